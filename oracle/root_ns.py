@@ -1,0 +1,131 @@
+"""Direct NVFP4 Newton-Schulz orthogonalisation (Q-Root), step by step.
+
+TEST INFRASTRUCTURE ONLY: imported by tests, by the smoke check and by the
+CPU-baseline leg of bench.py; never by the product path.
+
+Source: "Full-Stack FP4" (arXiv 2607.04422).
+  * Section 2, paragraph "Root optimizer": X_{k+1} = a X_k + b X_k (X_k^T X_k)
+    + c X_k (X_k^T X_k)^2, typically 5 iterations.  Written in the Gram-left
+    form used by Section 3.4, X (X^T X) = (X X^T) X, the Gram matrix is m x m
+    on the short side when X is m x n with m <= n.
+  * Section 3.4 "NVFP4 Root Optimizer", the iteration (with the random
+    Hadamard transform taken as the identity, as the method is specified for
+    this build):
+        qX_k  = Q1x16(X_k),            A_k = qX_k qX_k^T
+        qA_k  = Q1x16(A_k),  qA16_k = Q16x1(A_k),  B_k = b A_k + c qA_k qA16_k
+        qB_k  = Q1x16(B_k),  qX16_k = Q16x1(X_k),  X_{k+1} = a X_k + qB_k qX16_k
+  * Section 3.4 also clips outliers before the iteration; the clip used here
+    is a hard clamp at clip_k * RMS of the normalised matrix.
+
+Readings taken where the pages are silent (each is listed in the design doc):
+  * Frobenius normalisation X_0 = G / (||G||_F + eps), eps = 1e-7, ||G||_F
+    accumulated in float64; inv = fp32(1 / (||G||_F + eps)) and X_0 = fp32(G * inv).
+  * Clip: tau = fp32(clip_k * ||G||_F * inv / sqrt(m n)), X_0 = clamp(X_0, -tau, tau).
+  * Iterates X_k, A_k and B_k are FP32 tensors (the precision the quantiser
+    reads); every matrix product is taken in float64 on dequantised operands
+    and rounded once to FP32.  A_k is made exactly symmetric (upper triangle
+    mirrored), as the Gram matrix is by definition.
+  * A tall input (m0 > n0) is processed as its transpose and the result is
+    transposed back, so the Gram matrix is always min(m0, n0) square.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import nvfp4
+
+NS_EPS = 1e-7
+
+
+def normalise_and_clip(X: np.ndarray, clip_k: float | None, eps: float = NS_EPS):
+    """FP32 X_0 = clamp(fp32(X * inv), +-tau).  Returns (X0, inv, tau, norm)."""
+    X = np.asarray(X, dtype=np.float32)
+    m, n = X.shape
+    norm = float(np.sqrt(np.sum(X.astype(np.float64) ** 2)))
+    inv = np.float32(1.0 / (norm + eps))
+    X0 = X * inv
+    tau = None
+    if clip_k is not None and clip_k > 0:
+        tau = np.float32(clip_k * norm * float(inv) / np.sqrt(float(m) * float(n)))
+        X0 = np.clip(X0, -tau, tau).astype(np.float32)
+    return X0, inv, tau, norm
+
+
+def symmetric_from_upper(A: np.ndarray) -> np.ndarray:
+    """Mirror the upper triangle (diagonal included) into the lower one."""
+    return np.triu(A) + np.triu(A, 1).T
+
+
+def ns_iterations_nvfp4(X0, K, a, b, c, mode="pow2", trace=None):
+    """K NVFP4 Newton-Schulz iterations (Section 3.4) from the FP32 m x n X0 (m <= n)."""
+    X = np.asarray(X0, dtype=np.float32)
+    for k in range(K):
+        # qX_k = Q1x16(X_k); qX16_k = Q16x1(X_k) (held as the 1x16 quantisation of X_k^T)
+        qx, sx, gx = nvfp4.quantize_rows(X, mode=mode)
+        qxt, sxt, gxt = nvfp4.quantize_cols(X, mode=mode)
+        dX = nvfp4.dequantize_rows(qx, sx, gx)                     # m x n
+        dX16 = nvfp4.dequantize_cols(qxt, sxt, gxt)                # m x n, 16x1 blocks
+        # A_k = qX_k qX_k^T
+        A = symmetric_from_upper(dX @ dX.T).astype(np.float32)
+        # qA_k = Q1x16(A_k), qA16_k = Q16x1(A_k), B_k = b A_k + c qA_k qA16_k
+        qa, sa, ga = nvfp4.quantize_rows(A, mode=mode)
+        qa16, sa16, ga16 = nvfp4.quantize_cols(A, mode=mode)
+        P = nvfp4.dequantize_rows(qa, sa, ga) @ nvfp4.dequantize_cols(qa16, sa16, ga16)
+        B = (b * A.astype(np.float64) + c * P).astype(np.float32)
+        # qB_k = Q1x16(B_k), X_{k+1} = a X_k + qB_k qX16_k
+        qb, sb, gb = nvfp4.quantize_rows(B, mode=mode)
+        Xn = (a * X.astype(np.float64) + nvfp4.dequantize_rows(qb, sb, gb) @ dX16).astype(np.float32)
+        if trace is not None:
+            trace.append(dict(X=X, qX=(qx, sx, gx), qXT=(qxt, sxt, gxt), A=A,
+                              qA=(qa, sa, ga), P=P, B=B, qB=(qb, sb, gb), X_next=Xn))
+        X = Xn
+    return X
+
+
+def ns_iterations_f64(X0, K, a, b, c):
+    """K Newton-Schulz iterations in float64, no quantisation (Section 2)."""
+    X = np.asarray(X0, dtype=np.float64)
+    for _ in range(K):
+        A = X @ X.T
+        X = a * X + (b * A + c * (A @ A)) @ X
+    return X
+
+
+def root_ns(G, K=5, a=3.4445, b=-4.7750, c=2.0315, clip_k=3.0, eps=NS_EPS,
+            quantized=True, mode="pow2", trace=None):
+    """Normalise, clip and run K Newton-Schulz iterations on the FP32 matrix G.
+
+    quantized=True: the NVFP4 route of Section 3.4 (FP32 result).
+    quantized=False: the plain float64 iteration of Section 2 (float64 result;
+    normalisation and clip done in float64).
+    """
+    G = np.asarray(G)
+    if G.ndim != 2:
+        raise ValueError("G must be a matrix")
+    if not np.all(np.isfinite(G)):
+        raise ValueError("non-finite input")
+    tall = G.shape[0] > G.shape[1]
+    X = G.T if tall else G
+    if quantized:
+        X0, inv, tau, norm = normalise_and_clip(X.astype(np.float32), clip_k, eps)
+        if trace is not None:
+            trace.append(dict(X0=X0, inv=inv, tau=tau, norm=norm))
+        Y = ns_iterations_nvfp4(X0, K, a, b, c, mode=mode, trace=trace)
+    else:
+        X64 = np.asarray(X, dtype=np.float64)
+        norm = float(np.sqrt(np.sum(X64 ** 2)))
+        X0 = X64 / (norm + eps)
+        if clip_k is not None and clip_k > 0:
+            tau = clip_k * np.sqrt(np.sum(X0 ** 2)) / np.sqrt(X0.size)
+            X0 = np.clip(X0, -tau, tau)
+        Y = ns_iterations_f64(X0, K, a, b, c)
+    return np.ascontiguousarray(Y.T if tall else Y)
+
+
+def orthogonality_error(X) -> float:
+    """||X X^T - I||_F / sqrt(m) for m x n X (m <= n, else X^T)."""
+    X = np.asarray(X, dtype=np.float64)
+    if X.shape[0] > X.shape[1]:
+        X = X.T
+    m = X.shape[0]
+    return float(np.linalg.norm(X @ X.T - np.eye(m)) / np.sqrt(m))
