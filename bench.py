@@ -1,0 +1,379 @@
+#!/usr/bin/env python
+"""Benchmark of the direct NVFP4 Newton-Schulz step (Q-Root, "Full-Stack FP4"
+Section 3.4) on B200: one JSON line on rank 0.
+
+A step is one fs4_root_ns_batched call over every matrix of the workload
+(normalise + clip + quantise, then K iterations of the three NVFP4 products),
+inputs resident in HBM.  Default workload: four 3B-class decoder blocks
+(28 matrices: Q/K/V/O 3072x3072, gate/up 8192x3072, down 3072x8192), the
+analogue of the pages' own Root measurement over four decoder blocks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Multi-GPU (torchrun): every rank runs the whole workload on its own GPU (the
+matrices are independent; no collective on the data path), so per-GPU work is
+fixed and the scaling is weak; the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "3b_4blocks_gauss"
+METRIC = "NVFP4 Newton-Schulz matrices/s (K=5 iterations per matrix)"
+UNIT = "matrices/s"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "of measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "of fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def phase_kinds(K):
+    """Kernel launched in each timed phase of one call (3 + 3K events)."""
+    kinds = ["reduce", "preamble"]
+    for _ in range(K):
+        kinds += ["gram_x", "gram_a", "update"]
+    return kinds
+
+
+def flops_per_launch(w, kind):
+    tot = 0.0
+    for (r, c) in w.shapes:
+        m, n = min(r, c), max(r, c)
+        if kind == "gram_x":
+            tot += m * (m + 1) * n
+        elif kind == "gram_a":
+            tot += m * (m + 1) * m
+        elif kind == "update":
+            tot += 2 * m * m * n
+    return tot
+
+
+def bytes_per_launch(w, kind):
+    """Algorithmic HBM bytes of the memory-bound phases (read G once, write X_0 and both views)."""
+    tot = 0.0
+    for (r, c) in w.shapes:
+        e = r * c
+        if kind == "reduce":
+            tot += 4 * e
+        elif kind == "preamble":
+            tot += 4 * e + 4 * e + 2 * (e / 2 + e / 16)
+    return tot
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        nums = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if nums:
+            return int(max(nums))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample_rate(w, budget_s: float):
+    """Time the oracle (as it stands) on one bounded sample of the workload:
+    one NVFP4 Newton-Schulz iteration of an m x n slice of its first matrix.
+    Returns (matrices/s extrapolated by algorithmic FLOPs, seconds, description)."""
+    import numpy as np
+    from oracle import root_ns as R
+    from nvfp4_precision_optimizer_b200.workloads import BASE_SEED, generate
+    r0, c0 = w.shapes[0]
+    m_full, n_full = min(r0, c0), max(r0, c0)
+    G = generate((m_full, n_full), w.dist, BASE_SEED, "cpu").numpy()
+    m = m_full
+    while True:
+        X0, _, _, _ = R.normalise_and_clip(G[:m], w.clip_k)
+        t0 = time.perf_counter()
+        R.ns_iterations_nvfp4(X0, 1, *w.coeffs[0])
+        dt = time.perf_counter() - t0
+        if dt <= budget_s or m <= 256:
+            break
+        m //= 2
+    f_sample = m * (m + 1) * n_full + m * (m + 1) * m + 2 * m * m * n_full
+    f_matrix = w.K * (m_full * (m_full + 1) * n_full + m_full * (m_full + 1) * m_full
+                      + 2 * m_full * m_full * n_full)
+    per_matrix_s = dt * f_matrix / f_sample
+    desc = (f"oracle (numpy float64 products, exact NVFP4 emulation): one NVFP4 NS iteration of a "
+            f"{m}x{n_full} slice of the first {m_full}x{n_full} matrix, {dt:.2f} s, extrapolated by "
+            f"algorithmic FLOPs to K={w.K} iterations of one full matrix")
+    return 1.0 / per_matrix_s, dt, desc
+
+
+def run_reference(args):
+    from nvfp4_precision_optimizer_b200.workloads import WORKLOADS
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    budget = max(5.0, 150.0 / max(1, args.steps + args.warmup))
+    rates = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        rate, dt, desc = oracle_sample_rate(w, budget)
+        if i >= args.warmup:
+            rates.append(rate)
+    value = statistics.median(rates)
+    cores = cpu_cores()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * len(w.shapes) / value, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 products, fp32 tensors",
+        "data": "synthetic", "config": {"workload": w.name, "matrices": len(w.shapes), "K": w.K},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    import nvfp4_precision_optimizer_b200 as F
+    from nvfp4_precision_optimizer_b200.workloads import BASE_SEED, WORKLOADS, matrices
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    w = WORKLOADS[args.workload]
+    K = w.K
+    Gs = matrices(w, device="cuda", seed=BASE_SEED + 1000 * rank)
+    outs = [torch.empty_like(G) for G in Gs]
+    arr = F._descs(Gs, outs, w.coeffs)
+    lib = F._lib.lib()
+    need = int(lib.fs4_root_ns_batched_workspace_size(len(Gs), arr))
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    n_ev = 3 + 3 * K
+
+    def call(events=None):
+        if events is None:
+            st = lib.fs4_root_ns_batched(len(Gs), arr, K, w.clip_k, 0, ws.data_ptr(), need,
+                                         stream.cuda_stream)
+        else:
+            ev_arr = (F._lib.c_vp * n_ev)(*[e.cuda_event for e in events])
+            st = lib.fs4_root_ns_batched_timed(len(Gs), arr, K, w.clip_k, 0, ws.data_ptr(), need,
+                                               stream.cuda_stream, ev_arr, n_ev)
+        F.check(st, "fs4_root_ns_batched")
+
+    for _ in range(max(3, args.warmup)):
+        call()
+    torch.cuda.synchronize()
+    F.check(F.device_status(ws), "device status after warm-up")
+
+    step_events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    with sampler:
+        time.sleep(0.3)
+        t_start.record(stream)
+        for s in range(args.steps):
+            call(step_events[s])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    F.check(F.device_status(ws), "device status after timed steps")
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    ms_step = total_ms / args.steps
+
+    # per-phase kernel durations (CUDA events on the launching stream)
+    kinds = phase_kinds(K)
+    per_kind = {}
+    for evs in step_events:
+        for i, kind in enumerate(kinds):
+            per_kind.setdefault(kind, []).append(evs[i].elapsed_time(evs[i + 1]))
+    totals = {k: sum(v) for k, v in per_kind.items()}
+    dom = max(totals, key=totals.get)
+    dom_ms = statistics.mean(per_kind[dom])
+    peaks, peak_src = measured_peaks()
+    fp4_peak = 4.0 * peaks["bf16_tflops_sustained"]
+    if dom in ("gram_x", "gram_a", "update"):
+        achieved = flops_per_launch(w, dom) / (dom_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                "frac": achieved / fp4_peak}
+    else:
+        achieved = bytes_per_launch(w, dom) / (dom_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    roof["kernel"] = dom
+    roof["ms_per_launch"] = dom_ms
+    roof["peak_source"] = (f"dense FP4 = 4 x bf16_tflops_sustained ({peak_src} MEASURED_PEAKS.json; "
+                           f"4 = nominal FP4/BF16 dense ratio)" if roof["bound"] == "tensor"
+                           else f"hbm_gbs ({peak_src} MEASURED_PEAKS.json)")
+    roof["traffic"] = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            tr = json.load(f)
+        ent = tr.get(args.workload, {}).get(dom)
+        if ent and ent.get("source_sha") == F._source_digest():
+            roof["traffic"] = ent["bytes_per_launch"]
+
+    value = world * len(Gs) / (ms_step * 1e-3)
+    tflops = world * w.flops_algorithmic() / (ms_step * 1e-3) / 1e12
+    phase_ms = {k: statistics.mean(v) * (1 if k in ("reduce", "preamble") else K) for k, v in per_kind.items()}
+
+    # end to end through the public API with host buffers: H2D inputs, call, D2H outputs
+    e2e = None
+    if not args.no_e2e:
+        host_in = [G.cpu().pin_memory() for G in Gs]
+        host_out = [torch.empty(G.shape, dtype=torch.float32).pin_memory() for G in Gs]
+        e2e_steps = max(1, min(args.steps, 5))
+        for it in range(1 + e2e_steps):
+            if it == 1:
+                barrier()
+                torch.cuda.synchronize()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            for G, h in zip(Gs, host_in):
+                G.copy_(h, non_blocking=True)
+            F.root_ns_batched(Gs, K=K, coeffs=w.coeffs, clip_k=w.clip_k, outs=outs, workspace=ws)
+            for o, h in zip(outs, host_out):
+                h.copy_(o, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
+        nbytes = sum(G.numel() * 4 for G in Gs)
+        e2e = {"value": world * len(Gs) / (e2e_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
+               "ms_per_step": e2e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, dt, desc = oracle_sample_rate(w, 20.0)
+        cpu = {"value": rate, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3/16) products, fp32 accumulate",
+            "data": "synthetic",
+            "config": {"workload": w.name, "matrices": len(Gs), "shapes": sorted(set(map(tuple, w.shapes))),
+                       "K": K, "coeffs": "Muon (3.4445, -4.7750, 2.0315)", "clip": "3 x RMS",
+                       "parallelism": f"replicas x{world} (independent matrices, no collective)",
+                       "l2": "inputs larger than L2 (%.2f GB per step)" % (sum(G.numel() for G in Gs) * 4 / 1e9)},
+            "tflops_algorithmic": tflops,
+            "frac_fp4_peak_algorithmic": tflops / world / fp4_peak,
+            "tflops_dense_equivalent": world * w.flops_dense() / (ms_step * 1e-3) / 1e12,
+            "phase_ms_per_step": phase_ms,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": args.steps * (2 + 3 * K),
+            "clocks": sampler.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,228 @@
+/*
+ * fs4.h -- C ABI of libfs4: direct NVFP4 Newton-Schulz orthogonalisation on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method is the "NVFP4 Root Optimizer" of "Full-Stack FP4: Stable LLM
+ * Pretraining with Quantized Projections, Optimizers, and Attention"
+ * (arXiv 2607.04422):
+ *   - Section 2, paragraph "NVFP4 format": E2M1 values in 1x16 blocks, one
+ *     FP8 E4M3 scale s per block and one FP32 tensor scale s_g, with
+ *     x_hat = x_E2M1 * s * s_g.
+ *   - Section 2, paragraph "Root optimizer": the Newton-Schulz polynomial
+ *     X_{k+1} = a X + b X (X^T X) + c X (X^T X)^2, typically 5 iterations.
+ *   - Section 3.4, "NVFP4 Root Optimizer": outlier clipping, then the
+ *     iteration A = qX qX^T, B = b A + c qA qA^{16x1},
+ *     X_{k+1} = a X + qB qX^{16x1}, all quantisations round to nearest.
+ *
+ * Conventions shared by every entry point
+ *   - Pointers are DEVICE pointers unless a parameter says "host".  The caller
+ *     owns every buffer, including the workspace; the library never allocates
+ *     device memory and never synchronises, except fs4_device_status().
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All work is enqueued asynchronously on it.
+ *   - Matrices are row-major FP32 with a leading dimension `ld` (elements)
+ *     >= the number of columns.
+ *   - Argument errors are detected on the host, returned synchronously, and
+ *     nothing is enqueued.  Conditions only the device can see (non-finite
+ *     input, a bounded device-side wait that gave up) are recorded in a status
+ *     word inside the workspace; read it with fs4_device_status().  Device
+ *     code never traps.
+ *   - Functions are thread-safe; the only global state is a per-device cache
+ *     of the SM count and architecture check.
+ *
+ * NVFP4 storage
+ *   - Codes: 4-bit E2M1, (sign, e1, e0, m), element 2j of a block row in the
+ *     LOW nibble of byte j and element 2j+1 in the high nibble.
+ *   - Scales: one E4M3 byte per 16 consecutive elements of a row.
+ *   - Tensor scale: one FP32 (device) per tensor.  Default: the smallest power
+ *     of two s_g with 6 * 448 * s_g >= amax (s_g = 1 for an all-zero tensor).
+ *   - PLAIN layout (default): codes[r * (cols/2) + c/2], scales[r * (cols/16) + c/16].
+ *   - TILED layout (FS4_LAYOUT_TILED), the tensor-core operand layout: rows
+ *     padded to Rp = roundup(rows,128), columns to Cp = roundup(cols,256),
+ *     padding is zero.  Codes: tile (r/128, c/256) of 16384 bytes at
+ *     ((r/128)*(Cp/256) + c/256) * 16384; inside it row r%128 starts at byte
+ *     128*(r%128) and its 16-byte chunk j = (c%256)/32 is stored at chunk
+ *     position j ^ (r%8).  Scales: atom (r/128, c/64) of 512 bytes at
+ *     ((r/128)*(Cp/64) + c/64) * 512; inside it the scale of rows r and of
+ *     column block (c/16)%4 is byte 16*(r%32) + 4*((r%128)/32) + (c/16)%4.
+ *     Sizes: codes Rp*Cp/2 bytes, scales Rp*Cp/16 bytes.
+ */
+#ifndef FS4_H
+#define FS4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t fs4_status;
+
+enum {
+  FS4_OK = 0,
+  FS4_ERR_INVALID_ARG = -1, /* null pointer, bad leading dimension, misaligned buffer, bad flag */
+  FS4_ERR_SHAPE = -2,       /* a size is zero, negative, too large, or not a multiple of 16 */
+  FS4_ERR_ALIAS = -3,       /* an output overlaps an input */
+  FS4_ERR_WORKSPACE = -4,   /* workspace null, misaligned (256 B) or smaller than required */
+  FS4_ERR_ARCH = -5,        /* current device is not compute capability 10.0 */
+  FS4_ERR_CUDA = -6,        /* a CUDA runtime call or kernel launch failed */
+  FS4_ERR_NONFINITE = -7,   /* (device status) NaN or Inf in the input matrix */
+  FS4_ERR_TIMEOUT = -8      /* (device status) a bounded device-side wait gave up */
+};
+
+enum { FS4_AXIS_ROW = 0, /* 1x16 blocks along each row */
+       FS4_AXIS_COL = 1  /* 16x1 blocks along each column; stored as the quantisation of x^T */ };
+
+enum {
+  FS4_SG_AMAX = 1u << 0,      /* quantize only: s_g = fp32(amax / 2688) instead of a power of two */
+  FS4_LAYOUT_TILED = 1u << 1  /* quantize/dequantize: codes and scales in the TILED layout */
+};
+
+/* Debug stop for fs4_root_ns / fs4_root_ns_batched: run only the phases up to
+ * and including `phase` and return (the workspace then holds that state).
+ * phase 0 = preamble (normalise, clip, quantise X_0); phase 1 + 3k + j is the
+ * j-th product of iteration k (j = 0: A = qX qX^T, 1: P = qA qA^T and
+ * B = b A + c P, 2: X_{k+1} = a X_k + qB qX^{16x1}).  Encoded in flag bits 8..15
+ * as (phase + 1); 0 means run everything. */
+#define FS4_STOP_AFTER(phase) ((uint32_t)(((phase) + 1) & 0xFF) << 8)
+
+/* Upper limits checked on the host. */
+#define FS4_MAX_DIM 65536       /* m, n of one Newton-Schulz matrix */
+#define FS4_MAX_ITERS 32        /* K */
+#define FS4_MAX_BATCH 224       /* matrices per fs4_root_ns_batched call */
+
+/* ------------------------------------------------------------------ quantise */
+
+/* Bytes of workspace fs4_nvfp4_quantize needs (at least 256-byte aligned). */
+size_t fs4_nvfp4_quantize_workspace_size(void);
+
+/* NVFP4-quantise an FP32 matrix x (rows x cols, leading dimension ld).
+ * Source: Section 2 "NVFP4 format" (block scale per 16 elements, FP32 tensor
+ * scale) with round-to-nearest (Section 3.4).
+ *   axis FS4_AXIS_ROW: 1x16 blocks along rows; the result is rows x cols
+ *     (cols % 16 == 0 for the PLAIN layout).
+ *   axis FS4_AXIS_COL: 16x1 blocks along columns; the result is the
+ *     quantisation of x^T, a cols x rows matrix (rows % 16 == 0 for PLAIN).
+ *   codes, scales: outputs in the PLAIN or TILED layout (flags); s_g: output,
+ *   one device float.  Rule for each block: s = RN_e4m3(fp32(amax_b /
+ *   fp32(6 s_g))) saturating at 448; code = sign | RN_e2m1(fp32(|x| /
+ *   fp32(dec(s) * s_g))) saturating at 6, ties to the even code; a block whose
+ *   scale rounds to 0 gets all-zero codes.
+ *   Errors: FS4_ERR_SHAPE for empty or unaligned shapes; FS4_ERR_INVALID_ARG
+ *   for null pointers, ld < cols, codes/scales not 16-byte aligned (TILED);
+ *   FS4_ERR_WORKSPACE.  Non-finite input is recorded as FS4_ERR_NONFINITE in
+ *   the workspace status word (outputs then undefined). */
+fs4_status fs4_nvfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld,
+                              int32_t axis, uint8_t* codes, uint8_t* scales, float* s_g,
+                              uint32_t flags, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/* Dequantise a row-blocked NVFP4 matrix (rows x cols, as written by
+ * fs4_nvfp4_quantize in the layout given by flags) into FP32 y (leading
+ * dimension ld): y = fp32(fp32(code * s) * s_g).  Errors as above. */
+fs4_status fs4_nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* s_g,
+                                int64_t rows, int64_t cols, float* y, int64_t ld,
+                                uint32_t flags, void* stream);
+
+/* --------------------------------------------------------------------- GEMM */
+
+/* D = deq(A) * deq(B)^T on the tcgen05 block-scaled tensor cores
+ * (kind::mxf4nvf4, UE4M3 scales per 16 elements, FP32 accumulation in TMEM).
+ * The product is the one every step of Section 3.4 takes on NVFP4 operands.
+ * A is M x K and B is N x K, both row-blocked along K and in the TILED layout
+ * (as fs4_nvfp4_quantize writes with FS4_LAYOUT_TILED); a_sg, b_sg are their
+ * device tensor scales.  D is M x N FP32 with leading dimension ldd.
+ * K is rounded up to 256 with the zero padding of the TILED layout.
+ * Errors: FS4_ERR_SHAPE (M, N, K < 1 or > FS4_MAX_DIM), FS4_ERR_INVALID_ARG
+ * (null or non-16-byte-aligned operand, ldd < N), FS4_ERR_WORKSPACE (status
+ * word: workspace of fs4_nvfp4_quantize_workspace_size() bytes). */
+fs4_status fs4_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_sg,
+                          const uint8_t* b_codes, const uint8_t* b_scales, const float* b_sg,
+                          int64_t M, int64_t N, int64_t K, float* d, int64_t ldd,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* ----------------------------------------------------------- Newton-Schulz */
+
+/* One matrix of a batched call.  G (input) and out (output) are m x n FP32
+ * device matrices with leading dimensions ld and ld_out; out must not overlap
+ * G.  (a, b, c) are this matrix's polynomial coefficients (Section 3.4:
+ * Root's shape-dependent coefficients are passed per matrix). */
+typedef struct {
+  const float* G;
+  float* out;
+  int64_t m, n, ld, ld_out;
+  float a, b, c;
+} fs4_ns_desc;
+
+/* Workspace bytes fs4_root_ns needs for one m x n matrix. */
+size_t fs4_root_ns_workspace_size(int64_t m, int64_t n);
+
+/* Workspace bytes fs4_root_ns_batched needs for `count` matrices (host array). */
+size_t fs4_root_ns_batched_workspace_size(int32_t count, const fs4_ns_desc* descs);
+
+/* Direct NVFP4 Newton-Schulz step (Section 3.4) on one FP32 momentum matrix.
+ *   X_0 = clamp(G / (||G||_F + 1e-7), +-tau), tau = clip_k * RMS of the
+ *   normalised matrix (clip_k <= 0 disables the clamp); then K iterations of
+ *   qX = Q1x16(X), A = qX qX^T, B = b A + c Q1x16(A) Q16x1(A),
+ *   X <- a X + Q1x16(B) Q16x1(X).  A tall matrix (m > n) is processed as its
+ *   transpose so the Gram matrix is min(m,n) square; out has G's shape.
+ *   m, n multiples of 16 in [16, FS4_MAX_DIM]; 1 <= K <= FS4_MAX_ITERS;
+ *   a, b, c, clip_k finite.  Errors: FS4_ERR_SHAPE, FS4_ERR_INVALID_ARG,
+ *   FS4_ERR_ALIAS (out overlaps G), FS4_ERR_WORKSPACE, FS4_ERR_ARCH,
+ *   FS4_ERR_CUDA; device-side FS4_ERR_NONFINITE / FS4_ERR_TIMEOUT via
+ *   fs4_device_status (out is then zero or undefined-but-finite). */
+fs4_status fs4_root_ns(const float* G, int64_t m, int64_t n, int64_t ld, float* out,
+                       int64_t ld_out, int32_t K, float a, float b, float c, float clip_k,
+                       uint32_t flags, void* workspace, size_t workspace_bytes, void* stream);
+
+/* The same step on `count` independent matrices (descs is a HOST array),
+ * grouped so that each phase of the iteration is one launch over the tiles
+ * of all matrices (2 + 3K launches per call). */
+fs4_status fs4_root_ns_batched(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
+                               uint32_t flags, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* fs4_root_ns_batched, with CUDA events recorded on `stream` around each
+ * phase so a caller can time the kernels on the launching stream.
+ * phase_events: HOST array of n_events >= 3 + 3K cudaEvent_t handles (created
+ * by the caller with timing enabled).  Event 0 is recorded before the
+ * workspace reset and the reduction kernel, event 1 after it, event 2 after
+ * the preamble kernel, and event 3 + 3k + j after product j (0: A = qX qX^T,
+ * 1: B, 2: update) of iteration k.  Errors as fs4_root_ns_batched, plus
+ * FS4_ERR_INVALID_ARG for a missing event. */
+fs4_status fs4_root_ns_batched_timed(int32_t count, const fs4_ns_desc* descs, int32_t K,
+                                     float clip_k, uint32_t flags, void* workspace,
+                                     size_t workspace_bytes, void* stream,
+                                     void* const* phase_events, int32_t n_events);
+
+/* Synchronise `stream` and return the device status recorded in `workspace`
+ * by the last call that used it (FS4_OK, FS4_ERR_NONFINITE, FS4_ERR_TIMEOUT). */
+fs4_status fs4_device_status(const void* workspace, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* fs4_status_string(fs4_status status);
+
+/* Byte offsets (from the workspace base) of the internal tensors of matrix
+ * `index` of a batched call, for inspection after an FS4_STOP_AFTER run.
+ * mp, np: working dimensions padded to 256 (m <= n after the tall transpose).
+ * X: FP32 mp x np.  A: FP32 mp x mp (upper 256x256 tiles written).
+ * qX/qXT/qA/qB: TILED codes + scales of X (mp x np), X^T (np x mp, the 16x1
+ * view of X), A and B (mp x mp); qX and qXT alternate between two buffers by
+ * iteration parity (slot k%2 holds the view of X_k).  scalars: a float array
+ * with s_g of X_k at [k], of A_k at [64+k], of B_k at [128+k]. */
+typedef struct {
+  int64_t mp, np;
+  int64_t X, A;
+  int64_t qX_codes[2], qX_scales[2], qXT_codes[2], qXT_scales[2];
+  int64_t qA_codes, qA_scales, qB_codes, qB_scales;
+  int64_t scalars;
+} fs4_ns_layout;
+
+fs4_status fs4_root_ns_layout(int32_t count, const fs4_ns_desc* descs, int32_t index,
+                              fs4_ns_layout* layout);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FS4_H */

@@ -1,0 +1,198 @@
+"""Direct NVFP4 Newton-Schulz orthogonalisation (the Q-Root step of "Full-Stack
+FP4", arXiv 2607.04422, Section 3.4) on NVIDIA B200.
+
+Every step runs in the sm_100a kernels of libfs4.so behind the C ABI declared
+in include/fs4.h; this module only marshals torch tensors (device memory and
+streams) into those calls.  There is no CPU or fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Sequence
+
+import torch
+
+from . import _lib
+from ._lib import (FS4_AXIS_COL, FS4_AXIS_ROW, FS4_LAYOUT_TILED, FS4_SG_AMAX, Fs4Error, NsDesc,
+                   NsLayout, check, stop_after)
+
+MUON_COEFFS = (3.4445, -4.7750, 2.0315)
+
+__all__ = [
+    "quantize", "dequantize", "gemm", "root_ns", "root_ns_batched", "ns_workspace_size",
+    "ns_batched_workspace_size", "ns_layout", "device_status", "tiled_shape", "Fs4Error",
+    "MUON_COEFFS", "stop_after", "FS4_AXIS_ROW", "FS4_AXIS_COL",
+]
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _check_f32_matrix(x: torch.Tensor, name: str) -> None:
+    if not x.is_cuda or x.dtype != torch.float32 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError(f"{name} must be a CUDA float32 matrix with unit column stride")
+
+
+def _round_up(v: int, a: int) -> int:
+    return (v + a - 1) // a * a
+
+
+def tiled_shape(rows: int, cols: int) -> tuple[int, int]:
+    """(codes bytes, scales bytes) of a rows x cols matrix in the TILED layout."""
+    rp, cp = _round_up(rows, 128), _round_up(cols, 256)
+    return rp * cp // 2, rp * cp // 16
+
+
+def quantize(x: torch.Tensor, axis: int = FS4_AXIS_ROW, tiled: bool = False,
+             sg_mode: str = "pow2", workspace: torch.Tensor | None = None, stream=None):
+    """NVFP4-quantise x (fs4_nvfp4_quantize).  Returns (codes, scales, s_g)."""
+    _check_f32_matrix(x, "x")
+    rows, cols = x.shape
+    R, C = (rows, cols) if axis == FS4_AXIS_ROW else (cols, rows)
+    if tiled:
+        ncode, nscale = tiled_shape(R, C)
+        codes = torch.empty(ncode, dtype=torch.uint8, device=x.device)
+        scales = torch.empty(nscale, dtype=torch.uint8, device=x.device)
+    else:
+        codes = torch.empty((R, C // 2), dtype=torch.uint8, device=x.device)
+        scales = torch.empty((R, max(C // 16, 1)), dtype=torch.uint8, device=x.device)
+    s_g = torch.empty(1, dtype=torch.float32, device=x.device)
+    ws_bytes = _lib.lib().fs4_nvfp4_quantize_workspace_size()
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
+    flags = (FS4_LAYOUT_TILED if tiled else 0) | (FS4_SG_AMAX if sg_mode == "amax" else 0)
+    ld = x.stride(0) if rows > 1 else cols
+    check(_lib.lib().fs4_nvfp4_quantize(x.data_ptr(), rows, cols, ld, axis,
+                                        codes.data_ptr(), scales.data_ptr(), s_g.data_ptr(), flags,
+                                        workspace.data_ptr(), workspace.numel(), _stream(stream)),
+          "fs4_nvfp4_quantize")
+    return codes, scales, s_g
+
+
+def dequantize(codes: torch.Tensor, scales: torch.Tensor, s_g: torch.Tensor, rows: int, cols: int,
+               tiled: bool = False, stream=None) -> torch.Tensor:
+    """FP32 rows x cols matrix from an NVFP4 one (fs4_nvfp4_dequantize)."""
+    y = torch.empty((rows, cols), dtype=torch.float32, device=codes.device)
+    check(_lib.lib().fs4_nvfp4_dequantize(codes.data_ptr(), scales.data_ptr(), s_g.data_ptr(),
+                                          rows, cols, y.data_ptr(), cols,
+                                          FS4_LAYOUT_TILED if tiled else 0, _stream(stream)),
+          "fs4_nvfp4_dequantize")
+    return y
+
+
+def gemm(a, b, M: int, N: int, K: int, out: torch.Tensor | None = None,
+         workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """D = deq(A) deq(B)^T on the tensor cores (fs4_nvfp4_gemm); a, b are
+    (codes, scales, s_g) triples in the TILED layout, A M x K and B N x K."""
+    dev = a[0].device
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=dev)
+    check(_lib.lib().fs4_nvfp4_gemm(a[0].data_ptr(), a[1].data_ptr(), a[2].data_ptr(),
+                                    b[0].data_ptr(), b[1].data_ptr(), b[2].data_ptr(), M, N, K,
+                                    out.data_ptr(), _ld(out), workspace.data_ptr(),
+                                    workspace.numel(), _stream(stream)),
+          "fs4_nvfp4_gemm")
+    return out
+
+
+def _ld(t: torch.Tensor) -> int:
+    return t.stride(0) if t.shape[0] > 1 else t.shape[1]
+
+
+def _descs(Gs: Sequence[torch.Tensor], outs: Sequence[torch.Tensor], coeffs) -> ctypes.Array:
+    arr = (NsDesc * len(Gs))()
+    for i, (G, o) in enumerate(zip(Gs, outs)):
+        a, b, c = coeffs[i]
+        arr[i] = NsDesc(G.data_ptr(), o.data_ptr(), G.shape[0], G.shape[1], _ld(G), _ld(o), a, b, c)
+    return arr
+
+
+def ns_workspace_size(m: int, n: int) -> int:
+    return int(_lib.lib().fs4_root_ns_workspace_size(m, n))
+
+
+def _shape_descs(shapes: Sequence[tuple[int, int]]) -> ctypes.Array:
+    """Descriptors for size/layout queries: disjoint placeholder address ranges
+    (never dereferenced) so that the overlap checks pass."""
+    arr = (NsDesc * len(shapes))()
+    for i, (m, n) in enumerate(shapes):
+        arr[i] = NsDesc((2 * i + 1) << 36, (2 * i + 2) << 36, m, n, n, n, 1.0, 0.0, 0.0)
+    return arr
+
+
+def ns_batched_workspace_size(shapes: Sequence[tuple[int, int]]) -> int:
+    return int(_lib.lib().fs4_root_ns_batched_workspace_size(len(shapes), _shape_descs(shapes)))
+
+
+def root_ns(G: torch.Tensor, K: int = 5, a: float = MUON_COEFFS[0], b: float = MUON_COEFFS[1],
+            c: float = MUON_COEFFS[2], clip_k: float = 3.0, out: torch.Tensor | None = None,
+            workspace: torch.Tensor | None = None, flags: int = 0, stream=None) -> torch.Tensor:
+    """Direct NVFP4 Newton-Schulz step on one FP32 matrix (fs4_root_ns)."""
+    _check_f32_matrix(G, "G")
+    if out is None:
+        out = torch.empty_like(G)
+    m, n = G.shape
+    if workspace is None:
+        workspace = torch.empty(ns_workspace_size(m, n), dtype=torch.uint8, device=G.device)
+    check(_lib.lib().fs4_root_ns(G.data_ptr(), m, n, _ld(G), out.data_ptr(), _ld(out), K,
+                                 a, b, c, clip_k, flags, workspace.data_ptr(), workspace.numel(),
+                                 _stream(stream)),
+          "fs4_root_ns")
+    return out
+
+
+def root_ns_batched(Gs: Sequence[torch.Tensor], K: int = 5, coeffs=None, clip_k: float = 3.0,
+                    outs: Sequence[torch.Tensor] | None = None,
+                    workspace: torch.Tensor | None = None, flags: int = 0, stream=None):
+    """Direct NVFP4 Newton-Schulz step on a list of matrices in one grouped call
+    (fs4_root_ns_batched); coeffs is a list of per-matrix (a, b, c)."""
+    for G in Gs:
+        _check_f32_matrix(G, "G")
+    if coeffs is None:
+        coeffs = [MUON_COEFFS] * len(Gs)
+    if outs is None:
+        outs = [torch.empty_like(G) for G in Gs]
+    arr = _descs(Gs, outs, coeffs)
+    need = int(_lib.lib().fs4_root_ns_batched_workspace_size(len(Gs), arr))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=Gs[0].device)
+    check(_lib.lib().fs4_root_ns_batched(len(Gs), arr, K, clip_k, flags, workspace.data_ptr(),
+                                         workspace.numel(), _stream(stream)),
+          "fs4_root_ns_batched")
+    return outs
+
+
+def ns_layout(shapes: Sequence[tuple[int, int]], index: int = 0) -> NsLayout:
+    """Offsets of the internal tensors of matrix `index` (of a batched call on
+    matrices of these shapes) in the workspace."""
+    arr = _shape_descs(shapes)
+    lay = NsLayout()
+    check(_lib.lib().fs4_root_ns_layout(len(shapes), arr, index, ctypes.byref(lay)),
+          "fs4_root_ns_layout")
+    return lay
+
+
+def device_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise and return the device status word of the last call (0 = FS4_OK)."""
+    return int(_lib.lib().fs4_device_status(workspace.data_ptr(), _stream(stream)))
+
+
+def _source_digest() -> str:
+    """Short hash of the CUDA sources (ties stored ncu counters to the code they measured)."""
+    import hashlib
+    import os
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]

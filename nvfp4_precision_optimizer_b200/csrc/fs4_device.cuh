@@ -1,0 +1,332 @@
+// Device-side building blocks of libfs4 (sm_100a): PTX wrappers for mbarriers,
+// bulk copies and tcgen05, the TILED operand layout, and the 16-element NVFP4
+// block quantiser used by every kernel that writes an NVFP4 view.
+//
+// NVFP4 block rule ("Full-Stack FP4", Section 2, paragraph "NVFP4 format",
+// round-to-nearest per Section 3.4):
+//   s      = RN_e4m3(fp32(amax_b / fp32(6 s_g)))      (saturating at 448)
+//   code_i = sign_i | RN_e2m1(fp32(|x_i| / fp32(dec(s) s_g)))   (saturating at 6)
+//   a block whose scale rounds to 0 gets all-zero codes.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace fs4 {
+
+// ------------------------------------------------------------------ status word
+// Device-detected conditions are OR-ed into a 32-bit status word in the workspace.
+constexpr uint32_t kStatusNonFinite = 1u;
+constexpr uint32_t kStatusTimeout = 2u;
+// Bounded waits give up after this many nanoseconds of %globaltimer.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ------------------------------------------------------------------ TILED layout
+// Operand layout of a row-blocked NVFP4 matrix with Rp rows (multiple of 128)
+// and Cp columns (multiple of 256): 16 KB tiles of 128 rows x 256 elements in
+// the 128-byte-swizzled K-major form the tensor core reads, and 512-byte scale
+// atoms of 128 rows x 4 column blocks in the form tcgen05.cp copies to TMEM.
+constexpr int kTileRows = 128;
+constexpr int kTileK = 256;
+constexpr int kTileBytes = kTileRows * kTileK / 2;  // 16384
+constexpr int kAtomBytes = 512;
+
+// Byte offset of the 16-byte chunk that holds columns [c, c+32) of row r (c % 32 == 0).
+__host__ __device__ __forceinline__ int64_t tiled_chunk_offset(int64_t r, int64_t c, int64_t Cp) {
+  const int64_t tile = (r >> 7) * (Cp >> 8) + (c >> 8);
+  const int64_t rr = r & 127;
+  const int64_t j = (c & 255) >> 5;
+  return tile * kTileBytes + rr * 128 + ((j ^ (rr & 7)) << 4);
+}
+
+// Byte offset of the scale of row r, column block kb = c / 16.
+__host__ __device__ __forceinline__ int64_t tiled_scale_offset(int64_t r, int64_t kb, int64_t Cp) {
+  const int64_t atom = (r >> 7) * (Cp >> 6) + (kb >> 2);
+  return atom * kAtomBytes + 16 * (r & 31) + 4 * ((r & 127) >> 5) + (kb & 3);
+}
+
+// ------------------------------------------------------------------ conversions
+__device__ __forceinline__ uint32_t f32_to_e4m3(float v) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
+  return r & 0xFFu;
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)byte));
+  return __half2float(__ushort_as_half((uint16_t)(h2 & 0xFFFFu)));
+}
+
+// Eight FP32 values -> eight E2M1 codes packed low nibble first (RN, satfinite).
+__device__ __forceinline__ uint32_t pack8_e2m1(float q0, float q1, float q2, float q3, float q4,
+                                               float q5, float q6, float q7) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(q0), "f"(q1), "f"(q2), "f"(q3), "f"(q4), "f"(q5), "f"(q6), "f"(q7));
+  return out;
+}
+
+// Sum of the squared E2M1 values of the eight codes in `w`, accumulated into
+// a half2 (exact: every partial sum is a multiple of 1/4 below 512).
+__device__ __forceinline__ __half2 sq_e2m1_acc(uint32_t w, __half2 acc) {
+  uint32_t h0, h1, h2, h3;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
+      : "r"(w));
+  __half2 v0 = *reinterpret_cast<__half2*>(&h0), v1 = *reinterpret_cast<__half2*>(&h1);
+  __half2 v2 = *reinterpret_cast<__half2*>(&h2), v3 = *reinterpret_cast<__half2*>(&h3);
+  acc = __hfma2(v0, v0, acc);
+  acc = __hfma2(v1, v1, acc);
+  acc = __hfma2(v2, v2, acc);
+  acc = __hfma2(v3, v3, acc);
+  return acc;
+}
+
+// ------------------------------------------------------------------ tensor scale
+// Smallest power of two s_g with 2688 * s_g >= u, exponent clamped to [-116, 118];
+// 1 for u == 0.  Exact: 2688 = 1.3125 * 2^11, so compare u's mantissa with 1.3125.
+__host__ __device__ __forceinline__ float pow2_tensor_scale(float u) {
+  if (!(u > 0.0f)) return 1.0f;
+  uint32_t bits;
+#ifdef __CUDA_ARCH__
+  bits = __float_as_uint(u);
+#else
+  __builtin_memcpy(&bits, &u, 4);
+#endif
+  int e;
+  if ((bits >> 23) == 0) {
+    e = -126 - 11;  // subnormal u: far below the clamp
+  } else {
+    const int eu = (int)(bits >> 23) - 127;
+    const uint32_t mant = bits & 0x7FFFFFu;
+    e = (mant <= 0x280000u) ? eu - 11 : eu - 10;
+  }
+  e = e < -116 ? -116 : (e > 118 ? 118 : e);
+  uint32_t out = (uint32_t)(e + 127) << 23;
+  float f;
+#ifdef __CUDA_ARCH__
+  f = __uint_as_float(out);
+#else
+  __builtin_memcpy(&f, &out, 4);
+#endif
+  return f;
+}
+
+// ------------------------------------------------------------------ block quantiser
+struct QBlock16 {
+  uint32_t w0, w1;   // 16 codes, element 0 in the low nibble of w0
+  uint32_t scale;    // E4M3 byte
+  float sumsq;       // sum of the squared dequantised values
+};
+
+// Quantise 16 FP32 values with tensor scale s_g (six_sg = fp32(6 * s_g)).
+__device__ __forceinline__ QBlock16 quantize16(const float* x, float s_g, float six_sg) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  QBlock16 r;
+  r.scale = f32_to_e4m3(__fdiv_rn(amax, six_sg));
+  const float den = __fmul_rn(e4m3_to_f32(r.scale), s_g);
+  if (r.scale == 0u) {
+    r.w0 = r.w1 = 0u;
+    r.sumsq = 0.0f;
+    return r;
+  }
+  float q[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(x[i], den);
+  r.w0 = pack8_e2m1(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+  r.w1 = pack8_e2m1(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
+  __half2 acc = __float2half2_rn(0.0f);
+  acc = sq_e2m1_acc(r.w0, acc);
+  acc = sq_e2m1_acc(r.w1, acc);
+  const float s = __low2float(acc) + __high2float(acc);
+  r.sumsq = s * den * den;
+  return r;
+}
+
+// ------------------------------------------------------------------ shared memory / mbarriers
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0u;
+}
+
+// Wait for the phase with `parity` of `bar` to complete.  Gives up after
+// kWaitLimitNs (or at once if *abort is already set), records the timeout in
+// the status word and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status,
+                                          volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 63u) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(status, kStatusTimeout);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// 1-D bulk copy global -> shared (TMA engine), completion signalled on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// ------------------------------------------------------------------ tcgen05
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_addr(slot)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, K-major operand in 128-byte swizzled rows
+// (8-row groups 1024 bytes apart).  The start address must lie in a tile whose
+// base is 1024-byte aligned; advancing it by 32 bytes moves 64 FP4 along K.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);     // start address
+  d |= (uint64_t)1 << 16;                        // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;              // stride byte offset: 8 rows x 128 bytes
+  d |= (uint64_t)1 << 46;                        // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                        // 128-byte swizzle
+  return d;
+}
+
+// Descriptor of a plain 32-row x 16-byte block (one scale atom) for tcgen05.cp.
+__device__ __forceinline__ uint64_t sdesc_sf_atom(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(128 >> 4) << 32;               // 8-row core matrices 128 bytes apart
+  d |= (uint64_t)1 << 46;
+  return d;                                      // no swizzle
+}
+
+// Instruction descriptor: kind::mxf4nvf4, E2M1 x E2M1, UE4M3 scales, K-major A and B,
+// FP32 accumulate, M x N.
+__host__ __device__ constexpr uint32_t idesc_mxf4nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Copy one 512-byte scale atom from shared memory into 4 TMEM columns at
+// `taddr`, replicated to all four 32-lane quarters.
+__device__ __forceinline__ void tc_copy_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// D (TMEM) (+)= A(smem) * B(smem)^T with per-16 UE4M3 scales from TMEM; K = 64.
+__device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], "
+      "[%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Arrive on `bar` once every tcgen05 operation this thread issued so far has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_addr(bar))
+      : "memory");
+}
+
+// Load 32 consecutive 32-bit TMEM columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Named barrier among `count` threads (id 1..15; id 0 is __syncthreads).
+__device__ __forceinline__ void named_bar(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+}  // namespace fs4

@@ -1,0 +1,129 @@
+// Internal definitions shared by libfs4's kernels and its host-side planner.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fs4 {
+
+constexpr int kMaxBatch = 224;   // matrices per batched call (kernel-parameter table size)
+constexpr int kMaxIters = 32;
+constexpr int kPad = 256;        // working dimensions are padded to multiples of 256
+
+// ---------------------------------------------------------------- workspace header
+// Byte 0 of every workspace: the 32-bit device status word (kStatus* bits).
+// Bytes 4..7 of the quantize workspace: max |x| as float bits.
+constexpr size_t kHeaderBytes = 256;
+
+// ---------------------------------------------------------------- per-matrix state
+// One 4 KB block per matrix, zeroed at the start of every Newton-Schulz call.
+struct NsState {
+  double sumsq;            // sum of G^2 (float64)
+  uint32_t amaxG;          // max |G| as float bits
+  uint32_t nonfinite;      // G holds NaN or Inf
+  uint32_t done[4];        // finished work units per phase kind (preamble, G1, G2, G3)
+  uint32_t pad0[56];
+  float sg[192];           // tensor scales: X_k at [k], A_k at [64+k], B_k at [128+k]
+  float u_rowX[64];        // max_i sum_j deq(qX_k)_ij^2
+  float u_colX[64];        // max_j sum_i deq(qX16_k)_ij^2
+  float u_rowA[64];        // max_i sum_j deq(qA_k)_ij^2
+  float u_rowB[64];        // max_i sum_j deq(qB_k)_ij^2
+  uint32_t amaxX[64];      // max |X_k| as float bits
+  uint32_t pad1[448];
+};
+static_assert(sizeof(NsState) == 4096, "NsState must stay 4 KB");
+constexpr int kSgX = 0, kSgA = 64, kSgB = 128;
+
+// Offsets (bytes, from the workspace base) of one matrix's buffers.
+struct MatLayout {
+  int64_t state;                                 // NsState
+  int64_t rowsumX, colsumX, rowsumA, rowsumB;    // float [mp], [np], [mp], [mp]
+  int64_t X, A;                                  // float [mp*np], [mp*mp]
+  int64_t qX[2], sX[2], qXT[2], sXT[2];          // TILED codes/scales of X (mp x np), X^T (np x mp)
+  int64_t qA, sA, qB, sB;                        // TILED codes/scales of A, B (mp x mp)
+};
+
+__host__ __device__ inline int64_t align_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+// Bytes of the zero-initialised block (state + sums) of an mp x np matrix.
+__host__ __device__ inline int64_t state_block_bytes(int64_t mp, int64_t np) {
+  return align_up(4096 + 4 * (3 * mp + np), 256);
+}
+
+// Bytes of the large buffers of an mp x np matrix.
+__host__ __device__ inline int64_t big_block_bytes(int64_t mp, int64_t np) {
+  const int64_t xn = mp * np, aa = mp * mp;
+  return 4 * xn + 4 * aa + 2 * (xn / 2 + xn / 16) + 2 * (xn / 2 + xn / 16) + 2 * (aa / 2 + aa / 16);
+}
+
+__host__ __device__ inline MatLayout mat_layout(int64_t mp, int64_t np, int64_t state_off,
+                                                int64_t big_off) {
+  MatLayout L;
+  L.state = state_off;
+  L.rowsumX = state_off + 4096;
+  L.colsumX = L.rowsumX + 4 * mp;
+  L.rowsumA = L.colsumX + 4 * np;
+  L.rowsumB = L.rowsumA + 4 * mp;
+  const int64_t xn = mp * np, aa = mp * mp;
+  int64_t o = big_off;
+  L.X = o; o += 4 * xn;
+  L.A = o; o += 4 * aa;
+  for (int s = 0; s < 2; ++s) { L.qX[s] = o; o += xn / 2; L.sX[s] = o; o += xn / 16; }
+  for (int s = 0; s < 2; ++s) { L.qXT[s] = o; o += xn / 2; L.sXT[s] = o; o += xn / 16; }
+  L.qA = o; o += aa / 2; L.sA = o; o += aa / 16;
+  L.qB = o; o += aa / 2; L.sB = o; o += aa / 16;
+  return L;
+}
+
+// One matrix of a Newton-Schulz launch (kernel parameter, by value).
+struct MatDesc {
+  const float* G;          // caller's input, m0 x n0, leading dimension ldg
+  float* out;              // caller's output, m0 x n0, leading dimension ldo
+  int64_t ldg, ldo;
+  int64_t state_off, big_off;
+  int32_t m, n;            // working orientation, m <= n
+  int32_t mp, np;          // padded to multiples of 256
+  int32_t tall;            // 1: working X = G^T
+  float a, b, c;
+};
+
+// Kernel parameters of one Newton-Schulz phase over a batch of matrices.
+struct NsParams {
+  int32_t count;
+  int32_t iter;            // k of the current iteration
+  int32_t last;            // 1 on the final update product (writes `out`)
+  float clip_k;
+  uint32_t* status;
+  uint8_t* ws;             // workspace base
+  int32_t prefix[kMaxBatch + 1];   // prefix sums of this phase's work units per matrix
+  MatDesc mat[kMaxBatch];
+};
+static_assert(sizeof(NsParams) <= 32000, "kernel parameter block too large");
+
+// Parameters of the standalone block-scaled GEMM.
+struct GemmPlainArgs {
+  const uint8_t* a_codes; const uint8_t* a_scales; const float* a_sg;
+  const uint8_t* b_codes; const uint8_t* b_scales; const float* b_sg;
+  int32_t M, N, Kp;        // Kp: K padded to 256
+  int32_t Mp, Np;          // rows padded to 128
+  float* d;
+  int64_t ldd;
+  uint32_t* status;
+};
+
+enum class Epi : int { Plain = 0, GramX = 1, GramA = 2, Update = 3 };
+
+// ---------------------------------------------------------------- launchers (kernels.cu / gemm.cu)
+cudaError_t launch_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld, int axis,
+                            uint8_t* codes, uint8_t* scales, float* s_g, uint32_t flags,
+                            uint8_t* ws, cudaStream_t st, int num_sms);
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* s_g,
+                              int64_t rows, int64_t cols, float* y, int64_t ld, uint32_t flags,
+                              cudaStream_t st, int num_sms);
+cudaError_t launch_ns_reduce(const NsParams& p, cudaStream_t st, int num_sms);
+cudaError_t launch_ns_preamble(const NsParams& p, cudaStream_t st, int num_sms);
+cudaError_t launch_gemm_plain(const GemmPlainArgs& a, cudaStream_t st, int num_sms);
+cudaError_t launch_gemm_ns(Epi epi, const NsParams& p, cudaStream_t st, int num_sms);
+
+}  // namespace fs4

@@ -1,0 +1,539 @@
+// Block-scaled NVFP4 GEMMs on the 5th-generation tensor cores (sm_100a) with
+// the fused epilogues of the direct NVFP4 Newton-Schulz iteration.
+//
+// "Full-Stack FP4" (arXiv 2607.04422), Section 3.4, one iteration:
+//   G1  A   = qX qX^T                       epilogue: A (FP32), qA = Q1x16(A)
+//   G2  P   = qA qA16x1,  B = b A + c P     epilogue: qB = Q1x16(B)
+//   G3  X' = a X + qB qX16x1                epilogue: X' (FP32), Q1x16(X'), Q16x1(X')
+// A and B are symmetric, so G1 and G2 compute only the 256 x 256 tiles on and
+// above the diagonal; an off-diagonal tile also writes the transposed view,
+// which is the mirrored tile's 1x16 quantisation (Q16x1(A) = Q1x16(A)^T).
+//
+// Kernel structure (one persistent CTA per SM, 320 threads):
+//   warp 0     producer: 1-D bulk copies (TMA engine) of pre-tiled operand tiles
+//              and scale atoms into a 3-stage shared-memory ring
+//   warp 1     allocates 512 TMEM columns; one thread copies the scale atoms to
+//              TMEM (tcgen05.cp) and issues tcgen05.mma kind::mxf4nvf4
+//              (M=128, N=256, K=64, UE4M3 per-16 scales), FP32 accumulator in TMEM
+//   warps 2-9  epilogue: tcgen05.ld of the 128 x 256 accumulator, the fused
+//              element-wise step, requantisation of the next operand, and
+//              the row/column sums the next phase's tensor scales are bounded by
+// Every mbarrier wait is bounded (see mbar_wait); on a timeout the CTA stops
+// issuing work, drains what it issued, frees TMEM and returns.
+#include <cfloat>
+#include <cmath>
+
+#include "fs4_device.cuh"
+#include "fs4_internal.h"
+
+namespace fs4 {
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 256;
+constexpr int kStages = 3;
+constexpr int kThreads = 320;
+constexpr int kEpiThreads = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSfCol = 256;      // scale-factor columns follow the 256 accumulator columns
+constexpr uint32_t kSfBufCols = 48;   // 16 (A: 4 k-steps x 4) + 32 (B: 4 k-steps x 8)
+constexpr int A_BYTES = BM * BK / 2;
+constexpr int B_BYTES = BN * BK / 2;
+constexpr int SFA_BYTES = BM * BK / 16;
+constexpr int SFB_BYTES = BN * BK / 16;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+constexpr int TRANS_FLOATS = 32 * 33;
+constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + 8 * TRANS_FLOATS * 4 + 256;
+constexpr float kBoundInflate = 1.0f + 1.0f / 256.0f;
+constexpr uint32_t kIdesc = idesc_mxf4nvf4(BM, BN);
+static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
+
+struct Job {
+  int mat;
+  int64_t row0, col0;
+  int mirror;        // off-diagonal symmetric tile
+  int b_half;        // only the first 128 rows of the B tile exist
+  int kt;            // number of 256-wide K tiles
+  const uint8_t* a_codes; const uint8_t* a_sf;
+  const uint8_t* b_codes; const uint8_t* b_sf;
+  int64_t a_tile_row, b_tile_row;   // 128-row tile index of the A / B operand
+  int64_t ktiles_total;             // K tiles per operand row band (Kp / 256)
+};
+
+__device__ __forceinline__ int owner_of(const int32_t* prefix, int count, int64_t u) {
+  int lo = 0, hi = count - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= u) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Upper-triangle super tile s -> (P, Q), P <= Q, of a T x T grid, row-major.
+__device__ __forceinline__ void upper_tile(int64_t s, int64_t T, int64_t& P, int64_t& Q) {
+  P = 0;
+  while (s >= T - P) { s -= T - P; ++P; }
+  Q = P + s;
+}
+
+template <Epi E>
+__device__ __forceinline__ Job make_job(int64_t u, const NsParams& p, const GemmPlainArgs& g) {
+  Job j;
+  j.mirror = 0;
+  j.b_half = 0;
+  if constexpr (E == Epi::Plain) {
+    const int64_t nJ = (g.Np + BN - 1) / BN;
+    j.mat = 0;
+    j.row0 = (u / nJ) * BM;
+    j.col0 = (u % nJ) * BN;
+    j.b_half = (j.col0 + 128 >= g.Np) ? 1 : 0;
+    j.kt = g.Kp / BK;
+    j.ktiles_total = g.Kp / BK;
+    j.a_codes = g.a_codes; j.a_sf = g.a_scales;
+    j.b_codes = g.b_codes; j.b_sf = g.b_scales;
+  } else {
+    const int mi = owner_of(p.prefix, p.count, u);
+    const MatDesc& d = p.mat[mi];
+    const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
+    const int64_t lu = u - p.prefix[mi];
+    const int slot = p.iter & 1;
+    j.mat = mi;
+    if constexpr (E == Epi::GramX || E == Epi::GramA) {
+      const int64_t T = d.mp / 256;
+      int64_t P, Q;
+      upper_tile(lu >> 1, T, P, Q);
+      j.row0 = 256 * P + 128 * (lu & 1);
+      j.col0 = 256 * Q;
+      j.mirror = (P != Q) ? 1 : 0;
+      if constexpr (E == Epi::GramX) {
+        j.kt = d.np / BK;
+        j.a_codes = j.b_codes = p.ws + (slot ? L.qX[1] : L.qX[0]);
+        j.a_sf = j.b_sf = p.ws + (slot ? L.sX[1] : L.sX[0]);
+      } else {
+        j.kt = d.mp / BK;
+        j.a_codes = j.b_codes = p.ws + L.qA;
+        j.a_sf = j.b_sf = p.ws + L.sA;
+      }
+    } else {
+      const int64_t nJ = d.np / BN;
+      j.row0 = (lu / nJ) * BM;
+      j.col0 = (lu % nJ) * BN;
+      j.kt = d.mp / BK;
+      j.a_codes = p.ws + L.qB; j.a_sf = p.ws + L.sB;
+      j.b_codes = p.ws + (slot ? L.qXT[1] : L.qXT[0]);
+      j.b_sf = p.ws + (slot ? L.sXT[1] : L.sXT[0]);
+    }
+    j.ktiles_total = j.kt;
+  }
+  j.a_tile_row = j.row0 / 128;
+  j.b_tile_row = j.col0 / 128;
+  return j;
+}
+
+template <Epi E>
+__device__ __forceinline__ int64_t total_units(const NsParams& p, const GemmPlainArgs& g) {
+  if constexpr (E == Epi::Plain) {
+    return (int64_t)(g.Mp / BM) * ((g.Np + BN - 1) / BN);
+  } else {
+    return p.prefix[p.count];
+  }
+}
+
+// Max of a value over the 256 epilogue threads (named barrier 2); valid in epilogue thread 0.
+__device__ __forceinline__ float epi_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  const int et = threadIdx.x - 64;
+  named_bar(2, kEpiThreads);
+  if ((et & 31) == 0) red[et >> 5] = v;
+  named_bar(2, kEpiThreads);
+  if (et == 0) {
+    v = red[0];
+    for (int k = 1; k < 8; ++k) v = fmaxf(v, red[k]);
+  }
+  return v;
+}
+
+__device__ __forceinline__ float epi_drain_max(float* vec, int64_t len, float* red) {
+  float m = 0.0f;
+  for (int64_t i = threadIdx.x - 64; i < len; i += kEpiThreads) {
+    m = fmaxf(m, __ldcg(vec + i));
+    __stcg(vec + i, 0.0f);
+  }
+  return epi_max(m, red);
+}
+
+// 1x16 quantisation of 32 consecutive values of row r starting at column c (c % 32 == 0).
+__device__ __forceinline__ float store_row_chunk(const float* v, int64_t r, int64_t c, int64_t Cp,
+                                                 uint8_t* codes, uint8_t* scales, float sg,
+                                                 float six) {
+  const QBlock16 q0 = quantize16(v, sg, six);
+  const QBlock16 q1 = quantize16(v + 16, sg, six);
+  *reinterpret_cast<uint4*>(codes + tiled_chunk_offset(r, c, Cp)) =
+      make_uint4(q0.w0, q0.w1, q1.w0, q1.w1);
+  *reinterpret_cast<uint16_t*>(scales + tiled_scale_offset(r, c >> 4, Cp)) =
+      static_cast<uint16_t>(q0.scale | (q1.scale << 8));
+  return q0.sumsq + q1.sumsq;
+}
+
+// Transpose this warp's 32 x 32 chunk through shared memory: on return w[t]
+// holds the value of row t of the chunk in this lane's column.
+__device__ __forceinline__ void warp_transpose(const float* v, float* w, float* tb, int lane) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) tb[lane * 33 + j] = v[j];
+  __syncwarp();
+#pragma unroll
+  for (int t = 0; t < 32; ++t) w[t] = tb[t * 33 + lane];
+  __syncwarp();
+}
+
+template <Epi E>
+__global__ void __launch_bounds__(kThreads, 1)
+    nvfp4_gemm_kernel(const __grid_constant__ NsParams p, const __grid_constant__ GemmPlainArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  float* trans = reinterpret_cast<float*>(smem + kStages * STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * STAGE_BYTES + 8 * TRANS_FLOATS * 4);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kStages;
+  uint64_t* acc_full = bars + 2 * kStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* mma_done = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* s_last = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  volatile int* s_go = reinterpret_cast<volatile int*>(tmem_slot + 3);
+  float* red = reinterpret_cast<float*>(tmem_slot + 4);
+
+  uint32_t* status = (E == Epi::Plain) ? g.status : p.status;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 8);
+    mbar_init(mma_done, 1);
+    *abort_flag = (__ldcg(status) & kStatusTimeout) ? 1 : 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int64_t total = total_units<E>(p, g);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int64_t u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
+        const Job j = make_job<E>(u, p, g);
+        for (int kt = 0; kt < j.kt; ++kt, ++it) {
+          const uint32_t s = it % kStages, use = it / kStages;
+          if (!mbar_wait(&empty[s], (use & 1u) ^ 1u, status, abort_flag)) break;
+          uint8_t* st = stage_base + s * STAGE_BYTES;
+          const uint32_t bbytes = j.b_half ? (B_BYTES + SFB_BYTES) / 2 : (B_BYTES + SFB_BYTES);
+          mbar_arrive_expect_tx(&full[s], A_BYTES + SFA_BYTES + bbytes);
+          const int64_t at = j.a_tile_row * j.ktiles_total + kt;
+          bulk_g2s(st, j.a_codes + at * kTileBytes, A_BYTES, &full[s]);
+          bulk_g2s(st + A_BYTES + B_BYTES, j.a_sf + at * (4 * kAtomBytes), SFA_BYTES, &full[s]);
+          for (int h = 0; h < (j.b_half ? 1 : 2); ++h) {
+            const int64_t bt = (j.b_tile_row + h) * j.ktiles_total + kt;
+            bulk_g2s(st + A_BYTES + h * kTileBytes, j.b_codes + bt * kTileBytes, kTileBytes, &full[s]);
+            bulk_g2s(st + A_BYTES + B_BYTES + SFA_BYTES + h * (4 * kAtomBytes),
+                     j.b_sf + bt * (4 * kAtomBytes), 4 * kAtomBytes, &full[s]);
+          }
+        }
+      }
+      // drain: every issued copy must land before the CTA may exit
+      const uint32_t first = it > (uint32_t)kStages ? it - kStages : 0u;
+      for (uint32_t k = first; k < it; ++k) {
+        volatile int never = 0;
+        mbar_wait(&full[k % kStages], (k / kStages) & 1u, status, &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, tl = 0;
+      const uint32_t acc = tmem;   // lane 0, column 0
+      for (int64_t u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++tl) {
+        const Job j = make_job<E>(u, p, g);
+        if (!mbar_wait(acc_empty, (tl & 1u) ^ 1u, status, abort_flag)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int kt = 0; kt < j.kt; ++kt, ++it) {
+          const uint32_t s = it % kStages, use = it / kStages;
+          if (!mbar_wait(&full[s], use & 1u, status, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint8_t* st = stage_base + s * STAGE_BYTES;
+          const uint32_t sa = smem_addr(st), sb = sa + A_BYTES;
+          const uint32_t ssfa = sa + A_BYTES + B_BYTES, ssfb = ssfa + SFA_BYTES;
+          const uint32_t sf = tmem + kSfCol + (it & 1u) * kSfBufCols;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            tc_copy_sf(sf + 4 * ks, sdesc_sf_atom(ssfa + ks * kAtomBytes));
+            tc_copy_sf(sf + 16 + 8 * ks, sdesc_sf_atom(ssfb + ks * kAtomBytes));
+            tc_copy_sf(sf + 16 + 8 * ks + 4, sdesc_sf_atom(ssfb + 4 * kAtomBytes + ks * kAtomBytes));
+          }
+          const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sb);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            tc_mma_nvf4(acc, da + 2 * ks, db + 2 * ks, kIdesc, sf + 4 * ks, sf + 16 + 8 * ks,
+                        (kt | ks) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+      }
+      tc_commit(mma_done);
+      volatile int never = 0;
+      mbar_wait(mma_done, 0, status, &never);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;          // 0..7
+    const int quad = warp & 3;        // TMEM lanes 32*quad .. 32*quad+31
+    const int ch = ew >> 2;           // column half of the 256-wide tile
+    float* tb = trans + ew * TRANS_FLOATS;
+    uint32_t tl = 0;
+    for (int64_t u = blockIdx.x; u < total; u += gridDim.x, ++tl) {
+      const Job j = make_job<E>(u, p, g);
+      // every epilogue warp takes the same go / stop decision (they share named barriers)
+      mbar_wait(acc_full, tl & 1u, status, abort_flag);
+      named_bar(1, kEpiThreads);
+      if (threadIdx.x == 64) *s_go = *abort_flag ? 0 : 1;
+      named_bar(1, kEpiThreads);
+      if (!*s_go) break;
+      tc_fence_after();
+      const int64_t gr0 = j.row0 + 32 * quad;   // first row of this warp's band
+      const int64_t gr = gr0 + lane;             // this lane's row
+
+      // per-job constants
+      float acc_scale, sg_out = 1.0f, six_out = 6.0f, coef_a = 0.0f, coef_b = 0.0f, coef_c = 0.0f;
+      const MatDesc* d = nullptr;
+      NsState* st = nullptr;
+      MatLayout L;
+      const int k = p.iter;
+      if constexpr (E == Epi::Plain) {
+        acc_scale = __ldg(g.a_sg) * __ldg(g.b_sg);
+      } else {
+        d = &p.mat[j.mat];
+        st = reinterpret_cast<NsState*>(p.ws + d->state_off);
+        L = mat_layout(d->mp, d->np, d->state_off, d->big_off);
+        coef_a = d->a; coef_b = d->b; coef_c = d->c;
+        if constexpr (E == Epi::GramX) {
+          const float sx = __ldcg(&st->sg[kSgX + k]);
+          acc_scale = sx * sx;
+          sg_out = __ldcg(&st->sg[kSgA + k]);
+        } else if constexpr (E == Epi::GramA) {
+          const float sa = __ldcg(&st->sg[kSgA + k]);
+          acc_scale = sa * sa;
+          sg_out = __ldcg(&st->sg[kSgB + k]);
+        } else {
+          acc_scale = __ldcg(&st->sg[kSgB + k]) * __ldcg(&st->sg[kSgX + k]);
+          sg_out = p.last ? 1.0f : __ldcg(&st->sg[kSgX + k + 1]);
+        }
+        six_out = __fmul_rn(6.0f, sg_out);
+      }
+
+      float row_acc = 0.0f, amax = 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        const int64_t gc = j.col0 + 128 * ch + 32 * c;
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(128 * ch + 32 * c), v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] *= acc_scale;
+
+        if constexpr (E == Epi::Plain) {
+          if (gr < g.M) {
+            float* drow = g.d + gr * g.ldd;
+            if (gc + 32 <= g.N && (g.ldd & 3) == 0 && ((reinterpret_cast<uintptr_t>(g.d) & 15) == 0)) {
+#pragma unroll
+              for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<float4*>(drow + gc + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (gc + e < g.N) drow[gc + e] = v[e];
+            }
+          }
+        } else if constexpr (E == Epi::GramX) {
+          float* Arow = reinterpret_cast<float*>(p.ws + L.A) + gr * d->mp;
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(Arow + gc + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+          row_acc += store_row_chunk(v, gr, gc, d->mp, p.ws + L.qA, p.ws + L.sA, sg_out, six_out);
+          if (j.mirror) {
+            float w[32];
+            warp_transpose(v, w, tb, lane);
+            const float cs = store_row_chunk(w, gc + lane, gr0, d->mp, p.ws + L.qA, p.ws + L.sA,
+                                             sg_out, six_out);
+            if (cs != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.rowsumA) + gc + lane, cs);
+          }
+        } else if constexpr (E == Epi::GramA) {
+          const float* Arow = reinterpret_cast<const float*>(p.ws + L.A) + gr * d->mp;
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 a4 = __ldcg(reinterpret_cast<const float4*>(Arow + gc + e));
+            v[e] = fmaf(coef_b, a4.x, coef_c * v[e]);
+            v[e + 1] = fmaf(coef_b, a4.y, coef_c * v[e + 1]);
+            v[e + 2] = fmaf(coef_b, a4.z, coef_c * v[e + 2]);
+            v[e + 3] = fmaf(coef_b, a4.w, coef_c * v[e + 3]);
+          }
+          row_acc += store_row_chunk(v, gr, gc, d->mp, p.ws + L.qB, p.ws + L.sB, sg_out, six_out);
+          if (j.mirror) {
+            float w[32];
+            warp_transpose(v, w, tb, lane);
+            const float cs = store_row_chunk(w, gc + lane, gr0, d->mp, p.ws + L.qB, p.ws + L.sB,
+                                             sg_out, six_out);
+            if (cs != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.rowsumB) + gc + lane, cs);
+          }
+        } else {  // Update
+          float* Xrow = reinterpret_cast<float*>(p.ws + L.X) + gr * d->np;
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 x4 = __ldcg(reinterpret_cast<const float4*>(Xrow + gc + e));
+            v[e] = fmaf(coef_a, x4.x, v[e]);
+            v[e + 1] = fmaf(coef_a, x4.y, v[e + 1]);
+            v[e + 2] = fmaf(coef_a, x4.z, v[e + 2]);
+            v[e + 3] = fmaf(coef_a, x4.w, v[e + 3]);
+          }
+          if (p.last) {
+            if (gr < d->m) {
+              if (!d->tall) {
+                float* orow = d->out + gr * d->ldo;
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                  if (gc + e < d->n) orow[gc + e] = v[e];
+              } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                  if (gc + e < d->n) d->out[(gc + e) * d->ldo + gr] = v[e];
+              }
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(Xrow + gc + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(v[e]));
+            const int ns = (k + 1) & 1;
+            row_acc += store_row_chunk(v, gr, gc, d->np, p.ws + (ns ? L.qX[1] : L.qX[0]),
+                                       p.ws + (ns ? L.sX[1] : L.sX[0]), sg_out, six_out);
+            float w[32];
+            warp_transpose(v, w, tb, lane);
+            const float cs = store_row_chunk(w, gc + lane, gr0, d->mp, p.ws + (ns ? L.qXT[1] : L.qXT[0]),
+                                             p.ws + (ns ? L.sXT[1] : L.sXT[0]), sg_out, six_out);
+            if (cs != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.colsumX) + gc + lane, cs);
+          }
+        }
+      }
+      // accumulator drained: hand it back to the MMA warp
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+
+      if constexpr (E != Epi::Plain) {
+        float* rowsum = nullptr;
+        if constexpr (E == Epi::GramX) rowsum = reinterpret_cast<float*>(p.ws + L.rowsumA);
+        if constexpr (E == Epi::GramA) rowsum = reinterpret_cast<float*>(p.ws + L.rowsumB);
+        if constexpr (E == Epi::Update) rowsum = reinterpret_cast<float*>(p.ws + L.rowsumX);
+        if (row_acc != 0.0f) atomicAdd(rowsum + gr, row_acc);
+        if constexpr (E == Epi::Update) {
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+          if (lane == 0 && !p.last) atomicMax(&st->amaxX[k + 1], __float_as_uint(amax));
+        }
+        // the last CTA to finish a tile of this matrix derives the next tensor scale;
+        // every thread fences its own (fire-and-forget) sum atomics before the count
+        constexpr int kind = (E == Epi::GramX) ? 1 : (E == Epi::GramA ? 2 : 3);
+        __threadfence();
+        named_bar(1, kEpiThreads);
+        if (threadIdx.x == 64) {
+          const uint32_t units = (uint32_t)(p.prefix[j.mat + 1] - p.prefix[j.mat]);
+          *s_last = (atomicAdd(&st->done[kind], 1u) == units - 1u) ? 1 : 0;
+        }
+        named_bar(1, kEpiThreads);
+        if (*s_last) {
+          __threadfence();
+          if constexpr (E == Epi::GramX) {
+            const float ua = epi_drain_max(rowsum, d->mp, red);
+            if (threadIdx.x == 64) {
+              st->u_rowA[k] = ua;
+              const float ub = (fabsf(coef_b) * __ldcg(&st->u_rowX[k]) + fabsf(coef_c) * ua) * kBoundInflate;
+              st->sg[kSgB + k] = pow2_tensor_scale(ub);
+            }
+          } else if constexpr (E == Epi::GramA) {
+            const float ub = epi_drain_max(rowsum, d->mp, red);
+            if (threadIdx.x == 64) {
+              st->u_rowB[k] = ub;
+              const float ax = __uint_as_float(__ldcg(&st->amaxX[k]));
+              const float ux = (fabsf(coef_a) * ax + sqrtf(ub * __ldcg(&st->u_colX[k]))) * kBoundInflate;
+              st->sg[kSgX + k + 1] = pow2_tensor_scale(ux);
+            }
+          } else {
+            const float ur = epi_drain_max(rowsum, d->mp, red);
+            const float uc = epi_drain_max(reinterpret_cast<float*>(p.ws + L.colsumX), d->np, red);
+            if (threadIdx.x == 64 && !p.last) {
+              st->u_rowX[k + 1] = ur;
+              st->u_colX[k + 1] = uc;
+              st->sg[kSgA + k + 1] = pow2_tensor_scale(ur * kBoundInflate);
+            }
+          }
+          if (threadIdx.x == 64) st->done[kind] = 0u;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <Epi E>
+cudaError_t launch_impl(const NsParams* p, const GemmPlainArgs* g, int64_t units, cudaStream_t st,
+                        int num_sms) {
+  static unsigned long long attr_set = 0ull;   // one bit per device; a benign race
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !(attr_set & (1ull << dev))) {
+    e = cudaFuncSetAttribute(nvfp4_gemm_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_set |= 1ull << dev;
+  }
+  const int grid = (int)(units < num_sms ? (units > 0 ? units : 1) : num_sms);
+  static const NsParams zero_p{};
+  static const GemmPlainArgs zero_g{};
+  nvfp4_gemm_kernel<E><<<grid, kThreads, SMEM_BYTES, st>>>(p ? *p : zero_p, g ? *g : zero_g);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_plain(const GemmPlainArgs& a, cudaStream_t st, int num_sms) {
+  const int64_t units = (int64_t)(a.Mp / BM) * ((a.Np + BN - 1) / BN);
+  return launch_impl<Epi::Plain>(nullptr, &a, units, st, num_sms);
+}
+
+cudaError_t launch_gemm_ns(Epi epi, const NsParams& p, cudaStream_t st, int num_sms) {
+  const int64_t units = p.prefix[p.count];
+  switch (epi) {
+    case Epi::GramX: return launch_impl<Epi::GramX>(&p, nullptr, units, st, num_sms);
+    case Epi::GramA: return launch_impl<Epi::GramA>(&p, nullptr, units, st, num_sms);
+    case Epi::Update: return launch_impl<Epi::Update>(&p, nullptr, units, st, num_sms);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace fs4

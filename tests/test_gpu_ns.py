@@ -1,0 +1,201 @@
+"""GPU parity of the direct NVFP4 Newton-Schulz step (fs4_root_ns / _batched).
+
+Inputs are seeded synthetic momenta; expected values come from oracle/ on the
+same FP32 input.  Tolerances:
+  * preamble (normalise, clip, both NVFP4 views): bit-exact;
+  * first Gram product A_0 = qX_0 qX_0^T: relative Frobenius <= 1e-5 (the
+    operands are bit-identical to the oracle's at that point);
+  * end-to-end: relative Frobenius <= 2e-2 and orthogonality error within 10%
+    of the oracle's wherever the method itself is not chaotic (K <= 3 with the
+    Muon coefficients, K = 5 with the contractive quintic).  With the Muon
+    coefficients at K = 5 the NVFP4 iterate diverges, and two oracle runs that
+    differ only by one-ulp accumulation noise already differ by 2-18%; there
+    the orthogonality error within 10% and the singular-value spectrum are
+    asserted instead.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import nvfp4 as Q
+from oracle import root_ns as R
+from tests.helpers import rel_frob, tiled_to_plain, ws_f32
+
+
+def view(ws, codes_off, scales_off, rows, cols):
+    """PLAIN codes/scales of a rows x cols TILED view stored in the workspace."""
+    nc, ns = rows * cols // 2, rows * cols // 16
+    c, s, _, _ = tiled_to_plain(ws[codes_off:codes_off + nc], ws[scales_off:scales_off + ns], rows, cols)
+    return c, s
+
+pytestmark = pytest.mark.gpu
+
+MUON = (3.4445, -4.7750, 2.0315)
+QUINTIC = (15 / 8, -10 / 8, 3 / 8)
+CUBIC = (1.5, -0.5, 0.0)
+
+
+def momentum(m, n, kind="gauss", seed=0):
+    rng = np.random.default_rng(seed)
+    if kind == "gauss":
+        g = rng.standard_normal((m, n)) * 0.02
+    elif kind == "outliers":
+        g = rng.standard_normal((m, n)) * 0.02
+        g[rng.random((m, n)) < 0.001] *= 50
+    elif kind == "student":
+        t = rng.standard_t(3, (m, n))
+        g = t * (0.02 / np.sqrt(np.mean(t * t)))
+    else:
+        raise ValueError(kind)
+    return g.astype(np.float32)
+
+
+def run_gpu(F, G, K, coef, clip_k=3.0, flags=0):
+    Gt = torch.from_numpy(G).cuda()
+    ws = torch.zeros(F.ns_workspace_size(*G.shape), dtype=torch.uint8, device="cuda")
+    out = F.root_ns(Gt, K, *coef, clip_k=clip_k, workspace=ws, flags=flags)
+    assert F.device_status(ws) == 0
+    return out.cpu().numpy(), ws.cpu().numpy()
+
+
+def working(G):
+    return G.T if G.shape[0] > G.shape[1] else G
+
+
+@pytest.mark.parametrize("shape,kind", [((256, 256), "gauss"), ((48, 80), "gauss"),
+                                        ((1024, 4096), "outliers"), ((320, 96), "student"),
+                                        ((512, 272), "gauss")])
+def test_preamble_bit_exact(fs4, shape, kind):
+    G = momentum(*shape, kind=kind, seed=1)
+    _, ws = run_gpu(fs4, G, 1, MUON, flags=fs4.stop_after(0))
+    lay = fs4.ns_layout([shape], 0)
+    mp, np_ = lay.mp, lay.np
+    X0, inv, tau, _ = R.normalise_and_clip(working(G), 3.0)
+    m, n = X0.shape
+    Xg = ws_f32(ws, lay.X, mp * np_).reshape(mp, np_)
+    assert np.array_equal(Xg[:m, :n].view(np.uint32), X0.view(np.uint32))
+    assert not Xg[m:].any() and not Xg[:, n:].any()
+    sg = ws_f32(ws, lay.scalars, 192)
+    c, s, g = Q.quantize_rows(X0)
+    assert sg[0] == g
+    gc, gs = view(ws, lay.qX_codes[0], lay.qX_scales[0], mp, np_)
+    assert np.array_equal(gs[:m, :n // 16], s) and np.array_equal(gc[:m, :n // 2], c)
+    ct, st, gt = Q.quantize_cols(X0)
+    assert gt == g
+    gc, gs = view(ws, lay.qXT_codes[0], lay.qXT_scales[0], np_, mp)
+    assert np.array_equal(gs[:n, :m // 16], st) and np.array_equal(gc[:n, :m // 2], ct)
+
+
+@pytest.mark.parametrize("shape,kind", [((256, 256), "gauss"), ((1024, 4096), "outliers"),
+                                        ((512, 768), "student"), ((48, 80), "gauss")])
+def test_first_gram_product_and_its_requantisation(fs4, shape, kind):
+    G = momentum(*shape, kind=kind, seed=2)
+    _, ws = run_gpu(fs4, G, 1, MUON, flags=fs4.stop_after(1))
+    lay = fs4.ns_layout([shape], 0)
+    mp = lay.mp
+    X0, _, _, _ = R.normalise_and_clip(working(G), 3.0)
+    m = X0.shape[0]
+    c, s, g = Q.quantize_rows(X0)
+    dX = Q.dequantize_rows(c, s, g)
+    A = dX @ dX.T
+    Ag = ws_f32(ws, lay.A, mp * mp).reshape(mp, mp).astype(np.float64)
+    upper = (np.arange(mp)[:, None] // 256) <= (np.arange(mp)[None, :] // 256)
+    Aw = np.zeros((mp, mp))
+    Aw[:m, :m] = A
+    assert rel_frob(Ag[upper], Aw[upper]) <= 1e-5
+    assert not Ag[upper & ((np.arange(mp)[:, None] >= m) | (np.arange(mp)[None, :] >= m))].any()
+    # the GPU's tensor scale of A is a power of two that covers amax(A)
+    sga = ws_f32(ws, lay.scalars, 192)[64]
+    assert 2688 * sga >= np.abs(A).max() and np.log2(sga) == int(np.log2(sga))
+    # requantised A (both triangles, from the 1x16 view and the mirrored 16x1 view)
+    A32 = R.symmetric_from_upper(A).astype(np.float32)
+    oc, os_, og = Q.quantize_rows(A32)
+    want = Q.dequantize_rows(oc, os_, og)
+    gc, gs = view(ws, lay.qA_codes, lay.qA_scales, mp, mp)
+    got = Q.dequantize_rows(gc[:m, :m // 2], gs[:m, :m // 16], sga)
+    diff = got != want
+    assert diff.mean() <= 2e-3
+    # where they differ, the FP32 inputs straddled a rounding boundary: one grid step apart
+    assert np.all(np.abs(got - want)[diff] <= 0.51 * np.maximum(np.abs(got), np.abs(want))[diff] + 1e-30)
+
+
+def _spectrum_rel(a, b):
+    sa = np.linalg.svd(working(a).astype(np.float64), compute_uv=False)
+    sb = np.linalg.svd(working(b).astype(np.float64), compute_uv=False)
+    return float(np.linalg.norm(sa - sb) / np.linalg.norm(sb))
+
+
+@pytest.mark.parametrize("shape,kind,K,coef", [
+    ((256, 256), "gauss", 1, MUON), ((256, 256), "gauss", 3, MUON),
+    ((1024, 4096), "outliers", 2, MUON), ((1024, 4096), "outliers", 3, MUON),
+    ((48, 80), "gauss", 3, MUON), ((4096, 1024), "student", 2, MUON),
+    ((512, 1536), "gauss", 5, QUINTIC), ((1536, 512), "student", 5, QUINTIC),
+    ((272, 528), "outliers", 5, QUINTIC), ((256, 768), "gauss", 5, CUBIC),
+])
+def test_end_to_end_parity(fs4, shape, kind, K, coef):
+    G = momentum(*shape, kind=kind, seed=3)
+    got, _ = run_gpu(fs4, G, K, coef)
+    want = R.root_ns(G, K, *coef, clip_k=3.0)
+    assert got.shape == G.shape
+    assert rel_frob(got, want) <= 2e-2
+    eo, eg = R.orthogonality_error(want), R.orthogonality_error(got)
+    assert abs(eg - eo) <= 0.1 * eo
+
+
+@pytest.mark.parametrize("shape,kind", [((256, 256), "gauss"), ((1024, 4096), "outliers")])
+def test_five_muon_steps_orthogonality_and_spectrum(fs4, shape, kind):
+    G = momentum(*shape, kind=kind, seed=4)
+    got, _ = run_gpu(fs4, G, 5, MUON)
+    want = R.root_ns(G, 5, *MUON, clip_k=3.0)
+    eo, eg = R.orthogonality_error(want), R.orthogonality_error(got)
+    assert abs(eg - eo) <= 0.1 * eo
+    assert _spectrum_rel(got, want) <= 5e-2
+    assert np.all(np.isfinite(got))
+
+
+def test_batched_matches_single_calls_and_oracle(fs4):
+    specs = [((256, 256), "gauss", MUON), ((128, 384), "gauss", QUINTIC),
+             ((384, 128), "student", CUBIC), ((48, 80), "outliers", MUON),
+             ((512, 1024), "gauss", QUINTIC)]
+    Gs = [momentum(*s, kind=k, seed=10 + i) for i, (s, k, _) in enumerate(specs)]
+    coeffs = [c for _, _, c in specs]
+    Gt = [torch.from_numpy(G).cuda() for G in Gs]
+    outs = fs4.root_ns_batched(Gt, K=3, coeffs=coeffs, clip_k=3.0)
+    torch.cuda.synchronize()
+    for G, Gd, o, coef in zip(Gs, Gt, outs, coeffs):
+        single = fs4.root_ns(Gd, 3, *coef, clip_k=3.0).cpu().numpy()
+        got = o.cpu().numpy()
+        assert np.array_equal(got, single)
+        assert rel_frob(got, R.root_ns(G, 3, *coef, clip_k=3.0)) <= 2e-2
+
+
+def test_strided_input_and_output(fs4):
+    G = momentum(96, 160, seed=5)
+    big = torch.zeros((96, 200), device="cuda")
+    big[:, :160] = torch.from_numpy(G).cuda()
+    out = torch.full((96, 176), -1.0, device="cuda")
+    fs4.root_ns(big[:, :160], 3, *QUINTIC, out=out[:, :160])
+    got = out.cpu().numpy()
+    assert np.all(got[:, 160:] == -1.0)
+    assert rel_frob(got[:, :160], R.root_ns(G, 3, *QUINTIC)) <= 2e-2
+
+
+def test_no_clip(fs4):
+    G = momentum(128, 256, kind="outliers", seed=6)
+    got, _ = run_gpu(fs4, G, 3, QUINTIC, clip_k=0.0)
+    assert rel_frob(got, R.root_ns(G, 3, *QUINTIC, clip_k=None)) <= 2e-2
+
+
+def test_zero_input(fs4):
+    got, _ = run_gpu(fs4, np.zeros((64, 128), np.float32), 5, MUON)
+    assert not got.any()
+
+
+def test_nonfinite_input_reports_status_and_zero_output(fs4):
+    G = momentum(64, 128, seed=7)
+    G[5, 9] = np.inf
+    Gt = torch.from_numpy(G).cuda()
+    ws = torch.zeros(fs4.ns_workspace_size(64, 128), dtype=torch.uint8, device="cuda")
+    out = fs4.root_ns(Gt, 3, workspace=ws)
+    assert fs4.device_status(ws) == -7
+    assert not out.cpu().numpy().any()

@@ -1,0 +1,98 @@
+"""GPU parity of the standalone NVFP4 quantiser and dequantiser (bit-exact).
+
+Inputs are seeded; expected codes, scales and tensor scales come from the
+oracle (oracle/nvfp4.py) applied to the same FP32 input.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import nvfp4 as Q
+from tests.helpers import tiled_to_plain
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs():
+    rng = np.random.default_rng(2026)
+    cases = {
+        "gauss_64x64": rng.standard_normal((64, 64)) * 0.02,
+        "gauss_ragged_100x272": rng.standard_normal((100, 272)),
+        "student_t_257x1024": rng.standard_t(3, (257, 1024)) * 0.02,
+        "outliers_48x4096": rng.standard_normal((48, 4096)) * 0.02 * np.where(rng.random((48, 4096)) < 0.001, 50, 1),
+        "one_block_1x16": rng.standard_normal((1, 16)),
+        "wide_range_32x512": rng.standard_normal((32, 512)) * np.exp(rng.uniform(-14, 4, (32, 1))),
+        "ties_16x64": rng.choice([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0], (16, 64)) * rng.choice([-1, 1], (16, 64)),
+        "zeros_32x32": np.zeros((32, 32)),
+        "tiny_negative_16x32": -np.abs(rng.standard_normal((16, 32))) * np.where(rng.random((16, 32)) < 0.5, 1e-3, 1.0),
+        "large_2048x2048": rng.standard_normal((2048, 2048)),
+    }
+    return {k: v.astype(np.float32) for k, v in cases.items()}
+
+
+CASES = _inputs()
+
+
+def _gpu_quant(F, x, axis, tiled, mode):
+    xt = torch.from_numpy(x).cuda()
+    codes, scales, sg = F.quantize(xt, axis=axis, tiled=tiled, sg_mode=mode)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), scales.cpu().numpy(), sg.cpu().numpy()[0]
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+@pytest.mark.parametrize("axis", [0, 1])
+@pytest.mark.parametrize("tiled", [False, True])
+def test_quantize_bit_exact(fs4, name, axis, tiled):
+    x = CASES[name]
+    if axis == 1 and x.shape[0] % 16:
+        pytest.skip("column blocks need rows % 16 == 0")
+    for mode in ("pow2", "amax"):
+        want_c, want_s, want_g = (Q.quantize_rows(x, mode=mode) if axis == 0
+                                  else Q.quantize_cols(x, mode=mode))
+        c, s, g = _gpu_quant(fs4, x, axis, tiled, mode)
+        R, C = (x.shape if axis == 0 else x.shape[::-1])
+        if tiled:
+            c, s, cpad, spad = tiled_to_plain(c, s, R, C)
+            assert not cpad[R:].any() and not cpad[:, C // 2:].any()
+            assert not spad[R:].any() and not spad[:, C // 16:].any()
+        assert np.float32(g) == want_g, (name, mode)
+        assert np.array_equal(s, want_s), (name, mode, np.argwhere(s != want_s)[:5])
+        assert np.array_equal(c, want_c), (name, mode, np.argwhere(c != want_c)[:5])
+
+
+def test_hand_worked_blocks_on_gpu(fs4, golden_dir):
+    with open(os.path.join(golden_dir, "hand_blocks.json")) as f:
+        cases = json.load(f)["cases"]
+    for case in cases:
+        x = np.array(case["x"], np.float32)[None, :]
+        c, s, g = _gpu_quant(fs4, x, 0, False, "pow2")
+        assert float(g) == case["s_g"]
+        assert [f"{b:02x}" for b in s[0]] == case["scales_hex"]
+        assert [f"{b:02x}" for b in c[0]] == case["codes_hex"]
+
+
+@pytest.mark.parametrize("name", ["gauss_ragged_100x272", "wide_range_32x512", "student_t_257x1024"])
+@pytest.mark.parametrize("tiled", [False, True])
+def test_dequantize_bit_exact(fs4, name, tiled):
+    x = CASES[name]
+    xt = torch.from_numpy(x).cuda()
+    for mode in ("pow2", "amax"):
+        codes, scales, sg = fs4.quantize(xt, tiled=tiled, sg_mode=mode)
+        y = fs4.dequantize(codes, scales, sg, x.shape[0], x.shape[1], tiled=tiled).cpu().numpy()
+        wc, ws, wg = Q.quantize_rows(x, mode=mode)
+        want = Q.dequantize_rows(wc, ws, wg, dtype=np.float32)
+        assert np.array_equal(y.view(np.uint32), want.view(np.uint32))
+
+
+def test_nonfinite_input_sets_device_status(fs4):
+    x = torch.zeros((16, 32), device="cuda")
+    x[3, 7] = float("nan")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    fs4.quantize(x, workspace=ws)
+    assert fs4.device_status(ws) == -7
+    fs4.quantize(torch.ones((16, 32), device="cuda"), workspace=ws)
+    assert fs4.device_status(ws) == 0
