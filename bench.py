@@ -264,6 +264,9 @@ def main():
     F.check(F.device_status(ws), "device status after warm-up")
 
     step_events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    for evs in step_events:          # torch creates the CUDA event on its first record
+        for e in evs:
+            e.record(stream)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     barrier()

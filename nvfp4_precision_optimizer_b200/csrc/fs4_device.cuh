@@ -80,25 +80,23 @@ __device__ __forceinline__ uint32_t pack8_e2m1(float q0, float q1, float q2, flo
   return out;
 }
 
-// Sum of the squared E2M1 values of the eight codes in `w`, accumulated into
-// a half2 (exact: every partial sum is a multiple of 1/4 below 512).
-__device__ __forceinline__ __half2 sq_e2m1_acc(uint32_t w, __half2 acc) {
-  uint32_t h0, h1, h2, h3;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-      : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
-      : "r"(w));
-  __half2 v0 = *reinterpret_cast<__half2*>(&h0), v1 = *reinterpret_cast<__half2*>(&h1);
-  __half2 v2 = *reinterpret_cast<__half2*>(&h2), v3 = *reinterpret_cast<__half2*>(&h3);
-  acc = __hfma2(v0, v0, acc);
-  acc = __hfma2(v1, v1, acc);
-  acc = __hfma2(v2, v2, acc);
-  acc = __hfma2(v3, v3, acc);
-  return acc;
+// The two FP16 halves of a 32-bit register as FP32.
+__device__ __forceinline__ float half_lo(uint32_t h2) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+}
+__device__ __forceinline__ float half_hi(uint32_t h2) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
+}
+
+// 4 x the sum of the squared E2M1 values of the eight codes in `w`, in integer
+// arithmetic: byte permutes look up (2 v)^2 in {0, 1, 4, 9, 16, 36, 64, 144} for
+// each code magnitude (sign bits masked off) and dp4a adds the bytes.
+__device__ __forceinline__ uint32_t sq4_e2m1_sum8(uint32_t w) {
+  constexpr uint32_t kLutLo = 0x09040100u;   // codes 0..3: 0, 1, 4, 9
+  constexpr uint32_t kLutHi = 0x90402410u;   // codes 4..7: 16, 36, 64, 144
+  const uint32_t lo = __byte_perm(kLutLo, kLutHi, w & 0x7777u);
+  const uint32_t hi = __byte_perm(kLutLo, kLutHi, (w >> 16) & 0x7777u);
+  return __dp4a(lo, 0x01010101u, __dp4a(hi, 0x01010101u, 0u));
 }
 
 // ------------------------------------------------------------------ tensor scale
@@ -151,16 +149,20 @@ __device__ __forceinline__ QBlock16 quantize16(const float* x, float s_g, float 
     r.sumsq = 0.0f;
     return r;
   }
+  // x / den correctly rounded, by Markstein's FMA correction: with rcp = RN(1/den)
+  // and q0 = RN(x rcp), the residual x - q0 den is exact and q0 + residual * rcp
+  // rounds to RN(x / den) (no underflow/overflow here: |x / den| <= 6.2 or x = 0).
+  const float rcp = __frcp_rn(den);
   float q[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(x[i], den);
+  for (int i = 0; i < 16; ++i) {
+    const float q0 = x[i] * rcp;
+    q[i] = fmaf(fmaf(-q0, den, x[i]), rcp, q0);
+  }
   r.w0 = pack8_e2m1(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
   r.w1 = pack8_e2m1(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
-  __half2 acc = __float2half2_rn(0.0f);
-  acc = sq_e2m1_acc(r.w0, acc);
-  acc = sq_e2m1_acc(r.w1, acc);
-  const float s = __low2float(acc) + __high2float(acc);
-  r.sumsq = s * den * den;
+  const float s4 = static_cast<float>(sq4_e2m1_sum8(r.w0) + sq4_e2m1_sum8(r.w1));
+  r.sumsq = 0.25f * s4 * den * den;
   return r;
 }
 
@@ -322,6 +324,59 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Issue a load of 32 consecutive TMEM columns of this warp's 32 lanes; the
+// registers are valid only after tmem_wait_ld32.
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+// Wait for this thread's outstanding TMEM loads.  The 32 registers are passed
+// through the statement so that no use of them can be scheduled before the wait;
+// call it (or tmem_ld_order) once per register group filled by tmem_ld32_async.
+__device__ __forceinline__ void tmem_wait_ld32(uint32_t* r) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+        "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+        "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
+
+// Order a further register group after a preceding tmem_wait_ld32 (no instruction).
+__device__ __forceinline__ void tmem_ld_order(uint32_t* r) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+
+// Per-warpgroup register budget changes (all 128 threads of the warpgroup execute them).
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // Named barrier among `count` threads (id 1..15; id 0 is __syncthreads).

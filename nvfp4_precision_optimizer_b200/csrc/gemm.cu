@@ -34,6 +34,7 @@ constexpr int BM = 128, BN = 256, BK = 256;
 constexpr int kStages = 3;
 constexpr int kThreads = 320;
 constexpr int kEpiThreads = 256;
+constexpr int kEpiBase = 64;           // first epilogue thread
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCol = 256;      // scale-factor columns follow the 256 accumulator columns
 constexpr uint32_t kSfBufCols = 48;   // 16 (A: 4 k-steps x 4) + 32 (B: 4 k-steps x 8)
@@ -143,7 +144,7 @@ __device__ __forceinline__ int64_t total_units(const NsParams& p, const GemmPlai
 __device__ __forceinline__ float epi_max(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  const int et = threadIdx.x - 64;
+  const int et = threadIdx.x - kEpiBase;
   named_bar(2, kEpiThreads);
   if ((et & 31) == 0) red[et >> 5] = v;
   named_bar(2, kEpiThreads);
@@ -156,7 +157,7 @@ __device__ __forceinline__ float epi_max(float v, float* red) {
 
 __device__ __forceinline__ float epi_drain_max(float* vec, int64_t len, float* red) {
   float m = 0.0f;
-  for (int64_t i = threadIdx.x - 64; i < len; i += kEpiThreads) {
+  for (int64_t i = threadIdx.x - kEpiBase; i < len; i += kEpiThreads) {
     m = fmaxf(m, __ldcg(vec + i));
     __stcg(vec + i, 0.0f);
   }
@@ -223,7 +224,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int64_t total = total_units<E>(p, g);
-
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -305,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every epilogue warp takes the same go / stop decision (they share named barriers)
       mbar_wait(acc_full, tl & 1u, status, abort_flag);
       named_bar(1, kEpiThreads);
-      if (threadIdx.x == 64) *s_go = *abort_flag ? 0 : 1;
+      if (threadIdx.x == kEpiBase) *s_go = *abort_flag ? 0 : 1;
       named_bar(1, kEpiThreads);
       if (!*s_go) break;
       tc_fence_after();
@@ -349,68 +349,60 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] *= acc_scale;
 
+        // FP32 tiles are read and written after a per-warp transpose (lane = column,
+        // w[t] = row gr0 + t): every warp access is then one contiguous 128-byte line.
         if constexpr (E == Epi::Plain) {
-          if (gr < g.M) {
-            float* drow = g.d + gr * g.ldd;
-            if (gc + 32 <= g.N && (g.ldd & 3) == 0 && ((reinterpret_cast<uintptr_t>(g.d) & 15) == 0)) {
+          float w[32];
+          warp_transpose(v, w, tb, lane);
+          const int64_t col = gc + lane;
+          if (col < g.N) {
 #pragma unroll
-              for (int e = 0; e < 32; e += 4)
-                *reinterpret_cast<float4*>(drow + gc + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (gc + e < g.N) drow[gc + e] = v[e];
-            }
+            for (int t = 0; t < 32; ++t)
+              if (gr0 + t < g.M) g.d[(gr0 + t) * g.ldd + col] = w[t];
           }
         } else if constexpr (E == Epi::GramX) {
-          float* Arow = reinterpret_cast<float*>(p.ws + L.A) + gr * d->mp;
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(Arow + gc + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
           row_acc += store_row_chunk(v, gr, gc, d->mp, p.ws + L.qA, p.ws + L.sA, sg_out, six_out);
+          float w[32];
+          warp_transpose(v, w, tb, lane);
+          float* Acol = reinterpret_cast<float*>(p.ws + L.A) + gr0 * d->mp + gc + lane;
+#pragma unroll
+          for (int t = 0; t < 32; ++t) Acol[t * d->mp] = w[t];
           if (j.mirror) {
-            float w[32];
-            warp_transpose(v, w, tb, lane);
             const float cs = store_row_chunk(w, gc + lane, gr0, d->mp, p.ws + L.qA, p.ws + L.sA,
                                              sg_out, six_out);
             if (cs != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.rowsumA) + gc + lane, cs);
           }
         } else if constexpr (E == Epi::GramA) {
-          const float* Arow = reinterpret_cast<const float*>(p.ws + L.A) + gr * d->mp;
+          const float* Acol = reinterpret_cast<const float*>(p.ws + L.A) + gr0 * d->mp + gc + lane;
+          float w[32], a_row[32];
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const float4 a4 = __ldcg(reinterpret_cast<const float4*>(Arow + gc + e));
-            v[e] = fmaf(coef_b, a4.x, coef_c * v[e]);
-            v[e + 1] = fmaf(coef_b, a4.y, coef_c * v[e + 1]);
-            v[e + 2] = fmaf(coef_b, a4.z, coef_c * v[e + 2]);
-            v[e + 3] = fmaf(coef_b, a4.w, coef_c * v[e + 3]);
-          }
+          for (int t = 0; t < 32; ++t) w[t] = __ldcg(Acol + t * d->mp);
+          warp_transpose(w, a_row, tb, lane);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = fmaf(coef_b, a_row[e], coef_c * v[e]);
           row_acc += store_row_chunk(v, gr, gc, d->mp, p.ws + L.qB, p.ws + L.sB, sg_out, six_out);
           if (j.mirror) {
-            float w[32];
             warp_transpose(v, w, tb, lane);
             const float cs = store_row_chunk(w, gc + lane, gr0, d->mp, p.ws + L.qB, p.ws + L.sB,
                                              sg_out, six_out);
             if (cs != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.rowsumB) + gc + lane, cs);
           }
         } else {  // Update
-          float* Xrow = reinterpret_cast<float*>(p.ws + L.X) + gr * d->np;
+          float w[32];
+          warp_transpose(v, w, tb, lane);
+          float* Xcol = reinterpret_cast<float*>(p.ws + L.X) + gr0 * d->np + gc + lane;
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const float4 x4 = __ldcg(reinterpret_cast<const float4*>(Xrow + gc + e));
-            v[e] = fmaf(coef_a, x4.x, v[e]);
-            v[e + 1] = fmaf(coef_a, x4.y, v[e + 1]);
-            v[e + 2] = fmaf(coef_a, x4.z, v[e + 2]);
-            v[e + 3] = fmaf(coef_a, x4.w, v[e + 3]);
-          }
+          for (int t = 0; t < 32; ++t) w[t] = fmaf(coef_a, __ldcg(Xcol + t * d->np), w[t]);
           if (p.last) {
-            if (gr < d->m) {
-              if (!d->tall) {
-                float* orow = d->out + gr * d->ldo;
+            if (!d->tall) {
+              if (gc + lane < d->n) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                  if (gc + e < d->n) orow[gc + e] = v[e];
-              } else {
+                for (int t = 0; t < 32; ++t)
+                  if (gr0 + t < d->m) d->out[(gr0 + t) * d->ldo + gc + lane] = w[t];
+              }
+            } else {
+              warp_transpose(w, v, tb, lane);
+              if (gr < d->m) {
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
                   if (gc + e < d->n) d->out[(gc + e) * d->ldo + gr] = v[e];
@@ -418,21 +410,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           } else {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4*>(Xrow + gc + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(v[e]));
+            for (int t = 0; t < 32; ++t) {
+              Xcol[t * d->np] = w[t];
+              amax = fmaxf(amax, fabsf(w[t]));
+            }
             const int ns = (k + 1) & 1;
-            row_acc += store_row_chunk(v, gr, gc, d->np, p.ws + (ns ? L.qX[1] : L.qX[0]),
-                                       p.ws + (ns ? L.sX[1] : L.sX[0]), sg_out, six_out);
-            float w[32];
-            warp_transpose(v, w, tb, lane);
             const float cs = store_row_chunk(w, gc + lane, gr0, d->mp, p.ws + (ns ? L.qXT[1] : L.qXT[0]),
                                              p.ws + (ns ? L.sXT[1] : L.sXT[0]), sg_out, six_out);
             if (cs != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.colsumX) + gc + lane, cs);
+            warp_transpose(w, v, tb, lane);
+            row_acc += store_row_chunk(v, gr, gc, d->np, p.ws + (ns ? L.qX[1] : L.qX[0]),
+                                       p.ws + (ns ? L.sX[1] : L.sX[0]), sg_out, six_out);
           }
         }
       }
+
       // accumulator drained: hand it back to the MMA warp
       tc_fence_before();
       __syncwarp();
@@ -454,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kind = (E == Epi::GramX) ? 1 : (E == Epi::GramA ? 2 : 3);
         __threadfence();
         named_bar(1, kEpiThreads);
-        if (threadIdx.x == 64) {
+        if (threadIdx.x == kEpiBase) {
           const uint32_t units = (uint32_t)(p.prefix[j.mat + 1] - p.prefix[j.mat]);
           *s_last = (atomicAdd(&st->done[kind], 1u) == units - 1u) ? 1 : 0;
         }
@@ -463,14 +455,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           __threadfence();
           if constexpr (E == Epi::GramX) {
             const float ua = epi_drain_max(rowsum, d->mp, red);
-            if (threadIdx.x == 64) {
+            if (threadIdx.x == kEpiBase) {
               st->u_rowA[k] = ua;
               const float ub = (fabsf(coef_b) * __ldcg(&st->u_rowX[k]) + fabsf(coef_c) * ua) * kBoundInflate;
               st->sg[kSgB + k] = pow2_tensor_scale(ub);
             }
           } else if constexpr (E == Epi::GramA) {
             const float ub = epi_drain_max(rowsum, d->mp, red);
-            if (threadIdx.x == 64) {
+            if (threadIdx.x == kEpiBase) {
               st->u_rowB[k] = ub;
               const float ax = __uint_as_float(__ldcg(&st->amaxX[k]));
               const float ux = (fabsf(coef_a) * ax + sqrtf(ub * __ldcg(&st->u_colX[k]))) * kBoundInflate;
@@ -479,13 +471,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             const float ur = epi_drain_max(rowsum, d->mp, red);
             const float uc = epi_drain_max(reinterpret_cast<float*>(p.ws + L.colsumX), d->np, red);
-            if (threadIdx.x == 64 && !p.last) {
+            if (threadIdx.x == kEpiBase && !p.last) {
               st->u_rowX[k + 1] = ur;
               st->u_colX[k + 1] = uc;
               st->sg[kSgA + k + 1] = pow2_tensor_scale(ur * kBoundInflate);
             }
           }
-          if (threadIdx.x == 64) st->done[kind] = 0u;
+          if (threadIdx.x == kEpiBase) st->done[kind] = 0u;
         }
       }
     }

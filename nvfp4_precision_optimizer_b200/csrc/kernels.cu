@@ -189,10 +189,9 @@ __global__ void __launch_bounds__(kEwThreads) dequantize_kernel(
           : "r"(words[h]));
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
-        const __half2 hh = *reinterpret_cast<const __half2*>(&hv[p]);
         const int64_t c = j + h * 8 + p * 2;
-        y[i * ld + c] = __fmul_rn(__fmul_rn(__low2float(hh), s), s_g);
-        y[i * ld + c + 1] = __fmul_rn(__fmul_rn(__high2float(hh), s), s_g);
+        y[i * ld + c] = __fmul_rn(__fmul_rn(half_lo(hv[p]), s), s_g);
+        y[i * ld + c + 1] = __fmul_rn(__fmul_rn(half_hi(hv[p]), s), s_g);
       }
     }
   }

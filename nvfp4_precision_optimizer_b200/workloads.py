@@ -53,6 +53,7 @@ class Workload:
 WORKLOADS = {
     "single_256x256_gauss": Workload("single_256x256_gauss", [(256, 256)], "gauss"),
     "single_1024x4096_outliers": Workload("single_1024x4096_outliers", [(1024, 4096)], "outliers"),
+    "3b_1block_gauss": Workload("3b_1block_gauss", BLOCK_SHAPES, "gauss"),
     "3b_4blocks_gauss": Workload("3b_4blocks_gauss", BLOCK_SHAPES * 4, "gauss"),
     "3b_28blocks_student": Workload("3b_28blocks_student", BLOCK_SHAPES * 28, "student"),
     "single_8192x8192_student": Workload("single_8192x8192_student", [(8192, 8192)], "student"),

@@ -96,3 +96,42 @@ def test_nonfinite_input_sets_device_status(fs4):
     assert fs4.device_status(ws) == -7
     fs4.quantize(torch.ones((16, 32), device="cuda"), workspace=ws)
     assert fs4.device_status(ws) == 0
+
+
+def _threshold_sweep():
+    """Blocks whose scale decodes to each E4M3 mantissa 1 + m/8 and whose other
+    15 elements sweep 2^14 consecutive FP32 values on both sides of every E2M1
+    decision threshold (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5) times the decoded
+    scale.  The first element of each block is 6 * 2^-8 * (1 + m/8) * 256 /
+    256, which makes amax_b / (6 s_g) land exactly on that E4M3 value."""
+    rows = []
+    s_g = 2.0 ** -8
+    for m in range(8):
+        dec = (1 + m / 8) * 128                      # E4M3 value in [128, 256)
+        den = np.float32(dec * s_g)
+        head = np.float32(6.0 * dec * s_g)           # block amax -> scale exactly dec
+        for t in (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0):
+            centre = np.float32(t * den)
+            bits = centre.view(np.uint32).astype(np.int64)
+            vals = (np.arange(bits - 8190, bits + 8190)).astype(np.uint32).view(np.float32)
+            vals = vals.reshape(-1, 15)
+            blk = np.concatenate([np.full((vals.shape[0], 1), head, np.float32), vals], axis=1)
+            blk[1::2, 1:] *= -1
+            rows.append(blk)
+    x = np.concatenate(rows)
+    x = x[: x.shape[0] // 4 * 4].reshape(-1, 64)
+    # a whole-tensor amax equal to the block heads keeps s_g = 2^-8 (6 * 255 * 2^-8 < 2688 * 2^-8)
+    return x.astype(np.float32)
+
+
+def test_quantize_decisions_next_to_every_threshold(fs4):
+    x = _threshold_sweep()
+    want_c, want_s, want_g = Q.quantize_rows(x)
+    assert want_g == 2.0 ** -8
+    for tiled in (False, True):
+        c, s, g = _gpu_quant(fs4, x, 0, tiled, "pow2")
+        if tiled:
+            c, s, _, _ = tiled_to_plain(c, s, x.shape[0], x.shape[1])
+        assert g == want_g
+        assert np.array_equal(s, want_s)
+        assert np.array_equal(c, want_c), np.argwhere(c != want_c)[:5]
