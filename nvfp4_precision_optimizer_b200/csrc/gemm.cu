@@ -32,9 +32,16 @@ namespace {
 
 constexpr int BM = 128, BN = 256, BK = 256;
 constexpr int kStages = 3;
-constexpr int kThreads = 320;
+// 12 warps: warpgroup 0 = producer (warp 0), MMA issuer (warp 1), two idle warps;
+// warpgroups 1-2 = 8 epilogue warps.  Registers are rebalanced after launch:
+// 384 threads x 168 = 40 x 128 (warpgroup 0) + 232 x 256 (epilogue warpgroups).
+constexpr int kThreads = 384;
 constexpr int kEpiThreads = 256;
-constexpr int kEpiBase = 64;           // first epilogue thread
+constexpr int kEpiBase = 128;          // first epilogue thread
+constexpr uint32_t kRegsLaunch = 168;
+constexpr uint32_t kRegsCtl = 40;
+constexpr uint32_t kRegsEpi = 232;
+static_assert(kRegsCtl * 128 + kRegsEpi * 256 <= kRegsLaunch * kThreads, "register split over budget");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCol = 256;      // scale-factor columns follow the 256 accumulator columns
 constexpr uint32_t kSfBufCols = 48;   // 16 (A: 4 k-steps x 4) + 32 (B: 4 k-steps x 8)
@@ -224,6 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int64_t total = total_units<E>(p, g);
+  if (warp < 4) {
+    regs_dec<kRegsCtl>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -293,9 +302,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       volatile int never = 0;
       mbar_wait(mma_done, 0, status, &never);
     }
+  }
   } else {
+    regs_inc<kRegsEpi>();
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;          // 0..7
+    const int ew = warp - 4;          // 0..7
     const int quad = warp & 3;        // TMEM lanes 32*quad .. 32*quad+31
     const int ch = ew >> 2;           // column half of the 256-wide tile
     float* tb = trans + ew * TRANS_FLOATS;
@@ -340,14 +351,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         six_out = __fmul_rn(6.0f, sg_out);
       }
 
+      // drain this warp's 32 x 128 share of the accumulator into registers and hand
+      // the accumulator back at once: the next tile's MMAs overlap this epilogue
+      uint32_t accr[4][32];
+      const uint32_t taddr = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(128 * ch);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32_async(taddr + 32 * c, accr[c]);
+      tmem_wait_ld32(accr[0]);
+      tmem_ld_order(accr[1]);
+      tmem_ld_order(accr[2]);
+      tmem_ld_order(accr[3]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+
       float row_acc = 0.0f, amax = 0.0f;
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int64_t gc = j.col0 + 128 * ch + 32 * c;
         float v[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(128 * ch + 32 * c), v);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] *= acc_scale;
+        for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(accr[c][e]) * acc_scale;
 
         // FP32 tiles are read and written after a per-warp transpose (lane = column,
         // w[t] = row gr0 + t): every warp access is then one contiguous 128-byte line.
@@ -425,11 +449,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 
-      // accumulator drained: hand it back to the MMA warp
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
-
       if constexpr (E != Epi::Plain) {
         float* rowsum = nullptr;
         if constexpr (E == Epi::GramX) rowsum = reinterpret_cast<float*>(p.ws + L.rowsumA);
@@ -504,6 +523,12 @@ cudaError_t launch_impl(const NsParams* p, const GemmPlainArgs* g, int64_t units
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set |= 1ull << dev;
   }
+  // setmaxnreg.inc can only hand out what the block was launched with: refuse to
+  // launch unless the compiled register count is exactly the split's budget
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, nvfp4_gemm_kernel<E>);
+  if (e != cudaSuccess) return e;
+  if ((uint32_t)fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
   const int grid = (int)(units < num_sms ? (units > 0 ? units : 1) : num_sms);
   static const NsParams zero_p{};
   static const GemmPlainArgs zero_g{};
