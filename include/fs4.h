@@ -196,6 +196,31 @@ fs4_status fs4_root_ns_batched_timed(int32_t count, const fs4_ns_desc* descs, in
                                      size_t workspace_bytes, void* stream,
                                      void* const* phase_events, int32_t n_events);
 
+/* ------------------------------------------------------------ no-alloc variant */
+
+/* Bytes of the workspace array built into the library for fs4_root_ns_noalloc. */
+#define FS4_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* fs4_root_ns for callers that cannot allocate device memory (no counterpart in
+ * the paper; an interface addition).  Examples: code running while a stream is
+ * captured into a CUDA graph, where cudaMalloc is not allowed; plugins inside a
+ * host framework that owns all device memory and lends none; loops where a
+ * runtime allocation is forbidden.  Same arguments and result as fs4_root_ns
+ * with flags = 0, but the workspace is a fixed 16 MiB array compiled into the
+ * library (every device that loads the library holds it until the process
+ * exits).  Matrices whose fs4_root_ns_workspace_size(m, n) exceeds
+ * FS4_NOALLOC_SCRATCH_BYTES are rejected with FS4_ERR_WORKSPACE before anything
+ * is launched (1024 x 1024 needs 11.4 MiB and fits; 1024 x 2048 needs 17.6 MiB); other errors as fs4_root_ns.  The first call
+ * on each device looks up the array's device address with that device current
+ * (make it before any stream capture).  Every call shares the array and it keeps
+ * the last call's contents; each call clears what must start at zero, but calls
+ * whose work overlaps on the GPU race on it.  Device-side conditions (non-finite
+ * input: zero output) cannot be queried through fs4_device_status.  Allocates
+ * nothing. */
+fs4_status fs4_root_ns_noalloc(const float* G, int64_t m, int64_t n, int64_t ld, float* out,
+                               int64_t ld_out, int32_t K, float a, float b, float c,
+                               float clip_k, void* stream);
+
 /* Synchronise `stream` and return the device status recorded in `workspace`
  * by the last call that used it (FS4_OK, FS4_ERR_NONFINITE, FS4_ERR_TIMEOUT). */
 fs4_status fs4_device_status(const void* workspace, void* stream);
