@@ -314,7 +314,8 @@ def main():
         with open(tpath) as f:
             tr = json.load(f)
         ent = tr.get(args.workload, {}).get(dom)
-        if ent and ent.get("source_sha") == F._source_digest():
+        files = F.GEMM_SOURCES if dom in ("gram_x", "gram_a", "update") else F.ELEMENTWISE_SOURCES
+        if ent and ent.get("source_sha") == F._source_digest(files):
             roof["traffic"] = ent["bytes_per_launch"]
 
     value = world * len(Gs) / (ms_step * 1e-3)

@@ -185,14 +185,18 @@ def device_status(workspace: torch.Tensor, stream=None) -> int:
     return int(_lib.lib().fs4_device_status(workspace.data_ptr(), _stream(stream)))
 
 
-def _source_digest() -> str:
-    """Short hash of the CUDA sources (ties stored ncu counters to the code they measured)."""
+GEMM_SOURCES = ("gemm.cu", "fs4_device.cuh", "fs4_internal.h")
+ELEMENTWISE_SOURCES = ("kernels.cu", "fs4_device.cuh", "fs4_internal.h")
+
+
+def _source_digest(files=GEMM_SOURCES) -> str:
+    """Short hash of the CUDA sources that define a kernel (ties stored ncu counters
+    to the code they measured)."""
     import hashlib
     import os
     csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in sorted(files):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
