@@ -134,30 +134,49 @@ struct QBlock16 {
   uint32_t w0, w1;   // 16 codes, element 0 in the low nibble of w0
   uint32_t scale;    // E4M3 byte
   float sumsq;       // sum of the squared dequantised values
+  float amax;        // max |x| of the block
 };
 
+// Correctly rounded x / d from rcp = RN(1/d), by Markstein's FMA correction: the
+// residual x - q0 d of q0 = RN(x rcp) is exact and q0 + residual * rcp rounds to
+// RN(x / d).  Used where d has one of the eight 4-bit mantissas of an E4M3 value
+// times a power of two (decoded block scales and 6 s_g for a power-of-two s_g),
+// for which the identity is checked exhaustively, and |x / d| stays far from
+// the FP32 underflow and overflow ranges.
+__device__ __forceinline__ float div_rn_fma(float x, float d, float rcp) {
+  const float q0 = x * rcp;
+  return fmaf(fmaf(-q0, d, x), rcp, q0);
+}
+
 // Quantise 16 FP32 values with tensor scale s_g (six_sg = fp32(6 * s_g)).
-__device__ __forceinline__ QBlock16 quantize16(const float* x, float s_g, float six_sg) {
-  float amax = 0.0f;
+// kPow2: s_g is a power of two and rcp_six = RN(1 / six_sg), so the block scale
+// division may use the FMA-corrected form; otherwise IEEE division is used.
+template <bool kPow2>
+__device__ __forceinline__ QBlock16 quantize16(const float* x, float s_g, float six_sg, float rcp_six) {
+  // max |x| as a tree (depth 4 instead of a 16-long dependency chain)
+  float m8[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fabsf(x[i]), fabsf(x[i + 8]));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m8[i] = fmaxf(m8[i], m8[i + 4]);
+  const float amax = fmaxf(fmaxf(m8[0], m8[2]), fmaxf(m8[1], m8[3]));
   QBlock16 r;
-  r.scale = f32_to_e4m3(__fdiv_rn(amax, six_sg));
+  r.amax = amax;
+  r.scale = f32_to_e4m3(kPow2 ? div_rn_fma(amax, six_sg, rcp_six) : __fdiv_rn(amax, six_sg));
   const float den = __fmul_rn(e4m3_to_f32(r.scale), s_g);
   if (r.scale == 0u) {
     r.w0 = r.w1 = 0u;
     r.sumsq = 0.0f;
     return r;
   }
-  // x / den correctly rounded, by Markstein's FMA correction: with rcp = RN(1/den)
-  // and q0 = RN(x rcp), the residual x - q0 den is exact and q0 + residual * rcp
-  // rounds to RN(x / den) (no underflow/overflow here: |x / den| <= 6.2 or x = 0).
-  const float rcp = __frcp_rn(den);
   float q[16];
+  if (kPow2) {
+    const float rcp = __frcp_rn(den);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float q0 = x[i] * rcp;
-    q[i] = fmaf(fmaf(-q0, den, x[i]), rcp, q0);
+    for (int i = 0; i < 16; ++i) q[i] = div_rn_fma(x[i], den, rcp);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(x[i], den);
   }
   r.w0 = pack8_e2m1(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
   r.w1 = pack8_e2m1(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);

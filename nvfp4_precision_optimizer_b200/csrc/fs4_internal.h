@@ -22,8 +22,9 @@ struct NsState {
   double sumsq;            // sum of G^2 (float64)
   uint32_t amaxG;          // max |G| as float bits
   uint32_t nonfinite;      // G holds NaN or Inf
-  uint32_t done[4];        // finished work units per phase kind (preamble, G1, G2, G3)
-  uint32_t pad0[56];
+  uint32_t done[8];        // finished work units per phase kind (preamble, G1, G2, G3, reduce)
+  float inv0, tau0;        // fp32(1 / (||G|| + eps)) and the clip threshold (set after the reduction)
+  uint32_t pad0[50];
   float sg[192];           // tensor scales: X_k at [k], A_k at [64+k], B_k at [128+k]
   float u_rowX[64];        // max_i sum_j deq(qX_k)_ij^2
   float u_colX[64];        // max_j sum_i deq(qX16_k)_ij^2

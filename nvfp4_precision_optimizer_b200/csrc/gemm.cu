@@ -9,15 +9,21 @@
 // above the diagonal; an off-diagonal tile also writes the transposed view,
 // which is the mirrored tile's 1x16 quantisation (Q16x1(A) = Q1x16(A)^T).
 //
-// Kernel structure (one persistent CTA per SM, 320 threads):
+// Kernel structure (one persistent CTA per SM, 384 threads = 3 warpgroups):
 //   warp 0     producer: 1-D bulk copies (TMA engine) of pre-tiled operand tiles
 //              and scale atoms into a 3-stage shared-memory ring
 //   warp 1     allocates 512 TMEM columns; one thread copies the scale atoms to
 //              TMEM (tcgen05.cp) and issues tcgen05.mma kind::mxf4nvf4
 //              (M=128, N=256, K=64, UE4M3 per-16 scales), FP32 accumulator in TMEM
-//   warps 2-9  epilogue: tcgen05.ld of the 128 x 256 accumulator, the fused
-//              element-wise step, requantisation of the next operand, and
-//              the row/column sums the next phase's tensor scales are bounded by
+//   warp 2     tile counter: counts finished tiles per matrix and, in the CTA that
+//              finishes a matrix, derives the next phase's tensor scale
+//   warps 4-11 epilogue: tcgen05.ld of the 128 x 256 accumulator into registers
+//              (the accumulator is handed back to the MMA warp at once, so the
+//              next tile's MMAs overlap this epilogue), the fused element-wise
+//              step, requantisation of the next operand, and the row/column sums
+//              the next phase's tensor scales are bounded by
+// setmaxnreg moves registers from warpgroup 0 (control, 40 per thread) to the
+// two epilogue warpgroups (232 per thread).
 // Every mbarrier wait is bounded (see mbar_wait); on a timeout the CTA stops
 // issuing work, drains what it issued, frees TMEM and returns.
 #include <cfloat>
@@ -68,7 +74,7 @@ struct Job {
   int64_t ktiles_total;             // K tiles per operand row band (Kp / 256)
 };
 
-__device__ __forceinline__ int owner_of(const int32_t* prefix, int count, int64_t u) {
+__device__ __forceinline__ int owner_of(const int32_t* prefix, int count, int32_t u) {
   int lo = 0, hi = count - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -78,22 +84,23 @@ __device__ __forceinline__ int owner_of(const int32_t* prefix, int count, int64_
 }
 
 // Upper-triangle super tile s -> (P, Q), P <= Q, of a T x T grid, row-major.
-__device__ __forceinline__ void upper_tile(int64_t s, int64_t T, int64_t& P, int64_t& Q) {
+__device__ __forceinline__ void upper_tile(int32_t s, int32_t T, int32_t& P, int32_t& Q) {
   P = 0;
   while (s >= T - P) { s -= T - P; ++P; }
   Q = P + s;
 }
 
 template <Epi E>
-__device__ __forceinline__ Job make_job(int64_t u, const NsParams& p, const GemmPlainArgs& g) {
+__device__ __forceinline__ Job make_job(int32_t u, const NsParams& p, const GemmPlainArgs& g) {
   Job j;
   j.mirror = 0;
   j.b_half = 0;
   if constexpr (E == Epi::Plain) {
-    const int64_t nJ = (g.Np + BN - 1) / BN;
+    const int32_t nJ = (g.Np + BN - 1) / BN;
+    const int32_t I = u / nJ;
     j.mat = 0;
-    j.row0 = (u / nJ) * BM;
-    j.col0 = (u % nJ) * BN;
+    j.row0 = (int64_t)I * BM;
+    j.col0 = (int64_t)(u - I * nJ) * BN;
     j.b_half = (j.col0 + 128 >= g.Np) ? 1 : 0;
     j.kt = g.Kp / BK;
     j.ktiles_total = g.Kp / BK;
@@ -103,15 +110,15 @@ __device__ __forceinline__ Job make_job(int64_t u, const NsParams& p, const Gemm
     const int mi = owner_of(p.prefix, p.count, u);
     const MatDesc& d = p.mat[mi];
     const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
-    const int64_t lu = u - p.prefix[mi];
+    const int32_t lu = u - p.prefix[mi];
     const int slot = p.iter & 1;
     j.mat = mi;
     if constexpr (E == Epi::GramX || E == Epi::GramA) {
-      const int64_t T = d.mp / 256;
-      int64_t P, Q;
+      const int32_t T = d.mp / 256;
+      int32_t P, Q;
       upper_tile(lu >> 1, T, P, Q);
-      j.row0 = 256 * P + 128 * (lu & 1);
-      j.col0 = 256 * Q;
+      j.row0 = 256 * (int64_t)P + 128 * (lu & 1);
+      j.col0 = 256 * (int64_t)Q;
       j.mirror = (P != Q) ? 1 : 0;
       if constexpr (E == Epi::GramX) {
         j.kt = d.np / BK;
@@ -123,9 +130,10 @@ __device__ __forceinline__ Job make_job(int64_t u, const NsParams& p, const Gemm
         j.a_sf = j.b_sf = p.ws + L.sA;
       }
     } else {
-      const int64_t nJ = d.np / BN;
-      j.row0 = (lu / nJ) * BM;
-      j.col0 = (lu % nJ) * BN;
+      const int32_t nJ = d.np / BN;
+      const int32_t I = lu / nJ;
+      j.row0 = (int64_t)I * BM;
+      j.col0 = (int64_t)(lu - I * nJ) * BN;
       j.kt = d.mp / BK;
       j.a_codes = p.ws + L.qB; j.a_sf = p.ws + L.sB;
       j.b_codes = p.ws + (slot ? L.qXT[1] : L.qXT[0]);
@@ -139,49 +147,31 @@ __device__ __forceinline__ Job make_job(int64_t u, const NsParams& p, const Gemm
 }
 
 template <Epi E>
-__device__ __forceinline__ int64_t total_units(const NsParams& p, const GemmPlainArgs& g) {
+__device__ __forceinline__ int32_t total_units(const NsParams& p, const GemmPlainArgs& g) {
   if constexpr (E == Epi::Plain) {
-    return (int64_t)(g.Mp / BM) * ((g.Np + BN - 1) / BN);
+    return (g.Mp / BM) * ((g.Np + BN - 1) / BN);
   } else {
     return p.prefix[p.count];
   }
 }
 
-// Max of a value over the 256 epilogue threads (named barrier 2); valid in epilogue thread 0.
-__device__ __forceinline__ float epi_max(float v, float* red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  const int et = threadIdx.x - kEpiBase;
-  named_bar(2, kEpiThreads);
-  if ((et & 31) == 0) red[et >> 5] = v;
-  named_bar(2, kEpiThreads);
-  if (et == 0) {
-    v = red[0];
-    for (int k = 1; k < 8; ++k) v = fmaxf(v, red[k]);
-  }
-  return v;
-}
+struct ChunkSums {
+  float sumsq;   // sum of squared dequantised values of the 32 elements
+  float amax;    // max |x| of the 32 elements
+};
 
-__device__ __forceinline__ float epi_drain_max(float* vec, int64_t len, float* red) {
-  float m = 0.0f;
-  for (int64_t i = threadIdx.x - kEpiBase; i < len; i += kEpiThreads) {
-    m = fmaxf(m, __ldcg(vec + i));
-    __stcg(vec + i, 0.0f);
-  }
-  return epi_max(m, red);
-}
-
-// 1x16 quantisation of 32 consecutive values of row r starting at column c (c % 32 == 0).
-__device__ __forceinline__ float store_row_chunk(const float* v, int64_t r, int64_t c, int64_t Cp,
-                                                 uint8_t* codes, uint8_t* scales, float sg,
-                                                 float six) {
-  const QBlock16 q0 = quantize16(v, sg, six);
-  const QBlock16 q1 = quantize16(v + 16, sg, six);
+// 1x16 quantisation of 32 consecutive values of row r starting at column c (c % 32 == 0),
+// power-of-two tensor scale sg (six = 6 sg, rcp_six = RN(1 / six)).
+__device__ __forceinline__ ChunkSums store_row_chunk(const float* v, int64_t r, int64_t c, int64_t Cp,
+                                                     uint8_t* codes, uint8_t* scales, float sg,
+                                                     float six, float rcp_six) {
+  const QBlock16 q0 = quantize16<true>(v, sg, six, rcp_six);
+  const QBlock16 q1 = quantize16<true>(v + 16, sg, six, rcp_six);
   *reinterpret_cast<uint4*>(codes + tiled_chunk_offset(r, c, Cp)) =
       make_uint4(q0.w0, q0.w1, q1.w0, q1.w1);
   *reinterpret_cast<uint16_t*>(scales + tiled_scale_offset(r, c >> 4, Cp)) =
       static_cast<uint16_t>(q0.scale | (q1.scale << 8));
-  return q0.sumsq + q1.sumsq;
+  return {q0.sumsq + q1.sumsq, fmaxf(q0.amax, q1.amax)};
 }
 
 // Transpose this warp's 32 x 32 chunk through shared memory: on return w[t]
@@ -193,6 +183,77 @@ __device__ __forceinline__ void warp_transpose(const float* v, float* w, float* 
 #pragma unroll
   for (int t = 0; t < 32; ++t) w[t] = tb[t * 33 + lane];
   __syncwarp();
+}
+
+// Read-and-clear max of a float vector in global memory by one warp (values >= 0):
+// float4 loads, four in flight per lane.
+__device__ __forceinline__ float warp_drain_max4(float* vec, int64_t len, int lane) {
+  float m = 0.0f;
+  float4* v4 = reinterpret_cast<float4*>(vec);
+  const int64_t n4 = len >> 2;     // len is a multiple of 256
+  for (int64_t base = 0; base < n4; base += 128) {
+    float4 a[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int64_t i = base + k * 32 + lane;
+      a[k] = i < n4 ? __ldcg(v4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int64_t i = base + k * 32 + lane;
+      if (i < n4) __stcg(v4 + i, make_float4(0.f, 0.f, 0.f, 0.f));
+      m = fmaxf(m, fmaxf(fmaxf(a[k].x, a[k].y), fmaxf(a[k].z, a[k].w)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  return m;
+}
+
+// Count one finished tile of matrix mi; in the CTA that completes the matrix's
+// tiles of this launch, derive the next tensor scale from the row/column sums.
+template <Epi E>
+__device__ __forceinline__ void finalize_tile(const NsParams& p, int mi, int lane) {
+  if constexpr (E != Epi::Plain) {
+    const MatDesc& d = p.mat[mi];
+    NsState* st = reinterpret_cast<NsState*>(p.ws + d.state_off);
+    constexpr int kind = (E == Epi::GramX) ? 1 : (E == Epi::GramA ? 2 : 3);
+    int last = 0;
+    if (lane == 0) {
+      const uint32_t units = (uint32_t)(p.prefix[mi + 1] - p.prefix[mi]);
+      last = (atomicAdd(&st->done[kind], 1u) == units - 1u) ? 1 : 0;
+    }
+    last = __shfl_sync(0xFFFFFFFFu, last, 0);
+    if (!last) return;
+    __threadfence();
+    const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
+    const int k = p.iter;
+    if constexpr (E == Epi::GramX) {
+      const float ua = warp_drain_max4(reinterpret_cast<float*>(p.ws + L.rowsumA), d.mp, lane);
+      if (lane == 0) {
+        st->u_rowA[k] = ua;
+        const float ub = (fabsf(d.b) * __ldcg(&st->u_rowX[k]) + fabsf(d.c) * ua) * kBoundInflate;
+        st->sg[kSgB + k] = pow2_tensor_scale(ub);
+      }
+    } else if constexpr (E == Epi::GramA) {
+      const float ub = warp_drain_max4(reinterpret_cast<float*>(p.ws + L.rowsumB), d.mp, lane);
+      if (lane == 0) {
+        st->u_rowB[k] = ub;
+        const float ax = __uint_as_float(__ldcg(&st->amaxX[k]));
+        const float ux = (fabsf(d.a) * ax + sqrtf(ub * __ldcg(&st->u_colX[k]))) * kBoundInflate;
+        st->sg[kSgX + k + 1] = pow2_tensor_scale(ux);
+      }
+    } else {
+      const float ur = warp_drain_max4(reinterpret_cast<float*>(p.ws + L.rowsumX), d.mp, lane);
+      const float uc = warp_drain_max4(reinterpret_cast<float*>(p.ws + L.colsumX), d.np, lane);
+      if (lane == 0 && !p.last) {
+        st->u_rowX[k + 1] = ur;
+        st->u_colX[k + 1] = uc;
+        st->sg[kSgA + k + 1] = pow2_tensor_scale(ur * kBoundInflate);
+      }
+    }
+    if (lane == 0) st->done[kind] = 0u;
+  }
 }
 
 template <Epi E>
@@ -208,11 +269,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = bars + 2 * kStages;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* mma_done = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* s_last = reinterpret_cast<volatile int*>(tmem_slot + 2);
-  volatile int* s_go = reinterpret_cast<volatile int*>(tmem_slot + 3);
-  float* red = reinterpret_cast<float*>(tmem_slot + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 3);
+  uint32_t* arrivals = tmem_slot + 1;   // monotonic count of (epilogue warp, tile) completions
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   uint32_t* status = (E == Epi::Plain) ? g.status : p.status;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -222,6 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 8);
     mbar_init(mma_done, 1);
+    *arrivals = 0u;
     *abort_flag = (__ldcg(status) & kStatusTimeout) ? 1 : 0;
     fence_mbar_init();
   }
@@ -230,14 +290,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int64_t total = total_units<E>(p, g);
+  const int32_t total = total_units<E>(p, g);
   if (warp < 4) {
     regs_dec<kRegsCtl>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t it = 0;
-      for (int64_t u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
+      for (int32_t u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
         const Job j = make_job<E>(u, p, g);
         for (int kt = 0; kt < j.kt; ++kt, ++it) {
           const uint32_t s = it % kStages, use = it / kStages;
@@ -268,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t it = 0, tl = 0;
       const uint32_t acc = tmem;   // lane 0, column 0
-      for (int64_t u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++tl) {
+      for (int32_t u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++tl) {
         const Job j = make_job<E>(u, p, g);
         if (!mbar_wait(acc_empty, (tl & 1u) ^ 1u, status, abort_flag)) break;
         tc_fence_after();
@@ -302,29 +362,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       volatile int never = 0;
       mbar_wait(mma_done, 0, status, &never);
     }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ tile counter / finalizer
+    // Trails the epilogue warps: once all eight have published tile tl's sums, count
+    // the tile for its matrix; the CTA that finishes a matrix's last tile in this
+    // launch turns the matrix's sums into the next tensor scale.  The epilogue warps
+    // never wait for this warp.
+    if constexpr (E != Epi::Plain) {
+      uint32_t tl = 0;
+      for (int32_t u = blockIdx.x; u < total; u += gridDim.x, ++tl) {
+        const Job j = make_job<E>(u, p, g);
+        const uint32_t target = 8u * (tl + 1u);
+        bool seen = true;
+        if (*reinterpret_cast<volatile uint32_t*>(arrivals) < target) {
+          const uint64_t t0 = global_timer_ns();
+          while (*reinterpret_cast<volatile uint32_t*>(arrivals) < target) {
+            if (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs) { seen = false; break; }
+            __nanosleep(64);
+          }
+        }
+        if (!seen) {
+          if (lane == 0 && !*abort_flag) { atomicOr(status, kStatusTimeout); *abort_flag = 1; }
+          break;
+        }
+        __threadfence();
+        finalize_tile<E>(p, j.mat, lane);
+      }
+    }
   }
   } else {
     regs_inc<kRegsEpi>();
     // ------------------------------------------------------------ epilogue
+    // Every epilogue warp walks the same tile list and never leaves it early (a
+    // failed wait only skips that tile's work), so the block-wide barrier at the
+    // end is reached by all threads.  Per tile, each warp fences its row/column
+    // sum atomics and bumps the shared arrival counter that warp 2 trails.
     const int ew = warp - 4;          // 0..7
     const int quad = warp & 3;        // TMEM lanes 32*quad .. 32*quad+31
     const int ch = ew >> 2;           // column half of the 256-wide tile
     float* tb = trans + ew * TRANS_FLOATS;
     uint32_t tl = 0;
-    for (int64_t u = blockIdx.x; u < total; u += gridDim.x, ++tl) {
+    for (int32_t u = blockIdx.x; u < total; u += gridDim.x, ++tl) {
       const Job j = make_job<E>(u, p, g);
-      // every epilogue warp takes the same go / stop decision (they share named barriers)
-      mbar_wait(acc_full, tl & 1u, status, abort_flag);
-      named_bar(1, kEpiThreads);
-      if (threadIdx.x == kEpiBase) *s_go = *abort_flag ? 0 : 1;
-      named_bar(1, kEpiThreads);
-      if (!*s_go) break;
-      tc_fence_after();
+      const bool ok = mbar_wait(acc_full, tl & 1u, status, abort_flag);
       const int64_t gr0 = j.row0 + 32 * quad;   // first row of this warp's band
       const int64_t gr = gr0 + lane;             // this lane's row
 
       // per-job constants
-      float acc_scale, sg_out = 1.0f, six_out = 6.0f, coef_a = 0.0f, coef_b = 0.0f, coef_c = 0.0f;
+      float acc_scale, sg_out = 1.0f, six_out = 6.0f, rcp_six = 1.0f / 6.0f;
+      float coef_a = 0.0f, coef_b = 0.0f, coef_c = 0.0f;
       const MatDesc* d = nullptr;
       NsState* st = nullptr;
       MatLayout L;
@@ -349,102 +435,107 @@ __global__ void __launch_bounds__(kThreads, 1)
           sg_out = p.last ? 1.0f : __ldcg(&st->sg[kSgX + k + 1]);
         }
         six_out = __fmul_rn(6.0f, sg_out);
+        rcp_six = __frcp_rn(six_out);
       }
 
-      // drain this warp's 32 x 128 share of the accumulator into registers and hand
-      // the accumulator back at once: the next tile's MMAs overlap this epilogue
-      uint32_t accr[4][32];
-      const uint32_t taddr = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(128 * ch);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32_async(taddr + 32 * c, accr[c]);
-      tmem_wait_ld32(accr[0]);
-      tmem_ld_order(accr[1]);
-      tmem_ld_order(accr[2]);
-      tmem_ld_order(accr[3]);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
-
       float row_acc = 0.0f, amax = 0.0f;
+      if (ok) {
+        tc_fence_after();
+        // drain this warp's 32 x 128 share of the accumulator into registers and hand
+        // the accumulator back at once: the next tile's MMAs overlap this epilogue
+        uint32_t accr[4][32];
+        const uint32_t taddr = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(128 * ch);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int64_t gc = j.col0 + 128 * ch + 32 * c;
-        float v[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(accr[c][e]) * acc_scale;
+        for (int c = 0; c < 4; ++c) tmem_ld32_async(taddr + 32 * c, accr[c]);
+        tmem_wait_ld32(accr[0]);
+        tmem_ld_order(accr[1]);
+        tmem_ld_order(accr[2]);
+        tmem_ld_order(accr[3]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
 
-        // FP32 tiles are read and written after a per-warp transpose (lane = column,
-        // w[t] = row gr0 + t): every warp access is then one contiguous 128-byte line.
-        if constexpr (E == Epi::Plain) {
-          float w[32];
-          warp_transpose(v, w, tb, lane);
-          const int64_t col = gc + lane;
-          if (col < g.N) {
 #pragma unroll
-            for (int t = 0; t < 32; ++t)
-              if (gr0 + t < g.M) g.d[(gr0 + t) * g.ldd + col] = w[t];
-          }
-        } else if constexpr (E == Epi::GramX) {
-          row_acc += store_row_chunk(v, gr, gc, d->mp, p.ws + L.qA, p.ws + L.sA, sg_out, six_out);
-          float w[32];
-          warp_transpose(v, w, tb, lane);
-          float* Acol = reinterpret_cast<float*>(p.ws + L.A) + gr0 * d->mp + gc + lane;
+        for (int c = 0; c < 4; ++c) {
+          const int64_t gc = j.col0 + 128 * ch + 32 * c;
+          float v[32];
 #pragma unroll
-          for (int t = 0; t < 32; ++t) Acol[t * d->mp] = w[t];
-          if (j.mirror) {
-            const float cs = store_row_chunk(w, gc + lane, gr0, d->mp, p.ws + L.qA, p.ws + L.sA,
-                                             sg_out, six_out);
-            if (cs != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.rowsumA) + gc + lane, cs);
-          }
-        } else if constexpr (E == Epi::GramA) {
-          const float* Acol = reinterpret_cast<const float*>(p.ws + L.A) + gr0 * d->mp + gc + lane;
-          float w[32], a_row[32];
-#pragma unroll
-          for (int t = 0; t < 32; ++t) w[t] = __ldcg(Acol + t * d->mp);
-          warp_transpose(w, a_row, tb, lane);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = fmaf(coef_b, a_row[e], coef_c * v[e]);
-          row_acc += store_row_chunk(v, gr, gc, d->mp, p.ws + L.qB, p.ws + L.sB, sg_out, six_out);
-          if (j.mirror) {
+          for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(accr[c][e]) * acc_scale;
+
+          // FP32 tiles are read and written after a per-warp transpose (lane = column,
+          // w[t] = row gr0 + t): every warp access is then one contiguous 128-byte line.
+          if constexpr (E == Epi::Plain) {
+            float w[32];
             warp_transpose(v, w, tb, lane);
-            const float cs = store_row_chunk(w, gc + lane, gr0, d->mp, p.ws + L.qB, p.ws + L.sB,
-                                             sg_out, six_out);
-            if (cs != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.rowsumB) + gc + lane, cs);
-          }
-        } else {  // Update
-          float w[32];
-          warp_transpose(v, w, tb, lane);
-          float* Xcol = reinterpret_cast<float*>(p.ws + L.X) + gr0 * d->np + gc + lane;
+            const int64_t col = gc + lane;
+            if (col < g.N) {
+              float* dcol = g.d + gr0 * g.ldd + col;
 #pragma unroll
-          for (int t = 0; t < 32; ++t) w[t] = fmaf(coef_a, __ldcg(Xcol + t * d->np), w[t]);
-          if (p.last) {
-            if (!d->tall) {
-              if (gc + lane < d->n) {
+              for (int t = 0; t < 32; ++t)
+                if (gr0 + t < g.M) dcol[t * g.ldd] = w[t];
+            }
+          } else if constexpr (E == Epi::GramX) {
+            row_acc += store_row_chunk(v, gr, gc, d->mp, p.ws + L.qA, p.ws + L.sA, sg_out, six_out, rcp_six).sumsq;
+            float w[32];
+            warp_transpose(v, w, tb, lane);
+            float* Acol = reinterpret_cast<float*>(p.ws + L.A) + gr0 * d->mp + gc + lane;
 #pragma unroll
-                for (int t = 0; t < 32; ++t)
-                  if (gr0 + t < d->m) d->out[(gr0 + t) * d->ldo + gc + lane] = w[t];
+            for (int t = 0; t < 32; ++t) Acol[t * d->mp] = w[t];
+            if (j.mirror) {
+              const float cs = store_row_chunk(w, gc + lane, gr0, d->mp, p.ws + L.qA, p.ws + L.sA,
+                                               sg_out, six_out, rcp_six).sumsq;
+              if (cs != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.rowsumA) + gc + lane, cs);
+            }
+          } else if constexpr (E == Epi::GramA) {
+            const float* Acol = reinterpret_cast<const float*>(p.ws + L.A) + gr0 * d->mp + gc + lane;
+            float w[32], a_row[32];
+#pragma unroll
+            for (int t = 0; t < 32; ++t) w[t] = __ldcg(Acol + t * d->mp);
+            warp_transpose(w, a_row, tb, lane);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = fmaf(coef_b, a_row[e], coef_c * v[e]);
+            row_acc += store_row_chunk(v, gr, gc, d->mp, p.ws + L.qB, p.ws + L.sB, sg_out, six_out, rcp_six).sumsq;
+            if (j.mirror) {
+              warp_transpose(v, w, tb, lane);
+              const float cs = store_row_chunk(w, gc + lane, gr0, d->mp, p.ws + L.qB, p.ws + L.sB,
+                                               sg_out, six_out, rcp_six).sumsq;
+              if (cs != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.rowsumB) + gc + lane, cs);
+            }
+          } else {  // Update
+            float* Xcol = reinterpret_cast<float*>(p.ws + L.X) + gr0 * d->np + gc + lane;
+            float w[32];
+            warp_transpose(v, w, tb, lane);
+#pragma unroll
+            for (int t = 0; t < 32; ++t) w[t] = fmaf(coef_a, __ldcg(Xcol + t * d->np), w[t]);
+            if (p.last) {
+              if (!d->tall) {
+                if (gc + lane < d->n) {
+                  float* ocol = d->out + gr0 * d->ldo + gc + lane;
+#pragma unroll
+                  for (int t = 0; t < 32; ++t)
+                    if (gr0 + t < d->m) ocol[t * d->ldo] = w[t];
+                }
+              } else {
+                warp_transpose(w, v, tb, lane);
+                if (gr < d->m) {
+#pragma unroll
+                  for (int e = 0; e < 32; ++e)
+                    if (gc + e < d->n) d->out[(gc + e) * d->ldo + gr] = v[e];
+                }
               }
             } else {
+#pragma unroll
+              for (int t = 0; t < 32; ++t) Xcol[t * d->np] = w[t];
+              const int ns = (k + 1) & 1;
+              const ChunkSums cs = store_row_chunk(w, gc + lane, gr0, d->mp,
+                                                   p.ws + (ns ? L.qXT[1] : L.qXT[0]),
+                                                   p.ws + (ns ? L.sXT[1] : L.sXT[0]), sg_out, six_out, rcp_six);
+              amax = fmaxf(amax, cs.amax);
+              if (cs.sumsq != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.colsumX) + gc + lane, cs.sumsq);
               warp_transpose(w, v, tb, lane);
-              if (gr < d->m) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                  if (gc + e < d->n) d->out[(gc + e) * d->ldo + gr] = v[e];
-              }
+              row_acc += store_row_chunk(v, gr, gc, d->np, p.ws + (ns ? L.qX[1] : L.qX[0]),
+                                         p.ws + (ns ? L.sX[1] : L.sX[0]), sg_out, six_out, rcp_six).sumsq;
             }
-          } else {
-#pragma unroll
-            for (int t = 0; t < 32; ++t) {
-              Xcol[t * d->np] = w[t];
-              amax = fmaxf(amax, fabsf(w[t]));
-            }
-            const int ns = (k + 1) & 1;
-            const float cs = store_row_chunk(w, gc + lane, gr0, d->mp, p.ws + (ns ? L.qXT[1] : L.qXT[0]),
-                                             p.ws + (ns ? L.sXT[1] : L.sXT[0]), sg_out, six_out);
-            if (cs != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.colsumX) + gc + lane, cs);
-            warp_transpose(w, v, tb, lane);
-            row_acc += store_row_chunk(v, gr, gc, d->np, p.ws + (ns ? L.qX[1] : L.qX[0]),
-                                       p.ws + (ns ? L.sX[1] : L.sX[0]), sg_out, six_out);
           }
         }
       }
@@ -458,46 +549,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (E == Epi::Update) {
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-          if (lane == 0 && !p.last) atomicMax(&st->amaxX[k + 1], __float_as_uint(amax));
+          if (lane == 0 && !p.last && amax > 0.0f) atomicMax(&st->amaxX[k + 1], __float_as_uint(amax));
         }
-        // the last CTA to finish a tile of this matrix derives the next tensor scale;
-        // every thread fences its own (fire-and-forget) sum atomics before the count
-        constexpr int kind = (E == Epi::GramX) ? 1 : (E == Epi::GramA ? 2 : 3);
+        // publish this warp's sums for the counter warp (never waits)
         __threadfence();
-        named_bar(1, kEpiThreads);
-        if (threadIdx.x == kEpiBase) {
-          const uint32_t units = (uint32_t)(p.prefix[j.mat + 1] - p.prefix[j.mat]);
-          *s_last = (atomicAdd(&st->done[kind], 1u) == units - 1u) ? 1 : 0;
-        }
-        named_bar(1, kEpiThreads);
-        if (*s_last) {
-          __threadfence();
-          if constexpr (E == Epi::GramX) {
-            const float ua = epi_drain_max(rowsum, d->mp, red);
-            if (threadIdx.x == kEpiBase) {
-              st->u_rowA[k] = ua;
-              const float ub = (fabsf(coef_b) * __ldcg(&st->u_rowX[k]) + fabsf(coef_c) * ua) * kBoundInflate;
-              st->sg[kSgB + k] = pow2_tensor_scale(ub);
-            }
-          } else if constexpr (E == Epi::GramA) {
-            const float ub = epi_drain_max(rowsum, d->mp, red);
-            if (threadIdx.x == kEpiBase) {
-              st->u_rowB[k] = ub;
-              const float ax = __uint_as_float(__ldcg(&st->amaxX[k]));
-              const float ux = (fabsf(coef_a) * ax + sqrtf(ub * __ldcg(&st->u_colX[k]))) * kBoundInflate;
-              st->sg[kSgX + k + 1] = pow2_tensor_scale(ux);
-            }
-          } else {
-            const float ur = epi_drain_max(rowsum, d->mp, red);
-            const float uc = epi_drain_max(reinterpret_cast<float*>(p.ws + L.colsumX), d->np, red);
-            if (threadIdx.x == kEpiBase && !p.last) {
-              st->u_rowX[k + 1] = ur;
-              st->u_colX[k + 1] = uc;
-              st->sg[kSgA + k + 1] = pow2_tensor_scale(ur * kBoundInflate);
-            }
-          }
-          if (threadIdx.x == kEpiBase) st->done[kind] = 0u;
-        }
+        __syncwarp();
+        if (lane == 0) atomicAdd(arrivals, 1u);
       }
     }
   }

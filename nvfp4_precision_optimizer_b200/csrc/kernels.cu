@@ -24,7 +24,7 @@ __device__ __forceinline__ bool is_finite_bits(float v) {
 }
 
 // Index of the matrix that owns work unit u (prefix is ascending, prefix[0] == 0).
-__device__ __forceinline__ int owner_of(const int32_t* prefix, int count, int64_t u) {
+__device__ __forceinline__ int owner_of(const int32_t* prefix, int count, int32_t u) {
   int lo = 0, hi = count - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -59,12 +59,19 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return v;
 }
 
-// Read-and-clear max of a float vector in global memory (values >= 0), block-wide.
+// Read-and-clear max of a float vector in global memory (values >= 0), block-wide;
+// len is a multiple of 4 and vec 16-byte aligned.  Result valid in thread 0.
 __device__ float drain_max(float* vec, int64_t len, float* red) {
   float m = 0.0f;
-  for (int64_t i = threadIdx.x; i < len; i += kEwThreads) {
-    m = fmaxf(m, __ldcg(vec + i));
-    __stcg(vec + i, 0.0f);
+  float4* v4 = reinterpret_cast<float4*>(vec);
+  const int32_t n4 = (int32_t)(len >> 2);
+  for (int32_t i = threadIdx.x; i < n4; i += 2 * kEwThreads) {
+    const bool two = i + kEwThreads < n4;
+    const float4 a = __ldcg(v4 + i);
+    const float4 b = two ? __ldcg(v4 + i + kEwThreads) : make_float4(0.f, 0.f, 0.f, 0.f);
+    __stcg(v4 + i, make_float4(0.f, 0.f, 0.f, 0.f));
+    if (two) __stcg(v4 + i + kEwThreads, make_float4(0.f, 0.f, 0.f, 0.f));
+    m = fmaxf(m, fmaxf(fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w)), fmaxf(fmaxf(b.x, b.y), fmaxf(b.z, b.w))));
   }
   return block_max(m, red);
 }
@@ -118,6 +125,7 @@ __global__ void __launch_bounds__(kEwThreads) quantize_kernel(
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) *s_g_out = s_g;
   const float six_sg = __fmul_rn(6.0f, s_g);
+  const float rcp_six = __frcp_rn(six_sg);
 
   const int t = threadIdx.x;
   // stage: thread t covers 16 consecutive elements of one line of x
@@ -145,7 +153,8 @@ __global__ void __launch_bounds__(kEwThreads) quantize_kernel(
   float v[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) v[e] = tile[r][cb + e];
-  const QBlock16 q = quantize16(v, s_g, six_sg);
+  const QBlock16 q = sg_amax_mode ? quantize16<false>(v, s_g, six_sg, rcp_six)
+                                  : quantize16<true>(v, s_g, six_sg, rcp_six);
   if (tiled) {
     store_block_tiled(codes, scales, i, j, Cp, q);
   } else if (i < R && j < C) {
@@ -203,42 +212,77 @@ __device__ __forceinline__ NsState* state_of(const NsParams& p, const MatDesc& d
 }
 
 // Sum of G^2 (float64), max |G| and a non-finite flag per matrix; work unit =
-// 16 rows of one matrix in the caller's orientation.
+// 16 rows of one matrix in the caller's orientation.  The last CTA to finish a
+// matrix derives its normalisation and clip scalars and the tensor scale of X_0
+// (Section 3.4: normalise, clip, quantise), so the preamble only reads them.
 __global__ void __launch_bounds__(kEwThreads) ns_reduce_kernel(const __grid_constant__ NsParams p) {
   __shared__ float redf[kEwThreads / 32];
   __shared__ double redd[kEwThreads / 32];
-  const int64_t total = p.prefix[p.count];
-  for (int64_t u = blockIdx.x; u < total; u += gridDim.x) {
+  const int32_t total = p.prefix[p.count];
+  for (int32_t u = blockIdx.x; u < total; u += gridDim.x) {
     const int mi = owner_of(p.prefix, p.count, u);
     const MatDesc& d = p.mat[mi];
     const int64_t rows0 = d.tall ? d.n : d.m, cols0 = d.tall ? d.m : d.n;
     const int64_t r0 = (u - p.prefix[mi]) * 16;
+    const bool vec = ((reinterpret_cast<uintptr_t>(d.G) & 15) == 0) && ((d.ldg & 3) == 0);
     double s = 0.0;
     float mx = 0.0f;
     bool bad = false;
     for (int64_t r = r0; r < r0 + 16 && r < rows0; ++r) {
       const float* row = d.G + r * d.ldg;
-      for (int64_t c = threadIdx.x; c < cols0; c += kEwThreads) {
-        const float v = __ldg(row + c);
-        bad |= !is_finite_bits(v);
-        mx = fmaxf(mx, fabsf(v));
-        s += (double)v * (double)v;
+      if (vec) {
+        for (int64_t c = 4 * threadIdx.x; c < cols0; c += 4 * kEwThreads) {
+          const float4 v4 = __ldg(reinterpret_cast<const float4*>(row + c));
+          const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            bad |= !is_finite_bits(vv[e]);
+            mx = fmaxf(mx, fabsf(vv[e]));
+            s += (double)vv[e] * (double)vv[e];
+          }
+        }
+      } else {
+        for (int64_t c = threadIdx.x; c < cols0; c += kEwThreads) {
+          const float v = __ldg(row + c);
+          bad |= !is_finite_bits(v);
+          mx = fmaxf(mx, fabsf(v));
+          s += (double)v * (double)v;
+        }
       }
     }
     NsState* st = state_of(p, d);
-    if (__syncthreads_or(bad) && threadIdx.x == 0) {
-      atomicOr(&st->nonfinite, 1u);
-      atomicOr(p.status, kStatusNonFinite);
-    }
+    const bool any_bad = __syncthreads_or(bad);
     s = warp_sum(s);
     const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
     if (l == 0) redd[w] = s;
     mx = block_max(mx, redf);  // contains __syncthreads, orders the redd writes
     if (threadIdx.x == 0) {
+      if (any_bad) {
+        atomicOr(&st->nonfinite, 1u);
+        atomicOr(p.status, kStatusNonFinite);
+      }
       double tot = 0.0;
       for (int k = 0; k < kEwThreads / 32; ++k) tot += redd[k];
       atomicAdd(&st->sumsq, tot);
       atomicMax(&st->amaxG, __float_as_uint(mx));
+      __threadfence();
+      const uint32_t units = (uint32_t)(p.prefix[mi + 1] - p.prefix[mi]);
+      if (atomicAdd(&st->done[4], 1u) == units - 1u) {
+        __threadfence();
+        const bool dead = __ldcg(&st->nonfinite) != 0u;
+        const double norm = sqrt(__ldcg(&st->sumsq));
+        const float inv = dead ? 0.0f : (float)(1.0 / (norm + 1e-7));
+        float tau = FLT_MAX;
+        if (p.clip_k > 0.0f)
+          tau = (float)((double)p.clip_k * norm * (double)inv / sqrt((double)d.m * (double)d.n));
+        const float amaxG = __uint_as_float(__ldcg(&st->amaxG));
+        const float amax0 = dead ? 0.0f : fminf(__fmul_rn(amaxG, inv), tau);
+        st->inv0 = inv;
+        st->tau0 = tau;
+        st->sg[kSgX + 0] = pow2_tensor_scale(amax0);
+        st->amaxX[0] = __float_as_uint(amax0);
+        st->done[4] = 0u;
+      }
     }
     __syncthreads();
   }
@@ -246,105 +290,110 @@ __global__ void __launch_bounds__(kEwThreads) ns_reduce_kernel(const __grid_cons
 
 // Normalise, clip and quantise: X0 = clamp(fp32(G * inv), +-tau) written as FP32
 // and as both NVFP4 views, with row / column sums of the squared dequantised
-// values.  Work unit = one 64 x 64 tile of the padded working extent.
+// values.  Work unit = one 64 x 64 tile of the padded working extent; G and X
+// are read and written as float4 with 16 threads per 64-float row segment.
 __global__ void __launch_bounds__(kEwThreads) ns_preamble_kernel(const __grid_constant__ NsParams p) {
   __shared__ float tile[kT][kT + 1];
   __shared__ float red[kEwThreads / 32];
   __shared__ int s_last;
-  const int64_t total = p.prefix[p.count];
+  const int32_t total = p.prefix[p.count];
   const int t = threadIdx.x;
-  for (int64_t u = blockIdx.x; u < total; u += gridDim.x) {
+  for (int32_t u = blockIdx.x; u < total; u += gridDim.x) {
     const int mi = owner_of(p.prefix, p.count, u);
     const MatDesc& d = p.mat[mi];
     NsState* st = state_of(p, d);
     const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
-    const int64_t tiles_n = d.np / kT;
-    const int64_t lu = u - p.prefix[mi];
-    const int64_t i0 = (lu / tiles_n) * kT, j0 = (lu % tiles_n) * kT;
+    const int32_t tiles_n = d.np / kT;
+    const int32_t lu = u - p.prefix[mi];
+    const int32_t ti = lu / tiles_n;                       // 32-bit: units < 2^31
+    const int32_t i0 = ti * kT, j0 = (lu - ti * tiles_n) * kT;
 
-    // scalars of this matrix (identical in every CTA)
+    // scalars of this matrix, derived once by the reduction kernel
     const bool dead = __ldcg(&st->nonfinite) != 0u;
-    const double norm = sqrt(__ldcg(&st->sumsq));
-    const float inv = dead ? 0.0f : (float)(1.0 / (norm + 1e-7));
-    float tau = FLT_MAX;
-    if (p.clip_k > 0.0f)
-      tau = (float)((double)p.clip_k * norm * (double)inv / sqrt((double)d.m * (double)d.n));
-    const float amaxG = __uint_as_float(__ldcg(&st->amaxG));
-    const float amax0 = dead ? 0.0f : fminf(__fmul_rn(amaxG, inv), tau);
-    const float sg = pow2_tensor_scale(amax0);
+    const float inv = __ldcg(&st->inv0), tau = __ldcg(&st->tau0);
+    const float sg = __ldcg(&st->sg[kSgX + 0]);
     const float six_sg = __fmul_rn(6.0f, sg);
-    if (lu == 0 && t == 0) {
-      st->sg[kSgX + 0] = sg;
-      st->amaxX[0] = __float_as_uint(amax0);
-    }
+    const float rcp_six = __frcp_rn(six_sg);
+    const bool vec = ((reinterpret_cast<uintptr_t>(d.G) & 15) == 0) && ((d.ldg & 3) == 0);
 
-    // stage X0 tile (working orientation) in shared memory
-    {
-      const int line = t >> 2, part = (t & 3) * 16;
-      if (!d.tall) {
-        const int64_t i = i0 + line;
+    // stage the X0 tile (working orientation) in shared memory; a matrix with a
+    // non-finite entry is carried as all zeros (its output is zero)
+    const int32_t rows_g = d.tall ? d.n : d.m, cols_g = d.tall ? d.m : d.n;
+    const int32_t gr0 = d.tall ? j0 : i0, gc0 = d.tall ? i0 : j0;   // tile origin in G
+    const bool interior = vec && !dead && gr0 + kT <= rows_g && gc0 + kT <= cols_g;
+    const float* gtile = d.G + (int64_t)gr0 * d.ldg + gc0;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int64_t j = j0 + part + e;
-          float v = 0.0f;
-          if (!dead && i < d.m && j < d.n) v = fminf(fmaxf(__fmul_rn(__ldg(d.G + i * d.ldg + j), inv), -tau), tau);
-          tile[line][part + e] = v;
-        }
-      } else {  // X[i][j] = G[j][i]
-        const int64_t j = j0 + line;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int f = t + kEwThreads * pass;
+      const int line = f >> 4, c4 = (f & 15) * 4;       // 64 lines of 64 floats
+      float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      if (interior) {
+        const float4 x4 = __ldg(reinterpret_cast<const float4*>(gtile + (int64_t)line * d.ldg + c4));
+        v[0] = x4.x; v[1] = x4.y; v[2] = x4.z; v[3] = x4.w;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int64_t i = i0 + part + e;
-          float v = 0.0f;
-          if (!dead && i < d.m && j < d.n) v = fminf(fmaxf(__fmul_rn(__ldg(d.G + j * d.ldg + i), inv), -tau), tau);
-          tile[part + e][line] = v;
-        }
+        for (int e = 0; e < 4; ++e) v[e] = fminf(fmaxf(__fmul_rn(v[e], inv), -tau), tau);
+      } else if (!dead && gr0 + line < rows_g) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (gc0 + c4 + e < cols_g)
+            v[e] = fminf(fmaxf(__fmul_rn(__ldg(gtile + (int64_t)line * d.ldg + c4 + e), inv), -tau), tau);
+      }
+      // non-tall: line = row i of X; tall: line = row j of G = column j of X
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (!d.tall) tile[line][c4 + e] = v[e];
+        else tile[c4 + e][line] = v[e];
       }
     }
     __syncthreads();
-    // a matrix with a non-finite entry is carried as all zeros (its output is zero)
-    float* X = reinterpret_cast<float*>(p.ws + L.X);
-    {
-      const int r = t >> 2, cb = (t & 3) * 16;
-      const int64_t i = i0 + r, j = j0 + cb;
-      float v[16];
+    float* Xt = reinterpret_cast<float*>(p.ws + L.X) + (int64_t)i0 * d.np + j0;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = tile[r][cb + e];
-      float4* dst = reinterpret_cast<float4*>(X + i * d.np + j);
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
-      // 1x16 view (Gram operand): rows of X
-      const QBlock16 q = quantize16(v, sg, six_sg);
-      store_block_tiled(p.ws + L.qX[0], p.ws + L.sX[0], i, j, d.np, q);
-      float rs = q.sumsq;
-      rs += __shfl_xor_sync(0xFFFFFFFFu, rs, 1);
-      rs += __shfl_xor_sync(0xFFFFFFFFu, rs, 2);
-      if ((t & 3) == 0 && rs != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.rowsumX) + i, rs);
+    for (int pass = 0; pass < 4; ++pass) {
+      const int f = t + kEwThreads * pass;
+      const int r = f >> 4, c4 = (f & 15) * 4;
+      *reinterpret_cast<float4*>(Xt + r * d.np + c4) =
+          make_float4(tile[r][c4], tile[r][c4 + 1], tile[r][c4 + 2], tile[r][c4 + 3]);
     }
-    {
-      // 16x1 view (update operand), stored as the 1x16 quantisation of X^T
-      const int c = t >> 2, rb = (t & 3) * 16;
-      const int64_t j = j0 + c, i = i0 + rb;
+    // two views; thread t owns one 16-element block of line t/4 (four blocks per line)
+#pragma unroll
+    for (int view = 0; view < 2; ++view) {
+      const int line = t >> 2, blk = t & 3;
       float v[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = tile[rb + e][c];
-      const QBlock16 q = quantize16(v, sg, six_sg);
-      store_block_tiled(p.ws + L.qXT[0], p.ws + L.sXT[0], j, i, d.mp, q);
-      float cs = q.sumsq;
-      cs += __shfl_xor_sync(0xFFFFFFFFu, cs, 1);
-      cs += __shfl_xor_sync(0xFFFFFFFFu, cs, 2);
-      if ((t & 3) == 0 && cs != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.colsumX) + j, cs);
+      for (int e = 0; e < 16; ++e) v[e] = view == 0 ? tile[line][blk * 16 + e] : tile[blk * 16 + e][line];
+      const QBlock16 q = quantize16<true>(v, sg, six_sg, rcp_six);
+      // row (view 0: row i0+line of X, K = j0..) or row j0+line of X^T (view 1, K = i0..)
+      const int64_t R = (view == 0 ? i0 : j0) + line;
+      const int64_t K0 = view == 0 ? j0 : i0;
+      const int64_t Cp = view == 0 ? d.np : d.mp;
+      uint8_t* codes = p.ws + (view == 0 ? L.qX[0] : L.qXT[0]);
+      uint8_t* scales = p.ws + (view == 0 ? L.sX[0] : L.sXT[0]);
+      // pair blocks (0,1) and (2,3) into 16-byte chunks, the four scales into one word
+      const uint32_t o0 = __shfl_xor_sync(0xFFFFFFFFu, q.w0, 1);
+      const uint32_t o1 = __shfl_xor_sync(0xFFFFFFFFu, q.w1, 1);
+      uint32_t sc = q.scale << (8 * blk);
+      sc |= __shfl_xor_sync(0xFFFFFFFFu, sc, 1);
+      sc |= __shfl_xor_sync(0xFFFFFFFFu, sc, 2);
+      if ((blk & 1) == 0)
+        *reinterpret_cast<uint4*>(codes + tiled_chunk_offset(R, K0 + blk * 16, Cp)) =
+            make_uint4(q.w0, q.w1, o0, o1);
+      if (blk == 0) *reinterpret_cast<uint32_t*>(scales + tiled_scale_offset(R, K0 >> 4, Cp)) = sc;
+      float ss = q.sumsq;
+      ss += __shfl_xor_sync(0xFFFFFFFFu, ss, 1);
+      ss += __shfl_xor_sync(0xFFFFFFFFu, ss, 2);
+      if (blk == 0 && ss != 0.0f)
+        atomicAdd(reinterpret_cast<float*>(p.ws + (view == 0 ? L.rowsumX : L.colsumX)) + R, ss);
     }
     // the last CTA of this matrix turns the sums into the bounds the next phase needs;
-    // every thread fences its own (fire-and-forget) sum atomics before the count
-    __threadfence();
+    // the threads that issued (fire-and-forget) sum atomics fence them before the count
+    if ((t & 3) == 0) __threadfence();
     __syncthreads();
     if (t == 0) {
       const uint32_t units = (uint32_t)(p.prefix[mi + 1] - p.prefix[mi]);
       s_last = (atomicAdd(&st->done[0], 1u) == units - 1u);
     }
     __syncthreads();
-    if (s_last) {
+    if (s_last) {            // block-uniform
       __threadfence();
       const float ur = drain_max(reinterpret_cast<float*>(p.ws + L.rowsumX), d.mp, red);
       const float uc = drain_max(reinterpret_cast<float*>(p.ws + L.colsumX), d.np, red);
@@ -364,6 +413,22 @@ int grid_for(int64_t units, int num_sms, int per_sm) {
   return (int)(units < cap ? (units > 0 ? units : 1) : cap);
 }
 
+// Grid of a persistent (grid-stride) kernel: as many CTAs as are resident at once,
+// from the occupancy the compiled kernel actually reaches (a second wave would
+// leave SMs half empty while it runs).
+template <typename Kernel>
+int persistent_grid(Kernel kernel, int64_t units, int num_sms) {
+  static int resident = 0;    // per kernel; the same on every device of one architecture
+  if (resident == 0) {
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kEwThreads, 0) != cudaSuccess ||
+        occ < 1)
+      occ = 1;
+    resident = occ;
+  }
+  return grid_for(units, num_sms, resident);
+}
+
 }  // namespace
 
 cudaError_t launch_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld, int axis,
@@ -372,7 +437,7 @@ cudaError_t launch_quantize(const float* x, int64_t rows, int64_t cols, int64_t 
   cudaError_t e = cudaMemsetAsync(ws, 0, 8, st);
   if (e != cudaSuccess) return e;
   uint32_t* hdr = reinterpret_cast<uint32_t*>(ws);
-  amax_kernel<<<grid_for(rows, num_sms, 8), kEwThreads, 0, st>>>(x, rows, cols, ld, hdr);
+  amax_kernel<<<persistent_grid(amax_kernel, rows, num_sms), kEwThreads, 0, st>>>(x, rows, cols, ld, hdr);
   const int64_t R = axis ? cols : rows, C = axis ? rows : cols;
   const int tiled = (flags & 2u) ? 1 : 0;
   const int64_t Rext = tiled ? align_up(R, 128) : align_up(R, kT);
@@ -391,18 +456,18 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const
                               cudaStream_t st, int num_sms) {
   const int tiled = (flags & 2u) ? 1 : 0;
   const int64_t nblk = rows * (cols / 16);
-  dequantize_kernel<<<grid_for((nblk + kEwThreads - 1) / kEwThreads, num_sms, 8), kEwThreads, 0,
+  dequantize_kernel<<<persistent_grid(dequantize_kernel, (nblk + kEwThreads - 1) / kEwThreads, num_sms), kEwThreads, 0,
                       st>>>(codes, scales, s_g, rows, cols, tiled, align_up(cols, 256), y, ld);
   return cudaGetLastError();
 }
 
 cudaError_t launch_ns_reduce(const NsParams& p, cudaStream_t st, int num_sms) {
-  ns_reduce_kernel<<<grid_for(p.prefix[p.count], num_sms, 8), kEwThreads, 0, st>>>(p);
+  ns_reduce_kernel<<<persistent_grid(ns_reduce_kernel, p.prefix[p.count], num_sms), kEwThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_ns_preamble(const NsParams& p, cudaStream_t st, int num_sms) {
-  ns_preamble_kernel<<<grid_for(p.prefix[p.count], num_sms, 8), kEwThreads, 0, st>>>(p);
+  ns_preamble_kernel<<<persistent_grid(ns_preamble_kernel, p.prefix[p.count], num_sms), kEwThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 
