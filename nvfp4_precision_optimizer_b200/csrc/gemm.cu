@@ -42,8 +42,6 @@ constexpr int kStages = 3;
 // warpgroups 1-2 = 8 epilogue warps.  Registers are rebalanced after launch:
 // 384 threads x 168 = 40 x 128 (warpgroup 0) + 232 x 256 (epilogue warpgroups).
 constexpr int kThreads = 384;
-constexpr int kEpiThreads = 256;
-constexpr int kEpiBase = 128;          // first epilogue thread
 constexpr uint32_t kRegsLaunch = 168;
 constexpr uint32_t kRegsCtl = 40;
 constexpr uint32_t kRegsEpi = 232;
@@ -56,8 +54,21 @@ constexpr int B_BYTES = BN * BK / 2;
 constexpr int SFA_BYTES = BM * BK / 16;
 constexpr int SFB_BYTES = BN * BK / 16;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-constexpr int TRANS_FLOATS = 32 * 33;
-constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + 8 * TRANS_FLOATS * 4 + 256;
+constexpr int TRANS_FLOATS = 32 * 33;   // per-warp transpose buffer of the plain epilogue
+// Each epilogue warp owns a 32 x 128 share of the 128 x 256 tile and walks it in
+// chunks of 32 rows x 16 columns.  A chunk passes through a shared-memory stage
+// where row r starts at float 16 (r + r / 16) and its four 16-byte quads sit at
+// quad q ^ ((r / 2) % 4): one lane per row (the accumulator layout), one lane per
+// (column, row half) (the 16x1 view) and four lanes per row (coalesced global
+// traffic, rows r and r + 8 i) all hit 32 distinct banks.
+constexpr int kChunkCols = 16;
+constexpr int kChunks = 128 / kChunkCols;      // chunks per warp and tile
+constexpr int kStageFloats = 33 * 16;           // one staged chunk (2112 bytes)
+constexpr int kStageBufs = 3;                   // FP32 input runs two chunks ahead
+constexpr int EPI_WARP_FLOATS = kStageBufs * kStageFloats;
+static_assert(EPI_WARP_FLOATS >= TRANS_FLOATS, "the plain epilogue reuses the stage");
+constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + 8 * EPI_WARP_FLOATS * 4 + 256;
+static_assert(SMEM_BYTES <= 232448, "over the per-CTA shared-memory limit");
 constexpr float kBoundInflate = 1.0f + 1.0f / 256.0f;
 constexpr uint32_t kIdesc = idesc_mxf4nvf4(BM, BN);
 static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
@@ -155,25 +166,6 @@ __device__ __forceinline__ int32_t total_units(const NsParams& p, const GemmPlai
   }
 }
 
-struct ChunkSums {
-  float sumsq;   // sum of squared dequantised values of the 32 elements
-  float amax;    // max |x| of the 32 elements
-};
-
-// 1x16 quantisation of 32 consecutive values of row r starting at column c (c % 32 == 0),
-// power-of-two tensor scale sg (six = 6 sg, rcp_six = RN(1 / six)).
-__device__ __forceinline__ ChunkSums store_row_chunk(const float* v, int64_t r, int64_t c, int64_t Cp,
-                                                     uint8_t* codes, uint8_t* scales, float sg,
-                                                     float six, float rcp_six) {
-  const QBlock16 q0 = quantize16<true>(v, sg, six, rcp_six);
-  const QBlock16 q1 = quantize16<true>(v + 16, sg, six, rcp_six);
-  *reinterpret_cast<uint4*>(codes + tiled_chunk_offset(r, c, Cp)) =
-      make_uint4(q0.w0, q0.w1, q1.w0, q1.w1);
-  *reinterpret_cast<uint16_t*>(scales + tiled_scale_offset(r, c >> 4, Cp)) =
-      static_cast<uint16_t>(q0.scale | (q1.scale << 8));
-  return {q0.sumsq + q1.sumsq, fmaxf(q0.amax, q1.amax)};
-}
-
 // Transpose this warp's 32 x 32 chunk through shared memory: on return w[t]
 // holds the value of row t of the chunk in this lane's column.
 __device__ __forceinline__ void warp_transpose(const float* v, float* w, float* tb, int lane) {
@@ -256,14 +248,335 @@ __device__ __forceinline__ void finalize_tile(const NsParams& p, int mi, int lan
   }
 }
 
+// ---------------------------------------------------------------- epilogue staging
+__device__ __forceinline__ int stage_off(int r, int q) {
+  return 16 * (r + (r >> 4)) + 4 * (q ^ ((r >> 1) & 3));
+}
+
+__device__ __forceinline__ void cp_async16(float* smem_dst, const float* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem_dst)), "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Row r = lane of the stage <-> 16 registers.
+__device__ __forceinline__ void stage_load_row(const float* buf, int lane, float* x) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 t = *reinterpret_cast<const float4*>(buf + stage_off(lane, q));
+    x[4 * q] = t.x; x[4 * q + 1] = t.y; x[4 * q + 2] = t.z; x[4 * q + 3] = t.w;
+  }
+}
+__device__ __forceinline__ void stage_store_row(float* buf, int lane, const float* x) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<float4*>(buf + stage_off(lane, q)) =
+        make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+}
+// Column cc, rows 16 hh .. 16 hh + 15 of the stage -> 16 registers.
+__device__ __forceinline__ void stage_load_col(const float* buf, int cc, int hh, float* x) {
+#pragma unroll
+  for (int t = 0; t < 16; ++t) x[t] = buf[stage_off(16 * hh + t, cc >> 2) + (cc & 3)];
+}
+
+// FP32 rows of tile u for the four-lanes-per-row mapping: row row0 + 32 quad +
+// (lane / 4) + 8 i, i = 0..3, starts at base + i * step (step = 8 rows, in floats),
+// columns col0 + 128 ch + 4 (lane % 4) ...; the FP32 tile is A (GramX, GramA) or X (Update).
+struct TileRows {
+  float* base;
+  uint32_t step;
+};
+
+template <Epi E>
+__device__ __forceinline__ TileRows tile_rows(const NsParams& p, const GemmPlainArgs& g, int32_t u,
+                                              int quad, int ch, int lane) {
+  const Job j = make_job<E>(u, p, g);
+  const MatDesc& d = p.mat[j.mat];
+  const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
+  const int64_t pitch = (E == Epi::Update) ? d.np : d.mp;
+  TileRows t;
+  t.base = reinterpret_cast<float*>(p.ws + (E == Epi::Update ? L.X : L.A)) +
+           (j.row0 + 32 * quad + (lane >> 2)) * pitch + j.col0 + 128 * ch + 4 * (lane & 3);
+  t.step = (uint32_t)(8 * pitch);
+  return t;
+}
+
+// Asynchronous copy of chunk c of the FP32 tile rows into a stage buffer.
+__device__ __forceinline__ void stage_fetch(float* buf, TileRows t, int c, int lane) {
+  const int rr = lane >> 2, qq = lane & 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    cp_async16(buf + stage_off(rr + 8 * i, qq), t.base + (size_t)i * t.step + kChunkCols * c);
+}
+
+// Coalesced store of the staged chunk c to the FP32 tile rows.
+__device__ __forceinline__ void stage_flush(const float* buf, TileRows t, int c, int lane) {
+  const int rr = lane >> 2, qq = lane & 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    *reinterpret_cast<float4*>(t.base + (size_t)i * t.step + kChunkCols * c) =
+        *reinterpret_cast<const float4*>(buf + stage_off(rr + 8 * i, qq));
+}
+
+// Epilogue of the three Newton-Schulz GEMMs (one epilogue warp).
+//   GramX   A = sX^2 acc            -> A (FP32), qA = Q1x16(A); mirrored tile: Q1x16 of A^T
+//   GramA   B = b A + c sA^2 acc    -> qB = Q1x16(B);           mirrored tile: Q1x16 of B^T
+//   Update  X' = a X + sB sX acc    -> X' (FP32), Q1x16(X'), Q16x1(X') (or the output, last)
+template <Epi E>
+__device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainArgs& g,
+                                            uint32_t tmem, uint64_t* acc_full,
+                                            uint64_t* acc_empty, uint32_t* arrivals,
+                                            uint32_t* status, volatile int* abort_flag,
+                                            float* wbuf, int quad, int ch, int lane,
+                                            int32_t total) {
+  constexpr bool kIn = (E == Epi::GramA || E == Epi::Update);   // reads an FP32 tile
+  const int k = p.iter;
+  const int cc = lane & 15, hh = lane >> 4;
+  TileRows fp{nullptr, 0u};   // FP32 tile rows of the current tile
+  TileRows fn{nullptr, 0u};   // ... of the next tile (fetched ahead)
+  if constexpr (kIn) {
+    if ((int32_t)blockIdx.x < total) {
+      fp = tile_rows<E>(p, g, blockIdx.x, quad, ch, lane);
+      stage_fetch(wbuf, fp, 0, lane);
+      cp_async_commit();
+      stage_fetch(wbuf + kStageFloats, fp, 1, lane);
+      cp_async_commit();
+    }
+  }
+  int b = 0;   // stage buffer of the current chunk
+  uint32_t tl = 0;
+  for (int32_t u = blockIdx.x; u < total; u += gridDim.x, ++tl) {
+    const Job j = make_job<E>(u, p, g);
+    const MatDesc& d = p.mat[j.mat];
+    NsState* st = reinterpret_cast<NsState*>(p.ws + d.state_off);
+    const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
+    if constexpr (!kIn) fp = tile_rows<E>(p, g, u, quad, ch, lane);
+    // warp-uniform by construction: the chunk loop shuffles under this condition
+    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, tl & 1u, status, abort_flag));
+    const int64_t gr0 = j.row0 + 32 * quad;   // first row of this warp's band
+    const int64_t gr = gr0 + lane;             // this lane's row
+    const int64_t gc0 = j.col0 + 128 * ch;     // first column of this warp's half
+    const bool last = (E == Epi::Update) && p.last;
+
+    float acc_scale, sg_out;
+    if constexpr (E == Epi::GramX) {
+      const float sx = __ldcg(&st->sg[kSgX + k]);
+      acc_scale = sx * sx;
+      sg_out = __ldcg(&st->sg[kSgA + k]);
+    } else if constexpr (E == Epi::GramA) {
+      const float sa = __ldcg(&st->sg[kSgA + k]);
+      acc_scale = sa * sa;
+      sg_out = __ldcg(&st->sg[kSgB + k]);
+    } else {
+      acc_scale = __ldcg(&st->sg[kSgB + k]) * __ldcg(&st->sg[kSgX + k]);
+      sg_out = p.last ? 1.0f : __ldcg(&st->sg[kSgX + k + 1]);
+    }
+    const float six_out = __fmul_rn(6.0f, sg_out);
+    const float rcp_six = __frcp_rn(six_out);
+
+    // destinations of the two views and of their sums
+    const int ns = (k + 1) & 1;
+    uint8_t* row_codes = p.ws + (E == Epi::GramX ? L.qA : E == Epi::GramA ? L.qB : (ns ? L.qX[1] : L.qX[0]));
+    uint8_t* row_scales = p.ws + (E == Epi::GramX ? L.sA : E == Epi::GramA ? L.sB : (ns ? L.sX[1] : L.sX[0]));
+    const int64_t row_cp = (E == Epi::Update) ? d.np : d.mp;
+    uint8_t* col_codes = (E == Epi::Update) ? p.ws + (ns ? L.qXT[1] : L.qXT[0]) : row_codes;
+    uint8_t* col_scales = (E == Epi::Update) ? p.ws + (ns ? L.sXT[1] : L.sXT[0]) : row_scales;
+    float* rowsum = reinterpret_cast<float*>(
+        p.ws + (E == Epi::GramX ? L.rowsumA : E == Epi::GramA ? L.rowsumB : L.rowsumX));
+    float* colsum = (E == Epi::Update) ? reinterpret_cast<float*>(p.ws + L.colsumX) : rowsum;
+    const bool need_col = (E == Epi::Update) ? !last : (j.mirror != 0);
+
+    uint32_t accr[4][32];
+    if (ok) {
+      tc_fence_after();
+      // drain this warp's 32 x 128 share of the accumulator into registers and hand
+      // the accumulator back at once: the next tile's MMAs overlap this epilogue
+      const uint32_t taddr = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(128 * ch);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32_async(taddr + 32 * c, accr[c]);
+      tmem_wait_ld32(accr[0]);
+      tmem_ld_order(accr[1]);
+      tmem_ld_order(accr[2]);
+      tmem_ld_order(accr[3]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+    }
+
+    float row_acc = 0.0f, amax = 0.0f;
+    uint32_t prev_w0 = 0u, prev_w1 = 0u, scale_word = 0u;
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c) {
+      float* buf = wbuf + b * kStageFloats;
+      if constexpr (kIn) {
+        cp_async_wait<1>();   // this chunk's rows have landed (own copies) ...
+        __syncwarp();         // ... and every lane's
+      }
+      if (ok) {
+        const int64_t gcc = gc0 + kChunkCols * c;   // first column of the chunk
+        float y[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) y[e] = __uint_as_float(accr[c >> 1][16 * (c & 1) + e]) * acc_scale;
+        if constexpr (kIn) {
+          float xin[16];
+          stage_load_row(buf, lane, xin);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            if constexpr (E == Epi::Update) y[e] = fmaf(d.a, xin[e], y[e]);
+            else y[e] = fmaf(d.b, xin[e], d.c * y[e]);
+          }
+        }
+        if (last) {
+          // final iteration: write the output (transposed back for a tall input)
+          if (d.tall) {
+            if (gr < d.m) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                if (gcc + e < d.n) d.out[(gcc + e) * d.ldo + gr] = y[e];
+            }
+          } else {
+            stage_store_row(buf, lane, y);
+            __syncwarp();
+            float xc[16];
+            stage_load_col(buf, cc, hh, xc);
+            const int64_t col = gcc + cc;
+            if (col < d.n) {
+#pragma unroll
+              for (int t = 0; t < 16; ++t) {
+                const int64_t row = gr0 + 16 * hh + t;
+                if (row < d.m) d.out[row * d.ldo + col] = xc[t];
+              }
+            }
+          }
+        } else {
+          // 1x16 view along this lane's row
+          const QBlock16 q = quantize16<true>(y, sg_out, six_out, rcp_six);
+          row_acc += q.sumsq;
+          amax = fmaxf(amax, q.amax);
+          if (c & 1) {
+            *reinterpret_cast<uint4*>(row_codes + tiled_chunk_offset(gr, gcc - 16, row_cp)) =
+                make_uint4(prev_w0, prev_w1, q.w0, q.w1);
+          } else {
+            prev_w0 = q.w0;
+            prev_w1 = q.w1;
+          }
+          scale_word |= q.scale << (8 * (c & 3));
+          if ((c & 3) == 3) {
+            *reinterpret_cast<uint32_t*>(row_scales + tiled_scale_offset(gr, (gcc - 48) >> 4, row_cp)) =
+                scale_word;
+            scale_word = 0u;
+          }
+          if (E != Epi::GramA || need_col) {
+            stage_store_row(buf, lane, y);
+            __syncwarp();
+          }
+          if constexpr (E != Epi::GramA) stage_flush(buf, fp, c, lane);   // A or X' (FP32)
+          if (need_col) {
+            // 16x1 view: column gcc + cc, rows gr0 + 16 hh .. (the transposed view's row)
+            float xc[16];
+            stage_load_col(buf, cc, hh, xc);
+            const QBlock16 qc = quantize16<true>(xc, sg_out, six_out, rcp_six);
+            const uint32_t o0 = __shfl_xor_sync(0xFFFFFFFFu, qc.w0, 16);
+            const uint32_t o1 = __shfl_xor_sync(0xFFFFFFFFu, qc.w1, 16);
+            const uint32_t os = __shfl_xor_sync(0xFFFFFFFFu, qc.scale, 16);
+            const float s2 = qc.sumsq + __shfl_xor_sync(0xFFFFFFFFu, qc.sumsq, 16);
+            if (hh == 0) {
+              const int64_t rt = gcc + cc;
+              *reinterpret_cast<uint4*>(col_codes + tiled_chunk_offset(rt, gr0, d.mp)) =
+                  make_uint4(qc.w0, qc.w1, o0, o1);
+              *reinterpret_cast<uint16_t*>(col_scales + tiled_scale_offset(rt, gr0 >> 4, d.mp)) =
+                  static_cast<uint16_t>(qc.scale | (os << 8));
+              if (s2 != 0.0f) atomicAdd(colsum + rt, s2);
+            }
+          }
+        }
+      }
+      __syncwarp();   // every lane is done with this stage buffer
+      if constexpr (kIn) {
+        // fetch chunk c + 2 (of this tile or the next) into the buffer chunk c - 1 used
+        float* nb = wbuf + (b == 0 ? 2 : b - 1) * kStageFloats;
+        const bool more = u + (int32_t)gridDim.x < total;
+        if (c + 2 < kChunks) {
+          stage_fetch(nb, fp, c + 2, lane);
+        } else if (more) {
+          if (c + 2 == kChunks) fn = tile_rows<E>(p, g, u + gridDim.x, quad, ch, lane);
+          stage_fetch(nb, fn, c + 2 - kChunks, lane);
+        }
+        cp_async_commit();
+      }
+      b = (b == kStageBufs - 1) ? 0 : b + 1;
+    }
+
+    if (row_acc != 0.0f) atomicAdd(rowsum + gr, row_acc);
+    if constexpr (E == Epi::Update) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      if (lane == 0 && !p.last && amax > 0.0f) atomicMax(&st->amaxX[k + 1], __float_as_uint(amax));
+    }
+    // publish this warp's sums for the counter warp (never waits)
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) atomicAdd(arrivals, 1u);
+    if constexpr (kIn) fp = fn;
+  }
+  if constexpr (kIn) cp_async_wait<0>();
+}
+
+// Epilogue of the plain GEMM D = (sa sb) acc (one epilogue warp); tb is a 32 x 33
+// transpose buffer so that each store instruction writes one contiguous row segment.
+__device__ __forceinline__ void epilogue_plain(const NsParams& p, const GemmPlainArgs& g,
+                                               uint32_t tmem, uint64_t* acc_full,
+                                               uint64_t* acc_empty, uint32_t* status,
+                                               volatile int* abort_flag, float* tb, int quad,
+                                               int ch, int lane, int32_t total) {
+  uint32_t tl = 0;
+  for (int32_t u = blockIdx.x; u < total; u += gridDim.x, ++tl) {
+    const Job j = make_job<Epi::Plain>(u, p, g);
+    const bool ok = mbar_wait(acc_full, tl & 1u, status, abort_flag);
+    if (!ok) continue;
+    const int64_t gr0 = j.row0 + 32 * quad;
+    const float acc_scale = __ldg(g.a_sg) * __ldg(g.b_sg);
+    tc_fence_after();
+    uint32_t accr[4][32];
+    const uint32_t taddr = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(128 * ch);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld32_async(taddr + 32 * c, accr[c]);
+    tmem_wait_ld32(accr[0]);
+    tmem_ld_order(accr[1]);
+    tmem_ld_order(accr[2]);
+    tmem_ld_order(accr[3]);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(acc_empty);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float v[32], w[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(accr[c][e]) * acc_scale;
+      warp_transpose(v, w, tb, lane);
+      const int64_t col = j.col0 + 128 * ch + 32 * c + lane;
+      if (col < g.N) {
+        float* dcol = g.d + gr0 * g.ldd + col;
+#pragma unroll
+        for (int t = 0; t < 32; ++t)
+          if (gr0 + t < g.M) dcol[t * g.ldd] = w[t];
+      }
+    }
+  }
+}
+
 template <Epi E>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ NsParams p, const __grid_constant__ GemmPlainArgs g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
-  float* trans = reinterpret_cast<float*>(smem + kStages * STAGE_BYTES);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * STAGE_BYTES + 8 * TRANS_FLOATS * 4);
+  float* epi_smem = reinterpret_cast<float*>(smem + kStages * STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * STAGE_BYTES + 8 * EPI_WARP_FLOATS * 4);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
   uint64_t* acc_full = bars + 2 * kStages;
@@ -395,168 +708,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue
     // Every epilogue warp walks the same tile list and never leaves it early (a
     // failed wait only skips that tile's work), so the block-wide barrier at the
-    // end is reached by all threads.  Per tile, each warp fences its row/column
-    // sum atomics and bumps the shared arrival counter that warp 2 trails.
+    // end is reached by all threads.
     const int ew = warp - 4;          // 0..7
     const int quad = warp & 3;        // TMEM lanes 32*quad .. 32*quad+31
     const int ch = ew >> 2;           // column half of the 256-wide tile
-    float* tb = trans + ew * TRANS_FLOATS;
-    uint32_t tl = 0;
-    for (int32_t u = blockIdx.x; u < total; u += gridDim.x, ++tl) {
-      const Job j = make_job<E>(u, p, g);
-      const bool ok = mbar_wait(acc_full, tl & 1u, status, abort_flag);
-      const int64_t gr0 = j.row0 + 32 * quad;   // first row of this warp's band
-      const int64_t gr = gr0 + lane;             // this lane's row
-
-      // per-job constants
-      float acc_scale, sg_out = 1.0f, six_out = 6.0f, rcp_six = 1.0f / 6.0f;
-      float coef_a = 0.0f, coef_b = 0.0f, coef_c = 0.0f;
-      const MatDesc* d = nullptr;
-      NsState* st = nullptr;
-      MatLayout L;
-      const int k = p.iter;
-      if constexpr (E == Epi::Plain) {
-        acc_scale = __ldg(g.a_sg) * __ldg(g.b_sg);
-      } else {
-        d = &p.mat[j.mat];
-        st = reinterpret_cast<NsState*>(p.ws + d->state_off);
-        L = mat_layout(d->mp, d->np, d->state_off, d->big_off);
-        coef_a = d->a; coef_b = d->b; coef_c = d->c;
-        if constexpr (E == Epi::GramX) {
-          const float sx = __ldcg(&st->sg[kSgX + k]);
-          acc_scale = sx * sx;
-          sg_out = __ldcg(&st->sg[kSgA + k]);
-        } else if constexpr (E == Epi::GramA) {
-          const float sa = __ldcg(&st->sg[kSgA + k]);
-          acc_scale = sa * sa;
-          sg_out = __ldcg(&st->sg[kSgB + k]);
-        } else {
-          acc_scale = __ldcg(&st->sg[kSgB + k]) * __ldcg(&st->sg[kSgX + k]);
-          sg_out = p.last ? 1.0f : __ldcg(&st->sg[kSgX + k + 1]);
-        }
-        six_out = __fmul_rn(6.0f, sg_out);
-        rcp_six = __frcp_rn(six_out);
-      }
-
-      float row_acc = 0.0f, amax = 0.0f;
-      if (ok) {
-        tc_fence_after();
-        // drain this warp's 32 x 128 share of the accumulator into registers and hand
-        // the accumulator back at once: the next tile's MMAs overlap this epilogue
-        uint32_t accr[4][32];
-        const uint32_t taddr = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(128 * ch);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32_async(taddr + 32 * c, accr[c]);
-        tmem_wait_ld32(accr[0]);
-        tmem_ld_order(accr[1]);
-        tmem_ld_order(accr[2]);
-        tmem_ld_order(accr[3]);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acc_empty);
-
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int64_t gc = j.col0 + 128 * ch + 32 * c;
-          float v[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(accr[c][e]) * acc_scale;
-
-          // FP32 tiles are read and written after a per-warp transpose (lane = column,
-          // w[t] = row gr0 + t): every warp access is then one contiguous 128-byte line.
-          if constexpr (E == Epi::Plain) {
-            float w[32];
-            warp_transpose(v, w, tb, lane);
-            const int64_t col = gc + lane;
-            if (col < g.N) {
-              float* dcol = g.d + gr0 * g.ldd + col;
-#pragma unroll
-              for (int t = 0; t < 32; ++t)
-                if (gr0 + t < g.M) dcol[t * g.ldd] = w[t];
-            }
-          } else if constexpr (E == Epi::GramX) {
-            row_acc += store_row_chunk(v, gr, gc, d->mp, p.ws + L.qA, p.ws + L.sA, sg_out, six_out, rcp_six).sumsq;
-            float w[32];
-            warp_transpose(v, w, tb, lane);
-            float* Acol = reinterpret_cast<float*>(p.ws + L.A) + gr0 * d->mp + gc + lane;
-#pragma unroll
-            for (int t = 0; t < 32; ++t) Acol[t * d->mp] = w[t];
-            if (j.mirror) {
-              const float cs = store_row_chunk(w, gc + lane, gr0, d->mp, p.ws + L.qA, p.ws + L.sA,
-                                               sg_out, six_out, rcp_six).sumsq;
-              if (cs != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.rowsumA) + gc + lane, cs);
-            }
-          } else if constexpr (E == Epi::GramA) {
-            const float* Acol = reinterpret_cast<const float*>(p.ws + L.A) + gr0 * d->mp + gc + lane;
-            float w[32], a_row[32];
-#pragma unroll
-            for (int t = 0; t < 32; ++t) w[t] = __ldcg(Acol + t * d->mp);
-            warp_transpose(w, a_row, tb, lane);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = fmaf(coef_b, a_row[e], coef_c * v[e]);
-            row_acc += store_row_chunk(v, gr, gc, d->mp, p.ws + L.qB, p.ws + L.sB, sg_out, six_out, rcp_six).sumsq;
-            if (j.mirror) {
-              warp_transpose(v, w, tb, lane);
-              const float cs = store_row_chunk(w, gc + lane, gr0, d->mp, p.ws + L.qB, p.ws + L.sB,
-                                               sg_out, six_out, rcp_six).sumsq;
-              if (cs != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.rowsumB) + gc + lane, cs);
-            }
-          } else {  // Update
-            float* Xcol = reinterpret_cast<float*>(p.ws + L.X) + gr0 * d->np + gc + lane;
-            float w[32];
-            warp_transpose(v, w, tb, lane);
-#pragma unroll
-            for (int t = 0; t < 32; ++t) w[t] = fmaf(coef_a, __ldcg(Xcol + t * d->np), w[t]);
-            if (p.last) {
-              if (!d->tall) {
-                if (gc + lane < d->n) {
-                  float* ocol = d->out + gr0 * d->ldo + gc + lane;
-#pragma unroll
-                  for (int t = 0; t < 32; ++t)
-                    if (gr0 + t < d->m) ocol[t * d->ldo] = w[t];
-                }
-              } else {
-                warp_transpose(w, v, tb, lane);
-                if (gr < d->m) {
-#pragma unroll
-                  for (int e = 0; e < 32; ++e)
-                    if (gc + e < d->n) d->out[(gc + e) * d->ldo + gr] = v[e];
-                }
-              }
-            } else {
-#pragma unroll
-              for (int t = 0; t < 32; ++t) Xcol[t * d->np] = w[t];
-              const int ns = (k + 1) & 1;
-              const ChunkSums cs = store_row_chunk(w, gc + lane, gr0, d->mp,
-                                                   p.ws + (ns ? L.qXT[1] : L.qXT[0]),
-                                                   p.ws + (ns ? L.sXT[1] : L.sXT[0]), sg_out, six_out, rcp_six);
-              amax = fmaxf(amax, cs.amax);
-              if (cs.sumsq != 0.0f) atomicAdd(reinterpret_cast<float*>(p.ws + L.colsumX) + gc + lane, cs.sumsq);
-              warp_transpose(w, v, tb, lane);
-              row_acc += store_row_chunk(v, gr, gc, d->np, p.ws + (ns ? L.qX[1] : L.qX[0]),
-                                         p.ws + (ns ? L.sX[1] : L.sX[0]), sg_out, six_out, rcp_six).sumsq;
-            }
-          }
-        }
-      }
-
-      if constexpr (E != Epi::Plain) {
-        float* rowsum = nullptr;
-        if constexpr (E == Epi::GramX) rowsum = reinterpret_cast<float*>(p.ws + L.rowsumA);
-        if constexpr (E == Epi::GramA) rowsum = reinterpret_cast<float*>(p.ws + L.rowsumB);
-        if constexpr (E == Epi::Update) rowsum = reinterpret_cast<float*>(p.ws + L.rowsumX);
-        if (row_acc != 0.0f) atomicAdd(rowsum + gr, row_acc);
-        if constexpr (E == Epi::Update) {
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-          if (lane == 0 && !p.last && amax > 0.0f) atomicMax(&st->amaxX[k + 1], __float_as_uint(amax));
-        }
-        // publish this warp's sums for the counter warp (never waits)
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) atomicAdd(arrivals, 1u);
-      }
-    }
+    float* wbuf = epi_smem + ew * EPI_WARP_FLOATS;
+    if constexpr (E == Epi::Plain)
+      epilogue_plain(p, g, tmem, acc_full, acc_empty, status, abort_flag, wbuf, quad, ch, lane, total);
+    else
+      epilogue_ns<E>(p, g, tmem, acc_full, acc_empty, arrivals, status, abort_flag, wbuf, quad, ch,
+                     lane, total);
   }
 
   tc_fence_before();
