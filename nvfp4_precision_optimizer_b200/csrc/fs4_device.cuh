@@ -148,11 +148,31 @@ __device__ __forceinline__ float div_rn_fma(float x, float d, float rcp) {
   return fmaf(fmaf(-q0, d, x), rcp, q0);
 }
 
+// Per-CTA table of the positive E4M3 block scales: tab[b] = {value of byte b,
+// RN(1 / value)} for b = 1..126 (tab[0] and tab[127] unused).  With a
+// power-of-two tensor scale s_g = 2^k the decoded scale is den = value * 2^k and
+// RN(1 / den) = RN(1 / value) * 2^-k exactly, because the product stays a normal
+// number for every block scale reachable from a tensor scale of the form chosen by
+// pow2_tensor_scale (den <= 2^125.5, so 1 / den >= 2^-125.5).
+struct ScaleTab {
+  const float2* tab;   // 128 entries in shared memory
+  float rcp_sg;        // 1 / s_g, exact
+};
+
+__device__ __forceinline__ float2 scale_tab_entry(uint32_t b) {
+  if (b == 0u || b >= 127u) return make_float2(0.0f, 0.0f);
+  const float v = e4m3_to_f32(b);
+  return make_float2(v, __frcp_rn(v));
+}
+
 // Quantise 16 FP32 values with tensor scale s_g (six_sg = fp32(6 * s_g)).
 // kPow2: s_g is a power of two and rcp_six = RN(1 / six_sg), so the block scale
 // division may use the FMA-corrected form; otherwise IEEE division is used.
-template <bool kPow2>
-__device__ __forceinline__ QBlock16 quantize16(const float* x, float s_g, float six_sg, float rcp_six) {
+// With a table (kPow2 only) the decoded block scale and its reciprocal are looked up.
+template <bool kPow2, bool kTab = false>
+__device__ __forceinline__ QBlock16 quantize16(const float* x, float s_g, float six_sg, float rcp_six,
+                                               ScaleTab st = ScaleTab{nullptr, 0.0f}) {
+  static_assert(kPow2 || !kTab, "the scale table needs a power-of-two tensor scale");
   // max |x| as a tree (depth 4 instead of a 16-long dependency chain)
   float m8[8];
 #pragma unroll
@@ -163,15 +183,22 @@ __device__ __forceinline__ QBlock16 quantize16(const float* x, float s_g, float 
   QBlock16 r;
   r.amax = amax;
   r.scale = f32_to_e4m3(kPow2 ? div_rn_fma(amax, six_sg, rcp_six) : __fdiv_rn(amax, six_sg));
-  const float den = __fmul_rn(e4m3_to_f32(r.scale), s_g);
   if (r.scale == 0u) {
     r.w0 = r.w1 = 0u;
     r.sumsq = 0.0f;
     return r;
   }
+  float den, rcp = 0.0f;
+  if constexpr (kTab) {
+    const float2 t = st.tab[r.scale];
+    den = __fmul_rn(t.x, s_g);
+    rcp = t.y * st.rcp_sg;
+  } else {
+    den = __fmul_rn(e4m3_to_f32(r.scale), s_g);
+    if (kPow2) rcp = __frcp_rn(den);
+  }
   float q[16];
   if (kPow2) {
-    const float rcp = __frcp_rn(den);
 #pragma unroll
     for (int i = 0; i < 16; ++i) q[i] = div_rn_fma(x[i], den, rcp);
   } else {
@@ -208,14 +235,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// Test for completion of the phase with `parity`; if it is not complete the thread
+// may be suspended (it stops issuing) until it completes or about kSuspendNs pass.
+constexpr uint32_t kSuspendNs = 1000000u;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendNs)
       : "memory");
   return ok != 0u;
 }
@@ -227,15 +257,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
                                           volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t i = 0;; ++i) {
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 63u) {
-      if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
-        atomicOr(status, kStatusTimeout);
-        *abort = 1;
-        return false;
-      }
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(status, kStatusTimeout);
+      *abort = 1;
+      return false;
     }
   }
 }

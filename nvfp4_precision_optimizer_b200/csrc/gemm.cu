@@ -67,7 +67,7 @@ constexpr int kStageFloats = 33 * 16;           // one staged chunk (2112 bytes)
 constexpr int kStageBufs = 3;                   // FP32 input runs two chunks ahead
 constexpr int EPI_WARP_FLOATS = kStageBufs * kStageFloats;
 static_assert(EPI_WARP_FLOATS >= TRANS_FLOATS, "the plain epilogue reuses the stage");
-constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + 8 * EPI_WARP_FLOATS * 4 + 256;
+constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + 8 * EPI_WARP_FLOATS * 4 + 256 + 128 * 8;
 static_assert(SMEM_BYTES <= 232448, "over the per-CTA shared-memory limit");
 constexpr float kBoundInflate = 1.0f + 1.0f / 256.0f;
 constexpr uint32_t kIdesc = idesc_mxf4nvf4(BM, BN);
@@ -331,8 +331,8 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
                                             uint32_t tmem, uint64_t* acc_full,
                                             uint64_t* acc_empty, uint32_t* arrivals,
                                             uint32_t* status, volatile int* abort_flag,
-                                            float* wbuf, int quad, int ch, int lane,
-                                            int32_t total) {
+                                            float* wbuf, const float2* scale_tab, int quad, int ch,
+                                            int lane, int32_t total) {
   constexpr bool kIn = (E == Epi::GramA || E == Epi::Update);   // reads an FP32 tile
   const int k = p.iter;
   const int cc = lane & 15, hh = lane >> 4;
@@ -377,6 +377,7 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
     }
     const float six_out = __fmul_rn(6.0f, sg_out);
     const float rcp_six = __frcp_rn(six_out);
+    const ScaleTab stab{scale_tab, __frcp_rn(sg_out)};   // sg_out is a power of two
 
     // destinations of the two views and of their sums
     const int ns = (k + 1) & 1;
@@ -453,8 +454,23 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
             }
           }
         } else {
-          // 1x16 view along this lane's row
-          const QBlock16 q = quantize16<true>(y, sg_out, six_out, rcp_six);
+          // stage the chunk (FP32 store and/or the 16x1 view read it back)
+          if (E != Epi::GramA || need_col) {
+            stage_store_row(buf, lane, y);
+            __syncwarp();
+          }
+          if constexpr (E != Epi::GramA) stage_flush(buf, fp, c, lane);   // A or X' (FP32)
+          // 1x16 view along this lane's row and, where needed, the 16x1 view of column
+          // gcc + cc, rows gr0 + 16 hh ..: two independent quantiser chains side by side
+          QBlock16 q, qc;
+          if (need_col) {
+            float xc[16];
+            stage_load_col(buf, cc, hh, xc);
+            q = quantize16<true, true>(y, sg_out, six_out, rcp_six, stab);
+            qc = quantize16<true, true>(xc, sg_out, six_out, rcp_six, stab);
+          } else {
+            q = quantize16<true, true>(y, sg_out, six_out, rcp_six, stab);
+          }
           row_acc += q.sumsq;
           amax = fmaxf(amax, q.amax);
           if (c & 1) {
@@ -470,16 +486,8 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
                 scale_word;
             scale_word = 0u;
           }
-          if (E != Epi::GramA || need_col) {
-            stage_store_row(buf, lane, y);
-            __syncwarp();
-          }
-          if constexpr (E != Epi::GramA) stage_flush(buf, fp, c, lane);   // A or X' (FP32)
           if (need_col) {
-            // 16x1 view: column gcc + cc, rows gr0 + 16 hh .. (the transposed view's row)
-            float xc[16];
-            stage_load_col(buf, cc, hh, xc);
-            const QBlock16 qc = quantize16<true>(xc, sg_out, six_out, rcp_six);
+            // the two row halves of one column pair up into a 16-byte code chunk
             const uint32_t o0 = __shfl_xor_sync(0xFFFFFFFFu, qc.w0, 16);
             const uint32_t o1 = __shfl_xor_sync(0xFFFFFFFFu, qc.w1, 16);
             const uint32_t os = __shfl_xor_sync(0xFFFFFFFFu, qc.scale, 16);
@@ -585,6 +593,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 3);
   uint32_t* arrivals = tmem_slot + 1;   // monotonic count of (epilogue warp, tile) completions
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  float2* scale_tab = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(bars) + 256);
+  if (threadIdx.x >= 128 && threadIdx.x < 256) scale_tab[threadIdx.x - 128] = scale_tab_entry(threadIdx.x - 128);
 
   uint32_t* status = (E == Epi::Plain) ? g.status : p.status;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -691,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t t0 = global_timer_ns();
           while (*reinterpret_cast<volatile uint32_t*>(arrivals) < target) {
             if (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs) { seen = false; break; }
-            __nanosleep(64);
+            __nanosleep(500);
           }
         }
         if (!seen) {
@@ -716,8 +726,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (E == Epi::Plain)
       epilogue_plain(p, g, tmem, acc_full, acc_empty, status, abort_flag, wbuf, quad, ch, lane, total);
     else
-      epilogue_ns<E>(p, g, tmem, acc_full, acc_empty, arrivals, status, abort_flag, wbuf, quad, ch,
-                     lane, total);
+      epilogue_ns<E>(p, g, tmem, acc_full, acc_empty, arrivals, status, abort_flag, wbuf, scale_tab,
+                     quad, ch, lane, total);
   }
 
   tc_fence_before();

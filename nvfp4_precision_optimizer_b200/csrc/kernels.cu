@@ -295,9 +295,11 @@ __global__ void __launch_bounds__(kEwThreads) ns_reduce_kernel(const __grid_cons
 __global__ void __launch_bounds__(kEwThreads) ns_preamble_kernel(const __grid_constant__ NsParams p) {
   __shared__ float tile[kT][kT + 1];
   __shared__ float red[kEwThreads / 32];
+  __shared__ float2 scale_tab[128];
   __shared__ int s_last;
   const int32_t total = p.prefix[p.count];
   const int t = threadIdx.x;
+  if (t < 128) scale_tab[t] = scale_tab_entry(t);   // read after the first barrier below
   for (int32_t u = blockIdx.x; u < total; u += gridDim.x) {
     const int mi = owner_of(p.prefix, p.count, u);
     const MatDesc& d = p.mat[mi];
@@ -314,6 +316,7 @@ __global__ void __launch_bounds__(kEwThreads) ns_preamble_kernel(const __grid_co
     const float sg = __ldcg(&st->sg[kSgX + 0]);
     const float six_sg = __fmul_rn(6.0f, sg);
     const float rcp_six = __frcp_rn(six_sg);
+    const ScaleTab stab{scale_tab, __frcp_rn(sg)};   // sg is a power of two
     const bool vec = ((reinterpret_cast<uintptr_t>(d.G) & 15) == 0) && ((d.ldg & 3) == 0);
 
     // stage the X0 tile (working orientation) in shared memory; a matrix with a
@@ -361,7 +364,7 @@ __global__ void __launch_bounds__(kEwThreads) ns_preamble_kernel(const __grid_co
       float v[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) v[e] = view == 0 ? tile[line][blk * 16 + e] : tile[blk * 16 + e][line];
-      const QBlock16 q = quantize16<true>(v, sg, six_sg, rcp_six);
+      const QBlock16 q = quantize16<true, true>(v, sg, six_sg, rcp_six, stab);
       // row (view 0: row i0+line of X, K = j0..) or row j0+line of X^T (view 1, K = i0..)
       const int64_t R = (view == 0 ? i0 : j0) + line;
       const int64_t K0 = view == 0 ? j0 : i0;

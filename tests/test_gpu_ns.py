@@ -119,6 +119,45 @@ def test_first_gram_product_and_its_requantisation(fs4, shape, kind):
     assert np.all(np.abs(got - want)[diff] <= 0.51 * np.maximum(np.abs(got), np.abs(want))[diff] + 1e-30)
 
 
+def _upper_tiles_to_full(Ag, mp):
+    """Symmetric mp x mp matrix from the 256 x 256 tiles on and above the diagonal."""
+    t = np.arange(mp) // 256
+    upper = t[:, None] <= t[None, :]
+    return np.where(upper, Ag, Ag.T)
+
+
+@pytest.mark.parametrize("shape,kind", [((256, 256), "gauss"), ((48, 80), "gauss"),
+                                        ((1024, 4096), "outliers"), ((4096, 1024), "student"),
+                                        ((768, 1280), "gauss")])
+def test_epilogue_requantisation_bit_exact(fs4, shape, kind):
+    """The fused GEMM epilogues quantise their own FP32 results exactly as Q1x16 and
+    Q16x1 do (Section 3.4): the GPU's FP32 A_0 and X_1, quantised by the oracle with
+    the GPU's tensor scales, give the GPU's codes and scales byte for byte, on both
+    triangles of A (the lower one comes from the mirrored 16x1 view) and on both views
+    of X_1, padding included."""
+    G = momentum(*shape, kind=kind, seed=5)
+    lay = fs4.ns_layout([shape], 0)
+    mp, np_ = lay.mp, lay.np
+    # A_0 after the first Gram product
+    _, ws = run_gpu(fs4, G, 2, MUON, flags=fs4.stop_after(1))
+    A = _upper_tiles_to_full(ws_f32(ws, lay.A, mp * mp).reshape(mp, mp), mp)
+    sga = ws_f32(ws, lay.scalars, 192)[64]
+    oc, os_, _ = Q.quantize_rows(np.ascontiguousarray(A, dtype=np.float32), s_g=sga)
+    gc, gs = view(ws, lay.qA_codes, lay.qA_scales, mp, mp)
+    assert np.array_equal(gs, os_) and np.array_equal(gc, oc)
+    # X_1 after the first update (K = 2, so it is requantised for iteration 1)
+    _, ws = run_gpu(fs4, G, 2, MUON, flags=fs4.stop_after(3))
+    X1 = ws_f32(ws, lay.X, mp * np_).reshape(mp, np_)
+    sgx = ws_f32(ws, lay.scalars, 192)[1]
+    assert 2688 * sgx >= np.abs(X1).max()
+    oc, os_, _ = Q.quantize_rows(X1, s_g=sgx)
+    gc, gs = view(ws, lay.qX_codes[1], lay.qX_scales[1], mp, np_)
+    assert np.array_equal(gs, os_) and np.array_equal(gc, oc)
+    oc, os_, _ = Q.quantize_rows(np.ascontiguousarray(X1.T), s_g=sgx)
+    gc, gs = view(ws, lay.qXT_codes[1], lay.qXT_scales[1], np_, mp)
+    assert np.array_equal(gs, os_) and np.array_equal(gc, oc)
+
+
 def _spectrum_rel(a, b):
     sa = np.linalg.svd(working(a).astype(np.float64), compute_uv=False)
     sb = np.linalg.svd(working(b).astype(np.float64), compute_uv=False)
