@@ -300,7 +300,41 @@ __global__ void __launch_bounds__(kEwThreads) ns_preamble_kernel(const __grid_co
   const int32_t total = p.prefix[p.count];
   const int t = threadIdx.x;
   if (t < 128) scale_tab[t] = scale_tab_entry(t);   // read after the first barrier below
+
+  // The next unit's G tile is loaded into registers while this unit is quantised
+  // (interior tiles of 16-byte aligned inputs; edge tiles load on the guarded path).
+  float4 pf[4];
+  bool pf_fast = false;
+  auto prefetch = [&](int32_t uu) {
+    pf_fast = false;
+    if (uu >= total) return;
+    const int mi = owner_of(p.prefix, p.count, uu);
+    const MatDesc& d = p.mat[mi];
+    const int32_t tiles_n = d.np / kT;
+    const int32_t lu = uu - p.prefix[mi];
+    const int32_t ti = lu / tiles_n;
+    const int32_t i0 = ti * kT, j0 = (lu - ti * tiles_n) * kT;
+    const int32_t rows_g = d.tall ? d.n : d.m, cols_g = d.tall ? d.m : d.n;
+    const int32_t gr0 = d.tall ? j0 : i0, gc0 = d.tall ? i0 : j0;
+    const bool vec = ((reinterpret_cast<uintptr_t>(d.G) & 15) == 0) && ((d.ldg & 3) == 0);
+    if (vec && gr0 + kT <= rows_g && gc0 + kT <= cols_g) {
+      pf_fast = true;
+      const float* gtile = d.G + (int64_t)gr0 * d.ldg + gc0;
+#pragma unroll
+      for (int pass = 0; pass < 4; ++pass) {
+        const int f = t + kEwThreads * pass;
+        pf[pass] = __ldg(reinterpret_cast<const float4*>(gtile + (int64_t)(f >> 4) * d.ldg + (f & 15) * 4));
+      }
+    }
+  };
+  prefetch(blockIdx.x);
+
   for (int32_t u = blockIdx.x; u < total; u += gridDim.x) {
+    float4 cur[4];
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) cur[pass] = pf[pass];
+    const bool cur_fast = pf_fast;
+    prefetch(u + gridDim.x);
     const int mi = owner_of(p.prefix, p.count, u);
     const MatDesc& d = p.mat[mi];
     NsState* st = state_of(p, d);
@@ -317,25 +351,23 @@ __global__ void __launch_bounds__(kEwThreads) ns_preamble_kernel(const __grid_co
     const float six_sg = __fmul_rn(6.0f, sg);
     const float rcp_six = __frcp_rn(six_sg);
     const ScaleTab stab{scale_tab, __frcp_rn(sg)};   // sg is a power of two
-    const bool vec = ((reinterpret_cast<uintptr_t>(d.G) & 15) == 0) && ((d.ldg & 3) == 0);
 
     // stage the X0 tile (working orientation) in shared memory; a matrix with a
     // non-finite entry is carried as all zeros (its output is zero)
     const int32_t rows_g = d.tall ? d.n : d.m, cols_g = d.tall ? d.m : d.n;
     const int32_t gr0 = d.tall ? j0 : i0, gc0 = d.tall ? i0 : j0;   // tile origin in G
-    const bool interior = vec && !dead && gr0 + kT <= rows_g && gc0 + kT <= cols_g;
     const float* gtile = d.G + (int64_t)gr0 * d.ldg + gc0;
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass) {
       const int f = t + kEwThreads * pass;
       const int line = f >> 4, c4 = (f & 15) * 4;       // 64 lines of 64 floats
       float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      if (interior) {
-        const float4 x4 = __ldg(reinterpret_cast<const float4*>(gtile + (int64_t)line * d.ldg + c4));
-        v[0] = x4.x; v[1] = x4.y; v[2] = x4.z; v[3] = x4.w;
+      if (dead) {
+      } else if (cur_fast) {
+        v[0] = cur[pass].x; v[1] = cur[pass].y; v[2] = cur[pass].z; v[3] = cur[pass].w;
 #pragma unroll
         for (int e = 0; e < 4; ++e) v[e] = fminf(fmaxf(__fmul_rn(v[e], inv), -tau), tau);
-      } else if (!dead && gr0 + line < rows_g) {
+      } else if (gr0 + line < rows_g) {
 #pragma unroll
         for (int e = 0; e < 4; ++e)
           if (gc0 + c4 + e < cols_g)
