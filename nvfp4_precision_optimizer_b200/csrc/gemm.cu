@@ -301,8 +301,11 @@ __device__ __forceinline__ void stage_store_row(float* buf, int lane, const floa
 }
 // Column cc, rows 16 hh .. 16 hh + 15 of the stage -> 16 registers.
 __device__ __forceinline__ void stage_load_col(const float* buf, int cc, int hh, float* x) {
+  // stage_off(16 hh + t, cc / 4) + cc % 4 = 272 hh + 16 t + 4 ((cc / 4) ^ ((t / 2) % 4)) + cc % 4
+  const float* b = buf + 272 * hh + (cc & 3);
+  const int q = cc >> 2;
 #pragma unroll
-  for (int t = 0; t < 16; ++t) x[t] = buf[stage_off(16 * hh + t, cc >> 2) + (cc & 3)];
+  for (int t = 0; t < 16; ++t) x[t] = b[16 * t + 4 * (q ^ ((t >> 1) & 3))];
 }
 
 // FP32 rows of tile u for the four-lanes-per-row mapping: row row0 + 32 quad +
@@ -413,6 +416,18 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
         p.ws + (E == Epi::GramX ? L.rowsumA : E == Epi::GramA ? L.rowsumB : L.rowsumX));
     float* colsum = (E == Epi::Update) ? reinterpret_cast<float*>(p.ws + L.colsumX) : rowsum;
     const bool need_col = (E == Epi::Update) ? !last : (j.mirror != 0);
+    // TILED-layout addresses of this warp's share: a per-tile base plus a per-chunk
+    // constant (the share spans one 256-column tile of each view).  The update kernel,
+    // which is tighter on registers, measured faster recomputing them per chunk.
+    const int64_t rr = gr & 127;
+    uint8_t* const rowc = row_codes + ((gr >> 7) * (row_cp >> 8) + (gc0 >> 8)) * kTileBytes + rr * 128;
+    const uint32_t rjb = (uint32_t)((gc0 & 255) >> 5), rx = (uint32_t)(rr & 7);
+    uint8_t* const rows = row_scales + ((gr >> 7) * (row_cp >> 6) + (gc0 >> 6)) * kAtomBytes +
+                          16 * (gr & 31) + 4 * ((gr & 127) >> 5);
+    uint8_t* const colc = col_codes + ((gc0 >> 7) * (d.mp >> 8) + (gr0 >> 8)) * kTileBytes + cc * 128 +
+                          ((((gr0 & 255) >> 5) ^ (cc & 7)) << 4);
+    uint8_t* const cols = col_scales + ((gc0 >> 7) * (d.mp >> 6) + (gr0 >> 6)) * kAtomBytes + 16 * cc +
+                          ((gr0 >> 4) & 3);
 
     uint32_t accr[4][32];
     if (ok) {
@@ -501,16 +516,20 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
           row_acc += q.sumsq;
           amax = fmaxf(amax, q.amax);
           if (c & 1) {
-            *reinterpret_cast<uint4*>(row_codes + tiled_chunk_offset(gr, gcc - 16, row_cp)) =
-                make_uint4(prev_w0, prev_w1, q.w0, q.w1);
+            uint8_t* dst = (E == Epi::Update)
+                               ? row_codes + tiled_chunk_offset(gr, gcc - 16, row_cp)
+                               : rowc + (((rjb + (c >> 1)) ^ rx) << 4);
+            *reinterpret_cast<uint4*>(dst) = make_uint4(prev_w0, prev_w1, q.w0, q.w1);
           } else {
             prev_w0 = q.w0;
             prev_w1 = q.w1;
           }
           scale_word |= q.scale << (8 * (c & 3));
           if ((c & 3) == 3) {
-            *reinterpret_cast<uint32_t*>(row_scales + tiled_scale_offset(gr, (gcc - 48) >> 4, row_cp)) =
-                scale_word;
+            uint8_t* dst = (E == Epi::Update)
+                               ? row_scales + tiled_scale_offset(gr, (gcc - 48) >> 4, row_cp)
+                               : rows + kAtomBytes * (c >> 2);
+            *reinterpret_cast<uint32_t*>(dst) = scale_word;
             scale_word = 0u;
           }
           if (need_col) {
@@ -521,11 +540,13 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
             const float s2 = qc.sumsq + __shfl_xor_sync(0xFFFFFFFFu, qc.sumsq, 16);
             if (hh == 0) {
               const int64_t rt = gcc + cc;
-              *reinterpret_cast<uint4*>(col_codes + tiled_chunk_offset(rt, gr0, d.mp)) =
-                  make_uint4(qc.w0, qc.w1, o0, o1);
-              *reinterpret_cast<uint16_t*>(col_scales + tiled_scale_offset(rt, gr0 >> 4, d.mp)) =
-                  static_cast<uint16_t>(qc.scale | (os << 8));
-              if (s2 != 0.0f) atomicAdd(colsum + rt, s2);
+              uint8_t* dc = (E == Epi::Update) ? col_codes + tiled_chunk_offset(rt, gr0, d.mp)
+                                               : colc + 2048 * c;
+              uint8_t* ds = (E == Epi::Update) ? col_scales + tiled_scale_offset(rt, gr0 >> 4, d.mp)
+                                               : cols + 256 * (c & 1) + 4 * (c >> 1);
+              *reinterpret_cast<uint4*>(dc) = make_uint4(qc.w0, qc.w1, o0, o1);
+              *reinterpret_cast<uint16_t*>(ds) = static_cast<uint16_t>(qc.scale | (os << 8));
+              if (s2 != 0.0f) atomicAdd(colsum + gcc + cc, s2);
             }
           }
         }
