@@ -87,6 +87,15 @@ enum {
  * as (phase + 1); 0 means run everything. */
 #define FS4_STOP_AFTER(phase) ((uint32_t)(((phase) + 1) & 0xFF) << 8)
 
+/* Test-only flag for fs4_root_ns / fs4_root_ns_batched (no counterpart in the
+ * paper): the MMA issuer of the first Gram product waits on a barrier that
+ * nothing arrives on.  The bounded wait gives up after about 2 s, records the
+ * timeout in the status word, and every later kernel of the call skips its work;
+ * fs4_device_status then returns FS4_ERR_TIMEOUT and the outputs are undefined.
+ * The CUDA context stays usable: no trap, fault or unbounded wait is involved.
+ * It exists so that the device-side timeout path can be exercised on a GPU. */
+#define FS4_TEST_STALL (1u << 30)
+
 /* Upper limits checked on the host. */
 #define FS4_MAX_DIM 65536       /* m, n of one Newton-Schulz matrix */
 #define FS4_MAX_ITERS 32        /* K */

@@ -13,15 +13,15 @@ from typing import Sequence
 import torch
 
 from . import _lib
-from ._lib import (FS4_AXIS_COL, FS4_AXIS_ROW, FS4_LAYOUT_TILED, FS4_SG_AMAX, Fs4Error, NsDesc,
-                   NsLayout, check, stop_after)
+from ._lib import (FS4_AXIS_COL, FS4_AXIS_ROW, FS4_LAYOUT_TILED, FS4_SG_AMAX, FS4_TEST_STALL,
+                   Fs4Error, NsDesc, NsLayout, check, stop_after)
 
 MUON_COEFFS = (3.4445, -4.7750, 2.0315)
 
 __all__ = [
     "quantize", "dequantize", "gemm", "root_ns", "root_ns_batched", "ns_workspace_size",
     "ns_batched_workspace_size", "ns_layout", "device_status", "tiled_shape", "Fs4Error",
-    "MUON_COEFFS", "stop_after", "FS4_AXIS_ROW", "FS4_AXIS_COL",
+    "MUON_COEFFS", "stop_after", "FS4_AXIS_ROW", "FS4_AXIS_COL", "FS4_TEST_STALL",
 ]
 
 

@@ -168,7 +168,9 @@ fs4_status run_ns(const Plan& pl, int32_t K, float clip_k, uint32_t flags, uint8
     p.iter = k;
     p.last = 0;
     if (!fill_prefix(p, pl.units_gram)) return FS4_ERR_SHAPE;
+    p.stall = (k == 0 && (flags & FS4_TEST_STALL)) ? 1 : 0;
     if ((e = launch_gemm_ns(Epi::GramX, p, st, num_sms)) != cudaSuccess) return FS4_ERR_CUDA;
+    p.stall = 0;
     if (!mark()) return FS4_ERR_CUDA;
     if (stop == 1 + 3 * k) return FS4_OK;
     if ((e = launch_gemm_ns(Epi::GramA, p, st, num_sms)) != cudaSuccess) return FS4_ERR_CUDA;
@@ -271,7 +273,7 @@ static fs4_status batched_impl(int32_t count, const fs4_ns_desc* descs, int32_t 
                                void* stream, void* const* events, int32_t n_events) {
   if (K < 1 || K > FS4_MAX_ITERS) return FS4_ERR_SHAPE;
   if (!std::isfinite(clip_k)) return FS4_ERR_INVALID_ARG;
-  if (flags & ~(uint32_t)0xFF00u) return FS4_ERR_INVALID_ARG;
+  if (flags & ~(uint32_t)(0xFF00u | FS4_TEST_STALL)) return FS4_ERR_INVALID_ARG;
   static thread_local Plan pl;
   const fs4_status s = make_plan(count, descs, &pl);
   if (s != FS4_OK) return s;

@@ -236,8 +236,9 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 }
 
 // Test for completion of the phase with `parity`; if it is not complete the thread
-// may be suspended (it stops issuing) until it completes or about kSuspendNs pass.
-constexpr uint32_t kSuspendNs = 1000000u;
+// may be suspended (it stops issuing) until it completes or about kSuspendNs pass
+// (which also bounds how late a waiter notices an abort).
+constexpr uint32_t kSuspendNs = 20000u;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -251,15 +252,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with `parity` of `bar` to complete.  Gives up after
-// kWaitLimitNs (or at once if *abort is already set), records the timeout in
-// the status word and returns false.
+// kWaitLimitNs (or within about kSuspendNs of *abort being set), records the
+// timeout in the status word and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status,
                                           volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
+    if (mbar_try_wait(bar, parity)) return true;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       atomicOr(status, kStatusTimeout);
       *abort = 1;

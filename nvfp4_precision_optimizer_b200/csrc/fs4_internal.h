@@ -94,6 +94,7 @@ struct NsParams {
   int32_t count;
   int32_t iter;            // k of the current iteration
   int32_t last;            // 1 on the final update product (writes `out`)
+  int32_t stall;           // test only: the MMA issuer waits on a barrier nothing arrives on
   float clip_k;
   uint32_t* status;
   uint8_t* ws;             // workspace base

@@ -84,7 +84,7 @@ struct Cfg {
   static constexpr uint32_t kIdesc = idesc_mxf4nvf4(kPair ? 2 * BM : BM, BN);
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(SMEM_BYTES <= 232448, "over the per-CTA shared-memory limit");
-  static_assert((3 * kStages + 3) * 8 + 12 <= BAR_BYTES, "barrier block too small");
+  static_assert((3 * kStages + 4) * 8 + 12 <= BAR_BYTES, "barrier block too small");
 };
 
 struct Job {
@@ -643,7 +643,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = bars + 3 * kStages;
   uint64_t* acc_empty = acc_full + 1;         // (leader) both CTAs drained the accumulator
   uint64_t* mma_done = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 3);
+  uint64_t* stall_bar = acc_full + 3;        // test only: never arrived on
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 4);
   uint32_t* arrivals = tmem_slot + 1;   // monotonic count of (epilogue warp, tile) completions
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   float2* scale_tab = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(bars) + C::BAR_BYTES);
@@ -665,6 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, kPair ? 16 : 8);
     mbar_init(mma_done, 1);
+    mbar_init(stall_bar, 1);
     *arrivals = 0u;
     *abort_flag = (__ldcg(status) & kStatusTimeout) ? 1 : 0;
     fence_mbar_init();
@@ -748,6 +750,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint16_t kBoth = kPair ? 3 : 1;
       uint32_t it = 0, tl = 0;
       const uint32_t acc = tmem;   // lane 0, column 0
+      if constexpr (E != Epi::Plain) {
+        // test only: a wait that runs out (bounded), exercising the timeout path
+        if (p.stall) mbar_wait(stall_bar, 0, status, abort_flag);
+      }
       for (int32_t u = first; u < total && !*abort_flag; u += step, ++tl) {
         const Job j = make_job<E>(u, p, g, rank);
         if (!mbar_wait(acc_empty, (tl & 1u) ^ 1u, status, abort_flag)) break;

@@ -94,6 +94,9 @@ def test_root_ns_rejects_bad_arguments(F):
     assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 3.0, 0, G, ok, None) == -3         # ws overlaps G
     assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 3.0, 0, W + 4, ok, None) == -4     # misaligned ws
     assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 3.0, 1 << 3, W, ok, None) == -1    # unknown flag
+    assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 3.0, 1 << 29, W, ok, None) == -1   # unknown flag
+    # the test-only stall flag is accepted (the call then fails on the workspace size)
+    assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 3.0, F.FS4_TEST_STALL, W, ok - 1, None) == -4
 
 
 def test_batched_rejects_overlapping_outputs_and_bad_counts(F):

@@ -238,3 +238,22 @@ def test_nonfinite_input_reports_status_and_zero_output(fs4):
     out = fs4.root_ns(Gt, 3, workspace=ws)
     assert fs4.device_status(ws) == -7
     assert not out.cpu().numpy().any()
+
+
+def test_bounded_wait_timeout_reports_status_and_context_survives(fs4):
+    """A device wait that runs out (FS4_TEST_STALL: the first Gram product's MMA issuer
+    waits on a barrier nothing arrives on) ends the call with FS4_ERR_TIMEOUT in the
+    status word within a few seconds, with no fault; the next call on the same stream
+    is correct."""
+    import time
+    G = momentum(256, 256, seed=11)
+    Gt = torch.from_numpy(G).cuda()
+    ws = torch.zeros(fs4.ns_workspace_size(256, 256), dtype=torch.uint8, device="cuda")
+    t0 = time.time()
+    fs4.root_ns(Gt, 2, *MUON, workspace=ws, flags=fs4.FS4_TEST_STALL)
+    torch.cuda.synchronize()
+    assert time.time() - t0 < 30.0
+    assert fs4.device_status(ws) == -8          # FS4_ERR_TIMEOUT
+    got, ws2 = run_gpu(fs4, G, 2, MUON)         # fresh workspace, same context
+    want = R.root_ns(G, 2, *MUON, clip_k=3.0)
+    assert rel_frob(got, want) <= 2e-2
