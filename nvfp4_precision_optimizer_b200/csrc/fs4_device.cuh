@@ -165,11 +165,39 @@ __device__ __forceinline__ float2 scale_tab_entry(uint32_t b) {
   return make_float2(v, __frcp_rn(v));
 }
 
+// ------------------------------------------------------------------ packed FP32 pairs
+// sm_100 executes FP32 multiply and FMA on register pairs (f32x2); each lane of the
+// pair is rounded exactly like the scalar instruction.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+// div_rn_fma on a pair: nd = (-d, -d), rcp = (RN(1/d), RN(1/d)).
+__device__ __forceinline__ uint64_t div2_rn_fma(uint64_t x, uint64_t nd, uint64_t rcp) {
+  const uint64_t q0 = f2_mul(x, rcp);
+  return f2_fma(f2_fma(q0, nd, x), rcp, q0);
+}
+
 // Quantise 16 FP32 values with tensor scale s_g (six_sg = fp32(6 * s_g)).
 // kPow2: s_g is a power of two and rcp_six = RN(1 / six_sg), so the block scale
 // division may use the FMA-corrected form; otherwise IEEE division is used.
 // With a table (kPow2 only) the decoded block scale and its reciprocal are looked up.
-template <bool kPow2, bool kTab = false>
+// kPacked: divide in f32x2 pairs (fewer instructions; the same roundings).
+template <bool kPow2, bool kTab = false, bool kPacked = true>
 __device__ __forceinline__ QBlock16 quantize16(const float* x, float s_g, float six_sg, float rcp_six,
                                                ScaleTab st = ScaleTab{nullptr, 0.0f}) {
   static_assert(kPow2 || !kTab, "the scale table needs a power-of-two tensor scale");
@@ -198,7 +226,12 @@ __device__ __forceinline__ QBlock16 quantize16(const float* x, float s_g, float 
     if (kPow2) rcp = __frcp_rn(den);
   }
   float q[16];
-  if (kPow2) {
+  if (kPow2 && kPacked) {
+    const uint64_t nd2 = f2_pack(-den, -den), rcp2 = f2_pack(rcp, rcp);
+#pragma unroll
+    for (int i = 0; i < 16; i += 2)
+      f2_unpack(div2_rn_fma(f2_pack(x[i], x[i + 1]), nd2, rcp2), q[i], q[i + 1]);
+  } else if (kPow2) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) q[i] = div_rn_fma(x[i], den, rcp);
   } else {

@@ -360,6 +360,7 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
                                             int32_t first, int32_t step, int quad, int ch,
                                             int lane, int32_t total) {
   constexpr bool kIn = (E == Epi::GramA || E == Epi::Update);   // reads an FP32 tile
+  constexpr bool kPackedQ = (E != Epi::Update);   // f32x2 quantiser (measured per kernel)
   const int k = p.iter;
   const int cc = lane & 15, hh = lane >> 4;
   TileRows fp{nullptr, 0u};   // FP32 tile rows of the current tile
@@ -462,16 +463,33 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
       if (ok) {
         const int64_t gcc = gc0 + kChunkCols * c;   // first column of the chunk
         float y[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) y[e] = __uint_as_float(accr[c >> 1][16 * (c & 1) + e]) * acc_scale;
-        if constexpr (kIn) {
+        const uint64_t s2 = f2_pack(acc_scale, acc_scale);
+        if constexpr (E == Epi::Update) {
+          // (the paired update kernel measured faster with scalar arithmetic here)
           float xin[16];
           stage_load_row(buf, lane, xin);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            if constexpr (E == Epi::Update) y[e] = fmaf(d.a, xin[e], y[e]);
-            else y[e] = fmaf(d.b, xin[e], d.c * y[e]);
+          for (int e = 0; e < 16; ++e)
+            y[e] = fmaf(d.a, xin[e], __uint_as_float(accr[c >> 1][16 * (c & 1) + e]) * acc_scale);
+        } else if constexpr (kIn) {
+          // GramA: b A + c (s acc)   (pairs of columns at a time)
+          float xin[16];
+          stage_load_row(buf, lane, xin);
+          const uint64_t ca = f2_pack(d.b, d.b);
+          const uint64_t cc2 = f2_pack(d.c, d.c);
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            uint64_t v = f2_mul(f2_pack(__uint_as_float(accr[c >> 1][16 * (c & 1) + e]),
+                                        __uint_as_float(accr[c >> 1][16 * (c & 1) + e + 1])), s2);
+            if constexpr (E == Epi::GramA) v = f2_mul(cc2, v);
+            f2_unpack(f2_fma(ca, f2_pack(xin[e], xin[e + 1]), v), y[e], y[e + 1]);
           }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; e += 2)
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(accr[c >> 1][16 * (c & 1) + e]),
+                                     __uint_as_float(accr[c >> 1][16 * (c & 1) + e + 1])), s2),
+                      y[e], y[e + 1]);
         }
         if (last) {
           // final iteration: write the output (transposed back for a tall input)
@@ -508,10 +526,10 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
           if (need_col) {
             float xc[16];
             stage_load_col(buf, cc, hh, xc);
-            q = quantize16<true, true>(y, sg_out, six_out, rcp_six, stab);
-            qc = quantize16<true, true>(xc, sg_out, six_out, rcp_six, stab);
+            q = quantize16<true, true, kPackedQ>(y, sg_out, six_out, rcp_six, stab);
+            qc = quantize16<true, true, kPackedQ>(xc, sg_out, six_out, rcp_six, stab);
           } else {
-            q = quantize16<true, true>(y, sg_out, six_out, rcp_six, stab);
+            q = quantize16<true, true, kPackedQ>(y, sg_out, six_out, rcp_six, stab);
           }
           row_acc += q.sumsq;
           amax = fmaxf(amax, q.amax);
