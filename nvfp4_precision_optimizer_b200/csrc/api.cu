@@ -95,10 +95,9 @@ fs4_status make_plan(int32_t count, const fs4_ns_desc* descs, Plan* pl) {
     pl->units_reduce[i] = (d.m + 15) / 16;
     pl->units_pre[i] = (int64_t)(md.mp / 64) * (md.np / 64);
     const int64_t T = md.mp / 256;
-    // Gram units: 128-row halves of the 256 x 256 tiles on and above the diagonal;
-    // update units: 256 x 256 tiles, each computed by a CTA pair
+    // GEMM units: 128 x 256 tiles (Gram products: on and above the 256-block diagonal)
     pl->units_gram[i] = T * (T + 1);
-    pl->units_upd[i] = (int64_t)(md.mp / 256) * (md.np / 256);
+    pl->units_upd[i] = (int64_t)(md.mp / 128) * (md.np / 256);
   }
   pl->zero_bytes = align_up(off, 1024);
   off = pl->zero_bytes;

@@ -66,25 +66,20 @@ constexpr int EPI_WARP_FLOATS = kStageBufs * kStageFloats;
 static_assert(EPI_WARP_FLOATS >= TRANS_FLOATS, "the plain epilogue reuses the stage");
 constexpr float kBoundInflate = 1.0f + 1.0f / 256.0f;
 
-// Per-kernel configuration.  The plain GEMM and the two Gram products run one CTA
-// per 128 x 256 tile.  The update GEMM runs as CTA pairs (a cluster of 2) on
-// 256 x 256 tiles with tcgen05 cta_group::2: each CTA stages its own 128 rows of A
-// and 128 of B's 256 rows (the pair's tensor cores share both halves), so a stage
-// is 38 KB instead of 54 KB and four of them fit beside the epilogue staging.
+// Per-kernel configuration.
 template <Epi E>
 struct Cfg {
-  static constexpr bool kPair = (E == Epi::Update);
-  static constexpr int kG = kPair ? 2 : 1;                       // cta_group
-  static constexpr int kStages = kPair ? 4 : 3;
-  static constexpr int B_BYTES = (kPair ? BN / 2 : BN) * BK / 2;  // B rows staged per CTA
+  static constexpr int kStages = 3;
+  static constexpr int B_BYTES = BN * BK / 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int BAR_BYTES = 256;
+  static constexpr int EPI_FLOATS = kStageBufs * kStageFloats;
   static constexpr int SMEM_BYTES =
-      1024 + kStages * STAGE_BYTES + 8 * EPI_WARP_FLOATS * 4 + BAR_BYTES + 128 * 8;
-  static constexpr uint32_t kIdesc = idesc_mxf4nvf4(kPair ? 2 * BM : BM, BN);
+      1024 + kStages * STAGE_BYTES + 8 * EPI_FLOATS * 4 + BAR_BYTES + 128 * 8;
+  static constexpr uint32_t kIdesc = idesc_mxf4nvf4(BM, BN);
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(SMEM_BYTES <= 232448, "over the per-CTA shared-memory limit");
-  static_assert((3 * kStages + 4) * 8 + 12 <= BAR_BYTES, "barrier block too small");
+  static_assert((2 * kStages + 4) * 8 + 12 <= BAR_BYTES, "barrier block too small");
 };
 
 struct Job {
@@ -115,15 +110,15 @@ __device__ __forceinline__ void upper_tile(int32_t s, int32_t T, int32_t& P, int
   Q = P + s;
 }
 
-// Work unit u of kernel E for this CTA (rank = its place in a CTA pair).
+// Work unit u of kernel E: one 128 x 256 output tile.  The Newton-Schulz units of a
+// matrix go through its 256 x 256 blocks in order, the two 128-row halves of a block
+// one after the other (they share the block's B rows in L2).
 template <Epi E>
-__device__ __forceinline__ Job make_job(int32_t u, const NsParams& p, const GemmPlainArgs& g,
-                                        uint32_t rank) {
+__device__ __forceinline__ Job make_job(int32_t u, const NsParams& p, const GemmPlainArgs& g) {
   Job j;
   j.mirror = 0;
   j.b_half = 0;
   if constexpr (E == Epi::Plain) {
-    (void)rank;
     const int32_t nJ = (g.Np + BN - 1) / BN;
     const int32_t I = u / nJ;
     j.mat = 0;
@@ -141,10 +136,7 @@ __device__ __forceinline__ Job make_job(int32_t u, const NsParams& p, const Gemm
     const int32_t lu = u - p.prefix[mi];
     const int slot = p.iter & 1;
     j.mat = mi;
-    // a pair's unit is a 256 x 256 tile (this CTA: rows 128 * rank ..); a single
-    // CTA's unit is one 128-row half of it
-    const int32_t tu = Cfg<E>::kPair ? lu : (lu >> 1);
-    const int32_t half = Cfg<E>::kPair ? (int32_t)rank : (lu & 1);
+    const int32_t tu = lu >> 1, half = lu & 1;   // 256 x 256 block, 128-row half
     if constexpr (E == Epi::GramX || E == Epi::GramA) {
       const int32_t T = d.mp / 256;
       int32_t P, Q;
@@ -233,8 +225,7 @@ __device__ __forceinline__ void finalize_tile(const NsParams& p, int mi, int lan
     constexpr int kind = (E == Epi::GramX) ? 1 : (E == Epi::GramA ? 2 : 3);
     int last = 0;
     if (lane == 0) {
-      // a pair's unit is one 128-row tile in each of its two CTAs
-      const uint32_t tiles = (Cfg<E>::kPair ? 2u : 1u) * (uint32_t)(p.prefix[mi + 1] - p.prefix[mi]);
+      const uint32_t tiles = (uint32_t)(p.prefix[mi + 1] - p.prefix[mi]);
       last = (atomicAdd(&st->done[kind], 1u) == tiles - 1u) ? 1 : 0;
     }
     last = __shfl_sync(0xFFFFFFFFu, last, 0);
@@ -318,8 +309,8 @@ struct TileRows {
 
 template <Epi E>
 __device__ __forceinline__ TileRows tile_rows(const NsParams& p, const GemmPlainArgs& g, int32_t u,
-                                              uint32_t rank, int quad, int ch, int lane) {
-  const Job j = make_job<E>(u, p, g, rank);
+                                              int quad, int ch, int lane) {
+  const Job j = make_job<E>(u, p, g);
   const MatDesc& d = p.mat[j.mat];
   const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
   const int64_t pitch = (E == Epi::Update) ? d.np : d.mp;
@@ -356,9 +347,9 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
                                             uint32_t tmem, uint64_t* acc_full,
                                             uint64_t* acc_empty, uint32_t* arrivals,
                                             uint32_t* status, volatile int* abort_flag,
-                                            float* wbuf, const float2* scale_tab, uint32_t rank,
-                                            int32_t first, int32_t step, int quad, int ch,
+                                            float* wbuf, const float2* scale_tab, int quad, int ch,
                                             int lane, int32_t total) {
+  const int32_t first = blockIdx.x, step = gridDim.x;
   constexpr bool kIn = (E == Epi::GramA || E == Epi::Update);   // reads an FP32 tile
   constexpr bool kPackedQ = (E != Epi::Update);   // f32x2 quantiser (measured per kernel)
   const int k = p.iter;
@@ -367,7 +358,7 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
   TileRows fn{nullptr, 0u};   // ... of the next tile (fetched ahead)
   if constexpr (kIn) {
     if (first < total) {
-      fp = tile_rows<E>(p, g, first, rank, quad, ch, lane);
+      fp = tile_rows<E>(p, g, first, quad, ch, lane);
       stage_fetch(wbuf, fp, 0, lane);
       cp_async_commit();
       stage_fetch(wbuf + kStageFloats, fp, 1, lane);
@@ -377,11 +368,11 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
   int b = 0;   // stage buffer of the current chunk
   uint32_t tl = 0;
   for (int32_t u = first; u < total; u += step, ++tl) {
-    const Job j = make_job<E>(u, p, g, rank);
+    const Job j = make_job<E>(u, p, g);
     const MatDesc& d = p.mat[j.mat];
     NsState* st = reinterpret_cast<NsState*>(p.ws + d.state_off);
     const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
-    if constexpr (!kIn) fp = tile_rows<E>(p, g, u, rank, quad, ch, lane);
+    if constexpr (!kIn) fp = tile_rows<E>(p, g, u, quad, ch, lane);
     // warp-uniform by construction: the chunk loop shuffles under this condition
     const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, tl & 1u, status, abort_flag));
     const int64_t gr0 = j.row0 + 32 * quad;   // first row of this warp's band
@@ -444,11 +435,7 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
       tmem_ld_order(accr[3]);
       tc_fence_before();
       __syncwarp();
-      // the accumulator barrier lives in the pair's leader (rank 0)
-      if (lane == 0) {
-        if (rank == 0) mbar_arrive(acc_empty);
-        else mbar_arrive_cluster(acc_empty, 0);
-      }
+      if (lane == 0) mbar_arrive(acc_empty);
     }
 
     float row_acc = 0.0f, amax = 0.0f;
@@ -465,7 +452,7 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
         float y[16];
         const uint64_t s2 = f2_pack(acc_scale, acc_scale);
         if constexpr (E == Epi::Update) {
-          // (the paired update kernel measured faster with scalar arithmetic here)
+          // (the update kernel measured faster with scalar arithmetic here)
           float xin[16];
           stage_load_row(buf, lane, xin);
 #pragma unroll
@@ -577,7 +564,7 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
         if (c + 2 < kChunks) {
           stage_fetch(nb, fp, c + 2, lane);
         } else if (more) {
-          if (c + 2 == kChunks) fn = tile_rows<E>(p, g, u + step, rank, quad, ch, lane);
+          if (c + 2 == kChunks) fn = tile_rows<E>(p, g, u + step, quad, ch, lane);
           stage_fetch(nb, fn, c + 2 - kChunks, lane);
         }
         cp_async_commit();
@@ -609,7 +596,7 @@ __device__ __forceinline__ void epilogue_plain(const NsParams& p, const GemmPlai
                                                int ch, int lane, int32_t total) {
   uint32_t tl = 0;
   for (int32_t u = blockIdx.x; u < total; u += gridDim.x, ++tl) {
-    const Job j = make_job<Epi::Plain>(u, p, g, 0u);
+    const Job j = make_job<Epi::Plain>(u, p, g);
     const bool ok = mbar_wait(acc_full, tl & 1u, status, abort_flag);
     if (!ok) continue;
     const int64_t gr0 = j.row0 + 32 * quad;
@@ -647,19 +634,16 @@ template <Epi E>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ NsParams p, const __grid_constant__ GemmPlainArgs g) {
   using C = Cfg<E>;
-  constexpr bool kPair = C::kPair;
-  constexpr int G = C::kG;
   constexpr int kStages = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   float* epi_smem = reinterpret_cast<float*>(smem + kStages * C::STAGE_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * C::STAGE_BYTES + 8 * EPI_WARP_FLOATS * 4);
-  uint64_t* full = bars;                      // this CTA's operand stage landed
+  uint64_t* full = bars;                      // an operand stage landed
   uint64_t* empty = bars + kStages;           // the MMAs reading a stage finished
-  uint64_t* peer_full = bars + 2 * kStages;   // (leader) the peer's stage landed
-  uint64_t* acc_full = bars + 3 * kStages;
-  uint64_t* acc_empty = acc_full + 1;         // (leader) both CTAs drained the accumulator
+  uint64_t* acc_full = bars + 2 * kStages;
+  uint64_t* acc_empty = acc_full + 1;         // the epilogue warps drained the accumulator
   uint64_t* mma_done = acc_full + 2;
   uint64_t* stall_bar = acc_full + 3;        // test only: never arrived on
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 4);
@@ -670,29 +654,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint32_t* status = (E == Epi::Plain) ? g.status : p.status;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // CTA pairs: cluster c = CTAs 2c (leader, rank 0) and 2c + 1 walk the same units
-  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
-  const int32_t first = kPair ? (int32_t)(blockIdx.x >> 1) : (int32_t)blockIdx.x;
-  const int32_t step = kPair ? (int32_t)(gridDim.x >> 1) : (int32_t)gridDim.x;
+  const int32_t first = blockIdx.x, step = gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&peer_full[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, kPair ? 16 : 8);
+    mbar_init(acc_empty, 8);
     mbar_init(mma_done, 1);
     mbar_init(stall_bar, 1);
     *arrivals = 0u;
     *abort_flag = (__ldcg(status) & kStatusTimeout) ? 1 : 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc<G>(tmem_slot, kTmemCols);
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
-  if constexpr (kPair) cluster_sync();   // the peer's barriers exist before any remote arrive
-  else __syncthreads();
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int32_t total = total_units<E>(p, g);
@@ -703,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t it = 0;
       for (int32_t u = first; u < total && !*abort_flag; u += step) {
-        const Job j = make_job<E>(u, p, g, rank);
+        const Job j = make_job<E>(u, p, g);
         for (int kt = 0; kt < j.kt; ++kt, ++it) {
           const uint32_t s = it % kStages, use = it / kStages;
           if (!mbar_wait(&empty[s], (use & 1u) ^ 1u, status, abort_flag)) break;
@@ -712,29 +691,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* st_sfa = st_b + C::B_BYTES;
           uint8_t* st_sfb = st_sfa + SFA_BYTES;
           const int64_t at = j.a_tile_row * j.ktiles_total + kt;
-          if constexpr (kPair) {
-            // own 128 rows of A, own 128 of B's 256 rows, the scales of all 256 B rows
-            mbar_arrive_expect_tx(&full[s], A_BYTES + SFA_BYTES + C::B_BYTES + SFB_BYTES);
-            bulk_g2s(st, j.a_codes + at * kTileBytes, A_BYTES, &full[s]);
-            bulk_g2s(st_sfa, j.a_sf + at * (4 * kAtomBytes), SFA_BYTES, &full[s]);
-            const int64_t bt_own = (j.b_tile_row + rank) * j.ktiles_total + kt;
-            bulk_g2s(st_b, j.b_codes + bt_own * kTileBytes, kTileBytes, &full[s]);
-            for (int h = 0; h < 2; ++h) {
-              const int64_t bt = (j.b_tile_row + h) * j.ktiles_total + kt;
-              bulk_g2s(st_sfb + h * (4 * kAtomBytes), j.b_sf + bt * (4 * kAtomBytes), 4 * kAtomBytes,
-                       &full[s]);
-            }
-          } else {
-            const uint32_t bbytes = j.b_half ? (C::B_BYTES + SFB_BYTES) / 2 : (C::B_BYTES + SFB_BYTES);
-            mbar_arrive_expect_tx(&full[s], A_BYTES + SFA_BYTES + bbytes);
-            bulk_g2s(st, j.a_codes + at * kTileBytes, A_BYTES, &full[s]);
-            bulk_g2s(st_sfa, j.a_sf + at * (4 * kAtomBytes), SFA_BYTES, &full[s]);
-            for (int h = 0; h < (j.b_half ? 1 : 2); ++h) {
-              const int64_t bt = (j.b_tile_row + h) * j.ktiles_total + kt;
-              bulk_g2s(st_b + h * kTileBytes, j.b_codes + bt * kTileBytes, kTileBytes, &full[s]);
-              bulk_g2s(st_sfb + h * (4 * kAtomBytes), j.b_sf + bt * (4 * kAtomBytes), 4 * kAtomBytes,
-                       &full[s]);
-            }
+          const uint32_t bbytes = j.b_half ? (C::B_BYTES + SFB_BYTES) / 2 : (C::B_BYTES + SFB_BYTES);
+          mbar_arrive_expect_tx(&full[s], A_BYTES + SFA_BYTES + bbytes);
+          bulk_g2s(st, j.a_codes + at * kTileBytes, A_BYTES, &full[s]);
+          bulk_g2s(st_sfa, j.a_sf + at * (4 * kAtomBytes), SFA_BYTES, &full[s]);
+          for (int h = 0; h < (j.b_half ? 1 : 2); ++h) {
+            const int64_t bt = (j.b_tile_row + h) * j.ktiles_total + kt;
+            bulk_g2s(st_b + h * kTileBytes, j.b_codes + bt * kTileBytes, kTileBytes, &full[s]);
+            bulk_g2s(st_sfb + h * (4 * kAtomBytes), j.b_sf + bt * (4 * kAtomBytes), 4 * kAtomBytes,
+                     &full[s]);
           }
         }
       }
@@ -746,26 +711,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (kPair && rank != 0) {
-      // ---------------------------------------------------------- relay (pair's peer)
-      // Tell the leader's MMA thread each time one of this CTA's stages has landed.
-      if (lane == 0) {
-        uint32_t it = 0;
-        bool ok = true;
-        for (int32_t u = first; u < total && ok && !*abort_flag; u += step) {
-          const Job j = make_job<E>(u, p, g, rank);
-          for (int kt = 0; kt < j.kt; ++kt, ++it) {
-            const uint32_t s = it % kStages, use = it / kStages;
-            if (!mbar_wait(&full[s], use & 1u, status, abort_flag)) { ok = false; break; }
-            mbar_arrive_cluster(&peer_full[s], 0);
-          }
-        }
-      }
-    } else if (lane == 0) {
+    if (lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      // (the pair's leader issues for both CTAs: operands and accumulators of each
-      // CTA stay in that CTA; commits arrive on the barriers of both)
-      constexpr uint16_t kBoth = kPair ? 3 : 1;
       uint32_t it = 0, tl = 0;
       const uint32_t acc = tmem;   // lane 0, column 0
       if constexpr (E != Epi::Plain) {
@@ -773,14 +720,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (p.stall) mbar_wait(stall_bar, 0, status, abort_flag);
       }
       for (int32_t u = first; u < total && !*abort_flag; u += step, ++tl) {
-        const Job j = make_job<E>(u, p, g, rank);
+        const Job j = make_job<E>(u, p, g);
         if (!mbar_wait(acc_empty, (tl & 1u) ^ 1u, status, abort_flag)) break;
         tc_fence_after();
         bool ok = true;
         for (int kt = 0; kt < j.kt; ++kt, ++it) {
           const uint32_t s = it % kStages, use = it / kStages;
           if (!mbar_wait(&full[s], use & 1u, status, abort_flag)) { ok = false; break; }
-          if (kPair && !mbar_wait(&peer_full[s], use & 1u, status, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint8_t* st = stage_base + s * C::STAGE_BYTES;
           const uint32_t sa = smem_addr(st), sb = sa + A_BYTES;
@@ -788,22 +734,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sf = tmem + kSfCol + (it & 1u) * kSfBufCols;
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
-            tc_copy_sf<G>(sf + 4 * ks, sdesc_sf_atom(ssfa + ks * kAtomBytes));
-            tc_copy_sf<G>(sf + 16 + 8 * ks, sdesc_sf_atom(ssfb + ks * kAtomBytes));
-            tc_copy_sf<G>(sf + 16 + 8 * ks + 4, sdesc_sf_atom(ssfb + 4 * kAtomBytes + ks * kAtomBytes));
+            tc_copy_sf(sf + 4 * ks, sdesc_sf_atom(ssfa + ks * kAtomBytes));
+            tc_copy_sf(sf + 16 + 8 * ks, sdesc_sf_atom(ssfb + ks * kAtomBytes));
+            tc_copy_sf(sf + 16 + 8 * ks + 4, sdesc_sf_atom(ssfb + 4 * kAtomBytes + ks * kAtomBytes));
           }
           const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sb);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
-            tc_mma_nvf4<G>(acc, da + 2 * ks, db + 2 * ks, C::kIdesc, sf + 4 * ks, sf + 16 + 8 * ks,
-                           (kt | ks) != 0 ? 1u : 0u);
+            tc_mma_nvf4(acc, da + 2 * ks, db + 2 * ks, C::kIdesc, sf + 4 * ks, sf + 16 + 8 * ks,
+                        (kt | ks) != 0 ? 1u : 0u);
           }
-          tc_commit<G>(&empty[s], kBoth);
+          tc_commit(&empty[s]);
         }
         if (!ok) break;
-        tc_commit<G>(acc_full, kBoth);
+        tc_commit(acc_full);
       }
-      tc_commit<G>(mma_done, 1);
+      tc_commit(mma_done);
       volatile int never = 0;
       mbar_wait(mma_done, 0, status, &never);
     }
@@ -816,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (E != Epi::Plain) {
       uint32_t tl = 0;
       for (int32_t u = first; u < total; u += step, ++tl) {
-        const Job j = make_job<E>(u, p, g, rank);
+        const Job j = make_job<E>(u, p, g);
         const uint32_t target = 8u * (tl + 1u);
         bool seen = true;
         if (*reinterpret_cast<volatile uint32_t*>(arrivals) < target) {
@@ -849,17 +795,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       epilogue_plain(p, g, tmem, acc_full, acc_empty, status, abort_flag, wbuf, quad, ch, lane, total);
     else
       epilogue_ns<E>(p, g, tmem, acc_full, acc_empty, arrivals, status, abort_flag, wbuf, scale_tab,
-                     rank, first, step, quad, ch, lane, total);
+                     quad, ch, lane, total);
   }
 
   tc_fence_before();
-  // both CTAs of a pair are done with the TMEM (the leader's MMAs completed before
-  // its MMA thread got here) before either frees it
-  if constexpr (kPair) cluster_sync();
-  else __syncthreads();
+  __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc<G>(tmem, kTmemCols);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -868,7 +811,6 @@ cudaError_t launch_impl(const NsParams* p, const GemmPlainArgs* g, int64_t units
                         int num_sms) {
   using C = Cfg<E>;
   static unsigned long long attr_set = 0ull;   // one bit per device; a benign race
-  static int max_pairs = 0;                    // co-resident CTA pairs (same on every B200)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -884,38 +826,11 @@ cudaError_t launch_impl(const NsParams* p, const GemmPlainArgs* g, int64_t units
   e = cudaFuncGetAttributes(&fa, nvfp4_gemm_kernel<E>);
   if (e != cudaSuccess) return e;
   if ((uint32_t)fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
+  const int grid = (int)(units < num_sms ? (units > 0 ? units : 1) : num_sms);
   static const NsParams zero_p{};
   static const GemmPlainArgs zero_g{};
-  if constexpr (!C::kPair) {
-    const int grid = (int)(units < num_sms ? (units > 0 ? units : 1) : num_sms);
-    nvfp4_gemm_kernel<E><<<grid, kThreads, C::SMEM_BYTES, st>>>(p ? *p : zero_p, g ? *g : zero_g);
-    return cudaGetLastError();
-  } else {
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = C::SMEM_BYTES;
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (max_pairs == 0) {
-      cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
-      int n = 0;
-      e = cudaOccupancyMaxActiveClusters(&n, nvfp4_gemm_kernel<E>, &cfg);
-      if (e != cudaSuccess) return e;
-      if (n < 1) return cudaErrorInvalidConfiguration;
-      max_pairs = n;
-    }
-    const int64_t pairs = units < max_pairs ? (units > 0 ? units : 1) : max_pairs;
-    cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
-    e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<E>, p ? *p : zero_p, g ? *g : zero_g);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
-  }
+  nvfp4_gemm_kernel<E><<<grid, kThreads, C::SMEM_BYTES, st>>>(p ? *p : zero_p, g ? *g : zero_g);
+  return cudaGetLastError();
 }
 
 }  // namespace
