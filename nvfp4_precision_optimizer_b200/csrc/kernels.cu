@@ -294,9 +294,7 @@ __global__ void __launch_bounds__(kEwThreads) ns_reduce_kernel(const __grid_cons
 // are read and written as float4 with 16 threads per 64-float row segment.
 __global__ void __launch_bounds__(kEwThreads) ns_preamble_kernel(const __grid_constant__ NsParams p) {
   __shared__ float tile[kT][kT + 1];
-  __shared__ float red[kEwThreads / 32];
   __shared__ float2 scale_tab[128];
-  __shared__ int s_last;
   const int32_t total = p.prefix[p.count];
   const int t = threadIdx.x;
   if (t < 128) scale_tab[t] = scale_tab_entry(t);   // read after the first barrier below
@@ -419,27 +417,26 @@ __global__ void __launch_bounds__(kEwThreads) ns_preamble_kernel(const __grid_co
       if (blk == 0 && ss != 0.0f)
         atomicAdd(reinterpret_cast<float*>(p.ws + (view == 0 ? L.rowsumX : L.colsumX)) + R, ss);
     }
-    // the last CTA of this matrix turns the sums into the bounds the next phase needs;
-    // the threads that issued (fire-and-forget) sum atomics fence them before the count
-    if ((t & 3) == 0) __threadfence();
-    __syncthreads();
-    if (t == 0) {
-      const uint32_t units = (uint32_t)(p.prefix[mi + 1] - p.prefix[mi]);
-      s_last = (atomicAdd(&st->done[0], 1u) == units - 1u);
-    }
-    __syncthreads();
-    if (s_last) {            // block-uniform
-      __threadfence();
-      const float ur = drain_max(reinterpret_cast<float*>(p.ws + L.rowsumX), d.mp, red);
-      const float uc = drain_max(reinterpret_cast<float*>(p.ws + L.colsumX), d.np, red);
-      if (t == 0) {
-        st->u_rowX[0] = ur;
-        st->u_colX[0] = uc;
-        st->sg[kSgA + 0] = pow2_tensor_scale(ur * kBoundInflate);
-        st->done[0] = 0u;
-      }
-    }
-    __syncthreads();
+    __syncthreads();   // the tile is restaged by the next unit
+  }
+}
+
+// After the preamble: each matrix's bounds for the first Gram product from the row and
+// column sums of its quantised X_0 (one CTA per matrix; the sum vectors are cleared for
+// the update phases).  A separate launch orders the preamble's sum atomics before
+// these reads, so the preamble needs no fence or completion counter.
+__global__ void __launch_bounds__(kEwThreads) ns_preamble_bounds_kernel(const __grid_constant__ NsParams p) {
+  __shared__ float red[kEwThreads / 32];
+  const int mi = blockIdx.x;
+  const MatDesc& d = p.mat[mi];
+  NsState* st = state_of(p, d);
+  const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
+  const float ur = drain_max(reinterpret_cast<float*>(p.ws + L.rowsumX), d.mp, red);
+  const float uc = drain_max(reinterpret_cast<float*>(p.ws + L.colsumX), d.np, red);
+  if (threadIdx.x == 0) {
+    st->u_rowX[0] = ur;
+    st->u_colX[0] = uc;
+    st->sg[kSgA + 0] = pow2_tensor_scale(ur * kBoundInflate);
   }
 }
 
@@ -503,6 +500,9 @@ cudaError_t launch_ns_reduce(const NsParams& p, cudaStream_t st, int num_sms) {
 
 cudaError_t launch_ns_preamble(const NsParams& p, cudaStream_t st, int num_sms) {
   ns_preamble_kernel<<<persistent_grid(ns_preamble_kernel, p.prefix[p.count], num_sms), kEwThreads, 0, st>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  ns_preamble_bounds_kernel<<<p.count, kEwThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 
