@@ -371,7 +371,7 @@ def main():
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": args.steps * (3 + 3 * K),
+            "gpu_launches": args.steps * (2 + 6 * K),
             "clocks": sampler.summary(),
         }
         print(json.dumps(line), flush=True)

@@ -187,7 +187,7 @@ fs4_status fs4_root_ns(const float* G, int64_t m, int64_t n, int64_t ld, float* 
 
 /* The same step on `count` independent matrices (descs is a HOST array),
  * grouped so that each phase of the iteration is one launch over the tiles
- * of all matrices (3 + 3K launches per call). */
+ * of all matrices, each GEMM followed by a small bounds kernel (2 + 6K launches per call). */
 fs4_status fs4_root_ns_batched(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
                                uint32_t flags, void* workspace, size_t workspace_bytes,
                                void* stream);

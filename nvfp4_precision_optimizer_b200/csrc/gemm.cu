@@ -15,8 +15,8 @@
 //   warp 1     allocates 512 TMEM columns; one thread copies the scale atoms to
 //              TMEM (tcgen05.cp) and issues tcgen05.mma kind::mxf4nvf4
 //              (M=128, N=256, K=64, UE4M3 per-16 scales), FP32 accumulator in TMEM
-//   warp 2     tile counter: counts finished tiles per matrix and, in the CTA that
-//              finishes a matrix, derives the next phase's tensor scale
+//   (a one-CTA-per-matrix kernel after each launch turns the row/column sums
+//    into the next phase's tensor scale)
 //   warps 4-11 epilogue: tcgen05.ld of the 128 x 256 accumulator into registers
 //              (the accumulator is handed back to the MMA warp at once, so the
 //              next tile's MMAs overlap this epilogue), the fused element-wise
@@ -215,49 +215,60 @@ __device__ __forceinline__ float warp_drain_max4(float* vec, int64_t len, int la
   return m;
 }
 
-// Count one finished tile of matrix mi; in the CTA that completes the matrix's
-// tiles of this launch, derive the next tensor scale from the row/column sums.
+// After a Newton-Schulz GEMM launch: turn each matrix's row / column sums into the
+// bound that fixes the next tensor scale, and clear the sums for their next use (one
+// CTA per matrix; the launch boundary orders the GEMM's sum atomics before the reads).
+//   GramX:  u_rowA = max_i sum_j deq(qA)^2;  s_B from |b| u_rowX + |c| u_rowA
+//   GramA:  u_rowB = max_i sum_j deq(qB)^2;  s_X' from |a| amax(X) + sqrt(u_rowB u_colX)
+//   Update: u_rowX', u_colX' of the two views of X';  s_A' from u_rowX'
 template <Epi E>
-__device__ __forceinline__ void finalize_tile(const NsParams& p, int mi, int lane) {
-  if constexpr (E != Epi::Plain) {
-    const MatDesc& d = p.mat[mi];
-    NsState* st = reinterpret_cast<NsState*>(p.ws + d.state_off);
-    constexpr int kind = (E == Epi::GramX) ? 1 : (E == Epi::GramA ? 2 : 3);
-    int last = 0;
-    if (lane == 0) {
-      const uint32_t tiles = (uint32_t)(p.prefix[mi + 1] - p.prefix[mi]);
-      last = (atomicAdd(&st->done[kind], 1u) == tiles - 1u) ? 1 : 0;
+__global__ void __launch_bounds__(256) ns_bounds_kernel(const __grid_constant__ NsParams p) {
+  __shared__ float red[8];
+  const MatDesc& d = p.mat[blockIdx.x];
+  NsState* st = reinterpret_cast<NsState*>(p.ws + d.state_off);
+  const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
+  const int k = p.iter;
+  auto drain = [&](int64_t off, int64_t len) -> float {
+    float m = 0.0f;
+    float4* v4 = reinterpret_cast<float4*>(p.ws + off);
+    for (int64_t i = threadIdx.x; i < (len >> 2); i += 256) {
+      const float4 a = __ldcg(v4 + i);
+      __stcg(v4 + i, make_float4(0.f, 0.f, 0.f, 0.f));
+      m = fmaxf(m, fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w)));
     }
-    last = __shfl_sync(0xFFFFFFFFu, last, 0);
-    if (!last) return;
-    __threadfence();
-    const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
-    const int k = p.iter;
-    if constexpr (E == Epi::GramX) {
-      const float ua = warp_drain_max4(reinterpret_cast<float*>(p.ws + L.rowsumA), d.mp, lane);
-      if (lane == 0) {
-        st->u_rowA[k] = ua;
-        const float ub = (fabsf(d.b) * __ldcg(&st->u_rowX[k]) + fabsf(d.c) * ua) * kBoundInflate;
-        st->sg[kSgB + k] = pow2_tensor_scale(ub);
-      }
-    } else if constexpr (E == Epi::GramA) {
-      const float ub = warp_drain_max4(reinterpret_cast<float*>(p.ws + L.rowsumB), d.mp, lane);
-      if (lane == 0) {
-        st->u_rowB[k] = ub;
-        const float ax = __uint_as_float(__ldcg(&st->amaxX[k]));
-        const float ux = (fabsf(d.a) * ax + sqrtf(ub * __ldcg(&st->u_colX[k]))) * kBoundInflate;
-        st->sg[kSgX + k + 1] = pow2_tensor_scale(ux);
-      }
-    } else {
-      const float ur = warp_drain_max4(reinterpret_cast<float*>(p.ws + L.rowsumX), d.mp, lane);
-      const float uc = warp_drain_max4(reinterpret_cast<float*>(p.ws + L.colsumX), d.np, lane);
-      if (lane == 0 && !p.last) {
-        st->u_rowX[k + 1] = ur;
-        st->u_colX[k + 1] = uc;
-        st->sg[kSgA + k + 1] = pow2_tensor_scale(ur * kBoundInflate);
-      }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    float r = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) r = fmaxf(r, red[w]);
+    return r;
+  };
+  if constexpr (E == Epi::GramX) {
+    const float ua = drain(L.rowsumA, d.mp);
+    if (threadIdx.x == 0) {
+      st->u_rowA[k] = ua;
+      const float ub = (fabsf(d.b) * st->u_rowX[k] + fabsf(d.c) * ua) * kBoundInflate;
+      st->sg[kSgB + k] = pow2_tensor_scale(ub);
     }
-    if (lane == 0) st->done[kind] = 0u;
+  } else if constexpr (E == Epi::GramA) {
+    const float ub = drain(L.rowsumB, d.mp);
+    if (threadIdx.x == 0) {
+      st->u_rowB[k] = ub;
+      const float ax = __uint_as_float(st->amaxX[k]);
+      const float ux = (fabsf(d.a) * ax + sqrtf(ub * st->u_colX[k])) * kBoundInflate;
+      st->sg[kSgX + k + 1] = pow2_tensor_scale(ux);
+    }
+  } else {
+    const float ur = drain(L.rowsumX, d.mp);
+    const float uc = drain(L.colsumX, d.np);
+    if (threadIdx.x == 0 && !p.last) {
+      st->u_rowX[k + 1] = ur;
+      st->u_colX[k + 1] = uc;
+      st->sg[kSgA + k + 1] = pow2_tensor_scale(ur * kBoundInflate);
+    }
   }
 }
 
@@ -345,7 +356,7 @@ __device__ __forceinline__ void stage_flush(const float* buf, TileRows t, int c,
 template <Epi E>
 __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainArgs& g,
                                             uint32_t tmem, uint64_t* acc_full,
-                                            uint64_t* acc_empty, uint32_t* arrivals,
+                                            uint64_t* acc_empty,
                                             uint32_t* status, volatile int* abort_flag,
                                             float* wbuf, const float2* scale_tab, int quad, int ch,
                                             int lane, int32_t total) {
@@ -578,10 +589,6 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
       for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
       if (lane == 0 && !p.last && amax > 0.0f) atomicMax(&st->amaxX[k + 1], __float_as_uint(amax));
     }
-    // publish this warp's sums for the counter warp (never waits)
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) atomicAdd(arrivals, 1u);
     if constexpr (kIn) fp = fn;
   }
   if constexpr (kIn) cp_async_wait<0>();
@@ -647,7 +654,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* mma_done = acc_full + 2;
   uint64_t* stall_bar = acc_full + 3;        // test only: never arrived on
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 4);
-  uint32_t* arrivals = tmem_slot + 1;   // monotonic count of (epilogue warp, tile) completions
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   float2* scale_tab = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(bars) + C::BAR_BYTES);
   if (threadIdx.x >= 128 && threadIdx.x < 256) scale_tab[threadIdx.x - 128] = scale_tab_entry(threadIdx.x - 128);
@@ -665,7 +671,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(acc_empty, 8);
     mbar_init(mma_done, 1);
     mbar_init(stall_bar, 1);
-    *arrivals = 0u;
     *abort_flag = (__ldcg(status) & kStatusTimeout) ? 1 : 0;
     fence_mbar_init();
   }
@@ -753,33 +758,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       volatile int never = 0;
       mbar_wait(mma_done, 0, status, &never);
     }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ tile counter / finalizer
-    // Trails the epilogue warps: once all eight have published tile tl's sums, count
-    // the tile for its matrix; the CTA that finishes a matrix's last tile in this
-    // launch turns the matrix's sums into the next tensor scale.  The epilogue warps
-    // never wait for this warp.
-    if constexpr (E != Epi::Plain) {
-      uint32_t tl = 0;
-      for (int32_t u = first; u < total; u += step, ++tl) {
-        const Job j = make_job<E>(u, p, g);
-        const uint32_t target = 8u * (tl + 1u);
-        bool seen = true;
-        if (*reinterpret_cast<volatile uint32_t*>(arrivals) < target) {
-          const uint64_t t0 = global_timer_ns();
-          while (*reinterpret_cast<volatile uint32_t*>(arrivals) < target) {
-            if (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs) { seen = false; break; }
-            __nanosleep(500);
-          }
-        }
-        if (!seen) {
-          if (lane == 0 && !*abort_flag) { atomicOr(status, kStatusTimeout); *abort_flag = 1; }
-          break;
-        }
-        __threadfence();
-        finalize_tile<E>(p, j.mat, lane);
-      }
-    }
   }
   } else {
     regs_inc<kRegsEpi>();
@@ -794,7 +772,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (E == Epi::Plain)
       epilogue_plain(p, g, tmem, acc_full, acc_empty, status, abort_flag, wbuf, quad, ch, lane, total);
     else
-      epilogue_ns<E>(p, g, tmem, acc_full, acc_empty, arrivals, status, abort_flag, wbuf, scale_tab,
+      epilogue_ns<E>(p, g, tmem, acc_full, acc_empty, status, abort_flag, wbuf, scale_tab,
                      quad, ch, lane, total);
   }
 
@@ -842,12 +820,23 @@ cudaError_t launch_gemm_plain(const GemmPlainArgs& a, cudaStream_t st, int num_s
 
 cudaError_t launch_gemm_ns(Epi epi, const NsParams& p, cudaStream_t st, int num_sms) {
   const int64_t units = p.prefix[p.count];
+  cudaError_t e;
   switch (epi) {
-    case Epi::GramX: return launch_impl<Epi::GramX>(&p, nullptr, units, st, num_sms);
-    case Epi::GramA: return launch_impl<Epi::GramA>(&p, nullptr, units, st, num_sms);
-    case Epi::Update: return launch_impl<Epi::Update>(&p, nullptr, units, st, num_sms);
+    case Epi::GramX:
+      if ((e = launch_impl<Epi::GramX>(&p, nullptr, units, st, num_sms)) != cudaSuccess) return e;
+      ns_bounds_kernel<Epi::GramX><<<p.count, 256, 0, st>>>(p);
+      break;
+    case Epi::GramA:
+      if ((e = launch_impl<Epi::GramA>(&p, nullptr, units, st, num_sms)) != cudaSuccess) return e;
+      ns_bounds_kernel<Epi::GramA><<<p.count, 256, 0, st>>>(p);
+      break;
+    case Epi::Update:
+      if ((e = launch_impl<Epi::Update>(&p, nullptr, units, st, num_sms)) != cudaSuccess) return e;
+      if (!p.last) ns_bounds_kernel<Epi::Update><<<p.count, 256, 0, st>>>(p);
+      break;
     default: return cudaErrorInvalidValue;
   }
+  return cudaGetLastError();
 }
 
 }  // namespace fs4
