@@ -108,13 +108,48 @@ def global_scale(amax: float, mode: str = "pow2") -> np.float32:
     return np.float32(math.ldexp(1.0, e))
 
 
-def quantize_rows(x: np.ndarray, s_g: float | None = None, mode: str = "pow2"):
+def _quantize_blocks(blocks: np.ndarray, s_g: np.float32, M: float):
+    """Codes (4-bit, sign included), E4M3 scale bytes and FP32 dequantised values of
+    (rows, nb, 16) FP32 blocks with block scale RN_e4m3(amax / fp32(M * s_g))."""
+    amax_b = np.max(np.abs(blocks), axis=2)                      # exact
+    v = amax_b / (np.float32(M) * s_g)                           # FP32 division
+    scales = e4m3_encode(v)
+    den = E4M3_VALUES[scales].astype(np.float32) * s_g           # FP32 product
+    safe = np.where(den > 0, den, np.float32(1.0)).astype(np.float32)
+    q = np.abs(blocks) / safe[:, :, None]                        # FP32 division
+    mag = e2m1_encode_magnitude(q)
+    sign = np.signbit(blocks).astype(np.uint8) << 3
+    nib = np.where((den > 0)[:, :, None], mag | sign, 0).astype(np.uint8)
+    deq = (code_values(nib) * den[:, :, None]).astype(np.float32)   # exact in FP32
+    return nib, scales, deq
+
+
+def _block_sq_error_f32(blocks: np.ndarray, deq: np.ndarray) -> np.ndarray:
+    """sum_i (x_i - deq_i)^2 of each block, in FP32 with one rounding per operation,
+    summed in element order 0..15 (the order fixes the result bit for bit)."""
+    err = np.zeros(blocks.shape[:2], dtype=np.float32)
+    for i in range(BLOCK):
+        d = (blocks[:, :, i] - deq[:, :, i]).astype(np.float32)
+        err = (err + (d * d).astype(np.float32)).astype(np.float32)
+    return err
+
+
+def quantize_rows(x: np.ndarray, s_g: float | None = None, mode: str = "pow2",
+                  adaptive46: bool = False):
     """Q_1x16: quantise an FP32 matrix in blocks of 16 consecutive elements of a row.
 
     Returns (codes, scales, s_g): codes uint8 [rows, cols/2] (two elements per
     byte, low nibble first), scales uint8 [rows, cols/16] (E4M3 bytes), s_g
     float32.  ``s_g`` may be given (the value another implementation used);
     otherwise it is derived from the exact amax of ``x``.
+
+    adaptive46: the adaptive 4/6 block scaling named in Section 3.4 ("All
+    quantizations use RTN and adaptive 4/6 scaling"; Four Over Six, Section 2
+    "Others"): each block is quantised with its largest magnitude mapped to
+    M = 6 (the plain rule) and to M = 4, and keeps M = 4 only when that
+    candidate's squared error is strictly smaller (ties keep M = 6).  Reading:
+    the same tensor scale s_g serves both candidates; the error is the FP32
+    sum of _block_sq_error_f32.
     """
     x = np.asarray(x)
     if x.dtype != np.float32:
@@ -129,24 +164,75 @@ def quantize_rows(x: np.ndarray, s_g: float | None = None, mode: str = "pow2"):
         s_g = global_scale(amax, mode)
     s_g = np.float32(s_g)
     blocks = x.reshape(rows, cols // BLOCK, BLOCK)
-    amax_b = np.max(np.abs(blocks), axis=2)                      # exact
-    v = amax_b / (np.float32(6.0) * s_g)                         # FP32 division
-    scales = e4m3_encode(v)
-    den = E4M3_VALUES[scales].astype(np.float32) * s_g           # FP32 product
-    safe = np.where(den > 0, den, np.float32(1.0)).astype(np.float32)
-    q = np.abs(blocks) / safe[:, :, None]                        # FP32 division
-    mag = e2m1_encode_magnitude(q)
-    sign = np.signbit(blocks).astype(np.uint8) << 3
-    nib = np.where((den > 0)[:, :, None], mag | sign, 0).astype(np.uint8)
+    nib, scales, deq6 = _quantize_blocks(blocks, s_g, 6.0)
+    if adaptive46:
+        nib4, scales4, deq4 = _quantize_blocks(blocks, s_g, 4.0)
+        use4 = _block_sq_error_f32(blocks, deq4) < _block_sq_error_f32(blocks, deq6)
+        nib = np.where(use4[:, :, None], nib4, nib)
+        scales = np.where(use4, scales4, scales).astype(np.uint8)
     nib = nib.reshape(rows, cols)
     codes = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
     return codes, scales, s_g
 
 
-def quantize_cols(x: np.ndarray, s_g: float | None = None, mode: str = "pow2"):
+def quantize_cols(x: np.ndarray, s_g: float | None = None, mode: str = "pow2",
+                  adaptive46: bool = False):
     """Q_16x1: blocks of 16 consecutive elements of a column.  The result is
     laid out as the 1x16 quantisation of x^T (a cols x rows matrix)."""
-    return quantize_rows(np.ascontiguousarray(np.asarray(x).T), s_g, mode)
+    return quantize_rows(np.ascontiguousarray(np.asarray(x).T), s_g, mode, adaptive46)
+
+
+# ---------------------------------------------------------------- random Hadamard transform
+# Section 3.4 applies H16^r, "a fresh 16x16 random Hadamard transform", along the
+# K dimension of every quantised operand: qX = Q1x16(X H), qX16x1 = Q16x1(H^T X), so
+# that each product of two quantised operands carries H H^T = I.  Readings:
+#   * H16^r = D H16 / 4, with H16 the Sylvester Hadamard matrix (H16[i, j] =
+#     (-1)^popcount(i & j)) and D = diag of 16 random signs, given as a 16-bit mask
+#     (bit i set: element i of every block is negated before the transform).
+#   * One mask per product, shared by both of its operands and by every block.
+#   * In FP32 the transform is the in-place butterfly with strides 1, 2, 4, 8
+#     ((u, v) -> (u + v, u - v), one rounding per addition), then the exact * 0.25.
+
+def sylvester16() -> np.ndarray:
+    """H16 with entries (-1)^popcount(i & j) (float64)."""
+    i = np.arange(BLOCK)
+    pc = np.vectorize(lambda t: bin(int(t)).count("1"))(i[:, None] & i[None, :])
+    return np.where(pc % 2 == 0, 1.0, -1.0)
+
+
+def mask_signs(mask: int) -> np.ndarray:
+    """The 16 signs (+-1.0) of D for a sign mask."""
+    return np.array([-1.0 if (mask >> i) & 1 else 1.0 for i in range(BLOCK)])
+
+
+def hadamard_rows(x: np.ndarray, mask: int) -> np.ndarray:
+    """FP32 x H16^r on every 16-element block of each row (the butterfly reading)."""
+    x = np.asarray(x, dtype=np.float32)
+    rows, cols = x.shape
+    y = (x.reshape(rows, cols // BLOCK, BLOCK) * mask_signs(mask).astype(np.float32)).astype(np.float32)
+    y = y.copy()
+    h = 1
+    while h < BLOCK:
+        for i in range(0, BLOCK, 2 * h):
+            for j in range(i, i + h):
+                u, v = y[:, :, j].copy(), y[:, :, j + h].copy()
+                y[:, :, j] = (u + v).astype(np.float32)
+                y[:, :, j + h] = (u - v).astype(np.float32)
+        h *= 2
+    return (y * np.float32(0.25)).astype(np.float32).reshape(rows, cols)
+
+
+def hadamard_cols(x: np.ndarray, mask: int) -> np.ndarray:
+    """FP32 (H16^r)^T x on every 16-element block of each column."""
+    return np.ascontiguousarray(hadamard_rows(np.ascontiguousarray(np.asarray(x).T), mask).T)
+
+
+def hadamard_rows_f64(x: np.ndarray, mask: int) -> np.ndarray:
+    """x H16^r in float64 from the matrix definition (reference for the butterfly)."""
+    x = np.asarray(x, dtype=np.float64)
+    rows, cols = x.shape
+    Hr = np.diag(mask_signs(mask)) @ sylvester16() / 4.0
+    return (x.reshape(rows, cols // BLOCK, BLOCK) @ Hr).reshape(rows, cols)
 
 
 def unpack_codes(codes: np.ndarray) -> np.ndarray:

@@ -8,9 +8,10 @@ Source: "Full-Stack FP4" (arXiv 2607.04422).
     + c X_k (X_k^T X_k)^2, typically 5 iterations.  Written in the Gram-left
     form used by Section 3.4, X (X^T X) = (X X^T) X, the Gram matrix is m x m
     on the short side when X is m x n with m <= n.
-  * Section 3.4 "NVFP4 Root Optimizer", the iteration (with the random
-    Hadamard transform taken as the identity, as the method is specified for
-    this build):
+  * Section 3.4 "NVFP4 Root Optimizer", the iteration (by default with the
+    random Hadamard transform taken as the identity and plain M = 6 block
+    scaling; rht_masks / adaptive46 select the transform and the adaptive 4/6
+    scaling the section also names):
         qX_k  = Q1x16(X_k),            A_k = qX_k qX_k^T
         qA_k  = Q1x16(A_k),  qA16_k = Q16x1(A_k),  B_k = b A_k + c qA_k qA16_k
         qB_k  = Q1x16(B_k),  qX16_k = Q16x1(X_k),  X_{k+1} = a X_k + qB_k qX16_k
@@ -56,24 +57,34 @@ def symmetric_from_upper(A: np.ndarray) -> np.ndarray:
     return np.triu(A) + np.triu(A, 1).T
 
 
-def ns_iterations_nvfp4(X0, K, a, b, c, mode="pow2", trace=None):
-    """K NVFP4 Newton-Schulz iterations (Section 3.4) from the FP32 m x n X0 (m <= n)."""
+def ns_iterations_nvfp4(X0, K, a, b, c, mode="pow2", trace=None, rht_masks=None,
+                        adaptive46=False):
+    """K NVFP4 Newton-Schulz iterations (Section 3.4) from the FP32 m x n X0 (m <= n).
+
+    rht_masks: None (H = I) or 3K sign masks of H16^r (see nvfp4.hadamard_rows), one
+    per product: 3k for A_k = qX_k qX_k^T, 3k + 1 for qA_k qA16_k, 3k + 2 for
+    qB_k qX16_k.  adaptive46: adaptive 4/6 block scaling in every quantisation.
+    """
     X = np.asarray(X0, dtype=np.float32)
+    hr = (lambda t, j: t) if rht_masks is None else (lambda t, j: nvfp4.hadamard_rows(t, rht_masks[j]))
+    hc = (lambda t, j: t) if rht_masks is None else (lambda t, j: nvfp4.hadamard_cols(t, rht_masks[j]))
+    a46 = adaptive46
     for k in range(K):
-        # qX_k = Q1x16(X_k); qX16_k = Q16x1(X_k) (held as the 1x16 quantisation of X_k^T)
-        qx, sx, gx = nvfp4.quantize_rows(X, mode=mode)
-        qxt, sxt, gxt = nvfp4.quantize_cols(X, mode=mode)
+        # qX_k = Q1x16(X_k H); qX16_k = Q16x1(H'^T X_k) (held as the 1x16 quantisation of
+        # its transpose); H belongs to the Gram product, H' to the update product
+        qx, sx, gx = nvfp4.quantize_rows(hr(X, 3 * k), mode=mode, adaptive46=a46)
+        qxt, sxt, gxt = nvfp4.quantize_cols(hc(X, 3 * k + 2), mode=mode, adaptive46=a46)
         dX = nvfp4.dequantize_rows(qx, sx, gx)                     # m x n
         dX16 = nvfp4.dequantize_cols(qxt, sxt, gxt)                # m x n, 16x1 blocks
         # A_k = qX_k qX_k^T
         A = symmetric_from_upper(dX @ dX.T).astype(np.float32)
-        # qA_k = Q1x16(A_k), qA16_k = Q16x1(A_k), B_k = b A_k + c qA_k qA16_k
-        qa, sa, ga = nvfp4.quantize_rows(A, mode=mode)
-        qa16, sa16, ga16 = nvfp4.quantize_cols(A, mode=mode)
+        # qA_k = Q1x16(A_k H), qA16_k = Q16x1(H^T A_k), B_k = b A_k + c qA_k qA16_k
+        qa, sa, ga = nvfp4.quantize_rows(hr(A, 3 * k + 1), mode=mode, adaptive46=a46)
+        qa16, sa16, ga16 = nvfp4.quantize_cols(hc(A, 3 * k + 1), mode=mode, adaptive46=a46)
         P = nvfp4.dequantize_rows(qa, sa, ga) @ nvfp4.dequantize_cols(qa16, sa16, ga16)
         B = (b * A.astype(np.float64) + c * P).astype(np.float32)
-        # qB_k = Q1x16(B_k), X_{k+1} = a X_k + qB_k qX16_k
-        qb, sb, gb = nvfp4.quantize_rows(B, mode=mode)
+        # qB_k = Q1x16(B_k H'), X_{k+1} = a X_k + qB_k qX16_k
+        qb, sb, gb = nvfp4.quantize_rows(hr(B, 3 * k + 2), mode=mode, adaptive46=a46)
         Xn = (a * X.astype(np.float64) + nvfp4.dequantize_rows(qb, sb, gb) @ dX16).astype(np.float32)
         if trace is not None:
             trace.append(dict(X=X, qX=(qx, sx, gx), qXT=(qxt, sxt, gxt), A=A,
@@ -92,7 +103,7 @@ def ns_iterations_f64(X0, K, a, b, c):
 
 
 def root_ns(G, K=5, a=3.4445, b=-4.7750, c=2.0315, clip_k=3.0, eps=NS_EPS,
-            quantized=True, mode="pow2", trace=None):
+            quantized=True, mode="pow2", trace=None, rht_masks=None, adaptive46=False):
     """Normalise, clip and run K Newton-Schulz iterations on the FP32 matrix G.
 
     quantized=True: the NVFP4 route of Section 3.4 (FP32 result).
@@ -110,7 +121,8 @@ def root_ns(G, K=5, a=3.4445, b=-4.7750, c=2.0315, clip_k=3.0, eps=NS_EPS,
         X0, inv, tau, norm = normalise_and_clip(X.astype(np.float32), clip_k, eps)
         if trace is not None:
             trace.append(dict(X0=X0, inv=inv, tau=tau, norm=norm))
-        Y = ns_iterations_nvfp4(X0, K, a, b, c, mode=mode, trace=trace)
+        Y = ns_iterations_nvfp4(X0, K, a, b, c, mode=mode, trace=trace, rht_masks=rht_masks,
+                                adaptive46=adaptive46)
     else:
         X64 = np.asarray(X, dtype=np.float64)
         norm = float(np.sqrt(np.sum(X64 ** 2)))
