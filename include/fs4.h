@@ -87,6 +87,22 @@ enum {
  * as (phase + 1); 0 means run everything. */
 #define FS4_STOP_AFTER(phase) ((uint32_t)(((phase) + 1) & 0xFF) << 8)
 
+/* Quantiser options of the Newton-Schulz step (Section 3.4: "qX_k =
+ * Q1x16(X H16^r)" ... "All quantizations use RTN and adaptive 4/6 scaling").
+ * Off by default: the default step quantises plainly (H = I, M = 6).
+ * FS4_NS_ADAPTIVE46: every block is quantised with its amax mapped to 6 and to
+ *   4 and keeps the M = 4 candidate only if its squared error (FP32, summed in
+ *   element order) is strictly smaller; the tensor scale is shared.
+ * FS4_NS_RHT: every quantised operand is transformed along its K dimension by
+ *   H16^r = D H16 / 4 (H16 the Sylvester Hadamard matrix, D the diagonal of
+ *   signs of a 16-bit mask, bit i negating element i of each 16-element block;
+ *   FP32 butterfly with strides 1, 2, 4, 8, then * 0.25) before quantisation.
+ *   Both operands of a product carry the same mask, so the products are those
+ *   of the untransformed tensors.  Tensor scales then cover 4x the amax bound
+ *   (|x H| <= 4 amax).  Only fs4_root_ns_batched_ex takes the masks. */
+#define FS4_NS_ADAPTIVE46 (1u << 3)
+#define FS4_NS_RHT (1u << 2)
+
 /* Test-only flag for fs4_root_ns / fs4_root_ns_batched (no counterpart in the
  * paper): the MMA issuer of the first Gram product waits on a barrier that
  * nothing arrives on.  The bounded wait gives up after about 2 s, records the
@@ -191,6 +207,17 @@ fs4_status fs4_root_ns(const float* G, int64_t m, int64_t n, int64_t ld, float* 
 fs4_status fs4_root_ns_batched(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
                                uint32_t flags, void* workspace, size_t workspace_bytes,
                                void* stream);
+
+/* fs4_root_ns_batched with the quantiser options above.  rht_masks: HOST
+ * array of 3K sign masks when flags has FS4_NS_RHT (else ignored, may be
+ * NULL): entry 3k + j is the mask of product j of iteration k (j = 0:
+ * A = qX qX^T; 1: qA qA^T; 2: qB qX16x1), shared by both of its operands and
+ * drawn fresh by the caller (Section 3.4: "a fresh 16x16 random Hadamard
+ * transform").  Errors as fs4_root_ns_batched; FS4_ERR_INVALID_ARG also for
+ * FS4_NS_RHT without masks. */
+fs4_status fs4_root_ns_batched_ex(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
+                                  uint32_t flags, const uint16_t* rht_masks, void* workspace,
+                                  size_t workspace_bytes, void* stream);
 
 /* fs4_root_ns_batched, with CUDA events recorded on `stream` around each
  * phase so a caller can time the kernels on the launching stream.

@@ -13,8 +13,8 @@ from typing import Sequence
 import torch
 
 from . import _lib
-from ._lib import (FS4_AXIS_COL, FS4_AXIS_ROW, FS4_LAYOUT_TILED, FS4_SG_AMAX, FS4_TEST_STALL,
-                   Fs4Error, NsDesc, NsLayout, check, stop_after)
+from ._lib import (FS4_AXIS_COL, FS4_AXIS_ROW, FS4_LAYOUT_TILED, FS4_NS_ADAPTIVE46, FS4_NS_RHT,
+                   FS4_SG_AMAX, FS4_TEST_STALL, Fs4Error, NsDesc, NsLayout, check, stop_after)
 
 MUON_COEFFS = (3.4445, -4.7750, 2.0315)
 
@@ -22,6 +22,7 @@ __all__ = [
     "quantize", "dequantize", "gemm", "root_ns", "root_ns_batched", "ns_workspace_size",
     "ns_batched_workspace_size", "ns_layout", "device_status", "tiled_shape", "Fs4Error",
     "MUON_COEFFS", "stop_after", "FS4_AXIS_ROW", "FS4_AXIS_COL", "FS4_TEST_STALL",
+    "FS4_NS_RHT", "FS4_NS_ADAPTIVE46",
 ]
 
 
@@ -132,28 +133,47 @@ def ns_batched_workspace_size(shapes: Sequence[tuple[int, int]]) -> int:
     return int(_lib.lib().fs4_root_ns_batched_workspace_size(len(shapes), _shape_descs(shapes)))
 
 
+def _masks(rht_masks, K):
+    """Host uint16 array of the 3K H16^r sign masks (or None)."""
+    if rht_masks is None:
+        return None
+    masks = [int(v) & 0xFFFF for v in rht_masks]
+    if len(masks) < 3 * K:
+        raise ValueError(f"need 3K = {3 * K} sign masks, got {len(masks)}")
+    return (ctypes.c_uint16 * len(masks))(*masks)
+
+
 def root_ns(G: torch.Tensor, K: int = 5, a: float = MUON_COEFFS[0], b: float = MUON_COEFFS[1],
             c: float = MUON_COEFFS[2], clip_k: float = 3.0, out: torch.Tensor | None = None,
-            workspace: torch.Tensor | None = None, flags: int = 0, stream=None) -> torch.Tensor:
-    """Direct NVFP4 Newton-Schulz step on one FP32 matrix (fs4_root_ns)."""
+            workspace: torch.Tensor | None = None, flags: int = 0, stream=None,
+            rht_masks=None, adaptive46: bool = False) -> torch.Tensor:
+    """Direct NVFP4 Newton-Schulz step on one FP32 matrix (fs4_root_ns; with
+    rht_masks (3K sign masks of H16^r) or adaptive46, fs4_root_ns_batched_ex)."""
     _check_f32_matrix(G, "G")
     if out is None:
         out = torch.empty_like(G)
     m, n = G.shape
     if workspace is None:
         workspace = torch.empty(ns_workspace_size(m, n), dtype=torch.uint8, device=G.device)
-    check(_lib.lib().fs4_root_ns(G.data_ptr(), m, n, _ld(G), out.data_ptr(), _ld(out), K,
-                                 a, b, c, clip_k, flags, workspace.data_ptr(), workspace.numel(),
-                                 _stream(stream)),
-          "fs4_root_ns")
+    if rht_masks is None and not adaptive46:
+        check(_lib.lib().fs4_root_ns(G.data_ptr(), m, n, _ld(G), out.data_ptr(), _ld(out), K,
+                                     a, b, c, clip_k, flags, workspace.data_ptr(), workspace.numel(),
+                                     _stream(stream)),
+              "fs4_root_ns")
+        return out
+    root_ns_batched([G], K, [(a, b, c)], clip_k, [out], workspace, flags, stream, rht_masks,
+                    adaptive46)
     return out
 
 
 def root_ns_batched(Gs: Sequence[torch.Tensor], K: int = 5, coeffs=None, clip_k: float = 3.0,
                     outs: Sequence[torch.Tensor] | None = None,
-                    workspace: torch.Tensor | None = None, flags: int = 0, stream=None):
+                    workspace: torch.Tensor | None = None, flags: int = 0, stream=None,
+                    rht_masks=None, adaptive46: bool = False):
     """Direct NVFP4 Newton-Schulz step on a list of matrices in one grouped call
-    (fs4_root_ns_batched); coeffs is a list of per-matrix (a, b, c)."""
+    (fs4_root_ns_batched); coeffs is a list of per-matrix (a, b, c).  rht_masks
+    (3K sign masks of H16^r) and adaptive46 select the Section 3.4 quantiser
+    options (fs4_root_ns_batched_ex)."""
     for G in Gs:
         _check_f32_matrix(G, "G")
     if coeffs is None:
@@ -164,9 +184,18 @@ def root_ns_batched(Gs: Sequence[torch.Tensor], K: int = 5, coeffs=None, clip_k:
     need = int(_lib.lib().fs4_root_ns_batched_workspace_size(len(Gs), arr))
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=Gs[0].device)
-    check(_lib.lib().fs4_root_ns_batched(len(Gs), arr, K, clip_k, flags, workspace.data_ptr(),
-                                         workspace.numel(), _stream(stream)),
-          "fs4_root_ns_batched")
+    if rht_masks is None and not adaptive46:
+        check(_lib.lib().fs4_root_ns_batched(len(Gs), arr, K, clip_k, flags, workspace.data_ptr(),
+                                             workspace.numel(), _stream(stream)),
+              "fs4_root_ns_batched")
+        return outs
+    flags |= (FS4_NS_RHT if rht_masks is not None else 0) | (FS4_NS_ADAPTIVE46 if adaptive46 else 0)
+    masks = _masks(rht_masks, K)
+    check(_lib.lib().fs4_root_ns_batched_ex(len(Gs), arr, K, clip_k, flags,
+                                            ctypes.cast(masks, ctypes.c_void_p) if masks else None,
+                                            workspace.data_ptr(), workspace.numel(),
+                                            _stream(stream)),
+          "fs4_root_ns_batched_ex")
     return outs
 
 

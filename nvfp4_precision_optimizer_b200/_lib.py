@@ -23,6 +23,7 @@ STATUS_NAMES = {
 FS4_AXIS_ROW, FS4_AXIS_COL = 0, 1
 FS4_SG_AMAX, FS4_LAYOUT_TILED = 1, 2
 FS4_TEST_STALL = 1 << 30   # test only: a device wait that runs out (see include/fs4.h)
+FS4_NS_RHT, FS4_NS_ADAPTIVE46 = 1 << 2, 1 << 3
 MAX_BATCH = 224
 MAX_ITERS = 32
 
@@ -59,6 +60,8 @@ SIGNATURES = {
                             c_f32, c_u32, c_vp, c_sz, c_vp]),
     "fs4_root_ns_batched": (c_i32, [c_i32, ctypes.POINTER(NsDesc), c_i32, c_f32, c_u32, c_vp,
                                     c_sz, c_vp]),
+    "fs4_root_ns_batched_ex": (c_i32, [c_i32, ctypes.POINTER(NsDesc), c_i32, c_f32, c_u32, c_vp,
+                                       c_vp, c_sz, c_vp]),
     "fs4_root_ns_batched_timed": (c_i32, [c_i32, ctypes.POINTER(NsDesc), c_i32, c_f32, c_u32,
                                           c_vp, c_sz, c_vp, ctypes.POINTER(c_vp), c_i32]),
     "fs4_root_ns_noalloc": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i64, c_i32, c_f32, c_f32,

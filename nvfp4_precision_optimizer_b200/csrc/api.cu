@@ -137,7 +137,8 @@ bool fill_prefix(NsParams& p, const int64_t* units) {
 // Reused parameter block: 19 KB, too large for the stack of every caller thread.
 thread_local NsParams t_params;
 
-fs4_status run_ns(const Plan& pl, int32_t K, float clip_k, uint32_t flags, uint8_t* ws,
+fs4_status run_ns(const Plan& pl, int32_t K, float clip_k, uint32_t flags, const uint16_t* rht_masks,
+                  uint8_t* ws,
                   cudaStream_t st, int num_sms, void* const* events = nullptr) {
   int ev_i = 0;
   auto mark = [&]() -> bool {
@@ -151,6 +152,9 @@ fs4_status run_ns(const Plan& pl, int32_t K, float clip_k, uint32_t flags, uint8
   p.clip_k = clip_k;
   p.status = reinterpret_cast<uint32_t*>(ws);
   p.ws = ws;
+  p.opts = ((flags & FS4_NS_RHT) ? kOptRht : 0u) | ((flags & FS4_NS_ADAPTIVE46) ? kOpt46 : 0u);
+  if (flags & FS4_NS_RHT)
+    for (int i = 0; i < 3 * K; ++i) p.rht[i] = rht_masks[i];
   std::memcpy(p.mat, pl.mat, sizeof(MatDesc) * pl.count);
 
   if (!mark()) return FS4_ERR_CUDA;
@@ -268,11 +272,14 @@ size_t fs4_root_ns_workspace_size(int64_t m, int64_t n) {
 }
 
 static fs4_status batched_impl(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
-                               uint32_t flags, void* workspace, size_t workspace_bytes,
-                               void* stream, void* const* events, int32_t n_events) {
+                               uint32_t flags, const uint16_t* rht_masks, void* workspace,
+                               size_t workspace_bytes, void* stream, void* const* events,
+                               int32_t n_events) {
   if (K < 1 || K > FS4_MAX_ITERS) return FS4_ERR_SHAPE;
   if (!std::isfinite(clip_k)) return FS4_ERR_INVALID_ARG;
-  if (flags & ~(uint32_t)(0xFF00u | FS4_TEST_STALL)) return FS4_ERR_INVALID_ARG;
+  if (flags & ~(uint32_t)(0xFF00u | FS4_TEST_STALL | FS4_NS_RHT | FS4_NS_ADAPTIVE46))
+    return FS4_ERR_INVALID_ARG;
+  if ((flags & FS4_NS_RHT) && !rht_masks) return FS4_ERR_INVALID_ARG;
   static thread_local Plan pl;
   const fs4_status s = make_plan(count, descs, &pl);
   if (s != FS4_OK) return s;
@@ -294,14 +301,22 @@ static fs4_status batched_impl(int32_t count, const fs4_ns_desc* descs, int32_t 
   DeviceInfo di;
   const fs4_status ds = device_info(&di);
   if (ds != FS4_OK) return ds;
-  return run_ns(pl, K, clip_k, flags, static_cast<uint8_t*>(workspace),
+  return run_ns(pl, K, clip_k, flags, rht_masks, static_cast<uint8_t*>(workspace),
                 static_cast<cudaStream_t>(stream), di.num_sms, events);
 }
 
 fs4_status fs4_root_ns_batched(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
                                uint32_t flags, void* workspace, size_t workspace_bytes,
                                void* stream) {
-  return batched_impl(count, descs, K, clip_k, flags, workspace, workspace_bytes, stream, nullptr, 0);
+  return batched_impl(count, descs, K, clip_k, flags, nullptr, workspace, workspace_bytes, stream,
+                      nullptr, 0);
+}
+
+fs4_status fs4_root_ns_batched_ex(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
+                                  uint32_t flags, const uint16_t* rht_masks, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  return batched_impl(count, descs, K, clip_k, flags, rht_masks, workspace, workspace_bytes, stream,
+                      nullptr, 0);
 }
 
 fs4_status fs4_root_ns_batched_timed(int32_t count, const fs4_ns_desc* descs, int32_t K,
@@ -309,7 +324,7 @@ fs4_status fs4_root_ns_batched_timed(int32_t count, const fs4_ns_desc* descs, in
                                      size_t workspace_bytes, void* stream,
                                      void* const* phase_events, int32_t n_events) {
   if (!phase_events) return FS4_ERR_INVALID_ARG;
-  return batched_impl(count, descs, K, clip_k, flags, workspace, workspace_bytes, stream,
+  return batched_impl(count, descs, K, clip_k, flags, nullptr, workspace, workspace_bytes, stream,
                       phase_events, n_events);
 }
 

@@ -102,7 +102,9 @@ __device__ __forceinline__ uint32_t sq4_e2m1_sum8(uint32_t w) {
 // ------------------------------------------------------------------ tensor scale
 // Smallest power of two s_g with 2688 * s_g >= u, exponent clamped to [-116, 118];
 // 1 for u == 0.  Exact: 2688 = 1.3125 * 2^11, so compare u's mantissa with 1.3125.
-__host__ __device__ __forceinline__ float pow2_tensor_scale(float u) {
+// for46 (adaptive 4/6 block scaling): the denominator is 1792 = 4 * 448 = 1.75 * 2^10,
+// so that the M = 4 candidate's block scale cannot saturate either.
+__host__ __device__ __forceinline__ float pow2_tensor_scale(float u, bool for46 = false) {
   if (!(u > 0.0f)) return 1.0f;
   uint32_t bits;
 #ifdef __CUDA_ARCH__
@@ -116,7 +118,8 @@ __host__ __device__ __forceinline__ float pow2_tensor_scale(float u) {
   } else {
     const int eu = (int)(bits >> 23) - 127;
     const uint32_t mant = bits & 0x7FFFFFu;
-    e = (mant <= 0x280000u) ? eu - 11 : eu - 10;
+    if (for46) e = (mant <= 0x600000u) ? eu - 10 : eu - 9;
+    else e = (mant <= 0x280000u) ? eu - 11 : eu - 10;
   }
   e = e < -116 ? -116 : (e > 118 ? 118 : e);
   uint32_t out = (uint32_t)(e + 127) << 23;
@@ -196,10 +199,76 @@ __device__ __forceinline__ uint64_t div2_rn_fma(uint64_t x, uint64_t nd, uint64_
 // kPow2: s_g is a power of two and rcp_six = RN(1 / six_sg), so the block scale
 // division may use the FMA-corrected form; otherwise IEEE division is used.
 // With a table (kPow2 only) the decoded block scale and its reciprocal are looked up.
+// ------------------------------------------------------------------ random Hadamard transform
+// x <- x H16^r on one 16-element block, H16^r = D H16 / 4 ("Full-Stack FP4", Section 3.4):
+// bit i of `mask` negates element i, then the in-place butterfly with strides 1, 2, 4, 8
+// ((u, v) -> (u + v, u - v), FP32 round-to-nearest per addition), then the exact * 0.25.
+__device__ __forceinline__ void rht16(float* x, uint32_t mask) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) x[i] = __uint_as_float(__float_as_uint(x[i]) ^ (((mask >> i) & 1u) << 31));
+#pragma unroll
+  for (int h = 1; h < 16; h *= 2) {
+#pragma unroll
+    for (int i = 0; i < 16; i += 2 * h) {
+#pragma unroll
+      for (int j = i; j < i + h; ++j) {
+        const float u = x[j], v = x[j + h];
+        x[j] = __fadd_rn(u, v);
+        x[j + h] = __fsub_rn(u, v);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) x[i] = __fmul_rn(x[i], 0.25f);
+}
+
+// The 8 E2M1 values (signed) of one packed word as 4 f16x2: element 2i in the low
+// half of h[i] (byte i of w, low nibble first).
+__device__ __forceinline__ void e2m1_decode8(uint32_t w, uint32_t* h) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(w));
+}
+
+// The 16 E2M1 values (signed, as FP32) of a block's packed codes.
+__device__ __forceinline__ void e2m1_decode16(uint32_t w0, uint32_t w1, float* v) {
+  uint32_t h[8];
+  e2m1_decode8(w0, h);
+  e2m1_decode8(w1, h + 4);
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    v[2 * b] = half_lo(h[b]);
+    v[2 * b + 1] = half_hi(h[b]);
+  }
+}
+
+// sum_i (x_i - code_i * den)^2 in FP32, one rounding per operation, in element order.
+__device__ __forceinline__ float block_sq_error(const float* x, uint32_t w0, uint32_t w1, float den) {
+  float v[16];
+  e2m1_decode16(w0, w1, v);
+  float err = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float d = __fsub_rn(x[i], __fmul_rn(v[i], den));
+    err = __fadd_rn(err, __fmul_rn(d, d));
+  }
+  return err;
+}
+
 // kPacked: divide in f32x2 pairs (fewer instructions; the same roundings).
-template <bool kPow2, bool kTab = false, bool kPacked = true>
+// k46: adaptive 4/6 block scaling (Section 3.4): the block is also quantised with
+// its amax mapped to 4 (scale RN_e4m3(amax / (4 s_g)); 4 s_g is a power of two, so
+// that division is exact) and keeps that candidate only when its squared error is
+// strictly smaller.  Requires kPow2.
+template <bool kPow2, bool kTab = false, bool kPacked = true, bool k46 = false>
 __device__ __forceinline__ QBlock16 quantize16(const float* x, float s_g, float six_sg, float rcp_six,
                                                ScaleTab st = ScaleTab{nullptr, 0.0f}) {
+  static_assert(kPow2 || !k46, "adaptive 4/6 needs a power-of-two tensor scale");
   static_assert(kPow2 || !kTab, "the scale table needs a power-of-two tensor scale");
   // max |x| as a tree (depth 4 instead of a 16-long dependency chain)
   float m8[8];
@@ -208,41 +277,56 @@ __device__ __forceinline__ QBlock16 quantize16(const float* x, float s_g, float 
 #pragma unroll
   for (int i = 0; i < 4; ++i) m8[i] = fmaxf(m8[i], m8[i + 4]);
   const float amax = fmaxf(fmaxf(m8[0], m8[2]), fmaxf(m8[1], m8[3]));
-  QBlock16 r;
-  r.amax = amax;
-  r.scale = f32_to_e4m3(kPow2 ? div_rn_fma(amax, six_sg, rcp_six) : __fdiv_rn(amax, six_sg));
-  if (r.scale == 0u) {
-    r.w0 = r.w1 = 0u;
-    r.sumsq = 0.0f;
-    return r;
-  }
-  float den, rcp = 0.0f;
-  if constexpr (kTab) {
-    const float2 t = st.tab[r.scale];
-    den = __fmul_rn(t.x, s_g);
-    rcp = t.y * st.rcp_sg;
-  } else {
-    den = __fmul_rn(e4m3_to_f32(r.scale), s_g);
-    if (kPow2) rcp = __frcp_rn(den);
-  }
-  float q[16];
-  if (kPow2 && kPacked) {
-    const uint64_t nd2 = f2_pack(-den, -den), rcp2 = f2_pack(rcp, rcp);
+  // one candidate: block scale byte from the scaled amax, codes, den = value(scale) * s_g
+  auto candidate = [&](float scaled_amax, QBlock16& r, float& den) {
+    r.amax = amax;
+    r.scale = f32_to_e4m3(scaled_amax);
+    if (r.scale == 0u) {
+      r.w0 = r.w1 = 0u;
+      r.sumsq = 0.0f;
+      den = 0.0f;
+      return;
+    }
+    float rcp = 0.0f;
+    if constexpr (kTab) {
+      const float2 t = st.tab[r.scale];
+      den = __fmul_rn(t.x, s_g);
+      rcp = t.y * st.rcp_sg;
+    } else {
+      den = __fmul_rn(e4m3_to_f32(r.scale), s_g);
+      if (kPow2) rcp = __frcp_rn(den);
+    }
+    float q[16];
+    if (kPow2 && kPacked) {
+      const uint64_t nd2 = f2_pack(-den, -den), rcp2 = f2_pack(rcp, rcp);
 #pragma unroll
-    for (int i = 0; i < 16; i += 2)
-      f2_unpack(div2_rn_fma(f2_pack(x[i], x[i + 1]), nd2, rcp2), q[i], q[i + 1]);
-  } else if (kPow2) {
+      for (int i = 0; i < 16; i += 2)
+        f2_unpack(div2_rn_fma(f2_pack(x[i], x[i + 1]), nd2, rcp2), q[i], q[i + 1]);
+    } else if (kPow2) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) q[i] = div_rn_fma(x[i], den, rcp);
-  } else {
+      for (int i = 0; i < 16; ++i) q[i] = div_rn_fma(x[i], den, rcp);
+    } else {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(x[i], den);
+      for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(x[i], den);
+    }
+    r.w0 = pack8_e2m1(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+    r.w1 = pack8_e2m1(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
+    const float s4 = static_cast<float>(sq4_e2m1_sum8(r.w0) + sq4_e2m1_sum8(r.w1));
+    r.sumsq = 0.25f * s4 * den * den;
+  };
+  QBlock16 r6;
+  float den6;
+  candidate(kPow2 ? div_rn_fma(amax, six_sg, rcp_six) : __fdiv_rn(amax, six_sg), r6, den6);
+  if constexpr (k46) {
+    QBlock16 r4;
+    float den4;
+    // amax / (4 s_g): a division by a power of two, exact as a product
+    candidate(__fmul_rn(amax, __fmul_rn(0.25f, kTab ? st.rcp_sg : __frcp_rn(s_g))), r4, den4);
+    const float e6 = block_sq_error(x, r6.w0, r6.w1, den6);
+    const float e4 = block_sq_error(x, r4.w0, r4.w1, den4);
+    if (e4 < e6) return r4;
   }
-  r.w0 = pack8_e2m1(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
-  r.w1 = pack8_e2m1(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
-  const float s4 = static_cast<float>(sq4_e2m1_sum8(r.w0) + sq4_e2m1_sum8(r.w1));
-  r.sumsq = 0.25f * s4 * den * den;
-  return r;
+  return r6;
 }
 
 // ------------------------------------------------------------------ shared memory / mbarriers

@@ -90,14 +90,18 @@ struct MatDesc {
 };
 
 // Kernel parameters of one Newton-Schulz phase over a batch of matrices.
+constexpr uint32_t kOptRht = 1u, kOpt46 = 2u;   // NsParams::opts
+
 struct NsParams {
   int32_t count;
   int32_t iter;            // k of the current iteration
   int32_t last;            // 1 on the final update product (writes `out`)
   int32_t stall;           // test only: the MMA issuer waits on a barrier nothing arrives on
+  uint32_t opts;           // kOptRht | kOpt46
   float clip_k;
   uint32_t* status;
   uint8_t* ws;             // workspace base
+  uint16_t rht[3 * kMaxIters];   // H16^r sign mask of product j of iteration k at 3k + j
   int32_t prefix[kMaxBatch + 1];   // prefix sums of this phase's work units per matrix
   MatDesc mat[kMaxBatch];
 };

@@ -228,6 +228,9 @@ __global__ void __launch_bounds__(256) ns_bounds_kernel(const __grid_constant__ 
   NsState* st = reinterpret_cast<NsState*>(p.ws + d.state_off);
   const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
   const int k = p.iter;
+  // with the Hadamard transform the quantised tensor is T H: |T H| <= 4 max |T|
+  const float rht4 = (p.opts & kOptRht) ? 4.0f : 1.0f;
+  const bool for46 = (p.opts & kOpt46) != 0;   // tensor scales cover the M = 4 candidate
   auto drain = [&](int64_t off, int64_t len) -> float {
     float m = 0.0f;
     float4* v4 = reinterpret_cast<float4*>(p.ws + off);
@@ -251,7 +254,7 @@ __global__ void __launch_bounds__(256) ns_bounds_kernel(const __grid_constant__ 
     if (threadIdx.x == 0) {
       st->u_rowA[k] = ua;
       const float ub = (fabsf(d.b) * st->u_rowX[k] + fabsf(d.c) * ua) * kBoundInflate;
-      st->sg[kSgB + k] = pow2_tensor_scale(ub);
+      st->sg[kSgB + k] = pow2_tensor_scale(ub * rht4, for46);
     }
   } else if constexpr (E == Epi::GramA) {
     const float ub = drain(L.rowsumB, d.mp);
@@ -259,7 +262,7 @@ __global__ void __launch_bounds__(256) ns_bounds_kernel(const __grid_constant__ 
       st->u_rowB[k] = ub;
       const float ax = __uint_as_float(st->amaxX[k]);
       const float ux = (fabsf(d.a) * ax + sqrtf(ub * st->u_colX[k])) * kBoundInflate;
-      st->sg[kSgX + k + 1] = pow2_tensor_scale(ux);
+      st->sg[kSgX + k + 1] = pow2_tensor_scale(ux * rht4, for46);
     }
   } else {
     const float ur = drain(L.rowsumX, d.mp);
@@ -267,7 +270,7 @@ __global__ void __launch_bounds__(256) ns_bounds_kernel(const __grid_constant__ 
     if (threadIdx.x == 0 && !p.last) {
       st->u_rowX[k + 1] = ur;
       st->u_colX[k + 1] = uc;
-      st->sg[kSgA + k + 1] = pow2_tensor_scale(ur * kBoundInflate);
+      st->sg[kSgA + k + 1] = pow2_tensor_scale(ur * kBoundInflate * rht4, for46);
     }
   }
 }
@@ -353,7 +356,7 @@ __device__ __forceinline__ void stage_flush(const float* buf, TileRows t, int c,
 //   GramX   A = sX^2 acc            -> A (FP32), qA = Q1x16(A); mirrored tile: Q1x16 of A^T
 //   GramA   B = b A + c sA^2 acc    -> qB = Q1x16(B);           mirrored tile: Q1x16 of B^T
 //   Update  X' = a X + sB sX acc    -> X' (FP32), Q1x16(X'), Q16x1(X') (or the output, last)
-template <Epi E>
+template <Epi E, uint32_t kOpts>
 __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainArgs& g,
                                             uint32_t tmem, uint64_t* acc_full,
                                             uint64_t* acc_empty,
@@ -363,6 +366,17 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
   const int32_t first = blockIdx.x, step = gridDim.x;
   constexpr bool kIn = (E == Epi::GramA || E == Epi::Update);   // reads an FP32 tile
   constexpr bool kPackedQ = (E != Epi::Update);   // f32x2 quantiser (measured per kernel)
+  constexpr bool kRht = (kOpts & kOptRht) != 0;    // Hadamard transform before quantising
+  constexpr bool k46 = (kOpts & kOpt46) != 0;      // adaptive 4/6 block scaling
+  // H16^r masks of the tensors this epilogue quantises (Section 3.4): GramX -> qA (product
+  // qA qA^T of iteration k), GramA -> qB (update product of iteration k), Update -> the
+  // next iterate's Gram view and update view (iteration k + 1)
+  const int kk = p.iter;
+  const uint32_t mask_row = E == Epi::GramX ? p.rht[3 * kk + 1]
+                           : E == Epi::GramA ? p.rht[3 * kk + 2]
+                                             : (kk + 1 < kMaxIters ? p.rht[3 * (kk + 1)] : 0u);
+  const uint32_t mask_col = E == Epi::Update ? (kk + 1 < kMaxIters ? p.rht[3 * (kk + 1) + 2] : 0u)
+                                             : mask_row;
   const int k = p.iter;
   const int cc = lane & 15, hh = lane >> 4;
   TileRows fp{nullptr, 0u};   // FP32 tile rows of the current tile
@@ -521,16 +535,23 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
           // 1x16 view along this lane's row and, where needed, the 16x1 view of column
           // gcc + cc, rows gr0 + 16 hh ..: two independent quantiser chains side by side
           QBlock16 q, qc;
+          float yamax = 0.0f;   // max |X'| of the untransformed block (update bound)
+          if constexpr (kRht && E == Epi::Update) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) yamax = fmaxf(yamax, fabsf(y[e]));
+          }
+          if constexpr (kRht) rht16(y, mask_row);
           if (need_col) {
             float xc[16];
             stage_load_col(buf, cc, hh, xc);
-            q = quantize16<true, true, kPackedQ>(y, sg_out, six_out, rcp_six, stab);
-            qc = quantize16<true, true, kPackedQ>(xc, sg_out, six_out, rcp_six, stab);
+            if constexpr (kRht) rht16(xc, mask_col);
+            q = quantize16<true, true, kPackedQ, k46>(y, sg_out, six_out, rcp_six, stab);
+            qc = quantize16<true, true, kPackedQ, k46>(xc, sg_out, six_out, rcp_six, stab);
           } else {
-            q = quantize16<true, true, kPackedQ>(y, sg_out, six_out, rcp_six, stab);
+            q = quantize16<true, true, kPackedQ, k46>(y, sg_out, six_out, rcp_six, stab);
           }
           row_acc += q.sumsq;
-          amax = fmaxf(amax, q.amax);
+          amax = fmaxf(amax, kRht ? yamax : q.amax);
           if (c & 1) {
             uint8_t* dst = (E == Epi::Update)
                                ? row_codes + tiled_chunk_offset(gr, gcc - 16, row_cp)
@@ -637,7 +658,7 @@ __device__ __forceinline__ void epilogue_plain(const NsParams& p, const GemmPlai
   }
 }
 
-template <Epi E>
+template <Epi E, uint32_t kOpts>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ NsParams p, const __grid_constant__ GemmPlainArgs g) {
   using C = Cfg<E>;
@@ -772,7 +793,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (E == Epi::Plain)
       epilogue_plain(p, g, tmem, acc_full, acc_empty, status, abort_flag, wbuf, quad, ch, lane, total);
     else
-      epilogue_ns<E>(p, g, tmem, acc_full, acc_empty, status, abort_flag, wbuf, scale_tab,
+      epilogue_ns<E, kOpts>(p, g, tmem, acc_full, acc_empty, status, abort_flag, wbuf, scale_tab,
                      quad, ch, lane, total);
   }
 
@@ -784,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <Epi E>
+template <Epi E, uint32_t kOpts>
 cudaError_t launch_impl(const NsParams* p, const GemmPlainArgs* g, int64_t units, cudaStream_t st,
                         int num_sms) {
   using C = Cfg<E>;
@@ -793,7 +814,7 @@ cudaError_t launch_impl(const NsParams* p, const GemmPlainArgs* g, int64_t units
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !(attr_set & (1ull << dev))) {
-    e = cudaFuncSetAttribute(nvfp4_gemm_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(nvfp4_gemm_kernel<E, kOpts>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set |= 1ull << dev;
@@ -801,13 +822,13 @@ cudaError_t launch_impl(const NsParams* p, const GemmPlainArgs* g, int64_t units
   // setmaxnreg.inc can only hand out what the block was launched with: refuse to
   // launch unless the compiled register count is exactly the split's budget
   cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, nvfp4_gemm_kernel<E>);
+  e = cudaFuncGetAttributes(&fa, nvfp4_gemm_kernel<E, kOpts>);
   if (e != cudaSuccess) return e;
   if ((uint32_t)fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
   const int grid = (int)(units < num_sms ? (units > 0 ? units : 1) : num_sms);
   static const NsParams zero_p{};
   static const GemmPlainArgs zero_g{};
-  nvfp4_gemm_kernel<E><<<grid, kThreads, C::SMEM_BYTES, st>>>(p ? *p : zero_p, g ? *g : zero_g);
+  nvfp4_gemm_kernel<E, kOpts><<<grid, kThreads, C::SMEM_BYTES, st>>>(p ? *p : zero_p, g ? *g : zero_g);
   return cudaGetLastError();
 }
 
@@ -815,28 +836,42 @@ cudaError_t launch_impl(const NsParams* p, const GemmPlainArgs* g, int64_t units
 
 cudaError_t launch_gemm_plain(const GemmPlainArgs& a, cudaStream_t st, int num_sms) {
   const int64_t units = (int64_t)(a.Mp / BM) * ((a.Np + BN - 1) / BN);
-  return launch_impl<Epi::Plain>(nullptr, &a, units, st, num_sms);
+  return launch_impl<Epi::Plain, 0>(nullptr, &a, units, st, num_sms);
 }
 
-cudaError_t launch_gemm_ns(Epi epi, const NsParams& p, cudaStream_t st, int num_sms) {
+namespace {
+
+template <uint32_t kOpts>
+cudaError_t launch_ns_opts(Epi epi, const NsParams& p, cudaStream_t st, int num_sms) {
   const int64_t units = p.prefix[p.count];
   cudaError_t e;
   switch (epi) {
     case Epi::GramX:
-      if ((e = launch_impl<Epi::GramX>(&p, nullptr, units, st, num_sms)) != cudaSuccess) return e;
+      if ((e = launch_impl<Epi::GramX, kOpts>(&p, nullptr, units, st, num_sms)) != cudaSuccess) return e;
       ns_bounds_kernel<Epi::GramX><<<p.count, 256, 0, st>>>(p);
       break;
     case Epi::GramA:
-      if ((e = launch_impl<Epi::GramA>(&p, nullptr, units, st, num_sms)) != cudaSuccess) return e;
+      if ((e = launch_impl<Epi::GramA, kOpts>(&p, nullptr, units, st, num_sms)) != cudaSuccess) return e;
       ns_bounds_kernel<Epi::GramA><<<p.count, 256, 0, st>>>(p);
       break;
     case Epi::Update:
-      if ((e = launch_impl<Epi::Update>(&p, nullptr, units, st, num_sms)) != cudaSuccess) return e;
+      if ((e = launch_impl<Epi::Update, kOpts>(&p, nullptr, units, st, num_sms)) != cudaSuccess) return e;
       if (!p.last) ns_bounds_kernel<Epi::Update><<<p.count, 256, 0, st>>>(p);
       break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_ns(Epi epi, const NsParams& p, cudaStream_t st, int num_sms) {
+  switch (p.opts & (kOptRht | kOpt46)) {
+    case 0: return launch_ns_opts<0>(epi, p, st, num_sms);
+    case kOpt46: return launch_ns_opts<kOpt46>(epi, p, st, num_sms);
+    case kOptRht: return launch_ns_opts<kOptRht>(epi, p, st, num_sms);
+    default: return launch_ns_opts<kOptRht | kOpt46>(epi, p, st, num_sms);
+  }
 }
 
 }  // namespace fs4

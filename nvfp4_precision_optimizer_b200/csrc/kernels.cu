@@ -6,6 +6,7 @@
 // encoding; Section 3.4 for clipping before the NVFP4 iteration and for the two
 // views Q1x16(X) (Gram operand) and Q16x1(X) (update operand).
 #include <cfloat>
+#include <mutex>
 #include <cmath>
 
 #include "fs4_device.cuh"
@@ -279,7 +280,9 @@ __global__ void __launch_bounds__(kEwThreads) ns_reduce_kernel(const __grid_cons
         const float amax0 = dead ? 0.0f : fminf(__fmul_rn(amaxG, inv), tau);
         st->inv0 = inv;
         st->tau0 = tau;
-        st->sg[kSgX + 0] = pow2_tensor_scale(amax0);
+        // with the Hadamard transform the quantised tensor is X_0 H: |X_0 H| <= 4 amax
+        st->sg[kSgX + 0] = pow2_tensor_scale((p.opts & kOptRht) ? 4.0f * amax0 : amax0,
+                                             (p.opts & kOpt46) != 0);
         st->amaxX[0] = __float_as_uint(amax0);
         st->done[4] = 0u;
       }
@@ -292,6 +295,7 @@ __global__ void __launch_bounds__(kEwThreads) ns_reduce_kernel(const __grid_cons
 // and as both NVFP4 views, with row / column sums of the squared dequantised
 // values.  Work unit = one 64 x 64 tile of the padded working extent; G and X
 // are read and written as float4 with 16 threads per 64-float row segment.
+template <uint32_t kOpts>
 __global__ void __launch_bounds__(kEwThreads) ns_preamble_kernel(const __grid_constant__ NsParams p) {
   __shared__ float tile[kT][kT + 1];
   __shared__ float2 scale_tab[128];
@@ -394,7 +398,9 @@ __global__ void __launch_bounds__(kEwThreads) ns_preamble_kernel(const __grid_co
       float v[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) v[e] = view == 0 ? tile[line][blk * 16 + e] : tile[blk * 16 + e][line];
-      const QBlock16 q = quantize16<true, true>(v, sg, six_sg, rcp_six, stab);
+      // view 0 is the Gram operand of iteration 0, view 1 the update operand
+      if constexpr ((kOpts & kOptRht) != 0) rht16(v, view == 0 ? p.rht[0] : p.rht[2]);
+      const QBlock16 q = quantize16<true, true, true, (kOpts & kOpt46) != 0>(v, sg, six_sg, rcp_six, stab);
       // row (view 0: row i0+line of X, K = j0..) or row j0+line of X^T (view 1, K = i0..)
       const int64_t R = (view == 0 ? i0 : j0) + line;
       const int64_t K0 = view == 0 ? j0 : i0;
@@ -436,7 +442,8 @@ __global__ void __launch_bounds__(kEwThreads) ns_preamble_bounds_kernel(const __
   if (threadIdx.x == 0) {
     st->u_rowX[0] = ur;
     st->u_colX[0] = uc;
-    st->sg[kSgA + 0] = pow2_tensor_scale(ur * kBoundInflate);
+    st->sg[kSgA + 0] = pow2_tensor_scale(ur * kBoundInflate * ((p.opts & kOptRht) ? 4.0f : 1.0f),
+                                         (p.opts & kOpt46) != 0);
   }
 }
 
@@ -447,16 +454,29 @@ int grid_for(int64_t units, int num_sms, int per_sm) {
 
 // Grid of a persistent (grid-stride) kernel: as many CTAs as are resident at once,
 // from the occupancy the compiled kernel actually reaches (a second wave would
-// leave SMs half empty while it runs).
+// leave SMs half empty while it runs).  Cached per kernel address (kernels of one
+// signature share a pointer type, so a per-type cache would mix them up).
 template <typename Kernel>
 int persistent_grid(Kernel kernel, int64_t units, int num_sms) {
-  static int resident = 0;    // per kernel; the same on every device of one architecture
+  static std::mutex mu;
+  static const void* keys[16];
+  static int vals[16];
+  static int used = 0;
+  const void* key = reinterpret_cast<const void*>(kernel);
+  int resident = 0;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < used; ++i)
+      if (keys[i] == key) resident = vals[i];
+  }
   if (resident == 0) {
     int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kEwThreads, 0) != cudaSuccess ||
         occ < 1)
       occ = 1;
     resident = occ;
+    std::lock_guard<std::mutex> lk(mu);
+    if (used < 16) { keys[used] = key; vals[used] = occ; ++used; }
   }
   return grid_for(units, num_sms, resident);
 }
@@ -498,8 +518,19 @@ cudaError_t launch_ns_reduce(const NsParams& p, cudaStream_t st, int num_sms) {
   return cudaGetLastError();
 }
 
+template <uint32_t kOpts>
+void preamble_launch(const NsParams& p, cudaStream_t st, int num_sms) {
+  ns_preamble_kernel<kOpts><<<persistent_grid(ns_preamble_kernel<kOpts>, p.prefix[p.count], num_sms),
+                              kEwThreads, 0, st>>>(p);
+}
+
 cudaError_t launch_ns_preamble(const NsParams& p, cudaStream_t st, int num_sms) {
-  ns_preamble_kernel<<<persistent_grid(ns_preamble_kernel, p.prefix[p.count], num_sms), kEwThreads, 0, st>>>(p);
+  switch (p.opts & (kOptRht | kOpt46)) {
+    case 0: preamble_launch<0>(p, st, num_sms); break;
+    case kOpt46: preamble_launch<kOpt46>(p, st, num_sms); break;
+    case kOptRht: preamble_launch<kOptRht>(p, st, num_sms); break;
+    default: preamble_launch<kOptRht | kOpt46>(p, st, num_sms); break;
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   ns_preamble_bounds_kernel<<<p.count, kEwThreads, 0, st>>>(p);

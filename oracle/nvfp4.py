@@ -87,22 +87,30 @@ def e4m3_encode(v: np.ndarray) -> np.ndarray:
     return _nearest_even(v, _E4M3_POS)
 
 
-def global_scale(amax: float, mode: str = "pow2") -> np.float32:
-    """FP32 tensor scale s_g for a tensor whose largest |element| is ``amax``."""
+SG_DENOM_46 = 4.0 * E4M3_MAX  # 1792: under adaptive 4/6 the M = 4 candidate must fit too
+
+
+def global_scale(amax: float, mode: str = "pow2", denom: float = SG_DENOM) -> np.float32:
+    """FP32 tensor scale s_g for a tensor whose largest |element| is ``amax``.
+
+    denom: 2688 = 6 * 448 (a block's amax mapped to 6 fits the largest E4M3 scale);
+    SG_DENOM_46 = 1792 under adaptive 4/6.  Reading (the pages do not say): with
+    4/6 the tensor scale also covers the M = 4 candidate, so neither candidate's
+    block scale saturates."""
     amax = float(np.float32(amax))
     if not math.isfinite(amax) or amax < 0:
         raise ValueError("amax must be finite and non-negative")
     if amax == 0.0:
         return np.float32(1.0)
     if mode == "amax":
-        return np.float32(np.float32(amax) / np.float32(SG_DENOM))
+        return np.float32(np.float32(amax) / np.float32(denom))
     if mode != "pow2":
         raise ValueError(f"unknown tensor-scale mode {mode!r}")
-    # smallest integer e with 2688 * 2^e >= amax (exact float64 comparisons)
+    # smallest integer e with denom * 2^e >= amax (exact float64 comparisons)
     e = math.frexp(amax)[1] - 12
-    while math.ldexp(SG_DENOM, e) < amax:
+    while math.ldexp(denom, e) < amax:
         e += 1
-    while math.ldexp(SG_DENOM, e - 1) >= amax:
+    while math.ldexp(denom, e - 1) >= amax:
         e -= 1
     e = min(max(e, SG_EXP_MIN), SG_EXP_MAX)
     return np.float32(math.ldexp(1.0, e))
@@ -161,7 +169,7 @@ def quantize_rows(x: np.ndarray, s_g: float | None = None, mode: str = "pow2",
     rows, cols = x.shape
     if s_g is None:
         amax = float(np.max(np.abs(x))) if x.size else 0.0
-        s_g = global_scale(amax, mode)
+        s_g = global_scale(amax, mode, SG_DENOM_46 if adaptive46 else SG_DENOM)
     s_g = np.float32(s_g)
     blocks = x.reshape(rows, cols // BLOCK, BLOCK)
     nib, scales, deq6 = _quantize_blocks(blocks, s_g, 6.0)

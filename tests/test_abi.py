@@ -93,7 +93,16 @@ def test_root_ns_rejects_bad_arguments(F):
     assert ns(G, 64, 96, 96, G + 1024, 96, 5, 1.0, 0.0, 0.0, 3.0, 0, W, ok, None) == -3  # out overlaps G
     assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 3.0, 0, G, ok, None) == -3         # ws overlaps G
     assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 3.0, 0, W + 4, ok, None) == -4     # misaligned ws
-    assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 3.0, 1 << 3, W, ok, None) == -1    # unknown flag
+    assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 3.0, 1 << 5, W, ok, None) == -1    # unknown flag
+    # the Hadamard option needs the masks only the _ex entry point takes
+    assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 3.0, F.FS4_NS_RHT, W, ok, None) == -1
+    desc = (F.NsDesc * 1)()
+    desc[0].G, desc[0].out, desc[0].m, desc[0].n, desc[0].ld, desc[0].ld_out = G, O, 64, 96, 96, 96
+    desc[0].a, desc[0].b, desc[0].c = 1.0, 0.0, 0.0
+    ex = lib.fs4_root_ns_batched_ex
+    assert ex(1, desc, 5, 3.0, F.FS4_NS_RHT, None, W, ok, None) == -1                    # no masks
+    masks = (ctypes.c_uint16 * 15)(*range(15))
+    assert ex(1, desc, 5, 3.0, F.FS4_NS_RHT | F.FS4_NS_ADAPTIVE46, masks, W, ok - 1, None) == -4
     assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 3.0, 1 << 29, W, ok, None) == -1   # unknown flag
     # the test-only stall flag is accepted (the call then fails on the workspace size)
     assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 3.0, F.FS4_TEST_STALL, W, ok - 1, None) == -4

@@ -126,3 +126,16 @@ def test_rht46_route_stays_close_to_float64_for_contractive_quintic():
     yq = R.root_ns(G, 5, *quintic, rht_masks=masks, adaptive46=True)
     yf = R.root_ns(G, 5, *quintic, quantized=False)
     assert np.linalg.norm(yq - yf) / np.linalg.norm(yf) < 0.1
+
+
+@pytest.mark.parametrize("amax", [1e-30, 3e-5, 0.02, 1.0, 1.5, 1791.9, 1792.0, 1792.1, 3.0e30])
+def test_adaptive46_tensor_scale_covers_the_m4_candidate(amax):
+    """Under 4/6 the power-of-two s_g is the smallest with 4 * 448 * s_g >= amax, so the
+    largest block's M = 4 scale amax / (4 s_g) never exceeds the largest E4M3 value."""
+    sg = float(Q.global_scale(amax, denom=Q.SG_DENOM_46))
+    assert 1792.0 * sg >= float(np.float32(amax)) and 1792.0 * sg / 2 < float(np.float32(amax))
+    assert sg == 2.0 ** round(np.log2(sg))
+    x = np.zeros((1, 16), np.float32)
+    x[0, 0] = amax
+    codes, scales, got = Q.quantize_rows(x, adaptive46=True)
+    assert got == sg and Q.E4M3_VALUES[scales[0, 0]] * float(sg) * 6 >= float(np.float32(amax)) * 0.9
