@@ -17,6 +17,7 @@ fixed and the scaling is weak; the step time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import datetime
 import json
 import os
@@ -24,6 +25,8 @@ import statistics
 import subprocess
 import sys
 import time
+
+import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -42,6 +45,9 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quant", default="plain", choices=["plain", "rht46", "rht", "a46"],
+                    help="quantiser of the step: plain NVFP4 (default) or the Section 3.4 options "
+                         "(random Hadamard transform with fresh seeded sign masks, adaptive 4/6)")
     return ap.parse_args()
 
 
@@ -248,14 +254,22 @@ def main():
     stream = torch.cuda.current_stream()
     n_ev = 3 + 3 * K
 
+    qflags = {"plain": 0, "rht46": F.FS4_NS_RHT | F.FS4_NS_ADAPTIVE46, "rht": F.FS4_NS_RHT,
+              "a46": F.FS4_NS_ADAPTIVE46}[args.quant]
+    mask_rng = np.random.default_rng(BASE_SEED + 7)
+
     def call(events=None):
+        masks = None
+        if qflags & F.FS4_NS_RHT:        # fresh signs for every step (Section 3.4)
+            masks = (ctypes.c_uint16 * (3 * K))(*[int(v) for v in mask_rng.integers(0, 1 << 16, 3 * K)])
+        mptr = ctypes.cast(masks, ctypes.c_void_p) if masks is not None else None
         if events is None:
-            st = lib.fs4_root_ns_batched(len(Gs), arr, K, w.clip_k, 0, ws.data_ptr(), need,
-                                         stream.cuda_stream)
+            st = lib.fs4_root_ns_batched_ex(len(Gs), arr, K, w.clip_k, qflags, mptr, ws.data_ptr(),
+                                            need, stream.cuda_stream)
         else:
             ev_arr = (F._lib.c_vp * n_ev)(*[e.cuda_event for e in events])
-            st = lib.fs4_root_ns_batched_timed(len(Gs), arr, K, w.clip_k, 0, ws.data_ptr(), need,
-                                               stream.cuda_stream, ev_arr, n_ev)
+            st = lib.fs4_root_ns_batched_timed(len(Gs), arr, K, w.clip_k, qflags, mptr, ws.data_ptr(),
+                                               need, stream.cuda_stream, ev_arr, n_ev)
         F.check(st, "fs4_root_ns_batched")
 
     for _ in range(max(3, args.warmup)):
@@ -351,8 +365,11 @@ def main():
             stream.wait_event(ev["in"][b])
             if i >= 2:
                 stream.wait_event(ev["out"][b])           # step i - 2's outputs were copied out
+            masks = ([int(v) for v in mask_rng.integers(0, 1 << 16, 3 * K)]
+                     if qflags & F.FS4_NS_RHT else None)
             F.root_ns_batched(dev_in[b], K=K, coeffs=w.coeffs, clip_k=w.clip_k, outs=dev_out[b],
-                              workspace=ws, stream=stream)
+                              workspace=ws, stream=stream, rht_masks=masks,
+                              adaptive46=bool(qflags & F.FS4_NS_ADAPTIVE46))
             ev["done"][b].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev["done"][b])
@@ -397,6 +414,10 @@ def main():
             "data": "synthetic",
             "config": {"workload": w.name, "matrices": len(Gs), "shapes": sorted(set(map(tuple, w.shapes))),
                        "K": K, "coeffs": "Muon (3.4445, -4.7750, 2.0315)", "clip": "3 x RMS",
+                       "quantiser": {"plain": "NVFP4 RTN (H = I, M = 6)",
+                                     "rht46": "NVFP4 RTN with H16^r (fresh signs per step) and adaptive 4/6",
+                                     "rht": "NVFP4 RTN with H16^r (fresh signs per step)",
+                                     "a46": "NVFP4 RTN with adaptive 4/6"}[args.quant],
                        "parallelism": f"replicas x{world} (independent matrices, no collective)",
                        "l2": "inputs larger than L2 (%.2f GB per step)" % (sum(G.numel() for G in Gs) * 4 / 1e9)},
             "tflops_algorithmic": tflops,

@@ -219,17 +219,17 @@ fs4_status fs4_root_ns_batched_ex(int32_t count, const fs4_ns_desc* descs, int32
                                   uint32_t flags, const uint16_t* rht_masks, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
-/* fs4_root_ns_batched, with CUDA events recorded on `stream` around each
+/* fs4_root_ns_batched_ex, with CUDA events recorded on `stream` around each
  * phase so a caller can time the kernels on the launching stream.
  * phase_events: HOST array of n_events >= 3 + 3K cudaEvent_t handles (created
  * by the caller with timing enabled).  Event 0 is recorded before the
  * workspace reset and the reduction kernel, event 1 after it, event 2 after
- * the preamble kernel, and event 3 + 3k + j after product j (0: A = qX qX^T,
- * 1: B, 2: update) of iteration k.  Errors as fs4_root_ns_batched, plus
- * FS4_ERR_INVALID_ARG for a missing event. */
+ * the preamble kernels, and event 3 + 3k + j after product j (0: A = qX qX^T,
+ * 1: B, 2: update) of iteration k and its bounds kernel.  Errors as
+ * fs4_root_ns_batched_ex, plus FS4_ERR_INVALID_ARG for a missing event. */
 fs4_status fs4_root_ns_batched_timed(int32_t count, const fs4_ns_desc* descs, int32_t K,
-                                     float clip_k, uint32_t flags, void* workspace,
-                                     size_t workspace_bytes, void* stream,
+                                     float clip_k, uint32_t flags, const uint16_t* rht_masks,
+                                     void* workspace, size_t workspace_bytes, void* stream,
                                      void* const* phase_events, int32_t n_events);
 
 /* ------------------------------------------------------------ no-alloc variant */

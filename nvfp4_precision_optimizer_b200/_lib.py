@@ -63,7 +63,7 @@ SIGNATURES = {
     "fs4_root_ns_batched_ex": (c_i32, [c_i32, ctypes.POINTER(NsDesc), c_i32, c_f32, c_u32, c_vp,
                                        c_vp, c_sz, c_vp]),
     "fs4_root_ns_batched_timed": (c_i32, [c_i32, ctypes.POINTER(NsDesc), c_i32, c_f32, c_u32,
-                                          c_vp, c_sz, c_vp, ctypes.POINTER(c_vp), c_i32]),
+                                          c_vp, c_vp, c_sz, c_vp, ctypes.POINTER(c_vp), c_i32]),
     "fs4_root_ns_noalloc": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i64, c_i32, c_f32, c_f32,
                                     c_f32, c_f32, c_vp]),
     "fs4_device_status": (c_i32, [c_vp, c_vp]),
