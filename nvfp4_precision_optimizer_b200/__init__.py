@@ -77,11 +77,18 @@ def quantize(x: torch.Tensor, axis: int = FS4_AXIS_ROW, tiled: bool = False,
 
 
 def dequantize(codes: torch.Tensor, scales: torch.Tensor, s_g: torch.Tensor, rows: int, cols: int,
-               tiled: bool = False, stream=None) -> torch.Tensor:
-    """FP32 rows x cols matrix from an NVFP4 one (fs4_nvfp4_dequantize)."""
-    y = torch.empty((rows, cols), dtype=torch.float32, device=codes.device)
+               tiled: bool = False, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """FP32 rows x cols matrix from an NVFP4 one (fs4_nvfp4_dequantize); `out`, if
+    given, is a rows x cols FP32 view with unit column stride (any row stride)."""
+    if out is None:
+        y = torch.empty((rows, cols), dtype=torch.float32, device=codes.device)
+    else:
+        _check_f32_matrix(out, "out")
+        if tuple(out.shape) != (rows, cols):
+            raise ValueError(f"out must be {rows} x {cols}, got {tuple(out.shape)}")
+        y = out
     check(_lib.lib().fs4_nvfp4_dequantize(codes.data_ptr(), scales.data_ptr(), s_g.data_ptr(),
-                                          rows, cols, y.data_ptr(), cols,
+                                          rows, cols, y.data_ptr(), _ld(y),
                                           FS4_LAYOUT_TILED if tiled else 0, _stream(stream)),
           "fs4_nvfp4_dequantize")
     return y

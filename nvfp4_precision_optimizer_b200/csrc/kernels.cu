@@ -93,12 +93,23 @@ __global__ void __launch_bounds__(kEwThreads) amax_kernel(const float* __restric
   __shared__ float red[kEwThreads / 32];
   float m = 0.0f;
   bool bad = false;
+  const bool vec = ((reinterpret_cast<uintptr_t>(x) & 15) == 0) && ((ld & 3) == 0) && ((cols & 3) == 0);
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
     const float* row = x + r * ld;
-    for (int64_t c = threadIdx.x; c < cols; c += kEwThreads) {
-      const float v = __ldg(row + c);
-      bad |= !is_finite_bits(v);
-      m = fmaxf(m, fabsf(v));
+    if (vec) {  // float4 loads: one request per thread covers 16 bytes
+      const float4* row4 = reinterpret_cast<const float4*>(row);
+      for (int64_t c = threadIdx.x; c < (cols >> 2); c += kEwThreads) {
+        const float4 v = __ldg(row4 + c);
+        bad |= !(is_finite_bits(v.x) && is_finite_bits(v.y) && is_finite_bits(v.z) &&
+                 is_finite_bits(v.w));
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+      }
+    } else {
+      for (int64_t c = threadIdx.x; c < cols; c += kEwThreads) {
+        const float v = __ldg(row + c);
+        bad |= !is_finite_bits(v);
+        m = fmaxf(m, fabsf(v));
+      }
     }
   }
   if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(&hdr[0], kStatusNonFinite);
@@ -115,8 +126,12 @@ __global__ void __launch_bounds__(kEwThreads) quantize_kernel(
     int sg_amax_mode, int64_t Rext, int64_t Cext, int64_t Cp, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ scales, float* __restrict__ s_g_out, const uint32_t* __restrict__ hdr) {
   __shared__ float tile[kT][kT + 1];
-  const int64_t tiles_c = Cext / kT;
-  const int64_t i0 = (blockIdx.x / tiles_c) * kT, j0 = (blockIdx.x % tiles_c) * kT;
+  // Tiles are visited in x's row-major order, last tile first: the amax pass just
+  // streamed x top to bottom, so the tail of x is still resident in L2.
+  const int64_t xt = gridDim.x - 1 - blockIdx.x;
+  const int64_t xtiles_c = (col_axis ? Rext : Cext) / kT;
+  const int64_t xi0 = (xt / xtiles_c) * kT, xj0 = (xt % xtiles_c) * kT;
+  const int64_t i0 = col_axis ? xj0 : xi0, j0 = col_axis ? xi0 : xj0;
   const float amax = __uint_as_float(__ldcg(&hdr[1]));
   float s_g;
   if (sg_amax_mode) {
@@ -129,22 +144,32 @@ __global__ void __launch_bounds__(kEwThreads) quantize_kernel(
   const float rcp_six = __frcp_rn(six_sg);
 
   const int t = threadIdx.x;
-  // stage: thread t covers 16 consecutive elements of one line of x
+  // Stage the 64 x 64 tile of x (coalesced: 16 threads per 256-byte line segment, float4
+  // loads for interior tiles of 16-byte aligned inputs).  Row axis: x line = row i of the
+  // quantised matrix Y; column axis: x line = column of Y (Y = x^T), stored transposed.
   {
-    const int line = t >> 2, part = (t & 3) * 16;
-    if (!col_axis) {
-      const int64_t i = i0 + line;
+    const int64_t xr0 = col_axis ? j0 : i0, xc0 = col_axis ? i0 : j0;      // tile origin in x
+    const int64_t xrows = col_axis ? C : R, xcols = col_axis ? R : C;       // x's extent
+    const bool vec = ((reinterpret_cast<uintptr_t>(x) & 15) == 0) && ((ld & 3) == 0) &&
+                     xr0 + kT <= xrows && xc0 + kT <= xcols;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int64_t j = j0 + part + e;
-        tile[line][part + e] = (i < R && j < C) ? __ldg(x + i * ld + j) : 0.0f;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int f = t + kEwThreads * pass;
+      const int line = f >> 4, c4 = (f & 15) * 4;
+      const float* src = x + (xr0 + line) * ld + xc0 + c4;
+      float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      if (vec) {
+        const float4 x4 = __ldg(reinterpret_cast<const float4*>(src));
+        v[0] = x4.x; v[1] = x4.y; v[2] = x4.z; v[3] = x4.w;
+      } else if (xr0 + line < xrows) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (xc0 + c4 + e < xcols) v[e] = __ldg(src + e);
       }
-    } else {  // Y[i][j] = x[j][i]: read x row j0+line, columns i0+part..
-      const int64_t jx = j0 + line;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int64_t ix = i0 + part + e;
-        tile[part + e][line] = (jx < C && ix < R) ? __ldg(x + jx * ld + ix) : 0.0f;
+      for (int e = 0; e < 4; ++e) {
+        if (!col_axis) tile[line][c4 + e] = v[e];
+        else tile[c4 + e][line] = v[e];
       }
     }
   }
@@ -164,45 +189,53 @@ __global__ void __launch_bounds__(kEwThreads) quantize_kernel(
   }
 }
 
-// y = fp32(fp32(code * scale) * s_g), one thread per 16-element block.
+// y = fp32(fp32(code * scale) * s_g), one thread per group of 4 consecutive elements
+// of a row, so a warp writes 512 contiguous bytes (float4 stores when y is 16-byte
+// aligned with ld % 4 == 0).  The flat group index advances by a fixed (row, column)
+// stride, so the loop needs no 64-bit division.
 __global__ void __launch_bounds__(kEwThreads) dequantize_kernel(
     const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
     const float* __restrict__ s_g_ptr, int64_t R, int64_t C, int tiled, int64_t Cp,
     float* __restrict__ y, int64_t ld) {
   const float s_g = __ldg(s_g_ptr);
-  const int64_t nblk = R * (C / 16);
-  for (int64_t b = blockIdx.x * (int64_t)kEwThreads + threadIdx.x; b < nblk;
-       b += (int64_t)gridDim.x * kEwThreads) {
-    const int64_t i = b / (C / 16), j = (b % (C / 16)) * 16;
-    uint2 w;
-    uint32_t sb;
+  const int64_t C4 = C / 4;
+  if (R <= 0 || C4 <= 0) return;
+  const bool vec = ((reinterpret_cast<uintptr_t>(y) & 15) == 0) && ((ld & 3) == 0);
+  const int64_t g0 = blockIdx.x * (int64_t)kEwThreads + threadIdx.x;
+  const int64_t step = (int64_t)gridDim.x * kEwThreads;
+  const int64_t step_i = step / C4, step_c = step % C4;
+  int64_t i = g0 / C4, c4 = g0 % C4;
+  for (; i < R; i += step_i, c4 += step_c) {
+    if (c4 >= C4) { c4 -= C4; ++i; if (i >= R) break; }
+    const int64_t c = c4 * 4;
+    uint32_t w, sb;
     if (tiled) {
-      w = *reinterpret_cast<const uint2*>(codes + tiled_chunk_offset(i, j & ~int64_t(31), Cp) +
-                                          ((j & 16) ? 8 : 0));
-      sb = scales[tiled_scale_offset(i, j >> 4, Cp)];
+      w = *reinterpret_cast<const uint16_t*>(codes + tiled_chunk_offset(i, c & ~int64_t(31), Cp) +
+                                             ((c & 31) >> 1));
+      sb = scales[tiled_scale_offset(i, c >> 4, Cp)];
     } else {
-      w = *reinterpret_cast<const uint2*>(codes + i * (C / 2) + j / 2);
-      sb = scales[i * (C / 16) + j / 16];
+      w = *reinterpret_cast<const uint16_t*>(codes + i * (C / 2) + c / 2);
+      sb = scales[i * (C / 16) + c / 16];
     }
     const float s = e4m3_to_f32(sb);
-    uint32_t words[2] = {w.x, w.y};
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t hv[4];
-      asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-          "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-          "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-          "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-          "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-          "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-          : "=r"(hv[0]), "=r"(hv[1]), "=r"(hv[2]), "=r"(hv[3])
-          : "r"(words[h]));
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const int64_t c = j + h * 8 + p * 2;
-        y[i * ld + c] = __fmul_rn(__fmul_rn(half_lo(hv[p]), s), s_g);
-        y[i * ld + c + 1] = __fmul_rn(__fmul_rn(half_hi(hv[p]), s), s_g);
-      }
+    uint32_t hv[2];
+    // volatile: without it this decode of a 16-bit load came out wrong on sm_100a
+    // (nearly every output zero), while the same code with byte loads was exact.
+    asm volatile("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t}"
+        : "=r"(hv[0]), "=r"(hv[1])
+        : "r"(w));
+    const float4 o = make_float4(__fmul_rn(__fmul_rn(half_lo(hv[0]), s), s_g),
+                                 __fmul_rn(__fmul_rn(half_hi(hv[0]), s), s_g),
+                                 __fmul_rn(__fmul_rn(half_lo(hv[1]), s), s_g),
+                                 __fmul_rn(__fmul_rn(half_hi(hv[1]), s), s_g));
+    float* dst = y + i * ld + c;
+    if (vec) {
+      *reinterpret_cast<float4*>(dst) = o;
+    } else {
+      dst[0] = o.x; dst[1] = o.y; dst[2] = o.z; dst[3] = o.w;
     }
   }
 }
@@ -507,8 +540,8 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const
                               int64_t rows, int64_t cols, float* y, int64_t ld, uint32_t flags,
                               cudaStream_t st, int num_sms) {
   const int tiled = (flags & 2u) ? 1 : 0;
-  const int64_t nblk = rows * (cols / 16);
-  dequantize_kernel<<<persistent_grid(dequantize_kernel, (nblk + kEwThreads - 1) / kEwThreads, num_sms), kEwThreads, 0,
+  const int64_t ngrp = rows * (cols / 4);
+  dequantize_kernel<<<persistent_grid(dequantize_kernel, (ngrp + kEwThreads - 1) / kEwThreads, num_sms), kEwThreads, 0,
                       st>>>(codes, scales, s_g, rows, cols, tiled, align_up(cols, 256), y, ld);
   return cudaGetLastError();
 }

@@ -135,3 +135,62 @@ def test_quantize_decisions_next_to_every_threshold(fs4):
         assert g == want_g
         assert np.array_equal(s, want_s)
         assert np.array_equal(c, want_c), np.argwhere(c != want_c)[:5]
+
+
+@pytest.mark.parametrize("shape,axis", [((100, 272), 0), ((96, 200), 1), ((130, 1040), 0), ((272, 130), 1)])
+@pytest.mark.parametrize("tiled", [False, True])
+def test_quantize_strided_unaligned_input(fs4, shape, axis, tiled):
+    """x as a column-offset view of a wider matrix: its base is 4 bytes past a
+    16-byte boundary and its row stride is not a multiple of 4 floats, so the
+    quantiser takes its scalar staging path on every tile."""
+    R0, C0 = shape
+    rng = np.random.default_rng(17 + R0 + C0)
+    big = (rng.standard_normal((R0, C0 + 7)) * 0.05).astype(np.float32)
+    xt = torch.from_numpy(big).cuda()[:, 1:C0 + 1]
+    assert xt.stride(0) % 4 != 0 and (xt.data_ptr() % 16) != 0
+    x = np.ascontiguousarray(big[:, 1:C0 + 1])
+    want_c, want_s, want_g = Q.quantize_rows(x) if axis == 0 else Q.quantize_cols(x)
+    c, s, g = fs4.quantize(xt, axis=axis, tiled=tiled)
+    torch.cuda.synchronize()
+    c, s, g = c.cpu().numpy(), s.cpu().numpy(), s_g_value(g)
+    R, C = (R0, C0) if axis == 0 else (C0, R0)
+    if tiled:
+        c, s, _, _ = tiled_to_plain(c, s, R, C)
+    assert np.float32(g) == want_g
+    assert np.array_equal(s, want_s)
+    assert np.array_equal(c, want_c)
+
+
+def s_g_value(g):
+    return g.cpu().numpy()[0]
+
+
+@pytest.mark.parametrize("tiled", [False, True])
+def test_dequantize_into_strided_unaligned_view(fs4, tiled):
+    """Dequantise into a column-offset view (scalar store path): every element
+    matches the oracle bit for bit and the columns around the view keep their
+    sentinel."""
+    x = CASES["gauss_ragged_100x272"]
+    R, C = x.shape
+    codes, scales, sg = fs4.quantize(torch.from_numpy(x).cuda(), tiled=tiled)
+    big = torch.full((R, C + 5), 7.0, dtype=torch.float32, device="cuda")
+    view = big[:, 1:C + 1]
+    fs4.dequantize(codes, scales, sg, R, C, tiled=tiled, out=view)
+    got = big.cpu().numpy()
+    wc, ws, wg = Q.quantize_rows(x)
+    want = Q.dequantize_rows(wc, ws, wg, dtype=np.float32)
+    assert np.array_equal(got[:, 1:C + 1].view(np.uint32), want.view(np.uint32))
+    assert (got[:, 0] == 7.0).all() and (got[:, C + 1:] == 7.0).all()
+
+
+@pytest.mark.parametrize("shape", [(4096, 4096), (1000, 2064)])
+def test_dequantize_large_grid_stride(fs4, shape):
+    """Shapes with more 4-element groups than one persistent wave holds, so the
+    grid-stride loop wraps rows several times (including a ragged last row)."""
+    rng = np.random.default_rng(shape[0])
+    x = rng.standard_normal(shape).astype(np.float32)
+    codes, scales, sg = fs4.quantize(torch.from_numpy(x).cuda())
+    y = fs4.dequantize(codes, scales, sg, *shape).cpu().numpy()
+    wc, ws, wg = Q.quantize_rows(x)
+    want = Q.dequantize_rows(wc, ws, wg, dtype=np.float32)
+    assert np.array_equal(y.view(np.uint32), want.view(np.uint32))
