@@ -45,6 +45,11 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default="ns", choices=["ns", "quantize", "dequantize"],
+                    help="ns: the Newton-Schulz step (default); quantize / dequantize: the standalone "
+                         "NVFP4 calls over every matrix of the workload (row axis)")
+    ap.add_argument("--layout", default="plain", choices=["plain", "tiled"],
+                    help="NVFP4 layout of --op quantize / dequantize")
     ap.add_argument("--quant", default="plain", choices=["plain", "rht46", "rht", "a46"],
                     help="quantiser of the step: plain NVFP4 (default) or the Section 3.4 options "
                          "(random Hadamard transform with fresh seeded sign masks, adaptive 4/6)")
@@ -186,12 +191,66 @@ def oracle_sample_rate(w, budget_s: float):
     return 1.0 / per_matrix_s, dt, desc
 
 
+QD_BYTES = 4.5625          # algorithmic bytes per element: 4 B of FP32 + 0.5 B of codes + 1/16 B of scale
+QD_METRIC = {"quantize": "NVFP4 standalone quantise GB/s (4.5625 B per element)",
+             "dequantize": "NVFP4 standalone dequantise GB/s (4.5625 B per element)"}
+
+
+def oracle_qd_rate(w, op: str, budget_s: float):
+    """Time the oracle's quantiser (or dequantiser) on leading rows of the workload's
+    first matrix, growing the slice until it takes about budget_s / 4 seconds.
+    Returns (algorithmic GB/s, seconds, description)."""
+    from oracle import nvfp4 as Q
+    from nvfp4_precision_optimizer_b200.workloads import BASE_SEED, generate
+    G = generate(w.shapes[0], w.dist, BASE_SEED, "cpu").numpy()
+    rows = 16
+    while True:
+        x = G[:rows]
+        if op == "quantize":
+            t0 = time.perf_counter()
+            Q.quantize_rows(x)
+            dt = time.perf_counter() - t0
+        else:
+            c, sc, g = Q.quantize_rows(x)
+            t0 = time.perf_counter()
+            Q.dequantize_rows(c, sc, g, dtype=np.float32)
+            dt = time.perf_counter() - t0
+        if dt >= budget_s / 4 or rows >= G.shape[0]:
+            break
+        rows = min(G.shape[0], rows * 4)
+    rate = x.size * QD_BYTES / dt / 1e9
+    desc = (f"oracle {op} (numpy, exact NVFP4 emulation) of the first {rows} rows of a "
+            f"{G.shape[0]}x{G.shape[1]} workload matrix, {dt:.2f} s")
+    return rate, dt, desc
+
+
 def run_reference(args):
     from nvfp4_precision_optimizer_b200.workloads import WORKLOADS
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     w = WORKLOADS[args.workload]
+    if args.op != "ns":
+        rates, desc = [], ""
+        for i in range(args.warmup + args.steps):
+            rate, dt, desc = oracle_qd_rate(w, args.op, max(2.0, 120.0 / max(1, args.steps + args.warmup)))
+            if i >= args.warmup:
+                rates.append(rate)
+        value = statistics.median(rates)
+        total = sum(r * c for r, c in w.shapes) * QD_BYTES
+        line = {
+            "impl": "reference", "metric": QD_METRIC[args.op], "value": value, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * total / (value * 1e9), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32 values, exact NVFP4 emulation",
+            "data": "synthetic", "config": {"workload": w.name, "matrices": len(w.shapes), "op": args.op,
+                                            "layout": "plain"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return
     budget = max(5.0, 150.0 / max(1, args.steps + args.warmup))
     rates = []
     desc = ""
@@ -244,6 +303,11 @@ def main():
         return float(t.item())
 
     w = WORKLOADS[args.workload]
+    if args.op != "ns":
+        run_standalone(args, w, rank, world, local, barrier, max_over_ranks)
+        if world > 1:
+            dist.destroy_process_group()
+        return
     K = w.K
     Gs = matrices(w, device="cuda", seed=BASE_SEED + 1000 * rank)
     outs = [torch.empty_like(G) for G in Gs]
@@ -433,6 +497,190 @@ def main():
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def run_standalone(args, w, rank, world, local, barrier, max_over_ranks):
+    """--op quantize / dequantize: one step = one fs4_nvfp4_quantize (or _dequantize)
+    call per matrix of the workload, row axis, outputs preallocated."""
+    import torch
+    import nvfp4_precision_optimizer_b200 as F
+    from nvfp4_precision_optimizer_b200.workloads import BASE_SEED, matrices
+
+    lib = F._lib.lib()
+    tiled = args.layout == "tiled"
+    flags = F.FS4_LAYOUT_TILED if tiled else 0
+    Gs = matrices(w, device="cuda", seed=BASE_SEED + 1000 * rank)
+    stream = torch.cuda.current_stream()
+    qws_bytes = int(lib.fs4_nvfp4_quantize_workspace_size())
+    bufs = []
+    for G in Gs:
+        R, C = G.shape
+        nc, ns = F.tiled_shape(R, C) if tiled else (R * C // 2, R * C // 16)
+        bufs.append({"codes": torch.empty(nc, dtype=torch.uint8, device="cuda"),
+                     "scales": torch.empty(ns, dtype=torch.uint8, device="cuda"),
+                     "sg": torch.empty(1, dtype=torch.float32, device="cuda"),
+                     "ws": torch.zeros(qws_bytes, dtype=torch.uint8, device="cuda"),
+                     "y": torch.empty_like(G) if args.op == "dequantize" else None})
+
+    def quantize(i, x, st):
+        G, b = Gs[i], bufs[i]
+        F.check(lib.fs4_nvfp4_quantize(x.data_ptr(), G.shape[0], G.shape[1], G.shape[1], 0,
+                                       b["codes"].data_ptr(), b["scales"].data_ptr(), b["sg"].data_ptr(),
+                                       flags, b["ws"].data_ptr(), qws_bytes, st.cuda_stream),
+                "fs4_nvfp4_quantize")
+
+    def dequantize(i, y, st):
+        G, b = Gs[i], bufs[i]
+        F.check(lib.fs4_nvfp4_dequantize(b["codes"].data_ptr(), b["scales"].data_ptr(), b["sg"].data_ptr(),
+                                         G.shape[0], G.shape[1], y.data_ptr(), G.shape[1], flags,
+                                         st.cuda_stream), "fs4_nvfp4_dequantize")
+
+    def step():
+        for i in range(len(Gs)):
+            if args.op == "quantize":
+                quantize(i, Gs[i], stream)
+            else:
+                dequantize(i, bufs[i]["y"], stream)
+
+    for i in range(len(Gs)):              # codes for the dequantiser; warms the quantiser
+        quantize(i, Gs[i], stream)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    for b in bufs:
+        F.check(F.device_status(b["ws"]), "device status after warm-up")
+
+    call_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(Gs) + 1)] for _ in range(args.steps)]
+    for evs in call_ev:
+        for e in evs:
+            e.record(stream)
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    with sampler:
+        time.sleep(0.3)
+        for s in range(args.steps):
+            call_ev[s][0].record(stream)
+            for i in range(len(Gs)):
+                if args.op == "quantize":
+                    quantize(i, Gs[i], stream)
+                else:
+                    dequantize(i, bufs[i]["y"], stream)
+                call_ev[s][i + 1].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    total_ms = max_over_ranks(call_ev[0][0].elapsed_time(call_ev[-1][-1]))
+    ms_step = total_ms / args.steps
+    elems = sum(G.numel() for G in Gs)
+    value = world * elems * QD_BYTES / (ms_step * 1e-3) / 1e9
+
+    # roofline of one call (the amax and quantise launches of fs4_nvfp4_quantize, or
+    # the one dequantise launch), averaged over every call of the timed steps
+    call_ms = [evs[i].elapsed_time(evs[i + 1]) for evs in call_ev for i in range(len(Gs))]
+    call_bytes = elems * QD_BYTES / len(Gs)
+    mean_call = statistics.mean(call_ms)
+    peaks, peak_src = measured_peaks()
+    achieved = call_bytes / (mean_call * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+            "kernel": ("fs4_nvfp4_quantize call (amax_kernel + quantize_kernel)" if args.op == "quantize"
+                       else "fs4_nvfp4_dequantize call (dequantize_kernel)"),
+            "ms_per_launch": mean_call, "peak_source": f"hbm_gbs ({peak_src} MEASURED_PEAKS.json)"}
+
+    # end to end with host buffers: per matrix, copy in, call, copy out, pipelined over a
+    # copy-in, a compute and a copy-out stream (each matrix has its own device buffers)
+    e2e = None
+    if not args.no_e2e:
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        if args.op == "quantize":
+            host_in = [G.cpu().pin_memory() for G in Gs]
+            dev_in = [torch.empty_like(G) for G in Gs]
+            host_out = [(torch.empty(b["codes"].shape, dtype=torch.uint8).pin_memory(),
+                         torch.empty(b["scales"].shape, dtype=torch.uint8).pin_memory(),
+                         torch.empty(1, dtype=torch.float32).pin_memory()) for b in bufs]
+            dev_out = [(b["codes"], b["scales"], b["sg"]) for b in bufs]
+        else:
+            host_in = [(b["codes"].cpu().pin_memory(), b["scales"].cpu().pin_memory(),
+                        b["sg"].cpu().pin_memory()) for b in bufs]
+            dev_in = [(b["codes"], b["scales"], b["sg"]) for b in bufs]
+            host_out = [torch.empty(G.shape, dtype=torch.float32).pin_memory() for G in Gs]
+            dev_out = [b["y"] for b in bufs]
+        ev_in = [torch.cuda.Event() for _ in Gs]
+        ev_done = [torch.cuda.Event() for _ in Gs]
+        ev_out = [torch.cuda.Event() for _ in Gs]
+        for e in ev_in + ev_done + ev_out:
+            e.record(stream)
+
+        def copy(dst, src):
+            if isinstance(dst, tuple):
+                for d, h in zip(dst, src):
+                    d.copy_(h, non_blocking=True)
+            else:
+                dst.copy_(src, non_blocking=True)
+
+        def e2e_step():
+            for i in range(len(Gs)):
+                with torch.cuda.stream(s_in):
+                    s_in.wait_event(ev_done[i])        # the previous step's call read dev_in[i]
+                    copy(dev_in[i], host_in[i])
+                    ev_in[i].record(s_in)
+                stream.wait_event(ev_in[i])
+                stream.wait_event(ev_out[i])           # the previous step's outputs were copied out
+                if args.op == "quantize":
+                    quantize(i, dev_in[i], stream)
+                else:
+                    dequantize(i, dev_out[i], stream)
+                ev_done[i].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_done[i])
+                    copy(host_out[i], dev_out[i])
+                    ev_out[i].record(s_out)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e2e_steps = max(2, min(args.steps, 5))
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        s_in.wait_event(e0)
+        for _ in range(e2e_steps):
+            e2e_step()
+        for e in ev_out:
+            stream.wait_event(e)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
+        nb_fp32 = elems * 4
+        nb_q = sum(b["codes"].numel() + b["scales"].numel() + 4 for b in bufs)
+        e2e = {"value": world * elems * QD_BYTES / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": nb_fp32 if args.op == "quantize" else nb_q,
+               "d2h_bytes_per_step": nb_q if args.op == "quantize" else nb_fp32,
+               "ms_per_step": e2e_ms,
+               "pipeline": "per matrix: copy-in, call and copy-out overlap on three streams"}
+    for b in bufs:
+        F.check(F.device_status(b["ws"]), "device status after the timed steps")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, dt, desc = oracle_qd_rate(w, args.op, 20.0)
+        cpu = {"value": rate, "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle", "sample": desc}
+    if rank == 0:
+        line = {
+            "metric": QD_METRIC[args.op], "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32 <-> nvfp4 (e2m1 x e4m3/16, fp32 tensor scale)", "data": "synthetic",
+            "config": {"workload": w.name, "matrices": len(Gs), "op": args.op, "layout": args.layout,
+                       "axis": "row (1x16 blocks)", "s_g": "power of two",
+                       "parallelism": f"replicas x{world} (independent matrices, no collective)",
+                       "l2": "inputs larger than L2 (%.2f GB of FP32 per step)" % (elems * 4 / 1e9)},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps * len(Gs) * (2 if args.op == "quantize" else 1),
+            "clocks": sampler.summary(),
+        }
+        print(json.dumps(line), flush=True)
 
 
 if __name__ == "__main__":

@@ -157,15 +157,25 @@ __device__ __forceinline__ float div_rn_fma(float x, float d, float rcp) {
 // RN(1 / den) = RN(1 / value) * 2^-k exactly, because the product stays a normal
 // number for every block scale reachable from a tensor scale of the form chosen by
 // pow2_tensor_scale (den <= 2^125.5, so 1 / den >= 2^-125.5).
+// Decoded E4M3 block scales and their reciprocals, looked up by scale byte: tab[b] is
+// the value of byte b and tab[128 + b] = RN(1 / value), 256 floats in shared memory.
+// Two float arrays rather than one of float2: lanes with different bytes then share a
+// bank only when the bytes differ by a multiple of 32 (scales 16x apart), where
+// 8-byte entries collide already at bytes 16 apart (scales 4x apart).
 struct ScaleTab {
-  const float2* tab;   // 128 entries in shared memory
+  const float* tab;    // 256 floats in shared memory
   float rcp_sg;        // 1 / s_g, exact
 };
 
-__device__ __forceinline__ float2 scale_tab_entry(uint32_t b) {
-  if (b == 0u || b >= 127u) return make_float2(0.0f, 0.0f);
-  const float v = e4m3_to_f32(b);
-  return make_float2(v, __frcp_rn(v));
+// Fill entry b (0 <= b < 128) of a scale table.
+__device__ __forceinline__ void scale_tab_fill(float* tab, uint32_t b) {
+  float v = 0.0f, r = 0.0f;
+  if (b != 0u && b < 127u) {
+    v = e4m3_to_f32(b);
+    r = __frcp_rn(v);
+  }
+  tab[b] = v;
+  tab[128u + b] = r;
 }
 
 // ------------------------------------------------------------------ packed FP32 pairs
@@ -289,9 +299,8 @@ __device__ __forceinline__ QBlock16 quantize16(const float* x, float s_g, float 
     }
     float rcp = 0.0f;
     if constexpr (kTab) {
-      const float2 t = st.tab[r.scale];
-      den = __fmul_rn(t.x, s_g);
-      rcp = t.y * st.rcp_sg;
+      den = __fmul_rn(st.tab[r.scale], s_g);
+      rcp = st.tab[128u + r.scale] * st.rcp_sg;
     } else {
       den = __fmul_rn(e4m3_to_f32(r.scale), s_g);
       if (kPow2) rcp = __frcp_rn(den);

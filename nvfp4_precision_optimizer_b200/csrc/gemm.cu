@@ -361,7 +361,7 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
                                             uint32_t tmem, uint64_t* acc_full,
                                             uint64_t* acc_empty,
                                             uint32_t* status, volatile int* abort_flag,
-                                            float* wbuf, const float2* scale_tab, int quad, int ch,
+                                            float* wbuf, const float* scale_tab, int quad, int ch,
                                             int lane, int32_t total) {
   const int32_t first = blockIdx.x, step = gridDim.x;
   constexpr bool kIn = (E == Epi::GramA || E == Epi::Update);   // reads an FP32 tile
@@ -676,8 +676,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* stall_bar = acc_full + 3;        // test only: never arrived on
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
-  float2* scale_tab = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(bars) + C::BAR_BYTES);
-  if (threadIdx.x >= 128 && threadIdx.x < 256) scale_tab[threadIdx.x - 128] = scale_tab_entry(threadIdx.x - 128);
+  float* scale_tab = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + C::BAR_BYTES);
+  if (threadIdx.x >= 128 && threadIdx.x < 256) scale_tab_fill(scale_tab, threadIdx.x - 128);
 
   uint32_t* status = (E == Epi::Plain) ? g.status : p.status;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -5,6 +5,7 @@
 // "Full-Stack FP4" (arXiv 2607.04422): Section 2 "NVFP4 format" for the block
 // encoding; Section 3.4 for clipping before the NVFP4 iteration and for the two
 // views Q1x16(X) (Gram operand) and Q16x1(X) (update operand).
+#include <algorithm>
 #include <cfloat>
 #include <mutex>
 #include <cmath>
@@ -94,21 +95,39 @@ __global__ void __launch_bounds__(kEwThreads) amax_kernel(const float* __restric
   float m = 0.0f;
   bool bad = false;
   const bool vec = ((reinterpret_cast<uintptr_t>(x) & 15) == 0) && ((ld & 3) == 0) && ((cols & 3) == 0);
-  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-    const float* row = x + r * ld;
-    if (vec) {  // float4 loads: one request per thread covers 16 bytes
-      const float4* row4 = reinterpret_cast<const float4*>(row);
-      for (int64_t c = threadIdx.x; c < (cols >> 2); c += kEwThreads) {
-        const float4 v = __ldg(row4 + c);
-        bad |= !(is_finite_bits(v.x) && is_finite_bits(v.y) && is_finite_bits(v.z) &&
-                 is_finite_bits(v.w));
-        m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  if (vec && ld == cols) {  // contiguous: one flat float4 stream, four loads in flight per thread
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const int64_t n4 = rows * (cols >> 2);
+    const int64_t stride = (int64_t)gridDim.x * kEwThreads;
+    for (int64_t f = blockIdx.x * (int64_t)kEwThreads + threadIdx.x; f < n4; f += 4 * stride) {
+      float4 v[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        v[k] = f + k * stride < n4 ? __ldg(x4 + f + k * stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        bad |= !(is_finite_bits(v[k].x) && is_finite_bits(v[k].y) && is_finite_bits(v[k].z) &&
+                 is_finite_bits(v[k].w));
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(v[k].x), fabsf(v[k].y)), fmaxf(fabsf(v[k].z), fabsf(v[k].w))));
       }
-    } else {
-      for (int64_t c = threadIdx.x; c < cols; c += kEwThreads) {
-        const float v = __ldg(row + c);
-        bad |= !is_finite_bits(v);
-        m = fmaxf(m, fabsf(v));
+    }
+  } else {
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+      const float* row = x + r * ld;
+      if (vec) {  // float4 loads: one request per thread covers 16 bytes
+        const float4* row4 = reinterpret_cast<const float4*>(row);
+        for (int64_t c = threadIdx.x; c < (cols >> 2); c += kEwThreads) {
+          const float4 v = __ldg(row4 + c);
+          bad |= !(is_finite_bits(v.x) && is_finite_bits(v.y) && is_finite_bits(v.z) &&
+                   is_finite_bits(v.w));
+          m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        }
+      } else {
+        for (int64_t c = threadIdx.x; c < cols; c += kEwThreads) {
+          const float v = __ldg(row + c);
+          bad |= !is_finite_bits(v);
+          m = fmaxf(m, fabsf(v));
+        }
       }
     }
   }
@@ -192,7 +211,10 @@ __global__ void __launch_bounds__(kEwThreads) quantize_kernel(
 // y = fp32(fp32(code * scale) * s_g), one thread per group of 4 consecutive elements
 // of a row, so a warp writes 512 contiguous bytes (float4 stores when y is 16-byte
 // aligned with ld % 4 == 0).  The flat group index advances by a fixed (row, column)
-// stride, so the loop needs no 64-bit division.
+// stride, so the loop needs no 64-bit division; each pass handles kDqUnroll groups
+// whose code and scale loads are all issued before the first store.
+constexpr int kDqUnroll = 4;
+
 __global__ void __launch_bounds__(kEwThreads) dequantize_kernel(
     const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
     const float* __restrict__ s_g_ptr, int64_t R, int64_t C, int tiled, int64_t Cp,
@@ -205,37 +227,51 @@ __global__ void __launch_bounds__(kEwThreads) dequantize_kernel(
   const int64_t step = (int64_t)gridDim.x * kEwThreads;
   const int64_t step_i = step / C4, step_c = step % C4;
   int64_t i = g0 / C4, c4 = g0 % C4;
-  for (; i < R; i += step_i, c4 += step_c) {
-    if (c4 >= C4) { c4 -= C4; ++i; if (i >= R) break; }
-    const int64_t c = c4 * 4;
-    uint32_t w, sb;
-    if (tiled) {
-      w = *reinterpret_cast<const uint16_t*>(codes + tiled_chunk_offset(i, c & ~int64_t(31), Cp) +
-                                             ((c & 31) >> 1));
-      sb = scales[tiled_scale_offset(i, c >> 4, Cp)];
-    } else {
-      w = *reinterpret_cast<const uint16_t*>(codes + i * (C / 2) + c / 2);
-      sb = scales[i * (C / 16) + c / 16];
+  while (i < R) {
+    int64_t gi[kDqUnroll], gc[kDqUnroll];
+    uint32_t w[kDqUnroll], sb[kDqUnroll];
+#pragma unroll
+    for (int k = 0; k < kDqUnroll; ++k) {
+      gi[k] = i;
+      gc[k] = c4 * 4;
+      if (i < R) {
+        const int64_t c = gc[k];
+        if (tiled) {
+          w[k] = *reinterpret_cast<const uint16_t*>(
+              codes + tiled_chunk_offset(i, c & ~int64_t(31), Cp) + ((c & 31) >> 1));
+          sb[k] = scales[tiled_scale_offset(i, c >> 4, Cp)];
+        } else {
+          w[k] = *reinterpret_cast<const uint16_t*>(codes + i * (C / 2) + c / 2);
+          sb[k] = scales[i * (C / 16) + c / 16];
+        }
+      }
+      i += step_i;
+      c4 += step_c;
+      if (c4 >= C4) { c4 -= C4; ++i; }
     }
-    const float s = e4m3_to_f32(sb);
-    uint32_t hv[2];
-    // volatile: without it this decode of a 16-bit load came out wrong on sm_100a
-    // (nearly every output zero), while the same code with byte loads was exact.
-    asm volatile("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "mov.b32 {b0, b1, b2, b3}, %2;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t}"
-        : "=r"(hv[0]), "=r"(hv[1])
-        : "r"(w));
-    const float4 o = make_float4(__fmul_rn(__fmul_rn(half_lo(hv[0]), s), s_g),
-                                 __fmul_rn(__fmul_rn(half_hi(hv[0]), s), s_g),
-                                 __fmul_rn(__fmul_rn(half_lo(hv[1]), s), s_g),
-                                 __fmul_rn(__fmul_rn(half_hi(hv[1]), s), s_g));
-    float* dst = y + i * ld + c;
-    if (vec) {
-      *reinterpret_cast<float4*>(dst) = o;
-    } else {
-      dst[0] = o.x; dst[1] = o.y; dst[2] = o.z; dst[3] = o.w;
+#pragma unroll
+    for (int k = 0; k < kDqUnroll; ++k) {
+      if (gi[k] >= R) break;
+      const float s = e4m3_to_f32(sb[k]);
+      uint32_t hv[2];
+      // volatile: without it this decode of a 16-bit load came out wrong on sm_100a
+      // (nearly every output zero), while the same code with byte loads was exact.
+      asm volatile("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+                   "mov.b32 {b0, b1, b2, b3}, %2;\n\t"
+                   "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+                   "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t}"
+                   : "=r"(hv[0]), "=r"(hv[1])
+                   : "r"(w[k]));
+      const float4 o = make_float4(__fmul_rn(__fmul_rn(half_lo(hv[0]), s), s_g),
+                                   __fmul_rn(__fmul_rn(half_hi(hv[0]), s), s_g),
+                                   __fmul_rn(__fmul_rn(half_lo(hv[1]), s), s_g),
+                                   __fmul_rn(__fmul_rn(half_hi(hv[1]), s), s_g));
+      float* dst = y + gi[k] * ld + gc[k];
+      if (vec) {
+        *reinterpret_cast<float4*>(dst) = o;
+      } else {
+        dst[0] = o.x; dst[1] = o.y; dst[2] = o.z; dst[3] = o.w;
+      }
     }
   }
 }
@@ -331,10 +367,10 @@ __global__ void __launch_bounds__(kEwThreads) ns_reduce_kernel(const __grid_cons
 template <uint32_t kOpts>
 __global__ void __launch_bounds__(kEwThreads) ns_preamble_kernel(const __grid_constant__ NsParams p) {
   __shared__ float tile[kT][kT + 1];
-  __shared__ float2 scale_tab[128];
+  __shared__ float scale_tab[256];
   const int32_t total = p.prefix[p.count];
   const int t = threadIdx.x;
-  if (t < 128) scale_tab[t] = scale_tab_entry(t);   // read after the first barrier below
+  if (t < 128) scale_tab_fill(scale_tab, t);   // read after the first barrier below
 
   // The next unit's G tile is loaded into registers while this unit is quantised
   // (interior tiles of 16-byte aligned inputs; edge tiles load on the guarded path).
@@ -522,7 +558,8 @@ cudaError_t launch_quantize(const float* x, int64_t rows, int64_t cols, int64_t 
   cudaError_t e = cudaMemsetAsync(ws, 0, 8, st);
   if (e != cudaSuccess) return e;
   uint32_t* hdr = reinterpret_cast<uint32_t*>(ws);
-  amax_kernel<<<persistent_grid(amax_kernel, rows, num_sms), kEwThreads, 0, st>>>(x, rows, cols, ld, hdr);
+  const int64_t amax_units = std::max<int64_t>(rows, (rows * cols + 4095) / 4096);  // 4 float4 per thread
+  amax_kernel<<<persistent_grid(amax_kernel, amax_units, num_sms), kEwThreads, 0, st>>>(x, rows, cols, ld, hdr);
   const int64_t R = axis ? cols : rows, C = axis ? rows : cols;
   const int tiled = (flags & 2u) ? 1 : 0;
   const int64_t Rext = tiled ? align_up(R, 128) : align_up(R, kT);
