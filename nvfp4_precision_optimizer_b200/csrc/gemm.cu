@@ -398,8 +398,14 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
     NsState* st = reinterpret_cast<NsState*>(p.ws + d.state_off);
     const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
     if constexpr (!kIn) fp = tile_rows<E>(p, g, u, quad, ch, lane);
-    // warp-uniform by construction: the chunk loop shuffles under this condition
-    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, tl & 1u, status, abort_flag));
+    // One lane polls the barrier (32 lanes polling one mbarrier serialise on its bank);
+    // the warp then synchronises, which with tcgen05.fence::after_thread_sync below
+    // orders every lane's accumulator loads after the MMAs.  Warp-uniform by
+    // construction: the chunk loop shuffles under this condition.
+    const bool ok = __shfl_sync(0xFFFFFFFFu,
+                                lane == 0 ? (mbar_wait(acc_full, tl & 1u, status, abort_flag) ? 1 : 0) : 0,
+                                0) != 0;
+    __syncwarp();
     const int64_t gr0 = j.row0 + 32 * quad;   // first row of this warp's band
     const int64_t gr = gr0 + lane;             // this lane's row
     const int64_t gc0 = j.col0 + 128 * ch;     // first column of this warp's half
@@ -625,7 +631,11 @@ __device__ __forceinline__ void epilogue_plain(const NsParams& p, const GemmPlai
   uint32_t tl = 0;
   for (int32_t u = blockIdx.x; u < total; u += gridDim.x, ++tl) {
     const Job j = make_job<Epi::Plain>(u, p, g);
-    const bool ok = mbar_wait(acc_full, tl & 1u, status, abort_flag);
+    // one lane polls; the result is warp-uniform (the TMEM loads below are .sync.aligned)
+    const bool ok = __shfl_sync(0xFFFFFFFFu,
+                                lane == 0 ? (mbar_wait(acc_full, tl & 1u, status, abort_flag) ? 1 : 0) : 0,
+                                0) != 0;
+    __syncwarp();
     if (!ok) continue;
     const int64_t gr0 = j.row0 + 32 * quad;
     const float acc_scale = __ldg(g.a_sg) * __ldg(g.b_sg);
