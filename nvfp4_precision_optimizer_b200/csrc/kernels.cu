@@ -360,13 +360,27 @@ __global__ void __launch_bounds__(kEwThreads) ns_reduce_kernel(const __grid_cons
   }
 }
 
+// Preamble tile in shared memory: 64 rows of 64 floats in 16-byte chunks, chunk c of row
+// R stored at chunk c ^ pre_swz(R, c).  The XOR keeps every access of the kernel free of
+// bank conflicts: a quarter-warp reading four chunks of each of two adjacent rows (row
+// view, float4), a warp reading one column of four rows 16 apart (column view), and a
+// quarter-warp writing eight consecutive chunks of one row (staging); the transposed
+// staging of a tall matrix is 2-way.
+__device__ __forceinline__ int pre_swz(int R, int c) {
+  return (2 * (c >> 3)) ^ (R & 1) ^ ((R >> 2) & 1) ^ (2 * ((R >> 4) & 1)) ^ (4 * ((R >> 5) & 1));
+}
+__device__ __forceinline__ int pre_off(int R, int col) {   // float offset of (R, col)
+  const int c = col >> 2;
+  return R * kT + 4 * (c ^ pre_swz(R, c)) + (col & 3);
+}
+
 // Normalise, clip and quantise: X0 = clamp(fp32(G * inv), +-tau) written as FP32
 // and as both NVFP4 views, with row / column sums of the squared dequantised
 // values.  Work unit = one 64 x 64 tile of the padded working extent; G and X
 // are read and written as float4 with 16 threads per 64-float row segment.
 template <uint32_t kOpts>
-__global__ void __launch_bounds__(kEwThreads) ns_preamble_kernel(const __grid_constant__ NsParams p) {
-  __shared__ float tile[kT][kT + 1];
+__global__ void __launch_bounds__(kEwThreads, 4) ns_preamble_kernel(const __grid_constant__ NsParams p) {
+  __shared__ __align__(16) float tile[kT * kT];
   __shared__ float scale_tab[256];
   const int32_t total = p.prefix[p.count];
   const int t = threadIdx.x;
@@ -400,6 +414,12 @@ __global__ void __launch_bounds__(kEwThreads) ns_preamble_kernel(const __grid_co
   };
   prefetch(blockIdx.x);
 
+  // scalars of the current matrix (derived once by the reduction kernel), reloaded only
+  // when the unit belongs to another matrix than the previous one
+  int cur_mi = -1;
+  bool dead = false;
+  float inv = 0.0f, tau = 0.0f, sg = 1.0f, six_sg = 6.0f, rcp_six = 1.0f, rcp_sg = 1.0f;
+
   for (int32_t u = blockIdx.x; u < total; u += gridDim.x) {
     float4 cur[4];
 #pragma unroll
@@ -408,26 +428,32 @@ __global__ void __launch_bounds__(kEwThreads) ns_preamble_kernel(const __grid_co
     prefetch(u + gridDim.x);
     const int mi = owner_of(p.prefix, p.count, u);
     const MatDesc& d = p.mat[mi];
-    NsState* st = state_of(p, d);
     const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
     const int32_t tiles_n = d.np / kT;
     const int32_t lu = u - p.prefix[mi];
     const int32_t ti = lu / tiles_n;                       // 32-bit: units < 2^31
     const int32_t i0 = ti * kT, j0 = (lu - ti * tiles_n) * kT;
+    if (mi != cur_mi) {
+      const NsState* st = state_of(p, d);
+      cur_mi = mi;
+      dead = __ldcg(&st->nonfinite) != 0u;
+      inv = __ldcg(&st->inv0);
+      tau = __ldcg(&st->tau0);
+      sg = __ldcg(&st->sg[kSgX + 0]);
+      six_sg = __fmul_rn(6.0f, sg);
+      rcp_six = __frcp_rn(six_sg);
+      rcp_sg = __frcp_rn(sg);   // sg is a power of two
+    }
+    const ScaleTab stab{scale_tab, rcp_sg};
 
-    // scalars of this matrix, derived once by the reduction kernel
-    const bool dead = __ldcg(&st->nonfinite) != 0u;
-    const float inv = __ldcg(&st->inv0), tau = __ldcg(&st->tau0);
-    const float sg = __ldcg(&st->sg[kSgX + 0]);
-    const float six_sg = __fmul_rn(6.0f, sg);
-    const float rcp_six = __frcp_rn(six_sg);
-    const ScaleTab stab{scale_tab, __frcp_rn(sg)};   // sg is a power of two
-
-    // stage the X0 tile (working orientation) in shared memory; a matrix with a
-    // non-finite entry is carried as all zeros (its output is zero)
+    // X0 of this tile (working orientation); a matrix with a non-finite entry is carried
+    // as all zeros (its output is zero).  Non-tall: thread f holds X0 row f / 16, columns
+    // 4 (f % 16) .. + 3, written to X straight from registers and staged as one float4.
+    // Tall: it holds G row f / 16 = X0 column f / 16, staged transposed.
     const int32_t rows_g = d.tall ? d.n : d.m, cols_g = d.tall ? d.m : d.n;
     const int32_t gr0 = d.tall ? j0 : i0, gc0 = d.tall ? i0 : j0;   // tile origin in G
     const float* gtile = d.G + (int64_t)gr0 * d.ldg + gc0;
+    float* Xt = reinterpret_cast<float*>(p.ws + L.X) + (int64_t)i0 * d.np + j0;
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass) {
       const int f = t + kEwThreads * pass;
@@ -444,29 +470,39 @@ __global__ void __launch_bounds__(kEwThreads) ns_preamble_kernel(const __grid_co
           if (gc0 + c4 + e < cols_g)
             v[e] = fminf(fmaxf(__fmul_rn(__ldg(gtile + (int64_t)line * d.ldg + c4 + e), inv), -tau), tau);
       }
-      // non-tall: line = row i of X; tall: line = row j of G = column j of X
+      if (!d.tall) {
+        const float4 v4 = make_float4(v[0], v[1], v[2], v[3]);
+        *reinterpret_cast<float4*>(tile + pre_off(line, c4)) = v4;
+        *reinterpret_cast<float4*>(Xt + line * d.np + c4) = v4;
+      } else {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if (!d.tall) tile[line][c4 + e] = v[e];
-        else tile[c4 + e][line] = v[e];
+        for (int e = 0; e < 4; ++e) tile[pre_off(c4 + e, line)] = v[e];
       }
     }
     __syncthreads();
-    float* Xt = reinterpret_cast<float*>(p.ws + L.X) + (int64_t)i0 * d.np + j0;
+    if (d.tall) {
 #pragma unroll
-    for (int pass = 0; pass < 4; ++pass) {
-      const int f = t + kEwThreads * pass;
-      const int r = f >> 4, c4 = (f & 15) * 4;
-      *reinterpret_cast<float4*>(Xt + r * d.np + c4) =
-          make_float4(tile[r][c4], tile[r][c4 + 1], tile[r][c4 + 2], tile[r][c4 + 3]);
+      for (int pass = 0; pass < 4; ++pass) {
+        const int f = t + kEwThreads * pass;
+        const int r = f >> 4, c4 = (f & 15) * 4;
+        *reinterpret_cast<float4*>(Xt + r * d.np + c4) = *reinterpret_cast<const float4*>(tile + pre_off(r, c4));
+      }
     }
     // two views; thread t owns one 16-element block of line t/4 (four blocks per line)
 #pragma unroll
     for (int view = 0; view < 2; ++view) {
       const int line = t >> 2, blk = t & 3;
       float v[16];
+      if (view == 0) {
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = view == 0 ? tile[line][blk * 16 + e] : tile[blk * 16 + e][line];
+        for (int k = 0; k < 4; ++k) {
+          const float4 x4 = *reinterpret_cast<const float4*>(tile + pre_off(line, blk * 16 + 4 * k));
+          v[4 * k] = x4.x; v[4 * k + 1] = x4.y; v[4 * k + 2] = x4.z; v[4 * k + 3] = x4.w;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = tile[pre_off(blk * 16 + e, line)];
+      }
       // view 0 is the Gram operand of iteration 0, view 1 the update operand
       if constexpr ((kOpts & kOptRht) != 0) rht16(v, view == 0 ? p.rht[0] : p.rht[2]);
       const QBlock16 q = quantize16<true, true, true, (kOpts & kOpt46) != 0>(v, sg, six_sg, rcp_six, stab);
