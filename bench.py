@@ -56,6 +56,30 @@ def parse_args():
     return ap.parse_args()
 
 
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Seed of the workload matrices of one rank: every rank runs the whole workload on
+    its own matrices (replicas; the matrices are independent, no collective)."""
+    return base_seed + 1000 * rank
+
+
+def max_over_ranks(v: float, world: int, device: str = "cuda") -> float:
+    """The largest value over all ranks (step times: the job is as slow as its slowest
+    rank).  Uses the default process group; `device` is "cuda" under NCCL, "cpu" under gloo."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world: int, units_per_rank: float, ms_step: float) -> float:
+    """Whole-job throughput: the units every rank processed per step over the slowest
+    rank's step time."""
+    return world * units_per_rank / (ms_step * 1e-3)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -295,21 +319,17 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def ranks_max(v: float) -> float:
+        return max_over_ranks(v, world, "cuda")
 
     w = WORKLOADS[args.workload]
     if args.op != "ns":
-        run_standalone(args, w, rank, world, local, barrier, max_over_ranks)
+        run_standalone(args, w, rank, world, local, barrier, ranks_max)
         if world > 1:
             dist.destroy_process_group()
         return
     K = w.K
-    Gs = matrices(w, device="cuda", seed=BASE_SEED + 1000 * rank)
+    Gs = matrices(w, device="cuda", seed=rank_seed(BASE_SEED, rank))
     outs = [torch.empty_like(G) for G in Gs]
     arr = F._descs(Gs, outs, w.coeffs)
     lib = F._lib.lib()
@@ -359,7 +379,7 @@ def main():
         torch.cuda.synchronize()
     barrier()
     F.check(F.device_status(ws), "device status after timed steps")
-    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    total_ms = ranks_max(t_start.elapsed_time(t_end))
     ms_step = total_ms / args.steps
 
     # per-phase kernel durations (CUDA events on the launching stream)
@@ -396,7 +416,7 @@ def main():
         if ent and ent.get("source_sha") == F._source_digest(files):
             roof["traffic"] = ent["bytes_per_launch"]
 
-    value = world * len(Gs) / (ms_step * 1e-3)
+    value = job_rate(world, len(Gs), ms_step)
     tflops = world * w.flops_algorithmic() / (ms_step * 1e-3) / 1e12
     phase_ms = {k: statistics.mean(v) * (1 if k in ("reduce", "preamble") else K) for k, v in per_kind.items()}
 
@@ -457,9 +477,9 @@ def main():
         torch.cuda.synchronize()
         barrier()
         F.check(F.device_status(ws), "device status after the end-to-end steps")
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
+        e2e_ms = ranks_max(e0.elapsed_time(e1)) / e2e_steps
         nbytes = sum(G.numel() * 4 for G in Gs)
-        e2e = {"value": world * len(Gs) / (e2e_ms * 1e-3), "unit": UNIT,
+        e2e = {"value": job_rate(world, len(Gs), e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
                "ms_per_step": e2e_ms,
                "pipeline": "copy-in, compute and copy-out of consecutive steps overlap on three "
@@ -499,7 +519,7 @@ def main():
         dist.destroy_process_group()
 
 
-def run_standalone(args, w, rank, world, local, barrier, max_over_ranks):
+def run_standalone(args, w, rank, world, local, barrier, ranks_max):
     """--op quantize / dequantize: one step = one fs4_nvfp4_quantize (or _dequantize)
     call per matrix of the workload, row axis, outputs preallocated."""
     import torch
@@ -509,7 +529,7 @@ def run_standalone(args, w, rank, world, local, barrier, max_over_ranks):
     lib = F._lib.lib()
     tiled = args.layout == "tiled"
     flags = F.FS4_LAYOUT_TILED if tiled else 0
-    Gs = matrices(w, device="cuda", seed=BASE_SEED + 1000 * rank)
+    Gs = matrices(w, device="cuda", seed=rank_seed(BASE_SEED, rank))
     stream = torch.cuda.current_stream()
     qws_bytes = int(lib.fs4_nvfp4_quantize_workspace_size())
     bufs = []
@@ -569,10 +589,10 @@ def run_standalone(args, w, rank, world, local, barrier, max_over_ranks):
                 call_ev[s][i + 1].record(stream)
         torch.cuda.synchronize()
     barrier()
-    total_ms = max_over_ranks(call_ev[0][0].elapsed_time(call_ev[-1][-1]))
+    total_ms = ranks_max(call_ev[0][0].elapsed_time(call_ev[-1][-1]))
     ms_step = total_ms / args.steps
     elems = sum(G.numel() for G in Gs)
-    value = world * elems * QD_BYTES / (ms_step * 1e-3) / 1e9
+    value = job_rate(world, elems * QD_BYTES / 1e9, ms_step)
 
     # roofline of one call (the amax and quantise launches of fs4_nvfp4_quantize, or
     # the one dequantise launch), averaged over every call of the timed steps
@@ -651,10 +671,10 @@ def run_standalone(args, w, rank, world, local, barrier, max_over_ranks):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
+        e2e_ms = ranks_max(e0.elapsed_time(e1)) / e2e_steps
         nb_fp32 = elems * 4
         nb_q = sum(b["codes"].numel() + b["scales"].numel() + 4 for b in bufs)
-        e2e = {"value": world * elems * QD_BYTES / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e2e = {"value": job_rate(world, elems * QD_BYTES / 1e9, e2e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": nb_fp32 if args.op == "quantize" else nb_q,
                "d2h_bytes_per_step": nb_q if args.op == "quantize" else nb_fp32,
                "ms_per_step": e2e_ms,
