@@ -86,3 +86,42 @@ def test_full_size_batched_step_properties(fs4):
     want = R.root_ns(Gs[i].cpu().numpy(), w.K, *w.coeffs[i], clip_k=w.clip_k)
     eo, eg = R.orthogonality_error(want), R.orthogonality_error(got)
     assert abs(eg - eo) <= 0.1 * eo
+
+
+def test_full_size_first_iteration_per_shape_class(fs4):
+    """One complete iteration (GramX, GramA, Update) inside the full 3b_4blocks_gauss
+    batched call (bench.py's launch configuration), stopped after the first update:
+    X_1 of one matrix of each shape class (3072^2, tall 8192 x 3072, wide 3072 x 8192)
+    against the oracle's NVFP4 iteration from the same X_0.  One step is not chaotic,
+    so the relative Frobenius error is held to 2e-2."""
+    w = WORKLOADS["3b_4blocks_gauss"]
+    Gs = matrices(w, device="cuda", seed=BASE_SEED)
+    _, ws = _run(fs4, Gs, w, flags=fs4.stop_after(3))
+    shapes = [tuple(G.shape) for G in Gs]
+    picks = sorted({s: i for i, s in enumerate(shapes)}.values())
+    assert len(picks) == 3
+    for i in picks:
+        lay = fs4.ns_layout(shapes, i)
+        X0, _, _, _ = R.normalise_and_clip(working(Gs[i].cpu().numpy()), w.clip_k)
+        m, n = X0.shape
+        want = R.ns_iterations_nvfp4(X0, 1, *w.coeffs[i]).astype(np.float64)
+        Xg = ws[lay.X:lay.X + 4 * lay.mp * lay.np].cpu().numpy().view(np.float32)
+        got = Xg.reshape(lay.mp, lay.np)[:m, :n].astype(np.float64)
+        err = np.linalg.norm(got - want) / np.linalg.norm(want)
+        assert err <= 2e-2, (shapes[i], err)
+
+
+@pytest.mark.parametrize("axis", [0, 1])
+def test_full_size_standalone_quantise_bit_exact(fs4, axis):
+    """fs4_nvfp4_quantize on a whole 8192 x 3072 workload matrix (the bench's --op
+    quantize call), every code and scale against the oracle."""
+    w = WORKLOADS["3b_1block_gauss"]
+    G = matrices(w, device="cuda", seed=BASE_SEED)[4]
+    assert tuple(G.shape) == (8192, 3072)
+    x = G.cpu().numpy()
+    want_c, want_s, want_g = Q.quantize_rows(x) if axis == 0 else Q.quantize_cols(x)
+    c, s, g = fs4.quantize(G, axis=axis)
+    torch.cuda.synchronize()
+    assert np.float32(g.cpu().numpy()[0]) == want_g
+    assert np.array_equal(s.cpu().numpy(), want_s)
+    assert np.array_equal(c.cpu().numpy(), want_c)
