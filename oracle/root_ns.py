@@ -15,13 +15,19 @@ Source: "Full-Stack FP4" (arXiv 2607.04422).
         qX_k  = Q1x16(X_k),            A_k = qX_k qX_k^T
         qA_k  = Q1x16(A_k),  qA16_k = Q16x1(A_k),  B_k = b A_k + c qA_k qA16_k
         qB_k  = Q1x16(B_k),  qX16_k = Q16x1(X_k),  X_{k+1} = a X_k + qB_k qX16_k
-  * Section 3.4 also clips outliers before the iteration; the clip used here
-    is a hard clamp at clip_k * RMS of the normalised matrix.
+  * Section 3.4 also clips outliers before the iteration ("p99 outlier clipping";
+    Table 8: "Root quantile ratio 0.99").  Two clip rules are provided: a hard
+    clamp at clip_k * RMS of the normalised matrix (the default), and a hard clamp
+    at the q-quantile of |X_0| (clip_quantile = q).
 
 Readings taken where the pages are silent (each is listed in the design doc):
   * Frobenius normalisation X_0 = G / (||G||_F + eps), eps = 1e-7, ||G||_F
     accumulated in float64; inv = fp32(1 / (||G||_F + eps)) and X_0 = fp32(G * inv).
   * Clip: tau = fp32(clip_k * ||G||_F * inv / sqrt(m n)), X_0 = clamp(X_0, -tau, tau).
+  * Quantile clip: tau = the nearest-rank q-quantile of |X_0|, i.e. its k-th smallest
+    entry with k = ceil(fl64(q) * N) (1-based, clamped to [1, N]; N = m n; q is the
+    FP32 value the caller passes and the product is one IEEE float64 multiply), then
+    X_0 = clamp(X_0, -tau, tau).
   * Iterates X_k, A_k and B_k are FP32 tensors (the precision the quantiser
     reads); every matrix product is taken in float64 on dequantised operands
     and rounded once to FP32.  A_k is made exactly symmetric (upper triangle
@@ -38,15 +44,35 @@ from . import nvfp4
 NS_EPS = 1e-7
 
 
-def normalise_and_clip(X: np.ndarray, clip_k: float | None, eps: float = NS_EPS):
-    """FP32 X_0 = clamp(fp32(X * inv), +-tau).  Returns (X0, inv, tau, norm)."""
+def quantile_rank(q: float, N: int) -> int:
+    """1-based rank of the nearest-rank q-quantile of N values: ceil(fl64(q32) * N),
+    clamped to [1, N] (q32 = the FP32 value of q)."""
+    k = int(np.ceil(np.float64(np.float32(q)) * np.float64(N)))
+    return min(max(k, 1), N)
+
+
+def quantile_clip_threshold(X0: np.ndarray, q: float) -> np.float32:
+    """The nearest-rank q-quantile of |X0| (Section 3.4 "p99 outlier clipping", Table 8
+    "Root quantile ratio 0.99"): its k-th smallest entry, k = quantile_rank(q, N)."""
+    a = np.abs(np.asarray(X0, dtype=np.float32)).ravel()
+    k = quantile_rank(q, a.size)
+    return np.float32(np.partition(a, k - 1)[k - 1])
+
+
+def normalise_and_clip(X: np.ndarray, clip_k: float | None, eps: float = NS_EPS,
+                       clip_quantile: float | None = None):
+    """FP32 X_0 = clamp(fp32(X * inv), +-tau).  Returns (X0, inv, tau, norm).
+    clip_quantile = q: tau is the q-quantile of |fp32(X * inv)| instead of clip_k * RMS."""
     X = np.asarray(X, dtype=np.float32)
     m, n = X.shape
     norm = float(np.sqrt(np.sum(X.astype(np.float64) ** 2)))
     inv = np.float32(1.0 / (norm + eps))
     X0 = X * inv
     tau = None
-    if clip_k is not None and clip_k > 0:
+    if clip_quantile is not None:
+        tau = quantile_clip_threshold(X0, clip_quantile)
+        X0 = np.clip(X0, -tau, tau).astype(np.float32)
+    elif clip_k is not None and clip_k > 0:
         tau = np.float32(clip_k * norm * float(inv) / np.sqrt(float(m) * float(n)))
         X0 = np.clip(X0, -tau, tau).astype(np.float32)
     return X0, inv, tau, norm
@@ -103,7 +129,8 @@ def ns_iterations_f64(X0, K, a, b, c):
 
 
 def root_ns(G, K=5, a=3.4445, b=-4.7750, c=2.0315, clip_k=3.0, eps=NS_EPS,
-            quantized=True, mode="pow2", trace=None, rht_masks=None, adaptive46=False):
+            quantized=True, mode="pow2", trace=None, rht_masks=None, adaptive46=False,
+            clip_quantile=None):
     """Normalise, clip and run K Newton-Schulz iterations on the FP32 matrix G.
 
     quantized=True: the NVFP4 route of Section 3.4 (FP32 result).
@@ -118,7 +145,8 @@ def root_ns(G, K=5, a=3.4445, b=-4.7750, c=2.0315, clip_k=3.0, eps=NS_EPS,
     tall = G.shape[0] > G.shape[1]
     X = G.T if tall else G
     if quantized:
-        X0, inv, tau, norm = normalise_and_clip(X.astype(np.float32), clip_k, eps)
+        X0, inv, tau, norm = normalise_and_clip(X.astype(np.float32), clip_k, eps,
+                                                clip_quantile=clip_quantile)
         if trace is not None:
             trace.append(dict(X0=X0, inv=inv, tau=tau, norm=norm))
         Y = ns_iterations_nvfp4(X0, K, a, b, c, mode=mode, trace=trace, rht_masks=rht_masks,
@@ -127,7 +155,12 @@ def root_ns(G, K=5, a=3.4445, b=-4.7750, c=2.0315, clip_k=3.0, eps=NS_EPS,
         X64 = np.asarray(X, dtype=np.float64)
         norm = float(np.sqrt(np.sum(X64 ** 2)))
         X0 = X64 / (norm + eps)
-        if clip_k is not None and clip_k > 0:
+        if clip_quantile is not None:
+            a = np.abs(X0).ravel()
+            k = quantile_rank(clip_quantile, a.size)
+            tau = np.partition(a, k - 1)[k - 1]
+            X0 = np.clip(X0, -tau, tau)
+        elif clip_k is not None and clip_k > 0:
             tau = clip_k * np.sqrt(np.sum(X0 ** 2)) / np.sqrt(X0.size)
             X0 = np.clip(X0, -tau, tau)
         Y = ns_iterations_f64(X0, K, a, b, c)
