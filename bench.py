@@ -50,6 +50,9 @@ def parse_args():
                          "NVFP4 calls over every matrix of the workload (row axis)")
     ap.add_argument("--layout", default="plain", choices=["plain", "tiled"],
                     help="NVFP4 layout of --op quantize / dequantize")
+    ap.add_argument("--clip", default="rms", choices=["rms", "p99"],
+                    help="clip rule of the preamble: 3 x RMS (default) or the 0.99 quantile of "
+                         "|X_0| (Section 3.4 p99 outlier clipping, FS4_NS_CLIP_QUANTILE)")
     ap.add_argument("--quant", default="plain", choices=["plain", "rht46", "rht", "a46"],
                     help="quantiser of the step: plain NVFP4 (default) or the Section 3.4 options "
                          "(random Hadamard transform with fresh seeded sign masks, adaptive 4/6)")
@@ -340,6 +343,10 @@ def main():
 
     qflags = {"plain": 0, "rht46": F.FS4_NS_RHT | F.FS4_NS_ADAPTIVE46, "rht": F.FS4_NS_RHT,
               "a46": F.FS4_NS_ADAPTIVE46}[args.quant]
+    clip_arg = w.clip_k
+    if args.clip == "p99":
+        qflags |= F.FS4_NS_CLIP_QUANTILE
+        clip_arg = 0.99
     mask_rng = np.random.default_rng(BASE_SEED + 7)
 
     def call(events=None):
@@ -348,11 +355,11 @@ def main():
             masks = (ctypes.c_uint16 * (3 * K))(*[int(v) for v in mask_rng.integers(0, 1 << 16, 3 * K)])
         mptr = ctypes.cast(masks, ctypes.c_void_p) if masks is not None else None
         if events is None:
-            st = lib.fs4_root_ns_batched_ex(len(Gs), arr, K, w.clip_k, qflags, mptr, ws.data_ptr(),
+            st = lib.fs4_root_ns_batched_ex(len(Gs), arr, K, clip_arg, qflags, mptr, ws.data_ptr(),
                                             need, stream.cuda_stream)
         else:
             ev_arr = (F._lib.c_vp * n_ev)(*[e.cuda_event for e in events])
-            st = lib.fs4_root_ns_batched_timed(len(Gs), arr, K, w.clip_k, qflags, mptr, ws.data_ptr(),
+            st = lib.fs4_root_ns_batched_timed(len(Gs), arr, K, clip_arg, qflags, mptr, ws.data_ptr(),
                                                need, stream.cuda_stream, ev_arr, n_ev)
         F.check(st, "fs4_root_ns_batched")
 
@@ -453,7 +460,8 @@ def main():
                      if qflags & F.FS4_NS_RHT else None)
             F.root_ns_batched(dev_in[b], K=K, coeffs=w.coeffs, clip_k=w.clip_k, outs=dev_out[b],
                               workspace=ws, stream=stream, rht_masks=masks,
-                              adaptive46=bool(qflags & F.FS4_NS_ADAPTIVE46))
+                              adaptive46=bool(qflags & F.FS4_NS_ADAPTIVE46),
+                              clip_quantile=0.99 if args.clip == "p99" else None)
             ev["done"][b].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev["done"][b])
@@ -497,7 +505,8 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3/16) products, fp32 accumulate",
             "data": "synthetic",
             "config": {"workload": w.name, "matrices": len(Gs), "shapes": sorted(set(map(tuple, w.shapes))),
-                       "K": K, "coeffs": "Muon (3.4445, -4.7750, 2.0315)", "clip": "3 x RMS",
+                       "K": K, "coeffs": "Muon (3.4445, -4.7750, 2.0315)",
+                       "clip": "3 x RMS" if args.clip == "rms" else "0.99 quantile of |X_0| (nearest rank)",
                        "quantiser": {"plain": "NVFP4 RTN (H = I, M = 6)",
                                      "rht46": "NVFP4 RTN with H16^r (fresh signs per step) and adaptive 4/6",
                                      "rht": "NVFP4 RTN with H16^r (fresh signs per step)",
@@ -511,7 +520,7 @@ def main():
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": args.steps * (2 + 6 * K),
+            "gpu_launches": args.steps * (2 + 6 * K + (3 if args.clip == "p99" else 0)),
             "clocks": sampler.summary(),
         }
         print(json.dumps(line), flush=True)

@@ -103,6 +103,17 @@ enum {
 #define FS4_NS_ADAPTIVE46 (1u << 3)
 #define FS4_NS_RHT (1u << 2)
 
+/* Quantile clip of the Newton-Schulz step (Section 3.4: "p99 outlier clipping";
+ * Table 8: "Root quantile ratio 0.99").  With this flag clip_k is the quantile
+ * ratio q, 0 < q <= 1 (else FS4_ERR_INVALID_ARG), and tau is the nearest-rank
+ * q-quantile of |X_0|: the k-th smallest |x| of the normalised matrix with
+ * k = ceil(q * m * n) (q widened to double, one IEEE double multiply, k clamped to
+ * [1, m n]).  X_0 is clamped to [-tau, tau] as with the default rule.  The
+ * selection is exact (three radix digits of the 31-bit magnitude key) and adds
+ * three launches after the reduction; it uses the matrix's X buffer as scratch
+ * before the preamble writes X_0 there. */
+#define FS4_NS_CLIP_QUANTILE (1u << 4)
+
 /* Test-only flag for fs4_root_ns / fs4_root_ns_batched (no counterpart in the
  * paper): the MMA issuer of the first Gram product waits on a barrier that
  * nothing arrives on.  The bounded wait gives up after about 2 s, records the
@@ -188,7 +199,8 @@ size_t fs4_root_ns_batched_workspace_size(int32_t count, const fs4_ns_desc* desc
 
 /* Direct NVFP4 Newton-Schulz step (Section 3.4) on one FP32 momentum matrix.
  *   X_0 = clamp(G / (||G||_F + 1e-7), +-tau), tau = clip_k * RMS of the
- *   normalised matrix (clip_k <= 0 disables the clamp); then K iterations of
+ *   normalised matrix (clip_k <= 0 disables the clamp), or with
+ *   FS4_NS_CLIP_QUANTILE the clip_k-quantile of |X_0|; then K iterations of
  *   qX = Q1x16(X), A = qX qX^T, B = b A + c Q1x16(A) Q16x1(A),
  *   X <- a X + Q1x16(B) Q16x1(X).  A tall matrix (m > n) is processed as its
  *   transpose so the Gram matrix is min(m,n) square; out has G's shape.

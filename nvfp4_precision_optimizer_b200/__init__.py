@@ -13,7 +13,7 @@ from typing import Sequence
 import torch
 
 from . import _lib
-from ._lib import (FS4_AXIS_COL, FS4_AXIS_ROW, FS4_LAYOUT_TILED, FS4_NS_ADAPTIVE46, FS4_NS_RHT,
+from ._lib import (FS4_AXIS_COL, FS4_AXIS_ROW, FS4_LAYOUT_TILED, FS4_NS_ADAPTIVE46, FS4_NS_CLIP_QUANTILE, FS4_NS_RHT,
                    FS4_SG_AMAX, FS4_TEST_STALL, Fs4Error, NsDesc, NsLayout, check, stop_after)
 
 MUON_COEFFS = (3.4445, -4.7750, 2.0315)
@@ -22,7 +22,7 @@ __all__ = [
     "quantize", "dequantize", "gemm", "root_ns", "root_ns_batched", "ns_workspace_size",
     "ns_batched_workspace_size", "ns_layout", "device_status", "tiled_shape", "Fs4Error",
     "MUON_COEFFS", "stop_after", "FS4_AXIS_ROW", "FS4_AXIS_COL", "FS4_TEST_STALL",
-    "FS4_NS_RHT", "FS4_NS_ADAPTIVE46",
+    "FS4_NS_RHT", "FS4_NS_ADAPTIVE46", "FS4_NS_CLIP_QUANTILE",
 ]
 
 
@@ -153,10 +153,16 @@ def _masks(rht_masks, K):
 def root_ns(G: torch.Tensor, K: int = 5, a: float = MUON_COEFFS[0], b: float = MUON_COEFFS[1],
             c: float = MUON_COEFFS[2], clip_k: float = 3.0, out: torch.Tensor | None = None,
             workspace: torch.Tensor | None = None, flags: int = 0, stream=None,
-            rht_masks=None, adaptive46: bool = False) -> torch.Tensor:
+            rht_masks=None, adaptive46: bool = False,
+            clip_quantile: float | None = None) -> torch.Tensor:
     """Direct NVFP4 Newton-Schulz step on one FP32 matrix (fs4_root_ns; with
-    rht_masks (3K sign masks of H16^r) or adaptive46, fs4_root_ns_batched_ex)."""
+    rht_masks (3K sign masks of H16^r) or adaptive46, fs4_root_ns_batched_ex).
+    clip_quantile = q clips at the q-quantile of |X_0| (FS4_NS_CLIP_QUANTILE)
+    instead of clip_k * RMS."""
     _check_f32_matrix(G, "G")
+    if clip_quantile is not None:
+        flags |= FS4_NS_CLIP_QUANTILE
+        clip_k = clip_quantile
     if out is None:
         out = torch.empty_like(G)
     m, n = G.shape
@@ -176,11 +182,16 @@ def root_ns(G: torch.Tensor, K: int = 5, a: float = MUON_COEFFS[0], b: float = M
 def root_ns_batched(Gs: Sequence[torch.Tensor], K: int = 5, coeffs=None, clip_k: float = 3.0,
                     outs: Sequence[torch.Tensor] | None = None,
                     workspace: torch.Tensor | None = None, flags: int = 0, stream=None,
-                    rht_masks=None, adaptive46: bool = False):
+                    rht_masks=None, adaptive46: bool = False,
+                    clip_quantile: float | None = None):
     """Direct NVFP4 Newton-Schulz step on a list of matrices in one grouped call
     (fs4_root_ns_batched); coeffs is a list of per-matrix (a, b, c).  rht_masks
     (3K sign masks of H16^r) and adaptive46 select the Section 3.4 quantiser
-    options (fs4_root_ns_batched_ex)."""
+    options (fs4_root_ns_batched_ex); clip_quantile = q clips at the q-quantile
+    of |X_0| (FS4_NS_CLIP_QUANTILE) instead of clip_k * RMS."""
+    if clip_quantile is not None:
+        flags |= FS4_NS_CLIP_QUANTILE
+        clip_k = clip_quantile
     for G in Gs:
         _check_f32_matrix(G, "G")
     if coeffs is None:

@@ -23,7 +23,7 @@ STATUS_NAMES = {
 FS4_AXIS_ROW, FS4_AXIS_COL = 0, 1
 FS4_SG_AMAX, FS4_LAYOUT_TILED = 1, 2
 FS4_TEST_STALL = 1 << 30   # test only: a device wait that runs out (see include/fs4.h)
-FS4_NS_RHT, FS4_NS_ADAPTIVE46 = 1 << 2, 1 << 3
+FS4_NS_RHT, FS4_NS_ADAPTIVE46, FS4_NS_CLIP_QUANTILE = 1 << 2, 1 << 3, 1 << 4
 MAX_BATCH = 224
 MAX_ITERS = 32
 

@@ -152,7 +152,8 @@ fs4_status run_ns(const Plan& pl, int32_t K, float clip_k, uint32_t flags, const
   p.clip_k = clip_k;
   p.status = reinterpret_cast<uint32_t*>(ws);
   p.ws = ws;
-  p.opts = ((flags & FS4_NS_RHT) ? kOptRht : 0u) | ((flags & FS4_NS_ADAPTIVE46) ? kOpt46 : 0u);
+  p.opts = ((flags & FS4_NS_RHT) ? kOptRht : 0u) | ((flags & FS4_NS_ADAPTIVE46) ? kOpt46 : 0u) |
+           ((flags & FS4_NS_CLIP_QUANTILE) ? kOptQuantile : 0u);
   if (flags & FS4_NS_RHT)
     for (int i = 0; i < 3 * K; ++i) p.rht[i] = rht_masks[i];
   std::memcpy(p.mat, pl.mat, sizeof(MatDesc) * pl.count);
@@ -162,6 +163,8 @@ fs4_status run_ns(const Plan& pl, int32_t K, float clip_k, uint32_t flags, const
   if (e != cudaSuccess) return FS4_ERR_CUDA;
   if (!fill_prefix(p, pl.units_reduce)) return FS4_ERR_SHAPE;
   if ((e = launch_ns_reduce(p, st, num_sms)) != cudaSuccess) return FS4_ERR_CUDA;
+  if ((p.opts & kOptQuantile) && (e = launch_ns_quantile(p, st, num_sms)) != cudaSuccess)
+    return FS4_ERR_CUDA;
   if (!mark()) return FS4_ERR_CUDA;
   if (!fill_prefix(p, pl.units_pre)) return FS4_ERR_SHAPE;
   if ((e = launch_ns_preamble(p, st, num_sms)) != cudaSuccess) return FS4_ERR_CUDA;
@@ -277,8 +280,10 @@ static fs4_status batched_impl(int32_t count, const fs4_ns_desc* descs, int32_t 
                                int32_t n_events) {
   if (K < 1 || K > FS4_MAX_ITERS) return FS4_ERR_SHAPE;
   if (!std::isfinite(clip_k)) return FS4_ERR_INVALID_ARG;
-  if (flags & ~(uint32_t)(0xFF00u | FS4_TEST_STALL | FS4_NS_RHT | FS4_NS_ADAPTIVE46))
+  if (flags & ~(uint32_t)(0xFF00u | FS4_TEST_STALL | FS4_NS_RHT | FS4_NS_ADAPTIVE46 |
+                          FS4_NS_CLIP_QUANTILE))
     return FS4_ERR_INVALID_ARG;
+  if ((flags & FS4_NS_CLIP_QUANTILE) && !(clip_k > 0.0f && clip_k <= 1.0f)) return FS4_ERR_INVALID_ARG;
   if ((flags & FS4_NS_RHT) && !rht_masks) return FS4_ERR_INVALID_ARG;
   static thread_local Plan pl;
   const fs4_status s = make_plan(count, descs, &pl);

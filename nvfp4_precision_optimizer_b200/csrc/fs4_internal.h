@@ -24,7 +24,11 @@ struct NsState {
   uint32_t nonfinite;      // G holds NaN or Inf
   uint32_t done[8];        // finished work units per phase kind (preamble, G1, G2, G3, reduce)
   float inv0, tau0;        // fp32(1 / (||G|| + eps)) and the clip threshold (set after the reduction)
-  uint32_t pad0[50];
+  uint32_t q_bin1;         // quantile clip: top 11 key bits of the selected |G| (select pass 1)
+  uint32_t q_pad;
+  uint64_t q_rank1;        // quantile clip: rank of the selected key within that bin (1-based)
+  unsigned long long q_count;   // quantile clip: candidates gathered (keys in bin q_bin1)
+  uint32_t pad0[44];
   float sg[192];           // tensor scales: X_k at [k], A_k at [64+k], B_k at [128+k]
   float u_rowX[64];        // max_i sum_j deq(qX_k)_ij^2
   float u_colX[64];        // max_j sum_i deq(qX16_k)_ij^2
@@ -36,10 +40,16 @@ struct NsState {
 static_assert(sizeof(NsState) == 4096, "NsState must stay 4 KB");
 constexpr int kSgX = 0, kSgA = 64, kSgB = 128;
 
+// Quantile clip: the 31-bit key of |g| (its float bits without the sign) is selected
+// in three digits of 11, 11 and 9 bits; the first digit's histogram lives in the
+// zeroed state block.
+constexpr int kQBins1 = 2048, kQBins2 = 2048, kQBins3 = 512;
+
 // Offsets (bytes, from the workspace base) of one matrix's buffers.
 struct MatLayout {
   int64_t state;                                 // NsState
   int64_t rowsumX, colsumX, rowsumA, rowsumB;    // float [mp], [np], [mp], [mp]
+  int64_t qhist;                                 // uint32 [kQBins1] (quantile clip)
   int64_t X, A;                                  // float [mp*np], [mp*mp]
   int64_t qX[2], sX[2], qXT[2], sXT[2];          // TILED codes/scales of X (mp x np), X^T (np x mp)
   int64_t qA, sA, qB, sB;                        // TILED codes/scales of A, B (mp x mp)
@@ -49,7 +59,7 @@ __host__ __device__ inline int64_t align_up(int64_t v, int64_t a) { return (v + 
 
 // Bytes of the zero-initialised block (state + sums) of an mp x np matrix.
 __host__ __device__ inline int64_t state_block_bytes(int64_t mp, int64_t np) {
-  return align_up(4096 + 4 * (3 * mp + np), 256);
+  return align_up(4096 + 4 * (3 * mp + np) + 4 * kQBins1, 256);
 }
 
 // Bytes of the large buffers of an mp x np matrix.
@@ -66,6 +76,7 @@ __host__ __device__ inline MatLayout mat_layout(int64_t mp, int64_t np, int64_t 
   L.colsumX = L.rowsumX + 4 * mp;
   L.rowsumA = L.colsumX + 4 * np;
   L.rowsumB = L.rowsumA + 4 * mp;
+  L.qhist = L.rowsumB + 4 * mp;
   const int64_t xn = mp * np, aa = mp * mp;
   int64_t o = big_off;
   L.X = o; o += 4 * xn;
@@ -91,14 +102,15 @@ struct MatDesc {
 
 // Kernel parameters of one Newton-Schulz phase over a batch of matrices.
 constexpr uint32_t kOptRht = 1u, kOpt46 = 2u;   // NsParams::opts
+constexpr uint32_t kOptQuantile = 4u;            // clip at the clip_k-quantile of |X_0|
 
 struct NsParams {
   int32_t count;
   int32_t iter;            // k of the current iteration
   int32_t last;            // 1 on the final update product (writes `out`)
   int32_t stall;           // test only: the MMA issuer waits on a barrier nothing arrives on
-  uint32_t opts;           // kOptRht | kOpt46
-  float clip_k;
+  uint32_t opts;           // kOptRht | kOpt46 | kOptQuantile
+  float clip_k;            // clip_k * RMS, or with kOptQuantile the quantile ratio q in (0, 1]
   uint32_t* status;
   uint8_t* ws;             // workspace base
   uint16_t rht[3 * kMaxIters];   // H16^r sign mask of product j of iteration k at 3k + j
@@ -128,6 +140,7 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const
                               int64_t rows, int64_t cols, float* y, int64_t ld, uint32_t flags,
                               cudaStream_t st, int num_sms);
 cudaError_t launch_ns_reduce(const NsParams& p, cudaStream_t st, int num_sms);
+cudaError_t launch_ns_quantile(const NsParams& p, cudaStream_t st, int num_sms);
 cudaError_t launch_ns_preamble(const NsParams& p, cudaStream_t st, int num_sms);
 cudaError_t launch_gemm_plain(const GemmPlainArgs& a, cudaStream_t st, int num_sms);
 cudaError_t launch_gemm_ns(Epi epi, const NsParams& p, cudaStream_t st, int num_sms);

@@ -281,15 +281,27 @@ __device__ __forceinline__ NsState* state_of(const NsParams& p, const MatDesc& d
   return reinterpret_cast<NsState*>(p.ws + d.state_off);
 }
 
+// The 31-bit key of |g|: its float bits without the sign (non-negative floats order
+// like their bit patterns).
+__device__ __forceinline__ uint32_t abs_key(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
+
 // Sum of G^2 (float64), max |G| and a non-finite flag per matrix; work unit =
 // 16 rows of one matrix in the caller's orientation.  The last CTA to finish a
 // matrix derives its normalisation and clip scalars and the tensor scale of X_0
 // (Section 3.4: normalise, clip, quantise), so the preamble only reads them.
+// kHist (quantile clip): also a histogram of the top 11 bits of every |g| key,
+// accumulated per unit in shared memory and added to the matrix's histogram.
+template <bool kHist>
 __global__ void __launch_bounds__(kEwThreads) ns_reduce_kernel(const __grid_constant__ NsParams p) {
   __shared__ float redf[kEwThreads / 32];
   __shared__ double redd[kEwThreads / 32];
+  __shared__ uint32_t hist[kHist ? kQBins1 : 1];
   const int32_t total = p.prefix[p.count];
   for (int32_t u = blockIdx.x; u < total; u += gridDim.x) {
+    if constexpr (kHist) {
+      for (int b = threadIdx.x; b < kQBins1; b += kEwThreads) hist[b] = 0u;
+      __syncthreads();
+    }
     const int mi = owner_of(p.prefix, p.count, u);
     const MatDesc& d = p.mat[mi];
     const int64_t rows0 = d.tall ? d.n : d.m, cols0 = d.tall ? d.m : d.n;
@@ -309,6 +321,7 @@ __global__ void __launch_bounds__(kEwThreads) ns_reduce_kernel(const __grid_cons
             bad |= !is_finite_bits(vv[e]);
             mx = fmaxf(mx, fabsf(vv[e]));
             s += (double)vv[e] * (double)vv[e];
+            if constexpr (kHist) atomicAdd(&hist[abs_key(vv[e]) >> 20], 1u);
           }
         }
       } else {
@@ -317,11 +330,18 @@ __global__ void __launch_bounds__(kEwThreads) ns_reduce_kernel(const __grid_cons
           bad |= !is_finite_bits(v);
           mx = fmaxf(mx, fabsf(v));
           s += (double)v * (double)v;
+          if constexpr (kHist) atomicAdd(&hist[abs_key(v) >> 20], 1u);
         }
       }
     }
     NsState* st = state_of(p, d);
-    const bool any_bad = __syncthreads_or(bad);
+    const bool any_bad = __syncthreads_or(bad);   // also orders the histogram updates
+    if constexpr (kHist) {
+      uint32_t* gh = reinterpret_cast<uint32_t*>(
+          p.ws + mat_layout(d.mp, d.np, d.state_off, d.big_off).qhist);
+      for (int b = threadIdx.x; b < kQBins1; b += kEwThreads)
+        if (hist[b] != 0u) atomicAdd(&gh[b], hist[b]);
+    }
     s = warp_sum(s);
     const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
     if (l == 0) redd[w] = s;
@@ -342,8 +362,8 @@ __global__ void __launch_bounds__(kEwThreads) ns_reduce_kernel(const __grid_cons
         const bool dead = __ldcg(&st->nonfinite) != 0u;
         const double norm = sqrt(__ldcg(&st->sumsq));
         const float inv = dead ? 0.0f : (float)(1.0 / (norm + 1e-7));
-        float tau = FLT_MAX;
-        if (p.clip_k > 0.0f)
+        float tau = FLT_MAX;   // the quantile clip sets it after the selection
+        if (p.clip_k > 0.0f && !(p.opts & kOptQuantile))
           tau = (float)((double)p.clip_k * norm * (double)inv / sqrt((double)d.m * (double)d.n));
         const float amaxG = __uint_as_float(__ldcg(&st->amaxG));
         const float amax0 = dead ? 0.0f : fminf(__fmul_rn(amaxG, inv), tau);
@@ -357,6 +377,209 @@ __global__ void __launch_bounds__(kEwThreads) ns_reduce_kernel(const __grid_cons
       }
     }
     __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ quantile clip
+// tau = the nearest-rank q-quantile of |X_0| = fp32(|G|_(k) * inv), |G|_(k) the k-th
+// smallest |g| with k = ceil(fl64(q) * N) ("Full-Stack FP4" Section 3.4, "p99 outlier
+// clipping"; fp32(. * inv) is monotone, so the order statistic of |X_0| is that of |G|
+// scaled).  |G|_(k) is selected exactly on its 31-bit key, digit by digit: 11 bits from
+// the reduction's histogram, then the keys of that bin are gathered and the last 11 + 9
+// bits selected among them by one CTA per matrix.
+
+// 1-based rank of the quantile (IEEE double, as the oracle computes it).
+__device__ __forceinline__ uint64_t quantile_rank(float q, int64_t N) {
+  double k = ceil((double)q * (double)N);
+  if (k < 1.0) k = 1.0;
+  if (k > (double)N) k = (double)N;
+  return (uint64_t)k;
+}
+
+// Block-wide (kT threads): the bin b of `h` (nbins and kT powers of two) holding the
+// element of rank k (1-based; sum(h) >= k), and the rank of that element within bin b.
+// Result valid in every thread.
+template <int kT>
+__device__ void find_rank_bin(const uint32_t* h, int nbins, uint64_t k, int* bin_out,
+                              uint64_t* rank_out) {
+  __shared__ unsigned long long part[kT];
+  __shared__ int s_bin;
+  __shared__ unsigned long long s_rank;
+  const int per = nbins >= kT ? nbins / kT : 1, t = threadIdx.x;
+  const bool has = t * per < nbins;
+  unsigned long long sum = 0;
+  if (has)
+    for (int i = 0; i < per; ++i) sum += h[t * per + i];
+  part[t] = sum;
+  if (t == 0) { s_bin = nbins - 1; s_rank = 1; }
+  __syncthreads();
+  // inclusive scan of the per-thread sums (Hillis-Steele over kT entries)
+  for (int off = 1; off < kT; off <<= 1) {
+    const unsigned long long v = t >= off ? part[t - off] : 0ull;
+    __syncthreads();
+    part[t] += v;
+    __syncthreads();
+  }
+  const unsigned long long before = t > 0 ? part[t - 1] : 0ull;
+  if (has && before < k && k <= part[t]) {
+    unsigned long long acc = before;
+    for (int i = 0; i < per; ++i) {
+      const uint32_t c = h[t * per + i];
+      if (k <= acc + c) { s_bin = t * per + i; s_rank = k - acc; break; }
+      acc += c;
+    }
+  }
+  __syncthreads();
+  *bin_out = s_bin;
+  *rank_out = s_rank;
+  __syncthreads();
+}
+
+// One CTA per matrix: the first digit of the selected key and the rank within its bin.
+__global__ void __launch_bounds__(kEwThreads) ns_quantile_select1_kernel(const __grid_constant__ NsParams p) {
+  const MatDesc& d = p.mat[blockIdx.x];
+  NsState* st = state_of(p, d);
+  if (__ldcg(&st->nonfinite) != 0u) return;
+  const uint32_t* gh = reinterpret_cast<const uint32_t*>(p.ws + mat_layout(d.mp, d.np, d.state_off, d.big_off).qhist);
+  __shared__ uint32_t h[kQBins1];
+  for (int b = threadIdx.x; b < kQBins1; b += kEwThreads) h[b] = __ldcg(&gh[b]);
+  __syncthreads();
+  int bin;
+  uint64_t rank;
+  find_rank_bin<kEwThreads>(h, kQBins1, quantile_rank(p.clip_k, (int64_t)d.m * d.n), &bin, &rank);
+  if (threadIdx.x == 0) {
+    st->q_bin1 = (uint32_t)bin;
+    st->q_rank1 = rank;
+  }
+}
+
+// Gather the keys of every |g| whose top 11 bits equal the selected first digit into the
+// matrix's X buffer (unused until the preamble; it holds mp * np >= m * n words).  Work
+// unit = 16 rows of one matrix, as in the reduction.  Hits are staged in a shared buffer
+// (warp ballots, one shared atomic per warp and element step) and flushed with one global
+// atomic per flush, so the matrix's counter sees a few atomics per unit, not one per warp.
+constexpr int kGatherBuf = 8192;            // staged keys per CTA
+constexpr int kGatherStep = 4 * 4 * kEwThreads;   // elements per column step (4 float4 per thread)
+__global__ void __launch_bounds__(kEwThreads) ns_quantile_gather_kernel(const __grid_constant__ NsParams p) {
+  __shared__ uint32_t sbuf[kGatherBuf];
+  __shared__ uint32_t s_n;
+  __shared__ unsigned long long s_base;
+  const int32_t total = p.prefix[p.count];
+  const int lane = threadIdx.x & 31;
+  for (int32_t u = blockIdx.x; u < total; u += gridDim.x) {
+    const int mi = owner_of(p.prefix, p.count, u);
+    const MatDesc& d = p.mat[mi];
+    NsState* st = state_of(p, d);
+    if (__ldcg(&st->nonfinite) != 0u) continue;   // uniform over the CTA
+    const uint32_t bin = __ldcg(&st->q_bin1);
+    uint32_t* cand = reinterpret_cast<uint32_t*>(p.ws + mat_layout(d.mp, d.np, d.state_off, d.big_off).X);
+    const int64_t rows0 = d.tall ? d.n : d.m, cols0 = d.tall ? d.m : d.n;
+    const int64_t r0 = (u - p.prefix[mi]) * 16;
+    const bool vec = ((reinterpret_cast<uintptr_t>(d.G) & 15) == 0) && ((d.ldg & 3) == 0);
+    if (threadIdx.x == 0) s_n = 0u;
+    __syncthreads();
+    auto append = [&](uint32_t key, bool valid) {   // warp-wide: every lane calls it
+      const bool hit = valid && (key >> 20) == bin;
+      const unsigned m = __ballot_sync(0xFFFFFFFFu, hit);
+      if (m != 0u) {
+        const int leader = __ffs(m) - 1;
+        uint32_t pos = 0u;
+        if (lane == leader) pos = atomicAdd(&s_n, (uint32_t)__popc(m));
+        pos = __shfl_sync(0xFFFFFFFFu, pos, leader);
+        if (hit) sbuf[pos + __popc(m & ((1u << lane) - 1u))] = key;
+      }
+    };
+    // block-wide: move the staged keys to the matrix's candidate buffer
+    auto flush = [&]() {
+      __syncthreads();
+      const uint32_t n = s_n;
+      if (n != 0u) {
+        if (threadIdx.x == 0) s_base = atomicAdd(&st->q_count, (unsigned long long)n);
+        __syncthreads();
+        const unsigned long long base = s_base;
+        for (uint32_t i = threadIdx.x; i < n; i += kEwThreads) cand[base + i] = sbuf[i];
+        __syncthreads();
+        if (threadIdx.x == 0) s_n = 0u;
+      }
+      __syncthreads();
+    };
+    for (int64_t r = r0; r < r0 + 16 && r < rows0; ++r) {
+      const float* row = d.G + r * d.ldg;
+      // one column step adds at most kGatherStep keys: flush first when they might not fit
+      for (int64_t c0 = 0; c0 < cols0; c0 += kGatherStep) {   // uniform over the CTA
+        __syncthreads();
+        const bool full = s_n > (uint32_t)(kGatherBuf - kGatherStep);
+        __syncthreads();   // every thread has read s_n before any thread appends again
+        if (full) flush();
+        if (vec) {   // cols0 is a multiple of 16: a float4 is wholly inside or outside the row
+          float4 v[4];
+          bool valid[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int64_t c = c0 + 4 * (threadIdx.x + k * kEwThreads);
+            valid[k] = c < cols0;
+            v[k] = valid[k] ? __ldg(reinterpret_cast<const float4*>(row + c))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            append(abs_key(v[k].x), valid[k]);
+            append(abs_key(v[k].y), valid[k]);
+            append(abs_key(v[k].z), valid[k]);
+            append(abs_key(v[k].w), valid[k]);
+          }
+        } else {
+#pragma unroll 1
+          for (int k = 0; k < 16; ++k) {
+            const int64_t c = c0 + threadIdx.x + k * kEwThreads;
+            const bool valid = c < cols0;
+            append(valid ? abs_key(__ldg(row + c)) : 0u, valid);
+          }
+        }
+      }
+    }
+    flush();
+  }
+}
+
+// One CTA per matrix: the last two digits among the gathered keys, then tau, the clamp
+// bound of X_0 and the tensor scale of X_0.
+constexpr int kSelThreads = 1024;
+__global__ void __launch_bounds__(kSelThreads) ns_quantile_select2_kernel(const __grid_constant__ NsParams p) {
+  const MatDesc& d = p.mat[blockIdx.x];
+  NsState* st = state_of(p, d);
+  if (__ldcg(&st->nonfinite) != 0u) return;
+  const uint32_t* cand = reinterpret_cast<const uint32_t*>(p.ws + mat_layout(d.mp, d.np, d.state_off, d.big_off).X);
+  const uint64_t n = __ldcg(&st->q_count);
+  const uint32_t b1 = __ldcg(&st->q_bin1);
+  const uint64_t k1 = __ldcg(&st->q_rank1);
+  __shared__ uint32_t h[kQBins2];
+  for (int b = threadIdx.x; b < kQBins2; b += kSelThreads) h[b] = 0u;
+  __syncthreads();
+  for (uint64_t i = threadIdx.x; i < n; i += kSelThreads) atomicAdd(&h[(__ldcg(&cand[i]) >> 9) & (kQBins2 - 1)], 1u);
+  __syncthreads();
+  int b2;
+  uint64_t k2;
+  find_rank_bin<kSelThreads>(h, kQBins2, k1, &b2, &k2);
+  for (int b = threadIdx.x; b < kQBins3; b += kSelThreads) h[b] = 0u;
+  __syncthreads();
+  for (uint64_t i = threadIdx.x; i < n; i += kSelThreads) {
+    const uint32_t key = __ldcg(&cand[i]);
+    if (((key >> 9) & (kQBins2 - 1)) == (uint32_t)b2) atomicAdd(&h[key & (kQBins3 - 1)], 1u);
+  }
+  __syncthreads();
+  int b3;
+  uint64_t k3;
+  find_rank_bin<kSelThreads>(h, kQBins3, k2, &b3, &k3);
+  if (threadIdx.x == 0) {
+    const float gk = __uint_as_float((b1 << 20) | ((uint32_t)b2 << 9) | (uint32_t)b3);
+    const float inv = __ldcg(&st->inv0);
+    const float tau = __fmul_rn(gk, inv);
+    const float amax0 = fminf(__fmul_rn(__uint_as_float(__ldcg(&st->amaxG)), inv), tau);
+    st->tau0 = tau;
+    st->amaxX[0] = __float_as_uint(amax0);
+    st->sg[kSgX + 0] = pow2_tensor_scale((p.opts & kOptRht) ? 4.0f * amax0 : amax0,
+                                         (p.opts & kOpt46) != 0);
   }
 }
 
@@ -620,7 +843,22 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const
 }
 
 cudaError_t launch_ns_reduce(const NsParams& p, cudaStream_t st, int num_sms) {
-  ns_reduce_kernel<<<persistent_grid(ns_reduce_kernel, p.prefix[p.count], num_sms), kEwThreads, 0, st>>>(p);
+  if (p.opts & kOptQuantile)
+    ns_reduce_kernel<true><<<persistent_grid(ns_reduce_kernel<true>, p.prefix[p.count], num_sms), kEwThreads, 0, st>>>(p);
+  else
+    ns_reduce_kernel<false><<<persistent_grid(ns_reduce_kernel<false>, p.prefix[p.count], num_sms), kEwThreads, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+// Quantile clip selection after the reduction (p.prefix holds the reduction's units).
+cudaError_t launch_ns_quantile(const NsParams& p, cudaStream_t st, int num_sms) {
+  ns_quantile_select1_kernel<<<p.count, kEwThreads, 0, st>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  ns_quantile_gather_kernel<<<persistent_grid(ns_quantile_gather_kernel, p.prefix[p.count], num_sms),
+                              kEwThreads, 0, st>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  ns_quantile_select2_kernel<<<p.count, kSelThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 

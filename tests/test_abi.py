@@ -106,6 +106,13 @@ def test_root_ns_rejects_bad_arguments(F):
     assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 3.0, 1 << 29, W, ok, None) == -1   # unknown flag
     # the test-only stall flag is accepted (the call then fails on the workspace size)
     assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 3.0, F.FS4_TEST_STALL, W, ok - 1, None) == -4
+    # the quantile clip takes clip_k as a ratio in (0, 1]
+    qf = F.FS4_NS_CLIP_QUANTILE
+    assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 0.0, qf, W, ok, None) == -1
+    assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 3.0, qf, W, ok, None) == -1
+    assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, -0.5, qf, W, ok, None) == -1
+    assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 0.99, qf, W, ok - 1, None) == -4   # accepted
+    assert ns(G, 64, 96, 96, O, 96, 5, 1.0, 0.0, 0.0, 1.0, qf, W, ok - 1, None) == -4
 
 
 def test_batched_rejects_overlapping_outputs_and_bad_counts(F):
