@@ -45,9 +45,10 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="ns", choices=["ns", "quantize", "dequantize"],
+    ap.add_argument("--op", default="ns", choices=["ns", "quantize", "dequantize", "momentum"],
                     help="ns: the Newton-Schulz step (default); quantize / dequantize: the standalone "
-                         "NVFP4 calls over every matrix of the workload (row axis)")
+                         "NVFP4 calls over every matrix of the workload (row axis); momentum: one "
+                         "NVFP4 first-moment step (fs4_momentum_nvfp4) per matrix")
     ap.add_argument("--layout", default="plain", choices=["plain", "tiled"],
                     help="NVFP4 layout of --op quantize / dequantize")
     ap.add_argument("--clip", default="rms", choices=["rms", "p99"],
@@ -219,6 +220,8 @@ def oracle_sample_rate(w, budget_s: float):
 
 
 QD_BYTES = 4.5625          # algorithmic bytes per element: 4 B of FP32 + 0.5 B of codes + 1/16 B of scale
+MO_BYTES = 9.125   # momentum step: read g (4 B) and the state (0.5625 B), write m_t (4 B) and the state
+MO_METRIC = "NVFP4 first-moment step GB/s (9.125 B per element)"
 QD_METRIC = {"quantize": "NVFP4 standalone quantise GB/s (4.5625 B per element)",
              "dequantize": "NVFP4 standalone dequantise GB/s (4.5625 B per element)"}
 
@@ -257,6 +260,9 @@ def run_reference(args):
     if rank != 0:
         return
     w = WORKLOADS[args.workload]
+    if args.op == "momentum":
+        run_momentum_reference(args, w)
+        return
     if args.op != "ns":
         rates, desc = [], ""
         for i in range(args.warmup + args.steps):
@@ -326,6 +332,11 @@ def main():
         return max_over_ranks(v, world, "cuda")
 
     w = WORKLOADS[args.workload]
+    if args.op == "momentum":
+        run_momentum(args, w, rank, world, local, barrier, ranks_max)
+        if world > 1:
+            dist.destroy_process_group()
+        return
     if args.op != "ns":
         run_standalone(args, w, rank, world, local, barrier, ranks_max)
         if world > 1:
@@ -710,6 +721,191 @@ def run_standalone(args, w, rank, world, local, barrier, ranks_max):
             "clocks": sampler.summary(),
         }
         print(json.dumps(line), flush=True)
+
+
+def oracle_momentum_rate(w, budget_s: float):
+    """Time the oracle's momentum step (with a previous state) on leading rows of the
+    workload's first matrix.  Returns (algorithmic GB/s, seconds, description)."""
+    from oracle import momentum as M
+    from nvfp4_precision_optimizer_b200.workloads import BASE_SEED, generate
+    G = generate(w.shapes[0], w.dist, BASE_SEED, "cpu").numpy()
+    rows = 16
+    while True:
+        g = G[:rows]
+        _, state = M.update(g, 0.95, None, 0, 0x5A5A, 1)
+        t0 = time.perf_counter()
+        M.update(g, 0.95, state, 0x5A5A, 0xC3C3, 2)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s / 4 or rows >= G.shape[0]:
+            break
+        rows = min(G.shape[0], rows * 4)
+    desc = (f"oracle momentum step (numpy, exact emulation) of the first {rows} rows of a "
+            f"{G.shape[0]}x{G.shape[1]} workload matrix, {dt:.2f} s")
+    return g.size * MO_BYTES / dt / 1e9, dt, desc
+
+
+def run_momentum_reference(args, w):
+    rates, desc = [], ""
+    for i in range(args.warmup + args.steps):
+        rate, dt, desc = oracle_momentum_rate(w, max(2.0, 120.0 / max(1, args.steps + args.warmup)))
+        if i >= args.warmup:
+            rates.append(rate)
+    value = statistics.median(rates)
+    total = sum(r * c for r, c in w.shapes) * MO_BYTES
+    print(json.dumps({
+        "impl": "reference", "metric": MO_METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * total / (value * 1e9), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 values, exact NVFP4 emulation", "data": "synthetic",
+        "config": {"workload": w.name, "matrices": len(w.shapes), "op": "momentum"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def run_momentum(args, w, rank, world, local, barrier, ranks_max):
+    """--op momentum: one step = one fs4_momentum_nvfp4 call per matrix of the workload
+    (previous state present, updated in place; m_t written in FP32)."""
+    import torch
+    import nvfp4_precision_optimizer_b200 as F
+    from nvfp4_precision_optimizer_b200.workloads import BASE_SEED, matrices
+
+    lib = F._lib.lib()
+    Gs = matrices(w, device="cuda", seed=rank_seed(BASE_SEED, rank))
+    stream = torch.cuda.current_stream()
+    wsz = int(lib.fs4_momentum_workspace_size())
+    bufs = []
+    for G in Gs:
+        R, C = G.shape
+        bufs.append({"codes": torch.empty((R, C // 2), dtype=torch.uint8, device="cuda"),
+                     "scales": torch.empty((R, C // 16), dtype=torch.uint8, device="cuda"),
+                     "sg": torch.empty(1, dtype=torch.float32, device="cuda"),
+                     "m": torch.empty_like(G),
+                     "ws": torch.zeros(wsz, dtype=torch.uint8, device="cuda")})
+    step_no = [0]
+
+    def call(i, g, st, first=False):
+        b = bufs[i]
+        prev = (None, None, None) if first else (b["codes"].data_ptr(), b["scales"].data_ptr(),
+                                                 b["sg"].data_ptr())
+        k = step_no[0]
+        F.check(lib.fs4_momentum_nvfp4(g.data_ptr(), g.shape[0], g.shape[1], g.shape[1], 0.95,
+                                       prev[0], prev[1], prev[2], (0x5A5A + k) & 0xFFFF,
+                                       b["codes"].data_ptr(), b["scales"].data_ptr(), b["sg"].data_ptr(),
+                                       (0x5A5A + k + 1) & 0xFFFF, 1000 * k + i, b["m"].data_ptr(),
+                                       g.shape[1], b["ws"].data_ptr(), wsz, st.cuda_stream),
+                "fs4_momentum_nvfp4")
+
+    for i, G in enumerate(Gs):
+        call(i, G, stream, first=True)
+    step_no[0] += 1
+    for _ in range(max(3, args.warmup)):
+        for i, G in enumerate(Gs):
+            call(i, G, stream)
+        step_no[0] += 1
+    torch.cuda.synchronize()
+    for b in bufs:
+        F.check(F.device_status(b["ws"]), "device status after warm-up")
+    call_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(Gs) + 1)] for _ in range(args.steps)]
+    for evs in call_ev:
+        for e in evs:
+            e.record(stream)
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    with sampler:
+        time.sleep(0.3)
+        for s in range(args.steps):
+            call_ev[s][0].record(stream)
+            for i, G in enumerate(Gs):
+                call(i, G, stream)
+                call_ev[s][i + 1].record(stream)
+            step_no[0] += 1
+        torch.cuda.synchronize()
+    barrier()
+    total_ms = ranks_max(call_ev[0][0].elapsed_time(call_ev[-1][-1]))
+    ms_step = total_ms / args.steps
+    elems = sum(G.numel() for G in Gs)
+    value = job_rate(world, elems * MO_BYTES / 1e9, ms_step)
+    call_ms = [evs[i].elapsed_time(evs[i + 1]) for evs in call_ev for i in range(len(Gs))]
+    mean_call = statistics.mean(call_ms)
+    peaks, peak_src = measured_peaks()
+    achieved = elems * MO_BYTES / len(Gs) / (mean_call * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+            "kernel": "fs4_momentum_nvfp4 call (momentum_pass1_kernel + momentum_pass2_kernel)",
+            "ms_per_launch": mean_call, "peak_source": f"hbm_gbs ({peak_src} MEASURED_PEAKS.json)"}
+
+    # end to end: each matrix's gradient copied in from pinned host memory, the step, and
+    # m_t copied back (the state stays on the device), pipelined over three streams
+    e2e = None
+    if not args.no_e2e:
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        host_g = [G.cpu().pin_memory() for G in Gs]
+        dev_g = [torch.empty_like(G) for G in Gs]
+        host_m = [torch.empty(G.shape, dtype=torch.float32).pin_memory() for G in Gs]
+        ev_in = [torch.cuda.Event() for _ in Gs]
+        ev_done = [torch.cuda.Event() for _ in Gs]
+        ev_out = [torch.cuda.Event() for _ in Gs]
+        for e in ev_in + ev_done + ev_out:
+            e.record(stream)
+
+        def e2e_step():
+            for i in range(len(Gs)):
+                with torch.cuda.stream(s_in):
+                    s_in.wait_event(ev_done[i])
+                    dev_g[i].copy_(host_g[i], non_blocking=True)
+                    ev_in[i].record(s_in)
+                stream.wait_event(ev_in[i])
+                stream.wait_event(ev_out[i])
+                call(i, dev_g[i], stream)
+                ev_done[i].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_done[i])
+                    host_m[i].copy_(bufs[i]["m"], non_blocking=True)
+                    ev_out[i].record(s_out)
+            step_no[0] += 1
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e2e_steps = max(2, min(args.steps, 5))
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        s_in.wait_event(e0)
+        for _ in range(e2e_steps):
+            e2e_step()
+        for e in ev_out:
+            stream.wait_event(e)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = ranks_max(e0.elapsed_time(e1)) / e2e_steps
+        e2e = {"value": job_rate(world, elems * MO_BYTES / 1e9, e2e_ms), "unit": "GB/s",
+               "h2d_bytes_per_step": elems * 4, "d2h_bytes_per_step": elems * 4, "ms_per_step": e2e_ms,
+               "pipeline": "per matrix: gradient copy-in, step and m_t copy-out overlap on three streams"}
+    for b in bufs:
+        F.check(F.device_status(b["ws"]), "device status after the timed steps")
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, dt, desc = oracle_momentum_rate(w, 20.0)
+        cpu = {"value": rate, "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps({
+            "metric": MO_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32 momentum, nvfp4 state (e2m1 x e4m3/16, SR, adaptive 4/6, H16^r)",
+            "data": "synthetic",
+            "config": {"workload": w.name, "matrices": len(Gs), "op": "momentum", "beta": 0.95,
+                       "state": "previous state present, updated in place; m_t written in FP32",
+                       "parallelism": f"replicas x{world} (independent matrices, no collective)",
+                       "l2": "inputs larger than L2 (%.2f GB of FP32 per step)" % (elems * 4 / 1e9)},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps * len(Gs) * 2, "clocks": sampler.summary(),
+        }), flush=True)
 
 
 if __name__ == "__main__":

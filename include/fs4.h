@@ -161,6 +161,45 @@ fs4_status fs4_nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, con
                                 int64_t rows, int64_t cols, float* y, int64_t ld,
                                 uint32_t flags, void* stream);
 
+/* ------------------------------------------------------- momentum (first moment) */
+
+/* Bytes of workspace fs4_momentum_nvfp4 needs (at least 256-byte aligned). */
+size_t fs4_momentum_workspace_size(void);
+
+/* One step of the NVFP4-stored first moment of Q-Root (Section 3.3: "Hadamard mixing
+ * smooths the distribution before SR and adaptive 4/6 quantization"; Section 3.4: the
+ * first-order momentum follows that storage recipe).  Per element of the FP32 gradient
+ * g (rows x cols, leading dimension ld, cols % 16 == 0):
+ *   m_prev = 0, or the previous state decoded: fp32(fp32(code * s) * s_g) on each 1x16
+ *            block, then (H16^r)^-1 = H16 D / 4 with D the signs of prev_mask;
+ *   m_t    = fp32(fp32(beta * m_prev) + fp32(fp32(1 - beta) * g));
+ *   state  = NVFP4 of y = m_t H16^r (signs of `mask`, FP32 butterfly, * 0.25) in
+ *            PLAIN 1x16 row blocks: tensor scale the smallest power of two with
+ *            4 * 448 * s_g >= max |y|; per block the M = 6 and M = 4 candidates
+ *            (scale RN_e4m3(amax_b / (M s_g))) with stochastically rounded codes,
+ *            M = 4 kept only when its FP32 squared error (summed in element order)
+ *            is strictly smaller.  A code is rounded up from the E2M1 value lo below
+ *            v = fp32(|y| / den) to the next one, hi, when u < (v - lo) / (hi - lo);
+ *            v >= 6 gives 6.  u for element (i, j) is the top 24 bits of SplitMix64
+ *            at counter i * cols + j: z = seed + (i * cols + j + 1) * 0x9E3779B97F4A7C15,
+ *            z ^= z >> 30, z *= 0xBF58476D1CE4E5B9, z ^= z >> 27,
+ *            z *= 0x94D049BB133111EB, z ^= z >> 31; u = (z >> 40) * 2^-24.
+ * prev_codes, prev_scales, prev_sg: the previous state (all null on the first step);
+ * they may be the same buffers as codes, scales, s_g (in-place update).  m_out (may be
+ * null; leading dimension ld_out) receives m_t in FP32, the matrix the Newton-Schulz
+ * step consumes; it must not overlap g.  codes: rows x cols/2 bytes, scales:
+ * rows x cols/16 bytes (16-byte aligned), s_g: one device float.  Two launches.
+ * Errors: FS4_ERR_SHAPE, FS4_ERR_INVALID_ARG (null outputs, a partial previous state,
+ * non-finite beta, ld or ld_out too small, misalignment), FS4_ERR_ALIAS (m_out
+ * overlaps g), FS4_ERR_WORKSPACE; non-finite g is reported as FS4_ERR_NONFINITE
+ * through fs4_device_status. */
+fs4_status fs4_momentum_nvfp4(const float* g, int64_t rows, int64_t cols, int64_t ld,
+                              float beta, const uint8_t* prev_codes,
+                              const uint8_t* prev_scales, const float* prev_sg,
+                              uint32_t prev_mask, uint8_t* codes, uint8_t* scales, float* s_g,
+                              uint32_t mask, uint64_t seed, float* m_out, int64_t ld_out,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
 /* --------------------------------------------------------------------- GEMM */
 
 /* D = deq(A) * deq(B)^T on the tcgen05 block-scaled tensor cores

@@ -21,6 +21,7 @@ MUON_COEFFS = (3.4445, -4.7750, 2.0315)
 __all__ = [
     "quantize", "dequantize", "gemm", "root_ns", "root_ns_batched", "ns_workspace_size",
     "ns_batched_workspace_size", "ns_layout", "device_status", "tiled_shape", "Fs4Error",
+    "momentum_nvfp4",
     "MUON_COEFFS", "stop_after", "FS4_AXIS_ROW", "FS4_AXIS_COL", "FS4_TEST_STALL",
     "FS4_NS_RHT", "FS4_NS_ADAPTIVE46", "FS4_NS_CLIP_QUANTILE",
 ]
@@ -92,6 +93,32 @@ def dequantize(codes: torch.Tensor, scales: torch.Tensor, s_g: torch.Tensor, row
                                           FS4_LAYOUT_TILED if tiled else 0, _stream(stream)),
           "fs4_nvfp4_dequantize")
     return y
+
+
+def momentum_nvfp4(g: torch.Tensor, beta: float, state=None, prev_mask: int = 0, mask: int = 0,
+                   seed: int = 0, want_m: bool = True, out_state=None,
+                   workspace: torch.Tensor | None = None, stream=None):
+    """One step of the NVFP4-stored first moment (fs4_momentum_nvfp4).  state / out_state
+    are (codes, scales, s_g) triples in the PLAIN layout (out_state may be `state` for an
+    in-place step).  Returns (m_t FP32 or None, new state)."""
+    _check_f32_matrix(g, "g")
+    rows, cols = g.shape
+    dev = g.device
+    if out_state is None:
+        out_state = (torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev),
+                     torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev),
+                     torch.empty(1, dtype=torch.float32, device=dev))
+    m_out = torch.empty_like(g) if want_m else None
+    if workspace is None:
+        workspace = torch.empty(_lib.lib().fs4_momentum_workspace_size(), dtype=torch.uint8, device=dev)
+    prev = (None, None, None) if state is None else tuple(t.data_ptr() for t in state)
+    check(_lib.lib().fs4_momentum_nvfp4(g.data_ptr(), rows, cols, _ld(g), beta, prev[0], prev[1],
+                                        prev[2], prev_mask, out_state[0].data_ptr(),
+                                        out_state[1].data_ptr(), out_state[2].data_ptr(), mask,
+                                        seed, _ptr(m_out), _ld(m_out) if want_m else cols,
+                                        workspace.data_ptr(), workspace.numel(), _stream(stream)),
+          "fs4_momentum_nvfp4")
+    return m_out, out_state
 
 
 def gemm(a, b, M: int, N: int, K: int, out: torch.Tensor | None = None,

@@ -49,6 +49,10 @@ class NsLayout(ctypes.Structure):
 # name -> (restype, argtypes); the order follows include/fs4.h
 SIGNATURES = {
     "fs4_nvfp4_quantize_workspace_size": (c_sz, []),
+    "fs4_momentum_workspace_size": (c_sz, []),
+    "fs4_momentum_nvfp4": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_f32, c_vp, c_vp, c_vp, c_u32,
+                                   c_vp, c_vp, c_vp, c_u32, ctypes.c_uint64, c_vp, c_i64, c_vp,
+                                   c_sz, c_vp]),
     "fs4_nvfp4_quantize": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_i32, c_vp, c_vp, c_vp, c_u32,
                                    c_vp, c_sz, c_vp]),
     "fs4_nvfp4_dequantize": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_i64, c_u32, c_vp]),

@@ -197,6 +197,39 @@ extern "C" {
 
 size_t fs4_nvfp4_quantize_workspace_size(void) { return kHeaderBytes; }
 
+size_t fs4_momentum_workspace_size(void) { return kHeaderBytes; }
+
+fs4_status fs4_momentum_nvfp4(const float* g, int64_t rows, int64_t cols, int64_t ld,
+                              float beta, const uint8_t* prev_codes,
+                              const uint8_t* prev_scales, const float* prev_sg,
+                              uint32_t prev_mask, uint8_t* codes, uint8_t* scales, float* s_g,
+                              uint32_t mask, uint64_t seed, float* m_out, int64_t ld_out,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  if (!g || !codes || !scales || !s_g) return FS4_ERR_INVALID_ARG;
+  const int nprev = (prev_codes != nullptr) + (prev_scales != nullptr) + (prev_sg != nullptr);
+  if (nprev != 0 && nprev != 3) return FS4_ERR_INVALID_ARG;
+  if (!std::isfinite(beta) || prev_mask > 0xFFFFu || mask > 0xFFFFu) return FS4_ERR_INVALID_ARG;
+  if (rows < 1 || cols < 16 || rows > (1ll << 31) || cols > (1ll << 31) || cols % 16) return FS4_ERR_SHAPE;
+  if (ld < cols || (m_out && ld_out < cols)) return FS4_ERR_INVALID_ARG;
+  if (!aligned(g, 4) || (m_out && !aligned(m_out, 4)) || !aligned(codes, 16) || !aligned(scales, 16) ||
+      !aligned(s_g, 4) || (prev_codes && (!aligned(prev_codes, 16) || !aligned(prev_sg, 4))))
+    return FS4_ERR_INVALID_ARG;
+  if (m_out) {
+    uintptr_t glo, ghi, olo, ohi;
+    span(g, rows, cols, ld, &glo, &ghi);
+    span(m_out, rows, cols, ld_out, &olo, &ohi);
+    if (olo < ghi && glo < ohi) return FS4_ERR_ALIAS;
+  }
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < kHeaderBytes) return FS4_ERR_WORKSPACE;
+  DeviceInfo di;
+  const fs4_status ds = device_info(&di);
+  if (ds != FS4_OK) return ds;
+  return cuda_status(launch_momentum(g, rows, cols, ld, beta, prev_codes, prev_scales, prev_sg,
+                                     prev_mask, codes, scales, s_g, mask, seed, m_out, ld_out,
+                                     static_cast<uint8_t*>(workspace),
+                                     static_cast<cudaStream_t>(stream), di.num_sms));
+}
+
 fs4_status fs4_nvfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld, int32_t axis,
                               uint8_t* codes, uint8_t* scales, float* s_g, uint32_t flags,
                               void* workspace, size_t workspace_bytes, void* stream) {

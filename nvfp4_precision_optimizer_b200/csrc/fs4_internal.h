@@ -141,6 +141,12 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const
                               cudaStream_t st, int num_sms);
 cudaError_t launch_ns_reduce(const NsParams& p, cudaStream_t st, int num_sms);
 cudaError_t launch_ns_quantile(const NsParams& p, cudaStream_t st, int num_sms);
+cudaError_t launch_momentum(const float* g, int64_t rows, int64_t cols, int64_t ld, float beta,
+                            const uint8_t* prev_codes, const uint8_t* prev_scales,
+                            const float* prev_sg, uint32_t prev_mask, uint8_t* codes,
+                            uint8_t* scales, float* s_g, uint32_t mask, uint64_t seed,
+                            float* m_out, int64_t ld_out, uint8_t* ws, cudaStream_t st,
+                            int num_sms);
 cudaError_t launch_ns_preamble(const NsParams& p, cudaStream_t st, int num_sms);
 cudaError_t launch_gemm_plain(const GemmPlainArgs& a, cudaStream_t st, int num_sms);
 cudaError_t launch_gemm_ns(Epi epi, const NsParams& p, cudaStream_t st, int num_sms);

@@ -181,3 +181,32 @@ def test_tiled_layout_matches_header_formula():
     atom = (r // 128) * (Cp // 64) + c // 64
     soff = atom * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32) + (c // 16) % 4
     assert st[soff] == 0xCD and np.count_nonzero(st) == 1
+
+
+def test_momentum_argument_errors(F):
+    """fs4_momentum_nvfp4 rejects bad arguments on the host, before any launch."""
+    lib = F._lib.lib()
+    mo = lib.fs4_momentum_nvfp4
+    g, c, s, sg, W, mout = 1 << 20, 2 << 20, 3 << 20, 4 << 20, 5 << 20, 6 << 20   # fake aligned pointers
+    wsz = lib.fs4_momentum_workspace_size()
+    ok = (g, 32, 64, 64, 0.9, None, None, None, 0, c, s, sg, 0, 1, mout, 64, W, wsz, None)
+    def call(**kw):
+        args = list(ok)
+        names = ["g", "rows", "cols", "ld", "beta", "pc", "ps", "psg", "pmask", "c", "s", "sg",
+                 "mask", "seed", "m", "ldo", "ws", "wsb", "st"]
+        for k, v in kw.items():
+            args[names.index(k)] = v
+        return mo(*args)
+    assert call(cols=72) == -2                       # cols % 16
+    assert call(rows=0) == -2
+    assert call(g=None) == -1
+    assert call(c=None) == -1
+    assert call(beta=float("nan")) == -1
+    assert call(ld=48) == -1                         # ld < cols
+    assert call(ldo=48) == -1
+    assert call(pc=c) == -1                          # partial previous state
+    assert call(mask=1 << 16) == -1
+    assert call(c=c + 8) == -1                       # codes not 16-byte aligned
+    assert call(m=g + 1024) == -3                    # m_out overlaps g
+    assert call(ws=W + 4) == -4
+    assert call(wsb=wsz - 1) == -4
