@@ -257,3 +257,39 @@ def test_bounded_wait_timeout_reports_status_and_context_survives(fs4):
     got, ws2 = run_gpu(fs4, G, 2, MUON)         # fresh workspace, same context
     want = R.root_ns(G, 2, *MUON, clip_k=3.0)
     assert rel_frob(got, want) <= 2e-2
+
+
+@pytest.mark.parametrize("shape,kind,K,coef", [
+    ((16, 16), "gauss", 3, QUINTIC),          # the smallest legal matrix: one padded tile
+    ((16, 4096), "gauss", 3, QUINTIC),        # m = 16: a 16 x 16 Gram inside one 256 x 256 tile
+    ((4096, 16), "student", 3, QUINTIC),      # tall: processed as its 16 x 4096 transpose
+    ((272, 272), "outliers", 3, QUINTIC),     # one row and column past a 256 boundary
+    ((2064, 256), "gauss", 2, CUBIC),         # tall: working 256 x 2064, n padded to 2304
+])
+def test_extreme_shapes_parity(fs4, shape, kind, K, coef):
+    G = momentum(*shape, kind=kind, seed=6)
+    got, _ = run_gpu(fs4, G, K, coef)
+    want = R.root_ns(G, K, *coef, clip_k=3.0)
+    assert got.shape == G.shape and np.all(np.isfinite(got))
+    assert rel_frob(got, want) <= 2e-2
+
+
+def test_batch_of_random_shapes_matches_oracle(fs4):
+    """A batch of random multiple-of-16 shapes (both orientations, different paddings)
+    with per-matrix coefficients, against the oracle one by one."""
+    rng = np.random.default_rng(77)
+    specs = []
+    for i in range(9):
+        m, n = (int(v) * 16 for v in rng.integers(1, 40, 2))
+        coef = (QUINTIC, CUBIC)[i % 2]
+        specs.append(((m, n), coef))
+    Gs = [momentum(*s, kind=("gauss", "student", "outliers")[i % 3], seed=200 + i)
+          for i, (s, _) in enumerate(specs)]
+    coeffs = [c for _, c in specs]
+    Gt = [torch.from_numpy(G).cuda() for G in Gs]
+    outs = fs4.root_ns_batched(Gt, K=2, coeffs=coeffs, clip_k=3.0)
+    torch.cuda.synchronize()
+    for G, o, coef in zip(Gs, outs, coeffs):
+        got = o.cpu().numpy()
+        assert got.shape == G.shape
+        assert rel_frob(got, R.root_ns(G, 2, *coef, clip_k=3.0)) <= 2e-2, G.shape
