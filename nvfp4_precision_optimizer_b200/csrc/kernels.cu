@@ -137,20 +137,18 @@ __global__ void __launch_bounds__(kEwThreads) amax_kernel(const float* __restric
 }
 
 // Quantise the R x C matrix Y (Y = x for the row axis, Y = x^T for the column
-// axis) in 1x16 blocks along Y's rows.  One CTA per 64 x 64 tile of Y's
-// (padded) extent; the tile is staged through shared memory so both axes read
-// x with coalesced loads.
+// axis) in 1x16 blocks along Y's rows.  Work unit = one 64 x 64 tile of Y's (padded)
+// extent, staged through shared memory so both axes read x with coalesced loads.
+// Persistent CTAs: the next unit's x tile is loaded into registers while the current
+// one is quantised (interior tiles of 16-byte aligned inputs; edge tiles load on the
+// guarded path).  Tiles are visited in x's row-major order, last tile first: the amax
+// pass just streamed x top to bottom, so the tail of x is still resident in L2.
 __global__ void __launch_bounds__(kEwThreads) quantize_kernel(
     const float* __restrict__ x, int64_t ld, int64_t R, int64_t C, int col_axis, int tiled,
-    int sg_amax_mode, int64_t Rext, int64_t Cext, int64_t Cp, uint8_t* __restrict__ codes,
-    uint8_t* __restrict__ scales, float* __restrict__ s_g_out, const uint32_t* __restrict__ hdr) {
+    int sg_amax_mode, int64_t Rext, int64_t Cext, int64_t Cp, int64_t ntiles,
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, float* __restrict__ s_g_out,
+    const uint32_t* __restrict__ hdr) {
   __shared__ float tile[kT][kT + 1];
-  // Tiles are visited in x's row-major order, last tile first: the amax pass just
-  // streamed x top to bottom, so the tail of x is still resident in L2.
-  const int64_t xt = gridDim.x - 1 - blockIdx.x;
-  const int64_t xtiles_c = (col_axis ? Rext : Cext) / kT;
-  const int64_t xi0 = (xt / xtiles_c) * kT, xj0 = (xt % xtiles_c) * kT;
-  const int64_t i0 = col_axis ? xj0 : xi0, j0 = col_axis ? xi0 : xj0;
   const float amax = __uint_as_float(__ldcg(&hdr[1]));
   float s_g;
   if (sg_amax_mode) {
@@ -163,24 +161,52 @@ __global__ void __launch_bounds__(kEwThreads) quantize_kernel(
   const float rcp_six = __frcp_rn(six_sg);
 
   const int t = threadIdx.x;
-  // Stage the 64 x 64 tile of x (coalesced: 16 threads per 256-byte line segment, float4
-  // loads for interior tiles of 16-byte aligned inputs).  Row axis: x line = row i of the
-  // quantised matrix Y; column axis: x line = column of Y (Y = x^T), stored transposed.
-  {
-    const int64_t xr0 = col_axis ? j0 : i0, xc0 = col_axis ? i0 : j0;      // tile origin in x
-    const int64_t xrows = col_axis ? C : R, xcols = col_axis ? R : C;       // x's extent
-    const bool vec = ((reinterpret_cast<uintptr_t>(x) & 15) == 0) && ((ld & 3) == 0) &&
-                     xr0 + kT <= xrows && xc0 + kT <= xcols;
+  const int64_t xtiles_c = (col_axis ? Rext : Cext) / kT;
+  const int64_t xrows = col_axis ? C : R, xcols = col_axis ? R : C;       // x's extent
+  const bool aligned = ((reinterpret_cast<uintptr_t>(x) & 15) == 0) && ((ld & 3) == 0);
+  auto origin = [&](int64_t u, int64_t& xr0, int64_t& xc0) {   // tile origin in x
+    const int64_t xt = ntiles - 1 - u;
+    xr0 = (xt / xtiles_c) * kT;
+    xc0 = (xt % xtiles_c) * kT;
+  };
+  // 16 threads per 256-byte line segment of x, four passes of 16 lines
+  float4 pf[4];
+  bool pf_fast = false;
+  auto prefetch = [&](int64_t u) {
+    pf_fast = false;
+    if (u >= ntiles) return;
+    int64_t xr0, xc0;
+    origin(u, xr0, xc0);
+    if (aligned && xr0 + kT <= xrows && xc0 + kT <= xcols) {
+      pf_fast = true;
+#pragma unroll
+      for (int pass = 0; pass < 4; ++pass) {
+        const int f = t + kEwThreads * pass;
+        pf[pass] = __ldg(reinterpret_cast<const float4*>(x + (xr0 + (f >> 4)) * ld + xc0 + (f & 15) * 4));
+      }
+    }
+  };
+  prefetch(blockIdx.x);
+  for (int64_t u = blockIdx.x; u < ntiles; u += gridDim.x) {
+    float4 cur[4];
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) cur[pass] = pf[pass];
+    const bool cur_fast = pf_fast;
+    prefetch(u + gridDim.x);
+    int64_t xr0, xc0;
+    origin(u, xr0, xc0);
+    const int64_t i0 = col_axis ? xc0 : xr0, j0 = col_axis ? xr0 : xc0;
+    // Row axis: x line = row i of the quantised matrix Y; column axis: x line = column
+    // of Y (Y = x^T), stored transposed.
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass) {
       const int f = t + kEwThreads * pass;
       const int line = f >> 4, c4 = (f & 15) * 4;
-      const float* src = x + (xr0 + line) * ld + xc0 + c4;
       float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      if (vec) {
-        const float4 x4 = __ldg(reinterpret_cast<const float4*>(src));
-        v[0] = x4.x; v[1] = x4.y; v[2] = x4.z; v[3] = x4.w;
+      if (cur_fast) {
+        v[0] = cur[pass].x; v[1] = cur[pass].y; v[2] = cur[pass].z; v[3] = cur[pass].w;
       } else if (xr0 + line < xrows) {
+        const float* src = x + (xr0 + line) * ld + xc0 + c4;
 #pragma unroll
         for (int e = 0; e < 4; ++e)
           if (xc0 + c4 + e < xcols) v[e] = __ldg(src + e);
@@ -191,20 +217,21 @@ __global__ void __launch_bounds__(kEwThreads) quantize_kernel(
         else tile[c4 + e][line] = v[e];
       }
     }
-  }
-  __syncthreads();
-  const int r = t >> 2, cb = (t & 3) * 16;
-  const int64_t i = i0 + r, j = j0 + cb;
-  float v[16];
+    __syncthreads();
+    const int r = t >> 2, cb = (t & 3) * 16;
+    const int64_t i = i0 + r, j = j0 + cb;
+    float v[16];
 #pragma unroll
-  for (int e = 0; e < 16; ++e) v[e] = tile[r][cb + e];
-  const QBlock16 q = sg_amax_mode ? quantize16<false>(v, s_g, six_sg, rcp_six)
-                                  : quantize16<true>(v, s_g, six_sg, rcp_six);
-  if (tiled) {
-    store_block_tiled(codes, scales, i, j, Cp, q);
-  } else if (i < R && j < C) {
-    *reinterpret_cast<uint2*>(codes + i * (C / 2) + j / 2) = make_uint2(q.w0, q.w1);
-    scales[i * (C / 16) + j / 16] = static_cast<uint8_t>(q.scale);
+    for (int e = 0; e < 16; ++e) v[e] = tile[r][cb + e];
+    const QBlock16 q = sg_amax_mode ? quantize16<false>(v, s_g, six_sg, rcp_six)
+                                    : quantize16<true>(v, s_g, six_sg, rcp_six);
+    if (tiled) {
+      store_block_tiled(codes, scales, i, j, Cp, q);
+    } else if (i < R && j < C) {
+      *reinterpret_cast<uint2*>(codes + i * (C / 2) + j / 2) = make_uint2(q.w0, q.w1);
+      scales[i * (C / 16) + j / 16] = static_cast<uint8_t>(q.scale);
+    }
+    __syncthreads();   // the tile is restaged by the next unit
   }
 }
 
@@ -826,9 +853,8 @@ cudaError_t launch_quantize(const float* x, int64_t rows, int64_t cols, int64_t 
   const int64_t Cext = tiled ? Cp : align_up(C, kT);
   const int64_t ntiles = (Rext / kT) * (Cext / kT);
   if (ntiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
-  quantize_kernel<<<(unsigned)ntiles, kEwThreads, 0, st>>>(x, ld, R, C, axis, tiled,
-                                                          (flags & 1u) ? 1 : 0, Rext, Cext, Cp,
-                                                          codes, scales, s_g, hdr);
+  quantize_kernel<<<persistent_grid(quantize_kernel, ntiles, num_sms), kEwThreads, 0, st>>>(
+      x, ld, R, C, axis, tiled, (flags & 1u) ? 1 : 0, Rext, Cext, Cp, ntiles, codes, scales, s_g, hdr);
   return cudaGetLastError();
 }
 
