@@ -138,7 +138,7 @@ __device__ __forceinline__ void mo_block(const MoArgs& a, float prev_sg, int64_t
   rht16(y, a.mask);
 }
 
-__global__ void __launch_bounds__(kMoThreads) momentum_pass1_kernel(const __grid_constant__ MoArgs a) {
+__global__ void __launch_bounds__(kMoThreads, 4) momentum_pass1_kernel(const __grid_constant__ MoArgs a) {
   __shared__ float red[kMoThreads / 32];
   const float prev_sg = a.prev_codes ? __ldcg(a.prev_sg) : 0.0f;
   if (blockIdx.x == 0 && threadIdx.x == 0) a.hdr[2] = __float_as_uint(prev_sg);
@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(kMoThreads) momentum_pass1_kernel(const __grid
   if (threadIdx.x == 0) atomicMax(&a.hdr[1], __float_as_uint(mx));
 }
 
-__global__ void __launch_bounds__(kMoThreads) momentum_pass2_kernel(const __grid_constant__ MoArgs a) {
+__global__ void __launch_bounds__(kMoThreads, 4) momentum_pass2_kernel(const __grid_constant__ MoArgs a) {
   const float prev_sg = __uint_as_float(__ldcg(&a.hdr[2]));
   const float s_g = pow2_tensor_scale(__uint_as_float(__ldcg(&a.hdr[1])), true);
   if (blockIdx.x == 0 && threadIdx.x == 0) *a.s_g = s_g;
