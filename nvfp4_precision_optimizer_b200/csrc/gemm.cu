@@ -190,31 +190,6 @@ __device__ __forceinline__ void warp_transpose(const float* v, float* w, float* 
   __syncwarp();
 }
 
-// Read-and-clear max of a float vector in global memory by one warp (values >= 0):
-// float4 loads, four in flight per lane.
-__device__ __forceinline__ float warp_drain_max4(float* vec, int64_t len, int lane) {
-  float m = 0.0f;
-  float4* v4 = reinterpret_cast<float4*>(vec);
-  const int64_t n4 = len >> 2;     // len is a multiple of 256
-  for (int64_t base = 0; base < n4; base += 128) {
-    float4 a[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int64_t i = base + k * 32 + lane;
-      a[k] = i < n4 ? __ldcg(v4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int64_t i = base + k * 32 + lane;
-      if (i < n4) __stcg(v4 + i, make_float4(0.f, 0.f, 0.f, 0.f));
-      m = fmaxf(m, fmaxf(fmaxf(a[k].x, a[k].y), fmaxf(a[k].z, a[k].w)));
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  return m;
-}
-
 // After a Newton-Schulz GEMM launch: turn each matrix's row / column sums into the
 // bound that fixes the next tensor scale, and clear the sums for their next use (one
 // CTA per matrix; the launch boundary orders the GEMM's sum atomics before the reads).

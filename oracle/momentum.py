@@ -8,7 +8,7 @@ the first moment, Hadamard mixing smooths the distribution before stochastic rou
 (SR) and adaptive 4/6 quantisation; Section 3.4: Q-Root's first-order momentum follows
 that storage recipe.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
   * Update: m_t = fp32(fp32(beta * m_prev) + fp32(fp32(1 - beta) * g)), m_prev the
     decoded previous state (zero on the first step).
   * Storage: y = m_t H16^r (the FP32 butterfly of nvfp4.hadamard_rows with the caller's

@@ -9,7 +9,7 @@ one FP8 E4M3 scale per block of 1x16 elements, one FP32 tensor scale s_g, and
 x_hat = x_E2M1 * s * s_g.  Section 3.4 and the "Others" paragraph of Section 2:
 all quantisations round to nearest (RTN).
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
   * RTN is IEEE round-to-nearest, ties to the even code, saturating at the
     largest finite value (E2M1: 6, E4M3: 448).
   * Block scale s_b = RN_e4m3( fp32( amax_b / fp32(6 * s_g) ) ); element code

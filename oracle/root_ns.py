@@ -20,7 +20,7 @@ Source: "Full-Stack FP4" (arXiv 2607.04422).
     clamp at clip_k * RMS of the normalised matrix (the default), and a hard clamp
     at the q-quantile of |X_0| (clip_quantile = q).
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
   * Frobenius normalisation X_0 = G / (||G||_F + eps), eps = 1e-7, ||G||_F
     accumulated in float64; inv = fp32(1 / (||G||_F + eps)) and X_0 = fp32(G * inv).
   * Clip: tau = fp32(clip_k * ||G||_F * inv / sqrt(m n)), X_0 = clamp(X_0, -tau, tau).
