@@ -233,7 +233,8 @@ typedef struct {
 /* Workspace bytes fs4_root_ns needs for one m x n matrix. */
 size_t fs4_root_ns_workspace_size(int64_t m, int64_t n);
 
-/* Workspace bytes fs4_root_ns_batched needs for `count` matrices (host array). */
+/* Workspace bytes fs4_root_ns_batched (and _ex, _nvfp4) needs for `count` matrices
+ * (host array); it depends on the shapes only (pointers may be null or overlap). */
 size_t fs4_root_ns_batched_workspace_size(int32_t count, const fs4_ns_desc* descs);
 
 /* Direct NVFP4 Newton-Schulz step (Section 3.4) on one FP32 momentum matrix.
@@ -269,6 +270,32 @@ fs4_status fs4_root_ns_batched(int32_t count, const fs4_ns_desc* descs, int32_t 
 fs4_status fs4_root_ns_batched_ex(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
                                   uint32_t flags, const uint16_t* rht_masks, void* workspace,
                                   size_t workspace_bytes, void* stream);
+
+/* An NVFP4 first-moment state, as fs4_momentum_nvfp4 writes it: PLAIN 1x16 row blocks
+ * (codes m x n/2 bytes, scales m x n/16 bytes, both 16-byte aligned; s_g one device
+ * float) of m_t H16^r, with `mask` the sign mask of its H16^r. */
+typedef struct {
+  const uint8_t* codes;
+  const uint8_t* scales;
+  const float* s_g;
+  uint32_t mask;
+} fs4_nvfp4_state;
+
+/* fs4_root_ns_batched_ex on matrices given as NVFP4 first-moment states instead of FP32
+ * (the Newton-Schulz step consumes the stored momentum directly; Section 3.4: "The
+ * first-order momentum follows the first-moment storage recipe in Section 3.3").
+ * descs[i].G must be null and descs[i].ld is ignored; matrix i is the state states[i],
+ * decoded as fs4_momentum_nvfp4 decodes its previous state (fp32(fp32(code * s) * s_g)
+ * on each block, then (H16^r)^-1 = H16 D / 4), read by the reduction and the preamble in
+ * place of G.  Everything else (shapes, flags, masks, workspace, outputs) is as for
+ * fs4_root_ns_batched_ex; the workspace size and layout queries accept descriptors
+ * with a null G.  Errors as there; also FS4_ERR_INVALID_ARG for a null states array, a
+ * non-null G, or a state with null or misaligned pointers or mask > 0xFFFF. */
+fs4_status fs4_root_ns_batched_nvfp4(int32_t count, const fs4_ns_desc* descs,
+                                     const fs4_nvfp4_state* states, int32_t K, float clip_k,
+                                     uint32_t flags, const uint16_t* rht_masks, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
 
 /* fs4_root_ns_batched_ex, with CUDA events recorded on `stream` around each
  * phase so a caller can time the kernels on the launching stream.

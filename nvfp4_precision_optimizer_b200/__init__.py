@@ -21,7 +21,7 @@ MUON_COEFFS = (3.4445, -4.7750, 2.0315)
 __all__ = [
     "quantize", "dequantize", "gemm", "root_ns", "root_ns_batched", "ns_workspace_size",
     "ns_batched_workspace_size", "ns_layout", "device_status", "tiled_shape", "Fs4Error",
-    "momentum_nvfp4",
+    "momentum_nvfp4", "root_ns_batched_nvfp4",
     "MUON_COEFFS", "stop_after", "FS4_AXIS_ROW", "FS4_AXIS_COL", "FS4_TEST_STALL",
     "FS4_NS_RHT", "FS4_NS_ADAPTIVE46", "FS4_NS_CLIP_QUANTILE",
 ]
@@ -241,6 +241,43 @@ def root_ns_batched(Gs: Sequence[torch.Tensor], K: int = 5, coeffs=None, clip_k:
                                             workspace.data_ptr(), workspace.numel(),
                                             _stream(stream)),
           "fs4_root_ns_batched_ex")
+    return outs
+
+
+def root_ns_batched_nvfp4(states, K: int = 5, coeffs=None, clip_k: float = 3.0,
+                          outs: Sequence[torch.Tensor] | None = None,
+                          workspace: torch.Tensor | None = None, flags: int = 0, stream=None,
+                          rht_masks=None, adaptive46: bool = False,
+                          clip_quantile: float | None = None):
+    """The Newton-Schulz step on matrices given as NVFP4 first-moment states
+    (fs4_root_ns_batched_nvfp4): each state is (codes, scales, s_g, mask) as
+    momentum_nvfp4 returns it (plus the mask it was stored with); the matrix is
+    codes.shape[0] x 2 * codes.shape[1].  Other arguments as root_ns_batched."""
+    if clip_quantile is not None:
+        flags |= FS4_NS_CLIP_QUANTILE
+        clip_k = clip_quantile
+    shapes = [(int(st[0].shape[0]), int(st[0].shape[1]) * 2) for st in states]
+    dev = states[0][0].device
+    if coeffs is None:
+        coeffs = [MUON_COEFFS] * len(states)
+    if outs is None:
+        outs = [torch.empty(sh, dtype=torch.float32, device=dev) for sh in shapes]
+    arr = (NsDesc * len(states))()
+    sts = (_lib.Nvfp4State * len(states))()
+    for i, (st, o, sh) in enumerate(zip(states, outs, shapes)):
+        a, b, c = coeffs[i]
+        arr[i] = NsDesc(None, o.data_ptr(), sh[0], sh[1], sh[1], _ld(o), a, b, c)
+        sts[i] = _lib.Nvfp4State(st[0].data_ptr(), st[1].data_ptr(), st[2].data_ptr(), int(st[3]))
+    need = int(_lib.lib().fs4_root_ns_batched_workspace_size(len(states), arr))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    flags |= (FS4_NS_RHT if rht_masks is not None else 0) | (FS4_NS_ADAPTIVE46 if adaptive46 else 0)
+    masks = _masks(rht_masks, K)
+    check(_lib.lib().fs4_root_ns_batched_nvfp4(len(states), arr, sts, K, clip_k, flags,
+                                               ctypes.cast(masks, ctypes.c_void_p) if masks else None,
+                                               workspace.data_ptr(), workspace.numel(),
+                                               _stream(stream)),
+          "fs4_root_ns_batched_nvfp4")
     return outs
 
 

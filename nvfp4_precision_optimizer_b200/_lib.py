@@ -38,6 +38,10 @@ class NsDesc(ctypes.Structure):
                 ("ld_out", c_i64), ("a", c_f32), ("b", c_f32), ("c", c_f32)]
 
 
+class Nvfp4State(ctypes.Structure):
+    _fields_ = [("codes", c_vp), ("scales", c_vp), ("s_g", c_vp), ("mask", c_u32)]
+
+
 class NsLayout(ctypes.Structure):
     _fields_ = [("mp", c_i64), ("np", c_i64), ("X", c_i64), ("A", c_i64),
                 ("qX_codes", c_i64 * 2), ("qX_scales", c_i64 * 2),
@@ -66,6 +70,8 @@ SIGNATURES = {
                                     c_sz, c_vp]),
     "fs4_root_ns_batched_ex": (c_i32, [c_i32, ctypes.POINTER(NsDesc), c_i32, c_f32, c_u32, c_vp,
                                        c_vp, c_sz, c_vp]),
+    "fs4_root_ns_batched_nvfp4": (c_i32, [c_i32, ctypes.POINTER(NsDesc), ctypes.POINTER(Nvfp4State),
+                                          c_i32, c_f32, c_u32, c_vp, c_vp, c_sz, c_vp]),
     "fs4_root_ns_batched_timed": (c_i32, [c_i32, ctypes.POINTER(NsDesc), c_i32, c_f32, c_u32,
                                           c_vp, c_vp, c_sz, c_vp, ctypes.POINTER(c_vp), c_i32]),
     "fs4_root_ns_noalloc": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i64, c_i32, c_f32, c_f32,

@@ -59,30 +59,46 @@ struct Plan {
   int64_t total_bytes = 0;
 };
 
-fs4_status validate_desc(const fs4_ns_desc& d) {
-  if (!d.G || !d.out) return FS4_ERR_INVALID_ARG;
+fs4_status validate_desc(const fs4_ns_desc& d, const fs4_nvfp4_state* st, bool sizing) {
+  if (sizing) {   // workspace size / layout queries: shapes only
+    if (d.m < 16 || d.n < 16 || d.m > FS4_MAX_DIM || d.n > FS4_MAX_DIM) return FS4_ERR_SHAPE;
+    if (d.m % 16 || d.n % 16) return FS4_ERR_SHAPE;
+    return FS4_OK;
+  }
+  if (st) {   // NVFP4 source: G is not read
+    if (d.G || !st->codes || !st->scales || !st->s_g || st->mask > 0xFFFFu) return FS4_ERR_INVALID_ARG;
+    if (!aligned(st->codes, 16) || !aligned(st->scales, 16) || !aligned(st->s_g, 4)) return FS4_ERR_INVALID_ARG;
+  } else if (!d.G) {
+    return FS4_ERR_INVALID_ARG;
+  }
+  if (!d.out) return FS4_ERR_INVALID_ARG;
   if (d.m < 16 || d.n < 16 || d.m > FS4_MAX_DIM || d.n > FS4_MAX_DIM) return FS4_ERR_SHAPE;
   if (d.m % 16 || d.n % 16) return FS4_ERR_SHAPE;
-  if (d.ld < d.n || d.ld_out < d.n) return FS4_ERR_INVALID_ARG;
+  if ((!st && d.ld < d.n) || d.ld_out < d.n) return FS4_ERR_INVALID_ARG;
   if (!std::isfinite(d.a) || !std::isfinite(d.b) || !std::isfinite(d.c)) return FS4_ERR_INVALID_ARG;
-  if (!aligned(d.G, 4) || !aligned(d.out, 4)) return FS4_ERR_INVALID_ARG;
+  if ((!st && !aligned(d.G, 4)) || !aligned(d.out, 4)) return FS4_ERR_INVALID_ARG;
   return FS4_OK;
 }
 
 // Lay out the workspace: [header | state blocks of all matrices | big buffers of all matrices].
-fs4_status make_plan(int32_t count, const fs4_ns_desc* descs, Plan* pl) {
+fs4_status make_plan(int32_t count, const fs4_ns_desc* descs, Plan* pl,
+                     const fs4_nvfp4_state* states = nullptr, bool sizing = false) {
   if (count < 1 || count > kMaxBatch) return FS4_ERR_SHAPE;
   if (!descs) return FS4_ERR_INVALID_ARG;
   pl->count = count;
   int64_t off = kHeaderBytes;
   for (int i = 0; i < count; ++i) {
     const fs4_ns_desc& d = descs[i];
-    const fs4_status s = validate_desc(d);
+    const fs4_status s = validate_desc(d, states ? &states[i] : nullptr, sizing);
     if (s != FS4_OK) return s;
     MatDesc& md = pl->mat[i];
     md.G = d.G;
     md.out = d.out;
-    md.ldg = d.ld;
+    md.ldg = states ? d.n : d.ld;
+    md.qcodes = states ? states[i].codes : nullptr;
+    md.qscales = states ? states[i].scales : nullptr;
+    md.qsg = states ? states[i].s_g : nullptr;
+    md.qmask = states ? states[i].mask : 0u;
     md.ldo = d.ld_out;
     md.tall = d.m > d.n ? 1 : 0;
     md.m = (int32_t)(md.tall ? d.n : d.m);
@@ -106,13 +122,22 @@ fs4_status make_plan(int32_t count, const fs4_ns_desc* descs, Plan* pl) {
     off += align_up(big_block_bytes(pl->mat[i].mp, pl->mat[i].np), 1024);
   }
   pl->total_bytes = off;
+  if (sizing) return FS4_OK;
   // outputs must not overlap any input or any other output
   for (int i = 0; i < count; ++i) {
     uintptr_t olo, ohi;
     span(descs[i].out, descs[i].m, descs[i].n, descs[i].ld_out, &olo, &ohi);
     for (int k = 0; k < count; ++k) {
       uintptr_t glo, ghi;
-      span(descs[k].G, descs[k].m, descs[k].n, descs[k].ld, &glo, &ghi);
+      if (states) {   // the NVFP4 codes and scales are the inputs
+        glo = reinterpret_cast<uintptr_t>(states[k].codes);
+        ghi = glo + (uintptr_t)(descs[k].m * descs[k].n / 2);
+        if (olo < ghi && glo < ohi) return FS4_ERR_ALIAS;
+        glo = reinterpret_cast<uintptr_t>(states[k].scales);
+        ghi = glo + (uintptr_t)(descs[k].m * descs[k].n / 16);
+      } else {
+        span(descs[k].G, descs[k].m, descs[k].n, descs[k].ld, &glo, &ghi);
+      }
       if (olo < ghi && glo < ohi) return FS4_ERR_ALIAS;
       if (k != i) {
         span(descs[k].out, descs[k].m, descs[k].n, descs[k].ld_out, &glo, &ghi);
@@ -295,7 +320,7 @@ fs4_status fs4_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const
 
 size_t fs4_root_ns_batched_workspace_size(int32_t count, const fs4_ns_desc* descs) {
   static thread_local Plan pl;
-  if (make_plan(count, descs, &pl) != FS4_OK) return 0;
+  if (make_plan(count, descs, &pl, nullptr, true) != FS4_OK) return 0;
   return (size_t)pl.total_bytes;
 }
 
@@ -310,7 +335,7 @@ size_t fs4_root_ns_workspace_size(int64_t m, int64_t n) {
 static fs4_status batched_impl(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
                                uint32_t flags, const uint16_t* rht_masks, void* workspace,
                                size_t workspace_bytes, void* stream, void* const* events,
-                               int32_t n_events) {
+                               int32_t n_events, const fs4_nvfp4_state* states = nullptr) {
   if (K < 1 || K > FS4_MAX_ITERS) return FS4_ERR_SHAPE;
   if (!std::isfinite(clip_k)) return FS4_ERR_INVALID_ARG;
   if (flags & ~(uint32_t)(0xFF00u | FS4_TEST_STALL | FS4_NS_RHT | FS4_NS_ADAPTIVE46 |
@@ -319,7 +344,7 @@ static fs4_status batched_impl(int32_t count, const fs4_ns_desc* descs, int32_t 
   if ((flags & FS4_NS_CLIP_QUANTILE) && !(clip_k > 0.0f && clip_k <= 1.0f)) return FS4_ERR_INVALID_ARG;
   if ((flags & FS4_NS_RHT) && !rht_masks) return FS4_ERR_INVALID_ARG;
   static thread_local Plan pl;
-  const fs4_status s = make_plan(count, descs, &pl);
+  const fs4_status s = make_plan(count, descs, &pl, states);
   if (s != FS4_OK) return s;
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < (size_t)pl.total_bytes)
     return FS4_ERR_WORKSPACE;
@@ -327,7 +352,15 @@ static fs4_status batched_impl(int32_t count, const fs4_ns_desc* descs, int32_t 
   const uintptr_t wlo = reinterpret_cast<uintptr_t>(workspace), whi = wlo + (uintptr_t)pl.total_bytes;
   for (int i = 0; i < count; ++i) {
     uintptr_t lo, hi;
-    span(descs[i].G, descs[i].m, descs[i].n, descs[i].ld, &lo, &hi);
+    if (states) {
+      lo = reinterpret_cast<uintptr_t>(states[i].codes);
+      hi = lo + (uintptr_t)(descs[i].m * descs[i].n / 2);
+      if (lo < whi && wlo < hi) return FS4_ERR_ALIAS;
+      lo = reinterpret_cast<uintptr_t>(states[i].scales);
+      hi = lo + (uintptr_t)(descs[i].m * descs[i].n / 16);
+    } else {
+      span(descs[i].G, descs[i].m, descs[i].n, descs[i].ld, &lo, &hi);
+    }
     if (lo < whi && wlo < hi) return FS4_ERR_ALIAS;
     span(descs[i].out, descs[i].m, descs[i].n, descs[i].ld_out, &lo, &hi);
     if (lo < whi && wlo < hi) return FS4_ERR_ALIAS;
@@ -341,6 +374,15 @@ static fs4_status batched_impl(int32_t count, const fs4_ns_desc* descs, int32_t 
   if (ds != FS4_OK) return ds;
   return run_ns(pl, K, clip_k, flags, rht_masks, static_cast<uint8_t*>(workspace),
                 static_cast<cudaStream_t>(stream), di.num_sms, events);
+}
+
+fs4_status fs4_root_ns_batched_nvfp4(int32_t count, const fs4_ns_desc* descs,
+                                     const fs4_nvfp4_state* states, int32_t K, float clip_k,
+                                     uint32_t flags, const uint16_t* rht_masks, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  if (!states) return FS4_ERR_INVALID_ARG;
+  return batched_impl(count, descs, K, clip_k, flags, rht_masks, workspace, workspace_bytes, stream,
+                      nullptr, 0, states);
 }
 
 fs4_status fs4_root_ns_batched(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
@@ -405,7 +447,7 @@ fs4_status fs4_root_ns_layout(int32_t count, const fs4_ns_desc* descs, int32_t i
                               fs4_ns_layout* layout) {
   if (!layout) return FS4_ERR_INVALID_ARG;
   static thread_local Plan pl;
-  const fs4_status s = make_plan(count, descs, &pl);
+  const fs4_status s = make_plan(count, descs, &pl, nullptr, true);
   if (s != FS4_OK) return s;
   if (index < 0 || index >= count) return FS4_ERR_INVALID_ARG;
   const MatDesc& d = pl.mat[index];

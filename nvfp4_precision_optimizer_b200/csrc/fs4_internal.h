@@ -98,6 +98,12 @@ struct MatDesc {
   int32_t mp, np;          // padded to multiples of 256
   int32_t tall;            // 1: working X = G^T
   float a, b, c;
+  // NVFP4 source (G given as an NVFP4 state: PLAIN 1x16 row blocks of G H16^r, as the
+  // first-moment step stores it) or null (G is the FP32 matrix above)
+  const uint8_t* qcodes;
+  const uint8_t* qscales;
+  const float* qsg;
+  uint32_t qmask;
 };
 
 // Kernel parameters of one Newton-Schulz phase over a batch of matrices.

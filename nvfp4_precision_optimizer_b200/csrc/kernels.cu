@@ -312,6 +312,30 @@ __device__ __forceinline__ NsState* state_of(const NsParams& p, const MatDesc& d
 // like their bit patterns).
 __device__ __forceinline__ uint32_t abs_key(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
 
+// Elements c .. c + 3 of row r of a G given as an NVFP4 state (PLAIN 1x16 row blocks of
+// G H16^r with n0 columns, as the first-moment step stores it): fp32(fp32(code * s) * s_g),
+// then (H16^r)^-1 = H16 D / 4 across the quad of lanes holding the block.  c = 16 blk + 4q
+// with q = lane & 3 by construction of every caller; all 32 lanes call it, and lanes with
+// live = false (a whole quad at a time) contribute zeros.
+__device__ __forceinline__ void nvfp4_src_quad(const MatDesc& d, int64_t n0, int64_t r, int64_t c,
+                                               bool live, float (&v)[4]) {
+  const int q = threadIdx.x & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) v[j] = 0.0f;
+  if (live) {
+    const int64_t blk = r * (n0 / 16) + (c >> 4);
+    const uint32_t w = __ldg(reinterpret_cast<const uint16_t*>(d.qcodes) + 4 * blk + q);
+    const float sb = e4m3_to_f32(__ldg(d.qscales + blk));
+    const float sg = __ldg(d.qsg);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = __fmul_rn(__fmul_rn(e2m1_value((w >> (4 * j)) & 0xFu), sb), sg);
+  }
+  quad_butterfly(v, q);
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    v[j] = __uint_as_float(__float_as_uint(__fmul_rn(v[j], 0.25f)) ^ (((d.qmask >> (4 * q + j)) & 1u) << 31));
+}
+
 // Sum of G^2 (float64), max |G| and a non-finite flag per matrix; work unit =
 // 16 rows of one matrix in the caller's orientation.  The last CTA to finish a
 // matrix derives its normalisation and clip scalars and the tensor scale of X_0
@@ -339,7 +363,22 @@ __global__ void __launch_bounds__(kEwThreads) ns_reduce_kernel(const __grid_cons
     bool bad = false;
     for (int64_t r = r0; r < r0 + 16 && r < rows0; ++r) {
       const float* row = d.G + r * d.ldg;
-      if (vec) {
+      if (d.qcodes) {   // NVFP4 source: warp-uniform column steps (the decode is quad-wide)
+        for (int64_t c0 = 0; c0 < cols0; c0 += 4 * kEwThreads) {
+          const int64_t c = c0 + 4 * threadIdx.x;
+          float vv[4];
+          nvfp4_src_quad(d, cols0, r, c, c < cols0, vv);
+          if (c < cols0) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              bad |= !is_finite_bits(vv[e]);
+              mx = fmaxf(mx, fabsf(vv[e]));
+              s += (double)vv[e] * (double)vv[e];
+              if constexpr (kHist) atomicAdd(&hist[abs_key(vv[e]) >> 20], 1u);
+            }
+          }
+        }
+      } else if (vec) {
         for (int64_t c = 4 * threadIdx.x; c < cols0; c += 4 * kEwThreads) {
           const float4 v4 = __ldg(reinterpret_cast<const float4*>(row + c));
           const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
@@ -538,7 +577,19 @@ __global__ void __launch_bounds__(kEwThreads) ns_quantile_gather_kernel(const __
         const bool full = s_n > (uint32_t)(kGatherBuf - kGatherStep);
         __syncthreads();   // every thread has read s_n before any thread appends again
         if (full) flush();
-        if (vec) {   // cols0 is a multiple of 16: a float4 is wholly inside or outside the row
+        if (d.qcodes) {   // NVFP4 source: four quad-decoded elements per thread and step
+#pragma unroll 1
+          for (int k = 0; k < 4; ++k) {
+            const int64_t c = c0 + 4 * (threadIdx.x + k * kEwThreads);
+            const bool valid = c < cols0;
+            float v[4];
+            nvfp4_src_quad(d, cols0, r, c, valid, v);
+            append(abs_key(v[0]), valid);
+            append(abs_key(v[1]), valid);
+            append(abs_key(v[2]), valid);
+            append(abs_key(v[3]), valid);
+          }
+        } else if (vec) {   // cols0 is a multiple of 16: a float4 is wholly inside or outside the row
           float4 v[4];
           bool valid[4];
 #pragma unroll
@@ -652,7 +703,7 @@ __global__ void __launch_bounds__(kEwThreads, 4) ns_preamble_kernel(const __grid
     const int32_t rows_g = d.tall ? d.n : d.m, cols_g = d.tall ? d.m : d.n;
     const int32_t gr0 = d.tall ? j0 : i0, gc0 = d.tall ? i0 : j0;
     const bool vec = ((reinterpret_cast<uintptr_t>(d.G) & 15) == 0) && ((d.ldg & 3) == 0);
-    if (vec && gr0 + kT <= rows_g && gc0 + kT <= cols_g) {
+    if (!d.qcodes && vec && gr0 + kT <= rows_g && gc0 + kT <= cols_g) {
       pf_fast = true;
       const float* gtile = d.G + (int64_t)gr0 * d.ldg + gc0;
 #pragma unroll
@@ -710,6 +761,10 @@ __global__ void __launch_bounds__(kEwThreads, 4) ns_preamble_kernel(const __grid
       const int line = f >> 4, c4 = (f & 15) * 4;       // 64 lines of 64 floats
       float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       if (dead) {
+      } else if (d.qcodes) {   // NVFP4 source: the quad of lanes holding the block decodes it
+        nvfp4_src_quad(d, cols_g, gr0 + line, gc0 + c4, gr0 + line < rows_g && gc0 + c4 < cols_g, v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = fminf(fmaxf(__fmul_rn(v[e], inv), -tau), tau);
       } else if (cur_fast) {
         v[0] = cur[pass].x; v[1] = cur[pass].y; v[2] = cur[pass].z; v[3] = cur[pass].w;
 #pragma unroll

@@ -120,8 +120,9 @@ def test_batched_rejects_overlapping_outputs_and_bad_counts(F):
     arr = (F._lib.NsDesc * 2)()
     arr[0] = _desc(F, 1 << 30, 1 << 34, 32, 32)
     arr[1] = _desc(F, 1 << 31, (1 << 34) + 64, 32, 32)
+    # the size query looks at shapes only; the call itself rejects the overlapping outputs
     need = lib.fs4_root_ns_batched_workspace_size(2, arr)
-    assert need == 0   # overlapping outputs: no valid plan
+    assert need > 0 and need == F.ns_batched_workspace_size([(32, 32), (32, 32)])
     assert lib.fs4_root_ns_batched(2, arr, 5, 3.0, 0, 1 << 40, 1 << 30, None) == -3
     assert lib.fs4_root_ns_batched(0, arr, 5, 3.0, 0, 1 << 40, 1 << 30, None) == -2
     assert lib.fs4_root_ns_batched(225, arr, 5, 3.0, 0, 1 << 40, 1 << 30, None) == -2
@@ -210,3 +211,27 @@ def test_momentum_argument_errors(F):
     assert call(m=g + 1024) == -3                    # m_out overlaps g
     assert call(ws=W + 4) == -4
     assert call(wsb=wsz - 1) == -4
+
+
+def test_nvfp4_source_argument_errors(F):
+    """fs4_root_ns_batched_nvfp4 checks its states on the host, before any launch."""
+    lib = F._lib.lib()
+    nv = lib.fs4_root_ns_batched_nvfp4
+    arr = (F._lib.NsDesc * 1)()
+    arr[0] = F._lib.NsDesc(None, 1 << 34, 64, 96, 96, 96, 1.0, 0.0, 0.0)
+    st = (F._lib.Nvfp4State * 1)()
+    st[0] = F._lib.Nvfp4State(1 << 30, 1 << 31, 1 << 32, 0x1234)
+    need = lib.fs4_root_ns_batched_workspace_size(1, arr)   # a null G is fine for sizing
+    assert need > 0
+    W = 1 << 40
+    assert nv(1, arr, st, 5, 3.0, 0, None, W, need - 1, None) == -4       # accepted up to the size
+    assert nv(1, arr, None, 5, 3.0, 0, None, W, need, None) == -1         # no states
+    bad = (F._lib.Nvfp4State * 1)()
+    bad[0] = F._lib.Nvfp4State(1 << 30, (1 << 31) + 8, 1 << 32, 0)       # scales misaligned
+    assert nv(1, arr, bad, 5, 3.0, 0, None, W, need, None) == -1
+    bad[0] = F._lib.Nvfp4State(1 << 30, 1 << 31, 1 << 32, 1 << 16)       # mask too wide
+    assert nv(1, arr, bad, 5, 3.0, 0, None, W, need, None) == -1
+    arr[0] = F._lib.NsDesc(1 << 33, 1 << 34, 64, 96, 96, 96, 1.0, 0.0, 0.0)   # G must be null
+    assert nv(1, arr, st, 5, 3.0, 0, None, W, need, None) == -1
+    arr[0] = F._lib.NsDesc(None, (1 << 30) + 64, 64, 96, 96, 96, 1.0, 0.0, 0.0)  # out over the codes
+    assert nv(1, arr, st, 5, 3.0, 0, None, W, need, None) == -3

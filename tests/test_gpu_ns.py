@@ -293,3 +293,22 @@ def test_batch_of_random_shapes_matches_oracle(fs4):
         got = o.cpu().numpy()
         assert got.shape == G.shape
         assert rel_frob(got, R.root_ns(G, 2, *coef, clip_k=3.0)) <= 2e-2, G.shape
+
+
+def test_preamble_keeps_the_sign_of_negative_zeros(fs4):
+    """Exact -0.0 entries of G give -0.0 in X_0 and the sign code 0x8 in both views."""
+    G = momentum(64, 96, kind="gauss", seed=8)
+    rng = np.random.default_rng(8)
+    G[rng.random(G.shape) < 0.1] = -0.0
+    G[rng.random(G.shape) < 0.05] = 0.0
+    _, ws = run_gpu(fs4, G, 1, MUON, flags=fs4.stop_after(0))
+    lay = fs4.ns_layout([G.shape], 0)
+    X0, _, _, _ = R.normalise_and_clip(G, 3.0)
+    Xg = ws_f32(ws, lay.X, lay.mp * lay.np).reshape(lay.mp, lay.np)
+    assert np.array_equal(Xg[:64, :96].view(np.uint32), X0.view(np.uint32))
+    c, s, _ = Q.quantize_rows(X0)
+    gc, gs = view(ws, lay.qX_codes[0], lay.qX_scales[0], lay.mp, lay.np)
+    assert np.array_equal(gc[:64, :48], c) and np.array_equal(gs[:64, :6], s)
+    ct, st, _ = Q.quantize_cols(X0)
+    gc, gs = view(ws, lay.qXT_codes[0], lay.qXT_scales[0], lay.np, lay.mp)
+    assert np.array_equal(gc[:96, :32], ct) and np.array_equal(gs[:96, :4], st)

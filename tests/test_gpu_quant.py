@@ -29,6 +29,8 @@ def _inputs():
         "zeros_32x32": np.zeros((32, 32)),
         "tiny_negative_16x32": -np.abs(rng.standard_normal((16, 32))) * np.where(rng.random((16, 32)) < 0.5, 1e-3, 1.0),
         "large_2048x2048": rng.standard_normal((2048, 2048)),
+        # exact -0.0 entries keep their sign code (0x8); +0.0 gives 0x0
+        "signed_zeros_32x64": rng.choice([-0.0, 0.0, 1.0, -1.0, 5e-4, -5e-4], (32, 64)),
     }
     return {k: v.astype(np.float32) for k, v in cases.items()}
 
