@@ -178,7 +178,8 @@ fs4_status run_ns(const Plan& pl, int32_t K, float clip_k, uint32_t flags, const
   p.status = reinterpret_cast<uint32_t*>(ws);
   p.ws = ws;
   p.opts = ((flags & FS4_NS_RHT) ? kOptRht : 0u) | ((flags & FS4_NS_ADAPTIVE46) ? kOpt46 : 0u) |
-           ((flags & FS4_NS_CLIP_QUANTILE) ? kOptQuantile : 0u);
+           ((flags & FS4_NS_CLIP_QUANTILE) ? kOptQuantile : 0u) |
+           (pl.mat[0].qcodes ? kOptNvSrc : 0u);   // a call's matrices are all FP32 or all NVFP4
   if (flags & FS4_NS_RHT)
     for (int i = 0; i < 3 * K; ++i) p.rht[i] = rht_masks[i];
   std::memcpy(p.mat, pl.mat, sizeof(MatDesc) * pl.count);

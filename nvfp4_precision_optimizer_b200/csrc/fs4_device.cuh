@@ -232,41 +232,6 @@ __device__ __forceinline__ void rht16(float* x, uint32_t mask) {
   for (int i = 0; i < 16; ++i) x[i] = __fmul_rn(x[i], 0.25f);
 }
 
-// H16 butterfly of a 16-element block held by the four lanes of a quad, lane q owning
-// elements 4q .. 4q + 3 (lane q = lane & 3; all 32 lanes call it).  Strides 1 and 2 stay
-// inside a lane; strides 4 and 8 pair lane q with q ^ 1 and q ^ 2, the lower lane keeping
-// u + v and the upper u - v: the roundings of the one-thread butterfly of rht16.
-__device__ __forceinline__ void quad_butterfly(float (&x)[4], int q) {
-#pragma unroll
-  for (int j = 0; j < 4; j += 2) {
-    const float u = x[j], v = x[j + 1];
-    x[j] = __fadd_rn(u, v);
-    x[j + 1] = __fsub_rn(u, v);
-  }
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const float u = x[j], v = x[j + 2];
-    x[j] = __fadd_rn(u, v);
-    x[j + 2] = __fsub_rn(u, v);
-  }
-#pragma unroll
-  for (int m = 1; m <= 2; m <<= 1) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float p = __shfl_xor_sync(0xFFFFFFFFu, x[j], m);
-      x[j] = (q & m) ? __fsub_rn(p, x[j]) : __fadd_rn(x[j], p);
-    }
-  }
-}
-
-// Signed value of a 4-bit E2M1 code (sign bit 3), in plain arithmetic.
-__device__ __forceinline__ float e2m1_value(uint32_t nib) {
-  const uint32_t mag = nib & 7u;
-  const float v = mag < 4u ? 0.5f * (float)mag
-                           : (mag == 4u ? 2.0f : (mag == 5u ? 3.0f : (mag == 6u ? 4.0f : 6.0f)));
-  return (nib & 8u) ? -v : v;
-}
-
 // The 8 E2M1 values (signed) of one packed word as 4 f16x2: element 2i in the low
 // half of h[i] (byte i of w, low nibble first).
 __device__ __forceinline__ void e2m1_decode8(uint32_t w, uint32_t* h) {

@@ -109,6 +109,7 @@ struct MatDesc {
 // Kernel parameters of one Newton-Schulz phase over a batch of matrices.
 constexpr uint32_t kOptRht = 1u, kOpt46 = 2u;   // NsParams::opts
 constexpr uint32_t kOptQuantile = 4u;            // clip at the clip_k-quantile of |X_0|
+constexpr uint32_t kOptNvSrc = 8u;               // every G is an NVFP4 state (MatDesc::qcodes)
 
 struct NsParams {
   int32_t count;

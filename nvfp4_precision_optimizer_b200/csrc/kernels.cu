@@ -312,28 +312,22 @@ __device__ __forceinline__ NsState* state_of(const NsParams& p, const MatDesc& d
 // like their bit patterns).
 __device__ __forceinline__ uint32_t abs_key(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
 
-// Elements c .. c + 3 of row r of a G given as an NVFP4 state (PLAIN 1x16 row blocks of
-// G H16^r with n0 columns, as the first-moment step stores it): fp32(fp32(code * s) * s_g),
-// then (H16^r)^-1 = H16 D / 4 across the quad of lanes holding the block.  c = 16 blk + 4q
-// with q = lane & 3 by construction of every caller; all 32 lanes call it, and lanes with
-// live = false (a whole quad at a time) contribute zeros.
-__device__ __forceinline__ void nvfp4_src_quad(const MatDesc& d, int64_t n0, int64_t r, int64_t c,
-                                               bool live, float (&v)[4]) {
-  const int q = threadIdx.x & 3;
+// Block blk (16 elements from column 16 blk) of row r of a G given as an NVFP4 state
+// (PLAIN 1x16 row blocks of G H16^r with n0 columns, as the first-moment step stores it),
+// decoded by one thread: fp32(fp32(code * s) * s_g), then (H16^r)^-1 = H16 D / 4 (the
+// butterfly and * 0.25 of rht16 without signs, then the signs of the state's mask).
+__device__ __forceinline__ void nvfp4_src_block(const MatDesc& d, int64_t n0, int64_t r, int64_t blk,
+                                                float (&v)[16]) {
+  const int64_t b = r * (n0 / 16) + blk;
+  const uint2 w = __ldg(reinterpret_cast<const uint2*>(d.qcodes) + b);
+  const float sb = e4m3_to_f32(__ldg(d.qscales + b));
+  const float sg = __ldg(d.qsg);
+  e2m1_decode16(w.x, w.y, v);
 #pragma unroll
-  for (int j = 0; j < 4; ++j) v[j] = 0.0f;
-  if (live) {
-    const int64_t blk = r * (n0 / 16) + (c >> 4);
-    const uint32_t w = __ldg(reinterpret_cast<const uint16_t*>(d.qcodes) + 4 * blk + q);
-    const float sb = e4m3_to_f32(__ldg(d.qscales + blk));
-    const float sg = __ldg(d.qsg);
+  for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(__fmul_rn(v[i], sb), sg);
+  rht16(v, 0u);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) v[j] = __fmul_rn(__fmul_rn(e2m1_value((w >> (4 * j)) & 0xFu), sb), sg);
-  }
-  quad_butterfly(v, q);
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    v[j] = __uint_as_float(__float_as_uint(__fmul_rn(v[j], 0.25f)) ^ (((d.qmask >> (4 * q + j)) & 1u) << 31));
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(__float_as_uint(v[i]) ^ (((d.qmask >> i) & 1u) << 31));
 }
 
 // Sum of G^2 (float64), max |G| and a non-finite flag per matrix; work unit =
@@ -342,7 +336,7 @@ __device__ __forceinline__ void nvfp4_src_quad(const MatDesc& d, int64_t n0, int
 // (Section 3.4: normalise, clip, quantise), so the preamble only reads them.
 // kHist (quantile clip): also a histogram of the top 11 bits of every |g| key,
 // accumulated per unit in shared memory and added to the matrix's histogram.
-template <bool kHist>
+template <bool kHist, bool kNv>
 __global__ void __launch_bounds__(kEwThreads) ns_reduce_kernel(const __grid_constant__ NsParams p) {
   __shared__ float redf[kEwThreads / 32];
   __shared__ double redd[kEwThreads / 32];
@@ -363,19 +357,16 @@ __global__ void __launch_bounds__(kEwThreads) ns_reduce_kernel(const __grid_cons
     bool bad = false;
     for (int64_t r = r0; r < r0 + 16 && r < rows0; ++r) {
       const float* row = d.G + r * d.ldg;
-      if (d.qcodes) {   // NVFP4 source: warp-uniform column steps (the decode is quad-wide)
-        for (int64_t c0 = 0; c0 < cols0; c0 += 4 * kEwThreads) {
-          const int64_t c = c0 + 4 * threadIdx.x;
-          float vv[4];
-          nvfp4_src_quad(d, cols0, r, c, c < cols0, vv);
-          if (c < cols0) {
+      if constexpr (kNv) {   // NVFP4 source: one thread per 16-element block
+        for (int64_t blk = threadIdx.x; blk < cols0 / 16; blk += kEwThreads) {
+          float vv[16];
+          nvfp4_src_block(d, cols0, r, blk, vv);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              bad |= !is_finite_bits(vv[e]);
-              mx = fmaxf(mx, fabsf(vv[e]));
-              s += (double)vv[e] * (double)vv[e];
-              if constexpr (kHist) atomicAdd(&hist[abs_key(vv[e]) >> 20], 1u);
-            }
+          for (int e = 0; e < 16; ++e) {
+            bad |= !is_finite_bits(vv[e]);
+            mx = fmaxf(mx, fabsf(vv[e]));
+            s += (double)vv[e] * (double)vv[e];
+            if constexpr (kHist) atomicAdd(&hist[abs_key(vv[e]) >> 20], 1u);
           }
         }
       } else if (vec) {
@@ -526,6 +517,7 @@ __global__ void __launch_bounds__(kEwThreads) ns_quantile_select1_kernel(const _
 // atomic per flush, so the matrix's counter sees a few atomics per unit, not one per warp.
 constexpr int kGatherBuf = 8192;            // staged keys per CTA
 constexpr int kGatherStep = 4 * 4 * kEwThreads;   // elements per column step (4 float4 per thread)
+template <bool kNv>
 __global__ void __launch_bounds__(kEwThreads) ns_quantile_gather_kernel(const __grid_constant__ NsParams p) {
   __shared__ uint32_t sbuf[kGatherBuf];
   __shared__ uint32_t s_n;
@@ -577,18 +569,18 @@ __global__ void __launch_bounds__(kEwThreads) ns_quantile_gather_kernel(const __
         const bool full = s_n > (uint32_t)(kGatherBuf - kGatherStep);
         __syncthreads();   // every thread has read s_n before any thread appends again
         if (full) flush();
-        if (d.qcodes) {   // NVFP4 source: four quad-decoded elements per thread and step
-#pragma unroll 1
-          for (int k = 0; k < 4; ++k) {
-            const int64_t c = c0 + 4 * (threadIdx.x + k * kEwThreads);
-            const bool valid = c < cols0;
-            float v[4];
-            nvfp4_src_quad(d, cols0, r, c, valid, v);
-            append(abs_key(v[0]), valid);
-            append(abs_key(v[1]), valid);
-            append(abs_key(v[2]), valid);
-            append(abs_key(v[3]), valid);
+        if constexpr (kNv) {   // NVFP4 source: one 16-element block per thread and step
+          const int64_t blk = c0 / 16 + threadIdx.x;
+          const bool valid = blk < cols0 / 16;
+          float v[16];
+          if (valid) {
+            nvfp4_src_block(d, cols0, r, blk, v);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = 0.0f;
           }
+#pragma unroll
+          for (int e = 0; e < 16; ++e) append(abs_key(v[e]), valid);
         } else if (vec) {   // cols0 is a multiple of 16: a float4 is wholly inside or outside the row
           float4 v[4];
           bool valid[4];
@@ -703,7 +695,7 @@ __global__ void __launch_bounds__(kEwThreads, 4) ns_preamble_kernel(const __grid
     const int32_t rows_g = d.tall ? d.n : d.m, cols_g = d.tall ? d.m : d.n;
     const int32_t gr0 = d.tall ? j0 : i0, gc0 = d.tall ? i0 : j0;
     const bool vec = ((reinterpret_cast<uintptr_t>(d.G) & 15) == 0) && ((d.ldg & 3) == 0);
-    if (!d.qcodes && vec && gr0 + kT <= rows_g && gc0 + kT <= cols_g) {
+    if (!(kOpts & kOptNvSrc) && vec && gr0 + kT <= rows_g && gc0 + kT <= cols_g) {
       pf_fast = true;
       const float* gtile = d.G + (int64_t)gr0 * d.ldg + gc0;
 #pragma unroll
@@ -755,16 +747,35 @@ __global__ void __launch_bounds__(kEwThreads, 4) ns_preamble_kernel(const __grid
     const int32_t gr0 = d.tall ? j0 : i0, gc0 = d.tall ? i0 : j0;   // tile origin in G
     const float* gtile = d.G + (int64_t)gr0 * d.ldg + gc0;
     float* Xt = reinterpret_cast<float*>(p.ws + L.X) + (int64_t)i0 * d.np + j0;
+    if constexpr ((kOpts & kOptNvSrc) != 0) {
+      // NVFP4 source: thread t decodes block t % 4 of G row t / 4 of the tile
+      const int line = t >> 2, blk = t & 3;
+      float v[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[e] = 0.0f;
+      if (!dead && gr0 + line < rows_g && gc0 + 16 * blk < cols_g) {
+        nvfp4_src_block(d, cols_g, gr0 + line, gc0 / 16 + blk, v);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = fminf(fmaxf(__fmul_rn(v[e], inv), -tau), tau);
+      }
+      if (!d.tall) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float4 v4 = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+          *reinterpret_cast<float4*>(tile + pre_off(line, 16 * blk + 4 * k)) = v4;
+          *reinterpret_cast<float4*>(Xt + line * d.np + 16 * blk + 4 * k) = v4;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) tile[pre_off(16 * blk + e, line)] = v[e];
+      }
+    } else {
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass) {
       const int f = t + kEwThreads * pass;
       const int line = f >> 4, c4 = (f & 15) * 4;       // 64 lines of 64 floats
       float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       if (dead) {
-      } else if (d.qcodes) {   // NVFP4 source: the quad of lanes holding the block decodes it
-        nvfp4_src_quad(d, cols_g, gr0 + line, gc0 + c4, gr0 + line < rows_g && gc0 + c4 < cols_g, v);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) v[e] = fminf(fmaxf(__fmul_rn(v[e], inv), -tau), tau);
       } else if (cur_fast) {
         v[0] = cur[pass].x; v[1] = cur[pass].y; v[2] = cur[pass].z; v[3] = cur[pass].w;
 #pragma unroll
@@ -783,6 +794,7 @@ __global__ void __launch_bounds__(kEwThreads, 4) ns_preamble_kernel(const __grid
 #pragma unroll
         for (int e = 0; e < 4; ++e) tile[pre_off(c4 + e, line)] = v[e];
       }
+    }
     }
     __syncthreads();
     if (d.tall) {
@@ -924,10 +936,20 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const
 }
 
 cudaError_t launch_ns_reduce(const NsParams& p, cudaStream_t st, int num_sms) {
-  if (p.opts & kOptQuantile)
-    ns_reduce_kernel<true><<<persistent_grid(ns_reduce_kernel<true>, p.prefix[p.count], num_sms), kEwThreads, 0, st>>>(p);
-  else
-    ns_reduce_kernel<false><<<persistent_grid(ns_reduce_kernel<false>, p.prefix[p.count], num_sms), kEwThreads, 0, st>>>(p);
+  const unsigned units = (unsigned)p.prefix[p.count];
+  switch (p.opts & (kOptQuantile | kOptNvSrc)) {
+    case kOptQuantile:
+      ns_reduce_kernel<true, false><<<persistent_grid(ns_reduce_kernel<true, false>, units, num_sms), kEwThreads, 0, st>>>(p);
+      break;
+    case kOptNvSrc:
+      ns_reduce_kernel<false, true><<<persistent_grid(ns_reduce_kernel<false, true>, units, num_sms), kEwThreads, 0, st>>>(p);
+      break;
+    case kOptQuantile | kOptNvSrc:
+      ns_reduce_kernel<true, true><<<persistent_grid(ns_reduce_kernel<true, true>, units, num_sms), kEwThreads, 0, st>>>(p);
+      break;
+    default:
+      ns_reduce_kernel<false, false><<<persistent_grid(ns_reduce_kernel<false, false>, units, num_sms), kEwThreads, 0, st>>>(p);
+  }
   return cudaGetLastError();
 }
 
@@ -936,8 +958,12 @@ cudaError_t launch_ns_quantile(const NsParams& p, cudaStream_t st, int num_sms) 
   ns_quantile_select1_kernel<<<p.count, kEwThreads, 0, st>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  ns_quantile_gather_kernel<<<persistent_grid(ns_quantile_gather_kernel, p.prefix[p.count], num_sms),
-                              kEwThreads, 0, st>>>(p);
+  if (p.opts & kOptNvSrc)
+    ns_quantile_gather_kernel<true><<<persistent_grid(ns_quantile_gather_kernel<true>, p.prefix[p.count], num_sms),
+                                      kEwThreads, 0, st>>>(p);
+  else
+    ns_quantile_gather_kernel<false><<<persistent_grid(ns_quantile_gather_kernel<false>, p.prefix[p.count], num_sms),
+                                       kEwThreads, 0, st>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   ns_quantile_select2_kernel<<<p.count, kSelThreads, 0, st>>>(p);
   return cudaGetLastError();
@@ -950,11 +976,15 @@ void preamble_launch(const NsParams& p, cudaStream_t st, int num_sms) {
 }
 
 cudaError_t launch_ns_preamble(const NsParams& p, cudaStream_t st, int num_sms) {
-  switch (p.opts & (kOptRht | kOpt46)) {
+  switch (p.opts & (kOptRht | kOpt46 | kOptNvSrc)) {
     case 0: preamble_launch<0>(p, st, num_sms); break;
     case kOpt46: preamble_launch<kOpt46>(p, st, num_sms); break;
     case kOptRht: preamble_launch<kOptRht>(p, st, num_sms); break;
-    default: preamble_launch<kOptRht | kOpt46>(p, st, num_sms); break;
+    case kOptRht | kOpt46: preamble_launch<kOptRht | kOpt46>(p, st, num_sms); break;
+    case kOptNvSrc: preamble_launch<kOptNvSrc>(p, st, num_sms); break;
+    case kOptNvSrc | kOpt46: preamble_launch<kOptNvSrc | kOpt46>(p, st, num_sms); break;
+    case kOptNvSrc | kOptRht: preamble_launch<kOptNvSrc | kOptRht>(p, st, num_sms); break;
+    default: preamble_launch<kOptNvSrc | kOptRht | kOpt46>(p, st, num_sms); break;
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
