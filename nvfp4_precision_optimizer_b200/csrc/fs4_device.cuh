@@ -199,10 +199,14 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
   return r;
 }
-// div_rn_fma on a pair: nd = (-d, -d), rcp = (RN(1/d), RN(1/d)).
-__device__ __forceinline__ uint64_t div2_rn_fma(uint64_t x, uint64_t nd, uint64_t rcp) {
-  const uint64_t q0 = f2_mul(x, rcp);
-  return f2_fma(f2_fma(q0, nd, x), rcp, q0);
+// -RN(x / d) on a pair, by the same correction written for the negated quotient:
+// nq0 = x * (-rcp) = -q0, r = x + d * nq0 = x - q0 d (exact), result nq0 - r * rcp.
+// d2 = (d, d), nrcp = (-RN(1/d), -RN(1/d)).  A zero residual is +0, so the correction
+// never changes a zero quotient, whose sign is the opposite of x's (-(+0) for x = +0
+// and +0 for x = -0).
+__device__ __forceinline__ uint64_t ndiv2_rn_fma(uint64_t x, uint64_t d2, uint64_t nrcp) {
+  const uint64_t nq0 = f2_mul(x, nrcp);
+  return f2_fma(f2_fma(nq0, d2, x), nrcp, nq0);
 }
 
 // Quantise 16 FP32 values with tensor scale s_g (six_sg = fp32(6 * s_g)).
@@ -306,24 +310,31 @@ __device__ __forceinline__ QBlock16 quantize16(const float* x, float s_g, float 
       if (kPow2) rcp = __frcp_rn(den);
     }
     float q[16];
-    if (kPow2 && kPacked) {
-      const uint64_t nd2 = f2_pack(-den, -den), rcp2 = f2_pack(rcp, rcp);
+    if constexpr (kPow2) {
+      // the FMA-corrected quotient in negated form (ndiv2_rn_fma): a zero quotient then
+      // carries the opposite of x's sign, so flipping every code's sign bit afterwards
+      // gives each element x's sign, -0 included (the plain form turns x = -0 into +0)
+      if constexpr (kPacked) {
+        const uint64_t d2 = f2_pack(den, den), nrcp2 = f2_pack(-rcp, -rcp);
 #pragma unroll
-      for (int i = 0; i < 16; i += 2)
-        f2_unpack(div2_rn_fma(f2_pack(x[i], x[i + 1]), nd2, rcp2), q[i], q[i + 1]);
-      // the FMA correction turns x = -0 into +0 (+0 + -0 rounds to +0); the quotient's
-      // sign is x's (den > 0), and a -0 element must keep its sign code (0x8)
+        for (int i = 0; i < 16; i += 2)
+          f2_unpack(ndiv2_rn_fma(f2_pack(x[i], x[i + 1]), d2, nrcp2), q[i], q[i + 1]);
+      } else {
+        const float nrcp = -rcp;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) q[i] = copysignf(q[i], x[i]);
-    } else if (kPow2) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) q[i] = copysignf(div_rn_fma(x[i], den, rcp), x[i]);   // -0 as above
+        for (int i = 0; i < 16; ++i) {
+          const float nq0 = x[i] * nrcp;
+          q[i] = fmaf(fmaf(nq0, den, x[i]), nrcp, nq0);
+        }
+      }
+      r.w0 = pack8_e2m1(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]) ^ 0x88888888u;
+      r.w1 = pack8_e2m1(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]) ^ 0x88888888u;
     } else {
 #pragma unroll
       for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(x[i], den);
+      r.w0 = pack8_e2m1(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+      r.w1 = pack8_e2m1(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
     }
-    r.w0 = pack8_e2m1(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
-    r.w1 = pack8_e2m1(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
     const float s4 = static_cast<float>(sq4_e2m1_sum8(r.w0) + sq4_e2m1_sum8(r.w1));
     r.sumsq = 0.25f * s4 * den * den;
   };
