@@ -133,6 +133,21 @@ __host__ __device__ __forceinline__ float pow2_tensor_scale(float u, bool for46 
 }
 
 // ------------------------------------------------------------------ block quantiser
+// max(|a|, |b|, |c|) in one instruction (sm_100's three-input max with .abs); NaN
+// operands are ignored as by fmaxf.
+__device__ __forceinline__ float absmax3(float a, float b, float c) {
+  float r;
+  asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// max |x_i| of a 16-element block: a three-level tree of three-input maxima.
+__device__ __forceinline__ float absmax16(const float* x) {
+  const float m0 = absmax3(x[0], x[1], x[2]), m1 = absmax3(x[3], x[4], x[5]);
+  const float m2 = absmax3(x[6], x[7], x[8]), m3 = absmax3(x[9], x[10], x[11]);
+  const float m4 = absmax3(x[12], x[13], x[14]);
+  return fmaxf(absmax3(m0, m1, m2), absmax3(m3, m4, x[15]));
+}
+
 struct QBlock16 {
   uint32_t w0, w1;   // 16 codes, element 0 in the low nibble of w0
   uint32_t scale;    // E4M3 byte
@@ -284,13 +299,7 @@ __device__ __forceinline__ QBlock16 quantize16(const float* x, float s_g, float 
                                                ScaleTab st = ScaleTab{nullptr, 0.0f}) {
   static_assert(kPow2 || !k46, "adaptive 4/6 needs a power-of-two tensor scale");
   static_assert(kPow2 || !kTab, "the scale table needs a power-of-two tensor scale");
-  // max |x| as a tree (depth 4 instead of a 16-long dependency chain)
-  float m8[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fabsf(x[i]), fabsf(x[i + 8]));
-#pragma unroll
-  for (int i = 0; i < 4; ++i) m8[i] = fmaxf(m8[i], m8[i + 4]);
-  const float amax = fmaxf(fmaxf(m8[0], m8[2]), fmaxf(m8[1], m8[3]));
+  const float amax = absmax16(x);
   // one candidate: block scale byte from the scaled amax, codes, den = value(scale) * s_g
   auto candidate = [&](float scaled_amax, QBlock16& r, float& den) {
     r.amax = amax;

@@ -518,8 +518,7 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
           QBlock16 q, qc;
           float yamax = 0.0f;   // max |X'| of the untransformed block (update bound)
           if constexpr (kRht && E == Epi::Update) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) yamax = fmaxf(yamax, fabsf(y[e]));
+            yamax = absmax16(y);
           }
           if constexpr (kRht) rht16(y, mask_row);
           if (need_col) {
