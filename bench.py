@@ -54,6 +54,10 @@ def parse_args():
     ap.add_argument("--clip", default="rms", choices=["rms", "p99"],
                     help="clip rule of the preamble: 3 x RMS (default) or the 0.99 quantile of "
                          "|X_0| (Section 3.4 p99 outlier clipping, FS4_NS_CLIP_QUANTILE)")
+    ap.add_argument("--graph", action="store_true",
+                    help="ns: capture one call in a CUDA graph and replay it per step (for the "
+                         "launch-bound small workloads; per-phase times then come from a "
+                         "separate untimed pass of the event-recording call)")
     ap.add_argument("--quant", default="plain", choices=["plain", "rht46", "rht", "a46"],
                     help="quantiser of the step: plain NVFP4 (default) or the Section 3.4 options "
                          "(random Hadamard transform with fresh seeded sign masks, adaptive 4/6)")
@@ -360,45 +364,91 @@ def main():
         clip_arg = 0.99
     mask_rng = np.random.default_rng(BASE_SEED + 7)
 
+    if args.graph and qflags & F.FS4_NS_RHT:
+        raise SystemExit("--graph: a captured call would replay the same H16^r signs every step")
+
     def call(events=None):
         masks = None
         if qflags & F.FS4_NS_RHT:        # fresh signs for every step (Section 3.4)
             masks = (ctypes.c_uint16 * (3 * K))(*[int(v) for v in mask_rng.integers(0, 1 << 16, 3 * K)])
         mptr = ctypes.cast(masks, ctypes.c_void_p) if masks is not None else None
+        cur = torch.cuda.current_stream().cuda_stream   # the capture stream under --graph
         if events is None:
             st = lib.fs4_root_ns_batched_ex(len(Gs), arr, K, clip_arg, qflags, mptr, ws.data_ptr(),
-                                            need, stream.cuda_stream)
+                                            need, cur)
         else:
             ev_arr = (F._lib.c_vp * n_ev)(*[e.cuda_event for e in events])
             st = lib.fs4_root_ns_batched_timed(len(Gs), arr, K, clip_arg, qflags, mptr, ws.data_ptr(),
-                                               need, stream.cuda_stream, ev_arr, n_ev)
+                                               need, cur, ev_arr, n_ev)
         F.check(st, "fs4_root_ns_batched")
 
     for _ in range(max(3, args.warmup)):
         call()
     torch.cuda.synchronize()
     F.check(F.device_status(ws), "device status after warm-up")
+    graph = None
+    if args.graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            call()
+        for _ in range(max(3, args.warmup)):
+            graph.replay()
+        torch.cuda.synchronize()
+        F.check(F.device_status(ws), "device status after graph warm-up")
 
     step_events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     for evs in step_events:          # torch creates the CUDA event on its first record
         for e in evs:
             e.record(stream)
+    # Inputs that fit in L2 would be read from L2 by the next step: then L2 is flushed
+    # (a zero-fill of twice its size) before every step, and the step time is taken from
+    # the events around each call, so that the fill stays outside the timed work.
+    in_bytes = sum(G.numel() for G in Gs) * 4
+    l2_bytes = int(torch.cuda.get_device_properties(local).L2_cache_size)
+    flush = torch.empty(2 * l2_bytes, dtype=torch.uint8, device="cuda") if in_bytes <= 2 * l2_bytes else None
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(local)
+    replay_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                     for _ in range(args.steps)] if graph is not None else []
     with sampler:
         time.sleep(0.3)
         t_start.record(stream)
         for s in range(args.steps):
-            call(step_events[s])
+            if flush is not None:
+                flush.zero_()
+            if graph is not None:
+                replay_events[s][0].record(stream)
+                graph.replay()
+                replay_events[s][1].record(stream)
+            else:
+                call(step_events[s])
         t_end.record(stream)
         torch.cuda.synchronize()
     barrier()
     F.check(F.device_status(ws), "device status after timed steps")
-    total_ms = ranks_max(t_start.elapsed_time(t_end))
+    if graph is not None:
+        total_ms = ranks_max(sum(a.elapsed_time(b) for a, b in replay_events))
+    elif flush is None:
+        total_ms = ranks_max(t_start.elapsed_time(t_end))
+    else:
+        total_ms = ranks_max(sum(evs[0].elapsed_time(evs[-1]) for evs in step_events))
+    if flush is None:
+        l2_note = "inputs larger than L2 (%.2f GB per step)" % (in_bytes / 1e9)
+    else:
+        l2_note = ("L2 flushed before every step (zero-fill of %d MB; inputs %.1f MB); step time "
+                   "from events around each call" % (2 * l2_bytes >> 20, in_bytes / 1e6))
     ms_step = total_ms / args.steps
+    if graph is not None:
+        # per-phase times (roofline entry): a separate, untimed pass of the event-recording call
+        for s in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            call(step_events[s])
+        torch.cuda.synchronize()
+        F.check(F.device_status(ws), "device status after the per-phase pass")
 
     # per-phase kernel durations (CUDA events on the launching stream)
     kinds = phase_kinds(K)
@@ -523,7 +573,10 @@ def main():
                                      "rht": "NVFP4 RTN with H16^r (fresh signs per step)",
                                      "a46": "NVFP4 RTN with adaptive 4/6"}[args.quant],
                        "parallelism": f"replicas x{world} (independent matrices, no collective)",
-                       "l2": "inputs larger than L2 (%.2f GB per step)" % (sum(G.numel() for G in Gs) * 4 / 1e9)},
+                       "l2": l2_note,
+                       "launch": ("one CUDA graph replay per step (the call captured once); per-phase "
+                                  "times from a separate event-recording pass" if graph is not None
+                                  else "one library call per step (stream launches)")},
             "tflops_algorithmic": tflops,
             "frac_fp4_peak_algorithmic": tflops / world / fp4_peak,
             "tflops_dense_equivalent": world * w.flops_dense() / (ms_step * 1e-3) / 1e12,
@@ -715,7 +768,9 @@ def run_standalone(args, w, rank, world, local, barrier, ranks_max):
             "config": {"workload": w.name, "matrices": len(Gs), "op": args.op, "layout": args.layout,
                        "axis": "row (1x16 blocks)", "s_g": "power of two",
                        "parallelism": f"replicas x{world} (independent matrices, no collective)",
-                       "l2": "inputs larger than L2 (%.2f GB of FP32 per step)" % (elems * 4 / 1e9)},
+                       "l2": ("inputs larger than L2 (%.2f GB of FP32 per step)" % (elems * 4 / 1e9)
+                              if elems * 4 > torch.cuda.get_device_properties(local).L2_cache_size
+                              else "inputs of %.1f MB fit in L2 (not flushed)" % (elems * 4 / 1e6))},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * len(Gs) * (2 if args.op == "quantize" else 1),
             "clocks": sampler.summary(),
@@ -902,7 +957,9 @@ def run_momentum(args, w, rank, world, local, barrier, ranks_max):
             "config": {"workload": w.name, "matrices": len(Gs), "op": "momentum", "beta": 0.95,
                        "state": "previous state present, updated in place; m_t written in FP32",
                        "parallelism": f"replicas x{world} (independent matrices, no collective)",
-                       "l2": "inputs larger than L2 (%.2f GB of FP32 per step)" % (elems * 4 / 1e9)},
+                       "l2": ("inputs larger than L2 (%.2f GB of FP32 per step)" % (elems * 4 / 1e9)
+                              if elems * 4 > torch.cuda.get_device_properties(local).L2_cache_size
+                              else "inputs of %.1f MB fit in L2 (not flushed)" % (elems * 4 / 1e6))},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * len(Gs) * 2, "clocks": sampler.summary(),
         }), flush=True)
