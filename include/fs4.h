@@ -114,10 +114,12 @@ enum {
  * before the preamble writes X_0 there. */
 #define FS4_NS_CLIP_QUANTILE (1u << 4)
 
-/* Test-only flag for fs4_root_ns / fs4_root_ns_batched (no counterpart in the
- * paper): the MMA issuer of the first Gram product waits on a barrier that
- * nothing arrives on.  The bounded wait gives up after about 2 s, records the
- * timeout in the status word, and every later kernel of the call skips its work;
+/* Test-only flag for fs4_root_ns / fs4_root_ns_batched and fs4_nvfp4_quantize
+ * (no counterpart in the paper).  Newton-Schulz: the MMA issuer of the first
+ * Gram product waits on a barrier that nothing arrives on.  Quantise: the grid
+ * barrier between the amax pass and the quantise pass waits for one CTA more
+ * than the launch has.  The bounded wait gives up after about 2 s, records the
+ * timeout in the status word, and the rest of the call's work is skipped;
  * fs4_device_status then returns FS4_ERR_TIMEOUT and the outputs are undefined.
  * The CUDA context stays usable: no trap, fault or unbounded wait is involved.
  * It exists so that the device-side timeout path can be exercised on a GPU. */

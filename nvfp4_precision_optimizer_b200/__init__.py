@@ -52,8 +52,10 @@ def tiled_shape(rows: int, cols: int) -> tuple[int, int]:
 
 
 def quantize(x: torch.Tensor, axis: int = FS4_AXIS_ROW, tiled: bool = False,
-             sg_mode: str = "pow2", workspace: torch.Tensor | None = None, stream=None):
-    """NVFP4-quantise x (fs4_nvfp4_quantize).  Returns (codes, scales, s_g)."""
+             sg_mode: str = "pow2", workspace: torch.Tensor | None = None, stream=None,
+             flags: int = 0):
+    """NVFP4-quantise x (fs4_nvfp4_quantize).  Returns (codes, scales, s_g).
+    flags: extra call flags (FS4_TEST_STALL for the timeout test)."""
     _check_f32_matrix(x, "x")
     rows, cols = x.shape
     R, C = (rows, cols) if axis == FS4_AXIS_ROW else (cols, rows)
@@ -68,7 +70,7 @@ def quantize(x: torch.Tensor, axis: int = FS4_AXIS_ROW, tiled: bool = False,
     ws_bytes = _lib.lib().fs4_nvfp4_quantize_workspace_size()
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
-    flags = (FS4_LAYOUT_TILED if tiled else 0) | (FS4_SG_AMAX if sg_mode == "amax" else 0)
+    flags |= (FS4_LAYOUT_TILED if tiled else 0) | (FS4_SG_AMAX if sg_mode == "amax" else 0)
     ld = x.stride(0) if rows > 1 else cols
     check(_lib.lib().fs4_nvfp4_quantize(x.data_ptr(), rows, cols, ld, axis,
                                         codes.data_ptr(), scales.data_ptr(), s_g.data_ptr(), flags,

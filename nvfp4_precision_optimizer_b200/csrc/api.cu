@@ -261,7 +261,7 @@ fs4_status fs4_nvfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_
                               void* workspace, size_t workspace_bytes, void* stream) {
   if (!x || !codes || !scales || !s_g) return FS4_ERR_INVALID_ARG;
   if (axis != FS4_AXIS_ROW && axis != FS4_AXIS_COL) return FS4_ERR_INVALID_ARG;
-  if (flags & ~(uint32_t)(FS4_SG_AMAX | FS4_LAYOUT_TILED)) return FS4_ERR_INVALID_ARG;
+  if (flags & ~(uint32_t)(FS4_SG_AMAX | FS4_LAYOUT_TILED | FS4_TEST_STALL)) return FS4_ERR_INVALID_ARG;
   if (rows < 1 || cols < 1 || rows > (1ll << 31) || cols > (1ll << 31)) return FS4_ERR_SHAPE;
   if ((axis == FS4_AXIS_ROW ? cols : rows) % 16) return FS4_ERR_SHAPE;
   if (ld < cols) return FS4_ERR_INVALID_ARG;

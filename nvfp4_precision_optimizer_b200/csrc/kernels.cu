@@ -88,9 +88,9 @@ __device__ __forceinline__ void store_block_tiled(uint8_t* codes, uint8_t* scale
 }
 
 // ------------------------------------------------------------------ standalone quantise
-__global__ void __launch_bounds__(kEwThreads) amax_kernel(const float* __restrict__ x, int64_t rows,
-                                                          int64_t cols, int64_t ld,
-                                                          uint32_t* __restrict__ hdr) {
+// Pass 1: max |x| (hdr[1], as float bits) and a non-finite flag (hdr[0]) by atomics.
+__device__ __forceinline__ void amax_pass(const float* __restrict__ x, int64_t rows, int64_t cols,
+                                          int64_t ld, uint32_t* __restrict__ hdr) {
   __shared__ float red[kEwThreads / 32];
   float m = 0.0f;
   bool bad = false;
@@ -136,14 +136,14 @@ __global__ void __launch_bounds__(kEwThreads) amax_kernel(const float* __restric
   if (threadIdx.x == 0) atomicMax(&hdr[1], __float_as_uint(m));
 }
 
-// Quantise the R x C matrix Y (Y = x for the row axis, Y = x^T for the column
+// Pass 2: quantise the R x C matrix Y (Y = x for the row axis, Y = x^T for the column
 // axis) in 1x16 blocks along Y's rows.  Work unit = one 64 x 64 tile of Y's (padded)
 // extent, staged through shared memory so both axes read x with coalesced loads.
 // Persistent CTAs: the next unit's x tile is loaded into registers while the current
 // one is quantised (interior tiles of 16-byte aligned inputs; edge tiles load on the
 // guarded path).  Tiles are visited in x's row-major order, last tile first: the amax
 // pass just streamed x top to bottom, so the tail of x is still resident in L2.
-__global__ void __launch_bounds__(kEwThreads) quantize_kernel(
+__device__ __forceinline__ void quantize_pass(
     const float* __restrict__ x, int64_t ld, int64_t R, int64_t C, int col_axis, int tiled,
     int sg_amax_mode, int64_t Rext, int64_t Cext, int64_t Cp, int64_t ntiles,
     uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, float* __restrict__ s_g_out,
@@ -233,6 +233,54 @@ __global__ void __launch_bounds__(kEwThreads) quantize_kernel(
     }
     __syncthreads();   // the tile is restaged by the next unit
   }
+}
+
+// Arrive at a grid-wide barrier and wait (thread 0 of each CTA) until all `expected`
+// CTAs have arrived; the fence makes this CTA's earlier atomics visible to every CTA
+// that passes the barrier.  The wait is bounded: after kWaitLimitNs it records
+// kStatusTimeout and returns false (the CTA then skips the rest of its work).  Only
+// for cooperative launches, whose CTAs are all resident at once.
+__device__ __forceinline__ bool grid_barrier(uint32_t* count, uint32_t expected, uint32_t* status) {
+  __shared__ int passed;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(count, 1u);
+    const uint64_t t0 = global_timer_ns();
+    int ok = 0;
+    for (;;) {
+      uint32_t v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(count) : "memory");
+      if (v >= expected) { ok = 1; break; }
+      if (global_timer_ns() - t0 > kWaitLimitNs) { atomicOr(status, kStatusTimeout); break; }
+      __nanosleep(64);
+    }
+    passed = ok;
+  }
+  __syncthreads();
+  return passed != 0;
+}
+
+struct QuantArgs {
+  const float* x;
+  int64_t rows, cols, ld;             // x as given
+  int64_t R, C, Rext, Cext, Cp, ntiles;
+  int col_axis, tiled, sg_amax_mode;
+  int stall;                          // test only: the barrier waits for one CTA too many
+  uint8_t* codes;
+  uint8_t* scales;
+  float* s_g;
+  uint32_t* hdr;                      // [0] status, [1] amax bits, [2] barrier count (zeroed)
+};
+
+// Standalone quantise in one cooperative launch: the amax pass over x, a grid-wide
+// barrier, then the quantise pass.  The barrier takes the place of a second launch and
+// its ramp, and the quantise pass (last tile first) finds the tail of x in L2.
+__global__ void __launch_bounds__(kEwThreads) quantize_fused_kernel(const __grid_constant__ QuantArgs a) {
+  amax_pass(a.x, a.rows, a.cols, a.ld, a.hdr);
+  if (!grid_barrier(&a.hdr[2], gridDim.x + (a.stall ? 1u : 0u), &a.hdr[0])) return;
+  quantize_pass(a.x, a.ld, a.R, a.C, a.col_axis, a.tiled, a.sg_amax_mode, a.Rext, a.Cext, a.Cp,
+                a.ntiles, a.codes, a.scales, a.s_g, a.hdr);
 }
 
 // y = fp32(fp32(code * scale) * s_g), one thread per group of 4 consecutive elements
@@ -908,21 +956,30 @@ int persistent_grid(Kernel kernel, int64_t units, int num_sms) {
 cudaError_t launch_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld, int axis,
                             uint8_t* codes, uint8_t* scales, float* s_g, uint32_t flags,
                             uint8_t* ws, cudaStream_t st, int num_sms) {
-  cudaError_t e = cudaMemsetAsync(ws, 0, 8, st);
+  cudaError_t e = cudaMemsetAsync(ws, 0, 12, st);
   if (e != cudaSuccess) return e;
-  uint32_t* hdr = reinterpret_cast<uint32_t*>(ws);
-  const int64_t amax_units = std::max<int64_t>(rows, (rows * cols + 4095) / 4096);  // 4 float4 per thread
-  amax_kernel<<<persistent_grid(amax_kernel, amax_units, num_sms), kEwThreads, 0, st>>>(x, rows, cols, ld, hdr);
-  const int64_t R = axis ? cols : rows, C = axis ? rows : cols;
-  const int tiled = (flags & 2u) ? 1 : 0;
-  const int64_t Rext = tiled ? align_up(R, 128) : align_up(R, kT);
-  const int64_t Cp = align_up(C, 256);
-  const int64_t Cext = tiled ? Cp : align_up(C, kT);
-  const int64_t ntiles = (Rext / kT) * (Cext / kT);
-  if (ntiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
-  quantize_kernel<<<persistent_grid(quantize_kernel, ntiles, num_sms), kEwThreads, 0, st>>>(
-      x, ld, R, C, axis, tiled, (flags & 1u) ? 1 : 0, Rext, Cext, Cp, ntiles, codes, scales, s_g, hdr);
-  return cudaGetLastError();
+  QuantArgs a;
+  a.x = x; a.rows = rows; a.cols = cols; a.ld = ld;
+  a.R = axis ? cols : rows;
+  a.C = axis ? rows : cols;
+  a.tiled = (flags & 2u) ? 1 : 0;
+  a.Rext = a.tiled ? align_up(a.R, 128) : align_up(a.R, kT);
+  a.Cp = align_up(a.C, 256);
+  a.Cext = a.tiled ? a.Cp : align_up(a.C, kT);
+  a.ntiles = (a.Rext / kT) * (a.Cext / kT);
+  if (a.ntiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  a.col_axis = axis;
+  a.sg_amax_mode = (flags & 1u) ? 1 : 0;
+  a.stall = (flags & (1u << 30)) ? 1 : 0;   // FS4_TEST_STALL
+  a.codes = codes; a.scales = scales; a.s_g = s_g;
+  a.hdr = reinterpret_cast<uint32_t*>(ws);
+  // as many CTAs as are resident at once (a cooperative launch refuses more), fewer
+  // when neither pass has that much work (4 float4 per amax thread, one tile per unit)
+  const int64_t amax_units = std::max<int64_t>(rows, (rows * cols + 4095) / 4096);
+  const int grid = persistent_grid(quantize_fused_kernel, std::max<int64_t>(amax_units, a.ntiles), num_sms);
+  void* args[] = {&a};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(quantize_fused_kernel), dim3(grid),
+                                     dim3(kEwThreads), args, 0, st);
 }
 
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* s_g,

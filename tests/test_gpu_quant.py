@@ -100,6 +100,28 @@ def test_nonfinite_input_sets_device_status(fs4):
     assert fs4.device_status(ws) == 0
 
 
+def test_quantize_barrier_timeout_reports_status_and_context_survives(fs4):
+    """The quantise call's grid barrier (between its amax pass and its quantise pass)
+    is a bounded wait: with FS4_TEST_STALL it waits for one CTA more than the launch
+    has, gives up after about 2 s and records FS4_ERR_TIMEOUT, with no fault; the next
+    call on the same stream and workspace is bit-exact."""
+    import time
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((512, 1024)) * 0.02).astype(np.float32)
+    xd = torch.from_numpy(x).cuda()
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    t0 = time.time()
+    fs4.quantize(xd, workspace=ws, flags=fs4.FS4_TEST_STALL)
+    torch.cuda.synchronize()
+    assert time.time() - t0 < 30.0
+    assert fs4.device_status(ws) == -8          # FS4_ERR_TIMEOUT
+    codes, scales, sg = fs4.quantize(xd, workspace=ws)
+    assert fs4.device_status(ws) == 0
+    wc, wsc, wg = Q.quantize_rows(x)
+    assert np.array_equal(codes.cpu().numpy(), wc) and np.array_equal(scales.cpu().numpy(), wsc)
+    assert float(sg.item()) == float(wg)
+
+
 def _threshold_sweep():
     """Blocks whose scale decodes to each E4M3 mantissa 1 + m/8 and whose other
     15 elements sweep 2^14 consecutive FP32 values on both sides of every E2M1
