@@ -56,6 +56,8 @@ def test_quantize_rejects_bad_arguments_before_touching_the_device(F):
     assert q(fake, 4, 16, 16, 2, fake, fake, fake, 0, wsp, 256, None) == -1       # bad axis
     assert q(fake, 4, 16, 16, 0, fake + 8, fake, fake, 0, wsp, 256, None) == -1   # misaligned codes
     assert q(fake, 4, 16, 16, 0, fake, fake, fake, 1 << 7, wsp, 256, None) == -1  # unknown flag
+    # the test-only stall flag does not excuse another unknown bit
+    assert q(fake, 4, 16, 16, 0, fake, fake, fake, F.FS4_TEST_STALL | (1 << 7), wsp, 256, None) == -1
     assert q(fake, 4, 16, 16, 0, fake, fake, fake, 0, wsp, 100, None) == -4       # workspace too small
     assert q(fake, 4, 16, 16, 0, fake, fake, fake, 0, wsp + 8, 256, None) == -4   # misaligned workspace
 
