@@ -150,7 +150,11 @@ size_t fs4_nvfp4_quantize_workspace_size(void);
  *   Errors: FS4_ERR_SHAPE for empty or unaligned shapes; FS4_ERR_INVALID_ARG
  *   for null pointers, ld < cols, codes/scales not 16-byte aligned (TILED);
  *   FS4_ERR_WORKSPACE.  Non-finite input is recorded as FS4_ERR_NONFINITE in
- *   the workspace status word (outputs then undefined). */
+ *   the workspace status word (outputs then undefined).
+ *   One cooperative launch: a pass for the tensor amax, a grid-wide barrier
+ *   (a bounded wait: FS4_ERR_TIMEOUT in the status word if it runs out), then
+ *   the quantise pass.  The workspace holds the call's amax and barrier count,
+ *   so calls whose work may overlap on the GPU need separate workspaces. */
 fs4_status fs4_nvfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld,
                               int32_t axis, uint8_t* codes, uint8_t* scales, float* s_g,
                               uint32_t flags, void* workspace, size_t workspace_bytes,
