@@ -237,3 +237,36 @@ def test_nvfp4_source_argument_errors(F):
     assert nv(1, arr, st, 5, 3.0, 0, None, W, need, None) == -1
     arr[0] = F._lib.NsDesc(None, (1 << 30) + 64, 64, 96, 96, 96, 1.0, 0.0, 0.0)  # out over the codes
     assert nv(1, arr, st, 5, 3.0, 0, None, W, need, None) == -3
+
+
+def test_missing_library_fails_loudly():
+    """Without libfs4.so every call raises ImportError: there is no CPU or library
+    fallback.  Checked in a fresh interpreter whose loader points at a missing path."""
+    import subprocess
+    import sys
+    code = (
+        "import nvfp4_precision_optimizer_b200 as F\n"
+        "F._lib.LIB_PATH = '/nonexistent/libfs4.so'\n"
+        "F._lib._lib = None\n"
+        "import torch\n"
+        "# calls that reach the library first: ImportError\n"
+        "for call in (F._lib.lib, lambda: F.ns_workspace_size(256, 256),\n"
+        "             lambda: F.ns_batched_workspace_size([(256, 512)])):\n"
+        "    try:\n"
+        "        call()\n"
+        "    except ImportError:\n"
+        "        continue\n"
+        "    except Exception as e:\n"
+        "        raise SystemExit('wrong error: %r' % (e,))\n"
+        "    raise SystemExit('no error')\n"
+        "# compute calls on host tensors are refused before anything runs (no CPU path)\n"
+        "for call in (lambda: F.quantize(torch.zeros(16, 16)),\n"
+        "             lambda: F.root_ns(torch.zeros(16, 16))):\n"
+        "    try:\n"
+        "        call()\n"
+        "    except (ImportError, ValueError):\n"
+        "        continue\n"
+        "    raise SystemExit('a host tensor was accepted')\n"
+        "print('ok')\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
