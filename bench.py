@@ -194,9 +194,25 @@ def cpu_cores():
     return os.cpu_count() or 1
 
 
-def oracle_sample_rate(w, budget_s: float):
+QUANT_NAMES = {"plain": "NVFP4 RTN (H = I, M = 6)",
+               "rht46": "NVFP4 RTN with H16^r (fresh signs per step) and adaptive 4/6",
+               "rht": "NVFP4 RTN with H16^r (fresh signs per step)",
+               "a46": "NVFP4 RTN with adaptive 4/6"}
+
+
+def ns_config(w, quant: str, clip: str, world: int) -> dict:
+    """The workload keys of a Newton-Schulz bench line (the same for both arms)."""
+    return {"workload": w.name, "matrices": len(w.shapes), "shapes": sorted(set(map(tuple, w.shapes))),
+            "K": w.K, "coeffs": "Muon (3.4445, -4.7750, 2.0315)",
+            "clip": "3 x RMS" if clip == "rms" else "0.99 quantile of |X_0| (nearest rank)",
+            "quantiser": QUANT_NAMES[quant],
+            "parallelism": f"replicas x{world} (independent matrices, no collective)"}
+
+
+def oracle_sample_rate(w, budget_s: float, quant: str = "plain", clip: str = "rms"):
     """Time the oracle (as it stands) on one bounded sample of the workload:
-    one NVFP4 Newton-Schulz iteration of an m x n slice of its first matrix.
+    one NVFP4 Newton-Schulz iteration of an m x n slice of its first matrix, with the
+    quantiser options and clip rule of the run.
     Returns (matrices/s extrapolated by algorithmic FLOPs, seconds, description)."""
     import numpy as np
     from oracle import root_ns as R
@@ -204,11 +220,18 @@ def oracle_sample_rate(w, budget_s: float):
     r0, c0 = w.shapes[0]
     m_full, n_full = min(r0, c0), max(r0, c0)
     G = generate((m_full, n_full), w.dist, BASE_SEED, "cpu").numpy()
+    masks = None
+    if quant in ("rht", "rht46"):
+        masks = [int(v) for v in np.random.default_rng(BASE_SEED + 7).integers(0, 1 << 16, 3)]
+    a46 = quant in ("a46", "rht46")
     m = m_full
     while True:
-        X0, _, _, _ = R.normalise_and_clip(G[:m], w.clip_k)
+        if clip == "p99":
+            X0, _, _, _ = R.normalise_and_clip(G[:m], None, clip_quantile=0.99)
+        else:
+            X0, _, _, _ = R.normalise_and_clip(G[:m], w.clip_k)
         t0 = time.perf_counter()
-        R.ns_iterations_nvfp4(X0, 1, *w.coeffs[0])
+        R.ns_iterations_nvfp4(X0, 1, *w.coeffs[0], rht_masks=masks, adaptive46=a46)
         dt = time.perf_counter() - t0
         if dt <= budget_s or m <= 256:
             break
@@ -292,7 +315,7 @@ def run_reference(args):
     rates = []
     desc = ""
     for i in range(args.warmup + args.steps):
-        rate, dt, desc = oracle_sample_rate(w, budget)
+        rate, dt, desc = oracle_sample_rate(w, budget, args.quant, args.clip)
         if i >= args.warmup:
             rates.append(rate)
     value = statistics.median(rates)
@@ -302,7 +325,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * len(w.shapes) / value, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64 products, fp32 tensors",
-        "data": "synthetic", "config": {"workload": w.name, "matrices": len(w.shapes), "K": w.K},
+        "data": "synthetic", "config": ns_config(w, args.quant, args.clip, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -556,7 +579,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, dt, desc = oracle_sample_rate(w, 20.0)
+        rate, dt, desc = oracle_sample_rate(w, 20.0, args.quant, args.clip)
         cpu = {"value": rate, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": desc}
 
     if rank == 0:
@@ -565,14 +588,7 @@ def main():
             "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3/16) products, fp32 accumulate",
             "data": "synthetic",
-            "config": {"workload": w.name, "matrices": len(Gs), "shapes": sorted(set(map(tuple, w.shapes))),
-                       "K": K, "coeffs": "Muon (3.4445, -4.7750, 2.0315)",
-                       "clip": "3 x RMS" if args.clip == "rms" else "0.99 quantile of |X_0| (nearest rank)",
-                       "quantiser": {"plain": "NVFP4 RTN (H = I, M = 6)",
-                                     "rht46": "NVFP4 RTN with H16^r (fresh signs per step) and adaptive 4/6",
-                                     "rht": "NVFP4 RTN with H16^r (fresh signs per step)",
-                                     "a46": "NVFP4 RTN with adaptive 4/6"}[args.quant],
-                       "parallelism": f"replicas x{world} (independent matrices, no collective)",
+            "config": {**ns_config(w, args.quant, args.clip, world),
                        "l2": l2_note,
                        "launch": ("one CUDA graph replay per step (the call captured once); per-phase "
                                   "times from a separate event-recording pass" if graph is not None
