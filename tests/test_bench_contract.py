@@ -1,0 +1,59 @@
+"""CPU checks of bench.py's JSON contract on the arm that needs no GPU.
+
+`bench.py --impl reference` times the oracle on the host cores and prints one JSON
+line with the same metric, unit and workload description as the GPU arm.  Run on the
+smallest workload, so that the sample takes seconds.
+"""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def run_bench(*args):
+    r = subprocess.run([sys.executable, "bench.py", *args], cwd=ROOT, capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    return json.loads(r.stdout.strip().splitlines()[-1])
+
+
+@pytest.mark.parametrize("variant", [[], ["--quant", "rht46", "--clip", "p99"]])
+def test_reference_arm_line(variant):
+    import bench
+    from nvfp4_precision_optimizer_b200.workloads import WORKLOADS
+
+    line = run_bench("--impl", "reference", "--workload", "single_256x256_gauss",
+                     "--steps", "1", "--warmup", "0", *variant)
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["higher_is_better"] is True and line["vs_baseline"] is None
+    assert line["value"] > 0 and line["steps"] == 1
+    quant = variant[1] if variant else "plain"
+    clip = variant[3] if variant else "rms"
+    # the workload keys are those the GPU arm prints for the same flags
+    want = bench.ns_config(WORKLOADS["single_256x256_gauss"], quant, clip, 1)
+    assert line["config"] == json.loads(json.dumps(want))
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    e2e = line["e2e"]
+    assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+    # matrices/s and ms per step describe the same time
+    assert line["ms_per_step"] == pytest.approx(1000.0 * line["config"]["matrices"] / line["value"])
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    """Under torchrun only rank 0 runs the reference arm; the others exit 0 without work."""
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload",
+                        "single_256x256_gauss", "--steps", "1", "--warmup", "0"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 0 and r.stdout.strip() == ""
