@@ -247,3 +247,22 @@ def test_rejects_bad_input():
         Q.quantize_rows(np.array([[np.nan] * 16], np.float32))
     with pytest.raises(TypeError):
         Q.quantize_rows(np.ones((2, 16), np.float64))
+
+
+def test_exact_signed_zeros_keep_their_sign_bit():
+    """E2M1 is sign-magnitude (1 sign, 2 exponent, 1 mantissa bit), so in a block with a
+    non-zero scale a zero element keeps its sign: an exact -0.0 gets code 0x8 and +0.0
+    gets 0x0.  A block whose scale rounds to 0 (here an all-zero block) is written as
+    all-zero codes, signs included (the reading for a zero block scale)."""
+    x = np.zeros((2, 32), np.float32)
+    x[0, :16] = [-0.0, 0.0] * 8                       # all-zero block: scale byte 0
+    x[0, 16:] = [4.0, -0.0, 0.0, -4.0] + [0.0] * 12   # live block with signed zeros
+    x[1, :15] = 1.0
+    x[1, 15] = -0.0                                   # last element of a live block
+    codes, scales, _ = Q.quantize_rows(x)
+    nib = Q.unpack_codes(codes)
+    assert scales[0, 0] == 0 and np.all(nib[0, :16] == 0)
+    assert scales[0, 1] != 0
+    assert nib[0, 17] == 0x8 and nib[0, 18] == 0x0
+    assert nib[0, 16] & 8 == 0 and nib[0, 19] & 8 == 8
+    assert nib[1, 15] == 0x8 and np.all(nib[1, :15] == 0x7)   # the block amax maps to 6
