@@ -162,7 +162,16 @@ fs4_status fs4_nvfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_
 
 /* Dequantise a row-blocked NVFP4 matrix (rows x cols, as written by
  * fs4_nvfp4_quantize in the layout given by flags) into FP32 y (leading
- * dimension ld): y = fp32(fp32(code * s) * s_g).  Errors as above. */
+ * dimension ld): y = fp32(fp32(code * s) * s_g).
+ * Source: Section 2 "NVFP4 format": an element's value is its E2M1 value times
+ * its block's E4M3 scale times the FP32 tensor scale.
+ *   codes, scales: device, PLAIN (rows x cols/2 bytes, low nibble first;
+ *   rows x cols/16 bytes) or TILED (FS4_LAYOUT_TILED), 16-byte aligned; s_g:
+ *   one device float; y: device, caller-owned, rows x cols with ld >= cols, not
+ *   overlapping the inputs.  One launch, no workspace.
+ *   Errors: FS4_ERR_SHAPE (empty, or cols % 16 != 0), FS4_ERR_INVALID_ARG (null
+ *   pointers, unknown flags, ld < cols, misaligned pointers), FS4_ERR_ARCH,
+ *   FS4_ERR_CUDA. */
 fs4_status fs4_nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* s_g,
                                 int64_t rows, int64_t cols, float* y, int64_t ld,
                                 uint32_t flags, void* stream);
@@ -261,7 +270,20 @@ fs4_status fs4_root_ns(const float* G, int64_t m, int64_t n, int64_t ld, float* 
 
 /* The same step on `count` independent matrices (descs is a HOST array),
  * grouped so that each phase of the iteration is one launch over the tiles
- * of all matrices, each GEMM followed by a small bounds kernel (2 + 6K launches per call). */
+ * of all matrices, each GEMM followed by a small bounds kernel (2 + 6K launches per call).
+ * Source: Section 3.4 (the step of fs4_root_ns); the per-matrix (a, b, c) of each
+ * descriptor carry the shape-dependent coefficients of Section 2 "Root optimizer".
+ *   descs[i]: G (device, m x n, leading dimension ld), out (device, caller-owned,
+ *   same shape, leading dimension ld_out), a, b, c.  The workspace
+ *   (fs4_root_ns_batched_workspace_size, 256-byte aligned, caller-owned) holds
+ *   every matrix's iterates and views; it must not overlap any G or out, and no
+ *   out may overlap another out or any G.
+ *   Errors: FS4_ERR_SHAPE (count outside [1, FS4_MAX_BATCH], a shape as for
+ *   fs4_root_ns, K outside [1, FS4_MAX_ITERS]), FS4_ERR_INVALID_ARG (null
+ *   pointers, ld or ld_out < n, pointers not 4-byte aligned, non-finite
+ *   coefficients or clip_k, unknown flags),
+ *   FS4_ERR_ALIAS, FS4_ERR_WORKSPACE, FS4_ERR_ARCH, FS4_ERR_CUDA; device-side
+ *   conditions as for fs4_root_ns. */
 fs4_status fs4_root_ns_batched(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
                                uint32_t flags, void* workspace, size_t workspace_bytes,
                                void* stream);
