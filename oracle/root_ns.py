@@ -84,13 +84,21 @@ def symmetric_from_upper(A: np.ndarray) -> np.ndarray:
 
 
 def ns_iterations_nvfp4(X0, K, a, b, c, mode="pow2", trace=None, rht_masks=None,
-                        adaptive46=False):
+                        adaptive46=False, perturb=None, matmul=None):
     """K NVFP4 Newton-Schulz iterations (Section 3.4) from the FP32 m x n X0 (m <= n).
 
     rht_masks: None (H = I) or 3K sign masks of H16^r (see nvfp4.hadamard_rows), one
     per product: 3k for A_k = qX_k qX_k^T, 3k + 1 for qA_k qA16_k, 3k + 2 for
     qB_k qX16_k.  adaptive46: adaptive 4/6 block scaling in every quantisation.
+    perturb: None, or a function (k, name, T) -> T' applied to each FP32 tensor
+    ("A", "B", "X") right after it is formed; it lets a test study how the iteration
+    responds to other, equally valid FP32 roundings of the same values.  matmul: None
+    (float64 products), or a function (L, R) -> L R used for the three products
+    instead, e.g. one accumulating in FP32.  None for both leaves the arithmetic
+    above untouched.
     """
+    pert = (lambda k, name, t: t) if perturb is None else perturb
+    mm = (lambda l, r: l @ r) if matmul is None else matmul
     X = np.asarray(X0, dtype=np.float32)
     hr = (lambda t, j: t) if rht_masks is None else (lambda t, j: nvfp4.hadamard_rows(t, rht_masks[j]))
     hc = (lambda t, j: t) if rht_masks is None else (lambda t, j: nvfp4.hadamard_cols(t, rht_masks[j]))
@@ -103,15 +111,16 @@ def ns_iterations_nvfp4(X0, K, a, b, c, mode="pow2", trace=None, rht_masks=None,
         dX = nvfp4.dequantize_rows(qx, sx, gx)                     # m x n
         dX16 = nvfp4.dequantize_cols(qxt, sxt, gxt)                # m x n, 16x1 blocks
         # A_k = qX_k qX_k^T
-        A = symmetric_from_upper(dX @ dX.T).astype(np.float32)
+        A = pert(k, "A", symmetric_from_upper(mm(dX, dX.T)).astype(np.float32))
         # qA_k = Q1x16(A_k H), qA16_k = Q16x1(H^T A_k), B_k = b A_k + c qA_k qA16_k
         qa, sa, ga = nvfp4.quantize_rows(hr(A, 3 * k + 1), mode=mode, adaptive46=a46)
         qa16, sa16, ga16 = nvfp4.quantize_cols(hc(A, 3 * k + 1), mode=mode, adaptive46=a46)
-        P = nvfp4.dequantize_rows(qa, sa, ga) @ nvfp4.dequantize_cols(qa16, sa16, ga16)
-        B = (b * A.astype(np.float64) + c * P).astype(np.float32)
+        P = mm(nvfp4.dequantize_rows(qa, sa, ga), nvfp4.dequantize_cols(qa16, sa16, ga16))
+        B = pert(k, "B", (b * A.astype(np.float64) + c * P).astype(np.float32))
         # qB_k = Q1x16(B_k H'), X_{k+1} = a X_k + qB_k qX16_k
         qb, sb, gb = nvfp4.quantize_rows(hr(B, 3 * k + 2), mode=mode, adaptive46=a46)
-        Xn = (a * X.astype(np.float64) + nvfp4.dequantize_rows(qb, sb, gb) @ dX16).astype(np.float32)
+        Xn = (a * X.astype(np.float64) + mm(nvfp4.dequantize_rows(qb, sb, gb), dX16)).astype(np.float32)
+        Xn = pert(k, "X", Xn)
         if trace is not None:
             trace.append(dict(X=X, qX=(qx, sx, gx), qXT=(qxt, sxt, gxt), A=A,
                               qA=(qa, sa, ga), P=P, B=B, qB=(qb, sb, gb), X_next=Xn))

@@ -198,3 +198,48 @@ def test_update_uses_the_column_blocked_view():
     qb = Q.dequantize_rows(*trace[0]["qB"])
     want = (a * X0.astype(np.float64) + qb @ X0.astype(np.float64)).astype(np.float32)
     assert np.array_equal(trace[0]["X_next"], want)
+
+
+def test_combine_step_uses_the_quantised_square_and_the_fp32_gram_by_hand():
+    """One iteration worked out by hand (Section 3.4, second line of the iteration:
+    B = b A + c qA qA16x1).  X_0 is 16 x 16 with two non-zero rows, [6, 0, ...] and
+    [1, 1.5, 0, ...]; both of its NVFP4 views are exact (s_g = 2^-8, block scales
+    256 and 64).  Then, by hand:
+      A = X X^T:   A00 = 36, A01 = 6, A11 = 3.25 (FP32-exact, not NVFP4-exact);
+      qA:  s_g = 2^-6; row 0 [36, 6]: scale 384, den 6, codes 6, 1 (exact);
+           row 1 [6, 3.25]: scale 64, den 1, 3.25 rounds to the E2M1 value 3;
+           the 16x1 view of the symmetric A has the same values;
+      P = deq(qA) deq(qA16) = [[36, 6], [6, 3]]^2 = [[1332, 234], [234, 45]];
+      B = -0.5 A + 0.25 P = [[315, 55.5], [55.5, 9.625]];
+      qB:  s_g = 2^-3; row 0: 315 / 0.75 = 420 -> scale 416, den 52, codes 6 (312),
+           1 (52); row 1: 55.5 / 0.75 = 74 -> scale 72, den 9, codes 6 (54), 1 (9);
+      X_1 = 1 * X + deq(qB) X = [[1930, 78], [334, 15]] in the top-left corner.
+    The two plausible misreadings give different B: squaring the FP32 A
+    (P = A A: B01 = 55.875, B11 = 10.015625) and using deq(qA) in the b A term
+    (B11 = 9.75)."""
+    X0 = np.zeros((16, 16), np.float32)
+    X0[0, 0] = 6.0
+    X0[1, 0], X0[1, 1] = 1.0, 1.5
+    a, b, c = 1.0, -0.5, 0.25
+    trace = []
+    R.ns_iterations_nvfp4(X0, 1, a, b, c, trace=trace)
+    t = trace[0]
+
+    def corner(M, vals):
+        want = np.zeros((16, 16))
+        want[:2, :2] = vals
+        return np.array_equal(np.asarray(M, np.float64), want)
+
+    assert corner(t["A"], [[36.0, 6.0], [6.0, 3.25]])
+    assert corner(Q.dequantize_rows(*t["qA"]), [[36.0, 6.0], [6.0, 3.0]])
+    assert corner(t["P"], [[1332.0, 234.0], [234.0, 45.0]])
+    assert corner(t["B"], [[315.0, 55.5], [55.5, 9.625]])
+    assert corner(Q.dequantize_rows(*t["qB"]), [[312.0, 52.0], [54.0, 9.0]])
+    want_x1 = np.zeros((16, 16))
+    want_x1[:2, :2] = [[1930.0, 78.0], [334.0, 15.0]]
+    assert np.array_equal(t["X_next"].astype(np.float64), want_x1)
+    # the misreadings are distinguishable on this input
+    A = np.asarray(t["A"], np.float64)
+    assert not corner(b * A + c * (A @ A), [[315.0, 55.5], [55.5, 9.625]])
+    dqa = Q.dequantize_rows(*t["qA"])
+    assert not corner(b * dqa + c * np.asarray(t["P"]), [[315.0, 55.5], [55.5, 9.625]])
