@@ -22,4 +22,8 @@ Modules:
                           dequantise (numpy, exact emulation).
   * ``oracle.root_ns`` -- normalise + clip + K NVFP4 Newton-Schulz iterations,
                           products in float64 on dequantised operands.
+  * ``oracle.cpp_oracle`` -- ctypes binding of ``oracle/cpp/fs4_oracle.cpp``, the
+                          same steps restated in plain C++17 (OpenMP over rows,
+                          float64 triple loops, no BLAS); a second, independent
+                          implementation, and the one the CPU baseline times.
 """

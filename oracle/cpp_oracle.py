@@ -1,0 +1,161 @@
+"""ctypes binding of the C++ oracle (oracle/cpp/fs4_oracle.cpp).
+
+TEST INFRASTRUCTURE ONLY: loaded by the tests, by the smoke check and by the
+CPU-baseline / reference legs of bench.py; never by the product path.
+
+The C++ oracle is the plain, slow restatement of the direct NVFP4 Newton-Schulz
+step ("Full-Stack FP4", arXiv 2607.04422, Section 3.4): no BLAS, float64 triple
+loops over dequantised operands, nearest-value searches over the code tables,
+OpenMP over independent rows.  `build()` compiles it with g++ (no fast-math, no
+floating-point contraction); `lib()` builds it on first use if it is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "cpp", "fs4_oracle.cpp")
+LIB_PATH = os.path.join(HERE, "cpp", "libfs4_oracle.so")
+
+_lib = None
+_c = ctypes
+_fp = _c.POINTER(_c.c_float)
+_dp = _c.POINTER(_c.c_double)
+_up = _c.POINTER(_c.c_uint8)
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into oracle/cpp/libfs4_oracle.so (skipped when up to date)."""
+    if (not force and os.path.exists(LIB_PATH)
+            and os.path.getmtime(LIB_PATH) >= os.path.getmtime(SRC)):
+        return LIB_PATH
+    cmd = ["g++", "-std=c++17", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+           "-fPIC", "-shared", "-o", LIB_PATH + ".tmp", SRC]
+    subprocess.run(cmd, check=True)
+    os.replace(LIB_PATH + ".tmp", LIB_PATH)
+    return LIB_PATH
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = _c.CDLL(LIB_PATH)
+        L.fs4o_threads.restype = _c.c_int
+        L.fs4o_e2m1_value.restype = _c.c_double
+        L.fs4o_e2m1_value.argtypes = [_c.c_int]
+        L.fs4o_e4m3_value.restype = _c.c_double
+        L.fs4o_e4m3_value.argtypes = [_c.c_int]
+        L.fs4o_e2m1_encode.restype = _c.c_int
+        L.fs4o_e2m1_encode.argtypes = [_c.c_double]
+        L.fs4o_e4m3_encode.restype = _c.c_int
+        L.fs4o_e4m3_encode.argtypes = [_c.c_double]
+        L.fs4o_tensor_scale.restype = _c.c_float
+        L.fs4o_tensor_scale.argtypes = [_c.c_float, _c.c_int]
+        L.fs4o_quantize_rows.restype = _c.c_int
+        L.fs4o_quantize_rows.argtypes = [_fp, _c.c_int64, _c.c_int64, _c.c_float, _c.c_int, _up, _up,
+                                         _fp, _c.c_int]
+        L.fs4o_dequantize_rows.restype = _c.c_int
+        L.fs4o_dequantize_rows.argtypes = [_up, _up, _c.c_float, _c.c_int64, _c.c_int64, _dp, _c.c_int]
+        L.fs4o_product.restype = _c.c_int
+        L.fs4o_product.argtypes = [_dp, _dp, _c.c_int64, _c.c_int64, _c.c_int64, _dp, _c.c_int]
+        L.fs4o_normalise_and_clip.restype = _c.c_double
+        L.fs4o_normalise_and_clip.argtypes = [_fp, _c.c_int64, _c.c_int64, _c.c_double, _fp, _fp, _fp]
+        L.fs4o_ns_iterations_nvfp4.restype = _c.c_int
+        L.fs4o_ns_iterations_nvfp4.argtypes = [_fp, _c.c_int64, _c.c_int64, _c.c_int, _c.c_double,
+                                               _c.c_double, _c.c_double, _c.c_int]
+        L.fs4o_root_ns.restype = _c.c_int
+        L.fs4o_root_ns.argtypes = [_fp, _c.c_int64, _c.c_int64, _c.c_int, _c.c_double, _c.c_double,
+                                   _c.c_double, _c.c_double, _c.c_int, _fp, _dp, _c.c_int]
+        _lib = L
+    return _lib
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _ptr(a, t):
+    return a.ctypes.data_as(t)
+
+
+def threads() -> int:
+    return int(lib().fs4o_threads())
+
+
+def quantize_rows(x, s_g=None, mode="pow2", threads=0):
+    """Q1x16 of an FP32 matrix: (codes [rows, cols/2], scales [rows, cols/16], s_g)."""
+    x = _f32(x)
+    rows, cols = x.shape
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros((rows, cols // 16), np.uint8)
+    sg = np.zeros(1, np.float32)
+    st = lib().fs4o_quantize_rows(_ptr(x, _fp), rows, cols, float(s_g) if s_g is not None else -1.0,
+                                  1 if mode == "amax" else 0, _ptr(codes, _up), _ptr(scales, _up),
+                                  _ptr(sg, _fp), threads)
+    if st != 0:
+        raise ValueError("bad shape")
+    return codes, scales, np.float32(sg[0])
+
+
+def quantize_cols(x, s_g=None, mode="pow2", threads=0):
+    """Q16x1, laid out as the Q1x16 of x^T."""
+    return quantize_rows(np.ascontiguousarray(np.asarray(x, np.float32).T), s_g, mode, threads)
+
+
+def dequantize_rows(codes, scales, s_g, threads=0):
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    rows, cols = codes.shape[0], codes.shape[1] * 2
+    out = np.zeros((rows, cols), np.float64)
+    if lib().fs4o_dequantize_rows(_ptr(codes, _up), _ptr(scales, _up), float(s_g), rows, cols,
+                                  _ptr(out, _dp), threads) != 0:
+        raise ValueError("bad shape")
+    return out
+
+
+def product(L, R, threads=0):
+    L = np.ascontiguousarray(L, np.float64)
+    R = np.ascontiguousarray(R, np.float64)
+    out = np.zeros((L.shape[0], R.shape[1]), np.float64)
+    if lib().fs4o_product(_ptr(L, _dp), _ptr(R, _dp), L.shape[0], L.shape[1], R.shape[1],
+                          _ptr(out, _dp), threads) != 0:
+        raise ValueError("bad shape")
+    return out
+
+
+def normalise_and_clip(G, clip_k):
+    """(X0, inv, tau, norm) of an FP32 matrix already in working orientation."""
+    G = _f32(G)
+    X0 = np.zeros_like(G)
+    inv = np.zeros(1, np.float32)
+    tau = np.zeros(1, np.float32)
+    norm = lib().fs4o_normalise_and_clip(_ptr(G, _fp), G.shape[0], G.shape[1],
+                                         float(clip_k) if clip_k else 0.0, _ptr(X0, _fp),
+                                         _ptr(inv, _fp), _ptr(tau, _fp))
+    return X0, np.float32(inv[0]), (np.float32(tau[0]) if clip_k else None), float(norm)
+
+
+def ns_iterations_nvfp4(X0, K, a, b, c, threads=0):
+    X = _f32(X0).copy()
+    if lib().fs4o_ns_iterations_nvfp4(_ptr(X, _fp), X.shape[0], X.shape[1], int(K), float(a), float(b),
+                                      float(c), threads) != 0:
+        raise ValueError("bad shape")
+    return X
+
+
+def root_ns(G, K=5, a=3.4445, b=-4.7750, c=2.0315, clip_k=3.0, quantized=True, threads=0):
+    """The whole step (normalise, clip, K iterations) on an FP32 matrix of any orientation."""
+    G = _f32(G)
+    out32 = np.zeros(G.shape, np.float32)
+    out64 = np.zeros(G.shape, np.float64)
+    st = lib().fs4o_root_ns(_ptr(G, _fp), G.shape[0], G.shape[1], int(K), float(a), float(b), float(c),
+                            float(clip_k) if clip_k else 0.0, 1 if quantized else 0, _ptr(out32, _fp),
+                            _ptr(out64, _dp), threads)
+    if st != 0:
+        raise ValueError("bad shape or non-finite input")
+    return out32 if quantized else out64
