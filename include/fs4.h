@@ -84,7 +84,10 @@ enum {
  * phase 0 = preamble (normalise, clip, quantise X_0); phase 1 + 3k + j is the
  * j-th product of iteration k (j = 0: A = qX qX^T, 1: P = qA qA^T and
  * B = b A + c P, 2: X_{k+1} = a X_k + qB qX^{16x1}).  Encoded in flag bits 8..15
- * as (phase + 1); 0 means run everything. */
+ * as (phase + 1); 0 means run everything.  A stop right after product 1 of an
+ * iteration also writes that product's B (FP32) over the upper 256 x 256 tiles
+ * of A in the workspace (fs4_ns_layout.A), where B is otherwise never stored in
+ * FP32; without the stop the kernels never write it. */
 #define FS4_STOP_AFTER(phase) ((uint32_t)(((phase) + 1) & 0xFF) << 8)
 
 /* Quantiser options of the Newton-Schulz step (Section 3.4: "qX_k =
@@ -344,10 +347,9 @@ fs4_status fs4_root_ns_batched_timed(int32_t count, const fs4_ns_desc* descs, in
 #define FS4_NOALLOC_SCRATCH_BYTES (16u << 20)
 
 /* fs4_root_ns for callers that cannot allocate device memory (no counterpart in
- * the paper; an interface addition).  Examples: code running while a stream is
- * captured into a CUDA graph, where cudaMalloc is not allowed; plugins inside a
- * host framework that owns all device memory and lends none; loops where a
- * runtime allocation is forbidden.  Same arguments and result as fs4_root_ns
+ * the paper; an interface addition).  Examples: plugins inside a host framework
+ * that owns all device memory and lends none; loops in which a run-time
+ * allocation is forbidden.  Same arguments and result as fs4_root_ns
  * with flags = 0, but the workspace is a fixed 16 MiB array compiled into the
  * library (every device that loads the library holds it until the process
  * exits).  Matrices whose fs4_root_ns_workspace_size(m, n) exceeds

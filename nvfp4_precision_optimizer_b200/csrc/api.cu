@@ -205,7 +205,9 @@ fs4_status run_ns(const Plan& pl, int32_t K, float clip_k, uint32_t flags, const
     p.stall = 0;
     if (!mark()) return FS4_ERR_CUDA;
     if (stop == 1 + 3 * k) return FS4_OK;
+    p.dbg_b = (stop == 2 + 3 * k) ? 1 : 0;
     if ((e = launch_gemm_ns(Epi::GramA, p, st, num_sms)) != cudaSuccess) return FS4_ERR_CUDA;
+    p.dbg_b = 0;
     if (!mark()) return FS4_ERR_CUDA;
     if (stop == 2 + 3 * k) return FS4_OK;
     p.last = (k == K - 1) ? 1 : 0;

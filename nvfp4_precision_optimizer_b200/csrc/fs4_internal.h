@@ -116,6 +116,7 @@ struct NsParams {
   int32_t iter;            // k of the current iteration
   int32_t last;            // 1 on the final update product (writes `out`)
   int32_t stall;           // test only: the MMA issuer waits on a barrier nothing arrives on
+  int32_t dbg_b;           // debug stop after the second product: also write B (FP32) over A
   uint32_t opts;           // kOptRht | kOpt46 | kOptQuantile
   float clip_k;            // clip_k * RMS, or with kOptQuantile the quantile ratio q in (0, 1]
   uint32_t* status;

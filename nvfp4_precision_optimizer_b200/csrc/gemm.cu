@@ -507,12 +507,16 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
             }
           }
         } else {
-          // stage the chunk (FP32 store and/or the 16x1 view read it back)
-          if (E != Epi::GramA || need_col) {
+          // stage the chunk (FP32 store and/or the 16x1 view read it back); a debug
+          // stop after the second product also stores B (FP32) over this tile of A,
+          // whose chunk c was read already
+          const bool dbg_b = (E == Epi::GramA) && p.dbg_b;
+          if (E != Epi::GramA || need_col || dbg_b) {
             stage_store_row(buf, lane, y);
             __syncwarp();
           }
           if constexpr (E != Epi::GramA) stage_flush(buf, fp, c, lane);   // A or X' (FP32)
+          else if (dbg_b) stage_flush(buf, fp, c, lane);
           // 1x16 view along this lane's row and, where needed, the 16x1 view of column
           // gcc + cc, rows gr0 + 16 hh ..: two independent quantiser chains side by side
           QBlock16 q, qc;

@@ -1,18 +1,17 @@
 // fs4_root_ns_noalloc: the single-matrix Newton-Schulz step for callers that
 // cannot allocate device memory.
 //
-// Some callers have no way to obtain a workspace: code that runs while a stream
-// is being captured into a CUDA graph (cudaMalloc is not allowed during
-// capture), plugins living inside a host framework that owns every device
-// allocation and hands out none, or latency-critical loops where a runtime
-// allocation is not permitted.  This entry point gives them the same step with
-// the workspace taken from a fixed array compiled into the library.
+// Some callers have no way to obtain a workspace: plugins living inside a host
+// framework that owns every device allocation and hands out none, or loops in
+// which a run-time allocation is not permitted.  This entry point gives them the
+// same step with the workspace taken from a fixed array compiled into the
+// library.
 //
 // The array lives in every device that loads the library, for the life of the
 // process.  Its address is looked up once per device (cudaGetSymbolAddress on
-// the first call made with that device current; make that first call outside
-// any stream capture).  All calls share it: two calls whose work overlaps on
-// the GPU (different streams, or different host threads) race on it.  Each call
+// the first call made with that device current; make that first call before any
+// stream capture).  All calls share it: two calls whose work overlaps on the
+// GPU (different streams, or different host threads) race on it.  Each call
 // clears the parts that must start at zero before using them.
 #include <mutex>
 

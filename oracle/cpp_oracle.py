@@ -87,8 +87,12 @@ def threads() -> int:
     return int(lib().fs4o_threads())
 
 
-def quantize_rows(x, s_g=None, mode="pow2", threads=0):
-    """Q1x16 of an FP32 matrix: (codes [rows, cols/2], scales [rows, cols/16], s_g)."""
+def quantize_rows(x, s_g=None, mode="pow2", adaptive46=False, threads=0):
+    """Q1x16 of an FP32 matrix: (codes [rows, cols/2], scales [rows, cols/16], s_g).
+    The same signature as oracle.nvfp4.quantize_rows; adaptive 4/6 scaling is not
+    implemented here."""
+    if adaptive46:
+        raise NotImplementedError("the C++ oracle quantises with M = 6 only")
     x = _f32(x)
     rows, cols = x.shape
     codes = np.zeros((rows, cols // 2), np.uint8)
@@ -102,9 +106,10 @@ def quantize_rows(x, s_g=None, mode="pow2", threads=0):
     return codes, scales, np.float32(sg[0])
 
 
-def quantize_cols(x, s_g=None, mode="pow2", threads=0):
+def quantize_cols(x, s_g=None, mode="pow2", adaptive46=False, threads=0):
     """Q16x1, laid out as the Q1x16 of x^T."""
-    return quantize_rows(np.ascontiguousarray(np.asarray(x, np.float32).T), s_g, mode, threads)
+    return quantize_rows(np.ascontiguousarray(np.asarray(x, np.float32).T), s_g, mode, adaptive46,
+                         threads)
 
 
 def dequantize_rows(codes, scales, s_g, threads=0):
@@ -116,6 +121,11 @@ def dequantize_rows(codes, scales, s_g, threads=0):
                                   _ptr(out, _dp), threads) != 0:
         raise ValueError("bad shape")
     return out
+
+
+def dequantize_cols(codes, scales, s_g, threads=0):
+    """Inverse of quantize_cols: the rows x cols matrix (float64, exact)."""
+    return dequantize_rows(codes, scales, s_g, threads).T
 
 
 def product(L, R, threads=0):

@@ -40,6 +40,7 @@ from __future__ import annotations
 import numpy as np
 
 from . import nvfp4
+from . import nvfp4 as _nvfp4
 
 NS_EPS = 1e-7
 
@@ -84,7 +85,7 @@ def symmetric_from_upper(A: np.ndarray) -> np.ndarray:
 
 
 def ns_iterations_nvfp4(X0, K, a, b, c, mode="pow2", trace=None, rht_masks=None,
-                        adaptive46=False, perturb=None, matmul=None):
+                        adaptive46=False, perturb=None, matmul=None, codec=None):
     """K NVFP4 Newton-Schulz iterations (Section 3.4) from the FP32 m x n X0 (m <= n).
 
     rht_masks: None (H = I) or 3K sign masks of H16^r (see nvfp4.hadamard_rows), one
@@ -95,13 +96,17 @@ def ns_iterations_nvfp4(X0, K, a, b, c, mode="pow2", trace=None, rht_masks=None,
     responds to other, equally valid FP32 roundings of the same values.  matmul: None
     (float64 products), or a function (L, R) -> L R used for the three products
     instead, e.g. one accumulating in FP32.  None for both leaves the arithmetic
-    above untouched.
+    above untouched.  codec: None (this package's numpy codec, oracle.nvfp4) or
+    another module with the same quantize_rows / quantize_cols / dequantize_rows /
+    dequantize_cols, such as oracle.cpp_oracle (bit-identical, much faster on
+    large matrices).
     """
+    nvfp4 = _nvfp4 if codec is None else codec
     pert = (lambda k, name, t: t) if perturb is None else perturb
     mm = (lambda l, r: l @ r) if matmul is None else matmul
     X = np.asarray(X0, dtype=np.float32)
-    hr = (lambda t, j: t) if rht_masks is None else (lambda t, j: nvfp4.hadamard_rows(t, rht_masks[j]))
-    hc = (lambda t, j: t) if rht_masks is None else (lambda t, j: nvfp4.hadamard_cols(t, rht_masks[j]))
+    hr = (lambda t, j: t) if rht_masks is None else (lambda t, j: _nvfp4.hadamard_rows(t, rht_masks[j]))
+    hc = (lambda t, j: t) if rht_masks is None else (lambda t, j: _nvfp4.hadamard_cols(t, rht_masks[j]))
     a46 = adaptive46
     for k in range(K):
         # qX_k = Q1x16(X_k H); qX16_k = Q16x1(H'^T X_k) (held as the 1x16 quantisation of

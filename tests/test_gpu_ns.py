@@ -3,15 +3,19 @@
 Inputs are seeded synthetic momenta; expected values come from oracle/ on the
 same FP32 input.  Tolerances:
   * preamble (normalise, clip, both NVFP4 views): bit-exact;
-  * first Gram product A_0 = qX_0 qX_0^T: relative Frobenius <= 1e-5 (the
-    operands are bit-identical to the oracle's at that point);
+  * each product of an iteration (A = qX qX^T, B = b A + c qA qA16x1,
+    X' = a X + qB qX16x1): relative Frobenius <= 1e-5 against the float64
+    product of the GPU's own dequantised operands, and every NVFP4 view an
+    epilogue writes is the oracle's quantisation of the GPU's FP32 result,
+    byte for byte;
   * end-to-end: relative Frobenius <= 2e-2 and orthogonality error within 10%
-    of the oracle's wherever the method itself is not chaotic (K <= 3 with the
-    Muon coefficients, K = 5 with the contractive quintic).  With the Muon
-    coefficients at K = 5 the NVFP4 iterate diverges, and two oracle runs that
-    differ only by one-ulp accumulation noise already differ by 2-18%; there
-    the orthogonality error within 10% and the singular-value spectrum are
-    asserted instead.
+    of the oracle's wherever that is attainable: K <= 3 with the Muon
+    coefficients and K = 5 with the contractive quintic and cubic.  At K = 5 with
+    the Muon coefficients a one-ulp change in the FP32 rounding of B moves the
+    oracle's own output by about 10% (tests/test_oracle_sensitivity.py), so
+    there the orthogonality error within 10% and the singular-value spectrum
+    within 5% are asserted, and every iteration is checked on its own: one oracle
+    iteration from the GPU's X_k against the GPU's X_{k+1}, within 2e-2.
 """
 import numpy as np
 import pytest
@@ -312,3 +316,58 @@ def test_preamble_keeps_the_sign_of_negative_zeros(fs4):
     ct, st, _ = Q.quantize_cols(X0)
     gc, gs = view(ws, lay.qXT_codes[0], lay.qXT_scales[0], lay.np, lay.mp)
     assert np.array_equal(gc[:96, :32], ct) and np.array_equal(gs[:96, :4], st)
+
+
+def _ws_runs(fs4, G, K, coef, stops):
+    """One call per debug stop on the same input; returns a grab(off, n) per stop."""
+    out = {}
+    for s in stops:
+        _, ws = run_gpu(fs4, G, K, coef, flags=fs4.stop_after(s))
+        out[s] = (lambda w: (lambda off, n: w[off:off + n]))(ws)
+    return out
+
+
+@pytest.mark.parametrize("shape,kind", [((256, 256), "gauss"), ((48, 80), "gauss"),
+                                        ((1024, 4096), "outliers"), ((4096, 1024), "student"),
+                                        ((768, 1280), "gauss")])
+@pytest.mark.parametrize("coef", [(0.0, 0.0, 1.0), MUON])
+def test_second_and_third_products_against_float64(fs4, shape, kind, coef):
+    """Products 2 and 3 of the first iteration (Section 3.4: B = b A + c qA qA16x1 and
+    X_1 = a X_0 + qB qX16x1), each against the float64 product of the GPU's own
+    dequantised operands, within 1e-5; the epilogues' NVFP4 views of B and X_1 are
+    the oracle's quantisation of the GPU's FP32 results, byte for byte.  With
+    (a, b, c) = (0, 0, 1) the results are the bare products B = qA qA^T and
+    X_1 = qB qX16x1; with the Muon coefficients the fused combines are included."""
+    from tests import gemm_checks as GC
+    G = momentum(*shape, kind=kind, seed=12)
+    lay = fs4.ns_layout([shape], 0)
+    m, n = min(shape), max(shape)
+    g = _ws_runs(fs4, G, 2, coef, [1, 2, 3])
+    err_b, qb_ok = GC.check_second_product(g[1], g[2], lay, 0, coef[1], coef[2])
+    assert err_b <= 1e-5, err_b
+    assert qb_ok
+    err_x = GC.check_third_product(g[2], g[3], lay, 0, coef[0], m, n)
+    assert err_x <= 1e-5, err_x
+    assert GC.check_first_product_views(g[3], lay, 0, m, n)
+
+
+@pytest.mark.parametrize("shape,kind", [((256, 256), "gauss"), ((1024, 4096), "outliers"),
+                                        ((4096, 1024), "student"), ((512, 1536), "gauss")])
+def test_every_muon_iteration_from_the_gpu_iterate(fs4, shape, kind):
+    """K = 5 with the Muon coefficients, one iteration at a time: the oracle's NVFP4
+    iteration from the GPU's X_k against the GPU's X_{k+1} (the caller's output for
+    k = 4), within 2e-2 (Section 3.4)."""
+    G = momentum(*shape, kind=kind, seed=13)
+    lay = fs4.ns_layout([shape], 0)
+    m, n = min(shape), max(shape)
+    xs = []
+    for k in range(5):
+        _, ws = run_gpu(fs4, G, 5, MUON, flags=fs4.stop_after(3 * k))
+        xs.append(np.ascontiguousarray(ws_f32(ws, lay.X, lay.mp * lay.np).reshape(lay.mp, lay.np)[:m, :n]))
+    out, _ = run_gpu(fs4, G, 5, MUON)
+    xs.append(np.ascontiguousarray(working(out)))
+    X0 = R.normalise_and_clip(working(G), 3.0)[0]
+    assert np.array_equal(xs[0].view(np.uint32), X0.view(np.uint32))
+    for k in range(5):
+        want = R.ns_iterations_nvfp4(xs[k], 1, *MUON).astype(np.float64)
+        assert rel_frob(xs[k + 1], want) <= 2e-2, (k, rel_frob(xs[k + 1], want))

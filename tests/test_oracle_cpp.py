@@ -173,3 +173,15 @@ def test_nonfinite_input_is_refused():
     G[2, 3] = np.nan
     with pytest.raises(ValueError):
         C.root_ns(G, 1)
+
+
+@pytest.mark.parametrize("shape,K,coef", [((64, 160), 3, MUON), ((96, 320), 2, QUINTIC),
+                                          ((48, 48), 2, CUBIC)])
+def test_numpy_iteration_with_the_cpp_codec_is_bit_identical(shape, K, coef):
+    """The large-size GPU tests run the numpy oracle's iteration with the C++ codec
+    (codec=cpp_oracle) for speed; it must give the numpy codec's result bit for bit."""
+    rng = np.random.default_rng(6)
+    X0 = R.normalise_and_clip((rng.standard_normal(shape) * 0.02).astype(np.float32), 3.0)[0]
+    a = R.ns_iterations_nvfp4(X0, K, *coef)
+    b = R.ns_iterations_nvfp4(X0, K, *coef, codec=C)
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
