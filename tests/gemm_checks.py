@@ -50,14 +50,15 @@ def check_second_product(grab_after_1, grab_after_2, lay, k, b, c):
     grab_after_2: after product 2 with the debug stop (B written over A, qB).
     Returns (relative Frobenius error of B over the computed tiles, qB bit-exact)."""
     mp = lay.mp
-    A = f32(grab_after_1, lay.A, mp, mp).astype(np.float64)
+    up = upper_mask(mp)
+    # only the tiles on and above the diagonal are ever written: mask the rest
+    A = np.where(up, f32(grab_after_1, lay.A, mp, mp), np.float32(0)).astype(np.float64)
     qa_c, qa_s = view(grab_after_1, lay.qA_codes, lay.qA_scales, mp, mp)
     sg_a = scalars(grab_after_1, lay)[64 + k]
     dA = C.dequantize_rows(qa_c, qa_s, sg_a)
     P = dA @ dA.T
     want = np.float64(np.float32(b)) * symmetric_from_tiles(A, mp) + np.float64(np.float32(c)) * P
-    Bg = f32(grab_after_2, lay.A, mp, mp)
-    up = upper_mask(mp)
+    Bg = np.where(up, f32(grab_after_2, lay.A, mp, mp), np.float32(0))
     err = rel_frob(Bg.astype(np.float64)[up], want[up])
     sg_b = scalars(grab_after_2, lay)[128 + k]
     oc, os_, _ = C.quantize_rows(np.ascontiguousarray(symmetric_from_tiles(Bg, mp), np.float32), s_g=sg_b)
