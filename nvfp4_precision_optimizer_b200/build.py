@@ -11,7 +11,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libfs4.so")
-SOURCES = ["kernels.cu", "gemm.cu", "gemm_ns.cu", "momentum.cu", "api.cu", "noalloc.cu"]
+SOURCES = ["kernels.cu", "gemm.cu", "momentum.cu", "api.cu", "noalloc.cu"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",
