@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-bf16", action="store_true",
+                    help="skip the BF16 comparison step (same plan, BF16 operands)")
     ap.add_argument("--op", default="ns", choices=["ns", "quantize", "dequantize", "momentum"],
                     help="ns: the Newton-Schulz step (default); quantize / dequantize: the standalone "
                          "NVFP4 calls over every matrix of the workload (row axis); momentum: one "
@@ -173,15 +175,84 @@ def flops_per_launch(w, kind):
 
 
 def bytes_per_launch(w, kind):
-    """Algorithmic HBM bytes of the memory-bound phases (read G once, write X_0 and both views)."""
+    """Algorithmic HBM bytes of one launch of each phase: every tensor the phase must read
+    or write once (for the products: their FP32 inputs and outputs and their NVFP4
+    operands and views; the re-reads of operand tiles between output tiles are an
+    implementation cost and not counted).  Per matrix in working orientation m <= n:
+      reduce    4 mn (G)
+      preamble  4 mn (G) + 4 mn (X_0) + 2 x 0.5625 mn (both views)
+      gram_x    0.5625 mn (qX) + 4 m^2 (T+1)/(2T) (A, the 256 x 256 tiles on and above the
+                diagonal, T = m/256) + 0.5625 m^2 (qA, both triangles)
+      gram_a    4 m^2 (T+1)/(2T) (A) + 0.5625 m^2 (qA) + 0.5625 m^2 (qB)
+      update    0.5625 m^2 (qB) + 0.5625 mn (qX16x1) + 4 mn (X) + 4 mn (X') + 2 x 0.5625 mn
+                (both views of X'; the last update writes the FP32 output instead)"""
     tot = 0.0
     for (r, c) in w.shapes:
-        e = r * c
+        m, n = min(r, c), max(r, c)
+        e = m * n
+        tiles = max(1, (m + 255) // 256)
+        upper = 4.0 * m * m * (tiles + 1) / (2 * tiles)
         if kind == "reduce":
             tot += 4 * e
         elif kind == "preamble":
             tot += 4 * e + 4 * e + 2 * (e / 2 + e / 16)
+        elif kind == "gram_x":
+            tot += 0.5625 * e + upper + 0.5625 * m * m
+        elif kind == "gram_a":
+            tot += upper + 2 * 0.5625 * m * m
+        elif kind == "update":
+            tot += 0.5625 * m * m + 0.5625 * e + 8 * e + 2 * 0.5625 * e
     return tot
+
+
+def bf16_comparator(F, Gs, w, steps: int, flush, l2_bytes: int):
+    """Time the BF16 comparison step (fs4_root_ns_bf16_batched: the same Newton-Schulz
+    plan with BF16 operands on tcgen05 kind::f16) on the same matrices, per phase with
+    CUDA events on the launching stream; the pages compare Q-Root with an optimized
+    BF16 implementation of the same step (Full-Stack FP4, Section 4.4, Table 6)."""
+    import torch
+    lib = F._lib.lib()
+    K = w.K
+    outs = [torch.empty_like(G) for G in Gs]
+    arr = F._descs(Gs, outs, w.coeffs)
+    need = int(lib.fs4_root_ns_bf16_batched_workspace_size(len(Gs), arr))
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    n_ev = 3 + 3 * K
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(steps)]
+    for row in evs:
+        for e in row:
+            e.record(stream)
+
+    def call(row=None):
+        if row is None:
+            st = lib.fs4_root_ns_bf16_batched(len(Gs), arr, K, w.clip_k, 0, ws.data_ptr(), need,
+                                              stream.cuda_stream)
+        else:
+            ev_arr = (F._lib.c_vp * n_ev)(*[e.cuda_event for e in row])
+            st = lib.fs4_root_ns_bf16_batched_timed(len(Gs), arr, K, w.clip_k, 0, ws.data_ptr(), need,
+                                                    stream.cuda_stream, ev_arr, n_ev)
+        F.check(st, "fs4_root_ns_bf16_batched")
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    for row in evs:
+        if flush is not None:
+            flush.zero_()
+        call(row)
+    torch.cuda.synchronize()
+    F.check(F.device_status(ws), "device status after the BF16 comparison steps")
+    ms = statistics.mean(row[0].elapsed_time(row[-1]) for row in evs)
+    kinds = phase_kinds(K)
+    per_kind = {}
+    for row in evs:
+        for i, kind in enumerate(kinds):
+            per_kind.setdefault(kind, []).append(row[i].elapsed_time(row[i + 1]))
+    phase = {k: statistics.mean(v) * (1 if k in ("reduce", "preamble") else K) for k, v in per_kind.items()}
+    del ws, outs
+    torch.cuda.empty_cache()
+    return ms, phase
 
 
 def cpu_cores():
@@ -509,19 +580,28 @@ def main():
     # The GEMM kernels are timed one launch at a time (milliseconds each), so the
     # burst figure is the denominator: dense FP4 = 4 x the burst bf16 GEMM rate.
     fp4_peak = 4.0 * peaks["bf16_tflops"]
+    # The dominant kernel's roofline is the larger of its two floors: algorithmic FLOPs at
+    # the dense-FP4 peak and algorithmic bytes at the HBM peak.  (The update product of the
+    # 3072-row matrices moves 9.7 bytes of epilogue data per element of X for 2m FLOPs, so
+    # at m = 3072 its HBM floor is above its tensor floor.)
+    hbm_ach = bytes_per_launch(w, dom) / (dom_ms * 1e-3) / 1e9
+    hbm = {"bound": "hbm", "achieved": hbm_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+           "frac": hbm_ach / peaks["hbm_gbs"], "bytes_per_launch": bytes_per_launch(w, dom)}
     if dom in ("gram_x", "gram_a", "update"):
         achieved = flops_per_launch(w, dom) / (dom_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
-                "frac": achieved / fp4_peak}
+        ten = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+               "frac": achieved / fp4_peak, "flops_per_launch": flops_per_launch(w, dom)}
+        t_flop = flops_per_launch(w, dom) / (fp4_peak * 1e12)
+        t_byte = bytes_per_launch(w, dom) / (peaks["hbm_gbs"] * 1e9)
+        roof = dict(hbm if t_byte > t_flop else ten)
+        roof["other_bound"] = ten if t_byte > t_flop else hbm
     else:
-        achieved = bytes_per_launch(w, dom) / (dom_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"]}
+        roof = dict(hbm)
     roof["kernel"] = dom
     roof["ms_per_launch"] = dom_ms
     roof["peak_source"] = (f"dense FP4 = 4 x bf16_tflops, the burst figure ({peak_src} MEASURED_PEAKS.json; "
-                           f"4 = nominal FP4/BF16 dense ratio)" if roof["bound"] == "tensor"
-                           else f"hbm_gbs ({peak_src} MEASURED_PEAKS.json)")
+                           f"4 = nominal FP4/BF16 dense ratio); HBM = hbm_gbs ({peak_src} "
+                           f"MEASURED_PEAKS.json)")
     roof["traffic"] = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
@@ -535,6 +615,22 @@ def main():
     value = job_rate(world, len(Gs), ms_step)
     tflops = world * w.flops_algorithmic() / (ms_step * 1e-3) / 1e12
     phase_ms = {k: statistics.mean(v) * (1 if k in ("reduce", "preamble") else K) for k, v in per_kind.items()}
+
+    comparator = None
+    if not args.no_bf16 and args.quant == "plain" and args.clip == "rms":
+        bms, bphase = bf16_comparator(F, Gs, w, max(2, min(args.steps, 5)), flush, l2_bytes)
+        peaks_b, _ = measured_peaks()
+        bf16_tflops = w.flops_algorithmic() / (bms * 1e-3) / 1e12
+        comparator = {
+            "precision": "bf16 operands (tcgen05 kind::f16), fp32 accumulate, same plan and fusion",
+            "ms_per_step": bms, "value": job_rate(world, len(Gs), bms), "unit": UNIT,
+            "tflops_algorithmic": bf16_tflops,
+            "frac_bf16_peak": bf16_tflops / peaks_b["bf16_tflops"],
+            "nvfp4_speedup": bms / ms_step,
+            "phase_ms_per_step": bphase,
+            "context": "Full-Stack FP4 Table 6 (RTX 5090, d = 4096): Root BF16 344.55 ms vs NVFP4 "
+                       "109.80 ms per optimizer step (3.14x)",
+        }
 
     # end to end through the public API with host buffers: every step copies its inputs
     # in from pinned host memory, runs the call and copies its outputs back.  Steps are
@@ -625,6 +721,7 @@ def main():
             "tflops_dense_equivalent": world * w.flops_dense() / (ms_step * 1e-3) / 1e12,
             "phase_ms_per_step": phase_ms,
             "roofline": roof,
+            "comparator": comparator,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": args.steps * (2 + 6 * K + (3 if args.clip == "p99" else 0)),

@@ -341,6 +341,39 @@ fs4_status fs4_root_ns_batched_timed(int32_t count, const fs4_ns_desc* descs, in
                                      void* workspace, size_t workspace_bytes, void* stream,
                                      void* const* phase_events, int32_t n_events);
 
+/* -------------------------------------------------- BF16 comparison step */
+
+/* The same Newton-Schulz step with BF16 operands instead of NVFP4: the step of
+ * Section 2 "Root optimizer" as an optimized BF16 implementation takes it, the
+ * baseline that Section 4.4 and Table 6 (Root rows: BF16 344.55 ms, NVFP4
+ * 109.80 ms at d = 4096) compare the NVFP4 step against.  X_0 is normalised and
+ * clipped exactly as in fs4_root_ns; then K iterations of
+ *   Xb = bf16(X), A = Xb Xb^T, B = b A + c bf16(A) bf16(A)^T,
+ *   X <- a X + bf16(B) Xb,
+ * with bf16() rounding to nearest (ties to even), BF16 x BF16 products on the
+ * tensor cores (tcgen05 kind::f16) accumulated in FP32, and X, A, B held in FP32.
+ * Tall matrices are transposed as in fs4_root_ns.  There are no tensor scales, so
+ * a call launches 2 + 3K kernels.  Arguments, layouts, ownership, aliasing rules
+ * and errors as fs4_root_ns_batched; flags may hold FS4_STOP_AFTER,
+ * FS4_NS_CLIP_QUANTILE and FS4_TEST_STALL (FS4_NS_RHT and FS4_NS_ADAPTIVE46 give
+ * FS4_ERR_INVALID_ARG).  A stop after product 1 writes B (FP32) over A as in the
+ * NVFP4 step.  The workspace (larger than the NVFP4 step's: 2 bytes per element
+ * for each BF16 view) is sized by fs4_root_ns_bf16_batched_workspace_size. */
+size_t fs4_root_ns_bf16_batched_workspace_size(int32_t count, const fs4_ns_desc* descs);
+
+fs4_status fs4_root_ns_bf16_batched(int32_t count, const fs4_ns_desc* descs, int32_t K,
+                                    float clip_k, uint32_t flags, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/* fs4_root_ns_bf16_batched with CUDA events recorded around each phase, at the
+ * same 3 + 3K positions as fs4_root_ns_batched_timed. */
+fs4_status fs4_root_ns_bf16_batched_timed(int32_t count, const fs4_ns_desc* descs, int32_t K,
+                                          float clip_k, uint32_t flags, void* workspace,
+                                          size_t workspace_bytes, void* stream,
+                                          void* const* phase_events, int32_t n_events);
+
+
+
 /* ------------------------------------------------------------ no-alloc variant */
 
 /* Bytes of the workspace array built into the library for fs4_root_ns_noalloc. */
@@ -390,6 +423,14 @@ typedef struct {
 
 fs4_status fs4_root_ns_layout(int32_t count, const fs4_ns_desc* descs, int32_t index,
                               fs4_ns_layout* layout);
+
+/* Workspace offsets of matrix `index` of a BF16 step (see fs4_root_ns_layout).  The
+ * *_codes fields locate the BF16 views in the TILED BF16 layout: tiles of 128 rows x
+ * 64 elements (16384 bytes), tile (r/128, c/64) at ((r/128)*(Cp/64) + c/64)*16384,
+ * row r%128 at byte 128*(r%128), its 16-byte chunk j = (c%64)/8 at chunk position
+ * j ^ (r%8); the *_scales fields are unused. */
+fs4_status fs4_root_ns_bf16_layout(int32_t count, const fs4_ns_desc* descs, int32_t index,
+                                   fs4_ns_layout* layout);
 
 #ifdef __cplusplus
 }

@@ -21,7 +21,8 @@ MUON_COEFFS = (3.4445, -4.7750, 2.0315)
 __all__ = [
     "quantize", "dequantize", "gemm", "root_ns", "root_ns_batched", "ns_workspace_size",
     "ns_batched_workspace_size", "ns_layout", "device_status", "tiled_shape", "Fs4Error",
-    "momentum_nvfp4", "root_ns_batched_nvfp4",
+    "momentum_nvfp4", "root_ns_batched_nvfp4", "root_ns_bf16_batched", "ns_bf16_batched_workspace_size",
+    "ns_bf16_layout",
     "MUON_COEFFS", "stop_after", "FS4_AXIS_ROW", "FS4_AXIS_COL", "FS4_TEST_STALL",
     "FS4_NS_RHT", "FS4_NS_ADAPTIVE46", "FS4_NS_CLIP_QUANTILE",
 ]
@@ -281,6 +282,45 @@ def root_ns_batched_nvfp4(states, K: int = 5, coeffs=None, clip_k: float = 3.0,
                                                _stream(stream)),
           "fs4_root_ns_batched_nvfp4")
     return outs
+
+
+def root_ns_bf16_batched(Gs: Sequence[torch.Tensor], K: int = 5, coeffs=None, clip_k: float = 3.0,
+                         outs: Sequence[torch.Tensor] | None = None,
+                         workspace: torch.Tensor | None = None, flags: int = 0, stream=None,
+                         clip_quantile: float | None = None):
+    """The BF16 comparison step (fs4_root_ns_bf16_batched): the same Newton-Schulz
+    iteration with BF16 operands on the tensor cores instead of NVFP4.  Arguments as
+    root_ns_batched (no quantiser options)."""
+    if clip_quantile is not None:
+        flags |= FS4_NS_CLIP_QUANTILE
+        clip_k = clip_quantile
+    for G in Gs:
+        _check_f32_matrix(G, "G")
+    if coeffs is None:
+        coeffs = [MUON_COEFFS] * len(Gs)
+    if outs is None:
+        outs = [torch.empty_like(G) for G in Gs]
+    arr = _descs(Gs, outs, coeffs)
+    need = int(_lib.lib().fs4_root_ns_bf16_batched_workspace_size(len(Gs), arr))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=Gs[0].device)
+    check(_lib.lib().fs4_root_ns_bf16_batched(len(Gs), arr, K, clip_k, flags, workspace.data_ptr(),
+                                              workspace.numel(), _stream(stream)),
+          "fs4_root_ns_bf16_batched")
+    return outs
+
+
+def ns_bf16_batched_workspace_size(shapes: Sequence[tuple[int, int]]) -> int:
+    return int(_lib.lib().fs4_root_ns_bf16_batched_workspace_size(len(shapes), _shape_descs(shapes)))
+
+
+def ns_bf16_layout(shapes: Sequence[tuple[int, int]], index: int = 0) -> NsLayout:
+    """Workspace offsets of matrix `index` of a BF16 step on matrices of these shapes."""
+    arr = _shape_descs(shapes)
+    lay = NsLayout()
+    check(_lib.lib().fs4_root_ns_bf16_layout(len(shapes), arr, index, ctypes.byref(lay)),
+          "fs4_root_ns_bf16_layout")
+    return lay
 
 
 def ns_layout(shapes: Sequence[tuple[int, int]], index: int = 0) -> NsLayout:

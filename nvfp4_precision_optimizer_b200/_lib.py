@@ -74,11 +74,18 @@ SIGNATURES = {
                                           c_i32, c_f32, c_u32, c_vp, c_vp, c_sz, c_vp]),
     "fs4_root_ns_batched_timed": (c_i32, [c_i32, ctypes.POINTER(NsDesc), c_i32, c_f32, c_u32,
                                           c_vp, c_vp, c_sz, c_vp, ctypes.POINTER(c_vp), c_i32]),
+    "fs4_root_ns_bf16_batched_workspace_size": (c_sz, [c_i32, ctypes.POINTER(NsDesc)]),
+    "fs4_root_ns_bf16_batched": (c_i32, [c_i32, ctypes.POINTER(NsDesc), c_i32, c_f32, c_u32, c_vp,
+                                         c_sz, c_vp]),
+    "fs4_root_ns_bf16_batched_timed": (c_i32, [c_i32, ctypes.POINTER(NsDesc), c_i32, c_f32, c_u32,
+                                               c_vp, c_sz, c_vp, ctypes.POINTER(c_vp), c_i32]),
     "fs4_root_ns_noalloc": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i64, c_i32, c_f32, c_f32,
                                     c_f32, c_f32, c_vp]),
     "fs4_device_status": (c_i32, [c_vp, c_vp]),
     "fs4_status_string": (ctypes.c_char_p, [c_i32]),
     "fs4_root_ns_layout": (c_i32, [c_i32, ctypes.POINTER(NsDesc), c_i32, ctypes.POINTER(NsLayout)]),
+    "fs4_root_ns_bf16_layout": (c_i32, [c_i32, ctypes.POINTER(NsDesc), c_i32,
+                                        ctypes.POINTER(NsLayout)]),
 }
 
 _lib = None

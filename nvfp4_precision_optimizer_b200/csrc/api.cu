@@ -82,7 +82,7 @@ fs4_status validate_desc(const fs4_ns_desc& d, const fs4_nvfp4_state* st, bool s
 
 // Lay out the workspace: [header | state blocks of all matrices | big buffers of all matrices].
 fs4_status make_plan(int32_t count, const fs4_ns_desc* descs, Plan* pl,
-                     const fs4_nvfp4_state* states = nullptr, bool sizing = false) {
+                     const fs4_nvfp4_state* states = nullptr, bool sizing = false, bool bf16 = false) {
   if (count < 1 || count > kMaxBatch) return FS4_ERR_SHAPE;
   if (!descs) return FS4_ERR_INVALID_ARG;
   pl->count = count;
@@ -119,7 +119,7 @@ fs4_status make_plan(int32_t count, const fs4_ns_desc* descs, Plan* pl,
   off = pl->zero_bytes;
   for (int i = 0; i < count; ++i) {
     pl->mat[i].big_off = off;
-    off += align_up(big_block_bytes(pl->mat[i].mp, pl->mat[i].np), 1024);
+    off += align_up(big_block_bytes(pl->mat[i].mp, pl->mat[i].np, bf16), 1024);
   }
   pl->total_bytes = off;
   if (sizing) return FS4_OK;
@@ -164,7 +164,7 @@ thread_local NsParams t_params;
 
 fs4_status run_ns(const Plan& pl, int32_t K, float clip_k, uint32_t flags, const uint16_t* rht_masks,
                   uint8_t* ws,
-                  cudaStream_t st, int num_sms, void* const* events = nullptr) {
+                  cudaStream_t st, int num_sms, void* const* events = nullptr, bool bf16 = false) {
   int ev_i = 0;
   auto mark = [&]() -> bool {
     if (!events) return true;
@@ -179,7 +179,8 @@ fs4_status run_ns(const Plan& pl, int32_t K, float clip_k, uint32_t flags, const
   p.ws = ws;
   p.opts = ((flags & FS4_NS_RHT) ? kOptRht : 0u) | ((flags & FS4_NS_ADAPTIVE46) ? kOpt46 : 0u) |
            ((flags & FS4_NS_CLIP_QUANTILE) ? kOptQuantile : 0u) |
-           (pl.mat[0].qcodes ? kOptNvSrc : 0u);   // a call's matrices are all FP32 or all NVFP4
+           (pl.mat[0].qcodes ? kOptNvSrc : 0u) |  // a call's matrices are all FP32 or all NVFP4
+           (bf16 ? kOptBf16 : 0u);
   if (flags & FS4_NS_RHT)
     for (int i = 0; i < 3 * K; ++i) p.rht[i] = rht_masks[i];
   std::memcpy(p.mat, pl.mat, sizeof(MatDesc) * pl.count);
@@ -327,6 +328,33 @@ size_t fs4_root_ns_batched_workspace_size(int32_t count, const fs4_ns_desc* desc
   return (size_t)pl.total_bytes;
 }
 
+static fs4_status batched_impl(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
+                               uint32_t flags, const uint16_t* rht_masks, void* workspace,
+                               size_t workspace_bytes, void* stream, void* const* events,
+                               int32_t n_events, const fs4_nvfp4_state* states, bool bf16);
+
+size_t fs4_root_ns_bf16_batched_workspace_size(int32_t count, const fs4_ns_desc* descs) {
+  static thread_local Plan pl;
+  if (make_plan(count, descs, &pl, nullptr, true, true) != FS4_OK) return 0;
+  return (size_t)pl.total_bytes;
+}
+
+fs4_status fs4_root_ns_bf16_batched(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
+                                    uint32_t flags, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  return batched_impl(count, descs, K, clip_k, flags, nullptr, workspace, workspace_bytes, stream,
+                      nullptr, 0, nullptr, true);
+}
+
+fs4_status fs4_root_ns_bf16_batched_timed(int32_t count, const fs4_ns_desc* descs, int32_t K,
+                                          float clip_k, uint32_t flags, void* workspace,
+                                          size_t workspace_bytes, void* stream,
+                                          void* const* phase_events, int32_t n_events) {
+  if (!phase_events) return FS4_ERR_INVALID_ARG;
+  return batched_impl(count, descs, K, clip_k, flags, nullptr, workspace, workspace_bytes, stream,
+                      phase_events, n_events, nullptr, true);
+}
+
 size_t fs4_root_ns_workspace_size(int64_t m, int64_t n) {
   if (m < 16 || n < 16 || m > FS4_MAX_DIM || n > FS4_MAX_DIM || m % 16 || n % 16) return 0;
   const int64_t mm = m < n ? m : n, nn = m < n ? n : m;
@@ -338,7 +366,8 @@ size_t fs4_root_ns_workspace_size(int64_t m, int64_t n) {
 static fs4_status batched_impl(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
                                uint32_t flags, const uint16_t* rht_masks, void* workspace,
                                size_t workspace_bytes, void* stream, void* const* events,
-                               int32_t n_events, const fs4_nvfp4_state* states = nullptr) {
+                               int32_t n_events, const fs4_nvfp4_state* states,
+                               bool bf16) {
   if (K < 1 || K > FS4_MAX_ITERS) return FS4_ERR_SHAPE;
   if (!std::isfinite(clip_k)) return FS4_ERR_INVALID_ARG;
   if (flags & ~(uint32_t)(0xFF00u | FS4_TEST_STALL | FS4_NS_RHT | FS4_NS_ADAPTIVE46 |
@@ -346,8 +375,9 @@ static fs4_status batched_impl(int32_t count, const fs4_ns_desc* descs, int32_t 
     return FS4_ERR_INVALID_ARG;
   if ((flags & FS4_NS_CLIP_QUANTILE) && !(clip_k > 0.0f && clip_k <= 1.0f)) return FS4_ERR_INVALID_ARG;
   if ((flags & FS4_NS_RHT) && !rht_masks) return FS4_ERR_INVALID_ARG;
+  if (bf16 && (flags & (FS4_NS_RHT | FS4_NS_ADAPTIVE46))) return FS4_ERR_INVALID_ARG;
   static thread_local Plan pl;
-  const fs4_status s = make_plan(count, descs, &pl, states);
+  const fs4_status s = make_plan(count, descs, &pl, states, false, bf16);
   if (s != FS4_OK) return s;
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < (size_t)pl.total_bytes)
     return FS4_ERR_WORKSPACE;
@@ -376,7 +406,7 @@ static fs4_status batched_impl(int32_t count, const fs4_ns_desc* descs, int32_t 
   const fs4_status ds = device_info(&di);
   if (ds != FS4_OK) return ds;
   return run_ns(pl, K, clip_k, flags, rht_masks, static_cast<uint8_t*>(workspace),
-                static_cast<cudaStream_t>(stream), di.num_sms, events);
+                static_cast<cudaStream_t>(stream), di.num_sms, events, bf16);
 }
 
 fs4_status fs4_root_ns_batched_nvfp4(int32_t count, const fs4_ns_desc* descs,
@@ -385,21 +415,21 @@ fs4_status fs4_root_ns_batched_nvfp4(int32_t count, const fs4_ns_desc* descs,
                                      size_t workspace_bytes, void* stream) {
   if (!states) return FS4_ERR_INVALID_ARG;
   return batched_impl(count, descs, K, clip_k, flags, rht_masks, workspace, workspace_bytes, stream,
-                      nullptr, 0, states);
+                      nullptr, 0, states, false);
 }
 
 fs4_status fs4_root_ns_batched(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
                                uint32_t flags, void* workspace, size_t workspace_bytes,
                                void* stream) {
   return batched_impl(count, descs, K, clip_k, flags, nullptr, workspace, workspace_bytes, stream,
-                      nullptr, 0);
+                      nullptr, 0, nullptr, false);
 }
 
 fs4_status fs4_root_ns_batched_ex(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
                                   uint32_t flags, const uint16_t* rht_masks, void* workspace,
                                   size_t workspace_bytes, void* stream) {
   return batched_impl(count, descs, K, clip_k, flags, rht_masks, workspace, workspace_bytes, stream,
-                      nullptr, 0);
+                      nullptr, 0, nullptr, false);
 }
 
 fs4_status fs4_root_ns_batched_timed(int32_t count, const fs4_ns_desc* descs, int32_t K,
@@ -408,7 +438,7 @@ fs4_status fs4_root_ns_batched_timed(int32_t count, const fs4_ns_desc* descs, in
                                      void* const* phase_events, int32_t n_events) {
   if (!phase_events) return FS4_ERR_INVALID_ARG;
   return batched_impl(count, descs, K, clip_k, flags, rht_masks, workspace, workspace_bytes, stream,
-                      phase_events, n_events);
+                      phase_events, n_events, nullptr, false);
 }
 
 fs4_status fs4_root_ns(const float* G, int64_t m, int64_t n, int64_t ld, float* out,
@@ -446,15 +476,15 @@ const char* fs4_status_string(fs4_status s) {
   }
 }
 
-fs4_status fs4_root_ns_layout(int32_t count, const fs4_ns_desc* descs, int32_t index,
-                              fs4_ns_layout* layout) {
+static fs4_status layout_impl(int32_t count, const fs4_ns_desc* descs, int32_t index,
+                              fs4_ns_layout* layout, bool bf16) {
   if (!layout) return FS4_ERR_INVALID_ARG;
   static thread_local Plan pl;
-  const fs4_status s = make_plan(count, descs, &pl, nullptr, true);
+  const fs4_status s = make_plan(count, descs, &pl, nullptr, true, bf16);
   if (s != FS4_OK) return s;
   if (index < 0 || index >= count) return FS4_ERR_INVALID_ARG;
   const MatDesc& d = pl.mat[index];
-  const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
+  const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off, bf16);
   layout->mp = d.mp;
   layout->np = d.np;
   layout->X = L.X;
@@ -467,6 +497,16 @@ fs4_status fs4_root_ns_layout(int32_t count, const fs4_ns_desc* descs, int32_t i
   layout->qB_codes = L.qB; layout->qB_scales = L.sB;
   layout->scalars = L.state + (int64_t)offsetof(NsState, sg);
   return FS4_OK;
+}
+
+fs4_status fs4_root_ns_layout(int32_t count, const fs4_ns_desc* descs, int32_t index,
+                              fs4_ns_layout* layout) {
+  return layout_impl(count, descs, index, layout, false);
+}
+
+fs4_status fs4_root_ns_bf16_layout(int32_t count, const fs4_ns_desc* descs, int32_t index,
+                                   fs4_ns_layout* layout) {
+  return layout_impl(count, descs, index, layout, true);
 }
 
 }  // extern "C"

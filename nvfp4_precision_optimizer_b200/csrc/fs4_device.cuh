@@ -10,6 +10,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -44,6 +45,22 @@ __host__ __device__ __forceinline__ int64_t tiled_chunk_offset(int64_t r, int64_
   const int64_t rr = r & 127;
   const int64_t j = (c & 255) >> 5;
   return tile * kTileBytes + rr * 128 + ((j ^ (rr & 7)) << 4);
+}
+
+// The same TILED layout for BF16 operands (the BF16 comparison step): 16 KB tiles of
+// 128 rows x 64 elements (128-byte rows, chunk j of row r at chunk position j ^ (r % 8)).
+// Byte offset of the 16-byte chunk that holds columns [c, c+8) of row r (c % 8 == 0).
+__host__ __device__ __forceinline__ int64_t tiled_chunk_offset_bf16(int64_t r, int64_t c, int64_t Cp) {
+  const int64_t tile = (r >> 7) * (Cp >> 6) + (c >> 6);
+  const int64_t rr = r & 127;
+  const int64_t j = (c & 63) >> 3;
+  return tile * kTileBytes + rr * 128 + ((j ^ (rr & 7)) << 4);
+}
+
+// Two FP32 values rounded to BF16 (round to nearest, ties to even), the first in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // Byte offset of the scale of row r, column block kb = c / 16.
@@ -251,17 +268,20 @@ __device__ __forceinline__ void rht16(float* x, uint32_t mask) {
   for (int i = 0; i < 16; ++i) x[i] = __fmul_rn(x[i], 0.25f);
 }
 
+// The two E2M1 values (signed) of one code byte as an f16x2: the low nibble in the low
+// half.  The byte is handed to the conversion through its own 8-bit register, taken
+// from a 32-bit value with cvt, so no vector unpacking of a packed word is involved.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+  uint32_t h;
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h) : "r"(byte));
+  return h;
+}
+
 // The 8 E2M1 values (signed) of one packed word as 4 f16x2: element 2i in the low
 // half of h[i] (byte i of w, low nibble first).
 __device__ __forceinline__ void e2m1_decode8(uint32_t w, uint32_t* h) {
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
-      : "r"(w));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = e2m1x2_to_f16x2((w >> (8 * i)) & 0xFFu);
 }
 
 // The 16 E2M1 values (signed, as FP32) of a block's packed codes.
@@ -476,6 +496,22 @@ __device__ __forceinline__ uint64_t sdesc_sf_atom(uint32_t saddr) {
 // FP32 accumulate, M x N.
 __host__ __device__ constexpr uint32_t idesc_mxf4nvf4(int M, int N) {
   return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor: kind::f16 with BF16 A and B, FP32 accumulate, K-major A and B, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D (TMEM) (+)= A(smem) * B(smem)^T, BF16 operands, FP32 accumulator; K = 16.
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 // Copy one 512-byte scale atom from shared memory into 4 TMEM columns at

@@ -62,14 +62,19 @@ __host__ __device__ inline int64_t state_block_bytes(int64_t mp, int64_t np) {
   return align_up(4096 + 4 * (3 * mp + np) + 4 * kQBins1, 256);
 }
 
-// Bytes of the large buffers of an mp x np matrix.
-__host__ __device__ inline int64_t big_block_bytes(int64_t mp, int64_t np) {
-  const int64_t xn = mp * np, aa = mp * mp;
-  return 4 * xn + 4 * aa + 2 * (xn / 2 + xn / 16) + 2 * (xn / 2 + xn / 16) + 2 * (aa / 2 + aa / 16);
+// Bytes per element of one operand view: NVFP4 (codes 1/2 B + scales 1/16 B) or BF16 (2 B).
+// Returned as sixteenths of a byte so that both are integers.
+__host__ __device__ inline int64_t view_sixteenths(bool bf16) { return bf16 ? 32 : 9; }
+
+// Bytes of the large buffers of an mp x np matrix (bf16: the BF16 comparison step,
+// whose operand views are BF16 instead of NVFP4).
+__host__ __device__ inline int64_t big_block_bytes(int64_t mp, int64_t np, bool bf16 = false) {
+  const int64_t xn = mp * np, aa = mp * mp, v = view_sixteenths(bf16);
+  return 4 * xn + 4 * aa + 4 * (xn * v / 16) + 2 * (aa * v / 16);
 }
 
 __host__ __device__ inline MatLayout mat_layout(int64_t mp, int64_t np, int64_t state_off,
-                                                int64_t big_off) {
+                                                int64_t big_off, bool bf16 = false) {
   MatLayout L;
   L.state = state_off;
   L.rowsumX = state_off + 4096;
@@ -78,13 +83,16 @@ __host__ __device__ inline MatLayout mat_layout(int64_t mp, int64_t np, int64_t 
   L.rowsumB = L.rowsumA + 4 * mp;
   L.qhist = L.rowsumB + 4 * mp;
   const int64_t xn = mp * np, aa = mp * mp;
+  // NVFP4: codes (1/2 B per element) then scales (1/16 B); BF16: 2 B per element, no scales
+  const int64_t cx = bf16 ? 2 * xn : xn / 2, sx = bf16 ? 0 : xn / 16;
+  const int64_t ca = bf16 ? 2 * aa : aa / 2, sa = bf16 ? 0 : aa / 16;
   int64_t o = big_off;
   L.X = o; o += 4 * xn;
   L.A = o; o += 4 * aa;
-  for (int s = 0; s < 2; ++s) { L.qX[s] = o; o += xn / 2; L.sX[s] = o; o += xn / 16; }
-  for (int s = 0; s < 2; ++s) { L.qXT[s] = o; o += xn / 2; L.sXT[s] = o; o += xn / 16; }
-  L.qA = o; o += aa / 2; L.sA = o; o += aa / 16;
-  L.qB = o; o += aa / 2; L.sB = o; o += aa / 16;
+  for (int s = 0; s < 2; ++s) { L.qX[s] = o; o += cx; L.sX[s] = o; o += sx; }
+  for (int s = 0; s < 2; ++s) { L.qXT[s] = o; o += cx; L.sXT[s] = o; o += sx; }
+  L.qA = o; o += ca; L.sA = o; o += sa;
+  L.qB = o; o += ca; L.sB = o; o += sa;
   return L;
 }
 
@@ -110,6 +118,7 @@ struct MatDesc {
 constexpr uint32_t kOptRht = 1u, kOpt46 = 2u;   // NsParams::opts
 constexpr uint32_t kOptQuantile = 4u;            // clip at the clip_k-quantile of |X_0|
 constexpr uint32_t kOptNvSrc = 8u;               // every G is an NVFP4 state (MatDesc::qcodes)
+constexpr uint32_t kOptBf16 = 16u;               // BF16 operand views and kind::f16 products
 
 struct NsParams {
   int32_t count;

@@ -66,17 +66,22 @@ constexpr int EPI_WARP_FLOATS = kStageBufs * kStageFloats;
 static_assert(EPI_WARP_FLOATS >= TRANS_FLOATS, "the plain epilogue reuses the stage");
 constexpr float kBoundInflate = 1.0f + 1.0f / 256.0f;
 
-// Per-kernel configuration.
-template <Epi E>
+// Per-kernel configuration.  kBf16: the BF16 comparison step, whose operands are BF16
+// tiles of the same 128-byte rows (64 elements of K per tile instead of 256) and carry
+// no scale factors.
+template <Epi E, bool kBf16 = false>
 struct Cfg {
   static constexpr int kStages = 3;
-  static constexpr int B_BYTES = BN * BK / 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int kTileK = kBf16 ? 64 : BK;              // K elements per stage
+  static constexpr int B_BYTES = BN * 128;                    // 256 rows of 128 bytes
+  static constexpr int SFA = kBf16 ? 0 : SFA_BYTES;
+  static constexpr int SFB = kBf16 ? 0 : SFB_BYTES;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA + SFB;
   static constexpr int BAR_BYTES = 256;
   static constexpr int EPI_FLOATS = kStageBufs * kStageFloats;
   static constexpr int SMEM_BYTES =
       1024 + kStages * STAGE_BYTES + 8 * EPI_FLOATS * 4 + BAR_BYTES + 128 * 8;
-  static constexpr uint32_t kIdesc = idesc_mxf4nvf4(BM, BN);
+  static constexpr uint32_t kIdesc = kBf16 ? idesc_bf16(BM, BN) : idesc_mxf4nvf4(BM, BN);
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(SMEM_BYTES <= 232448, "over the per-CTA shared-memory limit");
   static_assert((2 * kStages + 4) * 8 + 12 <= BAR_BYTES, "barrier block too small");
@@ -87,11 +92,11 @@ struct Job {
   int64_t row0, col0;
   int mirror;        // off-diagonal symmetric tile
   int b_half;        // only the first 128 rows of the B tile exist
-  int kt;            // number of 256-wide K tiles
+  int kt;            // number of K tiles (256 NVFP4 or 64 BF16 elements each)
   const uint8_t* a_codes; const uint8_t* a_sf;
   const uint8_t* b_codes; const uint8_t* b_sf;
   int64_t a_tile_row, b_tile_row;   // 128-row tile index of the A / B operand
-  int64_t ktiles_total;             // K tiles per operand row band (Kp / 256)
+  int64_t ktiles_total;             // K tiles per operand row band
 };
 
 __device__ __forceinline__ int owner_of(const int32_t* prefix, int count, int32_t u) {
@@ -113,8 +118,9 @@ __device__ __forceinline__ void upper_tile(int32_t s, int32_t T, int32_t& P, int
 // Work unit u of kernel E: one 128 x 256 output tile.  The Newton-Schulz units of a
 // matrix go through its 256 x 256 blocks in order, the two 128-row halves of a block
 // one after the other (they share the block's B rows in L2).
-template <Epi E>
+template <Epi E, bool kBf16 = false>
 __device__ __forceinline__ Job make_job(int32_t u, const NsParams& p, const GemmPlainArgs& g) {
+  constexpr int TK = Cfg<E, kBf16>::kTileK;
   Job j;
   j.mirror = 0;
   j.b_half = 0;
@@ -132,7 +138,7 @@ __device__ __forceinline__ Job make_job(int32_t u, const NsParams& p, const Gemm
   } else {
     const int mi = owner_of(p.prefix, p.count, u);
     const MatDesc& d = p.mat[mi];
-    const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
+    const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off, kBf16);
     const int32_t lu = u - p.prefix[mi];
     const int slot = p.iter & 1;
     j.mat = mi;
@@ -145,11 +151,11 @@ __device__ __forceinline__ Job make_job(int32_t u, const NsParams& p, const Gemm
       j.col0 = 256 * (int64_t)Q;
       j.mirror = (P != Q) ? 1 : 0;
       if constexpr (E == Epi::GramX) {
-        j.kt = d.np / BK;
+        j.kt = d.np / TK;
         j.a_codes = j.b_codes = p.ws + (slot ? L.qX[1] : L.qX[0]);
         j.a_sf = j.b_sf = p.ws + (slot ? L.sX[1] : L.sX[0]);
       } else {
-        j.kt = d.mp / BK;
+        j.kt = d.mp / TK;
         j.a_codes = j.b_codes = p.ws + L.qA;
         j.a_sf = j.b_sf = p.ws + L.sA;
       }
@@ -158,7 +164,7 @@ __device__ __forceinline__ Job make_job(int32_t u, const NsParams& p, const Gemm
       const int32_t I = tu / nJ;
       j.row0 = 256 * (int64_t)I + 128 * (int64_t)half;
       j.col0 = (int64_t)(tu - I * nJ) * 256;
-      j.kt = d.mp / BK;
+      j.kt = d.mp / TK;
       j.a_codes = p.ws + L.qB; j.a_sf = p.ws + L.sB;
       j.b_codes = p.ws + (slot ? L.qXT[1] : L.qXT[0]);
       j.b_sf = p.ws + (slot ? L.sXT[1] : L.sXT[0]);
@@ -343,6 +349,7 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
   constexpr bool kPackedQ = true;   // f32x2 quantiser (measured faster in all three kernels)
   constexpr bool kRht = (kOpts & kOptRht) != 0;    // Hadamard transform before quantising
   constexpr bool k46 = (kOpts & kOpt46) != 0;      // adaptive 4/6 block scaling
+  constexpr bool kBf16 = (kOpts & kOptBf16) != 0;  // BF16 comparison step: BF16 views
   // H16^r masks of the tensors this epilogue quantises (Section 3.4): GramX -> qA (product
   // qA qA^T of iteration k), GramA -> qB (update product of iteration k), Update -> the
   // next iterate's Gram view and update view (iteration k + 1)
@@ -371,7 +378,7 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
     const Job j = make_job<E>(u, p, g);
     const MatDesc& d = p.mat[j.mat];
     NsState* st = reinterpret_cast<NsState*>(p.ws + d.state_off);
-    const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
+    const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off, kBf16);
     if constexpr (!kIn) fp = tile_rows<E>(p, g, u, quad, ch, lane);
     // One lane polls the barrier (32 lanes polling one mbarrier serialise on its bank);
     // the warp then synchronises, which with tcgen05.fence::after_thread_sync below
@@ -387,7 +394,10 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
     const bool last = (E == Epi::Update) && p.last;
 
     float acc_scale, sg_out;
-    if constexpr (E == Epi::GramX) {
+    if constexpr (kBf16) {
+      acc_scale = 1.0f;   // BF16 operands carry no tensor scales
+      sg_out = 1.0f;
+    } else if constexpr (E == Epi::GramX) {
       const float sx = __ldcg(&st->sg[kSgX + k]);
       acc_scale = sx * sx;
       sg_out = __ldcg(&st->sg[kSgA + k]);
@@ -517,6 +527,28 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
           }
           if constexpr (E != Epi::GramA) stage_flush(buf, fp, c, lane);   // A or X' (FP32)
           else if (dbg_b) stage_flush(buf, fp, c, lane);
+          if constexpr (kBf16) {
+            // BF16 views (round to nearest even): the row's 16 values, and where needed
+            // column gcc + cc, rows gr0 + 16 hh ..; two 16-byte chunks each
+            uint32_t w[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(y[2 * e], y[2 * e + 1]);
+            *reinterpret_cast<uint4*>(row_codes + tiled_chunk_offset_bf16(gr, gcc, row_cp)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(row_codes + tiled_chunk_offset_bf16(gr, gcc + 8, row_cp)) =
+                make_uint4(w[4], w[5], w[6], w[7]);
+            if (need_col) {
+              float xc[16];
+              stage_load_col(buf, cc, hh, xc);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(xc[2 * e], xc[2 * e + 1]);
+              const int64_t rt = gcc + cc, k0 = gr0 + 16 * hh;
+              *reinterpret_cast<uint4*>(col_codes + tiled_chunk_offset_bf16(rt, k0, d.mp)) =
+                  make_uint4(w[0], w[1], w[2], w[3]);
+              *reinterpret_cast<uint4*>(col_codes + tiled_chunk_offset_bf16(rt, k0 + 8, d.mp)) =
+                  make_uint4(w[4], w[5], w[6], w[7]);
+            }
+          } else {
           // 1x16 view along this lane's row and, where needed, the 16x1 view of column
           // gcc + cc, rows gr0 + 16 hh ..: two independent quantiser chains side by side
           QBlock16 q, qc;
@@ -569,6 +601,7 @@ __device__ __forceinline__ void epilogue_ns(const NsParams& p, const GemmPlainAr
               *reinterpret_cast<uint16_t*>(ds) = static_cast<uint16_t>(qc.scale | (os << 8));
               if (s2 != 0.0f) atomicAdd(colsum + gcc + cc, s2);
             }
+          }
           }
         }
       }
@@ -649,7 +682,8 @@ __device__ __forceinline__ void epilogue_plain(const NsParams& p, const GemmPlai
 template <Epi E, uint32_t kOpts>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ NsParams p, const __grid_constant__ GemmPlainArgs g) {
-  using C = Cfg<E>;
+  constexpr bool kBf16 = (kOpts & kOptBf16) != 0;
+  using C = Cfg<E, kBf16>;
   constexpr int kStages = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -696,24 +730,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t it = 0;
       for (int32_t u = first; u < total && !*abort_flag; u += step) {
-        const Job j = make_job<E>(u, p, g);
+        const Job j = make_job<E, kBf16>(u, p, g);
         for (int kt = 0; kt < j.kt; ++kt, ++it) {
           const uint32_t s = it % kStages, use = it / kStages;
           if (!mbar_wait(&empty[s], (use & 1u) ^ 1u, status, abort_flag)) break;
           uint8_t* st = stage_base + s * C::STAGE_BYTES;
           uint8_t* st_b = st + A_BYTES;
           uint8_t* st_sfa = st_b + C::B_BYTES;
-          uint8_t* st_sfb = st_sfa + SFA_BYTES;
+          uint8_t* st_sfb = st_sfa + C::SFA;
           const int64_t at = j.a_tile_row * j.ktiles_total + kt;
-          const uint32_t bbytes = j.b_half ? (C::B_BYTES + SFB_BYTES) / 2 : (C::B_BYTES + SFB_BYTES);
-          mbar_arrive_expect_tx(&full[s], A_BYTES + SFA_BYTES + bbytes);
+          const uint32_t bbytes = j.b_half ? (C::B_BYTES + C::SFB) / 2 : (C::B_BYTES + C::SFB);
+          mbar_arrive_expect_tx(&full[s], A_BYTES + C::SFA + bbytes);
           bulk_g2s(st, j.a_codes + at * kTileBytes, A_BYTES, &full[s]);
-          bulk_g2s(st_sfa, j.a_sf + at * (4 * kAtomBytes), SFA_BYTES, &full[s]);
+          if constexpr (!kBf16) bulk_g2s(st_sfa, j.a_sf + at * (4 * kAtomBytes), SFA_BYTES, &full[s]);
           for (int h = 0; h < (j.b_half ? 1 : 2); ++h) {
             const int64_t bt = (j.b_tile_row + h) * j.ktiles_total + kt;
             bulk_g2s(st_b + h * kTileBytes, j.b_codes + bt * kTileBytes, kTileBytes, &full[s]);
-            bulk_g2s(st_sfb + h * (4 * kAtomBytes), j.b_sf + bt * (4 * kAtomBytes), 4 * kAtomBytes,
-                     &full[s]);
+            if constexpr (!kBf16)
+              bulk_g2s(st_sfb + h * (4 * kAtomBytes), j.b_sf + bt * (4 * kAtomBytes), 4 * kAtomBytes,
+                       &full[s]);
           }
         }
       }
@@ -734,7 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (p.stall) mbar_wait(stall_bar, 0, status, abort_flag);
       }
       for (int32_t u = first; u < total && !*abort_flag; u += step, ++tl) {
-        const Job j = make_job<E>(u, p, g);
+        const Job j = make_job<E, kBf16>(u, p, g);
         if (!mbar_wait(acc_empty, (tl & 1u) ^ 1u, status, abort_flag)) break;
         tc_fence_after();
         bool ok = true;
@@ -744,19 +779,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint8_t* st = stage_base + s * C::STAGE_BYTES;
           const uint32_t sa = smem_addr(st), sb = sa + A_BYTES;
-          const uint32_t ssfa = sb + C::B_BYTES, ssfb = ssfa + SFA_BYTES;
-          const uint32_t sf = tmem + kSfCol + (it & 1u) * kSfBufCols;
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            tc_copy_sf(sf + 4 * ks, sdesc_sf_atom(ssfa + ks * kAtomBytes));
-            tc_copy_sf(sf + 16 + 8 * ks, sdesc_sf_atom(ssfb + ks * kAtomBytes));
-            tc_copy_sf(sf + 16 + 8 * ks + 4, sdesc_sf_atom(ssfb + 4 * kAtomBytes + ks * kAtomBytes));
-          }
           const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sb);
+          if constexpr (kBf16) {
+            // four K = 16 steps of BF16 per 128-byte row, no scale factors
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            tc_mma_nvf4(acc, da + 2 * ks, db + 2 * ks, C::kIdesc, sf + 4 * ks, sf + 16 + 8 * ks,
-                        (kt | ks) != 0 ? 1u : 0u);
+            for (int ks = 0; ks < 4; ++ks)
+              tc_mma_bf16(acc, da + 2 * ks, db + 2 * ks, C::kIdesc, (kt | ks) != 0 ? 1u : 0u);
+          } else {
+            const uint32_t ssfa = sb + C::B_BYTES, ssfb = ssfa + SFA_BYTES;
+            const uint32_t sf = tmem + kSfCol + (it & 1u) * kSfBufCols;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              tc_copy_sf(sf + 4 * ks, sdesc_sf_atom(ssfa + ks * kAtomBytes));
+              tc_copy_sf(sf + 16 + 8 * ks, sdesc_sf_atom(ssfb + ks * kAtomBytes));
+              tc_copy_sf(sf + 16 + 8 * ks + 4, sdesc_sf_atom(ssfb + 4 * kAtomBytes + ks * kAtomBytes));
+            }
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              tc_mma_nvf4(acc, da + 2 * ks, db + 2 * ks, C::kIdesc, sf + 4 * ks, sf + 16 + 8 * ks,
+                          (kt | ks) != 0 ? 1u : 0u);
+            }
           }
           tc_commit(&empty[s]);
         }
@@ -796,7 +838,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <Epi E, uint32_t kOpts>
 cudaError_t launch_impl(const NsParams* p, const GemmPlainArgs* g, int64_t units, cudaStream_t st,
                         int num_sms) {
-  using C = Cfg<E>;
+  using C = Cfg<E, (kOpts & kOptBf16) != 0>;
   static unsigned long long attr_set = 0ull;   // one bit per device; a benign race
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -834,17 +876,18 @@ cudaError_t launch_ns_opts(Epi epi, const NsParams& p, cudaStream_t st, int num_
   const int64_t units = p.prefix[p.count];
   cudaError_t e;
   switch (epi) {
+    // (the BF16 step has no tensor scales, hence no bounds kernels)
     case Epi::GramX:
       if ((e = launch_impl<Epi::GramX, kOpts>(&p, nullptr, units, st, num_sms)) != cudaSuccess) return e;
-      ns_bounds_kernel<Epi::GramX><<<p.count, 256, 0, st>>>(p);
+      if (!(kOpts & kOptBf16)) ns_bounds_kernel<Epi::GramX><<<p.count, 256, 0, st>>>(p);
       break;
     case Epi::GramA:
       if ((e = launch_impl<Epi::GramA, kOpts>(&p, nullptr, units, st, num_sms)) != cudaSuccess) return e;
-      ns_bounds_kernel<Epi::GramA><<<p.count, 256, 0, st>>>(p);
+      if (!(kOpts & kOptBf16)) ns_bounds_kernel<Epi::GramA><<<p.count, 256, 0, st>>>(p);
       break;
     case Epi::Update:
       if ((e = launch_impl<Epi::Update, kOpts>(&p, nullptr, units, st, num_sms)) != cudaSuccess) return e;
-      if (!p.last) ns_bounds_kernel<Epi::Update><<<p.count, 256, 0, st>>>(p);
+      if (!p.last && !(kOpts & kOptBf16)) ns_bounds_kernel<Epi::Update><<<p.count, 256, 0, st>>>(p);
       break;
     default: return cudaErrorInvalidValue;
   }
@@ -854,6 +897,7 @@ cudaError_t launch_ns_opts(Epi epi, const NsParams& p, cudaStream_t st, int num_
 }  // namespace
 
 cudaError_t launch_gemm_ns(Epi epi, const NsParams& p, cudaStream_t st, int num_sms) {
+  if (p.opts & kOptBf16) return launch_ns_opts<kOptBf16>(epi, p, st, num_sms);
   switch (p.opts & (kOptRht | kOpt46)) {
     case 0: return launch_ns_opts<0>(epi, p, st, num_sms);
     case kOpt46: return launch_ns_opts<kOpt46>(epi, p, st, num_sms);

@@ -328,15 +328,7 @@ __global__ void __launch_bounds__(kEwThreads) dequantize_kernel(
     for (int k = 0; k < kDqUnroll; ++k) {
       if (gi[k] >= R) break;
       const float s = e4m3_to_f32(sb[k]);
-      uint32_t hv[2];
-      // volatile: without it this decode of a 16-bit load came out wrong on sm_100a
-      // (nearly every output zero), while the same code with byte loads was exact.
-      asm volatile("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-                   "mov.b32 {b0, b1, b2, b3}, %2;\n\t"
-                   "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-                   "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t}"
-                   : "=r"(hv[0]), "=r"(hv[1])
-                   : "r"(w[k]));
+      const uint32_t hv[2] = {e2m1x2_to_f16x2(w[k] & 0xFFu), e2m1x2_to_f16x2((w[k] >> 8) & 0xFFu)};
       const float4 o = make_float4(__fmul_rn(__fmul_rn(half_lo(hv[0]), s), s_g),
                                    __fmul_rn(__fmul_rn(half_hi(hv[0]), s), s_g),
                                    __fmul_rn(__fmul_rn(half_lo(hv[1]), s), s_g),
@@ -769,7 +761,7 @@ __global__ void __launch_bounds__(kEwThreads, 4) ns_preamble_kernel(const __grid
     prefetch(u + gridDim.x);
     const int mi = owner_of(p.prefix, p.count, u);
     const MatDesc& d = p.mat[mi];
-    const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off);
+    const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off, (kOpts & kOptBf16) != 0);
     const int32_t tiles_n = d.np / kT;
     const int32_t lu = u - p.prefix[mi];
     const int32_t ti = lu / tiles_n;                       // 32-bit: units < 2^31
@@ -867,6 +859,20 @@ __global__ void __launch_bounds__(kEwThreads, 4) ns_preamble_kernel(const __grid
       } else {
 #pragma unroll
         for (int e = 0; e < 16; ++e) v[e] = tile[pre_off(blk * 16 + e, line)];
+      }
+      if constexpr ((kOpts & kOptBf16) != 0) {
+        // the BF16 comparison step: both views are BF16 copies (round to nearest even) of
+        // X0 (view 0) and of X0^T (view 1), two 16-byte chunks per block
+        const int64_t R = (view == 0 ? i0 : j0) + line;
+        const int64_t K0 = (view == 0 ? j0 : i0) + blk * 16;
+        const int64_t Cp = view == 0 ? d.np : d.mp;
+        uint8_t* dst = p.ws + (view == 0 ? L.qX[0] : L.qXT[0]);
+        uint32_t w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+        *reinterpret_cast<uint4*>(dst + tiled_chunk_offset_bf16(R, K0, Cp)) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(dst + tiled_chunk_offset_bf16(R, K0 + 8, Cp)) = make_uint4(w[4], w[5], w[6], w[7]);
+        continue;
       }
       // view 0 is the Gram operand of iteration 0, view 1 the update operand
       if constexpr ((kOpts & kOptRht) != 0) rht16(v, view == 0 ? p.rht[0] : p.rht[2]);
@@ -1033,6 +1039,11 @@ void preamble_launch(const NsParams& p, cudaStream_t st, int num_sms) {
 }
 
 cudaError_t launch_ns_preamble(const NsParams& p, cudaStream_t st, int num_sms) {
+  if (p.opts & kOptBf16) {
+    // BF16 views carry no tensor scale: no bounds kernel follows
+    preamble_launch<kOptBf16>(p, st, num_sms);
+    return cudaGetLastError();
+  }
   switch (p.opts & (kOptRht | kOpt46 | kOptNvSrc)) {
     case 0: preamble_launch<0>(p, st, num_sms); break;
     case kOpt46: preamble_launch<kOpt46>(p, st, num_sms); break;

@@ -133,6 +133,41 @@ def ns_iterations_nvfp4(X0, K, a, b, c, mode="pow2", trace=None, rht_masks=None,
     return X
 
 
+def bf16_round(x) -> np.ndarray:
+    """FP32 -> BF16 by round-to-nearest, ties to even, returned as the FP32 numbers
+    those BF16 values are.  BF16 keeps the sign, the 8 exponent bits and the top 7
+    mantissa bits of an FP32 number: the lower 16 bits are rounded away.  Finite
+    inputs only."""
+    x = np.asarray(x, dtype=np.float32)
+    bits = x.view(np.uint32).astype(np.uint64)
+    keep = bits >> 16
+    rest = bits & 0xFFFF
+    up = (rest > 0x8000) | ((rest == 0x8000) & ((keep & 1) == 1))
+    return ((keep + up.astype(np.uint64)) << 16).astype(np.uint32).view(np.float32)
+
+
+def ns_iterations_bf16(X0, K, a, b, c, trace=None):
+    """K Newton-Schulz iterations with BF16 operands (the optimized BF16 baseline the
+    pages compare Q-Root against, Section 4.4 and Table 6), from the FP32 m x n X0
+    (m <= n).  Same plan as the NVFP4 route with bf16() in place of each
+    quantisation: Xb = bf16(X), A = Xb Xb^T, B = b A + c bf16(A) bf16(A)^T,
+    X_{k+1} = a X + bf16(B) Xb.  Products in float64 on the BF16 values, rounded once
+    to FP32; A made exactly symmetric from its upper triangle; X, A, B FP32."""
+    X = np.asarray(X0, dtype=np.float32)
+    for _ in range(K):
+        Xb = bf16_round(X).astype(np.float64)
+        A = symmetric_from_upper(Xb @ Xb.T).astype(np.float32)
+        Ab = bf16_round(A).astype(np.float64)
+        P = Ab @ Ab.T
+        B = (b * A.astype(np.float64) + c * P).astype(np.float32)
+        Bb = bf16_round(B).astype(np.float64)
+        Xn = (a * X.astype(np.float64) + Bb @ Xb).astype(np.float32)
+        if trace is not None:
+            trace.append(dict(X=X, A=A, P=P, B=B, X_next=Xn))
+        X = Xn
+    return X
+
+
 def ns_iterations_f64(X0, K, a, b, c):
     """K Newton-Schulz iterations in float64, no quantisation (Section 2)."""
     X = np.asarray(X0, dtype=np.float64)
@@ -144,10 +179,11 @@ def ns_iterations_f64(X0, K, a, b, c):
 
 def root_ns(G, K=5, a=3.4445, b=-4.7750, c=2.0315, clip_k=3.0, eps=NS_EPS,
             quantized=True, mode="pow2", trace=None, rht_masks=None, adaptive46=False,
-            clip_quantile=None):
+            clip_quantile=None, bf16=False):
     """Normalise, clip and run K Newton-Schulz iterations on the FP32 matrix G.
 
-    quantized=True: the NVFP4 route of Section 3.4 (FP32 result).
+    quantized=True: the NVFP4 route of Section 3.4 (FP32 result); with bf16=True
+    the same plan with BF16 operands (ns_iterations_bf16) instead.
     quantized=False: the plain float64 iteration of Section 2 (float64 result;
     normalisation and clip done in float64).
     """
@@ -163,8 +199,11 @@ def root_ns(G, K=5, a=3.4445, b=-4.7750, c=2.0315, clip_k=3.0, eps=NS_EPS,
                                                 clip_quantile=clip_quantile)
         if trace is not None:
             trace.append(dict(X0=X0, inv=inv, tau=tau, norm=norm))
-        Y = ns_iterations_nvfp4(X0, K, a, b, c, mode=mode, trace=trace, rht_masks=rht_masks,
-                                adaptive46=adaptive46)
+        if bf16:
+            Y = ns_iterations_bf16(X0, K, a, b, c, trace=trace)
+        else:
+            Y = ns_iterations_nvfp4(X0, K, a, b, c, mode=mode, trace=trace, rht_masks=rht_masks,
+                                    adaptive46=adaptive46)
     else:
         X64 = np.asarray(X, dtype=np.float64)
         norm = float(np.sqrt(np.sum(X64 ** 2)))

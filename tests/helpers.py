@@ -67,3 +67,16 @@ def ws_f32(ws_np: np.ndarray, off: int, count: int) -> np.ndarray:
 
 def ws_bytes(ws_np: np.ndarray, off: int, count: int) -> np.ndarray:
     return ws_np[off:off + count]
+
+
+def tiled_bf16_to_plain(buf, rows: int, cols: int) -> np.ndarray:
+    """The TILED BF16 layout (tiles of 128 rows x 64 elements, 16-byte chunk j of row r
+    at position j ^ (r % 8)) of a rows x cols matrix -> its FP32 values, padding
+    included (shape Rp x Cp)."""
+    Rp, Cp = round_up(rows, 128), round_up(cols, 64)
+    t = np.asarray(buf, dtype=np.uint8).reshape(Rp // 128, Cp // 64, 128, 8, 16)
+    r, pos = _chunk_index()
+    t = t[:, :, r[:, None], pos, :]                    # logical chunk order
+    plain = np.ascontiguousarray(t.transpose(0, 2, 1, 3, 4)).reshape(Rp, Cp * 2)
+    u16 = plain.view(np.uint16)
+    return (u16.astype(np.uint32) << 16).view(np.float32)
