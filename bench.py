@@ -46,6 +46,9 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--per-matrix", action="store_true",
+                    help="--op quantize: one fs4_nvfp4_quantize call per matrix instead of one "
+                         "fs4_nvfp4_quantize_batched call per step")
     ap.add_argument("--no-bf16", action="store_true",
                     help="skip the BF16 comparison step (same plan, BF16 operands)")
     ap.add_argument("--op", default="ns", choices=["ns", "quantize", "dequantize", "momentum"],
@@ -733,8 +736,9 @@ def main():
 
 
 def run_standalone(args, w, rank, world, local, barrier, ranks_max):
-    """--op quantize / dequantize: one step = one fs4_nvfp4_quantize (or _dequantize)
-    call per matrix of the workload, row axis, outputs preallocated."""
+    """--op quantize / dequantize: one step = one fs4_nvfp4_quantize_batched call over every
+    matrix of the workload (--per-matrix: one fs4_nvfp4_quantize call per matrix), or one
+    fs4_nvfp4_dequantize call per matrix; row axis, outputs preallocated."""
     import torch
     import nvfp4_precision_optimizer_b200 as F
     from nvfp4_precision_optimizer_b200.workloads import BASE_SEED, matrices
@@ -768,7 +772,22 @@ def run_standalone(args, w, rank, world, local, barrier, ranks_max):
                                          G.shape[0], G.shape[1], y.data_ptr(), G.shape[1], flags,
                                          st.cuda_stream), "fs4_nvfp4_dequantize")
 
+    batched = args.op == "quantize" and not args.per_matrix
+    qarr = (F._lib.QuantDesc * len(Gs))()
+    for i, (G, b) in enumerate(zip(Gs, bufs)):
+        qarr[i] = F._lib.QuantDesc(G.data_ptr(), G.shape[0], G.shape[1], G.shape[1], 0, b["codes"].data_ptr(),
+                                   b["scales"].data_ptr(), b["sg"].data_ptr())
+    bws_bytes = int(lib.fs4_nvfp4_quantize_batched_workspace_size(len(Gs)))
+    bws = torch.zeros(max(bws_bytes, 256), dtype=torch.uint8, device="cuda")
+
+    def quantize_all(st):
+        F.check(lib.fs4_nvfp4_quantize_batched(len(Gs), qarr, flags, bws.data_ptr(), bws.numel(),
+                                               st.cuda_stream), "fs4_nvfp4_quantize_batched")
+
     def step():
+        if batched:
+            quantize_all(stream)
+            return
         for i in range(len(Gs)):
             if args.op == "quantize":
                 quantize(i, Gs[i], stream)
@@ -782,6 +801,7 @@ def run_standalone(args, w, rank, world, local, barrier, ranks_max):
     torch.cuda.synchronize()
     for b in bufs:
         F.check(F.device_status(b["ws"]), "device status after warm-up")
+    F.check(F.device_status(bws), "device status after warm-up")
 
     call_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(Gs) + 1)] for _ in range(args.steps)]
     for evs in call_ev:
@@ -794,6 +814,10 @@ def run_standalone(args, w, rank, world, local, barrier, ranks_max):
         time.sleep(0.3)
         for s in range(args.steps):
             call_ev[s][0].record(stream)
+            if batched:
+                quantize_all(stream)
+                call_ev[s][-1].record(stream)
+                continue
             for i in range(len(Gs)):
                 if args.op == "quantize":
                     quantize(i, Gs[i], stream)
@@ -801,6 +825,8 @@ def run_standalone(args, w, rank, world, local, barrier, ranks_max):
                     dequantize(i, bufs[i]["y"], stream)
                 call_ev[s][i + 1].record(stream)
         torch.cuda.synchronize()
+    if batched:
+        F.check(F.device_status(bws), "device status after the timed steps")
     barrier()
     total_ms = ranks_max(call_ev[0][0].elapsed_time(call_ev[-1][-1]))
     ms_step = total_ms / args.steps
@@ -809,15 +835,21 @@ def run_standalone(args, w, rank, world, local, barrier, ranks_max):
 
     # roofline of one call (the amax and quantise launches of fs4_nvfp4_quantize, or
     # the one dequantise launch), averaged over every call of the timed steps
-    call_ms = [evs[i].elapsed_time(evs[i + 1]) for evs in call_ev for i in range(len(Gs))]
-    call_bytes = elems * QD_BYTES / len(Gs)
+    if batched:
+        call_ms = [evs[0].elapsed_time(evs[-1]) for evs in call_ev]
+        call_bytes = elems * QD_BYTES
+    else:
+        call_ms = [evs[i].elapsed_time(evs[i + 1]) for evs in call_ev for i in range(len(Gs))]
+        call_bytes = elems * QD_BYTES / len(Gs)
     mean_call = statistics.mean(call_ms)
     peaks, peak_src = measured_peaks()
     achieved = call_bytes / (mean_call * 1e-3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-            "kernel": ("fs4_nvfp4_quantize call (quantize_fused_kernel: amax pass, grid barrier, quantise pass)" if args.op == "quantize"
-                       else "fs4_nvfp4_dequantize call (dequantize_kernel)"),
+            "kernel": ("fs4_nvfp4_quantize_batched call (quantize_batched_kernel: amax pass, grid "
+                       "barrier, quantise pass over every matrix)" if batched
+                       else "fs4_nvfp4_quantize call (quantize_fused_kernel: amax pass, grid barrier, quantise pass)"
+                       if args.op == "quantize" else "fs4_nvfp4_dequantize call (dequantize_kernel)"),
             "ms_per_launch": mean_call, "peak_source": f"hbm_gbs ({peak_src} MEASURED_PEAKS.json)"}
 
     # end to end with host buffers: per matrix, copy in, call, copy out, pipelined over a
@@ -912,7 +944,7 @@ def run_standalone(args, w, rank, world, local, barrier, ranks_max):
                               if elems * 4 > torch.cuda.get_device_properties(local).L2_cache_size
                               else "inputs of %.1f MB fit in L2 (not flushed)" % (elems * 4 / 1e6))},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps * len(Gs),   # one kernel per call (quantize: the fused kernel)
+            "gpu_launches": args.steps * (1 if batched else len(Gs)),   # one kernel per call
             "clocks": sampler.summary(),
         }
         print(json.dumps(line), flush=True)

@@ -163,7 +163,36 @@ fs4_status fs4_nvfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_
                               uint32_t flags, void* workspace, size_t workspace_bytes,
                               void* stream);
 
-/* Dequantise a row-blocked NVFP4 matrix (rows x cols, as written by
+/* One matrix of a batched quantise: x (device, rows x cols, leading dimension ld),
+ * axis (FS4_AXIS_ROW or FS4_AXIS_COL) and its outputs codes, scales, s_g, each as
+ * for fs4_nvfp4_quantize. */
+typedef struct {
+  const float* x;
+  int64_t rows, cols, ld;
+  int32_t axis;
+  uint8_t* codes;
+  uint8_t* scales;
+  float* s_g;
+} fs4_quant_desc;
+
+/* Bytes of workspace fs4_nvfp4_quantize_batched needs for `count` matrices (0 if
+ * count is outside [1, FS4_MAX_BATCH]). */
+size_t fs4_nvfp4_quantize_batched_workspace_size(int32_t count);
+
+/* fs4_nvfp4_quantize on `count` matrices (descs: HOST array) in one launch: each matrix
+ * gets its own tensor scale from its own amax and is quantised exactly as by
+ * fs4_nvfp4_quantize with the same axis and flags (Section 2 "NVFP4 format").  One
+ * cooperative launch covers every matrix: an amax pass, a grid-wide barrier (bounded:
+ * FS4_ERR_TIMEOUT in the status word if it runs out), then the quantise pass over the
+ * tiles of all matrices.  flags: FS4_SG_AMAX, FS4_LAYOUT_TILED (for all matrices),
+ * FS4_TEST_STALL.  Errors as fs4_nvfp4_quantize for each descriptor, plus
+ * FS4_ERR_SHAPE for count outside [1, FS4_MAX_BATCH]; a non-finite input anywhere is
+ * recorded as FS4_ERR_NONFINITE in the status word.  Outputs of different matrices
+ * must not overlap; calls whose work overlaps on the GPU need separate workspaces. */
+fs4_status fs4_nvfp4_quantize_batched(int32_t count, const fs4_quant_desc* descs, uint32_t flags,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Dequantise a row-blocked NVFP4 matrix (rows x cols, as written by/* Dequantise a row-blocked NVFP4 matrix (rows x cols, as written by
  * fs4_nvfp4_quantize in the layout given by flags) into FP32 y (leading
  * dimension ld): y = fp32(fp32(code * s) * s_g).
  * Source: Section 2 "NVFP4 format": an element's value is its E2M1 value times

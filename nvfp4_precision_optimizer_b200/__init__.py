@@ -19,7 +19,7 @@ from ._lib import (FS4_AXIS_COL, FS4_AXIS_ROW, FS4_LAYOUT_TILED, FS4_NS_ADAPTIVE
 MUON_COEFFS = (3.4445, -4.7750, 2.0315)
 
 __all__ = [
-    "quantize", "dequantize", "gemm", "root_ns", "root_ns_batched", "ns_workspace_size",
+    "quantize", "quantize_batched", "dequantize", "gemm", "root_ns", "root_ns_batched", "ns_workspace_size",
     "ns_batched_workspace_size", "ns_layout", "device_status", "tiled_shape", "Fs4Error",
     "momentum_nvfp4", "root_ns_batched_nvfp4", "root_ns_bf16_batched", "ns_bf16_batched_workspace_size",
     "ns_bf16_layout",
@@ -78,6 +78,39 @@ def quantize(x: torch.Tensor, axis: int = FS4_AXIS_ROW, tiled: bool = False,
                                         workspace.data_ptr(), workspace.numel(), _stream(stream)),
           "fs4_nvfp4_quantize")
     return codes, scales, s_g
+
+
+def quantize_batched(xs: Sequence[torch.Tensor], axis: int = FS4_AXIS_ROW, tiled: bool = False,
+                     sg_mode: str = "pow2", workspace: torch.Tensor | None = None, stream=None,
+                     flags: int = 0):
+    """fs4_nvfp4_quantize on every matrix of xs in one launch
+    (fs4_nvfp4_quantize_batched).  Returns a list of (codes, scales, s_g)."""
+    outs = []
+    arr = (_lib.QuantDesc * len(xs))()
+    for i, x in enumerate(xs):
+        _check_f32_matrix(x, "x")
+        rows, cols = x.shape
+        R, C = (rows, cols) if axis == FS4_AXIS_ROW else (cols, rows)
+        if tiled:
+            ncode, nscale = tiled_shape(R, C)
+            codes = torch.empty(ncode, dtype=torch.uint8, device=x.device)
+            scales = torch.empty(nscale, dtype=torch.uint8, device=x.device)
+        else:
+            codes = torch.empty((R, C // 2), dtype=torch.uint8, device=x.device)
+            scales = torch.empty((R, max(C // 16, 1)), dtype=torch.uint8, device=x.device)
+        s_g = torch.empty(1, dtype=torch.float32, device=x.device)
+        ld = x.stride(0) if rows > 1 else cols
+        arr[i] = _lib.QuantDesc(x.data_ptr(), rows, cols, ld, axis, codes.data_ptr(), scales.data_ptr(),
+                                s_g.data_ptr())
+        outs.append((codes, scales, s_g))
+    need = int(_lib.lib().fs4_nvfp4_quantize_batched_workspace_size(len(xs)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=xs[0].device)
+    flags |= (FS4_LAYOUT_TILED if tiled else 0) | (FS4_SG_AMAX if sg_mode == "amax" else 0)
+    check(_lib.lib().fs4_nvfp4_quantize_batched(len(xs), arr, flags, workspace.data_ptr(),
+                                                workspace.numel(), _stream(stream)),
+          "fs4_nvfp4_quantize_batched")
+    return outs
 
 
 def dequantize(codes: torch.Tensor, scales: torch.Tensor, s_g: torch.Tensor, rows: int, cols: int,

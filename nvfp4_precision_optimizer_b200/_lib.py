@@ -42,6 +42,11 @@ class Nvfp4State(ctypes.Structure):
     _fields_ = [("codes", c_vp), ("scales", c_vp), ("s_g", c_vp), ("mask", c_u32)]
 
 
+class QuantDesc(ctypes.Structure):
+    _fields_ = [("x", c_vp), ("rows", c_i64), ("cols", c_i64), ("ld", c_i64), ("axis", c_i32),
+                ("codes", c_vp), ("scales", c_vp), ("s_g", c_vp)]
+
+
 class NsLayout(ctypes.Structure):
     _fields_ = [("mp", c_i64), ("np", c_i64), ("X", c_i64), ("A", c_i64),
                 ("qX_codes", c_i64 * 2), ("qX_scales", c_i64 * 2),
@@ -59,6 +64,8 @@ SIGNATURES = {
                                    c_sz, c_vp]),
     "fs4_nvfp4_quantize": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_i32, c_vp, c_vp, c_vp, c_u32,
                                    c_vp, c_sz, c_vp]),
+    "fs4_nvfp4_quantize_batched_workspace_size": (c_sz, [c_i32]),
+    "fs4_nvfp4_quantize_batched": (c_i32, [c_i32, ctypes.POINTER(QuantDesc), c_u32, c_vp, c_sz, c_vp]),
     "fs4_nvfp4_dequantize": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_i64, c_u32, c_vp]),
     "fs4_nvfp4_gemm": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_vp,
                                c_i64, c_vp, c_sz, c_vp]),

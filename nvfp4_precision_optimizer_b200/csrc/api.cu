@@ -279,6 +279,38 @@ fs4_status fs4_nvfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_
                                      static_cast<cudaStream_t>(stream), di.num_sms));
 }
 
+size_t fs4_nvfp4_quantize_batched_workspace_size(int32_t count) {
+  if (count < 1 || count > kMaxBatch) return 0;
+  return quantize_batched_workspace_bytes(count);
+}
+
+fs4_status fs4_nvfp4_quantize_batched(int32_t count, const fs4_quant_desc* descs, uint32_t flags,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+  if (!descs) return FS4_ERR_INVALID_ARG;
+  if (count < 1 || count > kMaxBatch) return FS4_ERR_SHAPE;
+  if (flags & ~(uint32_t)(FS4_SG_AMAX | FS4_LAYOUT_TILED | FS4_TEST_STALL)) return FS4_ERR_INVALID_ARG;
+  static thread_local QuantDesc qd[kMaxBatch];
+  for (int i = 0; i < count; ++i) {
+    const fs4_quant_desc& d = descs[i];
+    if (!d.x || !d.codes || !d.scales || !d.s_g) return FS4_ERR_INVALID_ARG;
+    if (d.axis != FS4_AXIS_ROW && d.axis != FS4_AXIS_COL) return FS4_ERR_INVALID_ARG;
+    if (d.rows < 1 || d.cols < 1 || d.rows > (1ll << 31) || d.cols > (1ll << 31)) return FS4_ERR_SHAPE;
+    if ((d.axis == FS4_AXIS_ROW ? d.cols : d.rows) % 16) return FS4_ERR_SHAPE;
+    if (d.ld < d.cols) return FS4_ERR_INVALID_ARG;
+    if (!aligned(d.codes, 16) || !aligned(d.scales, 16) || !aligned(d.s_g, 4) || !aligned(d.x, 4))
+      return FS4_ERR_INVALID_ARG;
+    qd[i].x = d.x; qd[i].rows = d.rows; qd[i].cols = d.cols; qd[i].ld = d.ld; qd[i].axis = d.axis;
+    qd[i].codes = d.codes; qd[i].scales = d.scales; qd[i].s_g = d.s_g;
+  }
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < quantize_batched_workspace_bytes(count))
+    return FS4_ERR_WORKSPACE;
+  DeviceInfo di;
+  const fs4_status ds = device_info(&di);
+  if (ds != FS4_OK) return ds;
+  return cuda_status(launch_quantize_batched(count, qd, flags, static_cast<uint8_t*>(workspace),
+                                             static_cast<cudaStream_t>(stream), di.num_sms));
+}
+
 fs4_status fs4_nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* s_g,
                                 int64_t rows, int64_t cols, float* y, int64_t ld, uint32_t flags,
                                 void* stream) {

@@ -149,7 +149,20 @@ struct GemmPlainArgs {
 
 enum class Epi : int { Plain = 0, GramX = 1, GramA = 2, Update = 3 };
 
+// One matrix of a batched standalone quantise (host side; mirrors fs4_quant_desc).
+struct QuantDesc {
+  const float* x;
+  int64_t rows, cols, ld;
+  int32_t axis;
+  uint8_t* codes;
+  uint8_t* scales;
+  float* s_g;
+};
+
 // ---------------------------------------------------------------- launchers (kernels.cu / gemm.cu)
+size_t quantize_batched_workspace_bytes(int32_t count);
+cudaError_t launch_quantize_batched(int32_t count, const QuantDesc* descs, uint32_t flags, uint8_t* ws,
+                                    cudaStream_t st, int num_sms);
 cudaError_t launch_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld, int axis,
                             uint8_t* codes, uint8_t* scales, float* s_g, uint32_t flags,
                             uint8_t* ws, cudaStream_t st, int num_sms);

@@ -82,9 +82,16 @@ struct Cfg {
   static constexpr int SMEM_BYTES =
       1024 + kStages * STAGE_BYTES + 8 * EPI_FLOATS * 4 + BAR_BYTES + 128 * 8;
   static constexpr uint32_t kIdesc = kBf16 ? idesc_bf16(BM, BN) : idesc_mxf4nvf4(BM, BN);
+  // A separate warp copies the scale factors to TMEM (a ring of kSfBufs buffers) for the
+  // products whose time is set by the mainloop: issued by the MMA thread itself, each
+  // stage's copies queue behind its MMAs.  The update, whose time is set by its
+  // epilogue, measured slower with the extra warp and keeps the copies in the MMA thread.
+  static constexpr bool kSfWarp = !kBf16 && E != Epi::Update;
+  static constexpr int kSfBufs = kSfWarp ? 4 : 2;
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(SMEM_BYTES <= 232448, "over the per-CTA shared-memory limit");
-  static_assert((2 * kStages + 4) * 8 + 12 <= BAR_BYTES, "barrier block too small");
+  static_assert((2 * kStages + 4 + 2 * 4 + 1) * 8 + 12 <= BAR_BYTES, "barrier block too small");
+  static_assert(kSfCol + kSfBufs * kSfBufCols <= kTmemCols, "scale-factor ring over the TMEM columns");
 };
 
 struct Job {
@@ -696,7 +703,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_empty = acc_full + 1;         // the epilogue warps drained the accumulator
   uint64_t* mma_done = acc_full + 2;
   uint64_t* stall_bar = acc_full + 3;        // test only: never arrived on
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 4);
+  uint64_t* sf_full = acc_full + 4;           // [kSfBufs] scale copies into a TMEM buffer done
+  uint64_t* sf_empty = sf_full + C::kSfBufs;  // [kSfBufs] the MMAs reading that buffer done
+  uint64_t* sf_done = sf_empty + C::kSfBufs;  // the copier's last copies completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   float* scale_tab = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + C::BAR_BYTES);
   if (threadIdx.x >= 128 && threadIdx.x < 256) scale_tab_fill(scale_tab, threadIdx.x - 128);
@@ -714,6 +724,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(acc_empty, 8);
     mbar_init(mma_done, 1);
     mbar_init(stall_bar, 1);
+    for (int b = 0; b < C::kSfBufs; ++b) {
+      mbar_init(&sf_full[b], 1);
+      mbar_init(&sf_empty[b], 1);
+    }
+    mbar_init(sf_done, 1);
     *abort_flag = (__ldcg(status) & kStatusTimeout) ? 1 : 0;
     fence_mbar_init();
   }
@@ -786,19 +801,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int ks = 0; ks < 4; ++ks)
               tc_mma_bf16(acc, da + 2 * ks, db + 2 * ks, C::kIdesc, (kt | ks) != 0 ? 1u : 0u);
           } else {
-            const uint32_t ssfa = sb + C::B_BYTES, ssfb = ssfa + SFA_BYTES;
-            const uint32_t sf = tmem + kSfCol + (it & 1u) * kSfBufCols;
+            const uint32_t sfb_i = it % C::kSfBufs;
+            const uint32_t sf = tmem + kSfCol + sfb_i * kSfBufCols;
+            if constexpr (C::kSfWarp) {
+              // the copier warp filled this buffer from the same stage
+              if (!mbar_wait(&sf_full[sfb_i], (it / C::kSfBufs) & 1u, status, abort_flag)) { ok = false; break; }
+              tc_fence_after();
+            } else {
+              const uint32_t ssfa = sb + C::B_BYTES, ssfb = ssfa + SFA_BYTES;
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              tc_copy_sf(sf + 4 * ks, sdesc_sf_atom(ssfa + ks * kAtomBytes));
-              tc_copy_sf(sf + 16 + 8 * ks, sdesc_sf_atom(ssfb + ks * kAtomBytes));
-              tc_copy_sf(sf + 16 + 8 * ks + 4, sdesc_sf_atom(ssfb + 4 * kAtomBytes + ks * kAtomBytes));
+              for (int ks = 0; ks < 4; ++ks) {
+                tc_copy_sf(sf + 4 * ks, sdesc_sf_atom(ssfa + ks * kAtomBytes));
+                tc_copy_sf(sf + 16 + 8 * ks, sdesc_sf_atom(ssfb + ks * kAtomBytes));
+                tc_copy_sf(sf + 16 + 8 * ks + 4, sdesc_sf_atom(ssfb + 4 * kAtomBytes + ks * kAtomBytes));
+              }
             }
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
               tc_mma_nvf4(acc, da + 2 * ks, db + 2 * ks, C::kIdesc, sf + 4 * ks, sf + 16 + 8 * ks,
                           (kt | ks) != 0 ? 1u : 0u);
             }
+            if constexpr (C::kSfWarp) tc_commit(&sf_empty[sfb_i]);
           }
           tc_commit(&empty[s]);
         }
@@ -808,6 +831,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(mma_done);
       volatile int never = 0;
       mbar_wait(mma_done, 0, status, &never);
+    }
+  } else if (warp == 2 && C::kSfWarp) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- scale-factor copier
+      // For each stage: once its operands have landed and the MMAs of the stage that last
+      // used the TMEM buffer have completed, copy the stage's scale atoms into the buffer.
+      // The MMAs that read the stage's shared memory wait for these copies (sf_full), and
+      // the producer refills the stage only after those MMAs (empty), so the copies never
+      // read a refilled stage.
+      uint32_t it = 0;
+      bool ok = true;
+      for (int32_t u = first; u < total && ok && !*abort_flag; u += step) {
+        const Job j = make_job<E, kBf16>(u, p, g);
+        for (int kt = 0; kt < j.kt; ++kt, ++it) {
+          const uint32_t s = it % kStages, use = it / kStages;
+          const uint32_t b = it % C::kSfBufs;
+          if (!mbar_wait(&full[s], use & 1u, status, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&sf_empty[b], ((it / C::kSfBufs) & 1u) ^ 1u, status, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t ssfa = smem_addr(stage_base + s * C::STAGE_BYTES) + A_BYTES + C::B_BYTES;
+          const uint32_t ssfb = ssfa + SFA_BYTES;
+          const uint32_t sf = tmem + kSfCol + b * kSfBufCols;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            tc_copy_sf(sf + 4 * ks, sdesc_sf_atom(ssfa + ks * kAtomBytes));
+            tc_copy_sf(sf + 16 + 8 * ks, sdesc_sf_atom(ssfb + ks * kAtomBytes));
+            tc_copy_sf(sf + 16 + 8 * ks + 4, sdesc_sf_atom(ssfb + 4 * kAtomBytes + ks * kAtomBytes));
+          }
+          tc_commit(&sf_full[b]);
+        }
+      }
+      // every copy this thread issued completes before the TMEM is freed
+      tc_commit(sf_done);
+      volatile int never = 0;
+      mbar_wait(sf_done, 0, status, &never);
     }
   }
   } else {

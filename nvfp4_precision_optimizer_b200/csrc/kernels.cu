@@ -273,6 +273,32 @@ struct QuantArgs {
   uint32_t* hdr;                      // [0] status, [1] amax bits, [2] barrier count (zeroed)
 };
 
+// One matrix of a batched quantise (kernel parameter).
+struct QMat {
+  const float* x;
+  int64_t rows, cols, ld;             // x as given
+  int64_t R, C, Cp, xtiles_c;         // the quantised matrix Y (x or x^T), its padded width,
+                                      // tiles per line of x
+  int32_t col_axis, vec;              // 16x1 blocks; float4 loads possible
+  uint8_t* codes;
+  uint8_t* scales;
+  float* s_g;
+};
+// Workspace words of a batched quantise: [0] status, [kQBatchCountWord] barrier count,
+// [kQBatchAmaxWord + i] amax of matrix i (float bits); all zeroed by the launcher.
+constexpr int kQBatchCountWord = 2;
+constexpr int kQBatchAmaxWord = 64;
+
+struct QBatchArgs {
+  int32_t count;
+  int32_t tiled, sg_amax_mode, stall;
+  uint32_t* hdr;
+  int32_t pre_amax[kMaxBatch + 1];    // prefix sums of the 16-row amax units
+  int32_t pre_tiles[kMaxBatch + 1];   // prefix sums of the 64 x 64 tiles
+  QMat mat[kMaxBatch];
+};
+static_assert(sizeof(QBatchArgs) <= 32000, "kernel parameter block too large");
+
 // Standalone quantise in one cooperative launch: the amax pass over x, a grid-wide
 // barrier, then the quantise pass.  The barrier takes the place of a second launch and
 // its ramp, and the quantise pass (last tile first) finds the tail of x in L2.
@@ -281,6 +307,103 @@ __global__ void __launch_bounds__(kEwThreads) quantize_fused_kernel(const __grid
   if (!grid_barrier(&a.hdr[2], gridDim.x + (a.stall ? 1u : 0u), &a.hdr[0])) return;
   quantize_pass(a.x, a.ld, a.R, a.C, a.col_axis, a.tiled, a.sg_amax_mode, a.Rext, a.Cext, a.Cp,
                 a.ntiles, a.codes, a.scales, a.s_g, a.hdr);
+}
+
+// ------------------------------------------------------------------ batched quantise
+// Many matrices in one cooperative launch: the amax pass over units of 16 rows (one
+// atomic per unit on the matrix's amax), a grid-wide barrier, then the quantise pass
+// over the 64 x 64 tiles of every matrix, each staged through shared memory as in the
+// single-matrix quantise.  Work units of all matrices are numbered consecutively
+// (prefix sums), so one launch keeps every SM busy whatever the mix of sizes.
+__global__ void __launch_bounds__(kEwThreads) quantize_batched_kernel(const __grid_constant__ QBatchArgs a) {
+  __shared__ float red[kEwThreads / 32];
+  __shared__ float tile[kT][kT + 1];
+  uint32_t* status = a.hdr;
+  uint32_t* amaxv = a.hdr + kQBatchAmaxWord;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  // ---- pass 1: per-matrix max |x| and the non-finite flag
+  bool bad = false;
+  for (int32_t u = blockIdx.x; u < a.pre_amax[a.count]; u += gridDim.x) {
+    const int mi = owner_of(a.pre_amax, a.count, u);
+    const QMat& m = a.mat[mi];
+    const int64_t r0 = (int64_t)(u - a.pre_amax[mi]) * 16;
+    float mx = 0.0f;
+    for (int64_t r = r0 + warp; r < r0 + 16 && r < m.rows; r += kEwThreads / 32) {
+      const float* row = m.x + r * m.ld;
+      if (m.vec) {
+        const float4* row4 = reinterpret_cast<const float4*>(row);
+        for (int64_t c = lane; c < (m.cols >> 2); c += 32) {
+          const float4 v = __ldg(row4 + c);
+          bad |= !(is_finite_bits(v.x) && is_finite_bits(v.y) && is_finite_bits(v.z) &&
+                   is_finite_bits(v.w));
+          mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        }
+      } else {
+        for (int64_t c = lane; c < m.cols; c += 32) {
+          const float v = __ldg(row + c);
+          bad |= !is_finite_bits(v);
+          mx = fmaxf(mx, fabsf(v));
+        }
+      }
+    }
+    mx = block_max(mx, red);
+    if (t == 0 && mx > 0.0f) atomicMax(&amaxv[mi], __float_as_uint(mx));
+  }
+  if (__syncthreads_or(bad) && t == 0) atomicOr(&status[0], kStatusNonFinite);
+  if (!grid_barrier(&a.hdr[kQBatchCountWord], gridDim.x + (a.stall ? 1u : 0u), &status[0])) return;
+  // ---- pass 2: the tiles of every matrix
+  for (int32_t u = blockIdx.x; u < a.pre_tiles[a.count]; u += gridDim.x) {
+    const int mi = owner_of(a.pre_tiles, a.count, u);
+    const QMat& m = a.mat[mi];
+    const int64_t lu = u - a.pre_tiles[mi];
+    const float amax = __uint_as_float(__ldcg(&amaxv[mi]));
+    const float s_g = a.sg_amax_mode ? (amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f)
+                                     : pow2_tensor_scale(amax);
+    if (lu == 0 && t == 0) *m.s_g = s_g;
+    const float six_sg = __fmul_rn(6.0f, s_g);
+    const float rcp_six = __frcp_rn(six_sg);
+    // tile origin in x; Y = x (row axis) or x^T (column axis) is quantised along its rows
+    const int64_t xr0 = (lu / m.xtiles_c) * kT, xc0 = (lu % m.xtiles_c) * kT;
+    const int64_t xrows = m.col_axis ? m.C : m.R, xcols = m.col_axis ? m.R : m.C;
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+      const int f = t + kEwThreads * pass;
+      const int line = f >> 4, c4 = (f & 15) * 4;
+      float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      if (xr0 + line < xrows) {
+        const float* src = m.x + (xr0 + line) * m.ld + xc0 + c4;
+        if (m.vec && xc0 + c4 + 4 <= xcols) {
+          const float4 q4 = __ldg(reinterpret_cast<const float4*>(src));
+          v[0] = q4.x; v[1] = q4.y; v[2] = q4.z; v[3] = q4.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (xc0 + c4 + e < xcols) v[e] = __ldg(src + e);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (!m.col_axis) tile[line][c4 + e] = v[e];
+        else tile[c4 + e][line] = v[e];
+      }
+    }
+    __syncthreads();
+    const int64_t i0 = m.col_axis ? xc0 : xr0, j0 = m.col_axis ? xr0 : xc0;
+    const int r = t >> 2, cb = (t & 3) * 16;
+    const int64_t i = i0 + r, j = j0 + cb;
+    float v[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] = tile[r][cb + e];
+    const QBlock16 q = a.sg_amax_mode ? quantize16<false>(v, s_g, six_sg, rcp_six)
+                                      : quantize16<true>(v, s_g, six_sg, rcp_six);
+    if (a.tiled) {
+      store_block_tiled(m.codes, m.scales, i, j, m.Cp, q);
+    } else if (i < m.R && j < m.C) {
+      *reinterpret_cast<uint2*>(m.codes + i * (m.C / 2) + j / 2) = make_uint2(q.w0, q.w1);
+      m.scales[i * (m.C / 16) + j / 16] = static_cast<uint8_t>(q.scale);
+    }
+    __syncthreads();   // the tile is restaged by the next unit
+  }
 }
 
 // y = fp32(fp32(code * scale) * s_g), one thread per group of 4 consecutive elements
@@ -985,6 +1108,47 @@ cudaError_t launch_quantize(const float* x, int64_t rows, int64_t cols, int64_t 
   const int grid = persistent_grid(quantize_fused_kernel, std::max<int64_t>(amax_units, a.ntiles), num_sms);
   void* args[] = {&a};
   return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(quantize_fused_kernel), dim3(grid),
+                                     dim3(kEwThreads), args, 0, st);
+}
+
+size_t quantize_batched_workspace_bytes(int32_t count) {
+  return (size_t)align_up(4 * (kQBatchAmaxWord + count), 256);
+}
+
+cudaError_t launch_quantize_batched(int32_t count, const QuantDesc* d, uint32_t flags, uint8_t* ws,
+                                    cudaStream_t st, int num_sms) {
+  static thread_local QBatchArgs a;   // 27 KB: too large for every caller's stack
+  a.count = count;
+  a.tiled = (flags & 2u) ? 1 : 0;
+  a.sg_amax_mode = (flags & 1u) ? 1 : 0;
+  a.stall = (flags & (1u << 30)) ? 1 : 0;   // FS4_TEST_STALL
+  a.hdr = reinterpret_cast<uint32_t*>(ws);
+  int64_t na = 0, nt = 0;
+  a.pre_amax[0] = a.pre_tiles[0] = 0;
+  for (int i = 0; i < count; ++i) {
+    QMat& m = a.mat[i];
+    m.x = d[i].x; m.rows = d[i].rows; m.cols = d[i].cols; m.ld = d[i].ld;
+    m.col_axis = d[i].axis;
+    m.R = m.col_axis ? m.cols : m.rows;
+    m.C = m.col_axis ? m.rows : m.cols;
+    const int64_t Rext = a.tiled ? align_up(m.R, 128) : align_up(m.R, kT);
+    m.Cp = align_up(m.C, 256);
+    const int64_t Cext = a.tiled ? m.Cp : align_up(m.C, kT);
+    m.xtiles_c = (m.col_axis ? Rext : Cext) / kT;
+    m.vec = ((reinterpret_cast<uintptr_t>(m.x) & 15) == 0 && (m.ld & 3) == 0 && (m.cols & 3) == 0) ? 1 : 0;
+    m.codes = d[i].codes; m.scales = d[i].scales; m.s_g = d[i].s_g;
+    na += (m.rows + 15) / 16;
+    nt += (Rext / kT) * (Cext / kT);
+    if (na > 0x7FFFFFFF || nt > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    a.pre_amax[i + 1] = (int32_t)na;
+    a.pre_tiles[i + 1] = (int32_t)nt;
+  }
+  cudaError_t e = cudaMemsetAsync(ws, 0, quantize_batched_workspace_bytes(count), st);
+  if (e != cudaSuccess) return e;
+  // as many CTAs as are resident at once (a cooperative launch refuses more)
+  const int grid = persistent_grid(quantize_batched_kernel, std::max<int64_t>(na, nt), num_sms);
+  void* args[] = {&a};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(quantize_batched_kernel), dim3(grid),
                                      dim3(kEwThreads), args, 0, st);
 }
 

@@ -218,3 +218,80 @@ def test_dequantize_large_grid_stride(fs4, shape):
     wc, ws, wg = Q.quantize_rows(x)
     want = Q.dequantize_rows(wc, ws, wg, dtype=np.float32)
     assert np.array_equal(y.view(np.uint32), want.view(np.uint32))
+
+
+# ---------------------------------------------------------------- batched quantise
+
+def _batch_inputs():
+    """Every case of CASES whose shape suits the axis, in one batch."""
+    return {name: x for name, x in CASES.items()}
+
+
+@pytest.mark.parametrize("axis", [0, 1])
+@pytest.mark.parametrize("tiled", [False, True])
+@pytest.mark.parametrize("sg_mode", ["pow2", "amax"])
+def test_quantize_batched_matches_single_calls_and_oracle(fs4, axis, tiled, sg_mode):
+    """fs4_nvfp4_quantize_batched over a batch of mixed shapes (every case above whose
+    blocked dimension is a multiple of 16), each matrix byte for byte equal to its
+    single-matrix fs4_nvfp4_quantize result and to the oracle's quantisation with its own
+    tensor scale."""
+    names = [n for n, x in _batch_inputs().items() if (x.shape[1] if axis == 0 else x.shape[0]) % 16 == 0]
+    xs = [torch.from_numpy(CASES[n]).cuda() for n in names]
+    outs = fs4.quantize_batched(xs, axis=axis, tiled=tiled, sg_mode=sg_mode)
+    torch.cuda.synchronize()
+    for n, x, (c, s, g) in zip(names, xs, outs):
+        c1, s1, g1 = fs4.quantize(x, axis=axis, tiled=tiled, sg_mode=sg_mode)
+        assert torch.equal(c, c1) and torch.equal(s, s1) and torch.equal(g, g1), n
+        if not tiled:
+            xn = CASES[n]
+            wc, ws_, wg = (Q.quantize_rows if axis == 0 else Q.quantize_cols)(xn, mode=sg_mode)
+            assert np.float32(g.item()) == wg, n
+            assert np.array_equal(c.cpu().numpy(), wc) and np.array_equal(s.cpu().numpy(), ws_), n
+
+
+def test_quantize_batched_strided_and_unaligned_views(fs4):
+    rng = np.random.default_rng(41)
+    big = torch.from_numpy((rng.standard_normal((300, 1200)) * 0.02).astype(np.float32)).cuda()
+    xs = [big[:100, 1:273], big[10:150, 4:516], big[:, 16:16 + 1024]]   # odd offsets and strides
+    outs = fs4.quantize_batched(xs, axis=0)
+    for x, (c, s, g) in zip(xs, outs):
+        wc, ws_, wg = Q.quantize_rows(x.cpu().numpy())
+        assert np.float32(g.item()) == wg
+        assert np.array_equal(c.cpu().numpy(), wc) and np.array_equal(s.cpu().numpy(), ws_)
+
+
+def test_quantize_batched_full_size_3b_block(fs4):
+    """One 3B-class block (the bench's --op quantize workload unit): seven 3072 x 3072,
+    8192 x 3072 and 3072 x 8192 matrices in one launch, every byte against the single
+    calls, and two matrices against the C++ oracle."""
+    from nvfp4_precision_optimizer_b200.workloads import BASE_SEED, WORKLOADS, matrices
+    from oracle import cpp_oracle as C
+    Gs = matrices(WORKLOADS["3b_1block_gauss"], device="cuda", seed=BASE_SEED)
+    outs = fs4.quantize_batched(Gs, axis=0)
+    torch.cuda.synchronize()
+    for i, (G, (c, s, g)) in enumerate(zip(Gs, outs)):
+        c1, s1, g1 = fs4.quantize(G, axis=0)
+        assert torch.equal(c, c1) and torch.equal(s, s1) and torch.equal(g, g1)
+        if i in (0, 4):
+            wc, ws_, wg = C.quantize_rows(G.cpu().numpy())
+            assert np.float32(g.item()) == wg
+            assert np.array_equal(c.cpu().numpy(), wc) and np.array_equal(s.cpu().numpy(), ws_)
+
+
+def test_quantize_batched_nonfinite_and_timeout_status(fs4):
+    x = torch.zeros((32, 64), device="cuda")
+    y = torch.ones((16, 32), device="cuda")
+    x[3, 5] = float("nan")
+    ws = torch.zeros(fs4._lib.lib().fs4_nvfp4_quantize_batched_workspace_size(2), dtype=torch.uint8,
+                     device="cuda")
+    fs4.quantize_batched([x, y], workspace=ws)
+    assert fs4.device_status(ws) == -7
+    import time
+    t0 = time.time()
+    fs4.quantize_batched([y, y], workspace=ws, flags=fs4.FS4_TEST_STALL)
+    torch.cuda.synchronize()
+    assert time.time() - t0 < 30.0
+    assert fs4.device_status(ws) == -8
+    (c, s, g), = fs4.quantize_batched([y])
+    wc, ws_, wg = Q.quantize_rows(y.cpu().numpy())
+    assert np.array_equal(c.cpu().numpy(), wc) and np.float32(g.item()) == wg
