@@ -46,6 +46,9 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--source", default="fp32", choices=["fp32", "nvfp4"],
+                    help="ns: the momenta as FP32 matrices, or as NVFP4 first-moment states "
+                         "(fs4_root_ns_batched_nvfp4; states written once by fs4_momentum_nvfp4)")
     ap.add_argument("--per-matrix", action="store_true",
                     help="--op quantize: one fs4_nvfp4_quantize call per matrix instead of one "
                          "fs4_nvfp4_quantize_batched call per step")
@@ -487,12 +490,37 @@ def main():
     if args.graph and qflags & F.FS4_NS_RHT:
         raise SystemExit("--graph: a captured call would replay the same H16^r signs every step")
 
+    states = sarr = None
+    if args.source == "nvfp4":
+        # the momenta as NVFP4 first-moment states (one fs4_momentum_nvfp4 step from an empty
+        # state each); the step then reads the states in place of FP32 G
+        states = [F.momentum_nvfp4(G, 0.9, None, mask=0x5A5A, seed=BASE_SEED + i, want_m=False)[1]
+                  for i, G in enumerate(Gs)]
+        sarr = (F._lib.Nvfp4State * len(Gs))()
+        for i, (G, st) in enumerate(zip(Gs, states)):
+            sarr[i] = F._lib.Nvfp4State(st[0].data_ptr(), st[1].data_ptr(), st[2].data_ptr(), 0x5A5A)
+            arr[i].G = None
+        torch.cuda.synchronize()
+        del Gs
+        Gs = [torch.empty((1, 1), device="cuda") for _ in sarr]   # shapes come from the descriptors
+        need = int(lib.fs4_root_ns_batched_workspace_size(len(sarr), arr))
+
     def call(events=None):
         masks = None
         if qflags & F.FS4_NS_RHT:        # fresh signs for every step (Section 3.4)
             masks = (ctypes.c_uint16 * (3 * K))(*[int(v) for v in mask_rng.integers(0, 1 << 16, 3 * K)])
         mptr = ctypes.cast(masks, ctypes.c_void_p) if masks is not None else None
         cur = torch.cuda.current_stream().cuda_stream   # the capture stream under --graph
+        if sarr is not None:
+            ev_arr = None if events is None else (F._lib.c_vp * n_ev)(*[e.cuda_event for e in events])
+            if ev_arr is None:
+                st = lib.fs4_root_ns_batched_nvfp4(len(sarr), arr, sarr, K, clip_arg, qflags, mptr,
+                                                   ws.data_ptr(), need, cur)
+            else:
+                st = lib.fs4_root_ns_batched_nvfp4_timed(len(sarr), arr, sarr, K, clip_arg, qflags, mptr,
+                                                         ws.data_ptr(), need, cur, ev_arr, n_ev)
+            F.check(st, "fs4_root_ns_batched_nvfp4")
+            return
         if events is None:
             st = lib.fs4_root_ns_batched_ex(len(Gs), arr, K, clip_arg, qflags, mptr, ws.data_ptr(),
                                             need, cur)
@@ -523,7 +551,8 @@ def main():
     # Inputs that fit in L2 would be read from L2 by the next step: then L2 is flushed
     # (a zero-fill of twice its size) before every step, and the step time is taken from
     # the events around each call, so that the fill stays outside the timed work.
-    in_bytes = sum(G.numel() for G in Gs) * 4
+    in_bytes = (sum(G.numel() for G in Gs) * 4 if states is None
+                else sum(st[0].numel() + st[1].numel() for st in states))
     l2_bytes = int(torch.cuda.get_device_properties(local).L2_cache_size)
     flush = torch.empty(2 * l2_bytes, dtype=torch.uint8, device="cuda") if in_bytes <= 2 * l2_bytes else None
     t_start = torch.cuda.Event(enable_timing=True)
@@ -620,7 +649,7 @@ def main():
     phase_ms = {k: statistics.mean(v) * (1 if k in ("reduce", "preamble") else K) for k, v in per_kind.items()}
 
     comparator = None
-    if not args.no_bf16 and args.quant == "plain" and args.clip == "rms":
+    if not args.no_bf16 and args.quant == "plain" and args.clip == "rms" and states is None:
         bms, bphase = bf16_comparator(F, Gs, w, max(2, min(args.steps, 5)), flush, l2_bytes)
         peaks_b, _ = measured_peaks()
         bf16_tflops = w.flops_algorithmic() / (bms * 1e-3) / 1e12
@@ -640,7 +669,7 @@ def main():
     # pipelined on three streams (copy-in, compute, copy-out) with double-buffered
     # device tensors, so step i's copies overlap steps i - 1 and i + 1.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and states is None:
         host_in = [G.cpu().pin_memory() for G in Gs]
         # one pinned host set for the results: the copy-out stream writes it step after
         # step in order (nothing reads it in between), so the device side alone is
@@ -715,6 +744,8 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3/16) products, fp32 accumulate",
             "data": "synthetic",
             "config": {**ns_config(w, args.quant, args.clip, world),
+                       "source": ("NVFP4 first-moment states (fs4_root_ns_batched_nvfp4)"
+                                  if states is not None else "FP32 momenta"),
                        "l2": l2_note,
                        "launch": ("one CUDA graph replay per step (the call captured once); per-phase "
                                   "times from a separate event-recording pass" if graph is not None

@@ -357,6 +357,13 @@ fs4_status fs4_root_ns_batched_nvfp4(int32_t count, const fs4_ns_desc* descs,
                                      size_t workspace_bytes, void* stream);
 
 
+/* fs4_root_ns_batched_nvfp4 with the phase events of fs4_root_ns_batched_timed. */
+fs4_status fs4_root_ns_batched_nvfp4_timed(int32_t count, const fs4_ns_desc* descs,
+                                           const fs4_nvfp4_state* states, int32_t K, float clip_k,
+                                           uint32_t flags, const uint16_t* rht_masks,
+                                           void* workspace, size_t workspace_bytes, void* stream,
+                                           void* const* phase_events, int32_t n_events);
+
 /* fs4_root_ns_batched_ex, with CUDA events recorded on `stream` around each
  * phase so a caller can time the kernels on the launching stream.
  * phase_events: HOST array of n_events >= 3 + 3K cudaEvent_t handles (created

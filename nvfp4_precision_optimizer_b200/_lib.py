@@ -79,6 +79,9 @@ SIGNATURES = {
                                        c_vp, c_sz, c_vp]),
     "fs4_root_ns_batched_nvfp4": (c_i32, [c_i32, ctypes.POINTER(NsDesc), ctypes.POINTER(Nvfp4State),
                                           c_i32, c_f32, c_u32, c_vp, c_vp, c_sz, c_vp]),
+    "fs4_root_ns_batched_nvfp4_timed": (c_i32, [c_i32, ctypes.POINTER(NsDesc), ctypes.POINTER(Nvfp4State),
+                                                c_i32, c_f32, c_u32, c_vp, c_vp, c_sz, c_vp,
+                                                ctypes.POINTER(c_vp), c_i32]),
     "fs4_root_ns_batched_timed": (c_i32, [c_i32, ctypes.POINTER(NsDesc), c_i32, c_f32, c_u32,
                                           c_vp, c_vp, c_sz, c_vp, ctypes.POINTER(c_vp), c_i32]),
     "fs4_root_ns_bf16_batched_workspace_size": (c_sz, [c_i32, ctypes.POINTER(NsDesc)]),

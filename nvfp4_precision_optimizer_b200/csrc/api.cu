@@ -450,6 +450,16 @@ fs4_status fs4_root_ns_batched_nvfp4(int32_t count, const fs4_ns_desc* descs,
                       nullptr, 0, states, false);
 }
 
+fs4_status fs4_root_ns_batched_nvfp4_timed(int32_t count, const fs4_ns_desc* descs,
+                                           const fs4_nvfp4_state* states, int32_t K, float clip_k,
+                                           uint32_t flags, const uint16_t* rht_masks,
+                                           void* workspace, size_t workspace_bytes, void* stream,
+                                           void* const* phase_events, int32_t n_events) {
+  if (!states || !phase_events) return FS4_ERR_INVALID_ARG;
+  return batched_impl(count, descs, K, clip_k, flags, rht_masks, workspace, workspace_bytes, stream,
+                      phase_events, n_events, states, false);
+}
+
 fs4_status fs4_root_ns_batched(int32_t count, const fs4_ns_desc* descs, int32_t K, float clip_k,
                                uint32_t flags, void* workspace, size_t workspace_bytes,
                                void* stream) {

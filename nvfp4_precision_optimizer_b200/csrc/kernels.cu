@@ -834,27 +834,41 @@ __device__ __forceinline__ int pre_off(int R, int col) {   // float offset of (R
 // and as both NVFP4 views, with row / column sums of the squared dequantised
 // values.  Work unit = one 64 x 64 tile of the padded working extent; G and X
 // are read and written as float4 with 16 threads per 64-float row segment.
+// Each CTA takes one contiguous range of the unit sequence (matrix by matrix, the
+// tiles of X in row-major order), so the next unit's position follows from the
+// current one by an increment: the owning matrix is searched and the tile index
+// divided once per CTA.
 template <uint32_t kOpts>
 __global__ void __launch_bounds__(kEwThreads, 4) ns_preamble_kernel(const __grid_constant__ NsParams p) {
   __shared__ __align__(16) float tile[kT * kT];
   __shared__ float scale_tab[256];
-  const int32_t total = p.prefix[p.count];
   const int t = threadIdx.x;
   if (t < 128) scale_tab_fill(scale_tab, t);   // read after the first barrier below
+
+  const int32_t total = p.prefix[p.count];
+  const int32_t per = total / (int32_t)gridDim.x, extra = total % (int32_t)gridDim.x;
+  const int32_t bid = (int32_t)blockIdx.x;
+  const int32_t first = bid * per + min(bid, extra);
+  const int32_t n_units = per + (bid < extra ? 1 : 0);
+  if (n_units <= 0) return;
+
+  // position of the next unit to load: matrix, tile row and tile column of X
+  int nmi = owner_of(p.prefix, p.count, first);
+  int32_t ntn = p.mat[nmi].np / kT, ntm = p.mat[nmi].mp / kT, nti, ntj;
+  {
+    const int32_t lu = first - p.prefix[nmi];
+    nti = lu / ntn;
+    ntj = lu - nti * ntn;
+  }
 
   // The next unit's G tile is loaded into registers while this unit is quantised
   // (interior tiles of 16-byte aligned inputs; edge tiles load on the guarded path).
   float4 pf[4];
   bool pf_fast = false;
-  auto prefetch = [&](int32_t uu) {
+  auto prefetch = [&](int mi, int32_t ti, int32_t tj) {
     pf_fast = false;
-    if (uu >= total) return;
-    const int mi = owner_of(p.prefix, p.count, uu);
     const MatDesc& d = p.mat[mi];
-    const int32_t tiles_n = d.np / kT;
-    const int32_t lu = uu - p.prefix[mi];
-    const int32_t ti = lu / tiles_n;
-    const int32_t i0 = ti * kT, j0 = (lu - ti * tiles_n) * kT;
+    const int32_t i0 = ti * kT, j0 = tj * kT;
     const int32_t rows_g = d.tall ? d.n : d.m, cols_g = d.tall ? d.m : d.n;
     const int32_t gr0 = d.tall ? j0 : i0, gc0 = d.tall ? i0 : j0;
     const bool vec = ((reinterpret_cast<uintptr_t>(d.G) & 15) == 0) && ((d.ldg & 3) == 0);
@@ -868,7 +882,7 @@ __global__ void __launch_bounds__(kEwThreads, 4) ns_preamble_kernel(const __grid
       }
     }
   };
-  prefetch(blockIdx.x);
+  prefetch(nmi, nti, ntj);
 
   // scalars of the current matrix (derived once by the reduction kernel), reloaded only
   // when the unit belongs to another matrix than the previous one
@@ -876,19 +890,27 @@ __global__ void __launch_bounds__(kEwThreads, 4) ns_preamble_kernel(const __grid
   bool dead = false;
   float inv = 0.0f, tau = 0.0f, sg = 1.0f, six_sg = 6.0f, rcp_six = 1.0f, rcp_sg = 1.0f;
 
-  for (int32_t u = blockIdx.x; u < total; u += gridDim.x) {
+  for (int32_t it = 0; it < n_units; ++it) {
     float4 cur[4];
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass) cur[pass] = pf[pass];
     const bool cur_fast = pf_fast;
-    prefetch(u + gridDim.x);
-    const int mi = owner_of(p.prefix, p.count, u);
+    const int mi = nmi;
+    const int32_t i0 = nti * kT, j0 = ntj * kT;
+    if (it + 1 < n_units) {
+      if (++ntj == ntn) {
+        ntj = 0;
+        if (++nti == ntm) {
+          nti = 0;
+          ++nmi;
+          ntn = p.mat[nmi].np / kT;
+          ntm = p.mat[nmi].mp / kT;
+        }
+      }
+      prefetch(nmi, nti, ntj);
+    }
     const MatDesc& d = p.mat[mi];
     const MatLayout L = mat_layout(d.mp, d.np, d.state_off, d.big_off, (kOpts & kOptBf16) != 0);
-    const int32_t tiles_n = d.np / kT;
-    const int32_t lu = u - p.prefix[mi];
-    const int32_t ti = lu / tiles_n;                       // 32-bit: units < 2^31
-    const int32_t i0 = ti * kT, j0 = (lu - ti * tiles_n) * kT;
     if (mi != cur_mi) {
       const NsState* st = state_of(p, d);
       cur_mi = mi;
@@ -901,7 +923,6 @@ __global__ void __launch_bounds__(kEwThreads, 4) ns_preamble_kernel(const __grid
       rcp_sg = __frcp_rn(sg);   // sg is a power of two
     }
     const ScaleTab stab{scale_tab, rcp_sg};
-
     // X0 of this tile (working orientation); a matrix with a non-finite entry is carried
     // as all zeros (its output is zero).  Non-tall: thread f holds X0 row f / 16, columns
     // 4 (f % 16) .. + 3, written to X straight from registers and staged as one float4.
@@ -983,16 +1004,18 @@ __global__ void __launch_bounds__(kEwThreads, 4) ns_preamble_kernel(const __grid
 #pragma unroll
         for (int e = 0; e < 16; ++e) v[e] = tile[pre_off(blk * 16 + e, line)];
       }
+      // row r0 + line of the view (view 0: row i0 + line of X, K from j0; view 1: row
+      // j0 + line of X^T, K from i0)
+      const int32_t r0 = view == 0 ? i0 : j0, k0 = view == 0 ? j0 : i0;
+      const int32_t Cp = view == 0 ? d.np : d.mp;
       if constexpr ((kOpts & kOptBf16) != 0) {
         // the BF16 comparison step: both views are BF16 copies (round to nearest even) of
         // X0 (view 0) and of X0^T (view 1), two 16-byte chunks per block
-        const int64_t R = (view == 0 ? i0 : j0) + line;
-        const int64_t K0 = (view == 0 ? j0 : i0) + blk * 16;
-        const int64_t Cp = view == 0 ? d.np : d.mp;
         uint8_t* dst = p.ws + (view == 0 ? L.qX[0] : L.qXT[0]);
         uint32_t w[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+        const int64_t R = r0 + line, K0 = k0 + blk * 16;
         *reinterpret_cast<uint4*>(dst + tiled_chunk_offset_bf16(R, K0, Cp)) = make_uint4(w[0], w[1], w[2], w[3]);
         *reinterpret_cast<uint4*>(dst + tiled_chunk_offset_bf16(R, K0 + 8, Cp)) = make_uint4(w[4], w[5], w[6], w[7]);
         continue;
@@ -1000,12 +1023,16 @@ __global__ void __launch_bounds__(kEwThreads, 4) ns_preamble_kernel(const __grid
       // view 0 is the Gram operand of iteration 0, view 1 the update operand
       if constexpr ((kOpts & kOptRht) != 0) rht16(v, view == 0 ? p.rht[0] : p.rht[2]);
       const QBlock16 q = quantize16<true, true, true, (kOpts & kOpt46) != 0>(v, sg, six_sg, rcp_six, stab);
-      // row (view 0: row i0+line of X, K = j0..) or row j0+line of X^T (view 1, K = i0..)
-      const int64_t R = (view == 0 ? i0 : j0) + line;
-      const int64_t K0 = view == 0 ? j0 : i0;
-      const int64_t Cp = view == 0 ? d.np : d.mp;
-      uint8_t* codes = p.ws + (view == 0 ? L.qX[0] : L.qXT[0]);
-      uint8_t* scales = p.ws + (view == 0 ? L.sX[0] : L.sXT[0]);
+      // TILED destinations from the tile origin: r0 and k0 are multiples of 64, so the
+      // row stays in one 128-row tile (at rr = r0 % 128 + line) and the block pair in one
+      // 256-column tile (16-byte chunk (k0 % 256) / 32 + blk / 2, swizzled by rr % 8),
+      // and the four scales of the line fill one word of one scale atom
+      const int32_t rr = (r0 & 64) + line;
+      uint8_t* codes = p.ws + (view == 0 ? L.qX[0] : L.qXT[0]) +
+                       (int64_t)((r0 >> 7) * (Cp >> 8) + (k0 >> 8)) * kTileBytes + rr * 128;
+      uint8_t* scales = p.ws + (view == 0 ? L.sX[0] : L.sXT[0]) +
+                        (int64_t)((r0 >> 7) * (Cp >> 6) + (k0 >> 6)) * kAtomBytes + 16 * (rr & 31) +
+                        4 * (rr >> 5);
       // pair blocks (0,1) and (2,3) into 16-byte chunks, the four scales into one word
       const uint32_t o0 = __shfl_xor_sync(0xFFFFFFFFu, q.w0, 1);
       const uint32_t o1 = __shfl_xor_sync(0xFFFFFFFFu, q.w1, 1);
@@ -1013,14 +1040,14 @@ __global__ void __launch_bounds__(kEwThreads, 4) ns_preamble_kernel(const __grid
       sc |= __shfl_xor_sync(0xFFFFFFFFu, sc, 1);
       sc |= __shfl_xor_sync(0xFFFFFFFFu, sc, 2);
       if ((blk & 1) == 0)
-        *reinterpret_cast<uint4*>(codes + tiled_chunk_offset(R, K0 + blk * 16, Cp)) =
+        *reinterpret_cast<uint4*>(codes + (((((k0 & 255) >> 5) + (blk >> 1)) ^ (line & 7)) << 4)) =
             make_uint4(q.w0, q.w1, o0, o1);
-      if (blk == 0) *reinterpret_cast<uint32_t*>(scales + tiled_scale_offset(R, K0 >> 4, Cp)) = sc;
+      if (blk == 0) *reinterpret_cast<uint32_t*>(scales) = sc;
       float ss = q.sumsq;
       ss += __shfl_xor_sync(0xFFFFFFFFu, ss, 1);
       ss += __shfl_xor_sync(0xFFFFFFFFu, ss, 2);
       if (blk == 0 && ss != 0.0f)
-        atomicAdd(reinterpret_cast<float*>(p.ws + (view == 0 ? L.rowsumX : L.colsumX)) + R, ss);
+        atomicAdd(reinterpret_cast<float*>(p.ws + (view == 0 ? L.rowsumX : L.colsumX)) + r0 + line, ss);
     }
     __syncthreads();   // the tile is restaged by the next unit
   }
