@@ -12,9 +12,12 @@
 // Kernel structure (one persistent CTA per SM, 384 threads = 3 warpgroups):
 //   warp 0     producer: 1-D bulk copies (TMA engine) of pre-tiled operand tiles
 //              and scale atoms into a 3-stage shared-memory ring
-//   warp 1     allocates 512 TMEM columns; one thread copies the scale atoms to
-//              TMEM (tcgen05.cp) and issues tcgen05.mma kind::mxf4nvf4
-//              (M=128, N=256, K=64, UE4M3 per-16 scales), FP32 accumulator in TMEM
+//   warp 1     allocates 512 TMEM columns; one thread issues tcgen05.mma
+//              kind::mxf4nvf4 (M=128, N=256, K=64, UE4M3 per-16 scales), FP32
+//              accumulator in TMEM
+//   warps 2-3  scale-factor copiers: one or two threads copy every stage's scale atoms
+//              to TMEM (tcgen05.cp) into a ring of buffers (the update's MMA thread
+//              copies its own)
 //   (a one-CTA-per-matrix kernel after each launch turns the row/column sums
 //    into the next phase's tensor scale)
 //   warps 4-11 epilogue: tcgen05.ld of the 128 x 256 accumulator into registers
@@ -28,6 +31,7 @@
 // issuing work, drains what it issued, frees TMEM and returns.
 #include <cfloat>
 #include <cmath>
+#include <type_traits>
 
 #include "fs4_device.cuh"
 #include "fs4_internal.h"
@@ -37,7 +41,7 @@ namespace fs4 {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 256;
-// 12 warps: warpgroup 0 = producer (warp 0), MMA issuer (warp 1), two idle warps;
+// 12 warps: warpgroup 0 = producer (warp 0), MMA issuer (warp 1), scale copiers (2, 3);
 // warpgroups 1-2 = 8 epilogue warps.  Registers are rebalanced after launch:
 // 384 threads x 168 = 40 x 128 (warpgroup 0) + 232 x 256 (epilogue warpgroups).
 constexpr int kThreads = 384;
@@ -82,11 +86,16 @@ struct Cfg {
   static constexpr int SMEM_BYTES =
       1024 + kStages * STAGE_BYTES + 8 * EPI_FLOATS * 4 + BAR_BYTES + 128 * 8;
   static constexpr uint32_t kIdesc = kBf16 ? idesc_bf16(BM, BN) : idesc_mxf4nvf4(BM, BN);
-  // A separate warp copies the scale factors to TMEM (a ring of kSfBufs buffers) for the
-  // products whose time is set by the mainloop: issued by the MMA thread itself, each
-  // stage's copies queue behind its MMAs.  The update, whose time is set by its
-  // epilogue, measured slower with the extra warp and keeps the copies in the MMA thread.
-  static constexpr bool kSfWarp = !kBf16 && E != Epi::Update;
+  // Scale-factor copies to TMEM (a ring of kSfBufs buffers).  A tcgen05.cp takes about 50
+  // cycles to issue, so the twelve copies of a stage issued by the MMA thread take longer
+  // than the stage's MMAs take to run: the first Gram product (and the plain GEMM), whose
+  // time is set by the mainloop, leaves them to two copier threads (warps 2 and 3, six
+  // atoms each).  Each waiting copier thread shares a scheduler with two epilogue warps,
+  // and the products whose epilogue also streams an FP32 input measured best with fewer:
+  // one copier thread for the second Gram product, the copies in the MMA thread for the
+  // update.
+  static constexpr int kSfCopiers = kBf16 ? 0 : (E == Epi::Update ? 0 : (E == Epi::GramA ? 1 : 2));
+  static constexpr bool kSfWarp = kSfCopiers > 0;
   static constexpr int kSfBufs = kSfWarp ? 4 : 2;
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(SMEM_BYTES <= 232448, "over the per-CTA shared-memory limit");
@@ -725,10 +734,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(mma_done, 1);
     mbar_init(stall_bar, 1);
     for (int b = 0; b < C::kSfBufs; ++b) {
-      mbar_init(&sf_full[b], 1);
+      mbar_init(&sf_full[b], C::kSfCopiers > 0 ? C::kSfCopiers : 1);   // one arrival per copier thread
       mbar_init(&sf_empty[b], 1);
     }
-    mbar_init(sf_done, 1);
+    mbar_init(sf_done, C::kSfCopiers > 0 ? C::kSfCopiers : 1);
     *abort_flag = (__ldcg(status) & kStatusTimeout) ? 1 : 0;
     fence_mbar_init();
   }
@@ -740,31 +749,47 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int32_t total = total_units<E>(p, g);
   if (warp < 4) {
     regs_dec<kRegsCtl>();
+  // The control loops below each run on a single issuing thread, where every tcgen05 or
+  // bulk-copy instruction costs tens of cycles to issue: they keep per-stage work to those
+  // instructions, with the stage ring position, phases, descriptors and global addresses
+  // advanced by constant steps.
+  constexpr uint64_t kStageDesc = C::STAGE_BYTES >> 4;   // descriptor address units per stage
+  const uint32_t s_base = smem_addr(stage_base);
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t it = 0;
+      uint32_t it = 0, s = 0, ph = 0;   // stages issued; ring position and its phase
       for (int32_t u = first; u < total && !*abort_flag; u += step) {
         const Job j = make_job<E, kBf16>(u, p, g);
+        // k-tile kt of a 128-row band sits kt tiles after the band's first; the second
+        // half of the B tile is the next band
+        const int64_t band = j.ktiles_total * kTileBytes, sband = j.ktiles_total * (4 * kAtomBytes);
+        const uint8_t* pa = j.a_codes + j.a_tile_row * band;
+        const uint8_t* pb = j.b_codes + j.b_tile_row * band;
+        const uint8_t* psa = j.a_sf + j.a_tile_row * sband;
+        const uint8_t* psb = j.b_sf + j.b_tile_row * sband;
+        const uint32_t tx = A_BYTES + C::SFA + (j.b_half ? (C::B_BYTES + C::SFB) / 2 : (C::B_BYTES + C::SFB));
         for (int kt = 0; kt < j.kt; ++kt, ++it) {
-          const uint32_t s = it % kStages, use = it / kStages;
-          if (!mbar_wait(&empty[s], (use & 1u) ^ 1u, status, abort_flag)) break;
-          uint8_t* st = stage_base + s * C::STAGE_BYTES;
-          uint8_t* st_b = st + A_BYTES;
-          uint8_t* st_sfa = st_b + C::B_BYTES;
-          uint8_t* st_sfb = st_sfa + C::SFA;
-          const int64_t at = j.a_tile_row * j.ktiles_total + kt;
-          const uint32_t bbytes = j.b_half ? (C::B_BYTES + C::SFB) / 2 : (C::B_BYTES + C::SFB);
-          mbar_arrive_expect_tx(&full[s], A_BYTES + C::SFA + bbytes);
-          bulk_g2s(st, j.a_codes + at * kTileBytes, A_BYTES, &full[s]);
-          if constexpr (!kBf16) bulk_g2s(st_sfa, j.a_sf + at * (4 * kAtomBytes), SFA_BYTES, &full[s]);
-          for (int h = 0; h < (j.b_half ? 1 : 2); ++h) {
-            const int64_t bt = (j.b_tile_row + h) * j.ktiles_total + kt;
-            bulk_g2s(st_b + h * kTileBytes, j.b_codes + bt * kTileBytes, kTileBytes, &full[s]);
-            if constexpr (!kBf16)
-              bulk_g2s(st_sfb + h * (4 * kAtomBytes), j.b_sf + bt * (4 * kAtomBytes), 4 * kAtomBytes,
-                       &full[s]);
+          if (!mbar_wait(&empty[s], ph ^ 1u, status, abort_flag)) break;
+          const uint32_t st = s_base + s * C::STAGE_BYTES;
+          uint64_t* fb = &full[s];
+          mbar_arrive_expect_tx(fb, tx);
+          bulk_g2s_addr(st, pa, A_BYTES, fb);
+          bulk_g2s_addr(st + A_BYTES, pb, kTileBytes, fb);
+          if constexpr (!kBf16) {
+            bulk_g2s_addr(st + A_BYTES + C::B_BYTES, psa, SFA_BYTES, fb);
+            bulk_g2s_addr(st + A_BYTES + C::B_BYTES + C::SFA, psb, 4 * kAtomBytes, fb);
           }
+          if (!j.b_half) {
+            bulk_g2s_addr(st + A_BYTES + kTileBytes, pb + band, kTileBytes, fb);
+            if constexpr (!kBf16)
+              bulk_g2s_addr(st + A_BYTES + C::B_BYTES + C::SFA + 4 * kAtomBytes, psb + sband, 4 * kAtomBytes, fb);
+          }
+          pa += kTileBytes;
+          pb += kTileBytes;
+          psa += 4 * kAtomBytes;
+          psb += 4 * kAtomBytes;
+          if (++s == (uint32_t)kStages) { s = 0; ph ^= 1u; }
         }
       }
       // drain: every issued copy must land before the CTA may exit
@@ -777,8 +802,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      uint32_t it = 0, tl = 0;
+      uint32_t tl = 0, s = 0, ph = 0, b = 0, bph = 0;   // stage ring and scale-factor ring
       const uint32_t acc = tmem;   // lane 0, column 0
+      const uint64_t da0 = sdesc_sw128(s_base), db0 = sdesc_sw128(s_base + A_BYTES);
+      const uint64_t dsf0 = sdesc_sf_atom(s_base + A_BYTES + C::B_BYTES);
       if constexpr (E != Epi::Plain) {
         // test only: a wait that runs out (bounded), exercising the timeout path
         if (p.stall) mbar_wait(stall_bar, 0, status, abort_flag);
@@ -788,42 +815,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(acc_empty, (tl & 1u) ^ 1u, status, abort_flag)) break;
         tc_fence_after();
         bool ok = true;
-        for (int kt = 0; kt < j.kt; ++kt, ++it) {
-          const uint32_t s = it % kStages, use = it / kStages;
-          if (!mbar_wait(&full[s], use & 1u, status, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint8_t* st = stage_base + s * C::STAGE_BYTES;
-          const uint32_t sa = smem_addr(st), sb = sa + A_BYTES;
-          const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sb);
+        for (int kt = 0; kt < j.kt; ++kt) {
+          if (!mbar_wait(&full[s], ph, status, abort_flag)) { ok = false; break; }
+          const uint64_t da = da0 + s * kStageDesc, db = db0 + s * kStageDesc;
           if constexpr (kBf16) {
+            tc_fence_after();
             // four K = 16 steps of BF16 per 128-byte row, no scale factors
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
               tc_mma_bf16(acc, da + 2 * ks, db + 2 * ks, C::kIdesc, (kt | ks) != 0 ? 1u : 0u);
           } else {
-            const uint32_t sfb_i = it % C::kSfBufs;
-            const uint32_t sf = tmem + kSfCol + sfb_i * kSfBufCols;
+            const uint32_t sf = tmem + kSfCol + b * kSfBufCols;
             if constexpr (C::kSfWarp) {
-              // the copier warp filled this buffer from the same stage
-              if (!mbar_wait(&sf_full[sfb_i], (it / C::kSfBufs) & 1u, status, abort_flag)) { ok = false; break; }
+              // the copier threads filled scale-factor buffer b from this stage
+              if (!mbar_wait(&sf_full[b], bph, status, abort_flag)) { ok = false; break; }
               tc_fence_after();
             } else {
-              const uint32_t ssfa = sb + C::B_BYTES, ssfb = ssfa + SFA_BYTES;
+              // this thread copies the stage's twelve scale atoms (A, k-steps 0-3; B rows
+              // 0-127 and 128-255, k-steps 0-3; 512 bytes apart); the MMAs below queue
+              // behind them
+              tc_fence_after();
+              const uint64_t d = dsf0 + s * kStageDesc;
 #pragma unroll
-              for (int ks = 0; ks < 4; ++ks) {
-                tc_copy_sf(sf + 4 * ks, sdesc_sf_atom(ssfa + ks * kAtomBytes));
-                tc_copy_sf(sf + 16 + 8 * ks, sdesc_sf_atom(ssfb + ks * kAtomBytes));
-                tc_copy_sf(sf + 16 + 8 * ks + 4, sdesc_sf_atom(ssfb + 4 * kAtomBytes + ks * kAtomBytes));
-              }
+              for (int a = 0; a < 12; ++a)
+                tc_copy_sf(sf + (a < 4 ? 4 * a : (a < 8 ? 16 + 8 * (a - 4) : 20 + 8 * (a - 8))),
+                           d + (uint64_t)(a * (kAtomBytes >> 4)));
             }
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
               tc_mma_nvf4(acc, da + 2 * ks, db + 2 * ks, C::kIdesc, sf + 4 * ks, sf + 16 + 8 * ks,
                           (kt | ks) != 0 ? 1u : 0u);
             }
-            if constexpr (C::kSfWarp) tc_commit(&sf_empty[sfb_i]);
+            if constexpr (C::kSfWarp) tc_commit(&sf_empty[b]);
+            if (++b == (uint32_t)C::kSfBufs) { b = 0; bph ^= 1u; }
           }
           tc_commit(&empty[s]);
+          if (++s == (uint32_t)kStages) { s = 0; ph ^= 1u; }
         }
         if (!ok) break;
         tc_commit(acc_full);
@@ -832,40 +859,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       volatile int never = 0;
       mbar_wait(mma_done, 0, status, &never);
     }
-  } else if (warp == 2 && C::kSfWarp) {
-    if (lane == 0) {
-      // ---------------------------------------------------------- scale-factor copier
-      // For each stage: once its operands have landed and the MMAs of the stage that last
-      // used the TMEM buffer have completed, copy the stage's scale atoms into the buffer.
-      // The MMAs that read the stage's shared memory wait for these copies (sf_full), and
-      // the producer refills the stage only after those MMAs (empty), so the copies never
-      // read a refilled stage.
-      uint32_t it = 0;
+  } else if (warp >= 2 && C::kSfWarp) {
+    // ------------------------------------------------------------ scale-factor copiers
+    // For each stage: once its operands have landed and the MMAs of the stage that last
+    // used the TMEM buffer have completed, copy the stage's twelve scale atoms into the
+    // buffer: with two copiers lane 0 of warp 2 the first six (A, k-steps 0-3; B rows
+    // 0-127, k-steps 0-1) and lane 0 of warp 3 the other six, with one copier lane 0 of
+    // warp 2 all twelve; each copier thread commits once per stage (sf_full expects one
+    // arrival per copier thread).  The MMAs that read the stage's shared memory wait for these copies
+    // (sf_full), and the producer refills the stage only after those MMAs (empty), so
+    // the copies never read a refilled stage.
+    auto copier = [&](auto first_c) {
+      constexpr int kA0 = decltype(first_c)::value;           // first atom of this thread
+      constexpr int kNA = 12 / (C::kSfCopiers > 0 ? C::kSfCopiers : 1);   // atoms per copier thread
+      uint32_t s = 0, ph = 0, b = 0, bph = 0;
       bool ok = true;
+      const uint64_t dsf = sdesc_sf_atom(s_base + A_BYTES + C::B_BYTES);
       for (int32_t u = first; u < total && ok && !*abort_flag; u += step) {
         const Job j = make_job<E, kBf16>(u, p, g);
-        for (int kt = 0; kt < j.kt; ++kt, ++it) {
-          const uint32_t s = it % kStages, use = it / kStages;
-          const uint32_t b = it % C::kSfBufs;
-          if (!mbar_wait(&full[s], use & 1u, status, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&sf_empty[b], ((it / C::kSfBufs) & 1u) ^ 1u, status, abort_flag)) { ok = false; break; }
+        for (int kt = 0; kt < j.kt; ++kt) {
+          if (!mbar_wait(&full[s], ph, status, abort_flag) ||
+              !mbar_wait(&sf_empty[b], bph ^ 1u, status, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t ssfa = smem_addr(stage_base + s * C::STAGE_BYTES) + A_BYTES + C::B_BYTES;
-          const uint32_t ssfb = ssfa + SFA_BYTES;
           const uint32_t sf = tmem + kSfCol + b * kSfBufCols;
+          const uint64_t d = dsf + s * kStageDesc;
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            tc_copy_sf(sf + 4 * ks, sdesc_sf_atom(ssfa + ks * kAtomBytes));
-            tc_copy_sf(sf + 16 + 8 * ks, sdesc_sf_atom(ssfb + ks * kAtomBytes));
-            tc_copy_sf(sf + 16 + 8 * ks + 4, sdesc_sf_atom(ssfb + 4 * kAtomBytes + ks * kAtomBytes));
+          for (int q = 0; q < kNA; ++q) {
+            // atom a: 0-3 A k-step a, 4-7 B rows 0-127 k-step a - 4, 8-11 B rows 128-255
+            // k-step a - 8; atoms sit 512 bytes apart, A's then B's
+            const int a = kA0 + q;
+            const uint32_t col = a < 4 ? 4 * a : (a < 8 ? 16 + 8 * (a - 4) : 20 + 8 * (a - 8));
+            tc_copy_sf(sf + col, d + (uint64_t)(a * (kAtomBytes >> 4)));
           }
           tc_commit(&sf_full[b]);
+          if (++s == (uint32_t)kStages) { s = 0; ph ^= 1u; }
+          if (++b == (uint32_t)C::kSfBufs) { b = 0; bph ^= 1u; }
         }
       }
       // every copy this thread issued completes before the TMEM is freed
       tc_commit(sf_done);
       volatile int never = 0;
       mbar_wait(sf_done, 0, status, &never);
+    };
+    if (lane == 0) {
+      if (warp == 2) copier(std::integral_constant<int, 0>{});
+      else if (C::kSfCopiers == 2) copier(std::integral_constant<int, 6>{});
     }
   }
   } else {
