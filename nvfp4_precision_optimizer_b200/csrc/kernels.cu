@@ -830,6 +830,41 @@ __device__ __forceinline__ int pre_off(int R, int col) {   // float offset of (R
   return R * kT + 4 * (c ^ pre_swz(R, c)) + (col & 3);
 }
 
+// clamp(fp32(x * inv), +-tau) of four values.
+__device__ __forceinline__ float4 clip4(float4 x, float inv, float tau) {
+  return make_float4(fminf(fmaxf(__fmul_rn(x.x, inv), -tau), tau), fminf(fmaxf(__fmul_rn(x.y, inv), -tau), tau),
+                     fminf(fmaxf(__fmul_rn(x.z, inv), -tau), tau), fminf(fmaxf(__fmul_rn(x.w, inv), -tau), tau));
+}
+
+// Staging of a tile that the preamble's fast path does not take: an edge tile (rows_left
+// rows and cols_left columns of G remain from the tile origin), a G that is not 16-byte
+// aligned, or a matrix with a non-finite entry (dead: staged as zeros).  Kept out of line
+// so that its per-element guards stay off the interior tiles' path.
+__device__ __noinline__ void preamble_stage_guarded(float* tile, float* Xt, const float* gtile, int64_t ldg,
+                                                    int32_t np, bool tall, bool dead, float inv, float tau,
+                                                    int32_t rows_left, int32_t cols_left, int t) {
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {
+    const int f = t + kEwThreads * pass;
+    const int line = f >> 4, c4 = (f & 15) * 4;
+    float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (!dead && line < rows_left) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (c4 + e < cols_left)
+          v[e] = fminf(fmaxf(__fmul_rn(__ldg(gtile + (int64_t)line * ldg + c4 + e), inv), -tau), tau);
+    }
+    if (!tall) {
+      const float4 v4 = make_float4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<float4*>(tile + pre_off(line, c4)) = v4;
+      *reinterpret_cast<float4*>(Xt + line * np + c4) = v4;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) tile[pre_off(c4 + e, line)] = v[e];
+    }
+  }
+}
+
 // Normalise, clip and quantise: X0 = clamp(fp32(G * inv), +-tau) written as FP32
 // and as both NVFP4 views, with row / column sums of the squared dequantised
 // values.  Work unit = one 64 x 64 tile of the padded working extent; G and X
@@ -953,32 +988,33 @@ __global__ void __launch_bounds__(kEwThreads, 4) ns_preamble_kernel(const __grid
 #pragma unroll
         for (int e = 0; e < 16; ++e) tile[pre_off(16 * blk + e, line)] = v[e];
       }
-    } else {
-#pragma unroll
-    for (int pass = 0; pass < 4; ++pass) {
-      const int f = t + kEwThreads * pass;
-      const int line = f >> 4, c4 = (f & 15) * 4;       // 64 lines of 64 floats
-      float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      if (dead) {
-      } else if (cur_fast) {
-        v[0] = cur[pass].x; v[1] = cur[pass].y; v[2] = cur[pass].z; v[3] = cur[pass].w;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) v[e] = fminf(fmaxf(__fmul_rn(v[e], inv), -tau), tau);
-      } else if (gr0 + line < rows_g) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (gc0 + c4 + e < cols_g)
-            v[e] = fminf(fmaxf(__fmul_rn(__ldg(gtile + (int64_t)line * d.ldg + c4 + e), inv), -tau), tau);
-      }
+    } else if (cur_fast && !dead) {
+      // interior tile of a finite matrix, from the prefetched float4s (each case its own
+      // uniform branch, so that the other cases' code is not predicated into this one)
       if (!d.tall) {
-        const float4 v4 = make_float4(v[0], v[1], v[2], v[3]);
-        *reinterpret_cast<float4*>(tile + pre_off(line, c4)) = v4;
-        *reinterpret_cast<float4*>(Xt + line * d.np + c4) = v4;
+#pragma unroll
+        for (int pass = 0; pass < 4; ++pass) {
+          const int f = t + kEwThreads * pass;
+          const int line = f >> 4, c4 = (f & 15) * 4;       // 64 lines of 64 floats
+          const float4 v4 = clip4(cur[pass], inv, tau);
+          *reinterpret_cast<float4*>(tile + pre_off(line, c4)) = v4;
+          *reinterpret_cast<float4*>(Xt + line * d.np + c4) = v4;
+        }
       } else {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) tile[pre_off(c4 + e, line)] = v[e];
+        for (int pass = 0; pass < 4; ++pass) {
+          const int f = t + kEwThreads * pass;
+          const int line = f >> 4, c4 = (f & 15) * 4;
+          const float4 v4 = clip4(cur[pass], inv, tau);
+          tile[pre_off(c4, line)] = v4.x;
+          tile[pre_off(c4 + 1, line)] = v4.y;
+          tile[pre_off(c4 + 2, line)] = v4.z;
+          tile[pre_off(c4 + 3, line)] = v4.w;
+        }
       }
-    }
+    } else {
+      preamble_stage_guarded(tile, Xt, gtile, d.ldg, d.np, d.tall != 0, dead, inv, tau, rows_g - gr0,
+                             cols_g - gc0, t);
     }
     __syncthreads();
     if (d.tall) {
