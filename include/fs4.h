@@ -357,7 +357,12 @@ fs4_status fs4_root_ns_batched_nvfp4(int32_t count, const fs4_ns_desc* descs,
                                      size_t workspace_bytes, void* stream);
 
 
-/* fs4_root_ns_batched_nvfp4 with the phase events of fs4_root_ns_batched_timed. */
+/* fs4_root_ns_batched_nvfp4, with CUDA events recorded on `stream` around each
+ * phase at the 3 + 3K positions of fs4_root_ns_batched_timed (phase_events: HOST
+ * array of n_events >= 3 + 3K cudaEvent_t handles created by the caller with timing
+ * enabled).  Arguments, layouts and errors as fs4_root_ns_batched_nvfp4, plus
+ * FS4_ERR_INVALID_ARG for a missing event array or too few events, checked before
+ * anything is launched. */
 fs4_status fs4_root_ns_batched_nvfp4_timed(int32_t count, const fs4_ns_desc* descs,
                                            const fs4_nvfp4_state* states, int32_t K, float clip_k,
                                            uint32_t flags, const uint16_t* rht_masks,

@@ -99,7 +99,7 @@ struct Cfg {
   static constexpr int kSfBufs = kSfWarp ? 4 : 2;
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(SMEM_BYTES <= 232448, "over the per-CTA shared-memory limit");
-  static_assert((2 * kStages + 4 + 2 * 4 + 1) * 8 + 12 <= BAR_BYTES, "barrier block too small");
+  static_assert((3 * kStages + 4 + 2 * 4 + 1) * 8 + 12 <= BAR_BYTES, "barrier block too small");
   static_assert(kSfCol + kSfBufs * kSfBufCols <= kTmemCols, "scale-factor ring over the TMEM columns");
 };
 
@@ -715,7 +715,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* sf_full = acc_full + 4;           // [kSfBufs] scale copies into a TMEM buffer done
   uint64_t* sf_empty = sf_full + C::kSfBufs;  // [kSfBufs] the MMAs reading that buffer done
   uint64_t* sf_done = sf_empty + C::kSfBufs;  // the copier's last copies completed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_done + 1);
+  uint64_t* sf_land = sf_done + 1;            // [kStages] a stage's scale atoms landed (copier products)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_land + kStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   float* scale_tab = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + C::BAR_BYTES);
   if (threadIdx.x >= 128 && threadIdx.x < 256) scale_tab_fill(scale_tab, threadIdx.x - 128);
@@ -728,6 +729,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_land[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 8);
@@ -768,23 +770,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint8_t* pb = j.b_codes + j.b_tile_row * band;
         const uint8_t* psa = j.a_sf + j.a_tile_row * sband;
         const uint8_t* psb = j.b_sf + j.b_tile_row * sband;
-        const uint32_t tx = A_BYTES + C::SFA + (j.b_half ? (C::B_BYTES + C::SFB) / 2 : (C::B_BYTES + C::SFB));
+        // with copier threads the scale atoms land on a barrier of their own (sf_land) and
+        // are issued first, so the copies to TMEM start while the codes are still in flight
+        const uint32_t tx_sf = C::SFA + (j.b_half ? C::SFB / 2 : C::SFB);
+        const uint32_t tx_codes = A_BYTES + (j.b_half ? C::B_BYTES / 2 : C::B_BYTES);
         for (int kt = 0; kt < j.kt; ++kt, ++it) {
           if (!mbar_wait(&empty[s], ph ^ 1u, status, abort_flag)) break;
           const uint32_t st = s_base + s * C::STAGE_BYTES;
           uint64_t* fb = &full[s];
-          mbar_arrive_expect_tx(fb, tx);
+          if constexpr (!kBf16) {
+            uint64_t* sb = C::kSfWarp ? &sf_land[s] : fb;
+            if constexpr (C::kSfWarp) mbar_arrive_expect_tx(sb, tx_sf);
+            bulk_g2s_addr(st + A_BYTES + C::B_BYTES, psa, SFA_BYTES, sb);
+            bulk_g2s_addr(st + A_BYTES + C::B_BYTES + C::SFA, psb, 4 * kAtomBytes, sb);
+            if (!j.b_half)
+              bulk_g2s_addr(st + A_BYTES + C::B_BYTES + C::SFA + 4 * kAtomBytes, psb + sband, 4 * kAtomBytes, sb);
+          }
+          mbar_arrive_expect_tx(fb, C::kSfWarp ? tx_codes : tx_codes + (kBf16 ? 0u : tx_sf));
           bulk_g2s_addr(st, pa, A_BYTES, fb);
           bulk_g2s_addr(st + A_BYTES, pb, kTileBytes, fb);
-          if constexpr (!kBf16) {
-            bulk_g2s_addr(st + A_BYTES + C::B_BYTES, psa, SFA_BYTES, fb);
-            bulk_g2s_addr(st + A_BYTES + C::B_BYTES + C::SFA, psb, 4 * kAtomBytes, fb);
-          }
-          if (!j.b_half) {
-            bulk_g2s_addr(st + A_BYTES + kTileBytes, pb + band, kTileBytes, fb);
-            if constexpr (!kBf16)
-              bulk_g2s_addr(st + A_BYTES + C::B_BYTES + C::SFA + 4 * kAtomBytes, psb + sband, 4 * kAtomBytes, fb);
-          }
+          if (!j.b_half) bulk_g2s_addr(st + A_BYTES + kTileBytes, pb + band, kTileBytes, fb);
           pa += kTileBytes;
           pb += kTileBytes;
           psa += 4 * kAtomBytes;
@@ -797,6 +802,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t k = from; k < it; ++k) {
         volatile int never = 0;
         mbar_wait(&full[k % kStages], (k / kStages) & 1u, status, &never);
+        if constexpr (C::kSfWarp) mbar_wait(&sf_land[k % kStages], (k / kStages) & 1u, status, &never);
       }
     }
   } else if (warp == 1) {
@@ -861,9 +867,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 2 && C::kSfWarp) {
     // ------------------------------------------------------------ scale-factor copiers
-    // For each stage: once its operands have landed and the MMAs of the stage that last
-    // used the TMEM buffer have completed, copy the stage's twelve scale atoms into the
-    // buffer: with two copiers lane 0 of warp 2 the first six (A, k-steps 0-3; B rows
+    // For each stage: once its scale atoms have landed (sf_land) and the MMAs of the stage
+    // that last used the TMEM buffer have completed, copy the stage's twelve scale atoms
+    // into the buffer: with two copiers lane 0 of warp 2 the first six (A, k-steps 0-3; B rows
     // 0-127, k-steps 0-1) and lane 0 of warp 3 the other six, with one copier lane 0 of
     // warp 2 all twelve; each copier thread commits once per stage (sf_full expects one
     // arrival per copier thread).  The MMAs that read the stage's shared memory wait for these copies
@@ -878,7 +884,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int32_t u = first; u < total && ok && !*abort_flag; u += step) {
         const Job j = make_job<E, kBf16>(u, p, g);
         for (int kt = 0; kt < j.kt; ++kt) {
-          if (!mbar_wait(&full[s], ph, status, abort_flag) ||
+          if (!mbar_wait(&sf_land[s], ph, status, abort_flag) ||
               !mbar_wait(&sf_empty[b], bph ^ 1u, status, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sf = tmem + kSfCol + b * kSfBufCols;
