@@ -197,6 +197,18 @@ fs4_status run_ns(const Plan& pl, int32_t K, float clip_k, uint32_t flags, const
   if ((e = launch_ns_preamble(p, st, num_sms)) != cudaSuccess) return FS4_ERR_CUDA;
   if (!mark()) return FS4_ERR_CUDA;
   if (stop == 0) return FS4_OK;
+  // 8192-class batches (FLOP-weighted mean of the short side m at least 6144): the products'
+  // mainloops outlast their epilogues, and the kernels variant with more scale-factor
+  // copier threads is the faster one
+  {
+    double wsum = 0.0, wm = 0.0;
+    for (int i = 0; i < pl.count; ++i) {
+      const double m = (double)pl.mat[i].m, w = m * m * (double)pl.mat[i].n;
+      wsum += w;
+      wm += w * m;
+    }
+    if (wsum > 0.0 && wm >= 6144.0 * wsum) p.opts |= kOptWideK;
+  }
   for (int k = 0; k < K; ++k) {
     p.iter = k;
     p.last = 0;

@@ -119,6 +119,8 @@ constexpr uint32_t kOptRht = 1u, kOpt46 = 2u;   // NsParams::opts
 constexpr uint32_t kOptQuantile = 4u;            // clip at the clip_k-quantile of |X_0|
 constexpr uint32_t kOptNvSrc = 8u;               // every G is an NVFP4 state (MatDesc::qcodes)
 constexpr uint32_t kOptBf16 = 16u;               // BF16 operand views and kind::f16 products
+constexpr uint32_t kOptWideK = 32u;              // NVFP4 products of 8192-class matrices: their
+                                                 // mainloops set the time (two scale copiers each)
 
 struct NsParams {
   int32_t count;

@@ -73,7 +73,7 @@ constexpr float kBoundInflate = 1.0f + 1.0f / 256.0f;
 // Per-kernel configuration.  kBf16: the BF16 comparison step, whose operands are BF16
 // tiles of the same 128-byte rows (64 elements of K per tile instead of 256) and carry
 // no scale factors.
-template <Epi E, bool kBf16 = false>
+template <Epi E, bool kBf16 = false, bool kWide = false>
 struct Cfg {
   static constexpr int kStages = 3;
   static constexpr int kTileK = kBf16 ? 64 : BK;              // K elements per stage
@@ -91,10 +91,12 @@ struct Cfg {
   // than the stage's MMAs take to run: the first Gram product (and the plain GEMM), whose
   // time is set by the mainloop, leaves them to two copier threads (warps 2 and 3, six
   // atoms each).  Each waiting copier thread shares a scheduler with two epilogue warps,
-  // and the products whose epilogue also streams an FP32 input measured best with fewer:
-  // one copier thread for the second Gram product, the copies in the MMA thread for the
-  // update.
-  static constexpr int kSfCopiers = kBf16 ? 0 : (E == Epi::Update ? 0 : (E == Epi::GramA ? 1 : 2));
+  // and the products whose epilogue also streams an FP32 input measured best with fewer
+  // on 3072-wide matrices: one copier thread for the second Gram product, the copies in
+  // the MMA thread for the update.  With an inner dimension of 8192 (kWide) every product's
+  // mainloop outlasts its epilogue, and all three take two copier threads.
+  static constexpr int kSfCopiers =
+      kBf16 ? 0 : (kWide ? 2 : (E == Epi::Update ? 0 : (E == Epi::GramA ? 1 : 2)));
   static constexpr bool kSfWarp = kSfCopiers > 0;
   static constexpr int kSfBufs = kSfWarp ? 4 : 2;
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
@@ -699,7 +701,7 @@ template <Epi E, uint32_t kOpts>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ NsParams p, const __grid_constant__ GemmPlainArgs g) {
   constexpr bool kBf16 = (kOpts & kOptBf16) != 0;
-  using C = Cfg<E, kBf16>;
+  using C = Cfg<E, kBf16, (kOpts & kOptWideK) != 0>;
   constexpr int kStages = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -940,7 +942,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <Epi E, uint32_t kOpts>
 cudaError_t launch_impl(const NsParams* p, const GemmPlainArgs* g, int64_t units, cudaStream_t st,
                         int num_sms) {
-  using C = Cfg<E, (kOpts & kOptBf16) != 0>;
+  using C = Cfg<E, (kOpts & kOptBf16) != 0, (kOpts & kOptWideK) != 0>;
   static unsigned long long attr_set = 0ull;   // one bit per device; a benign race
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1000,11 +1002,15 @@ cudaError_t launch_ns_opts(Epi epi, const NsParams& p, cudaStream_t st, int num_
 
 cudaError_t launch_gemm_ns(Epi epi, const NsParams& p, cudaStream_t st, int num_sms) {
   if (p.opts & kOptBf16) return launch_ns_opts<kOptBf16>(epi, p, st, num_sms);
-  switch (p.opts & (kOptRht | kOpt46)) {
+  switch (p.opts & (kOptRht | kOpt46 | kOptWideK)) {
     case 0: return launch_ns_opts<0>(epi, p, st, num_sms);
     case kOpt46: return launch_ns_opts<kOpt46>(epi, p, st, num_sms);
     case kOptRht: return launch_ns_opts<kOptRht>(epi, p, st, num_sms);
-    default: return launch_ns_opts<kOptRht | kOpt46>(epi, p, st, num_sms);
+    case kOptRht | kOpt46: return launch_ns_opts<kOptRht | kOpt46>(epi, p, st, num_sms);
+    case kOptWideK: return launch_ns_opts<kOptWideK>(epi, p, st, num_sms);
+    case kOptWideK | kOpt46: return launch_ns_opts<kOptWideK | kOpt46>(epi, p, st, num_sms);
+    case kOptWideK | kOptRht: return launch_ns_opts<kOptWideK | kOptRht>(epi, p, st, num_sms);
+    default: return launch_ns_opts<kOptWideK | kOptRht | kOpt46>(epi, p, st, num_sms);
   }
 }
 
