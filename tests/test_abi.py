@@ -239,6 +239,38 @@ def test_nvfp4_source_argument_errors(F):
     assert nv(1, arr, st, 5, 3.0, 0, None, W, need, None) == -3
 
 
+def test_timed_entry_points_check_their_events_on_the_host(F):
+    """The phase-timed calls (fs4_root_ns_batched_timed, fs4_root_ns_batched_nvfp4_timed,
+    fs4_root_ns_bf16_batched_timed) refuse a missing event array, fewer than 3 + 3K events or
+    a null event handle before anything is launched (the handles are not touched here)."""
+    lib = F._lib.lib()
+    K = 2
+    n = 3 + 3 * K
+    arr = (F._lib.NsDesc * 1)()
+    arr[0] = F._lib.NsDesc(1 << 33, 1 << 34, 64, 96, 96, 96, 1.0, 0.0, 0.0)
+    W = 1 << 40
+    ev = (F._lib.c_vp * n)(*([1 << 20] * n))
+    ev_null = (F._lib.c_vp * n)(*([1 << 20] * (n - 1) + [None]))
+    need = lib.fs4_root_ns_batched_workspace_size(1, arr)
+    t = lib.fs4_root_ns_batched_timed
+    assert t(1, arr, K, 3.0, 0, None, W, need, None, None, n) == -1      # no event array
+    assert t(1, arr, K, 3.0, 0, None, W, need, None, ev, n - 1) == -1    # one event short
+    assert t(1, arr, K, 3.0, 0, None, W, need, None, ev_null, n) == -1   # a null handle
+    assert t(1, arr, K, 3.0, 0, None, W, need - 1, None, ev, n) == -4    # workspace first
+    need_b = lib.fs4_root_ns_bf16_batched_workspace_size(1, arr)
+    assert need_b > need                                                   # 2 B per view element
+    tb = lib.fs4_root_ns_bf16_batched_timed
+    assert tb(1, arr, K, 3.0, 0, W, need_b, None, None, n) == -1
+    assert tb(1, arr, K, 3.0, 0, W, need_b, None, ev, n - 1) == -1
+    st = (F._lib.Nvfp4State * 1)()
+    st[0] = F._lib.Nvfp4State(1 << 30, 1 << 31, 1 << 32, 0x1234)
+    arr[0] = F._lib.NsDesc(None, 1 << 34, 64, 96, 96, 96, 1.0, 0.0, 0.0)
+    tn = lib.fs4_root_ns_batched_nvfp4_timed
+    assert tn(1, arr, st, K, 3.0, 0, None, W, need, None, None, n) == -1
+    assert tn(1, arr, None, K, 3.0, 0, None, W, need, None, ev, n) == -1
+    assert tn(1, arr, st, K, 3.0, 0, None, W, need, None, ev, n - 1) == -1
+
+
 def test_missing_library_fails_loudly():
     """Without libfs4.so every call raises ImportError: there is no CPU or library
     fallback.  Checked in a fresh interpreter whose loader points at a missing path."""
