@@ -60,3 +60,23 @@ def test_reference_arm_other_ranks_exit_quietly():
                         "single_256x256_gauss", "--steps", "1", "--warmup", "0"],
                        cwd=ROOT, capture_output=True, text=True, timeout=300, env=env)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_committed_traffic_is_close_to_the_algorithmic_bytes():
+    """profiles/traffic.json holds each launch's measured DRAM bytes (ncu, scaled to the
+    workload by its units).  A product or element-wise phase that re-read its operands from
+    DRAM would show well above its algorithmic bytes; a capture of the wrong launch would
+    show far off either way.  Writes still in L2 when a kernel ends make the measurement a
+    little lower."""
+    import bench
+    from nvfp4_precision_optimizer_b200.workloads import WORKLOADS
+
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        traffic = json.load(f)
+    assert "3b_28blocks_student" in traffic
+    for workload, kinds in traffic.items():
+        for kind in ("reduce", "preamble", "gram_x", "gram_a", "update"):
+            ent = kinds[kind]
+            ratio = ent["bytes_per_launch"] / bench.bytes_per_launch(WORKLOADS[workload], kind)
+            assert 0.6 <= ratio <= 1.25, (workload, kind, ratio)
+            assert len(ent["source_sha"]) == 16 and ent["how"]
