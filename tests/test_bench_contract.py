@@ -80,3 +80,30 @@ def test_committed_traffic_is_close_to_the_algorithmic_bytes():
             ratio = ent["bytes_per_launch"] / bench.bytes_per_launch(WORKLOADS[workload], kind)
             assert 0.6 <= ratio <= 1.25, (workload, kind, ratio)
             assert len(ent["source_sha"]) == 16 and ent["how"]
+
+
+def test_roofline_helpers_by_hand():
+    """bench.py's per-launch algorithmic work, for one m x n matrix (m <= n) in working
+    orientation: the update is 2 m^2 n FLOPs over 0.5625 m^2 + 0.5625 mn + 8 mn + 1.125 mn
+    bytes, the Gram products m (m + 1) n and m (m + 1) m FLOPs (symmetric halves).  With
+    the measured peaks' ratio (about 992 FLOPs per byte for dense FP4) the update of a
+    3072-row matrix is HBM-bound and that of an 8192-row matrix tensor-bound."""
+    import bench
+    from nvfp4_precision_optimizer_b200.workloads import Workload
+
+    m, n = 3072, 8192
+    w = Workload("hand", [(n, m)], "gauss")          # a tall matrix, transposed to m x n
+    assert bench.flops_per_launch(w, "update") == 2 * m * m * n
+    assert bench.flops_per_launch(w, "gram_x") == m * (m + 1) * n
+    assert bench.flops_per_launch(w, "gram_a") == m * (m + 1) * m
+    e = m * n
+    assert bench.bytes_per_launch(w, "update") == pytest.approx(0.5625 * m * m + 0.5625 * e + 8 * e + 1.125 * e)
+    assert bench.bytes_per_launch(w, "reduce") == 4 * e
+    assert bench.bytes_per_launch(w, "preamble") == pytest.approx(9.125 * e)
+
+    fp4, hbm = 4.0 * 1622.9e12, 6540.8e9             # peaks of the pool's B200s
+    for side, bound in ((3072, "hbm"), (8192, "tensor")):
+        wm = Workload("hand", [(side, side)], "gauss")
+        t_flop = bench.flops_per_launch(wm, "update") / fp4
+        t_byte = bench.bytes_per_launch(wm, "update") / hbm
+        assert ("hbm" if t_byte > t_flop else "tensor") == bound, side
