@@ -209,9 +209,9 @@ def root_ns(G, K=5, a=3.4445, b=-4.7750, c=2.0315, clip_k=3.0, eps=NS_EPS,
         norm = float(np.sqrt(np.sum(X64 ** 2)))
         X0 = X64 / (norm + eps)
         if clip_quantile is not None:
-            a = np.abs(X0).ravel()
-            k = quantile_rank(clip_quantile, a.size)
-            tau = np.partition(a, k - 1)[k - 1]
+            mag = np.abs(X0).ravel()
+            k = quantile_rank(clip_quantile, mag.size)
+            tau = np.partition(mag, k - 1)[k - 1]
             X0 = np.clip(X0, -tau, tau)
         elif clip_k is not None and clip_k > 0:
             tau = clip_k * np.sqrt(np.sum(X0 ** 2)) / np.sqrt(X0.size)
