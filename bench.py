@@ -291,12 +291,11 @@ def oracle_sample_rate(w, budget_s: float, quant: str = "plain", clip: str = "rm
     """Time the oracle (as it stands) on one bounded sample of the workload:
     one NVFP4 Newton-Schulz iteration of an m x n slice of its first matrix (the whole
     matrix when that fits the budget), with the quantiser options and clip rule of the run.
-    The plain step (3 x RMS clip, no H16^r, no 4/6) runs the C++ oracle (OpenMP over
-    rows, float64 triple loops, no BLAS); the options run the numpy oracle, the only
-    one that implements them.
+    It runs the C++ oracle (OpenMP over rows, float64 triple loops, no BLAS), which
+    implements the plain step and every option (H16^r, adaptive 4/6, the quantile clip).
     Returns (matrices/s extrapolated by algorithmic FLOPs, seconds, description, cores)."""
     import numpy as np
-    from oracle import root_ns as R
+    from oracle import cpp_oracle as C
     from nvfp4_precision_optimizer_b200.workloads import BASE_SEED, generate
     r0, c0 = w.shapes[0]
     m_full, n_full = min(r0, c0), max(r0, c0)
@@ -305,27 +304,16 @@ def oracle_sample_rate(w, budget_s: float, quant: str = "plain", clip: str = "rm
     if quant in ("rht", "rht46"):
         masks = [int(v) for v in np.random.default_rng(BASE_SEED + 7).integers(0, 1 << 16, 3)]
     a46 = quant in ("a46", "rht46")
-    use_cpp = quant == "plain" and clip == "rms"
-    if use_cpp:
-        from oracle import cpp_oracle as C
-        cores = C.threads()
-    else:
-        cores = cpu_cores()
+    cores = C.threads()
     m = m_full
     while True:
-        if use_cpp:
-            X0 = C.normalise_and_clip(G[:m], w.clip_k)[0]
-            t0 = time.perf_counter()
-            C.ns_iterations_nvfp4(X0, 1, *w.coeffs[0])
-            dt = time.perf_counter() - t0
+        if clip == "p99":
+            X0 = C.normalise_and_clip(G[:m], None, clip_quantile=0.99)[0]
         else:
-            if clip == "p99":
-                X0, _, _, _ = R.normalise_and_clip(G[:m], None, clip_quantile=0.99)
-            else:
-                X0, _, _, _ = R.normalise_and_clip(G[:m], w.clip_k)
-            t0 = time.perf_counter()
-            R.ns_iterations_nvfp4(X0, 1, *w.coeffs[0], rht_masks=masks, adaptive46=a46)
-            dt = time.perf_counter() - t0
+            X0 = C.normalise_and_clip(G[:m], w.clip_k)[0]
+        t0 = time.perf_counter()
+        C.ns_iterations_nvfp4(X0, 1, *w.coeffs[0], rht_masks=masks, adaptive46=a46)
+        dt = time.perf_counter() - t0
         if dt <= budget_s or m <= 256:
             break
         m //= 2
@@ -333,8 +321,7 @@ def oracle_sample_rate(w, budget_s: float, quant: str = "plain", clip: str = "rm
     f_matrix = w.K * (m_full * (m_full + 1) * n_full + m_full * (m_full + 1) * m_full
                       + 2 * m_full * m_full * n_full)
     per_matrix_s = dt * f_matrix / f_sample
-    which = ("C++ oracle (OpenMP over rows, float64 triple loops, no BLAS, exact NVFP4 emulation)"
-             if use_cpp else "numpy oracle (float64 BLAS products, exact NVFP4 emulation)")
+    which = "C++ oracle (OpenMP over rows, float64 triple loops, no BLAS, exact NVFP4 emulation)"
     desc = (f"{which}: one NVFP4 NS iteration of a {m}x{n_full} slice of the first "
             f"{m_full}x{n_full} matrix, {dt:.2f} s on {cores} threads, extrapolated by algorithmic "
             f"FLOPs to K={w.K} iterations of one full matrix")

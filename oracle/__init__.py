@@ -24,6 +24,8 @@ Modules:
                           products in float64 on dequantised operands.
   * ``oracle.cpp_oracle`` -- ctypes binding of ``oracle/cpp/fs4_oracle.cpp``, the
                           same steps restated in plain C++17 (OpenMP over rows,
-                          float64 triple loops, no BLAS); a second, independent
-                          implementation, and the one the CPU baseline times.
+                          float64 triple loops, no BLAS), options included
+                          (H16^r, adaptive 4/6, quantile clip); a second,
+                          independent implementation, and the one the CPU
+                          baseline times.
 """

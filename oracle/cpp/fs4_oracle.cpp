@@ -31,6 +31,22 @@
 //   * A, B and X are FP32 tensors; products are float64 sums over dequantised
 //     operands, rounded once to FP32 (B and X' after the combine).  A is made
 //     exactly symmetric from its upper triangle.  Tall inputs are transposed.
+//
+// Options of Section 3.4 (off by default; the same readings as the numpy oracle):
+//   * Adaptive 4/6 ("All quantizations use RTN and adaptive 4/6 scaling"; Four
+//     Over Six): every block is quantised twice, with its amax mapped to M = 6 and
+//     to M = 4, and keeps M = 4 only when that candidate's squared error, summed
+//     in FP32 in element order, is strictly smaller.  Both candidates share s_g,
+//     whose denominator becomes 4 * 448 = 1792.
+//   * H16^r ("a fresh 16x16 random Hadamard transform" along K of every quantised
+//     operand): H16^r = D H16 / 4 with D the diagonal of 16 signs given by a 16-bit
+//     mask (bit i set: element i negated), one mask per product (3k: A_k, 3k + 1:
+//     qA qA16, 3k + 2: qB qX16), applied in FP32 as the butterfly with strides 1, 2,
+//     4, 8 ((u, v) -> (u + v, u - v)) and a final exact * 0.25.
+//   * Quantile clip ("p99 outlier clipping", Table 8 "Root quantile ratio 0.99"):
+//     tau is the k-th smallest |fp32(G inv)|, k = ceil(fl64(fp32(q)) N) clamped to
+//     [1, N] (the nearest-rank quantile), in place of clip_k * RMS.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -45,6 +61,9 @@ namespace {
 constexpr int kBlock = 16;
 constexpr double kE2m1Mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
 constexpr double kSgDenom = 6.0 * 448.0;   // 2688
+constexpr double kSgDenom46 = 4.0 * 448.0; // 1792: the M = 4 candidate fits too
+constexpr int kAmaxMode = 1;               // quantiser flags: s_g = amax / denom
+constexpr int kAdaptive46 = 2;             //                  adaptive 4/6 blocks
 constexpr double kEps = 1e-7;
 
 // Value of an FP8 E4M3 byte (bias 7, no infinities, S.1111.111 = NaN, exponent
@@ -93,40 +112,71 @@ const E4m3Grid& e4m3_grid() {
 int e2m1_encode(double q) { return nearest_even(q, kE2m1Mag, 8); }
 int e4m3_encode(double v) { return nearest_even(v, e4m3_grid().v, 127); }
 
-float tensor_scale(float amax, int amax_mode) {
+float tensor_scale(float amax, int amax_mode, double denom = kSgDenom) {
   if (!(amax > 0.0f)) return 1.0f;
-  if (amax_mode) return amax / 2688.0f;
+  if (amax_mode) return amax / (float)denom;
   int e = std::ilogb((double)amax) - 12;
-  while (std::ldexp(kSgDenom, e) < (double)amax) ++e;
-  while (std::ldexp(kSgDenom, e - 1) >= (double)amax) --e;
+  while (std::ldexp(denom, e) < (double)amax) ++e;
+  while (std::ldexp(denom, e - 1) >= (double)amax) --e;
   if (e < -116) e = -116;
   if (e > 118) e = 118;
   return (float)std::ldexp(1.0, e);
 }
 
+// One block of 16 FP32 values with its amax mapped to M: the E4M3 scale byte, the
+// 4-bit codes and the FP32 dequantised values.
+struct Block {
+  int scale;
+  uint8_t code[kBlock];
+  float deq[kBlock];
+};
+
+Block quantize_block(const float* xb, float s_g, float M) {
+  Block q;
+  float amax = 0.0f;
+  for (int i = 0; i < kBlock; ++i) amax = std::fmax(amax, std::fabs(xb[i]));
+  const float v = amax / (M * s_g);
+  q.scale = e4m3_encode((double)v);
+  const float den = (float)e4m3_value(q.scale) * s_g;
+  for (int i = 0; i < kBlock; ++i) {
+    uint8_t code = 0;
+    if (den > 0.0f) {
+      const float r = std::fabs(xb[i]) / den;
+      code = (uint8_t)(e2m1_encode((double)r) | (std::signbit(xb[i]) ? 8 : 0));
+    }
+    q.code[i] = code;
+    q.deq[i] = (float)(e2m1_value(code) * (double)den);
+  }
+  return q;
+}
+
+// sum_i (x_i - deq_i)^2 in FP32, one rounding per operation, i = 0 .. 15 in order.
+float block_sq_error(const float* xb, const Block& q) {
+  float e = 0.0f;
+  for (int i = 0; i < kBlock; ++i) {
+    const float d = xb[i] - q.deq[i];
+    const float d2 = d * d;
+    e = e + d2;
+  }
+  return e;
+}
+
 // Q1x16 of an FP32 rows x cols matrix (cols % 16 == 0) with tensor scale s_g:
-// 4-bit codes (one per element, unpacked) and E4M3 scale bytes.
-void quantize_rows(const float* x, int64_t rows, int64_t cols, float s_g, uint8_t* nib,
-                   uint8_t* scales) {
-  const float six_sg = 6.0f * s_g;
+// 4-bit codes (one per element, unpacked) and E4M3 scale bytes.  adaptive46: each
+// block keeps the M = 4 candidate when its squared error is strictly smaller.
+void quantize_rows(const float* x, int64_t rows, int64_t cols, float s_g, bool adaptive46,
+                   uint8_t* nib, uint8_t* scales) {
 #pragma omp parallel for schedule(static)
   for (int64_t r = 0; r < rows; ++r) {
     for (int64_t jb = 0; jb < cols / kBlock; ++jb) {
       const float* xb = x + r * cols + jb * kBlock;
-      float amax = 0.0f;
-      for (int i = 0; i < kBlock; ++i) amax = std::fmax(amax, std::fabs(xb[i]));
-      const float v = amax / six_sg;
-      const int s = e4m3_encode((double)v);
-      scales[r * (cols / kBlock) + jb] = (uint8_t)s;
-      const float den = (float)e4m3_value(s) * s_g;
-      for (int i = 0; i < kBlock; ++i) {
-        uint8_t code = 0;
-        if (den > 0.0f) {
-          const float q = std::fabs(xb[i]) / den;
-          code = (uint8_t)(e2m1_encode((double)q) | (std::signbit(xb[i]) ? 8 : 0));
-        }
-        nib[r * cols + jb * kBlock + i] = code;
+      Block q = quantize_block(xb, s_g, 6.0f);
+      if (adaptive46) {
+        const Block q4 = quantize_block(xb, s_g, 4.0f);
+        if (block_sq_error(xb, q4) < block_sq_error(xb, q)) q = q4;
       }
+      scales[r * (cols / kBlock) + jb] = (uint8_t)q.scale;
+      for (int i = 0; i < kBlock; ++i) nib[r * cols + jb * kBlock + i] = q.code[i];
     }
   }
 }
@@ -152,22 +202,59 @@ void transpose(const float* x, int64_t rows, int64_t cols, float* y) {
     for (int64_t c = 0; c < cols; ++c) y[c * rows + r] = x[r * cols + c];
 }
 
-// Dequantised Q1x16(x) (s_g from the exact amax) as a rows x cols float64 matrix.
-void q1x16(const float* x, int64_t rows, int64_t cols, double* out, float* sg_out) {
+// Quantiser options of one NS iteration: quantiser flags (kAmaxMode, kAdaptive46)
+// and the 3K sign masks of H16^r (null: H = I).
+struct Opts {
+  int flags = 0;
+  const uint16_t* masks = nullptr;
+};
+
+// x H16^r on every 16-element block of each row, in FP32 (rows x cols, in place):
+// signs of D, then the butterfly with strides 1, 2, 4, 8, then * 0.25.
+void hadamard_rows(float* x, int64_t rows, int64_t cols, uint16_t mask) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t jb = 0; jb < cols / kBlock; ++jb) {
+      float* y = x + r * cols + jb * kBlock;
+      for (int i = 0; i < kBlock; ++i)
+        if ((mask >> i) & 1) y[i] = -y[i];
+      for (int h = 1; h < kBlock; h *= 2)
+        for (int i = 0; i < kBlock; i += 2 * h)
+          for (int j = i; j < i + h; ++j) {
+            const float u = y[j], v = y[j + h];
+            y[j] = u + v;
+            y[j + h] = u - v;
+          }
+      for (int i = 0; i < kBlock; ++i) y[i] = y[i] * 0.25f;
+    }
+  }
+}
+
+// Dequantised Q1x16(x H) (s_g from the exact amax of x H) as a rows x cols float64
+// matrix; mask < 0: H = I.
+void q1x16(const float* x, int64_t rows, int64_t cols, int flags, int mask, double* out,
+           float* sg_out) {
+  std::vector<float> xh;
+  if (mask >= 0) {
+    xh.assign(x, x + rows * cols);
+    hadamard_rows(xh.data(), rows, cols, (uint16_t)mask);
+    x = xh.data();
+  }
   std::vector<uint8_t> nib((size_t)(rows * cols)), sc((size_t)(rows * cols / kBlock));
-  const float sg = tensor_scale(amax_of(x, rows * cols), 0);
-  quantize_rows(x, rows, cols, sg, nib.data(), sc.data());
+  const bool a46 = flags & kAdaptive46;
+  const float sg = tensor_scale(amax_of(x, rows * cols), flags & kAmaxMode, a46 ? kSgDenom46 : kSgDenom);
+  quantize_rows(x, rows, cols, sg, a46, nib.data(), sc.data());
   dequantize_rows(nib.data(), sc.data(), sg, rows, cols, out);
   if (sg_out) *sg_out = sg;
 }
 
-// Dequantised Q16x1(x): blocks of 16 down each column, returned as the rows x cols
-// matrix (the quantisation of x^T, transposed back).
-void q16x1(const float* x, int64_t rows, int64_t cols, double* out) {
+// Dequantised Q16x1(H^T x): blocks of 16 down each column, returned as the rows x
+// cols matrix.  Held as the Q1x16 of (H^T x)^T = x^T H, transposed back.
+void q16x1(const float* x, int64_t rows, int64_t cols, int flags, int mask, double* out) {
   std::vector<float> xt((size_t)(rows * cols));
   transpose(x, rows, cols, xt.data());
   std::vector<double> dt((size_t)(rows * cols));
-  q1x16(xt.data(), cols, rows, dt.data(), nullptr);
+  q1x16(xt.data(), cols, rows, flags, mask, dt.data(), nullptr);
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t c = 0; c < cols; ++c) out[r * cols + c] = dt[c * rows + r];
 }
@@ -186,48 +273,77 @@ void product(const double* L, const double* R, int64_t M, int64_t K, int64_t N, 
   }
 }
 
-// X_0 from G (m x n, working orientation): returns ||G||_F.
-double normalise_and_clip(const float* G, int64_t m, int64_t n, double clip_k, float* X0,
-                          float* inv_out, float* tau_out) {
+// 1-based rank of the nearest-rank q-quantile of N values: ceil(fl64(fp32(q)) N),
+// clamped to [1, N].
+int64_t quantile_rank(double q, int64_t N) {
+  int64_t k = (int64_t)std::ceil((double)(float)q * (double)N);
+  return k < 1 ? 1 : (k > N ? N : k);
+}
+
+// The k-th smallest of a[0 .. N) (1-based k): sort a copy and index it.
+template <class T>
+T kth_smallest(const T* a, int64_t N, int64_t k) {
+  std::vector<T> s(a, a + N);
+  std::sort(s.begin(), s.end());
+  return s[(size_t)(k - 1)];
+}
+
+// X_0 from G (m x n, working orientation): returns ||G||_F.  clip_quantile > 0:
+// tau is that quantile of |fp32(G inv)|; else clip_k > 0: tau = clip_k * RMS;
+// else no clip.
+double normalise_and_clip(const float* G, int64_t m, int64_t n, double clip_k,
+                          double clip_quantile, float* X0, float* inv_out, float* tau_out) {
   double s = 0.0;
   for (int64_t i = 0; i < m * n; ++i) s += (double)G[i] * (double)G[i];
   const double norm = std::sqrt(s);
   const float inv = (float)(1.0 / (norm + kEps));
   for (int64_t i = 0; i < m * n; ++i) X0[i] = G[i] * inv;
   float tau = 0.0f;
-  if (clip_k > 0.0) {
+  bool clip = false;
+  if (clip_quantile > 0.0) {
+    std::vector<float> a((size_t)(m * n));
+    for (int64_t i = 0; i < m * n; ++i) a[i] = std::fabs(X0[i]);
+    tau = kth_smallest(a.data(), m * n, quantile_rank(clip_quantile, m * n));
+    clip = true;
+  } else if (clip_k > 0.0) {
     tau = (float)(clip_k * norm * (double)inv / std::sqrt((double)m * (double)n));
-    for (int64_t i = 0; i < m * n; ++i) X0[i] = X0[i] > tau ? tau : (X0[i] < -tau ? -tau : X0[i]);
+    clip = true;
   }
+  if (clip)
+    for (int64_t i = 0; i < m * n; ++i) X0[i] = X0[i] > tau ? tau : (X0[i] < -tau ? -tau : X0[i]);
   if (inv_out) *inv_out = inv;
   if (tau_out) *tau_out = tau;
   return norm;
 }
 
-// One NVFP4 Newton-Schulz iteration on the FP32 m x n X (m <= n), in place.
-void nvfp4_iteration(float* X, int64_t m, int64_t n, double a, double b, double c) {
+// One NVFP4 Newton-Schulz iteration k on the FP32 m x n X (m <= n), in place.
+void nvfp4_iteration(float* X, int64_t m, int64_t n, double a, double b, double c, int k,
+                     const Opts& o) {
+  const int hX = o.masks ? o.masks[3 * k] : -1;       // H of A_k = qX qX^T
+  const int hA = o.masks ? o.masks[3 * k + 1] : -1;   // H of qA qA16
+  const int hU = o.masks ? o.masks[3 * k + 2] : -1;   // H' of qB qX16
   std::vector<double> dX((size_t)(m * n)), dX16((size_t)(m * n));
-  q1x16(X, m, n, dX.data(), nullptr);       // qX
-  q16x1(X, m, n, dX16.data());              // qX16x1
+  q1x16(X, m, n, o.flags, hX, dX.data(), nullptr);       // qX = Q1x16(X H)
+  q16x1(X, m, n, o.flags, hU, dX16.data());              // qX16x1 = Q16x1(H'^T X)
   // A = qX qX^T (upper triangle, mirrored), FP32
   std::vector<double> dXt((size_t)(m * n));
   for (int64_t r = 0; r < m; ++r)
-    for (int64_t k = 0; k < n; ++k) dXt[k * m + r] = dX[r * n + k];
+    for (int64_t kk = 0; kk < n; ++kk) dXt[kk * m + r] = dX[r * n + kk];
   std::vector<double> A64((size_t)(m * m));
   product(dX.data(), dXt.data(), m, n, m, A64.data());
   std::vector<float> A((size_t)(m * m));
   for (int64_t i = 0; i < m; ++i)
     for (int64_t j = i; j < m; ++j) A[i * m + j] = A[j * m + i] = (float)A64[i * m + j];
-  // B = b A + c qA qA16x1, FP32
+  // B = b A + c qA qA16x1 with qA = Q1x16(A H), qA16x1 = Q16x1(H^T A), FP32
   std::vector<double> dA((size_t)(m * m)), dA16((size_t)(m * m)), P((size_t)(m * m));
-  q1x16(A.data(), m, m, dA.data(), nullptr);
-  q16x1(A.data(), m, m, dA16.data());
+  q1x16(A.data(), m, m, o.flags, hA, dA.data(), nullptr);
+  q16x1(A.data(), m, m, o.flags, hA, dA16.data());
   product(dA.data(), dA16.data(), m, m, m, P.data());
   std::vector<float> B((size_t)(m * m));
   for (int64_t i = 0; i < m * m; ++i) B[i] = (float)(b * (double)A[i] + c * P[i]);
-  // X' = a X + qB qX16x1, FP32
+  // X' = a X + qB qX16x1 with qB = Q1x16(B H'), FP32
   std::vector<double> dB((size_t)(m * m)), U((size_t)(m * n));
-  q1x16(B.data(), m, m, dB.data(), nullptr);
+  q1x16(B.data(), m, m, o.flags, hU, dB.data(), nullptr);
   product(dB.data(), dX16.data(), m, m, n, U.data());
   for (int64_t i = 0; i < m * n; ++i) X[i] = (float)(a * (double)X[i] + U[i]);
 }
@@ -274,18 +390,32 @@ float fs4o_tensor_scale(float amax, int amax_mode) { return tensor_scale(amax, a
 
 // Q1x16 of x (rows x cols, cols % 16 == 0): packed codes (element 2j in the low
 // nibble of byte j), scale bytes, tensor scale.  s_g_in > 0 uses that tensor scale,
-// otherwise it is derived from the exact amax (amax_mode: 0 power of two,
-// 1 amax / 2688).  Returns 0, or -1 for a bad shape.
-int fs4o_quantize_rows(const float* x, int64_t rows, int64_t cols, float s_g_in, int amax_mode,
+// otherwise it is derived from the exact amax.  flags: bit 0 (1) s_g = amax / denom
+// instead of a power of two; bit 1 (2) adaptive 4/6 blocks (denom 1792, else 2688).
+// Returns 0, or -1 for a bad shape.
+int fs4o_quantize_rows(const float* x, int64_t rows, int64_t cols, float s_g_in, int flags,
                        uint8_t* codes, uint8_t* scales, float* s_g_out, int threads) {
   if (rows < 1 || cols < kBlock || cols % kBlock) return -1;
   set_threads(threads);
-  const float sg = s_g_in > 0.0f ? s_g_in : tensor_scale(amax_of(x, rows * cols), amax_mode);
+  const bool a46 = flags & kAdaptive46;
+  const float sg = s_g_in > 0.0f ? s_g_in
+                                 : tensor_scale(amax_of(x, rows * cols), flags & kAmaxMode,
+                                                a46 ? kSgDenom46 : kSgDenom);
   std::vector<uint8_t> nib((size_t)(rows * cols));
-  quantize_rows(x, rows, cols, sg, nib.data(), scales);
+  quantize_rows(x, rows, cols, sg, a46, nib.data(), scales);
   for (int64_t i = 0; i < rows * cols / 2; ++i)
     codes[i] = (uint8_t)(nib[2 * i] | (nib[2 * i + 1] << 4));
   *s_g_out = sg;
+  return 0;
+}
+
+// y = x H16^r (FP32, every 16-element block of each row; x and y rows x cols, may
+// alias), H16^r = D H16 / 4 with D from the sign mask.  Returns 0, or -1 for a bad
+// shape.
+int fs4o_hadamard_rows(const float* x, int64_t rows, int64_t cols, int mask, float* y) {
+  if (rows < 1 || cols < kBlock || cols % kBlock || mask < 0 || mask > 0xFFFF) return -1;
+  if (y != x) std::memcpy(y, x, sizeof(float) * (size_t)(rows * cols));
+  hadamard_rows(y, rows, cols, (uint16_t)mask);
   return 0;
 }
 
@@ -312,27 +442,36 @@ int fs4o_product(const double* L, const double* R, int64_t M, int64_t K, int64_t
   return 0;
 }
 
-// X_0 of an m x n FP32 matrix (already in working orientation); clip_k <= 0: no clip.
-double fs4o_normalise_and_clip(const float* G, int64_t m, int64_t n, double clip_k, float* X0,
-                               float* inv, float* tau) {
-  return normalise_and_clip(G, m, n, clip_k, X0, inv, tau);
+// X_0 of an m x n FP32 matrix (already in working orientation).  clip_quantile > 0:
+// nearest-rank quantile clip; else clip_k > 0: clip_k * RMS; else no clip.
+double fs4o_normalise_and_clip(const float* G, int64_t m, int64_t n, double clip_k,
+                               double clip_quantile, float* X0, float* inv, float* tau) {
+  return normalise_and_clip(G, m, n, clip_k, clip_quantile, X0, inv, tau);
 }
 
 // K NVFP4 iterations from an FP32 working-orientation X_0 (m <= n), in place.
+// masks: null (H = I) or 3K sign masks of H16^r; flags: as fs4o_quantize_rows,
+// applied to every quantisation.
 int fs4o_ns_iterations_nvfp4(float* X, int64_t m, int64_t n, int K, double a, double b, double c,
-                             int threads) {
+                             const uint16_t* masks, int flags, int threads) {
   if (m < 1 || n < 1 || m % kBlock || n % kBlock || K < 0) return -1;
   set_threads(threads);
-  for (int k = 0; k < K; ++k) nvfp4_iteration(X, m, n, a, b, c);
+  Opts o;
+  o.flags = flags;
+  o.masks = masks;
+  for (int k = 0; k < K; ++k) nvfp4_iteration(X, m, n, a, b, c, k, o);
   return 0;
 }
 
 // The whole step on an FP32 m0 x n0 matrix G: normalise, clip, K iterations.
-// quantized = 1: the NVFP4 route, result in out32 (m0 x n0 FP32).
+// quantized = 1: the NVFP4 route, result in out32 (m0 x n0 FP32), with the masks
+// and flags of fs4o_ns_iterations_nvfp4.
 // quantized = 0: the float64 route of Section 2 (normalisation and clip in float64),
-// result in out64.  Returns 0, or -1 for a bad shape or non-finite input.
+// result in out64.  clip_quantile > 0 replaces the clip_k * RMS clip on both routes.
+// Returns 0, or -1 for a bad shape or non-finite input.
 int fs4o_root_ns(const float* G, int64_t m0, int64_t n0, int K, double a, double b, double c,
-                 double clip_k, int quantized, float* out32, double* out64, int threads) {
+                 double clip_k, double clip_quantile, int quantized, const uint16_t* masks,
+                 int flags, float* out32, double* out64, int threads) {
   if (m0 < 1 || n0 < 1 || K < 0) return -1;
   for (int64_t i = 0; i < m0 * n0; ++i)
     if (!std::isfinite(G[i])) return -1;
@@ -345,8 +484,11 @@ int fs4o_root_ns(const float* G, int64_t m0, int64_t n0, int K, double a, double
   if (quantized) {
     if (m % kBlock || n % kBlock) return -1;
     std::vector<float> X((size_t)(m * n));
-    normalise_and_clip(W.data(), m, n, clip_k, X.data(), nullptr, nullptr);
-    for (int k = 0; k < K; ++k) nvfp4_iteration(X.data(), m, n, a, b, c);
+    normalise_and_clip(W.data(), m, n, clip_k, clip_quantile, X.data(), nullptr, nullptr);
+    Opts o;
+    o.flags = flags;
+    o.masks = masks;
+    for (int k = 0; k < K; ++k) nvfp4_iteration(X.data(), m, n, a, b, c, k, o);
     if (tall) transpose(X.data(), m, n, out32);
     else std::memcpy(out32, X.data(), sizeof(float) * (size_t)(m * n));
   } else {
@@ -355,12 +497,18 @@ int fs4o_root_ns(const float* G, int64_t m0, int64_t n0, int K, double a, double
     for (int64_t i = 0; i < m * n; ++i) s += (double)W[i] * (double)W[i];
     const double norm = std::sqrt(s);
     for (int64_t i = 0; i < m * n; ++i) X[i] = (double)W[i] / (norm + kEps);
-    if (clip_k > 0.0) {
+    double tau = -1.0;
+    if (clip_quantile > 0.0) {
+      std::vector<double> a0((size_t)(m * n));
+      for (int64_t i = 0; i < m * n; ++i) a0[i] = std::fabs(X[i]);
+      tau = kth_smallest(a0.data(), m * n, quantile_rank(clip_quantile, m * n));
+    } else if (clip_k > 0.0) {
       double s0 = 0.0;
       for (int64_t i = 0; i < m * n; ++i) s0 += X[i] * X[i];
-      const double tau = clip_k * std::sqrt(s0) / std::sqrt((double)(m * n));
-      for (int64_t i = 0; i < m * n; ++i) X[i] = X[i] > tau ? tau : (X[i] < -tau ? -tau : X[i]);
+      tau = clip_k * std::sqrt(s0) / std::sqrt((double)(m * n));
     }
+    if (tau >= 0.0)
+      for (int64_t i = 0; i < m * n; ++i) X[i] = X[i] > tau ? tau : (X[i] < -tau ? -tau : X[i]);
     for (int k = 0; k < K; ++k) f64_iteration(X.data(), m, n, a, b, c);
     for (int64_t r = 0; r < m; ++r)
       for (int64_t cc = 0; cc < n; ++cc) {

@@ -26,6 +26,10 @@ _c = ctypes
 _fp = _c.POINTER(_c.c_float)
 _dp = _c.POINTER(_c.c_double)
 _up = _c.POINTER(_c.c_uint8)
+_u16p = _c.POINTER(_c.c_uint16)
+
+AMAX_MODE = 1      # quantiser flags of the C ABI: s_g = amax / denom
+ADAPTIVE46 = 2     #                               adaptive 4/6 blocks
 
 
 def build(force: bool = False) -> str:
@@ -63,14 +67,18 @@ def lib():
         L.fs4o_dequantize_rows.argtypes = [_up, _up, _c.c_float, _c.c_int64, _c.c_int64, _dp, _c.c_int]
         L.fs4o_product.restype = _c.c_int
         L.fs4o_product.argtypes = [_dp, _dp, _c.c_int64, _c.c_int64, _c.c_int64, _dp, _c.c_int]
+        L.fs4o_hadamard_rows.restype = _c.c_int
+        L.fs4o_hadamard_rows.argtypes = [_fp, _c.c_int64, _c.c_int64, _c.c_int, _fp]
         L.fs4o_normalise_and_clip.restype = _c.c_double
-        L.fs4o_normalise_and_clip.argtypes = [_fp, _c.c_int64, _c.c_int64, _c.c_double, _fp, _fp, _fp]
+        L.fs4o_normalise_and_clip.argtypes = [_fp, _c.c_int64, _c.c_int64, _c.c_double, _c.c_double,
+                                              _fp, _fp, _fp]
         L.fs4o_ns_iterations_nvfp4.restype = _c.c_int
         L.fs4o_ns_iterations_nvfp4.argtypes = [_fp, _c.c_int64, _c.c_int64, _c.c_int, _c.c_double,
-                                               _c.c_double, _c.c_double, _c.c_int]
+                                               _c.c_double, _c.c_double, _u16p, _c.c_int, _c.c_int]
         L.fs4o_root_ns.restype = _c.c_int
         L.fs4o_root_ns.argtypes = [_fp, _c.c_int64, _c.c_int64, _c.c_int, _c.c_double, _c.c_double,
-                                   _c.c_double, _c.c_double, _c.c_int, _fp, _dp, _c.c_int]
+                                   _c.c_double, _c.c_double, _c.c_double, _c.c_int, _u16p, _c.c_int,
+                                   _fp, _dp, _c.c_int]
         _lib = L
     return _lib
 
@@ -87,19 +95,32 @@ def threads() -> int:
     return int(lib().fs4o_threads())
 
 
+def _flags(mode, adaptive46):
+    if mode not in ("pow2", "amax"):
+        raise ValueError(f"unknown tensor-scale mode {mode!r}")
+    return (AMAX_MODE if mode == "amax" else 0) | (ADAPTIVE46 if adaptive46 else 0)
+
+
+def _masks(rht_masks, K):
+    """The 3K sign masks of H16^r as a uint16 array (None: H = I)."""
+    if rht_masks is None:
+        return None
+    m = np.ascontiguousarray([int(v) for v in rht_masks], dtype=np.int64)
+    if m.size < 3 * K or np.any(m < 0) or np.any(m > 0xFFFF):
+        raise ValueError("rht_masks needs 3K masks in 0 .. 0xFFFF")
+    return m.astype(np.uint16)
+
+
 def quantize_rows(x, s_g=None, mode="pow2", adaptive46=False, threads=0):
     """Q1x16 of an FP32 matrix: (codes [rows, cols/2], scales [rows, cols/16], s_g).
-    The same signature as oracle.nvfp4.quantize_rows; adaptive 4/6 scaling is not
-    implemented here."""
-    if adaptive46:
-        raise NotImplementedError("the C++ oracle quantises with M = 6 only")
+    The same signature and result as oracle.nvfp4.quantize_rows."""
     x = _f32(x)
     rows, cols = x.shape
     codes = np.zeros((rows, cols // 2), np.uint8)
     scales = np.zeros((rows, cols // 16), np.uint8)
     sg = np.zeros(1, np.float32)
     st = lib().fs4o_quantize_rows(_ptr(x, _fp), rows, cols, float(s_g) if s_g is not None else -1.0,
-                                  1 if mode == "amax" else 0, _ptr(codes, _up), _ptr(scales, _up),
+                                  _flags(mode, adaptive46), _ptr(codes, _up), _ptr(scales, _up),
                                   _ptr(sg, _fp), threads)
     if st != 0:
         raise ValueError("bad shape")
@@ -138,33 +159,59 @@ def product(L, R, threads=0):
     return out
 
 
-def normalise_and_clip(G, clip_k):
-    """(X0, inv, tau, norm) of an FP32 matrix already in working orientation."""
+def hadamard_rows(x, mask):
+    """FP32 x H16^r on every 16-element block of each row (oracle.nvfp4.hadamard_rows)."""
+    x = _f32(x)
+    y = np.zeros_like(x)
+    if lib().fs4o_hadamard_rows(_ptr(x, _fp), x.shape[0], x.shape[1], int(mask), _ptr(y, _fp)) != 0:
+        raise ValueError("bad shape or mask")
+    return y
+
+
+def hadamard_cols(x, mask):
+    """FP32 (H16^r)^T x on every 16-element block of each column."""
+    return np.ascontiguousarray(hadamard_rows(np.ascontiguousarray(np.asarray(x, np.float32).T), mask).T)
+
+
+def normalise_and_clip(G, clip_k, clip_quantile=None):
+    """(X0, inv, tau, norm) of an FP32 matrix already in working orientation;
+    clip_quantile = q replaces the clip_k * RMS threshold by the q-quantile of |X0|."""
     G = _f32(G)
     X0 = np.zeros_like(G)
     inv = np.zeros(1, np.float32)
     tau = np.zeros(1, np.float32)
+    q = float(clip_quantile) if clip_quantile is not None else 0.0
     norm = lib().fs4o_normalise_and_clip(_ptr(G, _fp), G.shape[0], G.shape[1],
-                                         float(clip_k) if clip_k else 0.0, _ptr(X0, _fp),
+                                         float(clip_k) if clip_k else 0.0, q, _ptr(X0, _fp),
                                          _ptr(inv, _fp), _ptr(tau, _fp))
-    return X0, np.float32(inv[0]), (np.float32(tau[0]) if clip_k else None), float(norm)
+    clipped = clip_quantile is not None or bool(clip_k)
+    return X0, np.float32(inv[0]), (np.float32(tau[0]) if clipped else None), float(norm)
 
 
-def ns_iterations_nvfp4(X0, K, a, b, c, threads=0):
+def ns_iterations_nvfp4(X0, K, a, b, c, mode="pow2", rht_masks=None, adaptive46=False, threads=0):
+    """K NVFP4 iterations (oracle.root_ns.ns_iterations_nvfp4 with the same options)."""
     X = _f32(X0).copy()
+    masks = _masks(rht_masks, K)
+    mp = _ptr(masks, _u16p) if masks is not None else None
     if lib().fs4o_ns_iterations_nvfp4(_ptr(X, _fp), X.shape[0], X.shape[1], int(K), float(a), float(b),
-                                      float(c), threads) != 0:
+                                      float(c), mp, _flags(mode, adaptive46), threads) != 0:
         raise ValueError("bad shape")
     return X
 
 
-def root_ns(G, K=5, a=3.4445, b=-4.7750, c=2.0315, clip_k=3.0, quantized=True, threads=0):
-    """The whole step (normalise, clip, K iterations) on an FP32 matrix of any orientation."""
+def root_ns(G, K=5, a=3.4445, b=-4.7750, c=2.0315, clip_k=3.0, quantized=True, mode="pow2",
+            rht_masks=None, adaptive46=False, clip_quantile=None, threads=0):
+    """The whole step (normalise, clip, K iterations) on an FP32 matrix of any orientation,
+    with the options of oracle.root_ns.root_ns."""
     G = _f32(G)
     out32 = np.zeros(G.shape, np.float32)
     out64 = np.zeros(G.shape, np.float64)
+    masks = _masks(rht_masks, K) if quantized else None
+    mp = _ptr(masks, _u16p) if masks is not None else None
     st = lib().fs4o_root_ns(_ptr(G, _fp), G.shape[0], G.shape[1], int(K), float(a), float(b), float(c),
-                            float(clip_k) if clip_k else 0.0, 1 if quantized else 0, _ptr(out32, _fp),
+                            float(clip_k) if clip_k else 0.0,
+                            float(clip_quantile) if clip_quantile is not None else 0.0,
+                            1 if quantized else 0, mp, _flags(mode, adaptive46), _ptr(out32, _fp),
                             _ptr(out64, _dp), threads)
     if st != 0:
         raise ValueError("bad shape or non-finite input")

@@ -185,3 +185,170 @@ def test_numpy_iteration_with_the_cpp_codec_is_bit_identical(shape, K, coef):
     a = R.ns_iterations_nvfp4(X0, K, *coef)
     b = R.ns_iterations_nvfp4(X0, K, *coef, codec=C)
     assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+# ---------------------------------------------------------------- options of Section 3.4
+# H16^r ("a fresh 16x16 random Hadamard transform"), adaptive 4/6 block scaling and the
+# nearest-rank quantile clip ("p99 outlier clipping", Table 8 "Root quantile ratio").
+
+MASKS = [0x0000, 0x0001, 0x8000, 0xA5C3, 0x3A5C, 0xFFFF]
+
+
+def _awkward(shape, seed):
+    """Heavy-tailed values with signed zeros, an all-zero block and a few outliers."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_t(3, shape) * 0.02
+    x[rng.random(shape) < 0.02] *= 300.0
+    x[rng.random(shape) < 0.05] = -0.0
+    x[:, 16:32] = 0.0
+    return x.astype(np.float32)
+
+
+@pytest.mark.parametrize("mask", MASKS)
+def test_hadamard_bit_exact_against_the_numpy_oracle(mask):
+    x = _awkward((48, 96), 11)
+    for fc, fn in ((C.hadamard_rows, Q.hadamard_rows), (C.hadamard_cols, Q.hadamard_cols)):
+        got, want = fc(x, mask), fn(x, mask)
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+@pytest.mark.parametrize("mask", MASKS)
+def test_hadamard_matches_the_matrix_definition(mask):
+    """y = x D H16 / 4 from the Sylvester matrix: each FP32 output is four levels of
+    additions of the block's 16 inputs, so it lies within 4 * 2^-24 * sum|x_block|
+    (before the exact / 4) of the float64 value.  A block of unit vectors gives
+    the rows of D H16 / 4 exactly."""
+    x = _awkward((24, 64), 12)
+    got = C.hadamard_rows(x, mask).astype(np.float64)
+    want = Q.hadamard_rows_f64(x, mask)
+    bound = 4 * 2.0 ** -24 * np.abs(x.astype(np.float64)).reshape(24, 4, 16).sum(axis=2) / 4
+    assert np.all(np.abs(got - want).reshape(24, 4, 16) <= bound[:, :, None] + 1e-45)
+    eye = np.eye(16, dtype=np.float32)
+    Hr = np.diag(Q.mask_signs(mask)) @ Q.sylvester16() / 4.0
+    assert np.array_equal(C.hadamard_rows(eye, mask).astype(np.float64), Hr)
+
+
+def test_hadamard_refuses_a_bad_mask_or_shape():
+    with pytest.raises(ValueError):
+        C.hadamard_rows(np.zeros((2, 24), np.float32), 0)
+    with pytest.raises(ValueError):
+        C.hadamard_rows(np.zeros((2, 16), np.float32), 0x10000)
+
+
+def test_adaptive46_hand_worked_blocks(golden_dir):
+    with open(os.path.join(golden_dir, "adaptive46_blocks.json")) as f:
+        data = json.load(f)
+    for case in data["cases"]:
+        x = np.array(case["x"], dtype=np.float32).reshape(1, -1)
+        codes, scales, sg = C.quantize_rows(x, s_g=case["s_g"], adaptive46=True)
+        assert scales.tobytes().hex() == "".join(case["scales_hex"]), case["name"]
+        assert codes.tobytes().hex() == "".join(case["codes_hex"]), case["name"]
+
+
+@pytest.mark.parametrize("kind", ["gauss", "awkward", "half_steps", "tiny"])
+@pytest.mark.parametrize("mode", ["pow2", "amax"])
+def test_quantise_adaptive46_bit_exact_against_the_numpy_oracle(kind, mode):
+    rng = np.random.default_rng(13)
+    if kind == "gauss":
+        x = (rng.standard_normal((48, 192)) * rng.lognormal(0, 1, (48, 1))).astype(np.float32)
+    elif kind == "awkward":
+        x = _awkward((48, 192), 14)
+    elif kind == "half_steps":       # many blocks that one of the candidates holds exactly
+        x = (np.round(rng.standard_normal((48, 192)) * 4) / 2).astype(np.float32)
+    else:
+        x = (rng.standard_normal((48, 192)) * 1e-30).astype(np.float32)
+    for fc, fn in ((C.quantize_rows, Q.quantize_rows), (C.quantize_cols, Q.quantize_cols)):
+        c1, s1, g1 = fc(x, mode=mode, adaptive46=True)
+        c2, s2, g2 = fn(x, mode=mode, adaptive46=True)
+        assert g1 == g2 and np.array_equal(s1, s2) and np.array_equal(c1, c2)
+    # 4/6 changes some blocks, and keeps M = 6 on others
+    _, s46, g46 = C.quantize_rows(x, mode=mode, adaptive46=True)
+    _, s6, _ = C.quantize_rows(x, s_g=g46, mode=mode)
+    if kind != "tiny":
+        assert np.any(s6 != s46) and np.any(s6 == s46)
+
+
+def test_quantile_clip_hand_worked_vector():
+    # |G| = {5, 1, 3, 2, 4}; q = 0.5 -> rank 3 -> tau = fp32(3 inv); -5 and 4 clamp to -+tau
+    G = np.array([[-5.0, 1.0, 3.0, -2.0, 4.0]], np.float32)
+    X0, inv, tau, norm = C.normalise_and_clip(G, None, clip_quantile=0.5)
+    assert norm == pytest.approx(np.sqrt(55.0), rel=1e-15)
+    assert tau == np.float32(3.0) * inv
+    assert np.array_equal(X0, np.array([[-tau, 1.0 * inv, tau, -2.0 * inv, tau]], np.float32))
+
+
+@pytest.mark.parametrize("q", [0.99, 0.5, 0.999, 1.0, 1e-9])
+def test_quantile_clip_matches_the_numpy_oracle(q):
+    G = _awkward((64, 96), 15)
+    X1, inv1, tau1, n1 = C.normalise_and_clip(G, 3.0, clip_quantile=q)   # the quantile wins
+    X2, inv2, tau2, n2 = R.normalise_and_clip(G, 3.0, clip_quantile=q)
+    assert inv1 == inv2 and tau1 == tau2 and abs(n1 - n2) <= 1e-12 * n2
+    assert np.array_equal(X1.view(np.uint32), X2.view(np.uint32))
+
+
+OPTIONS = [dict(), dict(adaptive46=True), dict(rht=True), dict(rht=True, adaptive46=True),
+           dict(rht=True, adaptive46=True, mode="amax")]
+
+
+def _opts(o, K, seed):
+    o = dict(o)
+    masks = None
+    if o.pop("rht", False):
+        masks = [int(v) for v in np.random.default_rng(seed).integers(0, 1 << 16, 3 * K)]
+    return dict(o, rht_masks=masks)
+
+
+@pytest.mark.parametrize("opts", OPTIONS, ids=lambda o: "+".join(sorted(o)) or "plain")
+@pytest.mark.parametrize("shape,K,coef", [((48, 112), 3, MUON), ((32, 32), 2, QUINTIC)])
+def test_iteration_options_bit_identical_to_the_numpy_steps(opts, shape, K, coef):
+    """The numpy iteration with its own codec, H16^r and 4/6 and the C++ product in
+    place of BLAS (so that both sum every product in k order) gives the C++
+    iteration's FP32 iterate bit for bit: every quantisation, transform, mask
+    index and combine agrees."""
+    rng = np.random.default_rng(16)
+    X0 = R.normalise_and_clip((rng.standard_t(4, shape) * 0.02).astype(np.float32), 3.0)[0]
+    o = _opts(opts, K, 17)
+    got = C.ns_iterations_nvfp4(X0, K, *coef, **o)
+    want = R.ns_iterations_nvfp4(X0, K, *coef, matmul=C.product, **o)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+@pytest.mark.parametrize("opts", OPTIONS[1:4], ids=lambda o: "+".join(sorted(o)))
+@pytest.mark.parametrize("shape", [(64, 160), (160, 64)])
+def test_root_ns_options_match_the_numpy_oracle(opts, shape):
+    """The whole step with each option (and the 0.99 quantile clip) against the numpy
+    oracle with BLAS products: equal up to float64 summation order."""
+    K = 3
+    rng = np.random.default_rng(18)
+    G = (rng.standard_t(3, shape) * 0.02).astype(np.float32)
+    o = _opts(opts, K, 19)
+    for clip in (dict(clip_k=3.0), dict(clip_k=None, clip_quantile=0.99)):
+        got = C.root_ns(G, K, *MUON, **clip, **o)
+        want = R.root_ns(G, K, *MUON, **clip, **o)
+        assert got.shape == want.shape
+        assert np.linalg.norm(got - want) <= 1e-6 * np.linalg.norm(want)
+
+
+def test_float64_route_quantile_clip_matches_the_numpy_oracle():
+    """Both float64 routes with the 0.99 quantile clip agree; q = 1 clips nothing, so
+    that route equals the unclipped one, whose closed form is pinned above."""
+    rng = np.random.default_rng(20)
+    G = (rng.standard_t(3, (48, 80)) * 0.02).astype(np.float32)
+    for impl in (C, R):
+        got = impl.root_ns(G, 3, *MUON, clip_k=None, clip_quantile=0.99, quantized=False)
+        assert np.all(np.isfinite(got)) and got.shape == G.shape
+        q1 = impl.root_ns(G, 3, *MUON, clip_k=None, clip_quantile=1.0, quantized=False)
+        none = impl.root_ns(G, 3, *MUON, clip_k=None, quantized=False)
+        assert np.array_equal(q1, none)
+    got = C.root_ns(G, 3, *MUON, clip_k=None, clip_quantile=0.99, quantized=False)
+    want = R.root_ns(G, 3, *MUON, clip_k=None, clip_quantile=0.99, quantized=False)
+    assert np.linalg.norm(got - want) <= 1e-12 * np.linalg.norm(want)
+    assert np.linalg.norm(got - C.root_ns(G, 3, *MUON, clip_k=None, quantized=False)) > 0
+
+
+def test_too_few_masks_are_refused():
+    X0 = np.zeros((16, 16), np.float32)
+    with pytest.raises(ValueError):
+        C.ns_iterations_nvfp4(X0, 2, *MUON, rht_masks=[1, 2, 3, 4, 5])
+    with pytest.raises(ValueError):
+        C.root_ns(X0, 1, *MUON, rht_masks=[1, 2, 0x10000])
