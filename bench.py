@@ -70,6 +70,11 @@ def parse_args():
     ap.add_argument("--quant", default="plain", choices=["plain", "rht46", "rht", "a46"],
                     help="quantiser of the step: plain NVFP4 (default) or the Section 3.4 options "
                          "(random Hadamard transform with fresh seeded sign masks, adaptive 4/6)")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "lpt"],
+                    help="ns across ranks: replicas (default; every rank runs the whole workload on "
+                         "its own matrices, weak scaling, no collective) or lpt (one model's matrices "
+                         "split by longest processing time over the algorithmic FLOPs, one NCCL "
+                         "all-gather of the updates, strong scaling)")
     return ap.parse_args()
 
 
@@ -456,6 +461,11 @@ def main():
         if world > 1:
             dist.destroy_process_group()
         return
+    if args.shard == "lpt":
+        run_sharded(args, w, rank, world, local, barrier, ranks_max)
+        if world > 1:
+            dist.destroy_process_group()
+        return
     K = w.K
     Gs = matrices(w, device="cuda", seed=rank_seed(BASE_SEED, rank))
     outs = [torch.empty_like(G) for G in Gs]
@@ -751,6 +761,92 @@ def main():
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def run_sharded(args, w, rank, world, local, barrier, ranks_max):
+    """--shard lpt: one model's matrices split across the ranks (longest processing time
+    first over the algorithmic FLOPs; nvfp4_precision_optimizer_b200.shard).  Each rank runs
+    the step (fs4_root_ns_batched) on its share, then one NCCL all-gather returns every
+    update to every rank.  A step is both; its time is the maximum over ranks of the CUDA
+    events around them, and the value is the model's matrices over that time.  The total
+    work is fixed as N grows ("scaling": "strong").  The plain step on FP32 momenta only."""
+    import torch
+
+    import nvfp4_precision_optimizer_b200 as F
+    from nvfp4_precision_optimizer_b200 import shard
+    from nvfp4_precision_optimizer_b200.workloads import BASE_SEED, generate
+    if args.quant != "plain" or args.clip != "rms" or args.source != "fp32" or args.graph:
+        raise SystemExit("--shard lpt runs the plain step on FP32 momenta "
+                         "(no --quant, --clip, --source or --graph)")
+    K = w.K
+    S = shard.ShardedRootNS(w.shapes, K=K, coeffs=w.coeffs, rank=rank, world=world, device="cuda",
+                            clip_k=w.clip_k)
+    mine = set(S.local)
+    # one model on every rank: matrix i is seeded with BASE_SEED + i everywhere; a rank
+    # holds only the momenta it owns
+    Gs = [generate(s, w.dist, BASE_SEED + i, "cuda") if i in mine else None
+          for i, s in enumerate(w.shapes)]
+    stream = torch.cuda.current_stream()
+
+    def status(what):
+        if S.workspace is not None:
+            F.check(F.device_status(S.workspace), what)
+
+    for _ in range(max(3, args.warmup)):
+        S(Gs)
+    torch.cuda.synchronize()
+    status("device status after warm-up")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for evs in ev:                   # torch creates the CUDA event on its first record
+        for e in evs:
+            e.record(stream)
+    in_bytes = sum(G.numel() * 4 for G in Gs if G is not None)
+    l2_bytes = int(torch.cuda.get_device_properties(local).L2_cache_size)
+    flush = torch.empty(2 * l2_bytes, dtype=torch.uint8, device="cuda") if in_bytes <= 2 * l2_bytes else None
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    with sampler:
+        time.sleep(0.3)
+        for s in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            ev[s][0].record(stream)
+            S.compute_local(Gs)
+            ev[s][1].record(stream)
+            S.gather()
+            ev[s][2].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    status("device status after timed steps")
+    ms_step = ranks_max(sum(e[0].elapsed_time(e[2]) for e in ev)) / args.steps
+    ns_ms = ranks_max(statistics.mean(e[0].elapsed_time(e[1]) for e in ev))
+    ag_ms = ranks_max(statistics.mean(e[1].elapsed_time(e[2]) for e in ev))
+    n = len(w.shapes)
+    value = n / (ms_step * 1e-3)
+    gathered = world * S.plan.chunk * 4 if world > 1 else 0
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None,
+            "dtype": "nvfp4 (e2m1 x e4m3/16) products, fp32 accumulate", "data": "synthetic",
+            "config": {**ns_config(w, args.quant, args.clip, world),
+                       "parallelism": (f"lpt x{world}: the model's {n} matrices split by longest "
+                                       f"processing time over algorithmic FLOPs, one NCCL all-gather "
+                                       f"of the updates" if world > 1 else "one GPU, no collective"),
+                       "load_imbalance": S.plan.imbalance,
+                       "l2": ("inputs larger than L2 (%.2f GB per rank per step)" % (in_bytes / 1e9)
+                              if flush is None else "L2 flushed before every step")},
+            "split_ms": {"share_step_max_over_ranks": ns_ms, "all_gather_max_over_ranks": ag_ms},
+            "all_gather_recv_bytes_per_rank": gathered,
+            "tflops_algorithmic": w.flops_algorithmic() / (ms_step * 1e-3) / 1e12,
+            "roofline": None, "cpu_baseline": None, "e2e": None,
+            "note": "per-phase roofline, CPU baseline and end-to-end figures come from the default mode",
+            "gpu_launches": args.steps * (2 + 6 * K) if S.local else 0,
+            "clocks": sampler.summary(),
+        }
+        print(json.dumps(line), flush=True)
 
 
 def run_standalone(args, w, rank, world, local, barrier, ranks_max):
