@@ -10,10 +10,14 @@ decoder (196 matrices: per block Q/K/V/O 3072x3072, gate/up 8192x3072, down
 per matrix, K = 5, one batched call; the largest workload that fits one GPU.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                  [--shard replicas|lpt]
 
 Multi-GPU (torchrun): every rank runs the whole workload on its own GPU (the
 matrices are independent; no collective on the data path), so per-GPU work is
-fixed and the scaling is weak; the step time is the max over ranks.
+fixed and the scaling is weak; the step time is the max over ranks.  With
+--shard lpt the ranks instead split one workload (longest processing time first
+over the algorithmic FLOPs) and one NCCL all-gather returns every update to every
+rank: strong scaling.
 """
 from __future__ import annotations
 
