@@ -1069,30 +1069,31 @@ def run_standalone(args, w, rank, world, local, barrier, ranks_max):
 
 
 def oracle_momentum_rate(w, budget_s: float):
-    """Time the oracle's momentum step (with a previous state) on leading rows of the
-    workload's first matrix.  Returns (algorithmic GB/s, seconds, description)."""
-    from oracle import momentum as M
+    """Time the C++ oracle's momentum step (with a previous state) on leading rows of the
+    workload's first matrix.  Returns (algorithmic GB/s, seconds, description, cores)."""
+    from oracle import cpp_oracle as C
     from nvfp4_precision_optimizer_b200.workloads import BASE_SEED, generate
     G = generate(w.shapes[0], w.dist, BASE_SEED, "cpu").numpy()
     rows = 16
     while True:
         g = G[:rows]
-        _, state = M.update(g, 0.95, None, 0, 0x5A5A, 1)
+        _, state = C.momentum_update(g, 0.95, None, 0, 0x5A5A, 1)
         t0 = time.perf_counter()
-        M.update(g, 0.95, state, 0x5A5A, 0xC3C3, 2)
+        C.momentum_update(g, 0.95, state, 0x5A5A, 0xC3C3, 2)
         dt = time.perf_counter() - t0
         if dt >= budget_s / 4 or rows >= G.shape[0]:
             break
         rows = min(G.shape[0], rows * 4)
-    desc = (f"oracle momentum step (numpy, exact emulation) of the first {rows} rows of a "
-            f"{G.shape[0]}x{G.shape[1]} workload matrix, {dt:.2f} s")
-    return g.size * MO_BYTES / dt / 1e9, dt, desc
+    cores = C.threads()
+    desc = (f"C++ oracle momentum step (exact emulation; OpenMP over rows) of the first {rows} rows "
+            f"of a {G.shape[0]}x{G.shape[1]} workload matrix, {dt:.2f} s on {cores} threads")
+    return g.size * MO_BYTES / dt / 1e9, dt, desc, cores
 
 
 def run_momentum_reference(args, w):
-    rates, desc = [], ""
+    rates, desc, cores = [], "", 1
     for i in range(args.warmup + args.steps):
-        rate, dt, desc = oracle_momentum_rate(w, max(2.0, 120.0 / max(1, args.steps + args.warmup)))
+        rate, dt, desc, cores = oracle_momentum_rate(w, max(2.0, 120.0 / max(1, args.steps + args.warmup)))
         if i >= args.warmup:
             rates.append(rate)
     value = statistics.median(rates)
@@ -1103,7 +1104,7 @@ def run_momentum_reference(args, w):
         "ms_per_step": 1000.0 * total / (value * 1e9), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32 values, exact NVFP4 emulation", "data": "synthetic",
         "config": {"workload": w.name, "matrices": len(w.shapes), "op": "momentum"},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
@@ -1235,8 +1236,8 @@ def run_momentum(args, w, rank, world, local, barrier, ranks_max):
         F.check(F.device_status(b["ws"]), "device status after the timed steps")
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, dt, desc = oracle_momentum_rate(w, 20.0)
-        cpu = {"value": rate, "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle", "sample": desc}
+        rate, dt, desc, cores = oracle_momentum_rate(w, 20.0)
+        cpu = {"value": rate, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps({
             "metric": MO_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,

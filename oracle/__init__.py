@@ -25,7 +25,8 @@ Modules:
   * ``oracle.cpp_oracle`` -- ctypes binding of ``oracle/cpp/fs4_oracle.cpp``, the
                           same steps restated in plain C++17 (OpenMP over rows,
                           float64 triple loops, no BLAS), options included
-                          (H16^r, adaptive 4/6, quantile clip); a second,
+                          (H16^r, adaptive 4/6, quantile clip), with the BF16
+                          route and the NVFP4 first moment; a second,
                           independent implementation, and the one the CPU
                           baseline times.
 """

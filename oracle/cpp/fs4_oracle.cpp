@@ -46,6 +46,24 @@
 //   * Quantile clip ("p99 outlier clipping", Table 8 "Root quantile ratio 0.99"):
 //     tau is the k-th smallest |fp32(G inv)|, k = ceil(fl64(fp32(q)) N) clamped to
 //     [1, N] (the nearest-rank quantile), in place of clip_k * RMS.
+//
+// The BF16 route (the optimized BF16 baseline of Section 4.4 and Table 6): the same
+// plan with bf16() in place of every quantisation, bf16() = round to nearest, ties
+// to even, of the low 16 bits of the FP32 word.
+//
+// The NVFP4 first moment (Section 3.3 "Quantized-State AdamW", which Section 3.4's
+// momentum follows: Hadamard mixing, stochastic rounding, adaptive 4/6):
+//   * m_t = fp32(fp32(beta m_prev) + fp32(fp32(1 - beta) g)), m_prev the decoded
+//     previous state (zero on the first step);
+//   * state = Q(m_t H16^r) in 1x16 row blocks with 4/6 block scales (s_g by the 1792
+//     rule), every element code rounded stochastically: v = fp32(|y| / den) below 6
+//     goes to the upper of its two neighbouring E2M1 magnitudes when u < fp32((v - lo)
+//     / (hi - lo)), else to the lower; v >= 6 gives 6; both 4/6 candidates use the
+//     same u;
+//   * u of element i (row-major) = top 24 bits of SplitMix64 (Steele, Lea and Flood,
+//     OOPSLA 2014) at counter i + 1 from the seed, times 2^-24;
+//   * decode: fp32(fp32(code s_b) s_g), then (H16^r)^-1 = H16 D / 4 (the butterfly,
+//     the exact * 0.25, then the signs).
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -131,7 +149,19 @@ struct Block {
   float deq[kBlock];
 };
 
-Block quantize_block(const float* xb, float s_g, float M) {
+// Stochastic rounding of FP32 v >= 0 onto an E2M1 magnitude code with FP32 u in
+// [0, 1): lo = the largest magnitude <= v, hi the next; up when u < (v - lo) / (hi - lo).
+int e2m1_encode_sr(float v, float u) {
+  if (v >= 6.0f) return 7;
+  int lo = 0;
+  while (lo < 7 && kE2m1Mag[lo + 1] <= (double)v) ++lo;
+  const float gap = (float)(kE2m1Mag[lo + 1] - kE2m1Mag[lo]);
+  const float frac = (v - (float)kE2m1Mag[lo]) / gap;
+  return u < frac ? lo + 1 : lo;
+}
+
+// u: null for round to nearest, else the block's 16 stochastic-rounding draws.
+Block quantize_block(const float* xb, float s_g, float M, const float* u = nullptr) {
   Block q;
   float amax = 0.0f;
   for (int i = 0; i < kBlock; ++i) amax = std::fmax(amax, std::fabs(xb[i]));
@@ -142,7 +172,8 @@ Block quantize_block(const float* xb, float s_g, float M) {
     uint8_t code = 0;
     if (den > 0.0f) {
       const float r = std::fabs(xb[i]) / den;
-      code = (uint8_t)(e2m1_encode((double)r) | (std::signbit(xb[i]) ? 8 : 0));
+      const int mag = u ? e2m1_encode_sr(r, u[i]) : e2m1_encode((double)r);
+      code = (uint8_t)(mag | (std::signbit(xb[i]) ? 8 : 0));
     }
     q.code[i] = code;
     q.deq[i] = (float)(e2m1_value(code) * (double)den);
@@ -348,6 +379,98 @@ void nvfp4_iteration(float* X, int64_t m, int64_t n, double a, double b, double 
   for (int64_t i = 0; i < m * n; ++i) X[i] = (float)(a * (double)X[i] + U[i]);
 }
 
+// FP32 -> BF16 (round to nearest, ties to even, on the low 16 bits), returned as the
+// FP32 number that BF16 value is.  Finite inputs.
+float bf16_round(float x) {
+  uint32_t bits;
+  std::memcpy(&bits, &x, 4);
+  const uint32_t keep = bits >> 16, rest = bits & 0xFFFFu;
+  const uint32_t up = (rest > 0x8000u || (rest == 0x8000u && (keep & 1u))) ? 1u : 0u;
+  bits = (keep + up) << 16;
+  float y;
+  std::memcpy(&y, &bits, 4);
+  return y;
+}
+
+// One BF16 Newton-Schulz iteration on the FP32 m x n X (m <= n), in place:
+// Xb = bf16(X), A = Xb Xb^T, B = b A + c bf16(A) bf16(A)^T, X' = a X + bf16(B) Xb.
+void bf16_iteration(float* X, int64_t m, int64_t n, double a, double b, double c) {
+  std::vector<double> Xb((size_t)(m * n)), Xbt((size_t)(m * n));
+  for (int64_t r = 0; r < m; ++r)
+    for (int64_t k = 0; k < n; ++k) {
+      Xb[r * n + k] = (double)bf16_round(X[r * n + k]);
+      Xbt[k * m + r] = Xb[r * n + k];
+    }
+  std::vector<double> A64((size_t)(m * m));
+  product(Xb.data(), Xbt.data(), m, n, m, A64.data());
+  std::vector<float> A((size_t)(m * m));
+  for (int64_t i = 0; i < m; ++i)
+    for (int64_t j = i; j < m; ++j) A[i * m + j] = A[j * m + i] = (float)A64[i * m + j];
+  std::vector<double> Ab((size_t)(m * m)), Abt((size_t)(m * m)), P((size_t)(m * m));
+  for (int64_t i = 0; i < m; ++i)
+    for (int64_t j = 0; j < m; ++j) {
+      Ab[i * m + j] = (double)bf16_round(A[i * m + j]);
+      Abt[j * m + i] = Ab[i * m + j];
+    }
+  product(Ab.data(), Abt.data(), m, m, m, P.data());
+  std::vector<double> Bb((size_t)(m * m)), U((size_t)(m * n));
+  for (int64_t i = 0; i < m * m; ++i)
+    Bb[i] = (double)bf16_round((float)(b * (double)A[i] + c * P[i]));
+  product(Bb.data(), Xb.data(), m, m, n, U.data());
+  for (int64_t i = 0; i < m * n; ++i) X[i] = (float)(a * (double)X[i] + U[i]);
+}
+
+// SplitMix64 output at counter idx + 1 from seed (Steele, Lea and Flood, OOPSLA 2014).
+uint64_t splitmix64(uint64_t seed, uint64_t idx) {
+  uint64_t z = seed + (idx + 1) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// FP32 u in [0, 1): the top 24 bits of splitmix64 times 2^-24 (exact).
+float uniform24(uint64_t seed, uint64_t idx) {
+  return (float)std::ldexp((double)(splitmix64(seed, idx) >> 40), -24);
+}
+
+// NVFP4 state of the FP32 rows x cols momentum m_t: Q(m_t H16^r) with stochastically
+// rounded element codes and adaptive 4/6 block scales (1x16 row blocks, unpacked codes).
+void store_state(const float* m_t, int64_t rows, int64_t cols, uint16_t mask, uint64_t seed,
+                 uint8_t* nib, uint8_t* scales, float* s_g_out) {
+  std::vector<float> y(m_t, m_t + rows * cols);
+  hadamard_rows(y.data(), rows, cols, mask);
+  const float sg = tensor_scale(amax_of(y.data(), rows * cols), 0, kSgDenom46);
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t jb = 0; jb < cols / kBlock; ++jb) {
+      const float* xb = y.data() + r * cols + jb * kBlock;
+      float u[kBlock];
+      for (int i = 0; i < kBlock; ++i) u[i] = uniform24(seed, (uint64_t)(r * cols + jb * kBlock + i));
+      Block q = quantize_block(xb, sg, 6.0f, u);
+      const Block q4 = quantize_block(xb, sg, 4.0f, u);
+      if (block_sq_error(xb, q4) < block_sq_error(xb, q)) q = q4;
+      scales[r * (cols / kBlock) + jb] = (uint8_t)q.scale;
+      for (int i = 0; i < kBlock; ++i) nib[r * cols + jb * kBlock + i] = q.code[i];
+    }
+  }
+  *s_g_out = sg;
+}
+
+// FP32 momentum decoded from a state: fp32(fp32(code s_b) s_g), then (H16^r)^-1.
+void load_state(const uint8_t* nib, const uint8_t* scales, float s_g, uint16_t mask, int64_t rows,
+                int64_t cols, float* out) {
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t c = 0; c < cols; ++c) {
+      const float cs = (float)(e2m1_value(nib[r * cols + c]) *
+                               e4m3_value(scales[r * (cols / kBlock) + c / kBlock]));   // exact
+      out[r * cols + c] = cs * s_g;
+    }
+  hadamard_rows(out, rows, cols, 0);   // the butterfly and * 0.25, no signs
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t c = 0; c < cols; ++c)
+      if ((mask >> (c % kBlock)) & 1) out[r * cols + c] = -out[r * cols + c];
+}
+
 // One float64 Newton-Schulz iteration (Section 2), in place.
 void f64_iteration(double* X, int64_t m, int64_t n, double a, double b, double c) {
   std::vector<double> Xt((size_t)(m * n)), A((size_t)(m * m)), A2((size_t)(m * m)),
@@ -465,7 +588,8 @@ int fs4o_ns_iterations_nvfp4(float* X, int64_t m, int64_t n, int K, double a, do
 
 // The whole step on an FP32 m0 x n0 matrix G: normalise, clip, K iterations.
 // quantized = 1: the NVFP4 route, result in out32 (m0 x n0 FP32), with the masks
-// and flags of fs4o_ns_iterations_nvfp4.
+// and flags of fs4o_ns_iterations_nvfp4.  quantized = 2: the BF16 route (masks and
+// flags ignored), result in out32.
 // quantized = 0: the float64 route of Section 2 (normalisation and clip in float64),
 // result in out64.  clip_quantile > 0 replaces the clip_k * RMS clip on both routes.
 // Returns 0, or -1 for a bad shape or non-finite input.
@@ -488,7 +612,10 @@ int fs4o_root_ns(const float* G, int64_t m0, int64_t n0, int K, double a, double
     Opts o;
     o.flags = flags;
     o.masks = masks;
-    for (int k = 0; k < K; ++k) nvfp4_iteration(X.data(), m, n, a, b, c, k, o);
+    for (int k = 0; k < K; ++k) {
+      if (quantized == 2) bf16_iteration(X.data(), m, n, a, b, c);
+      else nvfp4_iteration(X.data(), m, n, a, b, c, k, o);
+    }
     if (tall) transpose(X.data(), m, n, out32);
     else std::memcpy(out32, X.data(), sizeof(float) * (size_t)(m * n));
   } else {
@@ -517,6 +644,78 @@ int fs4o_root_ns(const float* G, int64_t m0, int64_t n0, int K, double a, double
         else out64[r * n + cc] = v;
       }
   }
+  return 0;
+}
+
+// FP32 -> BF16 -> FP32 of n values (round to nearest, ties to even).
+void fs4o_bf16_round(const float* x, int64_t n, float* y) {
+  for (int64_t i = 0; i < n; ++i) y[i] = bf16_round(x[i]);
+}
+
+// K BF16 iterations from an FP32 working-orientation X_0 (m <= n), in place.
+int fs4o_ns_iterations_bf16(float* X, int64_t m, int64_t n, int K, double a, double b, double c,
+                            int threads) {
+  if (m < 1 || n < 1 || K < 0) return -1;
+  set_threads(threads);
+  for (int k = 0; k < K; ++k) bf16_iteration(X, m, n, a, b, c);
+  return 0;
+}
+
+// SplitMix64 outputs at counters idx[0 .. count) + 1, and the u24 draws.
+void fs4o_splitmix64(uint64_t seed, const uint64_t* idx, int64_t count, uint64_t* out) {
+  for (int64_t i = 0; i < count; ++i) out[i] = splitmix64(seed, idx[i]);
+}
+void fs4o_uniform24(uint64_t seed, const uint64_t* idx, int64_t count, float* out) {
+  for (int64_t i = 0; i < count; ++i) out[i] = uniform24(seed, idx[i]);
+}
+
+// Stochastic rounding of FP32 v >= 0 (finite) onto an E2M1 magnitude code 0..7.
+int fs4o_e2m1_encode_sr(float v, float u) { return e2m1_encode_sr(v, u); }
+
+// One NVFP4 first-moment step on a rows x cols FP32 gradient g (cols % 16 == 0):
+// m_t (FP32) and the new state (packed codes, scale bytes, s_g).  The previous state is
+// given by prev_codes / prev_scales / prev_sg with sign mask mask_prev, or
+// prev_codes = null for a zero previous moment.  Returns 0, or -1 for a bad shape.
+int fs4o_momentum_update(const float* g, int64_t rows, int64_t cols, double beta,
+                         const uint8_t* prev_codes, const uint8_t* prev_scales, float prev_sg,
+                         int mask_prev, int mask_next, uint64_t seed, float* m_t, uint8_t* codes,
+                         uint8_t* scales, float* s_g, int threads) {
+  if (rows < 1 || cols < kBlock || cols % kBlock) return -1;
+  if (mask_prev < 0 || mask_prev > 0xFFFF || mask_next < 0 || mask_next > 0xFFFF) return -1;
+  set_threads(threads);
+  std::vector<float> mp((size_t)(rows * cols), 0.0f);
+  if (prev_codes) {
+    std::vector<uint8_t> nib((size_t)(rows * cols));
+    for (int64_t i = 0; i < rows * cols / 2; ++i) {
+      nib[2 * i] = prev_codes[i] & 0xF;
+      nib[2 * i + 1] = prev_codes[i] >> 4;
+    }
+    load_state(nib.data(), prev_scales, prev_sg, (uint16_t)mask_prev, rows, cols, mp.data());
+  }
+  const float b = (float)beta;
+  const float omb = 1.0f - b;
+  for (int64_t i = 0; i < rows * cols; ++i) {
+    const float t1 = b * mp[i];
+    const float t2 = omb * g[i];
+    m_t[i] = t1 + t2;
+  }
+  std::vector<uint8_t> nib((size_t)(rows * cols));
+  store_state(m_t, rows, cols, (uint16_t)mask_next, seed, nib.data(), scales, s_g);
+  for (int64_t i = 0; i < rows * cols / 2; ++i)
+    codes[i] = (uint8_t)(nib[2 * i] | (nib[2 * i + 1] << 4));
+  return 0;
+}
+
+// FP32 momentum decoded from a state (packed codes).
+int fs4o_momentum_load(const uint8_t* codes, const uint8_t* scales, float s_g, int mask,
+                       int64_t rows, int64_t cols, float* out) {
+  if (rows < 1 || cols < kBlock || cols % kBlock || mask < 0 || mask > 0xFFFF) return -1;
+  std::vector<uint8_t> nib((size_t)(rows * cols));
+  for (int64_t i = 0; i < rows * cols / 2; ++i) {
+    nib[2 * i] = codes[i] & 0xF;
+    nib[2 * i + 1] = codes[i] >> 4;
+  }
+  load_state(nib.data(), scales, s_g, (uint16_t)mask, rows, cols, out);
   return 0;
 }
 

@@ -27,6 +27,7 @@ _fp = _c.POINTER(_c.c_float)
 _dp = _c.POINTER(_c.c_double)
 _up = _c.POINTER(_c.c_uint8)
 _u16p = _c.POINTER(_c.c_uint16)
+_u64p = _c.POINTER(_c.c_uint64)
 
 AMAX_MODE = 1      # quantiser flags of the C ABI: s_g = amax / denom
 ADAPTIVE46 = 2     #                               adaptive 4/6 blocks
@@ -75,6 +76,22 @@ def lib():
         L.fs4o_ns_iterations_nvfp4.restype = _c.c_int
         L.fs4o_ns_iterations_nvfp4.argtypes = [_fp, _c.c_int64, _c.c_int64, _c.c_int, _c.c_double,
                                                _c.c_double, _c.c_double, _u16p, _c.c_int, _c.c_int]
+        L.fs4o_bf16_round.restype = None
+        L.fs4o_bf16_round.argtypes = [_fp, _c.c_int64, _fp]
+        L.fs4o_ns_iterations_bf16.restype = _c.c_int
+        L.fs4o_ns_iterations_bf16.argtypes = [_fp, _c.c_int64, _c.c_int64, _c.c_int, _c.c_double,
+                                              _c.c_double, _c.c_double, _c.c_int]
+        L.fs4o_splitmix64.restype = None
+        L.fs4o_splitmix64.argtypes = [_c.c_uint64, _u64p, _c.c_int64, _u64p]
+        L.fs4o_uniform24.restype = None
+        L.fs4o_uniform24.argtypes = [_c.c_uint64, _u64p, _c.c_int64, _fp]
+        L.fs4o_e2m1_encode_sr.restype = _c.c_int
+        L.fs4o_e2m1_encode_sr.argtypes = [_c.c_float, _c.c_float]
+        L.fs4o_momentum_update.restype = _c.c_int
+        L.fs4o_momentum_update.argtypes = [_fp, _c.c_int64, _c.c_int64, _c.c_double, _up, _up, _c.c_float,
+                                           _c.c_int, _c.c_int, _c.c_uint64, _fp, _up, _up, _fp, _c.c_int]
+        L.fs4o_momentum_load.restype = _c.c_int
+        L.fs4o_momentum_load.argtypes = [_up, _up, _c.c_float, _c.c_int, _c.c_int64, _c.c_int64, _fp]
         L.fs4o_root_ns.restype = _c.c_int
         L.fs4o_root_ns.argtypes = [_fp, _c.c_int64, _c.c_int64, _c.c_int, _c.c_double, _c.c_double,
                                    _c.c_double, _c.c_double, _c.c_double, _c.c_int, _u16p, _c.c_int,
@@ -200,19 +217,94 @@ def ns_iterations_nvfp4(X0, K, a, b, c, mode="pow2", rht_masks=None, adaptive46=
 
 
 def root_ns(G, K=5, a=3.4445, b=-4.7750, c=2.0315, clip_k=3.0, quantized=True, mode="pow2",
-            rht_masks=None, adaptive46=False, clip_quantile=None, threads=0):
+            rht_masks=None, adaptive46=False, clip_quantile=None, bf16=False, threads=0):
     """The whole step (normalise, clip, K iterations) on an FP32 matrix of any orientation,
-    with the options of oracle.root_ns.root_ns."""
+    with the options of oracle.root_ns.root_ns (bf16=True: the BF16 route)."""
     G = _f32(G)
     out32 = np.zeros(G.shape, np.float32)
     out64 = np.zeros(G.shape, np.float64)
-    masks = _masks(rht_masks, K) if quantized else None
+    masks = _masks(rht_masks, K) if quantized and not bf16 else None
     mp = _ptr(masks, _u16p) if masks is not None else None
+    route = (2 if bf16 else 1) if quantized else 0
     st = lib().fs4o_root_ns(_ptr(G, _fp), G.shape[0], G.shape[1], int(K), float(a), float(b), float(c),
                             float(clip_k) if clip_k else 0.0,
                             float(clip_quantile) if clip_quantile is not None else 0.0,
-                            1 if quantized else 0, mp, _flags(mode, adaptive46), _ptr(out32, _fp),
+                            route, mp, _flags(mode, adaptive46), _ptr(out32, _fp),
                             _ptr(out64, _dp), threads)
     if st != 0:
         raise ValueError("bad shape or non-finite input")
     return out32 if quantized else out64
+
+
+def bf16_round(x):
+    """FP32 -> BF16 (round to nearest, ties to even) as FP32 values (oracle.root_ns.bf16_round)."""
+    x = _f32(x)
+    y = np.zeros_like(x)
+    lib().fs4o_bf16_round(_ptr(x, _fp), x.size, _ptr(y, _fp))
+    return y
+
+
+def ns_iterations_bf16(X0, K, a, b, c, threads=0):
+    """K BF16 iterations (oracle.root_ns.ns_iterations_bf16)."""
+    X = _f32(X0).copy()
+    if lib().fs4o_ns_iterations_bf16(_ptr(X, _fp), X.shape[0], X.shape[1], int(K), float(a), float(b),
+                                     float(c), threads) != 0:
+        raise ValueError("bad shape")
+    return X
+
+
+def splitmix64(seed, idx):
+    idx = np.ascontiguousarray(idx, dtype=np.uint64)
+    out = np.zeros(idx.shape, np.uint64)
+    lib().fs4o_splitmix64(int(seed) & (2 ** 64 - 1), _ptr(idx, _u64p), idx.size, _ptr(out, _u64p))
+    return out
+
+
+def uniform24(seed, idx):
+    idx = np.ascontiguousarray(idx, dtype=np.uint64)
+    out = np.zeros(idx.shape, np.float32)
+    lib().fs4o_uniform24(int(seed) & (2 ** 64 - 1), _ptr(idx, _u64p), idx.size, _ptr(out, _fp))
+    return out
+
+
+def sr_encode_magnitude(v, u):
+    """Stochastic rounding of FP32 v >= 0 onto E2M1 codes 0..7 (oracle.momentum.sr_encode_magnitude)."""
+    v = np.asarray(v, np.float32).ravel()
+    u = np.asarray(u, np.float32).ravel()
+    if not np.all(np.isfinite(v)) or np.any(v < 0):
+        raise ValueError("SR encode expects finite non-negative inputs")
+    return np.array([lib().fs4o_e2m1_encode_sr(float(a), float(b)) for a, b in zip(v, u)], np.uint8)
+
+
+def momentum_update(g, beta, state=None, mask_prev=0, mask_next=0, seed=0, threads=0):
+    """One NVFP4 first-moment step (oracle.momentum.update): (m_t, (codes, scales, s_g))."""
+    g = _f32(g)
+    rows, cols = g.shape
+    m_t = np.zeros_like(g)
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros((rows, cols // 16), np.uint8)
+    sg = np.zeros(1, np.float32)
+    if state is None:
+        pc = ps = None
+        psg = 0.0
+    else:
+        pcodes = np.ascontiguousarray(state[0], np.uint8)
+        pscales = np.ascontiguousarray(state[1], np.uint8)
+        pc, ps, psg = _ptr(pcodes, _up), _ptr(pscales, _up), float(state[2])
+    if lib().fs4o_momentum_update(_ptr(g, _fp), rows, cols, float(beta), pc, ps, psg, int(mask_prev),
+                                  int(mask_next), int(seed) & (2 ** 64 - 1), _ptr(m_t, _fp),
+                                  _ptr(codes, _up), _ptr(scales, _up), _ptr(sg, _fp), threads) != 0:
+        raise ValueError("bad shape or mask")
+    return m_t, (codes, scales, np.float32(sg[0]))
+
+
+def momentum_load(codes, scales, s_g, mask):
+    """FP32 momentum decoded from a state (oracle.momentum.load)."""
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    rows, cols = codes.shape[0], codes.shape[1] * 2
+    out = np.zeros((rows, cols), np.float32)
+    if lib().fs4o_momentum_load(_ptr(codes, _up), _ptr(scales, _up), float(s_g), int(mask), rows, cols,
+                                _ptr(out, _fp)) != 0:
+        raise ValueError("bad shape or mask")
+    return out

@@ -1,7 +1,8 @@
 """NVFP4 storage of the first moment (momentum) for Q-Root, step by step.
 
-TEST INFRASTRUCTURE ONLY: imported by tests, by the smoke check and by the
-CPU-baseline leg of bench.py; never by the product path.
+TEST INFRASTRUCTURE ONLY: imported by tests and by the smoke check; never by the
+product path.  (The CPU-baseline leg of bench.py times the C++ restatement of the
+same steps, oracle/cpp/fs4_oracle.cpp, which the tests pin to this module bit for bit.)
 
 Source: "Full-Stack FP4" (arXiv 2607.04422), Section 3.3 "Quantized-State AdamW": for
 the first moment, Hadamard mixing smooths the distribution before stochastic rounding

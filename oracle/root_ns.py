@@ -146,22 +146,25 @@ def bf16_round(x) -> np.ndarray:
     return ((keep + up.astype(np.uint64)) << 16).astype(np.uint32).view(np.float32)
 
 
-def ns_iterations_bf16(X0, K, a, b, c, trace=None):
+def ns_iterations_bf16(X0, K, a, b, c, trace=None, matmul=None):
     """K Newton-Schulz iterations with BF16 operands (the optimized BF16 baseline the
     pages compare Q-Root against, Section 4.4 and Table 6), from the FP32 m x n X0
     (m <= n).  Same plan as the NVFP4 route with bf16() in place of each
     quantisation: Xb = bf16(X), A = Xb Xb^T, B = b A + c bf16(A) bf16(A)^T,
     X_{k+1} = a X + bf16(B) Xb.  Products in float64 on the BF16 values, rounded once
-    to FP32; A made exactly symmetric from its upper triangle; X, A, B FP32."""
+    to FP32; A made exactly symmetric from its upper triangle; X, A, B FP32.
+    matmul: None (float64 products), or a function (L, R) -> L R used for the three
+    products instead (as in ns_iterations_nvfp4)."""
+    mm = (lambda l, r: l @ r) if matmul is None else matmul
     X = np.asarray(X0, dtype=np.float32)
     for _ in range(K):
         Xb = bf16_round(X).astype(np.float64)
-        A = symmetric_from_upper(Xb @ Xb.T).astype(np.float32)
+        A = symmetric_from_upper(mm(Xb, Xb.T)).astype(np.float32)
         Ab = bf16_round(A).astype(np.float64)
-        P = Ab @ Ab.T
+        P = mm(Ab, Ab.T)
         B = (b * A.astype(np.float64) + c * P).astype(np.float32)
         Bb = bf16_round(B).astype(np.float64)
-        Xn = (a * X.astype(np.float64) + Bb @ Xb).astype(np.float32)
+        Xn = (a * X.astype(np.float64) + mm(Bb, Xb)).astype(np.float32)
         if trace is not None:
             trace.append(dict(X=X, A=A, P=P, B=B, X_next=Xn))
         X = Xn

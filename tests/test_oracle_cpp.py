@@ -15,6 +15,7 @@ import numpy as np
 import pytest
 
 from oracle import cpp_oracle as C
+from oracle import momentum as M
 from oracle import nvfp4 as Q
 from oracle import root_ns as R
 
@@ -352,3 +353,100 @@ def test_too_few_masks_are_refused():
         C.ns_iterations_nvfp4(X0, 2, *MUON, rht_masks=[1, 2, 3, 4, 5])
     with pytest.raises(ValueError):
         C.root_ns(X0, 1, *MUON, rht_masks=[1, 2, 0x10000])
+
+
+# ---------------------------------------------------------------- BF16 route and NVFP4 momentum
+# The BF16 comparison step (Section 4.4, Table 6) and the NVFP4 first moment (Section 3.3,
+# which Section 3.4's momentum follows), restated in C++ and pinned to the same things as
+# the numpy oracle: the published SplitMix64 outputs, hand-checkable roundings, and the
+# numpy oracle bit for bit.
+
+def test_splitmix64_reference_outputs_and_draws():
+    z = C.splitmix64(0, np.arange(3, dtype=np.uint64))
+    assert [int(v) for v in z] == [0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4, 0x06C45D188009454F]
+    idx = np.arange(1 << 12, dtype=np.uint64)
+    for seed in (0, 1, 12345, 2 ** 63 + 5, 2 ** 64 - 1):
+        assert np.array_equal(C.splitmix64(seed, idx), M.splitmix64(seed, idx))
+        u = C.uniform24(seed, idx)
+        assert np.array_equal(u, M.uniform24(seed, idx))
+        assert u.min() >= 0.0 and u.max() < 1.0
+
+
+def test_stochastic_rounding_against_the_numpy_oracle_and_by_hand():
+    grid = Q.E2M1_MAGNITUDES.astype(np.float32)
+    for code, g in enumerate(grid):                 # grid points never move
+        for u in (0.0, 0.5, 1 - 2 ** -24):
+            assert C.sr_encode_magnitude([g], [u])[0] == code
+    # v = 2.5 lies halfway between 2 (code 4) and 3 (code 5): up exactly when u < 0.5
+    assert list(C.sr_encode_magnitude([2.5, 2.5, 2.5], [0.0, 0.4999999, 0.5])) == [5, 5, 4]
+    assert list(C.sr_encode_magnitude([6.0, 7.5, 1e30], [0.0, 0.0, 0.9])) == [7, 7, 7]
+    rng = np.random.default_rng(21)
+    v = np.concatenate([rng.uniform(0, 7, 3000), [0.25, 0.75, 5.999, 1e-30]]).astype(np.float32)
+    u = rng.uniform(0, 1, v.size).astype(np.float32)
+    assert np.array_equal(C.sr_encode_magnitude(v, u), M.sr_encode_magnitude(v, u))
+
+
+@pytest.mark.parametrize("masks,seeds", [((0x0000, 0x5A5A), (1, 2)), ((0xA5C3, 0xFFFF), (99, 2 ** 40 + 3))])
+def test_momentum_steps_bit_exact_against_the_numpy_oracle(masks, seeds):
+    rng = np.random.default_rng(22)
+    g1 = (rng.standard_t(3, (64, 96)) * 0.02).astype(np.float32)
+    g2 = (rng.standard_t(3, (64, 96)) * 0.02).astype(np.float32)
+    g1[:, 32:48] = 0.0                                # an all-zero block
+    state_c = state_n = None
+    mask_prev = 0
+    for g, mask, seed, beta in ((g1, masks[0], seeds[0], 0.9), (g2, masks[1], seeds[1], 0.95)):
+        mc, state_c = C.momentum_update(g, beta, state_c, mask_prev, mask, seed)
+        mn, state_n = M.update(g, beta, state_n, mask_prev, mask, seed)
+        assert np.array_equal(mc.view(np.uint32), mn.view(np.uint32))
+        assert state_c[2] == state_n[2]
+        assert np.array_equal(state_c[0], state_n[0]) and np.array_equal(state_c[1], state_n[1])
+        dc, dn = C.momentum_load(*state_c, mask), M.load(*state_n, mask)
+        assert np.array_equal(dc.view(np.uint32), dn.view(np.uint32))
+        mask_prev = mask
+
+
+def test_momentum_beta_zero_stores_the_gradient():
+    """beta = 0: m_t = g exactly.  Decoding the state undoes H16^r, which is orthogonal, so
+    each block's error has the L2 norm of its error in the transformed domain: at most
+    sqrt(16) elements x the widest E2M1 gap (2) x the block's scale s_b s_g (plus FP32
+    rounding of the two transforms)."""
+    rng = np.random.default_rng(23)
+    g = (rng.standard_normal((16, 64)) * 0.02).astype(np.float32)
+    m, st = C.momentum_update(g, 0.0, None, 0, 0x3C3C, 5)
+    assert np.array_equal(m, g)
+    back = C.momentum_load(*st, 0x3C3C).astype(np.float64)
+    den = Q.E4M3_VALUES[st[1]].astype(np.float64) * float(st[2])          # 16 x 4 blocks
+    err = np.linalg.norm((back - g).reshape(16, 4, 16), axis=2)
+    gb = np.linalg.norm(g.astype(np.float64).reshape(16, 4, 16), axis=2)
+    assert np.all(err <= 4 * 2 * den + 1e-5 * gb)
+    assert np.all(err > 0)                                                  # SR moved every block
+
+
+def test_bf16_round_against_the_numpy_oracle_and_by_hand():
+    # 1 + 2^-8 is a tie between 1 and 1 + 2^-7: it goes to the even mantissa (1);
+    # 1 + 3 * 2^-8 is a tie between 1 + 2^-7 and 1 + 2^-6: it goes to 1 + 2^-6
+    x = np.float32([1 + 2 ** -8, 1 + 3 * 2 ** -8, 1 + 2 ** -8 + 2 ** -20, -2.0, 0.0, -0.0])
+    want = np.float32([1.0, 1 + 2 ** -6, 1 + 2 ** -7, -2.0, 0.0, -0.0])
+    got = C.bf16_round(x)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    y = (np.random.default_rng(24).standard_normal((40, 64)) * 10.0 ** np.arange(-20, 20, 0.625)).astype(np.float32)
+    assert np.array_equal(C.bf16_round(y).view(np.uint32), R.bf16_round(y).view(np.uint32))
+
+
+@pytest.mark.parametrize("shape,K,coef", [((48, 112), 3, MUON), ((32, 32), 2, QUINTIC), ((16, 40), 5, CUBIC)])
+def test_bf16_iteration_bit_identical_to_the_numpy_steps(shape, K, coef):
+    rng = np.random.default_rng(25)
+    X0 = R.normalise_and_clip((rng.standard_t(4, shape) * 0.02).astype(np.float32), 3.0)[0]
+    got = C.ns_iterations_bf16(X0, K, *coef)
+    want = R.ns_iterations_bf16(X0, K, *coef, matmul=C.product)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+@pytest.mark.parametrize("shape", [(64, 160), (160, 64)])
+def test_bf16_route_matches_the_numpy_oracle(shape):
+    rng = np.random.default_rng(26)
+    G = (rng.standard_t(3, shape) * 0.02).astype(np.float32)
+    got = C.root_ns(G, 3, *MUON, clip_k=3.0, bf16=True)
+    want = R.root_ns(G, 3, *MUON, clip_k=3.0, bf16=True)
+    assert got.shape == want.shape
+    assert np.linalg.norm(got - want) <= 1e-6 * np.linalg.norm(want)
