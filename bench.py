@@ -270,17 +270,6 @@ def bf16_comparator(F, Gs, w, steps: int, flush, l2_bytes: int):
     return ms, phase
 
 
-def cpu_cores():
-    try:
-        from threadpoolctl import threadpool_info
-        nums = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        if nums:
-            return int(max(nums))
-    except Exception:
-        pass
-    return os.cpu_count() or 1
-
-
 QUANT_NAMES = {"plain": "NVFP4 RTN (H = I, M = 6)",
                "rht46": "NVFP4 RTN with H16^r (fresh signs per step) and adaptive 4/6",
                "rht": "NVFP4 RTN with H16^r (fresh signs per step)",
@@ -345,31 +334,32 @@ QD_METRIC = {"quantize": "NVFP4 standalone quantise GB/s (4.5625 B per element)"
 
 
 def oracle_qd_rate(w, op: str, budget_s: float):
-    """Time the oracle's quantiser (or dequantiser) on leading rows of the workload's
+    """Time the C++ oracle's quantiser (or dequantiser) on leading rows of the workload's
     first matrix, growing the slice until it takes about budget_s / 4 seconds.
-    Returns (algorithmic GB/s, seconds, description)."""
-    from oracle import nvfp4 as Q
+    Returns (algorithmic GB/s, seconds, description, cores)."""
+    from oracle import cpp_oracle as C
     from nvfp4_precision_optimizer_b200.workloads import BASE_SEED, generate
     G = generate(w.shapes[0], w.dist, BASE_SEED, "cpu").numpy()
     rows = 16
     while True:
-        x = G[:rows]
+        x = np.ascontiguousarray(G[:rows])
         if op == "quantize":
             t0 = time.perf_counter()
-            Q.quantize_rows(x)
+            C.quantize_rows(x)
             dt = time.perf_counter() - t0
         else:
-            c, sc, g = Q.quantize_rows(x)
+            c, sc, g = C.quantize_rows(x)
             t0 = time.perf_counter()
-            Q.dequantize_rows(c, sc, g, dtype=np.float32)
+            C.dequantize_rows(c, sc, g)
             dt = time.perf_counter() - t0
         if dt >= budget_s / 4 or rows >= G.shape[0]:
             break
         rows = min(G.shape[0], rows * 4)
     rate = x.size * QD_BYTES / dt / 1e9
-    desc = (f"oracle {op} (numpy, exact NVFP4 emulation) of the first {rows} rows of a "
-            f"{G.shape[0]}x{G.shape[1]} workload matrix, {dt:.2f} s")
-    return rate, dt, desc
+    cores = C.threads()
+    desc = (f"C++ oracle {op} (exact NVFP4 emulation, OpenMP over rows) of the first {rows} rows "
+            f"of a {G.shape[0]}x{G.shape[1]} workload matrix, {dt:.2f} s on {cores} threads")
+    return rate, dt, desc, cores
 
 
 def run_reference(args):
@@ -382,9 +372,9 @@ def run_reference(args):
         run_momentum_reference(args, w)
         return
     if args.op != "ns":
-        rates, desc = [], ""
+        rates, desc, cores = [], "", 1
         for i in range(args.warmup + args.steps):
-            rate, dt, desc = oracle_qd_rate(w, args.op, max(2.0, 120.0 / max(1, args.steps + args.warmup)))
+            rate, dt, desc, cores = oracle_qd_rate(w, args.op, max(2.0, 120.0 / max(1, args.steps + args.warmup)))
             if i >= args.warmup:
                 rates.append(rate)
         value = statistics.median(rates)
@@ -396,7 +386,7 @@ def run_reference(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32 values, exact NVFP4 emulation",
             "data": "synthetic", "config": {"workload": w.name, "matrices": len(w.shapes), "op": args.op,
                                             "layout": "plain"},
-            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }
@@ -1047,8 +1037,8 @@ def run_standalone(args, w, rank, world, local, barrier, ranks_max):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, dt, desc = oracle_qd_rate(w, args.op, 20.0)
-        cpu = {"value": rate, "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle", "sample": desc}
+        rate, dt, desc, cores = oracle_qd_rate(w, args.op, 20.0)
+        cpu = {"value": rate, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
     if rank == 0:
         line = {
             "metric": QD_METRIC[args.op], "value": value, "unit": "GB/s", "n_gpus": world,
