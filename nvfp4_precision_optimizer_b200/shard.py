@@ -97,9 +97,11 @@ class ShardedRootNS:
     does not own are not read and may be None.  It returns the updates of every
     matrix: views of one receive buffer, which the next call overwrites.
 
-    compute(Gs_local, outs_local) runs the step on this rank's share.  The default is
-    the CUDA path, fs4.root_ns_batched, with a workspace allocated once and the
-    options given here (K, coeffs, clip_k, rht_masks, adaptive46, clip_quantile).
+    compute(Gs_local, outs_local, **call_options) runs the step on this rank's share.  The
+    default is the CUDA path, fs4.root_ns_batched, with a workspace allocated once and the
+    options given here (K, coeffs, clip_k, rht_masks, adaptive46, clip_quantile).  Options
+    given to a call override these for that call: H16^r takes fresh sign masks every step,
+    e.g. S(Gs, rht_masks=masks).  Every rank should pass the same ones.
     The collective is torch.distributed's all_gather_into_tensor on the group (NCCL
     across GPUs).  It is skipped when the group has one rank.
     """
@@ -138,11 +140,12 @@ class ShardedRootNS:
             need = ns_batched_workspace_size([self.plan.shapes[i] for i in self.local])
             self.workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
 
-        def compute(Gs, outs):
-            root_ns_batched(Gs, K=K, coeffs=local_coeffs, outs=outs, workspace=self.workspace, **opts)
+        def compute(Gs, outs, **call_opts):
+            root_ns_batched(Gs, K=K, coeffs=local_coeffs, outs=outs, workspace=self.workspace,
+                            **{**opts, **call_opts})
         return compute
 
-    def compute_local(self, Gs: Sequence[torch.Tensor | None]) -> None:
+    def compute_local(self, Gs: Sequence[torch.Tensor | None], **call_options) -> None:
         """The step on this rank's share, into its send buffer (no collective)."""
         if len(Gs) != len(self.plan.shapes):
             raise ValueError("one momentum per matrix of the plan")
@@ -153,7 +156,7 @@ class ShardedRootNS:
             if G is None or tuple(G.shape) != self.plan.shapes[i]:
                 raise ValueError(f"matrix {i} is owned by rank {self.rank} and must have shape "
                                  f"{self.plan.shapes[i]}")
-        self.compute(local, self.local_outs)
+        self.compute(local, self.local_outs, **call_options)
 
     def gather(self) -> list[torch.Tensor]:
         """The all-gather of every rank's send buffer; returns the updates of every matrix."""
@@ -162,6 +165,6 @@ class ShardedRootNS:
             dist.all_gather_into_tensor(self.recv, self.send, group=self.group)
         return self.outs
 
-    def __call__(self, Gs: Sequence[torch.Tensor | None]) -> list[torch.Tensor]:
-        self.compute_local(Gs)
+    def __call__(self, Gs: Sequence[torch.Tensor | None], **call_options) -> list[torch.Tensor]:
+        self.compute_local(Gs, **call_options)
         return self.gather()

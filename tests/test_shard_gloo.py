@@ -74,9 +74,17 @@ def test_bench_workload_balance():
         assert shard.plan(w.shapes, w.K, world).imbalance < 1.05
 
 
-def _double(Gs, outs):
+def _double(Gs, outs, scale=2.0):
     for G, o in zip(Gs, outs):
-        o.copy_(2.0 * G)
+        o.copy_(scale * G)
+
+
+def test_call_options_reach_the_step():
+    shapes = [(32, 48), (16, 16)]
+    Gs = [torch.randn(s) for s in shapes]
+    S = shard.ShardedRootNS(shapes, K=3, rank=0, world=1, device="cpu", compute=_double)
+    outs = S(Gs, scale=3.0)
+    assert all(torch.equal(o, 3.0 * G) for o, G in zip(outs, Gs))
 
 
 def test_one_rank_needs_no_collective():
