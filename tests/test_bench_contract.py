@@ -107,3 +107,22 @@ def test_roofline_helpers_by_hand():
         t_flop = bench.flops_per_launch(wm, "update") / fp4
         t_byte = bench.bytes_per_launch(wm, "update") / hbm
         assert ("hbm" if t_byte > t_flop else "tensor") == bound, side
+
+
+def test_committed_register_report_matches_the_sources():
+    """profiles/ptxas_resources_all_kernels.md was made from the current CUDA sources (its
+    digest), lists one row per kernel, and records no spill on the default or 8192-class
+    GEMM variants."""
+    import re
+
+    from nvfp4_precision_optimizer_b200 import build
+    text = open(os.path.join(ROOT, "profiles", "ptxas_resources_all_kernels.md")).read()
+    m = re.search(r"(\d+) kernels; CUDA source digest ([0-9a-f]{16})", text)
+    assert m, "the report carries its kernel count and source digest"
+    assert m.group(2) == build.source_digest(), \
+        "CUDA sources changed: rerun python -m nvfp4_precision_optimizer_b200.build --ptxas-table"
+    rows = re.findall(r"^\| `([^`]+)` \| (\d+) \| (\d+) / (\d+) \|", text, re.M)
+    assert len(rows) == int(m.group(1))
+    for name, regs, st, ld in rows:
+        if name.startswith("nvfp4_gemm_kernel") and name.split()[-1] in ("plain", "wide-K"):
+            assert int(regs) == 168 and int(st) == 0 and int(ld) == 0, name
